@@ -1,0 +1,460 @@
+// C ABI of the library (declared in include/gla.h): argument checks, workspace layout and the
+// sequence of kernel launches for each operator.  Every check runs on the host before anything
+// is enqueued; nothing here allocates, frees or synchronises (except gla_device_error).
+#include <limits.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/gla.h"
+#include "common.cuh"
+#include "fast_path.cuh"
+#include "generic_kernels.cuh"
+
+using gla::bf16;
+namespace gk = gla::generic;
+
+// Device-side error latch written by bounded waits that run out (see gla_device_error).
+__device__ unsigned int g_gla_device_error = 0;
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Pointer rule: required pointers must be non-NULL; every non-NULL pointer 16-byte aligned.
+int check_ptr(const void* p, bool required) {
+  if (!p) return required ? GLA_ERR_INVALID_ARG : GLA_OK;
+  return aligned16(p) ? GLA_OK : GLA_ERR_INVALID_ARG;
+}
+
+int check_dim(int d) {
+  if (d <= 0) return GLA_ERR_INVALID_ARG;
+  if (d > 512 || d % 8 != 0) return GLA_ERR_UNSUPPORTED;
+  return GLA_OK;
+}
+
+int check_common(int B, int H, int T, int chunk, int dtype) {
+  if (B <= 0 || H <= 0 || T < 0) return GLA_ERR_INVALID_ARG;
+  if ((long long)B * H > INT_MAX) return GLA_ERR_INVALID_ARG;
+  if ((long long)B * H * (long long)(T > 0 ? T : 1) > (1LL << 40)) return GLA_ERR_INVALID_ARG;
+  if (dtype != GLA_DTYPE_F32 && dtype != GLA_DTYPE_BF16) return GLA_ERR_UNSUPPORTED;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return GLA_ERR_UNSUPPORTED;
+  return GLA_OK;
+}
+
+#define GLA_TRY(expr)              \
+  do {                             \
+    int _s = (expr);               \
+    if (_s != GLA_OK) return _s;   \
+  } while (0)
+
+#define GLA_CUDA(expr)                          \
+  do {                                          \
+    if ((expr) != cudaSuccess) return GLA_ERR_CUDA; \
+  } while (0)
+
+size_t esize(int dtype) { return dtype == GLA_DTYPE_BF16 ? 2 : 4; }
+
+// Bump allocator over the caller's workspace (or a dry run that only counts bytes).
+struct Carve {
+  char* base;
+  size_t used = 0;
+  explicit Carve(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + used) : nullptr;
+    used += gla::align256(count * sizeof(T));
+    return p;
+  }
+};
+
+// ----------------------------------------------------------------------------------------
+// GLA forward / backward (generic chunk-parallel passes)
+// ----------------------------------------------------------------------------------------
+struct GlaFwdWs {
+  float* states;
+};
+size_t carve_gla_fwd(Carve& c, int BH, int T, int dk, int dv, int chunk, GlaFwdWs* w) {
+  const size_t NC = gla::num_chunks(T, chunk);
+  float* s = c.take<float>((size_t)BH * NC * dk * dv);
+  if (w) w->states = s;
+  return c.used;
+}
+
+struct GlaBwdWs {
+  float *states, *dstates, *db, *hT;
+};
+size_t carve_gla_bwd(Carve& c, int BH, int T, int dk, int dv, int chunk, GlaBwdWs* w) {
+  const size_t NC = gla::num_chunks(T, chunk);
+  GlaBwdWs x;
+  x.states = c.take<float>((size_t)BH * NC * dk * dv);
+  x.dstates = c.take<float>((size_t)BH * NC * dk * dv);
+  x.db = c.take<float>((size_t)BH * T * dk);
+  x.hT = c.take<float>((size_t)BH * dk * dv);
+  if (w) *w = x;
+  return c.used;
+}
+
+template <typename TI>
+int gla_fwd_generic(const TI* q, const TI* k, const TI* v, const TI* g, const float* h0, TI* o, float* hT,
+                    gk::Shape s, void* ws, cudaStream_t st) {
+  Carve c(ws);
+  GlaFwdWs w;
+  carve_gla_fwd(c, s.BH, s.T, s.DK, s.DV, s.C, &w);
+  GLA_CUDA(gk::state_fwd<TI>(s, k, v, g, h0, 0, w.states, hT, 0, st));
+  GLA_CUDA((gk::out<TI, TI, TI>(s, q, k, v, g, w.states, o, st)));
+  return GLA_OK;
+}
+
+template <typename TI>
+int gla_bwd_generic(const TI* q, const TI* k, const TI* v, const TI* g, const float* h0, const TI* dO,
+                    const float* dhT, TI* dq, TI* dk, TI* dv, TI* dg, float* dh0, gk::Shape s, void* ws,
+                    cudaStream_t st) {
+  Carve c(ws);
+  GlaBwdWs w;
+  carve_gla_bwd(c, s.BH, s.T, s.DK, s.DV, s.C, &w);
+  GLA_CUDA(gk::state_fwd<TI>(s, k, v, g, h0, 0, w.states, w.hT, 0, st));
+  GLA_CUDA((gk::dstate_bwd<TI, TI>(s, q, g, dO, dhT, 0, w.dstates, dh0, 0, st)));
+  GLA_CUDA((gk::bwd_dqdk<TI, TI, TI>(s, q, k, v, g, dO, w.states, w.dstates, dq, dk, nullptr, w.db, st)));
+  GLA_CUDA((gk::bwd_dv<TI, TI, TI>(s, q, k, g, dO, w.dstates, dv, st)));
+  GLA_CUDA(gk::dg<TI>(s, w.db, w.hT, dhT, 0, nullptr, dg, st));
+  return GLA_OK;
+}
+
+// Copy src (or zeros when NULL) into dst, n floats; used for T == 0.
+int copy_or_zero(float* dst, const float* src, size_t n, cudaStream_t st) {
+  if (!dst) return GLA_OK;
+  if (src)
+    GLA_CUDA(cudaMemcpyAsync(dst, src, n * sizeof(float), cudaMemcpyDeviceToDevice, st));
+  else
+    GLA_CUDA(cudaMemsetAsync(dst, 0, n * sizeof(float), st));
+  return GLA_OK;
+}
+
+// ----------------------------------------------------------------------------------------
+// GSA (generic passes; pass 1 is the key-gated pass with roles exchanged: its state is kept
+// transposed, [m x dk], so that the slot axis is the gated row axis)
+// ----------------------------------------------------------------------------------------
+struct GsaFwdWs {
+  float *S1, *o1, *S2;
+  void* p;
+};
+size_t carve_gsa_fwd(Carve& c, int BH, int T, int dk, int dv, int m, int chunk, int dtype, bool need_p,
+                     GsaFwdWs* w) {
+  const size_t NC = gla::num_chunks(T, chunk);
+  GsaFwdWs x;
+  x.S1 = c.take<float>((size_t)BH * NC * m * dk);
+  x.o1 = c.take<float>((size_t)BH * T * m);
+  x.S2 = c.take<float>((size_t)BH * NC * m * dv);
+  x.p = need_p ? (void*)c.take<char>((size_t)BH * T * m * esize(dtype)) : nullptr;
+  if (w) *w = x;
+  return c.used;
+}
+
+struct GsaBwdWs {
+  float *S1, *o1, *S2, *dS2, *hT2, *db, *dp, *dphi2, *dg2, *do1, *dS1, *hT1;
+  void* p;
+};
+size_t carve_gsa_bwd(Carve& c, int BH, int T, int dk, int dv, int m, int chunk, int dtype, GsaBwdWs* w) {
+  const size_t NC = gla::num_chunks(T, chunk);
+  const size_t tm = (size_t)BH * T * m;
+  GsaBwdWs x;
+  x.S1 = c.take<float>((size_t)BH * NC * m * dk);
+  x.o1 = c.take<float>(tm);
+  x.S2 = c.take<float>((size_t)BH * NC * m * dv);
+  x.dS2 = c.take<float>((size_t)BH * NC * m * dv);
+  x.hT2 = c.take<float>((size_t)BH * m * dv);
+  x.db = c.take<float>(tm);
+  x.dp = c.take<float>(tm);
+  x.dphi2 = c.take<float>(tm);
+  x.dg2 = c.take<float>(tm);
+  x.do1 = c.take<float>(tm);
+  x.dS1 = c.take<float>((size_t)BH * NC * m * dk);
+  x.hT1 = c.take<float>((size_t)BH * m * dk);
+  x.p = (void*)c.take<char>(tm * esize(dtype));
+  if (w) *w = x;
+  return c.used;
+}
+
+template <typename TI>
+int gsa_fwd_impl(const TI* q, const TI* k, const TI* v, const TI* phi, const TI* g, const float* h01,
+                 const float* h02, TI* o, TI* p_save, float* hT1, float* hT2, int BH, int T, int dk, int dv, int m,
+                 int C, void* ws, cudaStream_t st) {
+  Carve c(ws);
+  GsaFwdWs w;
+  carve_gsa_fwd(c, BH, T, dk, dv, m, C, sizeof(TI) == 2 ? GLA_DTYPE_BF16 : GLA_DTYPE_F32, p_save == nullptr, &w);
+  TI* p = p_save ? p_save : static_cast<TI*>(w.p);
+  const gk::Shape s1{BH, T, m, dk, C}, s2{BH, T, m, dv, C};
+  // pass 1 state (transposed), then o1 = e^B (q S1) + gated intra term, via the dq formula.
+  GLA_CUDA(gk::state_fwd<TI>(s1, phi, k, g, h01, 1, w.S1, hT1, 1, st));
+  GLA_CUDA((gk::bwd_dqdk<TI, TI, float>(s1, phi, phi, k, g, q, w.S1, nullptr, w.o1, nullptr, nullptr, nullptr,
+                                        st)));
+  GLA_CUDA(gk::softmax_fwd<TI>(w.o1, p, nullptr, (long)BH * T, m, st));
+  GLA_CUDA(gk::state_fwd<TI>(s2, phi, v, g, h02, 0, w.S2, hT2, 0, st));
+  GLA_CUDA((gk::out<TI, TI, TI>(s2, p, phi, v, g, w.S2, o, st)));
+  return GLA_OK;
+}
+
+template <typename TI>
+int gsa_bwd_impl(const TI* q, const TI* k, const TI* v, const TI* phi, const TI* g, const float* h01,
+                 const float* h02, const TI* dO, const float* dhT1, const float* dhT2, TI* dq, TI* dk, TI* dv,
+                 TI* dphi, TI* dg, float* dh01, float* dh02, int BH, int T, int dkd, int dvd, int m, int C,
+                 void* ws, cudaStream_t st) {
+  Carve c(ws);
+  GsaBwdWs w;
+  carve_gsa_bwd(c, BH, T, dkd, dvd, m, C, sizeof(TI) == 2 ? GLA_DTYPE_BF16 : GLA_DTYPE_F32, &w);
+  TI* p = static_cast<TI*>(w.p);
+  const gk::Shape s1{BH, T, m, dkd, C}, s2{BH, T, m, dvd, C};
+  // recompute pass 1 and the slot softmax
+  GLA_CUDA(gk::state_fwd<TI>(s1, phi, k, g, h01, 1, w.S1, w.hT1, 0, st));
+  GLA_CUDA((gk::bwd_dqdk<TI, TI, float>(s1, phi, phi, k, g, q, w.S1, nullptr, w.o1, nullptr, nullptr, nullptr,
+                                        st)));
+  GLA_CUDA(gk::softmax_fwd<TI>(w.o1, p, nullptr, (long)BH * T, m, st));
+  // pass 2 backward (queries p, keys phi, values v)
+  GLA_CUDA(gk::state_fwd<TI>(s2, phi, v, g, h02, 0, w.S2, w.hT2, 0, st));
+  GLA_CUDA((gk::dstate_bwd<TI, TI>(s2, p, g, dO, dhT2, 0, w.dS2, dh02, 0, st)));
+  GLA_CUDA((gk::bwd_dqdk<TI, TI, float>(s2, p, phi, v, g, dO, w.S2, w.dS2, w.dp, w.dphi2, nullptr, w.db, st)));
+  GLA_CUDA((gk::bwd_dv<TI, TI, TI>(s2, p, phi, g, dO, w.dS2, dv, st)));
+  GLA_CUDA(gk::dg<float>(s2, w.db, w.hT2, dhT2, 0, nullptr, w.dg2, st));
+  // slot softmax Jacobian
+  GLA_CUDA(gk::softmax_bwd(w.o1, w.dp, w.do1, (long)BH * T, m, st));
+  // pass 1 backward with roles exchanged
+  GLA_CUDA((gk::dstate_bwd<float, TI>(s1, w.do1, g, q, dhT1, 1, w.dS1, dh01, 1, st)));
+  GLA_CUDA((gk::out<float, TI, TI>(s1, w.do1, phi, k, g, w.S1, dq, st)));
+  GLA_CUDA((gk::bwd_dv<float, TI, TI>(s1, w.do1, phi, g, q, w.dS1, dk, st)));
+  GLA_CUDA((gk::bwd_dqdk<float, TI, TI>(s1, w.do1, phi, k, g, q, w.S1, w.dS1, nullptr, dphi, w.dphi2, w.db, st)));
+  GLA_CUDA(gk::dg<TI>(s1, w.db, w.hT1, dhT1, 1, w.dg2, dg, st));
+  return GLA_OK;
+}
+
+}  // namespace
+
+// =========================================================================================
+// C ABI
+// =========================================================================================
+extern "C" {
+
+const char* gla_status_string(int status) {
+  switch (status) {
+    case GLA_OK: return "GLA_OK";
+    case GLA_ERR_INVALID_ARG: return "GLA_ERR_INVALID_ARG: NULL, misaligned or out-of-range argument";
+    case GLA_ERR_UNSUPPORTED: return "GLA_ERR_UNSUPPORTED: dtype, chunk or dimension not supported";
+    case GLA_ERR_WORKSPACE: return "GLA_ERR_WORKSPACE: workspace missing or too small";
+    case GLA_ERR_CUDA: return "GLA_ERR_CUDA: a CUDA call or kernel launch failed";
+    case GLA_ERR_TIMEOUT: return "GLA_ERR_TIMEOUT: a bounded device-side wait ran out";
+  }
+  return "unknown gla_status";
+}
+
+int gla_version(void) { return kVersion; }
+
+size_t gla_chunk_fwd_workspace(int B, int H, int T, int dk, int dv, int chunk, int dtype) {
+  if (check_common(B, H, T, chunk, dtype) || check_dim(dk) || check_dim(dv)) return 0;
+  if (T == 0) return 0;
+  if (gla::fast::fwd_supported(B * H, T, dk, dv, chunk, dtype)) return gla::fast::fwd_workspace(B * H, T, dk, dv);
+  Carve c(nullptr);
+  return carve_gla_fwd(c, B * H, T, dk, dv, chunk, nullptr);
+}
+
+int gla_chunk_fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
+                  int B, int H, int T, int dk, int dv, int chunk, int dtype, void* ws, size_t ws_bytes,
+                  void* stream) {
+  GLA_TRY(check_common(B, H, T, chunk, dtype));
+  GLA_TRY(check_dim(dk));
+  GLA_TRY(check_dim(dv));
+  const bool tok = T > 0;
+  GLA_TRY(check_ptr(q, tok));
+  GLA_TRY(check_ptr(k, tok));
+  GLA_TRY(check_ptr(v, tok));
+  GLA_TRY(check_ptr(g, tok));
+  GLA_TRY(check_ptr(o, tok));
+  GLA_TRY(check_ptr(h0, false));
+  GLA_TRY(check_ptr(hT, false));
+  const size_t need = gla_chunk_fwd_workspace(B, H, T, dk, dv, chunk, dtype);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return GLA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (T == 0) return copy_or_zero(hT, h0, (size_t)BH * dk * dv, st);
+  if (gla::fast::fwd_supported(BH, T, dk, dv, chunk, dtype))
+    return gla::fast::fwd(q, k, v, g, h0, o, hT, BH, T, dk, dv, ws, st) == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+  const gk::Shape s{BH, T, dk, dv, chunk};
+  if (dtype == GLA_DTYPE_BF16)
+    return gla_fwd_generic<bf16>((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)g, h0, (bf16*)o, hT,
+                                 s, ws, st);
+  return gla_fwd_generic<float>((const float*)q, (const float*)k, (const float*)v, (const float*)g, h0, (float*)o,
+                                hT, s, ws, st);
+}
+
+size_t gla_chunk_bwd_workspace(int B, int H, int T, int dk, int dv, int chunk, int dtype) {
+  if (check_common(B, H, T, chunk, dtype) || check_dim(dk) || check_dim(dv)) return 0;
+  if (T == 0) return 0;
+  if (gla::fast::bwd_supported(B * H, T, dk, dv, chunk, dtype)) return gla::fast::bwd_workspace(B * H, T, dk, dv);
+  Carve c(nullptr);
+  return carve_gla_bwd(c, B * H, T, dk, dv, chunk, nullptr);
+}
+
+int gla_chunk_bwd(const void* q, const void* k, const void* v, const void* g, const float* h0, const void* dO,
+                  const float* dhT, void* dq, void* dk, void* dv, void* dg, float* dh0, int B, int H, int T,
+                  int dkd, int dvd, int chunk, int dtype, void* ws, size_t ws_bytes, void* stream) {
+  GLA_TRY(check_common(B, H, T, chunk, dtype));
+  GLA_TRY(check_dim(dkd));
+  GLA_TRY(check_dim(dvd));
+  const bool tok = T > 0;
+  const void* req[] = {q, k, v, g, dO, dq, dk, dv, dg};
+  for (const void* p : req) GLA_TRY(check_ptr(p, tok));
+  GLA_TRY(check_ptr(h0, false));
+  GLA_TRY(check_ptr(dhT, false));
+  GLA_TRY(check_ptr(dh0, false));
+  const size_t need = gla_chunk_bwd_workspace(B, H, T, dkd, dvd, chunk, dtype);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return GLA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (T == 0) return copy_or_zero(dh0, dhT, (size_t)BH * dkd * dvd, st);
+  if (gla::fast::bwd_supported(BH, T, dkd, dvd, chunk, dtype))
+    return gla::fast::bwd(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, dkd, dvd, ws, st) == cudaSuccess
+               ? GLA_OK
+               : GLA_ERR_CUDA;
+  const gk::Shape s{BH, T, dkd, dvd, chunk};
+  if (dtype == GLA_DTYPE_BF16)
+    return gla_bwd_generic<bf16>((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)g, h0,
+                                 (const bf16*)dO, dhT, (bf16*)dq, (bf16*)dk, (bf16*)dv, (bf16*)dg, dh0, s, ws, st);
+  return gla_bwd_generic<float>((const float*)q, (const float*)k, (const float*)v, (const float*)g, h0,
+                                (const float*)dO, dhT, (float*)dq, (float*)dk, (float*)dv, (float*)dg, dh0, s, ws,
+                                st);
+}
+
+int gla_recurrent_step(const void* q, const void* k, const void* v, const void* g, float* S, void* o, int B, int H,
+                       int dk, int dv, int dtype, void* stream) {
+  GLA_TRY(check_common(B, H, 1, 64, dtype));
+  GLA_TRY(check_dim(dk));
+  GLA_TRY(check_dim(dv));
+  const void* req[] = {q, k, v, g, S, o};
+  for (const void* p : req) GLA_TRY(check_ptr(p, true));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (dtype == GLA_DTYPE_BF16)
+    GLA_CUDA(gk::decode<bf16>(BH, dk, dv, (const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)g, S,
+                              (bf16*)o, st));
+  else
+    GLA_CUDA(gk::decode<float>(BH, dk, dv, (const float*)q, (const float*)k, (const float*)v, (const float*)g, S,
+                               (float*)o, st));
+  return GLA_OK;
+}
+
+size_t gsa_fwd_workspace(int B, int H, int T, int dk, int dv, int m, int chunk, int dtype) {
+  if (check_common(B, H, T, chunk, dtype) || check_dim(dk) || check_dim(dv) || check_dim(m)) return 0;
+  if (T == 0) return 0;
+  Carve c(nullptr);
+  return carve_gsa_fwd(c, B * H, T, dk, dv, m, chunk, dtype, true, nullptr);
+}
+
+int gsa_fwd(const void* q, const void* k, const void* v, const void* phi, const void* g, const float* h0_1,
+            const float* h0_2, void* o, void* p_save, float* hT1, float* hT2, int B, int H, int T, int dk, int dv,
+            int m, int chunk, int dtype, void* ws, size_t ws_bytes, void* stream) {
+  GLA_TRY(check_common(B, H, T, chunk, dtype));
+  GLA_TRY(check_dim(dk));
+  GLA_TRY(check_dim(dv));
+  GLA_TRY(check_dim(m));
+  const bool tok = T > 0;
+  const void* req[] = {q, k, v, phi, g, o};
+  for (const void* p : req) GLA_TRY(check_ptr(p, tok));
+  const void* opt[] = {h0_1, h0_2, p_save, hT1, hT2};
+  for (const void* p : opt) GLA_TRY(check_ptr(p, false));
+  const size_t need = gsa_fwd_workspace(B, H, T, dk, dv, m, chunk, dtype);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return GLA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (T == 0) {
+    GLA_TRY(copy_or_zero(hT1, h0_1, (size_t)BH * dk * m, st));
+    return copy_or_zero(hT2, h0_2, (size_t)BH * m * dv, st);
+  }
+  if (dtype == GLA_DTYPE_BF16)
+    return gsa_fwd_impl<bf16>((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)phi, (const bf16*)g,
+                              h0_1, h0_2, (bf16*)o, (bf16*)p_save, hT1, hT2, BH, T, dk, dv, m, chunk, ws, st);
+  return gsa_fwd_impl<float>((const float*)q, (const float*)k, (const float*)v, (const float*)phi,
+                             (const float*)g, h0_1, h0_2, (float*)o, (float*)p_save, hT1, hT2, BH, T, dk, dv, m,
+                             chunk, ws, st);
+}
+
+size_t gsa_bwd_workspace(int B, int H, int T, int dk, int dv, int m, int chunk, int dtype) {
+  if (check_common(B, H, T, chunk, dtype) || check_dim(dk) || check_dim(dv) || check_dim(m)) return 0;
+  if (T == 0) return 0;
+  Carve c(nullptr);
+  return carve_gsa_bwd(c, B * H, T, dk, dv, m, chunk, dtype, nullptr);
+}
+
+int gsa_bwd(const void* q, const void* k, const void* v, const void* phi, const void* g, const float* h0_1,
+            const float* h0_2, const void* dO, const float* dhT1, const float* dhT2, void* dq, void* dk, void* dv,
+            void* dphi, void* dg, float* dh0_1, float* dh0_2, int B, int H, int T, int dkd, int dvd, int m,
+            int chunk, int dtype, void* ws, size_t ws_bytes, void* stream) {
+  GLA_TRY(check_common(B, H, T, chunk, dtype));
+  GLA_TRY(check_dim(dkd));
+  GLA_TRY(check_dim(dvd));
+  GLA_TRY(check_dim(m));
+  const bool tok = T > 0;
+  const void* req[] = {q, k, v, phi, g, dO, dq, dk, dv, dphi, dg};
+  for (const void* p : req) GLA_TRY(check_ptr(p, tok));
+  const void* opt[] = {h0_1, h0_2, dhT1, dhT2, dh0_1, dh0_2};
+  for (const void* p : opt) GLA_TRY(check_ptr(p, false));
+  const size_t need = gsa_bwd_workspace(B, H, T, dkd, dvd, m, chunk, dtype);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return GLA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (T == 0) {
+    GLA_TRY(copy_or_zero(dh0_1, dhT1, (size_t)BH * dkd * m, st));
+    return copy_or_zero(dh0_2, dhT2, (size_t)BH * m * dvd, st);
+  }
+  if (dtype == GLA_DTYPE_BF16)
+    return gsa_bwd_impl<bf16>((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)phi, (const bf16*)g,
+                              h0_1, h0_2, (const bf16*)dO, dhT1, dhT2, (bf16*)dq, (bf16*)dk, (bf16*)dv, (bf16*)dphi,
+                              (bf16*)dg, dh0_1, dh0_2, BH, T, dkd, dvd, m, chunk, ws, st);
+  return gsa_bwd_impl<float>((const float*)q, (const float*)k, (const float*)v, (const float*)phi,
+                             (const float*)g, h0_1, h0_2, (const float*)dO, dhT1, dhT2, (float*)dq, (float*)dk,
+                             (float*)dv, (float*)dphi, (float*)dg, dh0_1, dh0_2, BH, T, dkd, dvd, m, chunk, ws, st);
+}
+
+int gsa_recurrent_step(const void* q, const void* k, const void* v, const void* phi, const void* g, float* S1,
+                       float* S2, void* o, int B, int H, int dk, int dv, int m, int dtype, void* stream) {
+  GLA_TRY(check_common(B, H, 1, 64, dtype));
+  GLA_TRY(check_dim(dk));
+  GLA_TRY(check_dim(dv));
+  GLA_TRY(check_dim(m));
+  const void* req[] = {q, k, v, phi, g, S1, S2, o};
+  for (const void* p : req) GLA_TRY(check_ptr(p, true));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (dtype == GLA_DTYPE_BF16)
+    GLA_CUDA(gk::gsa_decode<bf16>(BH, dk, dv, m, (const bf16*)q, (const bf16*)k, (const bf16*)v,
+                                  (const bf16*)phi, (const bf16*)g, S1, S2, (bf16*)o, st));
+  else
+    GLA_CUDA(gk::gsa_decode<float>(BH, dk, dv, m, (const float*)q, (const float*)k, (const float*)v,
+                                   (const float*)phi, (const float*)g, S1, S2, (float*)o, st));
+  return GLA_OK;
+}
+
+int gla_device_error(void* stream, int reset, int* code) {
+  if (!code) return GLA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned int v = 0;
+  GLA_CUDA(cudaMemcpyFromSymbolAsync(&v, g_gla_device_error, sizeof(v), 0, cudaMemcpyDeviceToHost, st));
+  GLA_CUDA(cudaStreamSynchronize(st));
+  if (reset) {
+    const unsigned int zero = 0;
+    GLA_CUDA(cudaMemcpyToSymbolAsync(g_gla_device_error, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st));
+    GLA_CUDA(cudaStreamSynchronize(st));
+  }
+  *code = v == 0 ? GLA_OK : (int)v;
+  return GLA_OK;
+}
+
+}  // extern "C"
+
+// Address of the device error latch for kernels in other translation units.
+namespace gla {
+unsigned int* device_error_latch() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_gla_device_error) != cudaSuccess) return nullptr;
+  return static_cast<unsigned int*>(p);
+}
+}  // namespace gla

@@ -1,0 +1,169 @@
+/*
+ * gla.h - C ABI of the B200 (sm_100a) chunkwise Gated Linear Attention library.
+ *
+ * Operators
+ * ---------
+ * GLA (key-gated linear recurrence over a matrix memory, one head):
+ *     S_t = diag(exp g_t) . S_{t-1} + k_t^T v_t ,      o_t = q_t . S_t
+ *   q_t, k_t, g_t in R^dk, v_t in R^dv, S_t in R^{dk x dv}.
+ *   Described in words by "Gated Linear Attention for Efficient Long Sequences" (panels "Core
+ *   move" and "Step-by-step memory update") and by "MS-GLA: Multi-Scale Gated Linear
+ *   Attention ...", section 2.1 (data-dependent forget gate that scales rows of the memory;
+ *   chunkwise training with sequential inter-chunk and parallel intra-chunk work).
+ * GSA (Gated Slot Attention, m memory slots):
+ *     o1 = GLA_v(q, k, phi, g)  (pass 1: gate on the slot axis, which is the value axis)
+ *     p  = softmax over the m slots of o1
+ *     o  = GLA(p, phi, v, g)    (pass 2: keys phi, the same slot gates, now on the key axis)
+ *   "Gated Slot Attention for Efficient Linear-Time Sequence Modeling", abstract (two-layer
+ *   GLA linked via softmax) and "Approach" (two-pass linear attention, per-slot forget gates).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout      Per-token tensors are contiguous [B, H, T, D] (D fastest).  States and their
+ *             gradients (h0, hT, dhT, dh0, S) are contiguous float32 [B, H, rows, cols]:
+ *             GLA [B,H,dk,dv]; GSA pass 1 [B,H,dk,m]; GSA pass 2 [B,H,m,dv].
+ * dtype       GLA_DTYPE_BF16: q, k, v, g, phi, o, p and all per-token gradients are bf16;
+ *             arithmetic accumulates in fp32.  GLA_DTYPE_F32: all of them are fp32 and no
+ *             reduced-precision (bf16 or TF32) arithmetic is used anywhere.
+ * Gate        g is the log of the decay (alpha = exp g).  It must be finite and <= 0;
+ *             g = 0 means "keep", very negative g means "forget".  No scale is applied to q.
+ * chunk       Chunk length of the chunkwise algorithm: 16, 32 or 64.  It changes rounding
+ *             only, never the mathematical result.
+ * Tails       T need not be a multiple of chunk.  T == 0 is allowed: per-token pointers may
+ *             then be NULL, hT is set to h0 (or zeros) and dh0 to dhT (or zeros).
+ * Optional    A NULL optional input means zeros (h0, dhT).  A NULL optional output is not
+ *             written (hT, dh0, p_save).
+ * Ownership   The caller owns every buffer, including the workspace; nothing is allocated,
+ *             freed or retained by the library between calls.  Device pointers must be
+ *             16-byte aligned.  Buffers of one call must not overlap, except where stated.
+ * Streams     All work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
+ *             legacy default stream).  Calls return once the work is enqueued.
+ * Workspace   `*_workspace()` returns the bytes the matching call needs for those sizes (0 is
+ *             possible).  Pass at least that many bytes, 256-byte aligned.  The workspace
+ *             contents on entry do not matter; on exit they are unspecified.
+ * Errors      Invalid arguments are rejected before anything is enqueued:
+ *               GLA_ERR_INVALID_ARG   NULL required pointer, negative or zero size where a
+ *                                     positive one is required, misaligned pointer
+ *               GLA_ERR_UNSUPPORTED   dtype, chunk or a dimension outside the supported set
+ *               GLA_ERR_WORKSPACE     workspace NULL or smaller than *_workspace() returned
+ *             A failed kernel launch returns GLA_ERR_CUDA.  Kernels never trap: every wait on
+ *             an mbarrier is bounded, and a wait that runs out records GLA_ERR_TIMEOUT in a
+ *             device-side latch that gla_device_error() reads.
+ * Supported   1 <= dk, dv, m <= 512; dk, dv, m multiples of 8; B*H <= 2^31-1.
+ */
+#ifndef GLA_B200_H
+#define GLA_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GLA_OK = 0,
+  GLA_ERR_INVALID_ARG = 1,
+  GLA_ERR_UNSUPPORTED = 2,
+  GLA_ERR_WORKSPACE = 3,
+  GLA_ERR_CUDA = 4,
+  GLA_ERR_TIMEOUT = 5
+} gla_status;
+
+typedef enum { GLA_DTYPE_F32 = 0, GLA_DTYPE_BF16 = 1 } gla_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* gla_status_string(int status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int gla_version(void);
+
+/* ---------------------------------------------------------------------------------------
+ * gla_chunk_fwd - chunkwise GLA forward.
+ *   in : q, k, g [B,H,T,dk]; v [B,H,T,dv]; h0 [B,H,dk,dv] fp32 (optional, NULL = zeros)
+ *   out: o [B,H,T,dv]; hT = S_T [B,H,dk,dv] fp32 (optional)
+ * Chunkwise form ("MS-GLA", section 2.1): the state is carried chunk to chunk; inside a chunk
+ * the output is the inter-chunk term (q * exp(b)) S_in plus the gated causal intra-chunk term.
+ * ------------------------------------------------------------------------------------- */
+size_t gla_chunk_fwd_workspace(int B, int H, int T, int dk, int dv, int chunk, int dtype);
+int gla_chunk_fwd(const void* q, const void* k, const void* v, const void* g, const float* h0,
+                  void* o, float* hT, int B, int H, int T, int dk, int dv, int chunk, int dtype,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * gla_chunk_bwd - gradients of L(o, hT) for the same inputs as gla_chunk_fwd.
+ *   in : q, k, g, v, h0 (optional) as in gla_chunk_fwd; dO [B,H,T,dv];
+ *        dhT [B,H,dk,dv] fp32 (optional, NULL = zeros)
+ *   out: dq, dk, dg [B,H,T,dk]; dv [B,H,T,dv]; dh0 [B,H,dk,dv] fp32 (optional)
+ * The reverse-mode recurrence is derived from the forward recurrence; dg is the reverse
+ * cumulative sum over t of q*dq - k*dk plus, for every t, sum_j dhT[i,j] hT[i,j].
+ * ------------------------------------------------------------------------------------- */
+size_t gla_chunk_bwd_workspace(int B, int H, int T, int dk, int dv, int chunk, int dtype);
+int gla_chunk_bwd(const void* q, const void* k, const void* v, const void* g, const float* h0,
+                  const void* dO, const float* dhT, void* dq, void* dk, void* dv, void* dg,
+                  float* dh0, int B, int H, int T, int dk_dim, int dv_dim, int chunk, int dtype,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * gla_recurrent_step - one token of recurrent inference, in place on the state.
+ *   in : q, k, g [B,H,dk]; v [B,H,dv]; S [B,H,dk,dv] fp32 (read, then overwritten)
+ *   out: o [B,H,dv];  S <- diag(exp g) S + k^T v ; o = q S
+ * "MS-GLA", section 1 (O(1) inference memory per token).  No workspace.  S may not alias
+ * any other argument.
+ * ------------------------------------------------------------------------------------- */
+int gla_recurrent_step(const void* q, const void* k, const void* v, const void* g, float* S,
+                       void* o, int B, int H, int dk, int dv, int dtype, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * gsa_fwd - Gated Slot Attention forward.
+ *   in : q, k [B,H,T,dk]; v [B,H,T,dv]; phi, g [B,H,T,m] (g: per-slot log forget gate);
+ *        h0_1 [B,H,dk,m], h0_2 [B,H,m,dv] fp32 (optional)
+ *   out: o [B,H,T,dv]; p_save [B,H,T,m] (optional: the slot softmax p, in dtype);
+ *        hT1 [B,H,dk,m], hT2 [B,H,m,dv] fp32 (optional)
+ * ------------------------------------------------------------------------------------- */
+size_t gsa_fwd_workspace(int B, int H, int T, int dk, int dv, int m, int chunk, int dtype);
+int gsa_fwd(const void* q, const void* k, const void* v, const void* phi, const void* g,
+            const float* h0_1, const float* h0_2, void* o, void* p_save, float* hT1, float* hT2,
+            int B, int H, int T, int dk, int dv, int m, int chunk, int dtype, void* workspace,
+            size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * gsa_bwd - gradients of L(o, hT1, hT2) for the inputs of gsa_fwd.
+ *   in : as gsa_fwd, plus dO [B,H,T,dv]; dhT1 [B,H,dk,m], dhT2 [B,H,m,dv] fp32 (optional)
+ *   out: dq, dk [B,H,T,dk]; dv [B,H,T,dv]; dphi, dg [B,H,T,m];
+ *        dh0_1 [B,H,dk,m], dh0_2 [B,H,m,dv] fp32 (optional)
+ * Pass 2 is differentiated first, then the softmax Jacobian do1 = p * (dp - <p, dp>), then
+ * pass 1; dphi and dg sum the contributions of both passes.
+ * ------------------------------------------------------------------------------------- */
+size_t gsa_bwd_workspace(int B, int H, int T, int dk, int dv, int m, int chunk, int dtype);
+int gsa_bwd(const void* q, const void* k, const void* v, const void* phi, const void* g,
+            const float* h0_1, const float* h0_2, const void* dO, const float* dhT1,
+            const float* dhT2, void* dq, void* dk, void* dv, void* dphi, void* dg, float* dh0_1,
+            float* dh0_2, int B, int H, int T, int dk_dim, int dv_dim, int m, int chunk,
+            int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * gsa_recurrent_step - one token of GSA recurrent inference, in place on both states.
+ *   in : q, k [B,H,dk]; v [B,H,dv]; phi, g [B,H,m];
+ *        S1 [B,H,dk,m], S2 [B,H,m,dv] fp32 (read, then overwritten)
+ *   out: o [B,H,dv]
+ *   S1 <- S1 diag(exp g) + k^T phi ; p = softmax(q S1) ; S2 <- diag(exp g) S2 + phi^T v ;
+ *   o = p S2.  "Gated Slot Attention ...", abstract (efficient recurrent inference with a
+ *   small state).  No workspace.
+ * ------------------------------------------------------------------------------------- */
+int gsa_recurrent_step(const void* q, const void* k, const void* v, const void* phi,
+                       const void* g, float* S1, float* S2, void* o, int B, int H, int dk,
+                       int dv, int m, int dtype, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * gla_device_error - read (and optionally clear) the device-side error latch.
+ * Synchronises `stream`, then stores GLA_OK or the first error a kernel recorded since the
+ * last reset (GLA_ERR_TIMEOUT: a bounded wait ran out) in *code.  Returns GLA_ERR_CUDA if
+ * the copy fails, GLA_ERR_INVALID_ARG if code is NULL, else GLA_OK.
+ * ------------------------------------------------------------------------------------- */
+int gla_device_error(void* stream, int reset, int* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GLA_B200_H */

@@ -1,0 +1,97 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every function the
+header declares, answers workspace queries, and rejects invalid arguments before any launch."""
+import ctypes
+
+import pytest
+
+from chunkwise_linear_rnn_02_b200 import binding
+from chunkwise_linear_rnn_02_b200.build_lib import build
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+P = 0x7F0000000000  # a 16-byte aligned fake device address: never dereferenced by these tests
+BAD = P + 8         # misaligned
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load_library()
+
+
+def test_every_header_symbol_is_exported(lib):
+    names = binding.header_symbols()
+    expected = {"gla_status_string", "gla_version", "gla_chunk_fwd_workspace", "gla_chunk_fwd",
+                "gla_chunk_bwd_workspace", "gla_chunk_bwd", "gla_recurrent_step", "gsa_fwd_workspace",
+                "gsa_fwd", "gsa_bwd_workspace", "gsa_bwd", "gsa_recurrent_step", "gla_device_error"}
+    assert expected <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in binding._SIGNATURES, n
+
+
+def test_status_strings_and_version(lib):
+    for code in range(6):
+        assert binding.status_string(code).startswith("GLA_")
+    assert "unknown" in binding.status_string(99)
+    assert lib.gla_version() >= 10000
+
+
+def _fwd(lib, q=P, k=P, v=P, g=P, h0=None, o=P, hT=None, B=1, H=1, T=64, dk=64, dv=64, chunk=64, dtype=1,
+         ws=P, nb=1 << 40):
+    return lib.gla_chunk_fwd(q, k, v, g, h0, o, hT, B, H, T, dk, dv, chunk, dtype, ws, nb, None)
+
+
+def test_fwd_argument_checks(lib):
+    assert _fwd(lib, q=None) == INVALID
+    assert _fwd(lib, o=None) == INVALID
+    assert _fwd(lib, k=BAD) == INVALID
+    assert _fwd(lib, h0=BAD) == INVALID
+    assert _fwd(lib, B=0) == INVALID
+    assert _fwd(lib, T=-1) == INVALID
+    assert _fwd(lib, dk=0) == INVALID
+    assert _fwd(lib, dk=12) == UNSUPPORTED
+    assert _fwd(lib, dv=1024) == UNSUPPORTED
+    assert _fwd(lib, chunk=48) == UNSUPPORTED
+    assert _fwd(lib, dtype=7) == UNSUPPORTED
+    need = lib.gla_chunk_fwd_workspace(1, 1, 64, 64, 64, 64, 1)
+    assert need > 0
+    assert _fwd(lib, ws=None) == WORKSPACE
+    assert _fwd(lib, nb=need - 1) == WORKSPACE
+    assert _fwd(lib, ws=BAD) == WORKSPACE
+
+
+def test_bwd_and_gsa_argument_checks(lib):
+    # every call below is invalid: none may reach a launch with these fake pointers
+    args = [P] * 5 + [P, None] + [P] * 4 + [None]
+    bad = list(args)
+    bad[8] = None  # dv output missing
+    assert lib.gla_chunk_bwd(*bad, 1, 1, 64, 64, 64, 64, 1, P, 1 << 40, None) == INVALID
+    assert lib.gla_chunk_bwd(*args, 1, 1, 64, 64, 64, 64, 1, P, 8, None) == WORKSPACE
+    g11 = [P] * 5 + [None, None, P, None, None, None]
+    assert lib.gsa_fwd(*g11, 1, 1, 64, 64, 64, 20, 64, 1, P, 1 << 40, None) == UNSUPPORTED
+    assert lib.gsa_fwd(*g11, 1, 1, 64, 64, 64, 0, 64, 1, P, 1 << 40, None) == INVALID
+    assert lib.gsa_fwd(*g11, 1, 1, 64, 64, 64, 64, 64, 1, P, 16, None) == WORKSPACE
+    assert lib.gla_recurrent_step(P, P, P, P, None, P, 1, 1, 64, 64, 1, None) == INVALID
+    assert lib.gla_recurrent_step(P, P, P, P, P, P, 1, 1, 64, 64, 3, None) == UNSUPPORTED
+    assert lib.gsa_recurrent_step(P, P, P, P, P, P, BAD, P, 1, 1, 64, 64, 64, 1, None) == INVALID
+    assert lib.gla_device_error(None, 0, None) == INVALID
+
+
+def test_workspace_queries(lib):
+    # generic passes: fp32 per-chunk states (and, for bwd, state gradients, db and hT)
+    B, H, T, dk, dv, C = 2, 3, 130, 64, 128, 64
+    NC = 3
+    fwd_f32 = lib.gla_chunk_fwd_workspace(B, H, T, dk, dv, C, 0)
+    assert fwd_f32 >= B * H * NC * dk * dv * 4
+    assert fwd_f32 % 256 == 0
+    assert lib.gla_chunk_bwd_workspace(B, H, T, dk, dv, C, 0) >= 2 * fwd_f32
+    assert lib.gla_chunk_fwd_workspace(B, H, 0, dk, dv, C, 1) == 0
+    assert lib.gla_chunk_fwd_workspace(B, H, T, 7, dv, C, 1) == 0
+    assert lib.gsa_bwd_workspace(B, H, T, dk, dv, 64, C, 1) > lib.gsa_fwd_workspace(B, H, T, dk, dv, 64, C, 1)
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 1, 8, 8)
+    with pytest.raises(binding.GLAError):
+        binding.chunk_fwd(x, x, x, x)

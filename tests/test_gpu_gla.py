@@ -1,0 +1,133 @@
+"""GPU parity of the GLA entry points against the fp64 oracle at sizes the oracle finishes in
+seconds: several tiles in every dimension, ragged tails, all chunk sizes, both dtypes, and the
+degenerate cases (T = 0, T = 1, T < chunk, a near-reset gate, zero gate)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from chunkwise_linear_rnn_02_b200 import binding as gla
+from chunkwise_linear_rnn_02_b200.inputs import make_gla_inputs
+from helpers import assert_close, cuda, f64, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_fwd_bwd(inp, chunk, with_state=True, check_bwd=True):
+    dt = inp["q"].dtype
+    tol = tol_for(dt)
+    d = cuda(inp)
+    h0 = d.get("h0") if with_state else None
+    dhT = d.get("dhT") if with_state else None
+    o, hT = gla.chunk_fwd(d["q"], d["k"], d["v"], d["g"], h0=h0, chunk=chunk)
+    ro, rhT = O.gla_fwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]),
+                        f64(inp["h0"]) if h0 is not None else None)
+    errs = {"o": assert_close("o", o, ro, tol), "hT": assert_close("hT", hT, rhT, tol)}
+    if check_bwd:
+        dq, dk, dv, dg, dh0 = gla.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["do"], h0=h0, dhT=dhT, chunk=chunk)
+        ref = O.gla_bwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]),
+                        f64(inp["h0"]) if h0 is not None else None, f64(inp["do"]),
+                        f64(inp["dhT"]) if dhT is not None else None)
+        for name, x, r in zip(["dq", "dk", "dv", "dg", "dh0"], [dq, dk, dv, dg, dh0], ref):
+            errs[name] = assert_close(name, x, r, tol)
+    torch.cuda.synchronize()
+    assert gla.device_error() == 0
+    return errs
+
+
+def test_config_fwd_fp32_small():
+    """B=1, H=2, T=256, d_k=d_v=64, chunk 64, fp32: o and hT within 1e-4."""
+    inp = make_gla_inputs(1, 2, 256, 64, 64, torch.float32, seed=0, with_do=False)
+    _run_fwd_bwd(inp, 64, with_state=False, check_bwd=False)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("shape", [(2, 2, 200, 128, 192), (1, 3, 77, 64, 64), (1, 1, 130, 24, 40)])
+def test_fwd_bwd_multi_tile_ragged(dtype, shape):
+    B, H, T, dk, dv = shape
+    inp = make_gla_inputs(B, H, T, dk, dv, dtype, seed=1, with_h0=True, with_dhT=True)
+    _run_fwd_bwd(inp, 64)
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_every_chunk_size_gives_the_same_result(chunk):
+    inp = make_gla_inputs(1, 2, 100, 64, 64, torch.float32, seed=2, with_h0=True, with_dhT=True)
+    _run_fwd_bwd(inp, chunk)
+
+
+@pytest.mark.parametrize("T", [1, 5, 63, 64, 65])
+def test_short_sequences(T):
+    inp = make_gla_inputs(2, 1, T, 64, 128, torch.float32, seed=3, with_h0=True, with_dhT=True)
+    _run_fwd_bwd(inp, 64)
+
+
+def test_empty_sequence():
+    B, H, dk, dv = 2, 2, 64, 64
+    z = torch.empty(B, H, 0, dk, device="cuda")
+    h0 = torch.randn(B, H, dk, dv, device="cuda")
+    o, hT = gla.chunk_fwd(z, z, torch.empty(B, H, 0, dv, device="cuda"), z, h0=h0)
+    assert o.shape == (B, H, 0, dv)
+    torch.testing.assert_close(hT, h0, rtol=0, atol=0)
+    dq, dk_, dv_, dg, dh0 = gla.chunk_bwd(z, z, torch.empty(B, H, 0, dv, device="cuda"), z,
+                                          torch.empty(B, H, 0, dv, device="cuda"), h0=h0, dhT=h0)
+    torch.testing.assert_close(dh0, h0, rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_near_reset_and_zero_gates(dtype):
+    inp = make_gla_inputs(1, 2, 150, 64, 64, dtype, seed=4, with_h0=True, with_dhT=True)
+    inp["g"] = torch.full_like(inp["g"], -30.0)
+    _run_fwd_bwd(inp, 64)
+    inp["g"] = torch.zeros_like(inp["g"])
+    _run_fwd_bwd(inp, 64)
+
+
+@pytest.mark.parametrize("mu", [-2.0, 0.0, 3.0])
+def test_gate_bias_sweep_bf16(mu):
+    inp = make_gla_inputs(1, 2, 192, 128, 128, torch.bfloat16, seed=5, gate_mu=mu)
+    _run_fwd_bwd(inp, 64, with_state=False)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_steps_continue_chunked_forward(dtype):
+    B, H, T, n, dk, dv = 1, 2, 130, 20, 64, 128
+    inp = make_gla_inputs(B, H, T + n, dk, dv, dtype, seed=6, with_do=False)
+    d = cuda(inp)
+    o_full, hT_full = gla.chunk_fwd(d["q"], d["k"], d["v"], d["g"])
+    _, S = gla.chunk_fwd(d["q"][:, :, :T].contiguous(), d["k"][:, :, :T].contiguous(),
+                         d["v"][:, :, :T].contiguous(), d["g"][:, :, :T].contiguous())
+    steps = []
+    for t in range(T, T + n):
+        steps.append(gla.recurrent_step(d["q"][:, :, t].contiguous(), d["k"][:, :, t].contiguous(),
+                                        d["v"][:, :, t].contiguous(), d["g"][:, :, t].contiguous(), S))
+    ro, rhT = O.gla_fwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]))
+    tol = tol_for(dtype)
+    assert_close("decode o", torch.stack(steps, 2), ro[:, :, T:], tol)
+    assert_close("decode S", S, rhT, tol)
+    assert_close("chunked o", o_full[:, :, T:], ro[:, :, T:], tol)
+    assert_close("chunked hT", hT_full, rhT, tol)
+
+
+def test_decode_step_matches_oracle_step():
+    B, H, dk, dv = 2, 2, 64, 96
+    gen = torch.Generator().manual_seed(7)
+    q, k, g = (torch.randn(B, H, dk, generator=gen) for _ in range(3))
+    g = -torch.nn.functional.softplus(g)
+    v = torch.randn(B, H, dv, generator=gen)
+    S0 = torch.randn(B, H, dk, dv, generator=gen)
+    S = S0.cuda()
+    o = gla.recurrent_step(q.cuda(), k.cuda(), v.cuda(), g.cuda(), S)
+    ro, rS = O.gla_decode_step(f64(q), f64(k), f64(v), f64(g), f64(S0))
+    assert_close("o", o, ro, 1e-5)
+    assert_close("S", S, rS, 1e-5)
+
+
+def test_deterministic_repeat():
+    inp = cuda(make_gla_inputs(2, 2, 300, 128, 256, torch.bfloat16, seed=8))
+    a = gla.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"])
+    b = gla.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"])
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    ga = gla.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["do"])
+    gb = gla.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["do"])
+    for x, y in zip(ga, gb):
+        assert torch.equal(x, y)

@@ -1,0 +1,57 @@
+"""GPU parity of the GSA entry points (two GLA passes joined by a slot softmax) against the
+fp64 oracle, at small sizes with ragged tails, both dtypes, and the GSA decode step."""
+import pytest
+import torch
+
+import oracle as O
+from chunkwise_linear_rnn_02_b200 import binding as gla
+from chunkwise_linear_rnn_02_b200.inputs import make_gsa_inputs
+from helpers import assert_close, cuda, f64, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+def _states(B, H, dk, dv, m, seed):
+    gen = torch.Generator().manual_seed(seed)
+    return [torch.randn(s, generator=gen) * 0.5 for s in
+            [(B, H, dk, m), (B, H, m, dv), (B, H, dk, m), (B, H, m, dv)]]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("shape", [(1, 2, 130, 64, 64, 32), (2, 1, 70, 128, 64, 64)])
+def test_gsa_fwd_bwd(dtype, shape):
+    B, H, T, dk, dv, m = shape
+    tol = tol_for(dtype)
+    inp = make_gsa_inputs(B, H, T, dk, dv, m, dtype, seed=11)
+    h1, h2, d1, d2 = _states(B, H, dk, dv, m, 12)
+    d = cuda(inp)
+    o, p, hT1, hT2 = gla.gsa_fwd(d["q"], d["k"], d["v"], d["phi"], d["g"], h0_1=h1.cuda(), h0_2=h2.cuda(),
+                                 save_p=True)
+    a = [f64(inp[n]) for n in ["q", "k", "v", "phi", "g"]]
+    ro, rp, rhT1, rhT2 = O.gsa_fwd(*a, f64(h1), f64(h2))
+    assert_close("o", o, ro, tol)
+    assert_close("p", p, rp, tol)
+    assert_close("hT1", hT1, rhT1, tol)
+    assert_close("hT2", hT2, rhT2, tol)
+    grads = gla.gsa_bwd(d["q"], d["k"], d["v"], d["phi"], d["g"], d["do"], h0_1=h1.cuda(), h0_2=h2.cuda(),
+                        dhT1=d1.cuda(), dhT2=d2.cuda())
+    ref = O.gsa_bwd(*a, f64(h1), f64(h2), f64(inp["do"]), f64(d1), f64(d2))
+    for name, x, r in zip(["dq", "dk", "dv", "dphi", "dg", "dh0_1", "dh0_2"], grads, ref):
+        assert_close(name, x, r, tol)
+    assert gla.device_error() == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_gsa_decode_continues_forward(dtype):
+    B, H, T, n, dk, dv, m = 1, 2, 100, 12, 64, 64, 32
+    inp = make_gsa_inputs(B, H, T + n, dk, dv, m, dtype, seed=13, with_do=False)
+    d = cuda(inp)
+    sl = {k: v[:, :, :T].contiguous() for k, v in d.items()}
+    _, _, S1, S2 = gla.gsa_fwd(sl["q"], sl["k"], sl["v"], sl["phi"], sl["g"])
+    outs = [gla.gsa_recurrent_step(*(d[nm][:, :, t].contiguous() for nm in ["q", "k", "v", "phi", "g"]), S1, S2)
+            for t in range(T, T + n)]
+    ro, _, rhT1, rhT2 = O.gsa_fwd(*(f64(inp[nm]) for nm in ["q", "k", "v", "phi", "g"]))
+    tol = tol_for(dtype)
+    assert_close("o", torch.stack(outs, 2), ro[:, :, T:], tol)
+    assert_close("S1", S1, rhT1, tol)
+    assert_close("S2", S2, rhT2, tol)
