@@ -1,15 +1,481 @@
-// Fused sm_100a chunkwise kernels: not yet covering any shape; every call takes the generic path.
+// Fused sm_100a chunkwise GLA kernels (bf16 in, fp32 accumulate, chunk 64).
+//
+// Forward, one CTA per (head, 64 value columns); the CTA walks the chunks of its head in order
+// and keeps the recurrent state on chip ("MS-GLA ...", section 2.1: sequential inter-chunk
+// updates, parallel intra-chunk work; "Gated Linear Attention for Efficient Long Sequences":
+// chunking with on-chip reuse so that only inputs and outputs cross HBM).
+//
+// Per chunk of 64 tokens, with alpha_t = e^{g_t}, E1_j = prod_{t<=j} alpha_t = e^{B_j} and
+// E2_j = prod_{t>j} alpha_t = e^{gamma - B_j} (B_j the inclusive cumulative log-gate of the chunk,
+// gamma = B_63), everything is built from ONE exponential per (token, key dimension):
+//
+//   gate math (CUDA cores; each thread owns 2 adjacent key dimensions and a run of tokens):
+//     Qs = q E1 / e^{gamma} = q e^{B - gamma}     Kh = k E2 = k e^{gamma - B}
+//   tcgen05.mma (operands in shared memory, accumulators in TMEM):
+//     A   = Qs Kh^T                   [64 x 64]   = sum_d q_jd k_rd e^{B_jd - B_rd}, masked to r <= j
+//     O   = Qs (e^{gamma} S_i)        [64 x 64]   = (q e^{B}) S_i  (state copy pre-scaled by e^{gamma})
+//     dS  = Kh^T V                    [dk x 64]
+//     O  += A V
+//   state (fp32 registers, one thread per row d):   S_{i+1} = e^{gamma} S_i + dS
+//
+// Qs carries e^{B - gamma} <= e^{|gamma|}; it stays finite (and e^{gamma} S_i stays normal) while
+// the chunk keeps at least e^-80 of its state in every key dimension.  A chunk below that bound
+// (near-reset gates) switches to a safe form for that chunk: Qs = q e^{B} with an unscaled state
+// copy, and the intra-chunk matrix recomputed exactly in fp32 from e^{B_j - B_r} (r <= j).
+//
+// Operand layouts are the 128-byte-swizzled forms described in sm100.cuh; V comes straight from a
+// TMA tile load and serves as the MN-major B operand of two MMAs; Kh, stored [token][dim], is the
+// K-major B operand of A and the MN-major A operand of dS.
+#include <cudaTypedefs.h>
+#include <stdlib.h>
+#include <string.h>
+
 #include "fast_path.cuh"
+#include "sm100.cuh"
 
 namespace gla {
 namespace fast {
 
-bool fwd_supported(int, int, int, int, int, int) { return false; }
+using namespace sm100;
+
+constexpr int C = 64;        // chunk length
+constexpr int DVT = 64;      // value columns per CTA
+constexpr int NTHREADS = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kMinDecay = 1.8e-35f;  // e^-80: smallest chunk decay handled by the scaled form
+
+// ------------------------------------------------------------------------------------------
+// Host: tensor maps
+// ------------------------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D map over a [BH, T, D] bf16 tensor with box (box_d, 64 tokens, 1 head).
+static bool make_map(CUtensorMap* m, const void* base, int BH, int T, int D, int box_d, bool swizzle128) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  memset(m, 0, sizeof(*m));
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2 * (cuuint64_t)T};
+  cuuint32_t box[3] = {(cuuint32_t)box_d, (cuuint32_t)C, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static bool force_generic() {
+  const char* e = getenv("GLA_B200_GENERIC");
+  return e && e[0] && e[0] != '0';
+}
+
+// ------------------------------------------------------------------------------------------
+// Device helpers
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ float bf2f(const uint8_t* p) {
+  return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p)) << 16);
+}
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// Store 64 fp32 values as one swizzled 128-byte bf16 row r of a tile at `tile`.
+__device__ __forceinline__ void store_row_sw128(uint8_t* tile, int r, const float* v) {
+#pragma unroll
+  for (int cc = 0; cc < 8; ++cc) {
+    uint4 w;
+    w.x = pack2(v[8 * cc + 0], v[8 * cc + 1]);
+    w.y = pack2(v[8 * cc + 2], v[8 * cc + 3]);
+    w.z = pack2(v[8 * cc + 4], v[8 * cc + 5]);
+    w.w = pack2(v[8 * cc + 6], v[8 * cc + 7]);
+    *reinterpret_cast<uint4*>(tile + r * 128 + ((cc ^ (r & 7)) << 4)) = w;
+  }
+}
+__device__ __forceinline__ void store_row_sw128_scaled(uint8_t* tile, int r, const float* v, float s) {
+#pragma unroll
+  for (int cc = 0; cc < 8; ++cc) {
+    uint4 w;
+    w.x = pack2(s * v[8 * cc + 0], s * v[8 * cc + 1]);
+    w.y = pack2(s * v[8 * cc + 2], s * v[8 * cc + 3]);
+    w.z = pack2(s * v[8 * cc + 4], s * v[8 * cc + 5]);
+    w.w = pack2(s * v[8 * cc + 6], s * v[8 * cc + 7]);
+    *reinterpret_cast<uint4*>(tile + r * 128 + ((cc ^ (r & 7)) << 4)) = w;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Forward kernel
+// ------------------------------------------------------------------------------------------
+template <int DK>
+struct FwdLayout {
+  static constexpr int NPAIR = DK / 2;                      // dimension pairs
+  static constexpr int NSPLIT = NTHREADS / NPAIR;           // token runs per chunk
+  static constexpr int TS = C / NSPLIT;                     // tokens per run
+  static constexpr uint32_t RAW = C * DK * 2;               // one raw q / k / g tile
+  static constexpr uint32_t RAW_V = C * DVT * 2;            // raw v tile (swizzled)
+  static constexpr uint32_t STAGE = 3 * RAW + RAW_V;
+  static constexpr uint32_t OPS = 2 * STAGE;                // operand area
+  static constexpr uint32_t QS = OPS;                       // Qs [64 x DK]  K-major
+  static constexpr uint32_t KH = QS + C * DK * 2;           // Kh [64 x DK]  K-major B / MN-major A
+  static constexpr uint32_t SB = KH + C * DK * 2;           // scaled state copy [DK x 64] MN-major
+  static constexpr uint32_t AB = SB + DK * DVT * 2;         // A bf16 [64 x 64] K-major
+  static constexpr uint32_t DECAY = AB + C * C * 2;         // float[DK]       e^{gamma_d}
+  static constexpr uint32_t TOT = DECAY + DK * 4;           // float[NSPLIT][DK] run products
+  static constexpr uint32_t TOT_END = TOT + NSPLIT * DK * 4;
+  // Safe-mode scratch, used only after the first MMA group of a chunk has completed: fp32
+  // cumulative log-gates [64 x DK] over QS..KH, then the exact A [64 x 64] fp32 right after
+  // them when that still fits before AB, else in a region of its own.
+  static constexpr bool AEX_INSIDE = C * DK * 4 + C * C * 4 <= AB - QS;
+  static constexpr uint32_t AEX = AEX_INSIDE ? QS + C * DK * 4 : TOT_END;
+  static constexpr uint32_t TOTAL = AEX_INSIDE ? TOT_END : TOT_END + C * C * 4;
+  static constexpr uint32_t ALLOC = TOTAL + 1024;           // slack for 1024-byte alignment
+  static_assert(NSPLIT * NPAIR == NTHREADS && C % NSPLIT == 0, "thread split");
+  static_assert(STAGE % 1024 == 0 && RAW % 1024 == 0, "stage alignment");
+  static_assert(ALLOC <= 227 * 1024, "shared memory");
+  static_assert(C * DK * 4 <= AB - QS, "safe-mode gate scratch fits before AB");
+};
+
+template <int DK>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    fwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
+                     const float* __restrict__ h0, __nv_bfloat16* __restrict__ o, float* __restrict__ hT, int T,
+                     int DV, unsigned int* latch) {
+  using L = FwdLayout<DK>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_load[2], bar_mma1, bar_mma2;
+  __shared__ uint32_t tmem_base_sh;
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int dv0 = blockIdx.x * DVT, bh = blockIdx.y;
+  const int NC = (T + C - 1) / C;
+  float* decay_sm = reinterpret_cast<float*>(sm + L::DECAY);
+  float* tot_sm = reinterpret_cast<float*>(sm + L::TOT);
+
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, 256);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_g);
+    prefetch_tmap(&tm_v);
+    mbar_init(&bar_load[0], 1);
+    mbar_init(&bar_load[1], 1);
+    mbar_init(&bar_mma1, 1);
+    mbar_init(&bar_mma2, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue_load = [&](int chunk) {
+    const int s = chunk & 1;
+    uint8_t* st = sm + s * L::STAGE;
+    mbar_arrive_expect_tx(&bar_load[s], L::STAGE);
+    tma_load_3d(st, &tm_q, &bar_load[s], 0, chunk * C, bh);
+    tma_load_3d(st + L::RAW, &tm_k, &bar_load[s], 0, chunk * C, bh);
+    tma_load_3d(st + 2 * L::RAW, &tm_g, &bar_load[s], 0, chunk * C, bh);
+    tma_load_3d(st + 3 * L::RAW, &tm_v, &bar_load[s], dv0, chunk * C, bh);
+  };
+  if (tid == 0) {
+    issue_load(0);
+    if (NC > 1) issue_load(1);
+  }
+
+  // State rows owned by this thread: lane layout of the dS accumulator (M = DK).
+  const bool s_owner = (DK == 128) ? true : (lane < 16);
+  const int s_row = (DK == 128) ? tid : (warp * 16 + lane);
+  float S[DVT];
+#pragma unroll
+  for (int c = 0; c < DVT; ++c) S[c] = 0.f;
+  if (s_owner && h0) {
+    const float4* src = reinterpret_cast<const float4*>(h0 + ((size_t)bh * DK + s_row) * DV + dv0);
+#pragma unroll
+    for (int c = 0; c < DVT / 4; ++c) {
+      const float4 x = src[c];
+      S[4 * c] = x.x;
+      S[4 * c + 1] = x.y;
+      S[4 * c + 2] = x.z;
+      S[4 * c + 3] = x.w;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const uint32_t t_A = tmem, t_O = tmem + 64, t_dS = tmem + 128;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  // gate-math ownership: dimensions (2p, 2p+1), tokens [h*TS, (h+1)*TS)
+  const int gp = tid % L::NPAIR, gh = tid / L::NPAIR;
+  const int gd = 2 * gp;
+  const uint32_t g_blk = (gd >> 6) * (C * 128), g_col = gd & 63;
+
+  for (int i = 0; i < NC; ++i) {
+    const int s = i & 1;
+    uint8_t* st = sm + s * L::STAGE;
+    mbar_wait(&bar_load[s], (i >> 1) & 1, latch);
+
+    // ---------------- gate math: one ex2 per (token, dim); decays from running products -------
+    float a0[L::TS], a1[L::TS];
+    float run0 = 1.f, run1 = 1.f;
+#pragma unroll
+    for (int u = 0; u < L::TS; ++u) {
+      const int j = gh * L::TS + u;
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(st + 2 * L::RAW + (j * DK + gd) * 2);
+      a0[u] = ex2(bf_lo(w) * kLog2e);
+      a1[u] = ex2(bf_hi(w) * kLog2e);
+      run0 *= a0[u];
+      run1 *= a1[u];
+    }
+    tot_sm[gh * DK + gd] = run0;
+    tot_sm[gh * DK + gd + 1] = run1;
+    __syncthreads();
+    float pre0 = 1.f, pre1 = 1.f, suf0 = 1.f, suf1 = 1.f;
+#pragma unroll
+    for (int h = 0; h < L::NSPLIT; ++h) {
+      const float t0 = tot_sm[h * DK + gd], t1 = tot_sm[h * DK + gd + 1];
+      if (h < gh) {
+        pre0 *= t0;
+        pre1 *= t1;
+      } else if (h > gh) {
+        suf0 *= t0;
+        suf1 *= t1;
+      }
+    }
+    const float dec0 = pre0 * run0 * suf0, dec1 = pre1 * run1 * suf1;  // e^{gamma}
+    const bool weak = !(dec0 >= kMinDecay && dec1 >= kMinDecay);
+    if (gh == 0) {
+      decay_sm[gd] = dec0;
+      decay_sm[gd + 1] = dec1;
+    }
+    const int safe = __syncthreads_or(weak);
+    {
+      const float inv0 = safe ? 1.f : 1.f / dec0, inv1 = safe ? 1.f : 1.f / dec1;
+      float e0 = pre0, e1 = pre1;  // running E1 (inclusive)
+#pragma unroll
+      for (int u = 0; u < L::TS; ++u) {
+        const int j = gh * L::TS + u;
+        e0 *= a0[u];
+        e1 *= a1[u];
+        const uint32_t wq = *reinterpret_cast<const uint32_t*>(st + (j * DK + gd) * 2);
+        *reinterpret_cast<uint32_t*>(sm + L::QS + g_blk + sw128(j, g_col)) =
+            pack2(bf_lo(wq) * e0 * inv0, bf_hi(wq) * e1 * inv1);
+      }
+      float f0 = suf0, f1 = suf1;  // running E2 (exclusive of the token itself)
+#pragma unroll
+      for (int u = L::TS - 1; u >= 0; --u) {
+        const int j = gh * L::TS + u;
+        const uint32_t wk = *reinterpret_cast<const uint32_t*>(st + L::RAW + (j * DK + gd) * 2);
+        *reinterpret_cast<uint32_t*>(sm + L::KH + g_blk + sw128(j, g_col)) =
+            pack2(bf_lo(wk) * f0, bf_hi(wk) * f1);
+        f0 *= a0[u];
+        f1 *= a1[u];
+      }
+    }
+    // ---------------- state copy for the inter-chunk term: e^{gamma} S_i (or S_i in safe mode) ----
+    if (s_owner) store_row_sw128_scaled(sm + L::SB, s_row, S, safe ? 1.f : decay_sm[s_row]);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---------------- MMA group 1: A, O = Qs S', dS = Kh^T V ----------------
+    if (tid == 0) {
+      const uint32_t base = smem_u32(sm);
+      const uint32_t vbase = base + s * L::STAGE + 3 * L::RAW;
+      constexpr uint32_t id_A = idesc_bf16_f32(C, C, false, false);
+      constexpr uint32_t id_O = idesc_bf16_f32(C, DVT, false, true);
+      constexpr uint32_t id_S = idesc_bf16_f32(DK, DVT, true, true);
+#pragma unroll
+      for (int k = 0; k < DK / 16; ++k) {
+        const uint32_t koff = (k >> 2) * (C * 128) + (k & 3) * 32;
+        umma_bf16(t_A, desc_sw128(base + L::QS + koff, 16, 1024), desc_sw128(base + L::KH + koff, 16, 1024), id_A,
+                  k > 0);
+      }
+#pragma unroll
+      for (int k = 0; k < DK / 16; ++k) {
+        const uint32_t koff = (k >> 2) * (C * 128) + (k & 3) * 32;
+        umma_bf16(t_O, desc_sw128(base + L::QS + koff, 16, 1024), desc_sw128(base + L::SB + k * 2048, 16, 1024),
+                  id_O, k > 0);
+      }
+#pragma unroll
+      for (int k = 0; k < C / 16; ++k)
+        umma_bf16(t_dS, desc_sw128(base + L::KH + k * 2048, C * 128, 1024), desc_sw128(vbase + k * 2048, 16, 1024),
+                  id_S, k > 0);
+      umma_commit(&bar_mma1);
+    }
+    __syncwarp();
+    mbar_wait(&bar_mma1, i & 1, latch);
+    tc_fence_after();
+
+    // ---------------- safe mode: exact intra-chunk matrix ----------------
+    float* Aex = reinterpret_cast<float*>(sm + L::AEX);  // 64 x 64 fp32
+    if (safe) {
+      float* Bf = reinterpret_cast<float*>(sm + L::QS);  // 64 x DK fp32 cumulative log-gates
+      if (tid < DK) {
+        float b = 0.f;
+        for (int j = 0; j < C; ++j) {
+          b += bf2f(st + 2 * L::RAW + (j * DK + tid) * 2);
+          Bf[j * DK + tid] = b;
+        }
+      }
+      __syncthreads();
+      for (int e = tid; e < C * C; e += NTHREADS) {
+        const int j = e / C, r = e % C;
+        float acc = 0.f;
+        if (r <= j)
+          for (int d = 0; d < DK; ++d)
+            acc += bf2f(st + (j * DK + d) * 2) * bf2f(st + L::RAW + (r * DK + d) * 2) *
+                   __expf(Bf[j * DK + d] - Bf[r * DK + d]);
+        Aex[e] = acc;
+      }
+      __syncthreads();
+    }
+
+    // ---------------- A epilogue: mask, bf16, store as the K-major A operand ----------------
+    {
+      const int j = warp * 16 + lane;
+      float a[64];
+      tmem_ld32(t_A + lane_off, a);
+      tmem_ld32(t_A + lane_off + 32, a + 32);
+      tmem_ld_wait();
+      if (lane < 16) {
+        if (safe) {
+#pragma unroll
+          for (int r = 0; r < 64; ++r) a[r] = Aex[j * C + r];
+        }
+#pragma unroll
+        for (int r = 0; r < 64; ++r)
+          if (r > j) a[r] = 0.f;
+        store_row_sw128(sm + L::AB, j, a);
+      }
+    }
+    // ---------------- state update: S = e^gamma S + dS (fp32 registers) ----------------
+    {
+      float ds[64];
+      tmem_ld32(t_dS + lane_off, ds);
+      tmem_ld32(t_dS + lane_off + 32, ds + 32);
+      tmem_ld_wait();
+      if (s_owner) {
+        const float dec = decay_sm[s_row];
+#pragma unroll
+        for (int c = 0; c < DVT; ++c) S[c] = dec * S[c] + ds[c];
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---------------- MMA group 2: O += A V ----------------
+    if (tid == 0) {
+      const uint32_t base = smem_u32(sm);
+      const uint32_t vbase = base + s * L::STAGE + 3 * L::RAW;
+      constexpr uint32_t id_O = idesc_bf16_f32(C, DVT, false, true);
+#pragma unroll
+      for (int k = 0; k < C / 16; ++k)
+        umma_bf16(t_O, desc_sw128(base + L::AB + k * 32, 16, 1024), desc_sw128(vbase + k * 2048, 16, 1024), id_O, 1);
+      umma_commit(&bar_mma2);
+    }
+    __syncwarp();
+    mbar_wait(&bar_mma2, i & 1, latch);
+    tc_fence_after();
+
+    // ---------------- O epilogue: bf16 rows straight to global ----------------
+    {
+      const int j = warp * 16 + lane;
+      float ov[64];
+      tmem_ld32(t_O + lane_off, ov);
+      tmem_ld32(t_O + lane_off + 32, ov + 32);
+      tmem_ld_wait();
+      const int t = i * C + j;
+      if (lane < 16 && t < T) {
+        uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * T + t) * DV + dv0);
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint4 w;
+          w.x = pack2(ov[8 * cc + 0], ov[8 * cc + 1]);
+          w.y = pack2(ov[8 * cc + 2], ov[8 * cc + 3]);
+          w.z = pack2(ov[8 * cc + 4], ov[8 * cc + 5]);
+          w.w = pack2(ov[8 * cc + 6], ov[8 * cc + 7]);
+          dst[cc] = w;
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && i + 2 < NC) issue_load(i + 2);
+  }
+
+  if (s_owner && hT) {
+    float4* dst = reinterpret_cast<float4*>(hT + ((size_t)bh * DK + s_row) * DV + dv0);
+#pragma unroll
+    for (int c = 0; c < DVT / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ------------------------------------------------------------------------------------------
+// Host entry points
+// ------------------------------------------------------------------------------------------
+bool fwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype) {
+  if (force_generic()) return false;
+  if (dtype != 1 || chunk != C || T < 1 || BH < 1 || BH > 65535) return false;
+  if (dk != 64 && dk != 128) return false;
+  if (dv % DVT != 0) return false;
+  return encode_fn() != nullptr;
+}
+
 size_t fwd_workspace(int, int, int, int) { return 0; }
-cudaError_t fwd(const void*, const void*, const void*, const void*, const float*, void*, float*, int, int, int, int,
-                void*, cudaStream_t) {
+
+template <int DK>
+static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o,
+                              float* hT, int BH, int T, int dv, cudaStream_t st) {
+  CUtensorMap mq, mk, mg, mv;
+  if (!make_map(&mq, q, BH, T, DK, DK, false) || !make_map(&mk, k, BH, T, DK, DK, false) ||
+      !make_map(&mg, g, BH, T, DK, DK, false) || !make_map(&mv, v, BH, T, dv, DVT, true))
+    return cudaErrorInvalidValue;
+  auto kern = fwd_fused_kernel<DK>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdLayout<DK>::ALLOC);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid(dv / DVT, BH);
+  kern<<<grid, NTHREADS, FwdLayout<DK>::ALLOC, st>>>(mq, mk, mg, mv, h0, static_cast<__nv_bfloat16*>(o), hT, T, dv,
+                                                     device_error_latch());
+  return cudaGetLastError();
+}
+
+cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
+                int BH, int T, int dk, int dv, void*, cudaStream_t st) {
+  if (dk == 64) return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, st);
+  if (dk == 128) return launch_fwd<128>(q, k, v, g, h0, o, hT, BH, T, dv, st);
   return cudaErrorNotSupported;
 }
+
 bool bwd_supported(int, int, int, int, int, int) { return false; }
 size_t bwd_workspace(int, int, int, int) { return 0; }
 cudaError_t bwd(const void*, const void*, const void*, const void*, const float*, const void*, const float*, void*,

@@ -454,7 +454,12 @@ __global__ void __launch_bounds__(NT) bwd_dqdk_kernel(
       if (dk_addend) kk += dk_addend[row + u];
       if (dq) stf(dq + row + u, outq[u]);
       if (dk) stf(dk + row + u, kk);
-      if (db) db[row + u] = qs[jo * LD + co + u] * outq[u] - ks[jo * LD + co + u] * outk[u];
+      // The r = j = t terms of dq_t and dk_t (dA[t][t] k_t and dA[t][t] q_t) cancel exactly in
+      // q*dq - k*dk; leaving them out avoids cancellation when the gates decay strongly.
+      if (db) {
+        const float a = dAs[jo * (C + 1) + jo], qv = qs[jo * LD + co + u], kv = ks[jo * LD + co + u];
+        db[row + u] = qv * (outq[u] - a * kv) - kv * (outk[u] - a * qv);
+      }
     }
   }
 }

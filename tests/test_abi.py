@@ -36,7 +36,9 @@ def test_status_strings_and_version(lib):
     assert lib.gla_version() >= 10000
 
 
-def _fwd(lib, q=P, k=P, v=P, g=P, h0=None, o=P, hT=None, B=1, H=1, T=64, dk=64, dv=64, chunk=64, dtype=1,
+# fp32 (dtype 0) keeps every call below on the workspace-using path, so that a call which
+# passes the other checks still fails the workspace check and never reaches a launch.
+def _fwd(lib, q=P, k=P, v=P, g=P, h0=None, o=P, hT=None, B=1, H=1, T=64, dk=64, dv=64, chunk=64, dtype=0,
          ws=P, nb=1 << 40):
     return lib.gla_chunk_fwd(q, k, v, g, h0, o, hT, B, H, T, dk, dv, chunk, dtype, ws, nb, None)
 
@@ -53,7 +55,7 @@ def test_fwd_argument_checks(lib):
     assert _fwd(lib, dv=1024) == UNSUPPORTED
     assert _fwd(lib, chunk=48) == UNSUPPORTED
     assert _fwd(lib, dtype=7) == UNSUPPORTED
-    need = lib.gla_chunk_fwd_workspace(1, 1, 64, 64, 64, 64, 1)
+    need = lib.gla_chunk_fwd_workspace(1, 1, 64, 64, 64, 64, 0)
     assert need > 0
     assert _fwd(lib, ws=None) == WORKSPACE
     assert _fwd(lib, nb=need - 1) == WORKSPACE
@@ -65,12 +67,12 @@ def test_bwd_and_gsa_argument_checks(lib):
     args = [P] * 5 + [P, None] + [P] * 4 + [None]
     bad = list(args)
     bad[8] = None  # dv output missing
-    assert lib.gla_chunk_bwd(*bad, 1, 1, 64, 64, 64, 64, 1, P, 1 << 40, None) == INVALID
-    assert lib.gla_chunk_bwd(*args, 1, 1, 64, 64, 64, 64, 1, P, 8, None) == WORKSPACE
+    assert lib.gla_chunk_bwd(*bad, 1, 1, 64, 64, 64, 64, 0, P, 1 << 40, None) == INVALID
+    assert lib.gla_chunk_bwd(*args, 1, 1, 64, 64, 64, 64, 0, P, 8, None) == WORKSPACE
     g11 = [P] * 5 + [None, None, P, None, None, None]
     assert lib.gsa_fwd(*g11, 1, 1, 64, 64, 64, 20, 64, 1, P, 1 << 40, None) == UNSUPPORTED
     assert lib.gsa_fwd(*g11, 1, 1, 64, 64, 64, 0, 64, 1, P, 1 << 40, None) == INVALID
-    assert lib.gsa_fwd(*g11, 1, 1, 64, 64, 64, 64, 64, 1, P, 16, None) == WORKSPACE
+    assert lib.gsa_fwd(*g11, 1, 1, 64, 64, 64, 64, 64, 0, P, 16, None) == WORKSPACE
     assert lib.gla_recurrent_step(P, P, P, P, None, P, 1, 1, 64, 64, 1, None) == INVALID
     assert lib.gla_recurrent_step(P, P, P, P, P, P, 1, 1, 64, 64, 3, None) == UNSUPPORTED
     assert lib.gsa_recurrent_step(P, P, P, P, P, P, BAD, P, 1, 1, 64, 64, 64, 1, None) == INVALID
