@@ -26,130 +26,43 @@
 // Operand layouts are the 128-byte-swizzled forms described in sm100.cuh; V comes straight from a
 // TMA tile load and serves as the MN-major B operand of two MMAs; Kh, stored [token][dim], is the
 // K-major B operand of A and the MN-major A operand of dS.
-#include <cudaTypedefs.h>
-#include <stdlib.h>
-#include <string.h>
-
 #include "fast_path.cuh"
-#include "sm100.cuh"
+#include "fused_common.cuh"
 
 namespace gla {
 namespace fast {
 
 using namespace sm100;
 
-constexpr int C = 64;        // chunk length
 constexpr int DVT = 64;      // value columns per CTA
 constexpr int NTHREADS = 128;
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kMinDecay = 1.8e-35f;  // e^-80: smallest chunk decay handled by the scaled form
-
-// ------------------------------------------------------------------------------------------
-// Host: tensor maps
-// ------------------------------------------------------------------------------------------
-static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// 3-D map over a [BH, T, D] bf16 tensor with box (box_d, 64 tokens, 1 head).
-static bool make_map(CUtensorMap* m, const void* base, int BH, int T, int D, int box_d, bool swizzle128) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  memset(m, 0, sizeof(*m));
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2 * (cuuint64_t)T};
-  cuuint32_t box[3] = {(cuuint32_t)box_d, (cuuint32_t)C, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-static bool force_generic() {
-  const char* e = getenv("GLA_B200_GENERIC");
-  return e && e[0] && e[0] != '0';
-}
-
-// ------------------------------------------------------------------------------------------
-// Device helpers
-// ------------------------------------------------------------------------------------------
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-__device__ __forceinline__ float bf2f(const uint8_t* p) {
-  return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p)) << 16);
-}
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-// Store 64 fp32 values as one swizzled 128-byte bf16 row r of a tile at `tile`.
-__device__ __forceinline__ void store_row_sw128(uint8_t* tile, int r, const float* v) {
-#pragma unroll
-  for (int cc = 0; cc < 8; ++cc) {
-    uint4 w;
-    w.x = pack2(v[8 * cc + 0], v[8 * cc + 1]);
-    w.y = pack2(v[8 * cc + 2], v[8 * cc + 3]);
-    w.z = pack2(v[8 * cc + 4], v[8 * cc + 5]);
-    w.w = pack2(v[8 * cc + 6], v[8 * cc + 7]);
-    *reinterpret_cast<uint4*>(tile + r * 128 + ((cc ^ (r & 7)) << 4)) = w;
-  }
-}
-__device__ __forceinline__ void store_row_sw128_scaled(uint8_t* tile, int r, const float* v, float s) {
-#pragma unroll
-  for (int cc = 0; cc < 8; ++cc) {
-    uint4 w;
-    w.x = pack2(s * v[8 * cc + 0], s * v[8 * cc + 1]);
-    w.y = pack2(s * v[8 * cc + 2], s * v[8 * cc + 3]);
-    w.z = pack2(s * v[8 * cc + 4], s * v[8 * cc + 5]);
-    w.w = pack2(s * v[8 * cc + 6], s * v[8 * cc + 7]);
-    *reinterpret_cast<uint4*>(tile + r * 128 + ((cc ^ (r & 7)) << 4)) = w;
-  }
-}
 
 // ------------------------------------------------------------------------------------------
 // Forward kernel
 // ------------------------------------------------------------------------------------------
 template <int DK>
 struct FwdLayout {
-  static constexpr int NPAIR = DK / 2;                      // dimension pairs
-  static constexpr int NSPLIT = NTHREADS / NPAIR;           // token runs per chunk
-  static constexpr int TS = C / NSPLIT;                     // tokens per run
   static constexpr uint32_t RAW = C * DK * 2;               // one raw q / k / g tile
   static constexpr uint32_t RAW_V = C * DVT * 2;            // raw v tile (swizzled)
   static constexpr uint32_t STAGE = 3 * RAW + RAW_V;
   static constexpr uint32_t OPS = 2 * STAGE;                // operand area
-  static constexpr uint32_t QS = OPS;                       // Qs [64 x DK]  K-major
-  static constexpr uint32_t KH = QS + C * DK * 2;           // Kh [64 x DK]  K-major B / MN-major A
-  static constexpr uint32_t SB = KH + C * DK * 2;           // scaled state copy [DK x 64] MN-major
-  static constexpr uint32_t AB = SB + DK * DVT * 2;         // A bf16 [64 x 64] K-major
-  static constexpr uint32_t DECAY = AB + C * C * 2;         // float[DK]       e^{gamma_d}
+  static constexpr uint32_t QS_HI = OPS;                    // Qs hi / lo [64 x DK]  K-major
+  static constexpr uint32_t QS_LO = QS_HI + C * DK * 2;
+  static constexpr uint32_t KH = QS_LO + C * DK * 2;        // Kh [64 x DK]  K-major B / MN-major A
+  static constexpr uint32_t SB_HI = KH + C * DK * 2;        // scaled state copy hi / lo [DK x 64] MN-major
+  static constexpr uint32_t SB_LO = SB_HI + DK * DVT * 2;
+  static constexpr uint32_t AB_HI = SB_LO + DK * DVT * 2;   // A hi / lo [64 x 64] K-major
+  static constexpr uint32_t AB_LO = AB_HI + C * C * 2;
+  static constexpr uint32_t DECAY = AB_LO + C * C * 2;      // float[DK]       e^{gamma_d}
   static constexpr uint32_t TOT = DECAY + DK * 4;           // float[NSPLIT][DK] run products
-  static constexpr uint32_t TOT_END = TOT + NSPLIT * DK * 4;
-  // Safe-mode scratch, used only after the first MMA group of a chunk has completed: fp32
-  // cumulative log-gates [64 x DK] over QS..KH, then the exact A [64 x 64] fp32 right after
-  // them when that still fits before AB, else in a region of its own.
-  static constexpr bool AEX_INSIDE = C * DK * 4 + C * C * 4 <= AB - QS;
-  static constexpr uint32_t AEX = AEX_INSIDE ? QS + C * DK * 4 : TOT_END;
-  static constexpr uint32_t TOTAL = AEX_INSIDE ? TOT_END : TOT_END + C * C * 4;
+  static constexpr uint32_t TOTAL = TOT + GateRun<DK, NTHREADS>::NSPLIT * DK * 4;
   static constexpr uint32_t ALLOC = TOTAL + 1024;           // slack for 1024-byte alignment
-  static_assert(NSPLIT * NPAIR == NTHREADS && C % NSPLIT == 0, "thread split");
+  // Exact-path scratch, used after the first MMA group of a chunk has completed: fp32
+  // cumulative log-gates [64 x DK] over QS_HI..QS_LO, exact A [64 x 64] fp32 over KH..SB_HI.
+  static constexpr uint32_t XB = QS_HI, XA = KH;
   static_assert(STAGE % 1024 == 0 && RAW % 1024 == 0, "stage alignment");
   static_assert(ALLOC <= 227 * 1024, "shared memory");
-  static_assert(C * DK * 4 <= AB - QS, "safe-mode gate scratch fits before AB");
+  static_assert(C * DK * 4 <= KH - QS_HI && C * C * 4 <= SB_LO - KH, "exact-path scratch");
 };
 
 template <int DK>
@@ -159,6 +72,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                      const float* __restrict__ h0, __nv_bfloat16* __restrict__ o, float* __restrict__ hT, int T,
                      int DV, unsigned int* latch) {
   using L = FwdLayout<DK>;
+  using Gate = GateRun<DK, NTHREADS>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_load[2], bar_mma1, bar_mma2;
   __shared__ uint32_t tmem_base_sh;
@@ -224,10 +138,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = tmem_base_sh;
   const uint32_t t_A = tmem, t_O = tmem + 64, t_dS = tmem + 128;
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  // gate-math ownership: dimensions (2p, 2p+1), tokens [h*TS, (h+1)*TS)
-  const int gp = tid % L::NPAIR, gh = tid / L::NPAIR;
-  const int gd = 2 * gp;
-  const uint32_t g_blk = (gd >> 6) * (C * 128), g_col = gd & 63;
 
   for (int i = 0; i < NC; ++i) {
     const int s = i & 1;
@@ -235,64 +145,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_wait(&bar_load[s], (i >> 1) & 1, latch);
 
     // ---------------- gate math: one ex2 per (token, dim); decays from running products -------
-    float a0[L::TS], a1[L::TS];
-    float run0 = 1.f, run1 = 1.f;
-#pragma unroll
-    for (int u = 0; u < L::TS; ++u) {
-      const int j = gh * L::TS + u;
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(st + 2 * L::RAW + (j * DK + gd) * 2);
-      a0[u] = ex2(bf_lo(w) * kLog2e);
-      a1[u] = ex2(bf_hi(w) * kLog2e);
-      run0 *= a0[u];
-      run1 *= a1[u];
-    }
-    tot_sm[gh * DK + gd] = run0;
-    tot_sm[gh * DK + gd + 1] = run1;
-    __syncthreads();
-    float pre0 = 1.f, pre1 = 1.f, suf0 = 1.f, suf1 = 1.f;
-#pragma unroll
-    for (int h = 0; h < L::NSPLIT; ++h) {
-      const float t0 = tot_sm[h * DK + gd], t1 = tot_sm[h * DK + gd + 1];
-      if (h < gh) {
-        pre0 *= t0;
-        pre1 *= t1;
-      } else if (h > gh) {
-        suf0 *= t0;
-        suf1 *= t1;
-      }
-    }
-    const float dec0 = pre0 * run0 * suf0, dec1 = pre1 * run1 * suf1;  // e^{gamma}
-    const bool weak = !(dec0 >= kMinDecay && dec1 >= kMinDecay);
-    if (gh == 0) {
-      decay_sm[gd] = dec0;
-      decay_sm[gd + 1] = dec1;
+    Gate gr;
+    const bool weak = gr.run(st + 2 * L::RAW, DK, tot_sm);
+    if (gr.h == 0) {
+      decay_sm[gr.d] = gr.dec0;
+      decay_sm[gr.d + 1] = gr.dec1;
     }
     const int safe = __syncthreads_or(weak);
     {
-      const float inv0 = safe ? 1.f : 1.f / dec0, inv1 = safe ? 1.f : 1.f / dec1;
-      float e0 = pre0, e1 = pre1;  // running E1 (inclusive)
-#pragma unroll
-      for (int u = 0; u < L::TS; ++u) {
-        const int j = gh * L::TS + u;
-        e0 *= a0[u];
-        e1 *= a1[u];
-        const uint32_t wq = *reinterpret_cast<const uint32_t*>(st + (j * DK + gd) * 2);
-        *reinterpret_cast<uint32_t*>(sm + L::QS + g_blk + sw128(j, g_col)) =
-            pack2(bf_lo(wq) * e0 * inv0, bf_hi(wq) * e1 * inv1);
-      }
-      float f0 = suf0, f1 = suf1;  // running E2 (exclusive of the token itself)
-#pragma unroll
-      for (int u = L::TS - 1; u >= 0; --u) {
-        const int j = gh * L::TS + u;
-        const uint32_t wk = *reinterpret_cast<const uint32_t*>(st + L::RAW + (j * DK + gd) * 2);
-        *reinterpret_cast<uint32_t*>(sm + L::KH + g_blk + sw128(j, g_col)) =
-            pack2(bf_lo(wk) * f0, bf_hi(wk) * f1);
-        f0 *= a0[u];
-        f1 *= a1[u];
-      }
+      const float inv0 = safe ? 1.f : 1.f / gr.dec0, inv1 = safe ? 1.f : 1.f / gr.dec1;
+      const uint32_t blk = (gr.d >> 6) * (C * 128), col = gr.d & 63;
+      gr.forward([&](int j, float e0, float e1) {
+        const uint32_t wq = *reinterpret_cast<const uint32_t*>(st + (j * DK + gr.d) * 2);
+        uint32_t hi, lo;
+        split2(bf_lo(wq) * e0 * inv0, bf_hi(wq) * e1 * inv1, hi, lo);
+        *reinterpret_cast<uint32_t*>(sm + L::QS_HI + blk + sw128(j, col)) = hi;
+        *reinterpret_cast<uint32_t*>(sm + L::QS_LO + blk + sw128(j, col)) = lo;
+      });
+      gr.backward([&](int j, float e0, float e1) {
+        const uint32_t wk = *reinterpret_cast<const uint32_t*>(st + L::RAW + (j * DK + gr.d) * 2);
+        *reinterpret_cast<uint32_t*>(sm + L::KH + blk + sw128(j, col)) = pack2(bf_lo(wk) * e0, bf_hi(wk) * e1);
+      });
     }
     // ---------------- state copy for the inter-chunk term: e^{gamma} S_i (or S_i in safe mode) ----
-    if (s_owner) store_row_sw128_scaled(sm + L::SB, s_row, S, safe ? 1.f : decay_sm[s_row]);
+    if (s_owner) store_row_split(sm + L::SB_HI, sm + L::SB_LO, s_row, S, safe ? 1.f : decay_sm[s_row]);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -308,14 +184,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
       for (int k = 0; k < DK / 16; ++k) {
         const uint32_t koff = (k >> 2) * (C * 128) + (k & 3) * 32;
-        umma_bf16(t_A, desc_sw128(base + L::QS + koff, 16, 1024), desc_sw128(base + L::KH + koff, 16, 1024), id_A,
-                  k > 0);
+        const uint64_t kd = desc_sw128(base + L::KH + koff, 16, 1024);
+        umma_bf16(t_A, desc_sw128(base + L::QS_HI + koff, 16, 1024), kd, id_A, k > 0);
+        umma_bf16(t_A, desc_sw128(base + L::QS_LO + koff, 16, 1024), kd, id_A, 1);
       }
 #pragma unroll
       for (int k = 0; k < DK / 16; ++k) {
         const uint32_t koff = (k >> 2) * (C * 128) + (k & 3) * 32;
-        umma_bf16(t_O, desc_sw128(base + L::QS + koff, 16, 1024), desc_sw128(base + L::SB + k * 2048, 16, 1024),
-                  id_O, k > 0);
+        const uint64_t qh = desc_sw128(base + L::QS_HI + koff, 16, 1024);
+        const uint64_t sh = desc_sw128(base + L::SB_HI + k * 2048, 16, 1024);
+        umma_bf16(t_O, qh, sh, id_O, k > 0);
+        umma_bf16(t_O, qh, desc_sw128(base + L::SB_LO + k * 2048, 16, 1024), id_O, 1);
+        umma_bf16(t_O, desc_sw128(base + L::QS_LO + koff, 16, 1024), sh, id_O, 1);
       }
 #pragma unroll
       for (int k = 0; k < C / 16; ++k)
@@ -328,9 +208,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
 
     // ---------------- safe mode: exact intra-chunk matrix ----------------
-    float* Aex = reinterpret_cast<float*>(sm + L::AEX);  // 64 x 64 fp32
+    float* Aex = reinterpret_cast<float*>(sm + L::XA);  // 64 x 64 fp32
     if (safe) {
-      float* Bf = reinterpret_cast<float*>(sm + L::QS);  // 64 x DK fp32 cumulative log-gates
+      float* Bf = reinterpret_cast<float*>(sm + L::XB);  // 64 x DK fp32 cumulative log-gates
       if (tid < DK) {
         float b = 0.f;
         for (int j = 0; j < C; ++j) {
@@ -351,7 +231,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __syncthreads();
     }
 
-    // ---------------- A epilogue: mask, bf16, store as the K-major A operand ----------------
+    // ---------------- A epilogue: mask, hi/lo bf16, store as the K-major A operand ----------------
     {
       const int j = warp * 16 + lane;
       float a[64];
@@ -366,7 +246,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int r = 0; r < 64; ++r)
           if (r > j) a[r] = 0.f;
-        store_row_sw128(sm + L::AB, j, a);
+        store_row_split(sm + L::AB_HI, sm + L::AB_LO, j, a, 1.f);
       }
     }
     // ---------------- state update: S = e^gamma S + dS (fp32 registers) ----------------
@@ -392,8 +272,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t vbase = base + s * L::STAGE + 3 * L::RAW;
       constexpr uint32_t id_O = idesc_bf16_f32(C, DVT, false, true);
 #pragma unroll
-      for (int k = 0; k < C / 16; ++k)
-        umma_bf16(t_O, desc_sw128(base + L::AB + k * 32, 16, 1024), desc_sw128(vbase + k * 2048, 16, 1024), id_O, 1);
+      for (int k = 0; k < C / 16; ++k) {
+        const uint64_t vd = desc_sw128(vbase + k * 2048, 16, 1024);
+        umma_bf16(t_O, desc_sw128(base + L::AB_HI + k * 32, 16, 1024), vd, id_O, 1);
+        umma_bf16(t_O, desc_sw128(base + L::AB_LO + k * 32, 16, 1024), vd, id_O, 1);
+      }
       umma_commit(&bar_mma2);
     }
     __syncwarp();
@@ -408,18 +291,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tmem_ld32(t_O + lane_off + 32, ov + 32);
       tmem_ld_wait();
       const int t = i * C + j;
-      if (lane < 16 && t < T) {
-        uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * T + t) * DV + dv0);
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          uint4 w;
-          w.x = pack2(ov[8 * cc + 0], ov[8 * cc + 1]);
-          w.y = pack2(ov[8 * cc + 2], ov[8 * cc + 3]);
-          w.z = pack2(ov[8 * cc + 4], ov[8 * cc + 5]);
-          w.w = pack2(ov[8 * cc + 6], ov[8 * cc + 7]);
-          dst[cc] = w;
-        }
-      }
+      if (lane < 16 && t < T) store_row_global_bf16(o + ((size_t)bh * T + t) * DV + dv0, ov);
     }
     tc_fence_before();
     __syncthreads();
@@ -473,13 +345,6 @@ cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, cons
                 int BH, int T, int dk, int dv, void*, cudaStream_t st) {
   if (dk == 64) return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, st);
   if (dk == 128) return launch_fwd<128>(q, k, v, g, h0, o, hT, BH, T, dv, st);
-  return cudaErrorNotSupported;
-}
-
-bool bwd_supported(int, int, int, int, int, int) { return false; }
-size_t bwd_workspace(int, int, int, int) { return 0; }
-cudaError_t bwd(const void*, const void*, const void*, const void*, const float*, const void*, const float*, void*,
-                void*, void*, void*, float*, int, int, int, int, void*, cudaStream_t) {
   return cudaErrorNotSupported;
 }
 

@@ -1,0 +1,868 @@
+// Fused sm_100a chunkwise GLA backward (bf16 in, fp32 accumulate, chunk 64, d_k = 128).
+//
+// Reverse-mode of the chunkwise recurrence.  With G_{i+1} = dL/dS at the end of chunk i
+// (G_N = dhT), per chunk (B_j the inclusive cumulative log-gate, gamma = B_63, E1 = e^{B},
+// E2 = e^{gamma - B}, dec = e^{gamma}, Kh = k E2, Qt = q E1, Qs = Qt / dec):
+//
+//   dA  = mask(dO V^T)                        A = mask(Qs Kh^T)
+//   dq  = E1 (dO S_i^T) + (E1 / dec) (dA Kh)
+//   dk  = E2 (V G_{i+1}^T) + (E2 / dec) (dA^T Qt)
+//   dv  = Kh G_{i+1} + A^T dO
+//   G_i = dec G_{i+1} + Qt^T dO               S_{i+1} = dec S_i + Kh^T V
+//   db  = q (dq - dA_jj k) - k (dk - dA_jj q) ;  dg_t = sum_{s>=t} db_s + rowsum(dhT * hT)
+//
+// (the dA_jj terms of dq_j and dk_j cancel exactly in q dq - k dk and are left out of db).
+//
+// One launch, two kinds of CTA, all resident at once:
+//   * key-tile CTAs, one per (head, 64 key dimensions): a forward walk that rebuilds S on chip
+//     and writes dq, then a reverse walk that carries G on chip and writes dk, dg and dh0 (dg
+//     needs dq, which it reads back with TMA);
+//   * value-tile CTAs, one per (head, 128 value columns): one reverse walk carrying G[:, tile]
+//     that writes dv.
+// States live in TMEM as fp32 accumulators; their bf16 copies in shared memory feed the MMAs.
+// A chunk that keeps less than e^-40 of its state in some dimension computes its intra-chunk
+// terms exactly in fp32 (CUDA cores) instead of through the scaled operands.
+#include "fast_path.cuh"
+#include "fused_common.cuh"
+
+namespace gla {
+namespace fast {
+
+using namespace sm100;
+
+constexpr int BT = 128;  // threads per CTA
+constexpr int KT = 64;   // key dimensions per key-tile CTA
+constexpr int VT = 128;  // value columns per value-tile CTA
+
+struct BwdMaps {
+  CUtensorMap v, dO;                 // box (64 cols, 64 tokens), 128-byte swizzle
+  CUtensorMap k64, g64, q64;         // box (64 dims, 64 tokens), plain
+  CUtensorMap q_all, k_all, g_all;   // box (DK dims, 64 tokens), plain
+};
+
+struct BwdArgs {
+  const float* h0;
+  const float* dhT;
+  __nv_bfloat16 *dq, *dk, *dv, *dg;
+  float* dh0;
+  float* ws_qx;    // [BH][NC][DK] chunk sums of Qt X
+  float* ws_part;  // [BH][T][DK] forward-walk part of dg
+  int T, n_key_ctas;
+  unsigned int* latch;
+};
+
+// ------------------------------------------------------------------------------------------
+// Key-tile CTA
+//
+// Gate gradient, evaluated chunk by chunk so that rounding never accumulates over the sequence:
+// for token t at local position tau of chunk i (Qt = q E1, Kh = k E2, X = dO S_i^T, Z = V G_{i+1}^T),
+//   dg_t = c_i + sum_{r<tau} Kh_r Z_r + sum_{j>=tau} Qt_j X_j
+//              + sum_{r<tau} ( k_r dk^intra_r - q_r dq^intra_r )        (intra terms without j = r)
+//   c_i  = e^{gamma_i} rowsum(G_{i+1} * S_i), carried backwards over chunk boundaries as
+//   c_{N-1} = rowsum(dhT * hT) - sum_r (Kh Z)_{N-1},  c_i = c_{i+1} + sum_j (Qt X)_{i+1} - sum_r (Kh Z)_i.
+// The forward walk writes the Qt X and q dq^intra parts (chunk-local, fp32) and the chunk sums of
+// Qt X into the workspace; the reverse walk adds the rest.  The chunk sums use Qt and Kh exactly as
+// the G and S updates see them (bf16 hi + lo), so the recurrence for c telescopes exactly for the
+// states the kernel carries and its rounding does not accumulate over chunks.  Because the four
+// parts of dg are several times larger than dg, every MMA operand of this CTA is a bf16 hi + lo
+// pair (three products per MMA), which keeps them near fp32 accuracy.  The state copies feeding X and Z
+// are split into bf16 hi + lo parts, because the chunk sums they produce are carried over the
+// whole sequence.
+// ------------------------------------------------------------------------------------------
+template <int DK, int DV>
+struct KeyLayout {
+  static constexpr uint32_t VB = C * DV * 2;        // a v or dO tile [64 x DV] (DV/64 swizzled boxes)
+  static constexpr uint32_t TILE = C * KT * 2;      // a [64 x 64] bf16 tile
+  static constexpr uint32_t PA_V = 0, PA_DO = VB;   // part A: v, dO
+  static constexpr uint32_t PB = 2 * VB;            // part B: k, g, q tiles
+  static constexpr uint32_t PB_K = PB, PB_G = PB + TILE, PB_Q = PB + 2 * TILE;
+  static constexpr uint32_t KQ_HI = PB + 3 * TILE; // Kh (forward walk) / Qt (reverse walk), hi / lo
+  static constexpr uint32_t KQ_LO = KQ_HI + TILE;
+  static constexpr uint32_t SG_HI = KQ_LO + TILE;   // bf16 hi / lo copies of S or G rows [64 x DV], K-major
+  static constexpr uint32_t SG_LO = SG_HI + KT * DV * 2;
+  static constexpr uint32_t DA_HI = SG_LO + KT * DV * 2;  // masked dA, bf16 hi / lo [64 x 64]
+  static constexpr uint32_t DA_LO = DA_HI + TILE;
+  static constexpr uint32_t EF = DA_LO + TILE;      // fp32 [64][64]: E1 / E2, then a per-token term
+  static constexpr uint32_t SCR = EF + C * KT * 4;  // fp32 [64][64]: a per-token term
+  static constexpr uint32_t DEC = SCR + C * KT * 4;
+  static constexpr uint32_t TOT = DEC + KT * 4;     // [4][64]
+  static constexpr uint32_t DIAG = TOT + 4 * KT * 4;
+  static constexpr uint32_t CARRY = DIAG + C * 4;
+  static constexpr uint32_t TOTAL = CARRY + KT * 4;
+  // exact-path scratch (only when the part-A prefetch is held back): B and dA in fp32
+  static constexpr uint32_t XB = PA_V, XA = PA_DO;
+  // TMEM columns
+  static constexpr uint32_t T_SG = 0, T_DA = DV, T_X = DV + 64, T_Y = DV + 128;
+  static_assert(VB >= C * KT * 4, "exact-path scratch fits in a part-A tile");
+  static_assert(DV + 192 <= 512, "TMEM columns");
+};
+
+template <int DK, int DV>
+__device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int tau, uint64_t* bars,
+                              uint32_t tmem) {
+  using L = KeyLayout<DK, DV>;
+  using Gate = GateRun<KT, BT>;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int T = a.T, NC = (T + C - 1) / C, d0 = tau * KT;
+  const uint32_t base = smem_u32(sm);
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const bool row_owner = lane < 16;
+  const int row = warp * 16 + lane;  // row of an M=64 accumulator owned by this thread
+  uint64_t* bar_pa = bars + 0;
+  uint64_t* bar_pb = bars + 1;
+  uint64_t* bar_m1 = bars + 3;
+  uint64_t* bar_m2 = bars + 4;
+  uint32_t ph_pa = 0, ph_pb = 0, ph_m1 = 0, ph_m2 = 0;
+  float* DEC = reinterpret_cast<float*>(sm + L::DEC);
+  float* TOT = reinterpret_cast<float*>(sm + L::TOT);
+  float* EF = reinterpret_cast<float*>(sm + L::EF);
+  float* SCR = reinterpret_cast<float*>(sm + L::SCR);
+  float* DIAG = reinterpret_cast<float*>(sm + L::DIAG);
+  float* CARRY = reinterpret_cast<float*>(sm + L::CARRY);
+  float* qx_sums = a.ws_qx + (size_t)bh * NC * DK + d0;  // [NC][DK] slice of this head and key tile
+  float* part = a.ws_part + (size_t)bh * T * DK + d0;      // [T][DK] slice: forward-walk part of dg
+
+  auto load_a = [&](int chunk) {
+    mbar_arrive_expect_tx(bar_pa, 2 * L::VB);
+    for (int b = 0; b < DV / 64; ++b) {
+      tma_load_3d(sm + L::PA_V + b * (C * 128), &mp.v, bar_pa, b * 64, chunk * C, bh);
+      tma_load_3d(sm + L::PA_DO + b * (C * 128), &mp.dO, bar_pa, b * 64, chunk * C, bh);
+    }
+  };
+  auto load_b = [&](int chunk) {
+    mbar_arrive_expect_tx(bar_pb, 3 * L::TILE);
+    tma_load_3d(sm + L::PB_K, &mp.k64, bar_pb, d0, chunk * C, bh);
+    tma_load_3d(sm + L::PB_G, &mp.g64, bar_pb, d0, chunk * C, bh);
+    tma_load_3d(sm + L::PB_Q, &mp.q64, bar_pb, d0, chunk * C, bh);
+  };
+  auto sync_tc = [&]() {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  };
+  // Initialise the TMEM state rows and their hi/lo bf16 copies from a [DK x DV] fp32 source (or zeros).
+  auto init_state = [&](const float* src) {
+    float v[64];
+    for (int c0 = 0; c0 < DV; c0 += 64) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c)
+        v[c] = (src && row_owner) ? src[((size_t)bh * DK + d0 + row) * DV + c0 + c] : 0.f;
+      tmem_st32(tmem + L::T_SG + lane_off + c0, v);
+      tmem_st32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
+      if (row_owner)
+        store_row_split(sm + L::SG_HI + (c0 / 64) * (KT * 128), sm + L::SG_LO + (c0 / 64) * (KT * 128), row, v, 1.f);
+    }
+    tmem_st_wait();
+  };
+  // Rescale the TMEM state rows by DEC[row] (all lanes take part; only owners' rows matter).
+  auto rescale_state = [&]() {
+    const float s = row_owner ? DEC[row] : 0.f;
+    float v[32];
+    for (int c0 = 0; c0 < DV; c0 += 32) {
+      tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 32; ++c) v[c] *= s;
+      tmem_st32(tmem + L::T_SG + lane_off + c0, v);
+    }
+    tmem_st_wait();
+  };
+  // Copy the TMEM state rows into the hi/lo bf16 K-major operands.
+  auto copy_state = [&]() {
+    float v[64];
+    for (int c0 = 0; c0 < DV; c0 += 64) {
+      tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
+      tmem_ld32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
+      tmem_ld_wait();
+      if (row_owner)
+        store_row_split(sm + L::SG_HI + (c0 / 64) * (KT * 128), sm + L::SG_LO + (c0 / 64) * (KT * 128), row, v, 1.f);
+    }
+  };
+  // Cumulative log-gates of the key tile, fp32 [64][64], for the exact path.
+  auto exact_gates = [&]() {
+    float* XB = reinterpret_cast<float*>(sm + L::XB);
+    if (tid < KT) {
+      float b = 0.f;
+      for (int j = 0; j < C; ++j) {
+        b += bf2f(sm + L::PB_G + (j * KT + tid) * 2);
+        XB[j * KT + tid] = b;
+      }
+    }
+  };
+  // dA epilogue: masked bf16 operand, its diagonal, and (exact path) an fp32 copy.
+  auto dA_epilogue = [&](int safe) {
+    float v[64];
+    tmem_ld32(tmem + L::T_DA + lane_off, v);
+    tmem_ld32(tmem + L::T_DA + lane_off + 32, v + 32);
+    tmem_ld_wait();
+    if (row_owner) {
+      float diag = 0.f;
+#pragma unroll
+      for (int r = 0; r < 64; ++r) {
+        if (r > row) v[r] = 0.f;
+        if (r == row) diag = v[r];
+      }
+      DIAG[row] = diag;
+      store_row_split(sm + L::DA_HI, sm + L::DA_LO, row, v, 1.f);
+      if (safe) {
+        float* XA = reinterpret_cast<float*>(sm + L::XA);
+#pragma unroll
+        for (int r = 0; r < 64; ++r) XA[row * C + r] = v[r];
+      }
+    }
+  };
+  auto mma_dA = [&](int k, uint32_t ko) {
+    constexpr uint32_t id_dA = idesc_bf16_f32(C, C, false, false);
+    umma_bf16(tmem + L::T_DA, desc_sw128(base + L::PA_DO + ko, 16, 1024), desc_sw128(base + L::PA_V + ko, 16, 1024),
+              id_dA, k > 0);
+  };
+
+  // ============================ forward walk: dq, first part of dg ============================
+  if (tid == 0) {
+    load_a(0);
+    load_b(0);
+  }
+  init_state(a.h0);
+  for (int i = 0; i < NC; ++i) {
+    mbar_wait(bar_pa, ph_pa, a.latch);
+    ph_pa ^= 1;
+    mbar_wait(bar_pb, ph_pb, a.latch);
+    ph_pb ^= 1;
+    Gate gr;
+    const bool weak = gr.run(sm + L::PB_G, KT, TOT);
+    gr.backward([&](int j, float e0, float e1) {
+      const uint32_t wk = *reinterpret_cast<const uint32_t*>(sm + L::PB_K + (j * KT + gr.d) * 2);
+      uint32_t hi, lo;
+      split2(bf_lo(wk) * e0, bf_hi(wk) * e1, hi, lo);
+      *reinterpret_cast<uint32_t*>(sm + L::KQ_HI + sw128(j, gr.d)) = hi;
+      *reinterpret_cast<uint32_t*>(sm + L::KQ_LO + sw128(j, gr.d)) = lo;
+    });
+    gr.forward([&](int j, float e0, float e1) {
+      *reinterpret_cast<float2*>(EF + j * KT + gr.d) = make_float2(e0, e1);
+    });
+    if (gr.h == 0) {
+      DEC[gr.d] = gr.dec0;
+      DEC[gr.d + 1] = gr.dec1;
+    }
+    const int safe = __syncthreads_or(weak);
+    rescale_state();
+    fence_async_smem();
+    sync_tc();
+    if (tid == 0) {
+      constexpr uint32_t id_X = idesc_bf16_f32(C, KT, false, false);
+      constexpr uint32_t id_S = idesc_bf16_f32(KT, DV, true, true);
+#pragma unroll
+      for (int k = 0; k < DV / 16; ++k) {
+        const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
+        const uint64_t ad = desc_sw128(base + L::PA_DO + ko, 16, 1024);
+        mma_dA(k, ko);
+        umma_bf16(tmem + L::T_X, ad, desc_sw128(base + L::SG_HI + ko, 16, 1024), id_X, k > 0);
+        umma_bf16(tmem + L::T_X, ad, desc_sw128(base + L::SG_LO + ko, 16, 1024), id_X, 1);
+      }
+#pragma unroll
+      for (int k = 0; k < C / 16; ++k) {
+        const uint64_t vd = desc_sw128(base + L::PA_V + k * 2048, C * 128, 1024);
+        umma_bf16(tmem + L::T_SG, desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024), vd, id_S, 1);
+        umma_bf16(tmem + L::T_SG, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), vd, id_S, 1);
+      }
+      umma_commit(bar_m1);
+    }
+    __syncwarp();
+    mbar_wait(bar_m1, ph_m1, a.latch);
+    ph_m1 ^= 1;
+    tc_fence_after();
+    if (tid == 0 && !safe && i + 1 < NC) load_a(i + 1);
+    dA_epilogue(safe);
+    fence_async_smem();
+    sync_tc();
+    if (tid == 0 && !safe) {
+      constexpr uint32_t id_Y = idesc_bf16_f32(C, KT, false, true);
+#pragma unroll
+      for (int k = 0; k < C / 16; ++k) {
+        const uint64_t ah = desc_sw128(base + L::DA_HI + k * 32, 16, 1024);
+        const uint64_t bh = desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024);
+        umma_bf16(tmem + L::T_Y, ah, bh, id_Y, k > 0);
+        umma_bf16(tmem + L::T_Y, ah, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), id_Y, 1);
+        umma_bf16(tmem + L::T_Y, desc_sw128(base + L::DA_LO + k * 32, 16, 1024), bh, id_Y, 1);
+      }
+      umma_commit(bar_m2);
+    }
+    copy_state();
+    if (safe) {
+      exact_gates();
+      __syncthreads();
+    } else {
+      __syncwarp();
+      mbar_wait(bar_m2, ph_m2, a.latch);
+      ph_m2 ^= 1;
+      tc_fence_after();
+    }
+    {  // dq epilogue; per-token terms q e^B X (-> SCR) and q dq^intra without j = r (-> EF)
+      float x[64], y[64];
+      tmem_ld32(tmem + L::T_X + lane_off, x);
+      tmem_ld32(tmem + L::T_X + lane_off + 32, x + 32);
+      if (!safe) {
+        tmem_ld32(tmem + L::T_Y + lane_off, y);
+        tmem_ld32(tmem + L::T_Y + lane_off + 32, y + 32);
+      }
+      tmem_ld_wait();
+      if (row_owner) {
+        const int j = row;
+        float* e1 = EF + j * KT;
+        const float ajj = DIAG[j];
+        if (safe) {
+          const float* XB = reinterpret_cast<const float*>(sm + L::XB);
+          const float* XA = reinterpret_cast<const float*>(sm + L::XA);
+#pragma unroll
+          for (int d = 0; d < 64; ++d) {
+            float acc = 0.f;
+            for (int r = 0; r <= j; ++r)
+              acc += XA[j * C + r] * bf2f(sm + L::PB_K + (r * KT + d) * 2) * __expf(XB[j * KT + d] - XB[r * KT + d]);
+            y[d] = acc;  // exact intra term
+          }
+        } else {
+#pragma unroll
+          for (int d = 0; d < 64; ++d) y[d] *= e1[d] / DEC[d];
+        }
+#pragma unroll
+        for (int d = 0; d < 64; ++d) {
+          const float qv = bf2f(sm + L::PB_Q + (j * KT + d) * 2), kv = bf2f(sm + L::PB_K + (j * KT + d) * 2);
+          const float ev = e1[d];
+          SCR[j * KT + d] = bf_split_sum(qv * ev) * x[d];  // Qt as the G update sees it
+          e1[d] = qv * (y[d] - ajj * kv);
+          x[d] = ev * x[d] + y[d];
+        }
+        const int t = i * C + j;
+        if (t < T) store_row_global_bf16(a.dq + ((size_t)bh * T + t) * DK + d0, x);
+      }
+    }
+    __syncthreads();
+    if (tid < KT) {  // chunk-local parts of dg: suffix of Qt X minus prefix of q dq^intra
+      const int d = tid;
+      float suf = 0.f;
+      for (int j = C - 1; j >= 0; --j) {
+        suf += SCR[j * KT + d];
+        SCR[j * KT + d] = suf;
+      }
+      float pre = 0.f;
+      for (int j = 0; j < C; ++j) {
+        const int t = i * C + j;
+        if (t < T) part[(size_t)t * DK + d] = SCR[j * KT + d] - pre;
+        pre += EF[j * KT + d];
+      }
+      qx_sums[(size_t)i * DK + d] = suf;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      if (safe && i + 1 < NC) load_a(i + 1);
+      if (i + 1 < NC) load_b(i + 1);
+    }
+  }
+
+  // rowsum(dhT * hT): hT rows = the state after the forward walk
+  {
+    float v[32];
+    float acc = 0.f;
+    for (int c0 = 0; c0 < DV; c0 += 32) {
+      tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
+      tmem_ld_wait();
+      if (row_owner && a.dhT) {
+        const float* src = a.dhT + ((size_t)bh * DK + d0 + row) * DV + c0;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) acc += src[c] * v[c];
+      }
+    }
+    if (row_owner) CARRY[row] = acc;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  // ============================ reverse walk: dk, dg, dh0 ============================
+  if (tid == 0) {
+    load_a(NC - 1);
+    load_b(NC - 1);
+  }
+  init_state(a.dhT);
+  for (int n = 0; n < NC; ++n) {
+    const int i = NC - 1 - n;
+    mbar_wait(bar_pa, ph_pa, a.latch);
+    ph_pa ^= 1;
+    mbar_wait(bar_pb, ph_pb, a.latch);
+    ph_pb ^= 1;
+    Gate gr;
+    const bool weak = gr.run(sm + L::PB_G, KT, TOT);
+    gr.forward([&](int j, float e0, float e1) {
+      const uint32_t wq = *reinterpret_cast<const uint32_t*>(sm + L::PB_Q + (j * KT + gr.d) * 2);
+      uint32_t hi, lo;
+      split2(bf_lo(wq) * e0, bf_hi(wq) * e1, hi, lo);
+      *reinterpret_cast<uint32_t*>(sm + L::KQ_HI + sw128(j, gr.d)) = hi;
+      *reinterpret_cast<uint32_t*>(sm + L::KQ_LO + sw128(j, gr.d)) = lo;
+    });
+    gr.backward([&](int j, float e0, float e1) {
+      *reinterpret_cast<float2*>(EF + j * KT + gr.d) = make_float2(e0, e1);
+    });
+    if (gr.h == 0) {
+      DEC[gr.d] = gr.dec0;
+      DEC[gr.d + 1] = gr.dec1;
+    }
+    const int safe = __syncthreads_or(weak);
+    rescale_state();
+    fence_async_smem();
+    sync_tc();
+    if (tid == 0) {
+      constexpr uint32_t id_Z = idesc_bf16_f32(C, KT, false, false);
+      constexpr uint32_t id_G = idesc_bf16_f32(KT, DV, true, true);
+#pragma unroll
+      for (int k = 0; k < DV / 16; ++k) {
+        const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
+        const uint64_t vd = desc_sw128(base + L::PA_V + ko, 16, 1024);
+        mma_dA(k, ko);
+        umma_bf16(tmem + L::T_X, vd, desc_sw128(base + L::SG_HI + ko, 16, 1024), id_Z, k > 0);
+        umma_bf16(tmem + L::T_X, vd, desc_sw128(base + L::SG_LO + ko, 16, 1024), id_Z, 1);
+      }
+#pragma unroll
+      for (int k = 0; k < C / 16; ++k) {
+        const uint64_t dd = desc_sw128(base + L::PA_DO + k * 2048, C * 128, 1024);
+        umma_bf16(tmem + L::T_SG, desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024), dd, id_G, 1);
+        umma_bf16(tmem + L::T_SG, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), dd, id_G, 1);
+      }
+      umma_commit(bar_m1);
+    }
+    __syncwarp();
+    mbar_wait(bar_m1, ph_m1, a.latch);
+    ph_m1 ^= 1;
+    tc_fence_after();
+    if (tid == 0 && !safe && n + 1 < NC) load_a(i - 1);
+    dA_epilogue(safe);
+    fence_async_smem();
+    sync_tc();
+    if (tid == 0 && !safe) {
+      constexpr uint32_t id_W = idesc_bf16_f32(C, KT, true, true);
+#pragma unroll
+      for (int k = 0; k < C / 16; ++k) {
+        const uint64_t ah = desc_sw128(base + L::DA_HI + k * 2048, C * 128, 1024);
+        const uint64_t bh = desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024);
+        umma_bf16(tmem + L::T_Y, ah, bh, id_W, k > 0);
+        umma_bf16(tmem + L::T_Y, ah, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), id_W, 1);
+        umma_bf16(tmem + L::T_Y, desc_sw128(base + L::DA_LO + k * 2048, C * 128, 1024), bh, id_W, 1);
+      }
+      umma_commit(bar_m2);
+    }
+    copy_state();
+    if (safe) {
+      exact_gates();
+      __syncthreads();
+    } else {
+      __syncwarp();
+      mbar_wait(bar_m2, ph_m2, a.latch);
+      ph_m2 ^= 1;
+      tc_fence_after();
+    }
+    {  // dk epilogue; per-token terms Kh Z (-> EF) and Kh Z + k dk^intra without j = r (-> SCR)
+      float z[64], w[64];
+      tmem_ld32(tmem + L::T_X + lane_off, z);
+      tmem_ld32(tmem + L::T_X + lane_off + 32, z + 32);
+      if (!safe) {
+        tmem_ld32(tmem + L::T_Y + lane_off, w);
+        tmem_ld32(tmem + L::T_Y + lane_off + 32, w + 32);
+      }
+      tmem_ld_wait();
+      if (row_owner) {
+        const int r = row;
+        float* e2 = EF + r * KT;
+        const float arr = DIAG[r];
+        if (safe) {
+          const float* XB = reinterpret_cast<const float*>(sm + L::XB);
+          const float* XA = reinterpret_cast<const float*>(sm + L::XA);
+#pragma unroll
+          for (int d = 0; d < 64; ++d) {
+            float acc = 0.f;
+            for (int j = r; j < C; ++j)
+              acc += XA[j * C + r] * bf2f(sm + L::PB_Q + (j * KT + d) * 2) * __expf(XB[j * KT + d] - XB[r * KT + d]);
+            w[d] = acc;
+          }
+        } else {
+#pragma unroll
+          for (int d = 0; d < 64; ++d) w[d] *= e2[d] / DEC[d];
+        }
+#pragma unroll
+        for (int d = 0; d < 64; ++d) {
+          const float qv = bf2f(sm + L::PB_Q + (r * KT + d) * 2), kv = bf2f(sm + L::PB_K + (r * KT + d) * 2);
+          const float ev = e2[d];
+          const float kz = bf_split_sum(kv * ev) * z[d];  // Kh as the S update sees it
+          e2[d] = kz;
+          SCR[r * KT + d] = kz + kv * (w[d] - arr * qv);
+          z[d] = ev * z[d] + w[d];
+        }
+        const int t = i * C + r;
+        if (t < T) store_row_global_bf16(a.dk + ((size_t)bh * T + t) * DK + d0, z);
+      }
+    }
+    __syncthreads();
+    if (tid < KT) {  // dg = c_i + prefix of (Kh Z + k dk^intra) + the forward walk's partial
+      const int d = tid;
+      float kz = 0.f;
+      for (int r = 0; r < C; ++r) kz += EF[r * KT + d];
+      const float ci = (n == 0 ? CARRY[d] : CARRY[d] + qx_sums[(size_t)(i + 1) * DK + d]) - kz;
+      float pre = 0.f;
+      for (int r = 0; r < C; ++r) {
+        const int t = i * C + r;
+        if (t < T)
+          a.dg[((size_t)bh * T + t) * DK + d0 + d] =
+              __float2bfloat16_rn(ci + pre + part[(size_t)t * DK + d]);
+        pre += SCR[r * KT + d];
+      }
+      CARRY[d] = ci;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && n + 1 < NC) {
+      if (safe) load_a(i - 1);
+      load_b(i - 1);
+    }
+  }
+  // dh0 rows = G_0
+  if (a.dh0) {
+    tc_fence_after();
+    float v[32];
+    for (int c0 = 0; c0 < DV; c0 += 32) {
+      tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
+      tmem_ld_wait();
+      if (row_owner) {
+        float4* dst = reinterpret_cast<float4*>(a.dh0 + ((size_t)bh * DK + d0 + row) * DV + c0);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Value-tile CTA: reverse walk carrying G[:, tile] (fp32, TMEM); dv = Kh G_{i+1} + A^T dO.
+// Qs, Kh, the G copy and A enter the MMAs as bf16 hi + lo pairs.  One array holds the queries of
+// both A and the G update: Qs = Qt / dec (then G <- dec (G + Qs^T dO)), or Qt itself in a chunk on
+// the exact path (then G <- dec G + Qt^T dO, the intra-chunk A computed exactly in fp32).
+// ------------------------------------------------------------------------------------------
+template <int DK>
+struct ValLayout {
+  static constexpr uint32_t RAW = C * DK * 2;       // q, k, g [64][DK] row-major
+  static constexpr uint32_t DOT = C * VT * 2;       // dO tile, VT/64 swizzled boxes
+  static constexpr uint32_t STAGE = 3 * RAW + DOT;  // single-buffered
+  static constexpr uint32_t QP_HI = STAGE;          // Qs (or Qt) hi / lo [64 x DK] K-major
+  static constexpr uint32_t QP_LO = QP_HI + C * DK * 2;
+  static constexpr uint32_t KH_HI = QP_LO + C * DK * 2;  // Kh hi / lo [64 x DK] K-major
+  static constexpr uint32_t KH_LO = KH_HI + C * DK * 2;
+  static constexpr uint32_t GC_HI = KH_LO + C * DK * 2;  // G[:, tile] copy hi / lo [DK rows x VT] MN-major
+  static constexpr uint32_t GC_LO = GC_HI + DK * VT * 2;
+  static constexpr uint32_t AB_HI = GC_LO + DK * VT * 2;  // A hi / lo [64 x 64]
+  static constexpr uint32_t AB_LO = AB_HI + C * C * 2;
+  static constexpr uint32_t DEC = AB_LO + C * C * 2;
+  static constexpr uint32_t TOT = DEC + DK * 4;
+  static constexpr uint32_t TOTAL = TOT + GateRun<DK, BT>::NSPLIT * DK * 4;
+  static constexpr uint32_t XB = QP_HI, XA = KH_HI;  // exact-path scratch (after the first MMA group)
+  static constexpr uint32_t T_G = 0, T_A = VT, T_DV = VT + 64;
+  static_assert(STAGE % 1024 == 0, "stage alignment");
+  static_assert(C * DK * 4 <= KH_HI - QP_HI && C * C * 4 <= GC_HI - KH_HI, "exact-path scratch");
+};
+
+template <int DK>
+__device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int vt, int DV,
+                              uint64_t* bars, uint32_t tmem) {
+  using L = ValLayout<DK>;
+  using Gate = GateRun<DK, BT>;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int T = a.T, NC = (T + C - 1) / C, c0 = vt * VT;
+  const uint32_t base = smem_u32(sm);
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const bool row_owner = lane < 16;
+  const int row = warp * 16 + lane;
+  uint64_t* bar_ld = bars + 0;
+  uint64_t* bar_m1 = bars + 3;
+  uint64_t* bar_m2 = bars + 4;
+  uint32_t ph_ld = 0, ph_m1 = 0, ph_m2 = 0;
+  float* DEC = reinterpret_cast<float*>(sm + L::DEC);
+  float* TOT = reinterpret_cast<float*>(sm + L::TOT);
+
+  auto load = [&](int chunk) {
+    mbar_arrive_expect_tx(bar_ld, L::STAGE);
+    tma_load_3d(sm, &mp.q_all, bar_ld, 0, chunk * C, bh);
+    tma_load_3d(sm + L::RAW, &mp.k_all, bar_ld, 0, chunk * C, bh);
+    tma_load_3d(sm + 2 * L::RAW, &mp.g_all, bar_ld, 0, chunk * C, bh);
+    for (int b = 0; b < VT / 64; ++b)
+      tma_load_3d(sm + 3 * L::RAW + b * (C * 128), &mp.dO, bar_ld, c0 + b * 64, chunk * C, bh);
+  };
+  auto sync_tc = [&]() {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  };
+  // G <- DEC[row] * G for this thread's row of the M=128 accumulator.
+  auto rescale_G = [&]() {
+    const float sc = DEC[tid];
+    float v[32];
+    for (int cb = 0; cb < VT; cb += 32) {
+      tmem_ld32(tmem + L::T_G + lane_off + cb, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 32; ++c) v[c] *= sc;
+      tmem_st32(tmem + L::T_G + lane_off + cb, v);
+    }
+    tmem_st_wait();
+  };
+  // G rows (this thread owns row tid of the M=128 accumulator): init from dhT[:, tile]
+  {
+    float v[64];
+    for (int cb = 0; cb < VT; cb += 64) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c) v[c] = a.dhT ? a.dhT[((size_t)bh * DK + tid) * DV + c0 + cb + c] : 0.f;
+      tmem_st32(tmem + L::T_G + lane_off + cb, v);
+      tmem_st32(tmem + L::T_G + lane_off + cb + 32, v + 32);
+      store_row_split(sm + L::GC_HI + (cb / 64) * (DK * 128), sm + L::GC_LO + (cb / 64) * (DK * 128), tid, v, 1.f);
+    }
+    tmem_st_wait();
+  }
+  if (tid == 0) load(NC - 1);
+  for (int n = 0; n < NC; ++n) {
+    const int i = NC - 1 - n;
+    mbar_wait(bar_ld, ph_ld, a.latch);
+    ph_ld ^= 1;
+    Gate gr;
+    const bool weak = gr.run(sm + 2 * L::RAW, DK, TOT);
+    if (gr.h == 0) {
+      DEC[gr.d] = gr.dec0;
+      DEC[gr.d + 1] = gr.dec1;
+    }
+    const int safe = __syncthreads_or(weak);
+    {
+      const float inv0 = safe ? 1.f : 1.f / gr.dec0, inv1 = safe ? 1.f : 1.f / gr.dec1;
+      const uint32_t blk = (gr.d >> 6) * (C * 128), col = gr.d & 63;
+      gr.forward([&](int j, float e0, float e1) {
+        const uint32_t wq = *reinterpret_cast<const uint32_t*>(sm + (j * DK + gr.d) * 2);
+        uint32_t hi, lo;
+        split2(bf_lo(wq) * e0 * inv0, bf_hi(wq) * e1 * inv1, hi, lo);
+        *reinterpret_cast<uint32_t*>(sm + L::QP_HI + blk + sw128(j, col)) = hi;
+        *reinterpret_cast<uint32_t*>(sm + L::QP_LO + blk + sw128(j, col)) = lo;
+      });
+      gr.backward([&](int j, float e0, float e1) {
+        const uint32_t wk = *reinterpret_cast<const uint32_t*>(sm + L::RAW + (j * DK + gr.d) * 2);
+        uint32_t hi, lo;
+        split2(bf_lo(wk) * e0, bf_hi(wk) * e1, hi, lo);
+        *reinterpret_cast<uint32_t*>(sm + L::KH_HI + blk + sw128(j, col)) = hi;
+        *reinterpret_cast<uint32_t*>(sm + L::KH_LO + blk + sw128(j, col)) = lo;
+      });
+    }
+    if (safe) rescale_G();
+    fence_async_smem();
+    sync_tc();
+    if (tid == 0) {
+      const uint32_t dob = base + 3 * L::RAW;
+      constexpr uint32_t id_A = idesc_bf16_f32(C, C, false, false);
+      constexpr uint32_t id_dv = idesc_bf16_f32(C, VT, false, true);
+      constexpr uint32_t id_G = idesc_bf16_f32(DK, VT, true, true);
+#pragma unroll
+      for (int k = 0; k < DK / 16; ++k) {
+        const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
+        const uint64_t qh = desc_sw128(base + L::QP_HI + ko, 16, 1024), ql = desc_sw128(base + L::QP_LO + ko, 16, 1024);
+        const uint64_t kh = desc_sw128(base + L::KH_HI + ko, 16, 1024), kl = desc_sw128(base + L::KH_LO + ko, 16, 1024);
+        umma_bf16(tmem + L::T_A, qh, kh, id_A, k > 0);
+        umma_bf16(tmem + L::T_A, qh, kl, id_A, 1);
+        umma_bf16(tmem + L::T_A, ql, kh, id_A, 1);
+        const uint64_t gh = desc_sw128(base + L::GC_HI + k * 2048, DK * 128, 1024);
+        umma_bf16(tmem + L::T_DV, kh, gh, id_dv, k > 0);
+        umma_bf16(tmem + L::T_DV, kh, desc_sw128(base + L::GC_LO + k * 2048, DK * 128, 1024), id_dv, 1);
+        umma_bf16(tmem + L::T_DV, kl, gh, id_dv, 1);
+      }
+#pragma unroll
+      for (int k = 0; k < C / 16; ++k) {
+        const uint64_t dd = desc_sw128(dob + k * 2048, C * 128, 1024);
+        umma_bf16(tmem + L::T_G, desc_sw128(base + L::QP_HI + k * 2048, C * 128, 1024), dd, id_G, 1);
+        umma_bf16(tmem + L::T_G, desc_sw128(base + L::QP_LO + k * 2048, C * 128, 1024), dd, id_G, 1);
+      }
+      umma_commit(bar_m1);
+    }
+    __syncwarp();
+    mbar_wait(bar_m1, ph_m1, a.latch);
+    ph_m1 ^= 1;
+    tc_fence_after();
+    if (!safe) rescale_G();
+    float* XA = reinterpret_cast<float*>(sm + L::XA);
+    if (safe) {  // exact A = sum_d q_jd k_rd e^{B_jd - B_rd}, r <= j
+      float* XB = reinterpret_cast<float*>(sm + L::XB);
+      if (tid < DK) {
+        float b = 0.f;
+        for (int j = 0; j < C; ++j) {
+          b += bf2f(sm + 2 * L::RAW + (j * DK + tid) * 2);
+          XB[j * DK + tid] = b;
+        }
+      }
+      __syncthreads();
+      for (int e = tid; e < C * C; e += BT) {
+        const int j = e / C, r = e % C;
+        float acc = 0.f;
+        if (r <= j)
+          for (int d = 0; d < DK; ++d)
+            acc += bf2f(sm + (j * DK + d) * 2) * bf2f(sm + L::RAW + (r * DK + d) * 2) *
+                   __expf(XB[j * DK + d] - XB[r * DK + d]);
+        XA[e] = acc;
+      }
+      __syncthreads();
+    }
+    {  // A epilogue
+      float v[64];
+      tmem_ld32(tmem + L::T_A + lane_off, v);
+      tmem_ld32(tmem + L::T_A + lane_off + 32, v + 32);
+      tmem_ld_wait();
+      if (row_owner) {
+        if (safe) {
+#pragma unroll
+          for (int r = 0; r < 64; ++r) v[r] = XA[row * C + r];
+        }
+#pragma unroll
+        for (int r = 0; r < 64; ++r)
+          if (r > row) v[r] = 0.f;
+        store_row_split(sm + L::AB_HI, sm + L::AB_LO, row, v, 1.f);
+      }
+    }
+    {  // hi / lo copy of G_i for the next (earlier) chunk
+      float v[64];
+      for (int cb = 0; cb < VT; cb += 64) {
+        tmem_ld32(tmem + L::T_G + lane_off + cb, v);
+        tmem_ld32(tmem + L::T_G + lane_off + cb + 32, v + 32);
+        tmem_ld_wait();
+        store_row_split(sm + L::GC_HI + (cb / 64) * (DK * 128), sm + L::GC_LO + (cb / 64) * (DK * 128), tid, v, 1.f);
+      }
+    }
+    fence_async_smem();
+    sync_tc();
+    if (tid == 0) {
+      const uint32_t dob = base + 3 * L::RAW;
+      constexpr uint32_t id_dv2 = idesc_bf16_f32(C, VT, true, true);
+#pragma unroll
+      for (int k = 0; k < C / 16; ++k) {
+        const uint64_t dd = desc_sw128(dob + k * 2048, C * 128, 1024);
+        umma_bf16(tmem + L::T_DV, desc_sw128(base + L::AB_HI + k * 2048, C * 128, 1024), dd, id_dv2, 1);
+        umma_bf16(tmem + L::T_DV, desc_sw128(base + L::AB_LO + k * 2048, C * 128, 1024), dd, id_dv2, 1);
+      }
+      umma_commit(bar_m2);
+    }
+    __syncwarp();
+    mbar_wait(bar_m2, ph_m2, a.latch);
+    ph_m2 ^= 1;
+    tc_fence_after();
+    {  // dv epilogue
+      float v[64];
+      const int t = i * C + row;
+      for (int cb = 0; cb < VT; cb += 64) {
+        tmem_ld32(tmem + L::T_DV + lane_off + cb, v);
+        tmem_ld32(tmem + L::T_DV + lane_off + cb + 32, v + 32);
+        tmem_ld_wait();
+        if (row_owner && t < T) store_row_global_bf16(a.dv + ((size_t)bh * T + t) * DV + c0 + cb, v);
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && n + 1 < NC) load(i - 1);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Kernel and host entry points
+// ------------------------------------------------------------------------------------------
+template <int DK, int DV>
+struct BwdSmem {
+  static constexpr uint32_t K = KeyLayout<DK, DV>::TOTAL, V = ValLayout<DK>::TOTAL;
+  static constexpr uint32_t ALLOC = (K > V ? K : V) + 1024;
+  static_assert(ALLOC <= 227 * 1024, "shared memory");
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bars[5];
+  __shared__ uint32_t tmem_base_sh;
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  const int warp = threadIdx.x >> 5;
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < 5; ++b) mbar_init(&bars[b], 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  constexpr int per_head = DK / KT + DV / VT;
+  const int bh = blockIdx.x / per_head, role = blockIdx.x % per_head;
+  if (role < DK / KT)
+    key_tile_body<DK, DV>(sm, mp, a, bh, role, bars, tmem);
+  else
+    val_tile_body<DK>(sm, mp, a, bh, role - DK / KT, DV, bars, tmem);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+bool bwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype) {
+  if (force_generic()) return false;
+  if (dtype != 1 || chunk != C || T < 1 || BH < 1) return false;
+  if (dk != 128 || (dv != 128 && dv != 256)) return false;
+  return encode_fn() != nullptr;
+}
+
+size_t bwd_workspace(int BH, int T, int dk, int) {
+  return align256((size_t)BH * ((T + C - 1) / C) * dk * sizeof(float)) +
+         align256((size_t)BH * T * dk * sizeof(float));
+}
+
+template <int DK, int DV>
+static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* g, const float* h0,
+                              const void* dO, const float* dhT, void* dq, void* dk, void* dv, void* dg, float* dh0,
+                              int BH, int T, void* ws, cudaStream_t st) {
+  BwdMaps mp;
+  if (!make_map(&mp.v, v, BH, T, DV, 64, true) || !make_map(&mp.dO, dO, BH, T, DV, 64, true) ||
+      !make_map(&mp.k64, k, BH, T, DK, KT, false) || !make_map(&mp.g64, g, BH, T, DK, KT, false) ||
+      !make_map(&mp.q64, q, BH, T, DK, KT, false) ||
+      !make_map(&mp.q_all, q, BH, T, DK, DK, false) || !make_map(&mp.k_all, k, BH, T, DK, DK, false) ||
+      !make_map(&mp.g_all, g, BH, T, DK, DK, false))
+    return cudaErrorInvalidValue;
+  BwdArgs a;
+  a.h0 = h0;
+  a.dhT = dhT;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.dg = static_cast<__nv_bfloat16*>(dg);
+  a.dh0 = dh0;
+  a.T = T;
+  a.n_key_ctas = BH * (DK / KT);
+  a.ws_qx = static_cast<float*>(ws);
+  a.ws_part = a.ws_qx + align256((size_t)BH * ((T + C - 1) / C) * DK * sizeof(float)) / sizeof(float);
+  a.latch = device_error_latch();
+  auto kern = bwd_fused_kernel<DK, DV>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<DK, DV>::ALLOC);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int grid = BH * (DK / KT + DV / VT);
+  kern<<<grid, BT, BwdSmem<DK, DV>::ALLOC, st>>>(mp, a);
+  return cudaGetLastError();
+}
+
+cudaError_t bwd(const void* q, const void* k, const void* v, const void* g, const float* h0, const void* dO,
+                const float* dhT, void* dq, void* dk, void* dv, void* dg, float* dh0, int BH, int T, int dkd, int dvd,
+                void* ws, cudaStream_t st) {
+  if (dkd == 128 && dvd == 256) return launch_bwd<128, 256>(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, ws, st);
+  if (dkd == 128 && dvd == 128) return launch_bwd<128, 128>(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, ws, st);
+  return cudaErrorNotSupported;
+}
+
+}  // namespace fast
+}  // namespace gla

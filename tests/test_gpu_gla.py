@@ -161,3 +161,21 @@ def test_fused_forward_is_selected_for_bf16_shapes():
     assert gla.workspace_bytes("gla_chunk_fwd", 8, 4, 2048, 128, 256, 64, 1) == 0
     assert gla.workspace_bytes("gla_chunk_fwd", 1, 1, 100, 64, 64, 64, 1) == 0
     assert gla.workspace_bytes("gla_chunk_fwd", 1, 1, 100, 64, 64, 64, 0) > 0  # fp32: generic passes
+
+
+@pytest.mark.parametrize("dv", [128, 256])
+@pytest.mark.parametrize("T", [1, 40, 64, 150, 300])
+def test_fused_shapes_fwd_bwd(dv, T):
+    """d_k = 128 bf16 shapes served by the fused kernels, with initial and final state gradients."""
+    inp = make_gla_inputs(2, 2, T, 128, dv, torch.bfloat16, seed=20 + T, with_h0=True, with_dhT=True)
+    _run_fwd_bwd(inp, 64)
+
+
+def test_fused_shapes_mixed_strong_gates():
+    """Some chunks keep less than e^-40 of their state (exact fp32 intra-chunk path), others do not."""
+    inp = make_gla_inputs(1, 2, 320, 128, 256, torch.bfloat16, seed=31, with_h0=True, with_dhT=True)
+    g = inp["g"].float()
+    g[:, :, 64:128] -= 2.0      # chunk 1: ~ -128 over the chunk in every dimension
+    g[:, 1, 200:210, :7] = -9.0  # part of chunk 3, a few dimensions
+    inp["g"] = g.to(torch.bfloat16)
+    _run_fwd_bwd(inp, 64)
