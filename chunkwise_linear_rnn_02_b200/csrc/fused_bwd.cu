@@ -36,7 +36,7 @@ constexpr int VT = 128;  // value columns per value-tile CTA
 
 struct BwdMaps {
   CUtensorMap v, dO;                 // box (64 cols, 64 tokens), 128-byte swizzle
-  CUtensorMap k64, g64, q64;         // box (64 dims, 64 tokens), plain
+  CUtensorMap k64, g64, q64;         // box (64 dims, 64 tokens), 128-byte swizzle
   CUtensorMap q_all, k_all, g_all;   // box (DK dims, 64 tokens), plain
 };
 
@@ -82,9 +82,10 @@ struct KeyLayout {
   static constexpr uint32_t SG_LO = SG_HI + KT * DV * 2;
   static constexpr uint32_t DA_HI = SG_LO + KT * DV * 2;  // masked dA, bf16 hi / lo [64 x 64]
   static constexpr uint32_t DA_LO = DA_HI + TILE;
-  static constexpr uint32_t EF = DA_LO + TILE;      // fp32 [64][64]: E1 / E2, then a per-token term
-  static constexpr uint32_t SCR = EF + C * KT * 4;  // fp32 [64][64]: a per-token term
-  static constexpr uint32_t DEC = SCR + C * KT * 4;
+  static constexpr int FS = 66;                     // padded row stride of the fp32 [64][64] scratch
+  static constexpr uint32_t EF = DA_LO + TILE;      // fp32 [64][FS]: E1 / E2, then a per-token term
+  static constexpr uint32_t SCR = EF + C * FS * 4;  // fp32 [64][FS]: a per-token term
+  static constexpr uint32_t DEC = SCR + C * FS * 4;
   static constexpr uint32_t TOT = DEC + KT * 4;     // [4][64]
   static constexpr uint32_t DIAG = TOT + 4 * KT * 4;
   static constexpr uint32_t CARRY = DIAG + C * 4;
@@ -140,6 +141,9 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     __syncthreads();
     tc_fence_after();
   };
+  // Element (token j, dim d) of a raw k / g / q tile (TMA 128-byte swizzle).
+  auto raw = [&](uint32_t tile, int j, int d) { return bf2f(sm + tile + sw128(j, d)); };
+  auto raw2 = [&](uint32_t tile, int j, int d) { return *reinterpret_cast<const uint32_t*>(sm + tile + sw128(j, d)); };
   // Initialise the TMEM state rows and their hi/lo bf16 copies from a [DK x DV] fp32 source (or zeros).
   auto init_state = [&](const float* src) {
     float v[64];
@@ -157,13 +161,15 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   // Rescale the TMEM state rows by DEC[row] (all lanes take part; only owners' rows matter).
   auto rescale_state = [&]() {
     const float s = row_owner ? DEC[row] : 0.f;
-    float v[32];
-    for (int c0 = 0; c0 < DV; c0 += 32) {
+    float v[64];
+    for (int c0 = 0; c0 < DV; c0 += 64) {
       tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
+      tmem_ld32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
       tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < 32; ++c) v[c] *= s;
+      for (int c = 0; c < 64; ++c) v[c] *= s;
       tmem_st32(tmem + L::T_SG + lane_off + c0, v);
+      tmem_st32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
     }
     tmem_st_wait();
   };
@@ -184,7 +190,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     if (tid < KT) {
       float b = 0.f;
       for (int j = 0; j < C; ++j) {
-        b += bf2f(sm + L::PB_G + (j * KT + tid) * 2);
+        b += raw(L::PB_G, j, tid);
         XB[j * KT + tid] = b;
       }
     }
@@ -229,16 +235,16 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     mbar_wait(bar_pb, ph_pb, a.latch);
     ph_pb ^= 1;
     Gate gr;
-    const bool weak = gr.run(sm + L::PB_G, KT, TOT);
+    const bool weak = gr.run_swizzled(sm + L::PB_G, TOT);
     gr.backward([&](int j, float e0, float e1) {
-      const uint32_t wk = *reinterpret_cast<const uint32_t*>(sm + L::PB_K + (j * KT + gr.d) * 2);
+      const uint32_t wk = raw2(L::PB_K, j, gr.d);
       uint32_t hi, lo;
       split2(bf_lo(wk) * e0, bf_hi(wk) * e1, hi, lo);
       *reinterpret_cast<uint32_t*>(sm + L::KQ_HI + sw128(j, gr.d)) = hi;
       *reinterpret_cast<uint32_t*>(sm + L::KQ_LO + sw128(j, gr.d)) = lo;
     });
     gr.forward([&](int j, float e0, float e1) {
-      *reinterpret_cast<float2*>(EF + j * KT + gr.d) = make_float2(e0, e1);
+      *reinterpret_cast<float2*>(EF + j * L::FS + gr.d) = make_float2(e0, e1);
     });
     if (gr.h == 0) {
       DEC[gr.d] = gr.dec0;
@@ -308,7 +314,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       tmem_ld_wait();
       if (row_owner) {
         const int j = row;
-        float* e1 = EF + j * KT;
+        float* e1 = EF + j * L::FS;
         const float ajj = DIAG[j];
         if (safe) {
           const float* XB = reinterpret_cast<const float*>(sm + L::XB);
@@ -317,7 +323,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
           for (int d = 0; d < 64; ++d) {
             float acc = 0.f;
             for (int r = 0; r <= j; ++r)
-              acc += XA[j * C + r] * bf2f(sm + L::PB_K + (r * KT + d) * 2) * __expf(XB[j * KT + d] - XB[r * KT + d]);
+              acc += XA[j * C + r] * raw(L::PB_K, r, d) * __expf(XB[j * KT + d] - XB[r * KT + d]);
             y[d] = acc;  // exact intra term
           }
         } else {
@@ -326,9 +332,9 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         }
 #pragma unroll
         for (int d = 0; d < 64; ++d) {
-          const float qv = bf2f(sm + L::PB_Q + (j * KT + d) * 2), kv = bf2f(sm + L::PB_K + (j * KT + d) * 2);
+          const float qv = raw(L::PB_Q, j, d), kv = raw(L::PB_K, j, d);
           const float ev = e1[d];
-          SCR[j * KT + d] = bf_split_sum(qv * ev) * x[d];  // Qt as the G update sees it
+          SCR[j * L::FS + d] = bf_split_sum(qv * ev) * x[d];  // Qt as the G update sees it
           e1[d] = qv * (y[d] - ajj * kv);
           x[d] = ev * x[d] + y[d];
         }
@@ -341,14 +347,14 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       const int d = tid;
       float suf = 0.f;
       for (int j = C - 1; j >= 0; --j) {
-        suf += SCR[j * KT + d];
-        SCR[j * KT + d] = suf;
+        suf += SCR[j * L::FS + d];
+        SCR[j * L::FS + d] = suf;
       }
       float pre = 0.f;
       for (int j = 0; j < C; ++j) {
         const int t = i * C + j;
-        if (t < T) part[(size_t)t * DK + d] = SCR[j * KT + d] - pre;
-        pre += EF[j * KT + d];
+        if (t < T) part[(size_t)t * DK + d] = SCR[j * L::FS + d] - pre;
+        pre += EF[j * L::FS + d];
       }
       qx_sums[(size_t)i * DK + d] = suf;
     }
@@ -392,16 +398,16 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     mbar_wait(bar_pb, ph_pb, a.latch);
     ph_pb ^= 1;
     Gate gr;
-    const bool weak = gr.run(sm + L::PB_G, KT, TOT);
+    const bool weak = gr.run_swizzled(sm + L::PB_G, TOT);
     gr.forward([&](int j, float e0, float e1) {
-      const uint32_t wq = *reinterpret_cast<const uint32_t*>(sm + L::PB_Q + (j * KT + gr.d) * 2);
+      const uint32_t wq = raw2(L::PB_Q, j, gr.d);
       uint32_t hi, lo;
       split2(bf_lo(wq) * e0, bf_hi(wq) * e1, hi, lo);
       *reinterpret_cast<uint32_t*>(sm + L::KQ_HI + sw128(j, gr.d)) = hi;
       *reinterpret_cast<uint32_t*>(sm + L::KQ_LO + sw128(j, gr.d)) = lo;
     });
     gr.backward([&](int j, float e0, float e1) {
-      *reinterpret_cast<float2*>(EF + j * KT + gr.d) = make_float2(e0, e1);
+      *reinterpret_cast<float2*>(EF + j * L::FS + gr.d) = make_float2(e0, e1);
     });
     if (gr.h == 0) {
       DEC[gr.d] = gr.dec0;
@@ -471,7 +477,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       tmem_ld_wait();
       if (row_owner) {
         const int r = row;
-        float* e2 = EF + r * KT;
+        float* e2 = EF + r * L::FS;
         const float arr = DIAG[r];
         if (safe) {
           const float* XB = reinterpret_cast<const float*>(sm + L::XB);
@@ -480,7 +486,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
           for (int d = 0; d < 64; ++d) {
             float acc = 0.f;
             for (int j = r; j < C; ++j)
-              acc += XA[j * C + r] * bf2f(sm + L::PB_Q + (j * KT + d) * 2) * __expf(XB[j * KT + d] - XB[r * KT + d]);
+              acc += XA[j * C + r] * raw(L::PB_Q, j, d) * __expf(XB[j * KT + d] - XB[r * KT + d]);
             w[d] = acc;
           }
         } else {
@@ -489,11 +495,11 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         }
 #pragma unroll
         for (int d = 0; d < 64; ++d) {
-          const float qv = bf2f(sm + L::PB_Q + (r * KT + d) * 2), kv = bf2f(sm + L::PB_K + (r * KT + d) * 2);
+          const float qv = raw(L::PB_Q, r, d), kv = raw(L::PB_K, r, d);
           const float ev = e2[d];
           const float kz = bf_split_sum(kv * ev) * z[d];  // Kh as the S update sees it
           e2[d] = kz;
-          SCR[r * KT + d] = kz + kv * (w[d] - arr * qv);
+          SCR[r * L::FS + d] = kz + kv * (w[d] - arr * qv);
           z[d] = ev * z[d] + w[d];
         }
         const int t = i * C + r;
@@ -504,15 +510,19 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     if (tid < KT) {  // dg = c_i + prefix of (Kh Z + k dk^intra) + the forward walk's partial
       const int d = tid;
       float kz = 0.f;
-      for (int r = 0; r < C; ++r) kz += EF[r * KT + d];
+      for (int r = 0; r < C; ++r) kz += EF[r * L::FS + d];
       const float ci = (n == 0 ? CARRY[d] : CARRY[d] + qx_sums[(size_t)(i + 1) * DK + d]) - kz;
       float pre = 0.f;
-      for (int r = 0; r < C; ++r) {
-        const int t = i * C + r;
-        if (t < T)
-          a.dg[((size_t)bh * T + t) * DK + d0 + d] =
-              __float2bfloat16_rn(ci + pre + part[(size_t)t * DK + d]);
-        pre += SCR[r * KT + d];
+      for (int r0 = 0; r0 < C; r0 += 16) {
+        float pv[16];  // issue the 16 loads before the dependent prefix sum
+#pragma unroll
+        for (int u = 0; u < 16; ++u) pv[u] = (i * C + r0 + u < T) ? part[(size_t)(i * C + r0 + u) * DK + d] : 0.f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int t = i * C + r0 + u;
+          if (t < T) a.dg[((size_t)bh * T + t) * DK + d0 + d] = __float2bfloat16_rn(ci + pre + pv[u]);
+          pre += SCR[(r0 + u) * L::FS + d];
+        }
       }
       CARRY[d] = ci;
     }
@@ -826,8 +836,8 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
                               int BH, int T, void* ws, cudaStream_t st) {
   BwdMaps mp;
   if (!make_map(&mp.v, v, BH, T, DV, 64, true) || !make_map(&mp.dO, dO, BH, T, DV, 64, true) ||
-      !make_map(&mp.k64, k, BH, T, DK, KT, false) || !make_map(&mp.g64, g, BH, T, DK, KT, false) ||
-      !make_map(&mp.q64, q, BH, T, DK, KT, false) ||
+      !make_map(&mp.k64, k, BH, T, DK, KT, true) || !make_map(&mp.g64, g, BH, T, DK, KT, true) ||
+      !make_map(&mp.q64, q, BH, T, DK, KT, true) ||
       !make_map(&mp.q_all, q, BH, T, DK, DK, false) || !make_map(&mp.k_all, k, BH, T, DK, DK, false) ||
       !make_map(&mp.g_all, g, BH, T, DK, DK, false))
     return cudaErrorInvalidValue;

@@ -151,6 +151,13 @@ struct GateRun {
 
   // Returns true when this thread's dimensions keep less than kMinDecay of the state.
   __device__ __forceinline__ bool run(const uint8_t* graw, int gstride, float* tot) {
+    return run_impl(graw, gstride, tot, false);
+  }
+  // Same for a [64][64] tile stored with the 128-byte swizzle (ND == 64).
+  __device__ __forceinline__ bool run_swizzled(const uint8_t* graw, float* tot) {
+    return run_impl(graw, 64, tot, true);
+  }
+  __device__ __forceinline__ bool run_impl(const uint8_t* graw, int gstride, float* tot, bool swz) {
     const int tid = threadIdx.x;
     p = tid % NPAIR;
     h = tid / NPAIR;
@@ -159,7 +166,7 @@ struct GateRun {
 #pragma unroll
     for (int u = 0; u < TS; ++u) {
       const int j = h * TS + u;
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(graw + (j * gstride + d) * 2);
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(graw + (swz ? sm100::sw128(j, d) : (j * gstride + d) * 2));
       a0[u] = ex2(bf_lo(w) * kLog2e);
       a1[u] = ex2(bf_hi(w) * kLog2e);
       r0 *= a0[u];
