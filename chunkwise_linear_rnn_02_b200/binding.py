@@ -39,6 +39,7 @@ _SIGNATURES = {
     "gsa_bwd": (_i, [_vp] * 17 + [_i] * 8 + [_vp, _sz, _vp]),
     "gsa_recurrent_step": (_i, [_vp] * 8 + [_i] * 6 + [_vp]),
     "gla_device_error": (_i, [_vp, _i, ctypes.POINTER(_i)]),
+    "gla_chunk_bwd_noalloc": (_i, [_vp] * 12 + [_i] * 7 + [_vp]),
 }
 
 

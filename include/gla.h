@@ -155,6 +155,29 @@ int gsa_recurrent_step(const void* q, const void* k, const void* v, const void* 
                        int dv, int m, int dtype, void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * gla_chunk_bwd_noalloc - gla_chunk_bwd without a workspace argument, for callers that cannot
+ * provide one.  (A library entry point only; the source pages have no counterpart of it.)
+ *
+ * Who needs it: callers that have no means to obtain device memory for a workspace, such as a
+ * plain C host without a device allocator, a runtime that has carved up device memory in advance
+ * and hands it out only for tensors, or code that must not call cudaMalloc because that call may
+ * synchronise the device while its work is in flight.
+ * What it uses instead: a fixed 64 MiB scratch array compiled into the library, reserved on every
+ * device that loads this part of the library and held until the process exits.  The first call on
+ * a device looks up that array's device address (cudaGetSymbolAddress); make the first call on each
+ * device before any stream capture.  All calls share the array: calls that overlap on the GPU
+ * (different streams or host threads) race on it.  Nothing in it needs to start at zero.
+ * Arguments, layouts and outputs are those of gla_chunk_bwd.  Supported: bf16, chunk 64,
+ * d_k = 128, d_v in {128, 256}, T >= 1 (else GLA_ERR_UNSUPPORTED / GLA_ERR_INVALID_ARG), and
+ * B*H*(T + ceil(T/64))*d_k*4 bytes of scratch within the 64 MiB (else GLA_ERR_WORKSPACE).
+ * It allocates nothing.
+ * ------------------------------------------------------------------------------------- */
+int gla_chunk_bwd_noalloc(const void* q, const void* k, const void* v, const void* g, const float* h0,
+                          const void* dO, const float* dhT, void* dq, void* dk, void* dv, void* dg,
+                          float* dh0, int B, int H, int T, int dk_dim, int dv_dim, int chunk, int dtype,
+                          void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * gla_device_error - read (and optionally clear) the device-side error latch.
  * Synchronises `stream`, then stores GLA_OK or the first error a kernel recorded since the
  * last reset (GLA_ERR_TIMEOUT: a bounded wait ran out) in *code.  Returns GLA_ERR_CUDA if

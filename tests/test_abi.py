@@ -77,6 +77,14 @@ def test_bwd_and_gsa_argument_checks(lib):
     assert lib.gla_recurrent_step(P, P, P, P, P, P, 1, 1, 64, 64, 3, None) == UNSUPPORTED
     assert lib.gsa_recurrent_step(P, P, P, P, P, P, BAD, P, 1, 1, 64, 64, 64, 1, None) == INVALID
     assert lib.gla_device_error(None, 0, None) == INVALID
+    # the workspace-free backward rejects what it cannot run before touching the device
+    nb = [P] * 5 + [P, None] + [P] * 4 + [None]
+    assert lib.gla_chunk_bwd_noalloc(*nb, 1, 1, 64, 128, 256, 64, 0, None) == UNSUPPORTED   # fp32
+    assert lib.gla_chunk_bwd_noalloc(*nb, 1, 1, 64, 64, 256, 64, 1, None) == UNSUPPORTED    # d_k
+    assert lib.gla_chunk_bwd_noalloc(*nb, 1, 1, 0, 128, 256, 64, 1, None) == INVALID        # T = 0
+    bad_nb = list(nb)
+    bad_nb[0] = None
+    assert lib.gla_chunk_bwd_noalloc(*bad_nb, 1, 1, 64, 128, 256, 64, 1, None) == INVALID
 
 
 def test_workspace_queries(lib):
