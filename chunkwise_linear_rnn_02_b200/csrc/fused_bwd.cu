@@ -30,7 +30,7 @@ namespace fast {
 
 using namespace sm100;
 
-constexpr int BT = 128;  // threads per CTA
+constexpr int BT = 256;  // threads per CTA: warps w and w+4 share TMEM lanes and split columns
 constexpr int KT = 64;   // key dimensions per key-tile CTA
 constexpr int VT = 128;  // value columns per value-tile CTA
 
@@ -86,10 +86,11 @@ struct KeyLayout {
   static constexpr uint32_t EF = DA_LO + TILE;      // fp32 [64][FS]: E1 / E2, then a per-token term
   static constexpr uint32_t SCR = EF + C * FS * 4;  // fp32 [64][FS]: a per-token term
   static constexpr uint32_t DEC = SCR + C * FS * 4;
-  static constexpr uint32_t TOT = DEC + KT * 4;     // [4][64]
-  static constexpr uint32_t DIAG = TOT + 4 * KT * 4;
+  static constexpr uint32_t TOT = DEC + KT * 4;     // [NSPLIT][64]
+  static constexpr uint32_t DIAG = TOT + GateRun<KT, BT>::NSPLIT * KT * 4;
   static constexpr uint32_t CARRY = DIAG + C * 4;
-  static constexpr uint32_t TOTAL = CARRY + KT * 4;
+  static constexpr uint32_t CARRYP = CARRY + KT * 4;  // [2][64] per-column-half partial row sums
+  static constexpr uint32_t TOTAL = CARRYP + 2 * KT * 4;
   // exact-path scratch (only when the part-A prefetch is held back): B and dA in fp32
   static constexpr uint32_t XB = PA_V, XA = PA_DO;
   // TMEM columns
@@ -104,11 +105,13 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   using L = KeyLayout<DK, DV>;
   using Gate = GateRun<KT, BT>;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
   const int T = a.T, NC = (T + C - 1) / C, d0 = tau * KT;
   const uint32_t base = smem_u32(sm);
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
   const bool row_owner = lane < 16;
-  const int row = warp * 16 + lane;  // row of an M=64 accumulator owned by this thread
+  const int row = q4 * 16 + lane;  // row of an M=64 accumulator owned by this thread
+  constexpr int HV = DV / 2;       // state columns per warp
   uint64_t* bar_pa = bars + 0;
   uint64_t* bar_pb = bars + 1;
   uint64_t* bar_m1 = bars + 3;
@@ -147,7 +150,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   // Initialise the TMEM state rows and their hi/lo bf16 copies from a [DK x DV] fp32 source (or zeros).
   auto init_state = [&](const float* src) {
     float v[64];
-    for (int c0 = 0; c0 < DV; c0 += 64) {
+    for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 64) {
 #pragma unroll
       for (int c = 0; c < 64; ++c)
         v[c] = (src && row_owner) ? src[((size_t)bh * DK + d0 + row) * DV + c0 + c] : 0.f;
@@ -162,7 +165,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   auto rescale_state = [&]() {
     const float s = row_owner ? DEC[row] : 0.f;
     float v[64];
-    for (int c0 = 0; c0 < DV; c0 += 64) {
+    for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 64) {
       tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
       tmem_ld32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
       tmem_ld_wait();
@@ -176,7 +179,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   // Copy the TMEM state rows into the hi/lo bf16 K-major operands.
   auto copy_state = [&]() {
     float v[64];
-    for (int c0 = 0; c0 < DV; c0 += 64) {
+    for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 64) {
       tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
       tmem_ld32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
       tmem_ld_wait();
@@ -197,23 +200,20 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   };
   // dA epilogue: masked bf16 operand, its diagonal, and (exact path) an fp32 copy.
   auto dA_epilogue = [&](int safe) {
-    float v[64];
-    tmem_ld32(tmem + L::T_DA + lane_off, v);
-    tmem_ld32(tmem + L::T_DA + lane_off + 32, v + 32);
+    float v[32];
+    tmem_ld32(tmem + L::T_DA + lane_off + half * 32, v);
     tmem_ld_wait();
     if (row_owner) {
-      float diag = 0.f;
 #pragma unroll
-      for (int r = 0; r < 64; ++r) {
-        if (r > row) v[r] = 0.f;
-        if (r == row) diag = v[r];
+      for (int c = 0; c < 32; ++c) {
+        if (half * 32 + c > row) v[c] = 0.f;
+        if (half * 32 + c == row) DIAG[row] = v[c];
       }
-      DIAG[row] = diag;
-      store_row_split(sm + L::DA_HI, sm + L::DA_LO, row, v, 1.f);
+      store_half_split(sm + L::DA_HI, sm + L::DA_LO, row, v, half);
       if (safe) {
         float* XA = reinterpret_cast<float*>(sm + L::XA);
 #pragma unroll
-        for (int r = 0; r < 64; ++r) XA[row * C + r] = v[r];
+        for (int c = 0; c < 32; ++c) XA[row * C + half * 32 + c] = v[c];
       }
     }
   };
@@ -304,42 +304,38 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       tc_fence_after();
     }
     {  // dq epilogue; per-token terms q e^B X (-> SCR) and q dq^intra without j = r (-> EF)
-      float x[64], y[64];
-      tmem_ld32(tmem + L::T_X + lane_off, x);
-      tmem_ld32(tmem + L::T_X + lane_off + 32, x + 32);
-      if (!safe) {
-        tmem_ld32(tmem + L::T_Y + lane_off, y);
-        tmem_ld32(tmem + L::T_Y + lane_off + 32, y + 32);
-      }
+      float x[32], y[32];
+      tmem_ld32(tmem + L::T_X + lane_off + half * 32, x);
+      if (!safe) tmem_ld32(tmem + L::T_Y + lane_off + half * 32, y);
       tmem_ld_wait();
       if (row_owner) {
-        const int j = row;
-        float* e1 = EF + j * L::FS;
+        const int j = row, cb = half * 32;
+        float* e1 = EF + j * L::FS + cb;
         const float ajj = DIAG[j];
         if (safe) {
           const float* XB = reinterpret_cast<const float*>(sm + L::XB);
           const float* XA = reinterpret_cast<const float*>(sm + L::XA);
 #pragma unroll
-          for (int d = 0; d < 64; ++d) {
+          for (int c = 0; c < 32; ++c) {
             float acc = 0.f;
             for (int r = 0; r <= j; ++r)
-              acc += XA[j * C + r] * raw(L::PB_K, r, d) * __expf(XB[j * KT + d] - XB[r * KT + d]);
-            y[d] = acc;  // exact intra term
+              acc += XA[j * C + r] * raw(L::PB_K, r, cb + c) * __expf(XB[j * KT + cb + c] - XB[r * KT + cb + c]);
+            y[c] = acc;  // exact intra term
           }
         } else {
 #pragma unroll
-          for (int d = 0; d < 64; ++d) y[d] *= e1[d] / DEC[d];
+          for (int c = 0; c < 32; ++c) y[c] *= e1[c] / DEC[cb + c];
         }
 #pragma unroll
-        for (int d = 0; d < 64; ++d) {
-          const float qv = raw(L::PB_Q, j, d), kv = raw(L::PB_K, j, d);
-          const float ev = e1[d];
-          SCR[j * L::FS + d] = bf_split_sum(qv * ev) * x[d];  // Qt as the G update sees it
-          e1[d] = qv * (y[d] - ajj * kv);
-          x[d] = ev * x[d] + y[d];
+        for (int c = 0; c < 32; ++c) {
+          const float qv = raw(L::PB_Q, j, cb + c), kv = raw(L::PB_K, j, cb + c);
+          const float ev = e1[c];
+          SCR[j * L::FS + cb + c] = bf_split_sum(qv * ev) * x[c];  // Qt as the G update sees it
+          e1[c] = qv * (y[c] - ajj * kv);
+          x[c] = ev * x[c] + y[c];
         }
         const int t = i * C + j;
-        if (t < T) store_row_global_bf16(a.dq + ((size_t)bh * T + t) * DK + d0, x);
+        if (t < T) store_half_global_bf16(a.dq + ((size_t)bh * T + t) * DK + d0 + cb, x);
       }
     }
     __syncthreads();
@@ -368,9 +364,10 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
 
   // rowsum(dhT * hT): hT rows = the state after the forward walk
   {
+    float* CARRYP = reinterpret_cast<float*>(sm + L::CARRYP);
     float v[32];
     float acc = 0.f;
-    for (int c0 = 0; c0 < DV; c0 += 32) {
+    for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 32) {
       tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
       tmem_ld_wait();
       if (row_owner && a.dhT) {
@@ -379,7 +376,9 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         for (int c = 0; c < 32; ++c) acc += src[c] * v[c];
       }
     }
-    if (row_owner) CARRY[row] = acc;
+    if (row_owner) CARRYP[half * KT + row] = acc;
+    __syncthreads();
+    if (tid < KT) CARRY[tid] = CARRYP[tid] + CARRYP[KT + tid];
   }
   tc_fence_before();
   __syncthreads();
@@ -467,43 +466,39 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       tc_fence_after();
     }
     {  // dk epilogue; per-token terms Kh Z (-> EF) and Kh Z + k dk^intra without j = r (-> SCR)
-      float z[64], w[64];
-      tmem_ld32(tmem + L::T_X + lane_off, z);
-      tmem_ld32(tmem + L::T_X + lane_off + 32, z + 32);
-      if (!safe) {
-        tmem_ld32(tmem + L::T_Y + lane_off, w);
-        tmem_ld32(tmem + L::T_Y + lane_off + 32, w + 32);
-      }
+      float z[32], w[32];
+      tmem_ld32(tmem + L::T_X + lane_off + half * 32, z);
+      if (!safe) tmem_ld32(tmem + L::T_Y + lane_off + half * 32, w);
       tmem_ld_wait();
       if (row_owner) {
-        const int r = row;
-        float* e2 = EF + r * L::FS;
+        const int r = row, cb = half * 32;
+        float* e2 = EF + r * L::FS + cb;
         const float arr = DIAG[r];
         if (safe) {
           const float* XB = reinterpret_cast<const float*>(sm + L::XB);
           const float* XA = reinterpret_cast<const float*>(sm + L::XA);
 #pragma unroll
-          for (int d = 0; d < 64; ++d) {
+          for (int c = 0; c < 32; ++c) {
             float acc = 0.f;
             for (int j = r; j < C; ++j)
-              acc += XA[j * C + r] * raw(L::PB_Q, j, d) * __expf(XB[j * KT + d] - XB[r * KT + d]);
-            w[d] = acc;
+              acc += XA[j * C + r] * raw(L::PB_Q, j, cb + c) * __expf(XB[j * KT + cb + c] - XB[r * KT + cb + c]);
+            w[c] = acc;
           }
         } else {
 #pragma unroll
-          for (int d = 0; d < 64; ++d) w[d] *= e2[d] / DEC[d];
+          for (int c = 0; c < 32; ++c) w[c] *= e2[c] / DEC[cb + c];
         }
 #pragma unroll
-        for (int d = 0; d < 64; ++d) {
-          const float qv = raw(L::PB_Q, r, d), kv = raw(L::PB_K, r, d);
-          const float ev = e2[d];
-          const float kz = bf_split_sum(kv * ev) * z[d];  // Kh as the S update sees it
-          e2[d] = kz;
-          SCR[r * L::FS + d] = kz + kv * (w[d] - arr * qv);
-          z[d] = ev * z[d] + w[d];
+        for (int c = 0; c < 32; ++c) {
+          const float qv = raw(L::PB_Q, r, cb + c), kv = raw(L::PB_K, r, cb + c);
+          const float ev = e2[c];
+          const float kz = bf_split_sum(kv * ev) * z[c];  // Kh as the S update sees it
+          e2[c] = kz;
+          SCR[r * L::FS + cb + c] = kz + kv * (w[c] - arr * qv);
+          z[c] = ev * z[c] + w[c];
         }
         const int t = i * C + r;
-        if (t < T) store_row_global_bf16(a.dk + ((size_t)bh * T + t) * DK + d0, z);
+        if (t < T) store_half_global_bf16(a.dk + ((size_t)bh * T + t) * DK + d0 + cb, z);
       }
     }
     __syncthreads();
@@ -537,7 +532,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   if (a.dh0) {
     tc_fence_after();
     float v[32];
-    for (int c0 = 0; c0 < DV; c0 += 32) {
+    for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 32) {
       tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
       tmem_ld_wait();
       if (row_owner) {
@@ -585,9 +580,12 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = a.T, NC = (T + C - 1) / C, c0 = vt * VT;
   const uint32_t base = smem_u32(sm);
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int q4 = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
+  const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
   const bool row_owner = lane < 16;
-  const int row = warp * 16 + lane;
+  const int row = q4 * 16 + lane;   // row of an M=64 accumulator
+  const int grow = q4 * 32 + lane;  // row of the M=128 G accumulator
+  constexpr int HT = VT / 2;        // G / dv columns per warp
   uint64_t* bar_ld = bars + 0;
   uint64_t* bar_m1 = bars + 3;
   uint64_t* bar_m2 = bars + 4;
@@ -610,9 +608,9 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   };
   // G <- DEC[row] * G for this thread's row of the M=128 accumulator.
   auto rescale_G = [&]() {
-    const float sc = DEC[tid];
+    const float sc = DEC[grow];
     float v[32];
-    for (int cb = 0; cb < VT; cb += 32) {
+    for (int cb = half * HT; cb < (half + 1) * HT; cb += 32) {
       tmem_ld32(tmem + L::T_G + lane_off + cb, v);
       tmem_ld_wait();
 #pragma unroll
@@ -621,15 +619,15 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     }
     tmem_st_wait();
   };
-  // G rows (this thread owns row tid of the M=128 accumulator): init from dhT[:, tile]
+  // G rows (this thread owns row grow of the M=128 accumulator): init from dhT[:, tile]
   {
     float v[64];
-    for (int cb = 0; cb < VT; cb += 64) {
+    for (int cb = half * HT; cb < (half + 1) * HT; cb += 64) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) v[c] = a.dhT ? a.dhT[((size_t)bh * DK + tid) * DV + c0 + cb + c] : 0.f;
+      for (int c = 0; c < 64; ++c) v[c] = a.dhT ? a.dhT[((size_t)bh * DK + grow) * DV + c0 + cb + c] : 0.f;
       tmem_st32(tmem + L::T_G + lane_off + cb, v);
       tmem_st32(tmem + L::T_G + lane_off + cb + 32, v + 32);
-      store_row_split(sm + L::GC_HI + (cb / 64) * (DK * 128), sm + L::GC_LO + (cb / 64) * (DK * 128), tid, v, 1.f);
+      store_row_split(sm + L::GC_HI + (cb / 64) * (DK * 128), sm + L::GC_LO + (cb / 64) * (DK * 128), grow, v, 1.f);
     }
     tmem_st_wait();
   }
@@ -720,28 +718,27 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       __syncthreads();
     }
     {  // A epilogue
-      float v[64];
-      tmem_ld32(tmem + L::T_A + lane_off, v);
-      tmem_ld32(tmem + L::T_A + lane_off + 32, v + 32);
+      float v[32];
+      tmem_ld32(tmem + L::T_A + lane_off + half * 32, v);
       tmem_ld_wait();
       if (row_owner) {
         if (safe) {
 #pragma unroll
-          for (int r = 0; r < 64; ++r) v[r] = XA[row * C + r];
+          for (int c = 0; c < 32; ++c) v[c] = XA[row * C + half * 32 + c];
         }
 #pragma unroll
-        for (int r = 0; r < 64; ++r)
-          if (r > row) v[r] = 0.f;
-        store_row_split(sm + L::AB_HI, sm + L::AB_LO, row, v, 1.f);
+        for (int c = 0; c < 32; ++c)
+          if (half * 32 + c > row) v[c] = 0.f;
+        store_half_split(sm + L::AB_HI, sm + L::AB_LO, row, v, half);
       }
     }
     {  // hi / lo copy of G_i for the next (earlier) chunk
       float v[64];
-      for (int cb = 0; cb < VT; cb += 64) {
+      for (int cb = half * HT; cb < (half + 1) * HT; cb += 64) {
         tmem_ld32(tmem + L::T_G + lane_off + cb, v);
         tmem_ld32(tmem + L::T_G + lane_off + cb + 32, v + 32);
         tmem_ld_wait();
-        store_row_split(sm + L::GC_HI + (cb / 64) * (DK * 128), sm + L::GC_LO + (cb / 64) * (DK * 128), tid, v, 1.f);
+        store_row_split(sm + L::GC_HI + (cb / 64) * (DK * 128), sm + L::GC_LO + (cb / 64) * (DK * 128), grow, v, 1.f);
       }
     }
     fence_async_smem();
@@ -764,7 +761,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     {  // dv epilogue
       float v[64];
       const int t = i * C + row;
-      for (int cb = 0; cb < VT; cb += 64) {
+      for (int cb = half * HT; cb < (half + 1) * HT; cb += 64) {
         tmem_ld32(tmem + L::T_DV + lane_off + cb, v);
         tmem_ld32(tmem + L::T_DV + lane_off + cb + 32, v + 32);
         tmem_ld_wait();

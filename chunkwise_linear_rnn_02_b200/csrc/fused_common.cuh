@@ -133,6 +133,34 @@ __device__ __forceinline__ void store_row_split(uint8_t* th, uint8_t* tl, int r,
   }
 }
 
+// Store 32 fp32 values as hi / lo bf16 into columns 32*hb .. 32*hb+31 of swizzled 64-column row r.
+__device__ __forceinline__ void store_half_split(uint8_t* th, uint8_t* tl, int r, const float* v, int hb) {
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    uint4 h, l;
+    split2(v[8 * cc + 0], v[8 * cc + 1], h.x, l.x);
+    split2(v[8 * cc + 2], v[8 * cc + 3], h.y, l.y);
+    split2(v[8 * cc + 4], v[8 * cc + 5], h.z, l.z);
+    split2(v[8 * cc + 6], v[8 * cc + 7], h.w, l.w);
+    const uint32_t off = r * 128 + ((((4 * hb + cc) ^ (r & 7)) & 7) << 4);
+    *reinterpret_cast<uint4*>(th + off) = h;
+    *reinterpret_cast<uint4*>(tl + off) = l;
+  }
+}
+// Store 32 fp32 values as bf16 to global (16-byte aligned destination).
+__device__ __forceinline__ void store_half_global_bf16(__nv_bfloat16* dst, const float* v) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    uint4 w;
+    w.x = pack2(v[8 * cc + 0], v[8 * cc + 1]);
+    w.y = pack2(v[8 * cc + 2], v[8 * cc + 3]);
+    w.z = pack2(v[8 * cc + 4], v[8 * cc + 5]);
+    w.w = pack2(v[8 * cc + 6], v[8 * cc + 7]);
+    d[cc] = w;
+  }
+}
+
 // Gate math shared by the fused kernels.  The CTA's NTH threads cover ND key dimensions of one
 // chunk: thread t owns dimensions (2p, 2p+1), p = t % (ND/2), and the run of TS = 64 * (ND/2) / NTH
 // tokens starting at h * TS, h = t / (ND/2).  It loads the raw log-gates g (row-major [64][gstride]
