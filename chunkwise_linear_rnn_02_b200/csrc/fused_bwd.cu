@@ -46,7 +46,7 @@ struct BwdArgs {
   __nv_bfloat16 *dq, *dk, *dv, *dg;
   float* dh0;
   float* ws_qx;    // [BH][NC][DK] chunk sums of Qt X
-  float* ws_part;  // [BH][T][DK] forward-walk part of dg
+  float* ws_part;  // [BH][NC][DK][64] forward-walk part of dg, one row of 64 tokens per chunk and dim
   int T, n_key_ctas;
   unsigned int* latch;
 };
@@ -83,13 +83,13 @@ struct KeyLayout {
   static constexpr uint32_t DA_HI = SG_LO + KT * DV * 2;  // masked dA, bf16 hi / lo [64 x 64]
   static constexpr uint32_t DA_LO = DA_HI + TILE;
   static constexpr int FS = 66;                     // padded row stride of the fp32 [64][64] scratch
-  static constexpr uint32_t EF = DA_LO + TILE;      // fp32 [64][FS]: E1 / E2, then a per-token term
-  static constexpr uint32_t SCR = EF + C * FS * 4;  // fp32 [64][FS]: a per-token term
-  static constexpr uint32_t DEC = SCR + C * FS * 4;
+  static constexpr uint32_t EF = DA_LO + TILE;      // fp32 [64][FS]: E1 (forward walk) / E2 (reverse walk)
+  static constexpr uint32_t XCH = EF + C * FS * 4;  // float2 [2][64]: token-half sums exchanged per dim
+  static constexpr uint32_t DEC = XCH + 2 * KT * 8;
   static constexpr uint32_t TOT = DEC + KT * 4;     // [NSPLIT][64]
   static constexpr uint32_t DIAG = TOT + GateRun<KT, BT>::NSPLIT * KT * 4;
-  static constexpr uint32_t CARRY = DIAG + C * 4;
-  static constexpr uint32_t CARRYP = CARRY + KT * 4;  // [2][64] per-column-half partial row sums
+  static constexpr uint32_t CARRY = DIAG + C * 4;    // [2][64] c_i, double-buffered over chunks
+  static constexpr uint32_t CARRYP = CARRY + 2 * KT * 4;  // [2][64] per-column-half partial row sums
   static constexpr uint32_t TOTAL = CARRYP + 2 * KT * 4;
   // exact-path scratch (only when the part-A prefetch is held back): B and dA in fp32
   static constexpr uint32_t XB = PA_V, XA = PA_DO;
@@ -120,11 +120,11 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   float* DEC = reinterpret_cast<float*>(sm + L::DEC);
   float* TOT = reinterpret_cast<float*>(sm + L::TOT);
   float* EF = reinterpret_cast<float*>(sm + L::EF);
-  float* SCR = reinterpret_cast<float*>(sm + L::SCR);
+  float2* XCH = reinterpret_cast<float2*>(sm + L::XCH);
   float* DIAG = reinterpret_cast<float*>(sm + L::DIAG);
   float* CARRY = reinterpret_cast<float*>(sm + L::CARRY);
   float* qx_sums = a.ws_qx + (size_t)bh * NC * DK + d0;  // [NC][DK] slice of this head and key tile
-  float* part = a.ws_part + (size_t)bh * T * DK + d0;      // [T][DK] slice: forward-walk part of dg
+  float* part = a.ws_part + ((size_t)bh * NC * DK + d0) * C;  // [NC][DK][64] slice: forward-walk part of dg
 
   auto load_a = [&](int chunk) {
     mbar_arrive_expect_tx(bar_pa, 2 * L::VB);
@@ -255,15 +255,15 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     fence_async_smem();
     sync_tc();
     if (tid == 0) {
-      constexpr uint32_t id_X = idesc_bf16_f32(C, KT, false, false);
+      constexpr uint32_t id_X = idesc_bf16_f32(KT, C, false, false);  // X^T = S dO^T
       constexpr uint32_t id_S = idesc_bf16_f32(KT, DV, true, true);
 #pragma unroll
       for (int k = 0; k < DV / 16; ++k) {
         const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
-        const uint64_t ad = desc_sw128(base + L::PA_DO + ko, 16, 1024);
+        const uint64_t bd = desc_sw128(base + L::PA_DO + ko, 16, 1024);
         mma_dA(k, ko);
-        umma_bf16(tmem + L::T_X, ad, desc_sw128(base + L::SG_HI + ko, 16, 1024), id_X, k > 0);
-        umma_bf16(tmem + L::T_X, ad, desc_sw128(base + L::SG_LO + ko, 16, 1024), id_X, 1);
+        umma_bf16(tmem + L::T_X, desc_sw128(base + L::SG_HI + ko, 16, 1024), bd, id_X, k > 0);
+        umma_bf16(tmem + L::T_X, desc_sw128(base + L::SG_LO + ko, 16, 1024), bd, id_X, 1);
       }
 #pragma unroll
       for (int k = 0; k < C / 16; ++k) {
@@ -282,14 +282,14 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     fence_async_smem();
     sync_tc();
     if (tid == 0 && !safe) {
-      constexpr uint32_t id_Y = idesc_bf16_f32(C, KT, false, true);
+      constexpr uint32_t id_Y = idesc_bf16_f32(KT, C, true, false);  // Y^T = Kh^T dA^T
 #pragma unroll
       for (int k = 0; k < C / 16; ++k) {
-        const uint64_t ah = desc_sw128(base + L::DA_HI + k * 32, 16, 1024);
-        const uint64_t bh = desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024);
+        const uint64_t ah = desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024);
+        const uint64_t bh = desc_sw128(base + L::DA_HI + k * 32, 16, 1024);
         umma_bf16(tmem + L::T_Y, ah, bh, id_Y, k > 0);
-        umma_bf16(tmem + L::T_Y, ah, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), id_Y, 1);
-        umma_bf16(tmem + L::T_Y, desc_sw128(base + L::DA_LO + k * 32, 16, 1024), bh, id_Y, 1);
+        umma_bf16(tmem + L::T_Y, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), bh, id_Y, 1);
+        umma_bf16(tmem + L::T_Y, ah, desc_sw128(base + L::DA_LO + k * 32, 16, 1024), id_Y, 1);
       }
       umma_commit(bar_m2);
     }
@@ -303,63 +303,70 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       ph_m2 ^= 1;
       tc_fence_after();
     }
-    {  // dq epilogue; per-token terms q e^B X (-> SCR) and q dq^intra without j = r (-> EF)
-      float x[32], y[32];
+    {  // dq epilogue: this thread owns key dimension d = row and the tokens jb .. jb+31
+      float x[32], y[32];  // rows of X^T and Y^T
       tmem_ld32(tmem + L::T_X + lane_off + half * 32, x);
       if (!safe) tmem_ld32(tmem + L::T_Y + lane_off + half * 32, y);
       tmem_ld_wait();
       if (row_owner) {
-        const int j = row, cb = half * 32;
-        float* e1 = EF + j * L::FS + cb;
-        const float ajj = DIAG[j];
+        const int d = row, jb = half * 32;
         if (safe) {
           const float* XB = reinterpret_cast<const float*>(sm + L::XB);
           const float* XA = reinterpret_cast<const float*>(sm + L::XA);
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
+            const int j = jb + c;
+            const float bj = XB[j * KT + d];
             float acc = 0.f;
-            for (int r = 0; r <= j; ++r)
-              acc += XA[j * C + r] * raw(L::PB_K, r, cb + c) * __expf(XB[j * KT + cb + c] - XB[r * KT + cb + c]);
+            for (int r = 0; r <= j; ++r) acc += XA[j * C + r] * raw(L::PB_K, r, d) * __expf(bj - XB[r * KT + d]);
             y[c] = acc;  // exact intra term
           }
         } else {
+          const float inv = 1.f / DEC[d];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) y[c] *= e1[c] / DEC[cb + c];
+          for (int c = 0; c < 32; ++c) y[c] *= EF[(jb + c) * L::FS + d] * inv;
+        }
+        __nv_bfloat16* dst = a.dq + ((size_t)bh * T + i * C + jb) * DK + d0 + d;
+        float tot_s = 0.f, tot_e = 0.f;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int j = jb + c;
+          const float qv = raw(L::PB_Q, j, d), kv = raw(L::PB_K, j, d), ev = EF[j * L::FS + d];
+          if (i * C + j < T) dst[(size_t)c * DK] = __float2bfloat16_rn(ev * x[c] + y[c]);
+          x[c] = bf_split_sum(qv * ev) * x[c];  // Qt X, with Qt as the G update sees it
+          y[c] = qv * (y[c] - DIAG[j] * kv);    // q dq^intra without j = r
+          tot_s += x[c];
+          tot_e += y[c];
+        }
+        XCH[half * KT + d] = make_float2(tot_s, tot_e);
+      }
+      __syncthreads();
+      if (tid == 0 && i + 1 < NC) {
+        if (safe) load_a(i + 1);
+        load_b(i + 1);
+      }
+      if (row_owner) {  // part = suffix (inclusive) of Qt X minus prefix (exclusive) of q dq^intra
+        const int d = row, jb = half * 32;
+        const float2 o = XCH[(half ^ 1) * KT + d];
+        float suf = half == 0 ? o.x : 0.f, pre = half == 1 ? o.y : 0.f;
+#pragma unroll
+        for (int c = 31; c >= 0; --c) {
+          suf += x[c];
+          x[c] = suf;
         }
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float qv = raw(L::PB_Q, j, cb + c), kv = raw(L::PB_K, j, cb + c);
-          const float ev = e1[c];
-          SCR[j * L::FS + cb + c] = bf_split_sum(qv * ev) * x[c];  // Qt as the G update sees it
-          e1[c] = qv * (y[c] - ajj * kv);
-          x[c] = ev * x[c] + y[c];
+          x[c] -= pre;
+          pre += y[c];
         }
-        const int t = i * C + j;
-        if (t < T) store_half_global_bf16(a.dq + ((size_t)bh * T + t) * DK + d0 + cb, x);
+        float4* dst = reinterpret_cast<float4*>(part + ((size_t)i * DK + d) * C + jb);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+        if (half == 0) qx_sums[(size_t)i * DK + d] = suf;
       }
-    }
-    __syncthreads();
-    if (tid < KT) {  // chunk-local parts of dg: suffix of Qt X minus prefix of q dq^intra
-      const int d = tid;
-      float suf = 0.f;
-      for (int j = C - 1; j >= 0; --j) {
-        suf += SCR[j * L::FS + d];
-        SCR[j * L::FS + d] = suf;
-      }
-      float pre = 0.f;
-      for (int j = 0; j < C; ++j) {
-        const int t = i * C + j;
-        if (t < T) part[(size_t)t * DK + d] = SCR[j * L::FS + d] - pre;
-        pre += EF[j * L::FS + d];
-      }
-      qx_sums[(size_t)i * DK + d] = suf;
     }
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
-      if (safe && i + 1 < NC) load_a(i + 1);
-      if (i + 1 < NC) load_b(i + 1);
-    }
   }
 
   // rowsum(dhT * hT): hT rows = the state after the forward walk
@@ -378,7 +385,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     }
     if (row_owner) CARRYP[half * KT + row] = acc;
     __syncthreads();
-    if (tid < KT) CARRY[tid] = CARRYP[tid] + CARRYP[KT + tid];
+    if (tid < KT) CARRY[tid] = CARRYP[tid] + CARRYP[KT + tid];  // c for the last chunk: buffer 0
   }
   tc_fence_before();
   __syncthreads();
@@ -417,15 +424,15 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     fence_async_smem();
     sync_tc();
     if (tid == 0) {
-      constexpr uint32_t id_Z = idesc_bf16_f32(C, KT, false, false);
+      constexpr uint32_t id_Z = idesc_bf16_f32(KT, C, false, false);  // Z^T = G V^T
       constexpr uint32_t id_G = idesc_bf16_f32(KT, DV, true, true);
 #pragma unroll
       for (int k = 0; k < DV / 16; ++k) {
         const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
         const uint64_t vd = desc_sw128(base + L::PA_V + ko, 16, 1024);
         mma_dA(k, ko);
-        umma_bf16(tmem + L::T_X, vd, desc_sw128(base + L::SG_HI + ko, 16, 1024), id_Z, k > 0);
-        umma_bf16(tmem + L::T_X, vd, desc_sw128(base + L::SG_LO + ko, 16, 1024), id_Z, 1);
+        umma_bf16(tmem + L::T_X, desc_sw128(base + L::SG_HI + ko, 16, 1024), vd, id_Z, k > 0);
+        umma_bf16(tmem + L::T_X, desc_sw128(base + L::SG_LO + ko, 16, 1024), vd, id_Z, 1);
       }
 #pragma unroll
       for (int k = 0; k < C / 16; ++k) {
@@ -444,14 +451,14 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     fence_async_smem();
     sync_tc();
     if (tid == 0 && !safe) {
-      constexpr uint32_t id_W = idesc_bf16_f32(C, KT, true, true);
+      constexpr uint32_t id_W = idesc_bf16_f32(KT, C, true, true);  // W^T = Qt^T dA
 #pragma unroll
       for (int k = 0; k < C / 16; ++k) {
-        const uint64_t ah = desc_sw128(base + L::DA_HI + k * 2048, C * 128, 1024);
-        const uint64_t bh = desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024);
+        const uint64_t ah = desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024);
+        const uint64_t bh = desc_sw128(base + L::DA_HI + k * 2048, C * 128, 1024);
         umma_bf16(tmem + L::T_Y, ah, bh, id_W, k > 0);
-        umma_bf16(tmem + L::T_Y, ah, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), id_W, 1);
-        umma_bf16(tmem + L::T_Y, desc_sw128(base + L::DA_LO + k * 2048, C * 128, 1024), bh, id_W, 1);
+        umma_bf16(tmem + L::T_Y, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), bh, id_W, 1);
+        umma_bf16(tmem + L::T_Y, ah, desc_sw128(base + L::DA_LO + k * 2048, C * 128, 1024), id_W, 1);
       }
       umma_commit(bar_m2);
     }
@@ -465,68 +472,77 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       ph_m2 ^= 1;
       tc_fence_after();
     }
-    {  // dk epilogue; per-token terms Kh Z (-> EF) and Kh Z + k dk^intra without j = r (-> SCR)
-      float z[32], w[32];
+    {  // dk epilogue: this thread owns key dimension d = row and the tokens rb .. rb+31
+      const int d = row, rb = half * 32;
+      float pv[32];  // the forward walk's part of dg for these tokens
+      float qxn = 0.f;
+      if (row_owner) {
+        const float4* src = reinterpret_cast<const float4*>(part + ((size_t)i * DK + d) * C + rb);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float4 u = src[c];
+          pv[4 * c] = u.x;
+          pv[4 * c + 1] = u.y;
+          pv[4 * c + 2] = u.z;
+          pv[4 * c + 3] = u.w;
+        }
+        if (n > 0) qxn = qx_sums[(size_t)(i + 1) * DK + d];
+      }
+      float z[32], w[32];  // rows of Z^T and W^T
       tmem_ld32(tmem + L::T_X + lane_off + half * 32, z);
       if (!safe) tmem_ld32(tmem + L::T_Y + lane_off + half * 32, w);
       tmem_ld_wait();
+      float tot_k = 0.f, tot_s = 0.f;
       if (row_owner) {
-        const int r = row, cb = half * 32;
-        float* e2 = EF + r * L::FS + cb;
-        const float arr = DIAG[r];
         if (safe) {
           const float* XB = reinterpret_cast<const float*>(sm + L::XB);
           const float* XA = reinterpret_cast<const float*>(sm + L::XA);
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
+            const int r = rb + c;
+            const float br = XB[r * KT + d];
             float acc = 0.f;
-            for (int j = r; j < C; ++j)
-              acc += XA[j * C + r] * raw(L::PB_Q, j, cb + c) * __expf(XB[j * KT + cb + c] - XB[r * KT + cb + c]);
-            w[c] = acc;
+            for (int j = r; j < C; ++j) acc += XA[j * C + r] * raw(L::PB_Q, j, d) * __expf(XB[j * KT + d] - br);
+            w[c] = acc;  // exact intra term
           }
         } else {
+          const float inv = 1.f / DEC[d];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) w[c] *= e2[c] / DEC[cb + c];
+          for (int c = 0; c < 32; ++c) w[c] *= EF[(rb + c) * L::FS + d] * inv;
         }
+        __nv_bfloat16* dst = a.dk + ((size_t)bh * T + i * C + rb) * DK + d0 + d;
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float qv = raw(L::PB_Q, r, cb + c), kv = raw(L::PB_K, r, cb + c);
-          const float ev = e2[c];
-          const float kz = bf_split_sum(kv * ev) * z[c];  // Kh as the S update sees it
-          e2[c] = kz;
-          SCR[r * L::FS + cb + c] = kz + kv * (w[c] - arr * qv);
-          z[c] = ev * z[c] + w[c];
+          const int r = rb + c;
+          const float qv = raw(L::PB_Q, r, d), kv = raw(L::PB_K, r, d), ev = EF[r * L::FS + d];
+          if (i * C + r < T) dst[(size_t)c * DK] = __float2bfloat16_rn(ev * z[c] + w[c]);
+          const float kz = bf_split_sum(kv * ev) * z[c];  // Kh Z, with Kh as the S update sees it
+          w[c] = kz + kv * (w[c] - DIAG[r] * qv);        // plus k dk^intra without j = r
+          tot_k += kz;
+          tot_s += w[c];
         }
-        const int t = i * C + r;
-        if (t < T) store_half_global_bf16(a.dk + ((size_t)bh * T + t) * DK + d0 + cb, z);
+        XCH[half * KT + d] = make_float2(tot_k, tot_s);
       }
-    }
-    __syncthreads();
-    if (tid < KT) {  // dg = c_i + prefix of (Kh Z + k dk^intra) + the forward walk's partial
-      const int d = tid;
-      float kz = 0.f;
-      for (int r = 0; r < C; ++r) kz += EF[r * L::FS + d];
-      const float ci = (n == 0 ? CARRY[d] : CARRY[d] + qx_sums[(size_t)(i + 1) * DK + d]) - kz;
-      float pre = 0.f;
-      for (int r0 = 0; r0 < C; r0 += 16) {
-        float pv[16];  // issue the 16 loads before the dependent prefix sum
+      __syncthreads();
+      if (tid == 0 && n + 1 < NC) {
+        if (safe) load_a(i - 1);
+        load_b(i - 1);
+      }
+      if (row_owner) {  // dg = c_i + prefix (exclusive) of (Kh Z + k dk^intra) + the forward walk's part
+        const float2 o = XCH[(half ^ 1) * KT + d];
+        const float ci = CARRY[(n & 1) * KT + d] + qxn - (tot_k + o.x);
+        float pre = half == 1 ? o.y : 0.f;
+        __nv_bfloat16* dst = a.dg + ((size_t)bh * T + i * C + rb) * DK + d0 + d;
 #pragma unroll
-        for (int u = 0; u < 16; ++u) pv[u] = (i * C + r0 + u < T) ? part[(size_t)(i * C + r0 + u) * DK + d] : 0.f;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int t = i * C + r0 + u;
-          if (t < T) a.dg[((size_t)bh * T + t) * DK + d0 + d] = __float2bfloat16_rn(ci + pre + pv[u]);
-          pre += SCR[(r0 + u) * L::FS + d];
+        for (int c = 0; c < 32; ++c) {
+          if (i * C + rb + c < T) dst[(size_t)c * DK] = __float2bfloat16_rn(ci + pre + pv[c]);
+          pre += w[c];
         }
+        if (half == 0) CARRY[((n + 1) & 1) * KT + d] = ci;
       }
-      CARRY[d] = ci;
     }
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && n + 1 < NC) {
-      if (safe) load_a(i - 1);
-      load_b(i - 1);
-    }
   }
   // dh0 rows = G_0
   if (a.dh0) {
@@ -823,8 +839,8 @@ bool bwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype) {
 }
 
 size_t bwd_workspace(int BH, int T, int dk, int) {
-  return align256((size_t)BH * ((T + C - 1) / C) * dk * sizeof(float)) +
-         align256((size_t)BH * T * dk * sizeof(float));
+  const size_t NC = (T + C - 1) / C;
+  return align256((size_t)BH * NC * dk * sizeof(float)) + align256((size_t)BH * NC * C * dk * sizeof(float));
 }
 
 template <int DK, int DV>
