@@ -225,10 +225,9 @@ def run_ours(args, cfg, name):
 
     from chunkwise_linear_rnn_02_b200 import binding as gla
     from chunkwise_linear_rnn_02_b200.inputs import make_gla_inputs
+    from chunkwise_linear_rnn_02_b200.ranks import batch_seed, max_over_ranks, rank_env, sum_over_ranks
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     if world > 1:
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -238,7 +237,7 @@ def run_ours(args, cfg, name):
     dev = torch.device("cuda", torch.cuda.current_device())
     gla.load_library()
 
-    inp = make_gla_inputs(cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.dtype, seed=1000 + rank)
+    inp = make_gla_inputs(cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.dtype, seed=batch_seed(1000, rank))
     d = {k: v.to(dev) for k, v in inp.items()}
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
@@ -278,10 +277,7 @@ def run_ours(args, cfg, name):
     bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     step_ms = fwd_ms + bwd_ms
     clocks = sampler.stop()
-    if world > 1:
-        t = torch.tensor([step_ms, fwd_ms, bwd_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms, fwd_ms, bwd_ms = t.tolist()
+    step_ms, fwd_ms, bwd_ms = max_over_ranks([step_ms, fwd_ms, bwd_ms], dev)
 
     # end-to-end through the public API with host buffers: H2D inputs, fwd, bwd, D2H results
     names_in = ["q", "k", "v", "g", "do"]
@@ -308,15 +304,12 @@ def run_ours(args, cfg, name):
             e2e_times.append(e0.elapsed_time(e1))
     d2h = sum(x.numel() * x.element_size() for x in outs_host)
     e2e_ms = statistics.mean(e2e_times)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
+    (e2e_ms,) = max_over_ranks([e2e_ms], dev)
 
     launches_per_step, kernel_names = (None, ["not counted"]) if args.no_launch_count else count_launches(step)
     peaks = load_peaks()
     fb, bb, ff, bf = algorithmic(cfg)
-    tokens = cfg.B * cfg.T * world
+    (tokens,) = sum_over_ranks([cfg.B * cfg.T], dev)
     t_roof = max((fb + bb) / (peaks["hbm_gbs"] * 1e9), (ff + bf) / (peaks["bf16_tflops"] * 1e12))
     # dominant call: the larger of the fwd and bwd device times
     if bwd_ms >= fwd_ms:
