@@ -35,7 +35,7 @@ namespace fast {
 using namespace sm100;
 
 constexpr int DVT = 64;      // value columns per CTA
-constexpr int NTHREADS = 128;
+constexpr int NTHREADS = 256;  // warps w and w+4 share TMEM lanes and split accumulator columns
 
 // ------------------------------------------------------------------------------------------
 // Forward kernel
@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
   const int dv0 = blockIdx.x * DVT, bh = blockIdx.y;
   const int NC = (T + C - 1) / C;
   float* decay_sm = reinterpret_cast<float*>(sm + L::DECAY);
@@ -114,16 +115,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (NC > 1) issue_load(1);
   }
 
-  // State rows owned by this thread: lane layout of the dS accumulator (M = DK).
+  // State owned by this thread: row s_row (lane layout of the dS accumulator, M = DK), columns
+  // sc0 .. sc0+31 of the CTA's 64.
+  constexpr int SW = DVT / 2;
   const bool s_owner = (DK == 128) ? true : (lane < 16);
-  const int s_row = (DK == 128) ? tid : (warp * 16 + lane);
-  float S[DVT];
+  const int s_row = (DK == 128) ? (q4 * 32 + lane) : (q4 * 16 + lane);
+  const int sc0 = half * SW;
+  float S[SW];
 #pragma unroll
-  for (int c = 0; c < DVT; ++c) S[c] = 0.f;
+  for (int c = 0; c < SW; ++c) S[c] = 0.f;
   if (s_owner && h0) {
-    const float4* src = reinterpret_cast<const float4*>(h0 + ((size_t)bh * DK + s_row) * DV + dv0);
+    const float4* src = reinterpret_cast<const float4*>(h0 + ((size_t)bh * DK + s_row) * DV + dv0 + sc0);
 #pragma unroll
-    for (int c = 0; c < DVT / 4; ++c) {
+    for (int c = 0; c < SW / 4; ++c) {
       const float4 x = src[c];
       S[4 * c] = x.x;
       S[4 * c + 1] = x.y;
@@ -137,7 +141,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   const uint32_t t_A = tmem, t_O = tmem + 64, t_dS = tmem + 128;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
 
   for (int i = 0; i < NC; ++i) {
     const int s = i & 1;
@@ -168,7 +172,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       });
     }
     // ---------------- state copy for the inter-chunk term: e^{gamma} S_i (or S_i in safe mode) ----
-    if (s_owner) store_row_split(sm + L::SB_HI, sm + L::SB_LO, s_row, S, safe ? 1.f : decay_sm[s_row]);
+    if (s_owner) {
+      const float sc = safe ? 1.f : decay_sm[s_row];
+      float sv[SW];
+#pragma unroll
+      for (int c = 0; c < SW; ++c) sv[c] = S[c] * sc;
+      store_half_split(sm + L::SB_HI, sm + L::SB_LO, s_row, sv, half);
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -233,32 +243,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     // ---------------- A epilogue: mask, hi/lo bf16, store as the K-major A operand ----------------
     {
-      const int j = warp * 16 + lane;
-      float a[64];
-      tmem_ld32(t_A + lane_off, a);
-      tmem_ld32(t_A + lane_off + 32, a + 32);
+      const int j = q4 * 16 + lane, cb = half * 32;
+      float a[32];
+      tmem_ld32(t_A + lane_off + cb, a);
       tmem_ld_wait();
       if (lane < 16) {
         if (safe) {
 #pragma unroll
-          for (int r = 0; r < 64; ++r) a[r] = Aex[j * C + r];
+          for (int c = 0; c < 32; ++c) a[c] = Aex[j * C + cb + c];
         }
 #pragma unroll
-        for (int r = 0; r < 64; ++r)
-          if (r > j) a[r] = 0.f;
-        store_row_split(sm + L::AB_HI, sm + L::AB_LO, j, a, 1.f);
+        for (int c = 0; c < 32; ++c)
+          if (cb + c > j) a[c] = 0.f;
+        store_half_split(sm + L::AB_HI, sm + L::AB_LO, j, a, half);
       }
     }
     // ---------------- state update: S = e^gamma S + dS (fp32 registers) ----------------
     {
-      float ds[64];
-      tmem_ld32(t_dS + lane_off, ds);
-      tmem_ld32(t_dS + lane_off + 32, ds + 32);
+      float ds[SW];
+      tmem_ld32(t_dS + lane_off + sc0, ds);
       tmem_ld_wait();
       if (s_owner) {
         const float dec = decay_sm[s_row];
 #pragma unroll
-        for (int c = 0; c < DVT; ++c) S[c] = dec * S[c] + ds[c];
+        for (int c = 0; c < SW; ++c) S[c] = dec * S[c] + ds[c];
       }
     }
     fence_async_smem();
@@ -285,13 +293,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     // ---------------- O epilogue: bf16 rows straight to global ----------------
     {
-      const int j = warp * 16 + lane;
-      float ov[64];
-      tmem_ld32(t_O + lane_off, ov);
-      tmem_ld32(t_O + lane_off + 32, ov + 32);
+      const int j = q4 * 16 + lane, cb = half * 32;
+      float ov[32];
+      tmem_ld32(t_O + lane_off + cb, ov);
       tmem_ld_wait();
       const int t = i * C + j;
-      if (lane < 16 && t < T) store_row_global_bf16(o + ((size_t)bh * T + t) * DV + dv0, ov);
+      if (lane < 16 && t < T) store_half_global_bf16(o + ((size_t)bh * T + t) * DV + dv0 + cb, ov);
     }
     tc_fence_before();
     __syncthreads();
@@ -299,9 +306,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 
   if (s_owner && hT) {
-    float4* dst = reinterpret_cast<float4*>(hT + ((size_t)bh * DK + s_row) * DV + dv0);
+    float4* dst = reinterpret_cast<float4*>(hT + ((size_t)bh * DK + s_row) * DV + dv0 + sc0);
 #pragma unroll
-    for (int c = 0; c < DVT / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
+    for (int c = 0; c < SW / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
   }
   tc_fence_before();
   __syncthreads();
