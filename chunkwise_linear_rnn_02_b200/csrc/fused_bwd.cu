@@ -73,37 +73,45 @@ template <int DK, int DV>
 struct KeyLayout {
   static constexpr uint32_t VB = C * DV * 2;        // a v or dO tile [64 x DV] (DV/64 swizzled boxes)
   static constexpr uint32_t TILE = C * KT * 2;      // a [64 x 64] bf16 tile
-  static constexpr uint32_t PA_V = 0, PA_DO = VB;   // part A: v, dO
-  static constexpr uint32_t PB = 2 * VB;            // part B: k, g, q tiles
-  static constexpr uint32_t PB_K = PB, PB_G = PB + TILE, PB_Q = PB + 2 * TILE;
-  static constexpr uint32_t KQ_HI = PB + 3 * TILE; // Kh (forward walk) / Qt (reverse walk), hi / lo
+  static constexpr uint32_t PA_V = 0, PA_DO = VB;   // part A: v, dO (one buffer)
+  static constexpr uint32_t PB = 2 * VB;            // part B: k, g, q tiles (two buffers)
+  static constexpr uint32_t PB_STAGE = 3 * TILE;
+  static constexpr uint32_t PB_K = 0, PB_G = TILE, PB_Q = 2 * TILE;  // offsets inside a part-B buffer
+  static constexpr uint32_t KQ_HI = PB + 2 * PB_STAGE;  // Kh (forward walk) / Qt (reverse walk), hi / lo
   static constexpr uint32_t KQ_LO = KQ_HI + TILE;
   static constexpr uint32_t SG_HI = KQ_LO + TILE;   // bf16 hi / lo copies of S or G rows [64 x DV], K-major
   static constexpr uint32_t SG_LO = SG_HI + KT * DV * 2;
   static constexpr uint32_t DA_HI = SG_LO + KT * DV * 2;  // masked dA, bf16 hi / lo [64 x 64]
   static constexpr uint32_t DA_LO = DA_HI + TILE;
-  static constexpr int FS = 66;                     // padded row stride of the fp32 [64][64] scratch
-  static constexpr uint32_t EF = DA_LO + TILE;      // fp32 [64][FS]: E1 (forward walk) / E2 (reverse walk)
-  static constexpr uint32_t XCH = EF + C * FS * 4;  // float2 [2][64]: token-half sums exchanged per dim
-  static constexpr uint32_t DEC = XCH + 2 * KT * 8;
-  static constexpr uint32_t TOT = DEC + KT * 4;     // [NSPLIT][64]
-  static constexpr uint32_t DIAG = TOT + GateRun<KT, BT>::NSPLIT * KT * 4;
-  static constexpr uint32_t CARRY = DIAG + C * 4;    // [2][64] c_i, double-buffered over chunks
+  static constexpr int NS = GateRun<KT, BT>::NSPLIT;
+  static constexpr uint32_t XCH = DA_LO + TILE;         // float2 [2][64]: token-half sums exchanged per dim
+  static constexpr uint32_t DEC = XCH + 2 * KT * 8;     // float [2][64]: chunk decays, per part-B buffer
+  static constexpr uint32_t TOT = DEC + 2 * KT * 4;     // float [2][NS][64]: gate run products, per buffer
+  static constexpr uint32_t DIAG = TOT + 2 * NS * KT * 4;
+  static constexpr uint32_t CARRY = DIAG + C * 4;       // [2][64] c_i, double-buffered over chunks
   static constexpr uint32_t CARRYP = CARRY + 2 * KT * 4;  // [2][64] per-column-half partial row sums
   static constexpr uint32_t TOTAL = CARRYP + 2 * KT * 4;
-  // exact-path scratch (only when the part-A prefetch is held back): B and dA in fp32
-  static constexpr uint32_t XB = PA_V, XA = PA_DO;
   // TMEM columns
   static constexpr uint32_t T_SG = 0, T_DA = DV, T_X = DV + 64, T_Y = DV + 128;
-  static_assert(VB >= C * KT * 4, "exact-path scratch fits in a part-A tile");
   static_assert(DV + 192 <= 512, "TMEM columns");
+  static_assert(PB % 1024 == 0 && PB_STAGE % 1024 == 0 && KQ_HI % 1024 == 0 && SG_HI % 1024 == 0 &&
+                    DA_HI % 1024 == 0,
+                "operand alignment");
 };
 
+// Key-tile schedule: chunk i's epilogue runs while chunk i+1's first MMA group is on the tensor
+// pipe.  Per chunk step: wait for MMA group 1 of chunk i, move its dA and X^T (Z^T) rows into
+// registers, issue group 2 (Y^T or W^T); then prepare chunk i+1 (gate run from the second part-B
+// buffer, Kh or Qt operand, state copy and rescale) and issue its group 1; then finish chunk i's
+// outputs.  The epilogue forms E1 / E2 itself from the raw gates and the run products of the gate
+// run, multiplying in the same order, so its values equal the ones behind the MMA operands.
 template <int DK, int DV>
 __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int tau, uint64_t* bars,
                               uint32_t tmem) {
   using L = KeyLayout<DK, DV>;
   using Gate = GateRun<KT, BT>;
+  constexpr int NS = L::NS, TS = Gate::TS;
+  static_assert(TS == 8 && NS == 8, "epilogue runs: four gate runs of eight tokens per token half");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
   const int T = a.T, NC = (T + C - 1) / C, d0 = tau * KT;
@@ -111,43 +119,67 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
   const bool row_owner = lane < 16;
   const int row = q4 * 16 + lane;  // row of an M=64 accumulator owned by this thread
+  const int tb = half * 32;        // first column (token) of this thread's half
   constexpr int HV = DV / 2;       // state columns per warp
   uint64_t* bar_pa = bars + 0;
-  uint64_t* bar_pb = bars + 1;
+  uint64_t* bar_pb = bars + 1;     // two barriers, one per part-B buffer
   uint64_t* bar_m1 = bars + 3;
   uint64_t* bar_m2 = bars + 4;
   uint32_t ph_pa = 0, ph_pb = 0, ph_m1 = 0, ph_m2 = 0;
   float* DEC = reinterpret_cast<float*>(sm + L::DEC);
   float* TOT = reinterpret_cast<float*>(sm + L::TOT);
-  float* EF = reinterpret_cast<float*>(sm + L::EF);
   float2* XCH = reinterpret_cast<float2*>(sm + L::XCH);
   float* DIAG = reinterpret_cast<float*>(sm + L::DIAG);
   float* CARRY = reinterpret_cast<float*>(sm + L::CARRY);
-  float* qx_sums = a.ws_qx + (size_t)bh * NC * DK + d0;  // [NC][DK] slice of this head and key tile
+  float* qx_sums = a.ws_qx + (size_t)bh * NC * DK + d0;          // [NC][DK] slice of this head and key tile
   float* part = a.ws_part + ((size_t)bh * NC * DK + d0) * C;  // [NC][DK][64] slice: forward-walk part of dg
 
+  auto pbo = [&](int b) { return L::PB + (uint32_t)b * L::PB_STAGE; };
   auto load_a = [&](int chunk) {
     mbar_arrive_expect_tx(bar_pa, 2 * L::VB);
-    for (int b = 0; b < DV / 64; ++b) {
-      tma_load_3d(sm + L::PA_V + b * (C * 128), &mp.v, bar_pa, b * 64, chunk * C, bh);
-      tma_load_3d(sm + L::PA_DO + b * (C * 128), &mp.dO, bar_pa, b * 64, chunk * C, bh);
+    for (int bb = 0; bb < DV / 64; ++bb) {
+      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, bar_pa, bb * 64, chunk * C, bh);
+      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, bar_pa, bb * 64, chunk * C, bh);
     }
   };
-  auto load_b = [&](int chunk) {
-    mbar_arrive_expect_tx(bar_pb, 3 * L::TILE);
-    tma_load_3d(sm + L::PB_K, &mp.k64, bar_pb, d0, chunk * C, bh);
-    tma_load_3d(sm + L::PB_G, &mp.g64, bar_pb, d0, chunk * C, bh);
-    tma_load_3d(sm + L::PB_Q, &mp.q64, bar_pb, d0, chunk * C, bh);
+  auto load_b = [&](int chunk, int b) {
+    uint8_t* pb = sm + pbo(b);
+    mbar_arrive_expect_tx(bar_pb + b, L::PB_STAGE);
+    tma_load_3d(pb + L::PB_K, &mp.k64, bar_pb + b, d0, chunk * C, bh);
+    tma_load_3d(pb + L::PB_G, &mp.g64, bar_pb + b, d0, chunk * C, bh);
+    tma_load_3d(pb + L::PB_Q, &mp.q64, bar_pb + b, d0, chunk * C, bh);
+  };
+  auto wait_b = [&](int b) {
+    mbar_wait(bar_pb + b, (ph_pb >> b) & 1u, a.latch);
+    ph_pb ^= 1u << b;
   };
   auto sync_tc = [&]() {
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
   };
-  // Element (token j, dim d) of a raw k / g / q tile (TMA 128-byte swizzle).
-  auto raw = [&](uint32_t tile, int j, int d) { return bf2f(sm + tile + sw128(j, d)); };
-  auto raw2 = [&](uint32_t tile, int j, int d) { return *reinterpret_cast<const uint32_t*>(sm + tile + sw128(j, d)); };
-  // Initialise the TMEM state rows and their hi/lo bf16 copies from a [DK x DV] fp32 source (or zeros).
+  // Element (token j, dim d) of a raw tile at shared-memory offset off (TMA 128-byte swizzle).
+  auto raw = [&](uint32_t off, int j, int d) { return bf2f(sm + off + sw128(j, d)); };
+  auto raw2 = [&](uint32_t off, int j, int d) { return *reinterpret_cast<const uint32_t*>(sm + off + sw128(j, d)); };
+  // dA (masked, as the MMAs see it: hi + lo) at (j, r).
+  auto dA_at = [&](int j, int r) { return raw(L::DA_HI, j, r) + raw(L::DA_LO, j, r); };
+  // Gate run of the chunk in part-B buffer b: run products into TOT[b], decays into DEC[b].
+  auto gate = [&](Gate& gr, int b) {
+    const bool weak = gr.run_swizzled(sm + pbo(b) + L::PB_G, TOT + b * NS * KT);
+    if (gr.h == 0) {
+      DEC[b * KT + gr.d] = gr.dec0;
+      DEC[b * KT + gr.d + 1] = gr.dec1;
+    }
+    return __syncthreads_or(weak);
+  };
+  auto write_kq = [&](uint32_t off, int j, int d, float e0, float e1) {
+    const uint32_t w = raw2(off, j, d);
+    uint32_t hi, lo;
+    split2(bf_lo(w) * e0, bf_hi(w) * e1, hi, lo);
+    *reinterpret_cast<uint32_t*>(sm + L::KQ_HI + sw128(j, d)) = hi;
+    *reinterpret_cast<uint32_t*>(sm + L::KQ_LO + sw128(j, d)) = lo;
+  };
+  // Initialise the TMEM state rows from a [DK x DV] fp32 source (or zeros).
   auto init_state = [&](const float* src) {
     float v[64];
     for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 64) {
@@ -156,217 +188,203 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         v[c] = (src && row_owner) ? src[((size_t)bh * DK + d0 + row) * DV + c0 + c] : 0.f;
       tmem_st32(tmem + L::T_SG + lane_off + c0, v);
       tmem_st32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
-      if (row_owner)
-        store_row_split(sm + L::SG_HI + (c0 / 64) * (KT * 128), sm + L::SG_LO + (c0 / 64) * (KT * 128), row, v, 1.f);
     }
     tmem_st_wait();
   };
-  // Rescale the TMEM state rows by DEC[row] (all lanes take part; only owners' rows matter).
-  auto rescale_state = [&]() {
-    const float s = row_owner ? DEC[row] : 0.f;
+  // TMEM state rows -> hi/lo bf16 K-major operand copy; then the rows scaled by DEC[b] (all lanes
+  // take part; only owners' rows matter).
+  auto state_pass = [&](int b) {
+    const float sc = row_owner ? DEC[b * KT + row] : 0.f;
     float v[64];
     for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 64) {
       tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
       tmem_ld32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
       tmem_ld_wait();
+      if (row_owner)
+        store_row_split(sm + L::SG_HI + (c0 / 64) * (KT * 128), sm + L::SG_LO + (c0 / 64) * (KT * 128), row, v, 1.f);
 #pragma unroll
-      for (int c = 0; c < 64; ++c) v[c] *= s;
+      for (int c = 0; c < 64; ++c) v[c] *= sc;
       tmem_st32(tmem + L::T_SG + lane_off + c0, v);
       tmem_st32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
     }
     tmem_st_wait();
   };
-  // Copy the TMEM state rows into the hi/lo bf16 K-major operands.
-  auto copy_state = [&]() {
-    float v[64];
-    for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 64) {
-      tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
-      tmem_ld32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
-      tmem_ld_wait();
-      if (row_owner)
-        store_row_split(sm + L::SG_HI + (c0 / 64) * (KT * 128), sm + L::SG_LO + (c0 / 64) * (KT * 128), row, v, 1.f);
-    }
-  };
-  // Cumulative log-gates of the key tile, fp32 [64][64], for the exact path.
-  auto exact_gates = [&]() {
-    float* XB = reinterpret_cast<float*>(sm + L::XB);
-    if (tid < KT) {
-      float b = 0.f;
-      for (int j = 0; j < C; ++j) {
-        b += raw(L::PB_G, j, tid);
-        XB[j * KT + tid] = b;
-      }
-    }
-  };
-  // dA epilogue: masked bf16 operand, its diagonal, and (exact path) an fp32 copy.
-  auto dA_epilogue = [&](int safe) {
+  // dA epilogue: masked bf16 hi / lo operand and its diagonal.
+  auto dA_epilogue = [&]() {
     float v[32];
-    tmem_ld32(tmem + L::T_DA + lane_off + half * 32, v);
+    tmem_ld32(tmem + L::T_DA + lane_off + tb, v);
     tmem_ld_wait();
     if (row_owner) {
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        if (half * 32 + c > row) v[c] = 0.f;
-        if (half * 32 + c == row) DIAG[row] = v[c];
+        if (tb + c > row) v[c] = 0.f;
+        if (tb + c == row) DIAG[row] = v[c];
       }
       store_half_split(sm + L::DA_HI, sm + L::DA_LO, row, v, half);
-      if (safe) {
-        float* XA = reinterpret_cast<float*>(sm + L::XA);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) XA[row * C + half * 32 + c] = v[c];
-      }
     }
   };
-  auto mma_dA = [&](int k, uint32_t ko) {
+  // MMA group 1: dA = dO V^T; X^T = S dO^T (forward) or Z^T = G V^T (reverse); and the state
+  // update S += Kh^T V (forward) or G += Qt^T dO (reverse).
+  auto issue_m1 = [&](bool fwd) {
+    if (tid != 0) return;
+    mbar_wait(bar_pa, ph_pa, a.latch);
+    ph_pa ^= 1;
+    tc_fence_after();
     constexpr uint32_t id_dA = idesc_bf16_f32(C, C, false, false);
-    umma_bf16(tmem + L::T_DA, desc_sw128(base + L::PA_DO + ko, 16, 1024), desc_sw128(base + L::PA_V + ko, 16, 1024),
-              id_dA, k > 0);
+    constexpr uint32_t id_X = idesc_bf16_f32(KT, C, false, false);
+    constexpr uint32_t id_S = idesc_bf16_f32(KT, DV, true, true);
+    const uint32_t xb = fwd ? L::PA_DO : L::PA_V, sb = fwd ? L::PA_V : L::PA_DO;
+#pragma unroll
+    for (int k = 0; k < DV / 16; ++k) {
+      const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
+      const uint64_t bd = desc_sw128(base + xb + ko, 16, 1024);
+      umma_bf16(tmem + L::T_DA, desc_sw128(base + L::PA_DO + ko, 16, 1024),
+                desc_sw128(base + L::PA_V + ko, 16, 1024), id_dA, k > 0);
+      umma_bf16(tmem + L::T_X, desc_sw128(base + L::SG_HI + ko, 16, 1024), bd, id_X, k > 0);
+      umma_bf16(tmem + L::T_X, desc_sw128(base + L::SG_LO + ko, 16, 1024), bd, id_X, 1);
+    }
+#pragma unroll
+    for (int k = 0; k < C / 16; ++k) {
+      const uint64_t dd = desc_sw128(base + sb + k * 2048, C * 128, 1024);
+      umma_bf16(tmem + L::T_SG, desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024), dd, id_S, 1);
+      umma_bf16(tmem + L::T_SG, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), dd, id_S, 1);
+    }
+    umma_commit(bar_m1);
+  };
+  // MMA group 2: Y^T = Kh^T dA^T (forward) or W^T = Qt^T dA (reverse).
+  auto issue_m2 = [&](bool fwd) {
+    if (tid != 0) return;
+    constexpr uint32_t id_Y = idesc_bf16_f32(KT, C, true, false);
+    constexpr uint32_t id_W = idesc_bf16_f32(KT, C, true, true);
+#pragma unroll
+    for (int k = 0; k < C / 16; ++k) {
+      const uint64_t ah = desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024);
+      const uint64_t al = desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024);
+      const uint64_t bh = fwd ? desc_sw128(base + L::DA_HI + k * 32, 16, 1024)
+                              : desc_sw128(base + L::DA_HI + k * 2048, C * 128, 1024);
+      const uint64_t bl = fwd ? desc_sw128(base + L::DA_LO + k * 32, 16, 1024)
+                              : desc_sw128(base + L::DA_LO + k * 2048, C * 128, 1024);
+      const uint32_t id = fwd ? id_Y : id_W;
+      umma_bf16(tmem + L::T_Y, ah, bh, id, k > 0);
+      umma_bf16(tmem + L::T_Y, al, bh, id, 1);
+      umma_bf16(tmem + L::T_Y, ah, bl, id, 1);
+    }
+    umma_commit(bar_m2);
+  };
+  auto wait_m2 = [&]() {
+    mbar_wait(bar_m2, ph_m2, a.latch);
+    ph_m2 ^= 1;
+    tc_fence_after();
+  };
+  // Chunk i+1 (or i-1): gate run from buffer nb, Kh / Qt operand, state copy + rescale, group 1.
+  // The operand area KQ is free once group 2 of the current chunk has completed.
+  auto prepare = [&](bool fwd, int nb, int m2_pending) {
+    wait_b(nb);
+    Gate gr;
+    const int safe = gate(gr, nb);
+    if (m2_pending) wait_m2();
+    const uint32_t off = pbo(nb) + (fwd ? L::PB_K : L::PB_Q);
+    if (fwd)
+      gr.backward([&](int j, float e0, float e1) { write_kq(off, j, gr.d, e0, e1); });
+    else
+      gr.forward([&](int j, float e0, float e1) { write_kq(off, j, gr.d, e0, e1); });
+    state_pass(nb);
+    fence_async_smem();
+    sync_tc();
+    issue_m1(fwd);
+    return safe;
   };
 
   // ============================ forward walk: dq, first part of dg ============================
   if (tid == 0) {
     load_a(0);
-    load_b(0);
+    load_b(0, 0);
+    if (NC > 1) load_b(1, 1);
   }
   init_state(a.h0);
+  int safe_next = prepare(true, 0, 0);
   for (int i = 0; i < NC; ++i) {
-    mbar_wait(bar_pa, ph_pa, a.latch);
-    ph_pa ^= 1;
-    mbar_wait(bar_pb, ph_pb, a.latch);
-    ph_pb ^= 1;
-    Gate gr;
-    const bool weak = gr.run_swizzled(sm + L::PB_G, TOT);
-    gr.backward([&](int j, float e0, float e1) {
-      const uint32_t wk = raw2(L::PB_K, j, gr.d);
-      uint32_t hi, lo;
-      split2(bf_lo(wk) * e0, bf_hi(wk) * e1, hi, lo);
-      *reinterpret_cast<uint32_t*>(sm + L::KQ_HI + sw128(j, gr.d)) = hi;
-      *reinterpret_cast<uint32_t*>(sm + L::KQ_LO + sw128(j, gr.d)) = lo;
-    });
-    gr.forward([&](int j, float e0, float e1) {
-      *reinterpret_cast<float2*>(EF + j * L::FS + gr.d) = make_float2(e0, e1);
-    });
-    if (gr.h == 0) {
-      DEC[gr.d] = gr.dec0;
-      DEC[gr.d + 1] = gr.dec1;
-    }
-    const int safe = __syncthreads_or(weak);
-    rescale_state();
-    fence_async_smem();
-    sync_tc();
-    if (tid == 0) {
-      constexpr uint32_t id_X = idesc_bf16_f32(KT, C, false, false);  // X^T = S dO^T
-      constexpr uint32_t id_S = idesc_bf16_f32(KT, DV, true, true);
-#pragma unroll
-      for (int k = 0; k < DV / 16; ++k) {
-        const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
-        const uint64_t bd = desc_sw128(base + L::PA_DO + ko, 16, 1024);
-        mma_dA(k, ko);
-        umma_bf16(tmem + L::T_X, desc_sw128(base + L::SG_HI + ko, 16, 1024), bd, id_X, k > 0);
-        umma_bf16(tmem + L::T_X, desc_sw128(base + L::SG_LO + ko, 16, 1024), bd, id_X, 1);
-      }
-#pragma unroll
-      for (int k = 0; k < C / 16; ++k) {
-        const uint64_t vd = desc_sw128(base + L::PA_V + k * 2048, C * 128, 1024);
-        umma_bf16(tmem + L::T_SG, desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024), vd, id_S, 1);
-        umma_bf16(tmem + L::T_SG, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), vd, id_S, 1);
-      }
-      umma_commit(bar_m1);
-    }
-    __syncwarp();
+    const int b = i & 1, safe = safe_next;
     mbar_wait(bar_m1, ph_m1, a.latch);
     ph_m1 ^= 1;
     tc_fence_after();
-    if (tid == 0 && !safe && i + 1 < NC) load_a(i + 1);
-    dA_epilogue(safe);
+    if (tid == 0 && i + 1 < NC) load_a(i + 1);
+    float x[32];  // this thread's row of X^T: key dim d = row, tokens tb .. tb+31
+    tmem_ld32(tmem + L::T_X + lane_off + tb, x);
+    dA_epilogue();
     fence_async_smem();
     sync_tc();
-    if (tid == 0 && !safe) {
-      constexpr uint32_t id_Y = idesc_bf16_f32(KT, C, true, false);  // Y^T = Kh^T dA^T
-#pragma unroll
-      for (int k = 0; k < C / 16; ++k) {
-        const uint64_t ah = desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024);
-        const uint64_t bh = desc_sw128(base + L::DA_HI + k * 32, 16, 1024);
-        umma_bf16(tmem + L::T_Y, ah, bh, id_Y, k > 0);
-        umma_bf16(tmem + L::T_Y, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), bh, id_Y, 1);
-        umma_bf16(tmem + L::T_Y, ah, desc_sw128(base + L::DA_LO + k * 32, 16, 1024), id_Y, 1);
-      }
-      umma_commit(bar_m2);
-    }
-    copy_state();
-    if (safe) {
-      exact_gates();
-      __syncthreads();
-    } else {
-      __syncwarp();
-      mbar_wait(bar_m2, ph_m2, a.latch);
-      ph_m2 ^= 1;
-      tc_fence_after();
-    }
-    {  // dq epilogue: this thread owns key dimension d = row and the tokens jb .. jb+31
-      float x[32], y[32];  // rows of X^T and Y^T
-      tmem_ld32(tmem + L::T_X + lane_off + half * 32, x);
-      if (!safe) tmem_ld32(tmem + L::T_Y + lane_off + half * 32, y);
+    if (!safe) issue_m2(true);
+    if (i + 1 < NC)
+      safe_next = prepare(true, b ^ 1, !safe);
+    else if (!safe)
+      wait_m2();
+    float y[32];  // this thread's row of Y^T
+    if (!safe) {
+      tmem_ld32(tmem + L::T_Y + lane_off + tb, y);
       tmem_ld_wait();
-      if (row_owner) {
-        const int d = row, jb = half * 32;
-        if (safe) {
-          const float* XB = reinterpret_cast<const float*>(sm + L::XB);
-          const float* XA = reinterpret_cast<const float*>(sm + L::XA);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int j = jb + c;
-            const float bj = XB[j * KT + d];
-            float acc = 0.f;
-            for (int r = 0; r <= j; ++r) acc += XA[j * C + r] * raw(L::PB_K, r, d) * __expf(bj - XB[r * KT + d]);
-            y[c] = acc;  // exact intra term
-          }
-        } else {
-          const float inv = 1.f / DEC[d];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) y[c] *= EF[(jb + c) * L::FS + d] * inv;
-        }
-        __nv_bfloat16* dst = a.dq + ((size_t)bh * T + i * C + jb) * DK + d0 + d;
-        float tot_s = 0.f, tot_e = 0.f;
+    }
+    float tot_s = 0.f, tot_e = 0.f;
+    if (row_owner) {  // dq; per-token terms Qt X (-> x) and q dq^intra without j = r (-> y)
+      const int d = row;
+      const uint32_t pk = pbo(b) + L::PB_K, pg = pbo(b) + L::PB_G, pq = pbo(b) + L::PB_Q;
+      const float* tot = TOT + b * NS * KT;
+      if (safe) {  // exact intra term y_j = sum_{r<=j} dA_jr k_r e^{B_j - B_r}
+        float bj = 0.f;
+        for (int t = 0; t < tb; ++t) bj += raw(pg, t, d);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const int j = jb + c;
-          const float qv = raw(L::PB_Q, j, d), kv = raw(L::PB_K, j, d), ev = EF[j * L::FS + d];
-          if (i * C + j < T) dst[(size_t)c * DK] = __float2bfloat16_rn(ev * x[c] + y[c]);
-          x[c] = bf_split_sum(qv * ev) * x[c];  // Qt X, with Qt as the G update sees it
-          y[c] = qv * (y[c] - DIAG[j] * kv);    // q dq^intra without j = r
+          bj += raw(pg, tb + c, d);
+          float acc = 0.f, br = 0.f;
+          for (int r = 0; r <= tb + c; ++r) {
+            br += raw(pg, r, d);
+            acc += dA_at(tb + c, r) * raw(pk, r, d) * __expf(bj - br);
+          }
+          y[c] = acc;
+        }
+      }
+      const float inv = 1.f / DEC[b * KT + d];
+      __nv_bfloat16* dst = a.dq + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        float e = 1.f;  // E1 = e^{B_j}, formed as GateRun::forward forms it
+        for (int hh = 0; hh < half * 4 + rr; ++hh) e *= tot[hh * KT + d];
+#pragma unroll
+        for (int u = 0; u < TS; ++u) {
+          const int c = rr * TS + u, j = tb + c;
+          e *= ex2(raw(pg, j, d) * kLog2e);
+          if (!safe) y[c] *= e * inv;
+          const float qv = raw(pq, j, d), kv = raw(pk, j, d);
+          if (i * C + j < T) dst[(size_t)c * DK] = __float2bfloat16_rn(e * x[c] + y[c]);
+          x[c] = bf_split_sum(qv * e) * x[c];  // Qt X, with Qt as the G update sees it
+          y[c] = qv * (y[c] - DIAG[j] * kv);   // q dq^intra without j = r
           tot_s += x[c];
           tot_e += y[c];
         }
-        XCH[half * KT + d] = make_float2(tot_s, tot_e);
       }
-      __syncthreads();
-      if (tid == 0 && i + 1 < NC) {
-        if (safe) load_a(i + 1);
-        load_b(i + 1);
-      }
-      if (row_owner) {  // part = suffix (inclusive) of Qt X minus prefix (exclusive) of q dq^intra
-        const int d = row, jb = half * 32;
-        const float2 o = XCH[(half ^ 1) * KT + d];
-        float suf = half == 0 ? o.x : 0.f, pre = half == 1 ? o.y : 0.f;
-#pragma unroll
-        for (int c = 31; c >= 0; --c) {
-          suf += x[c];
-          x[c] = suf;
-        }
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] -= pre;
-          pre += y[c];
-        }
-        float4* dst = reinterpret_cast<float4*>(part + ((size_t)i * DK + d) * C + jb);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
-        if (half == 0) qx_sums[(size_t)i * DK + d] = suf;
-      }
+      XCH[half * KT + d] = make_float2(tot_s, tot_e);
     }
-    tc_fence_before();
     __syncthreads();
+    if (tid == 0 && i + 2 < NC) load_b(i + 2, b);
+    if (row_owner) {  // part = suffix (inclusive) of Qt X minus prefix (exclusive) of q dq^intra
+      const int d = row;
+      const float2 o = XCH[(half ^ 1) * KT + d];
+      float suf = half == 0 ? o.x : 0.f, pre = half == 1 ? o.y : 0.f;
+#pragma unroll
+      for (int c = 31; c >= 0; --c) {
+        suf += x[c];
+        x[c] = suf;
+      }
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        x[c] -= pre;
+        pre += y[c];
+      }
+      float4* dst = reinterpret_cast<float4*>(part + ((size_t)i * DK + d) * C + tb);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+      if (half == 0) qx_sums[(size_t)i * DK + d] = suf;
+    }
   }
 
   // rowsum(dhT * hT): hT rows = the state after the forward walk
@@ -394,159 +412,111 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   // ============================ reverse walk: dk, dg, dh0 ============================
   if (tid == 0) {
     load_a(NC - 1);
-    load_b(NC - 1);
+    load_b(NC - 1, 0);
+    if (NC > 1) load_b(NC - 2, 1);
   }
   init_state(a.dhT);
+  safe_next = prepare(false, 0, 0);
   for (int n = 0; n < NC; ++n) {
-    const int i = NC - 1 - n;
-    mbar_wait(bar_pa, ph_pa, a.latch);
-    ph_pa ^= 1;
-    mbar_wait(bar_pb, ph_pb, a.latch);
-    ph_pb ^= 1;
-    Gate gr;
-    const bool weak = gr.run_swizzled(sm + L::PB_G, TOT);
-    gr.forward([&](int j, float e0, float e1) {
-      const uint32_t wq = raw2(L::PB_Q, j, gr.d);
-      uint32_t hi, lo;
-      split2(bf_lo(wq) * e0, bf_hi(wq) * e1, hi, lo);
-      *reinterpret_cast<uint32_t*>(sm + L::KQ_HI + sw128(j, gr.d)) = hi;
-      *reinterpret_cast<uint32_t*>(sm + L::KQ_LO + sw128(j, gr.d)) = lo;
-    });
-    gr.backward([&](int j, float e0, float e1) {
-      *reinterpret_cast<float2*>(EF + j * L::FS + gr.d) = make_float2(e0, e1);
-    });
-    if (gr.h == 0) {
-      DEC[gr.d] = gr.dec0;
-      DEC[gr.d + 1] = gr.dec1;
-    }
-    const int safe = __syncthreads_or(weak);
-    rescale_state();
-    fence_async_smem();
-    sync_tc();
-    if (tid == 0) {
-      constexpr uint32_t id_Z = idesc_bf16_f32(KT, C, false, false);  // Z^T = G V^T
-      constexpr uint32_t id_G = idesc_bf16_f32(KT, DV, true, true);
-#pragma unroll
-      for (int k = 0; k < DV / 16; ++k) {
-        const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
-        const uint64_t vd = desc_sw128(base + L::PA_V + ko, 16, 1024);
-        mma_dA(k, ko);
-        umma_bf16(tmem + L::T_X, desc_sw128(base + L::SG_HI + ko, 16, 1024), vd, id_Z, k > 0);
-        umma_bf16(tmem + L::T_X, desc_sw128(base + L::SG_LO + ko, 16, 1024), vd, id_Z, 1);
-      }
-#pragma unroll
-      for (int k = 0; k < C / 16; ++k) {
-        const uint64_t dd = desc_sw128(base + L::PA_DO + k * 2048, C * 128, 1024);
-        umma_bf16(tmem + L::T_SG, desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024), dd, id_G, 1);
-        umma_bf16(tmem + L::T_SG, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), dd, id_G, 1);
-      }
-      umma_commit(bar_m1);
-    }
-    __syncwarp();
+    const int i = NC - 1 - n, b = n & 1, safe = safe_next;
     mbar_wait(bar_m1, ph_m1, a.latch);
     ph_m1 ^= 1;
     tc_fence_after();
-    if (tid == 0 && !safe && n + 1 < NC) load_a(i - 1);
-    dA_epilogue(safe);
+    if (tid == 0 && n + 1 < NC) load_a(i - 1);
+    float z[32];  // this thread's row of Z^T: key dim d = row, tokens tb .. tb+31
+    tmem_ld32(tmem + L::T_X + lane_off + tb, z);
+    dA_epilogue();
     fence_async_smem();
     sync_tc();
-    if (tid == 0 && !safe) {
-      constexpr uint32_t id_W = idesc_bf16_f32(KT, C, true, true);  // W^T = Qt^T dA
+    if (!safe) issue_m2(false);
+    float pv[32];  // the forward walk's part of dg for these tokens
+    float qxn = 0.f;
+    if (row_owner) {
+      const float4* src = reinterpret_cast<const float4*>(part + ((size_t)i * DK + row) * C + tb);
 #pragma unroll
-      for (int k = 0; k < C / 16; ++k) {
-        const uint64_t ah = desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024);
-        const uint64_t bh = desc_sw128(base + L::DA_HI + k * 2048, C * 128, 1024);
-        umma_bf16(tmem + L::T_Y, ah, bh, id_W, k > 0);
-        umma_bf16(tmem + L::T_Y, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), bh, id_W, 1);
-        umma_bf16(tmem + L::T_Y, ah, desc_sw128(base + L::DA_LO + k * 2048, C * 128, 1024), id_W, 1);
+      for (int c = 0; c < 8; ++c) {
+        const float4 u = src[c];
+        pv[4 * c] = u.x;
+        pv[4 * c + 1] = u.y;
+        pv[4 * c + 2] = u.z;
+        pv[4 * c + 3] = u.w;
       }
-      umma_commit(bar_m2);
+      if (n > 0) qxn = qx_sums[(size_t)(i + 1) * DK + row];
     }
-    copy_state();
-    if (safe) {
-      exact_gates();
-      __syncthreads();
-    } else {
-      __syncwarp();
-      mbar_wait(bar_m2, ph_m2, a.latch);
-      ph_m2 ^= 1;
-      tc_fence_after();
-    }
-    {  // dk epilogue: this thread owns key dimension d = row and the tokens rb .. rb+31
-      const int d = row, rb = half * 32;
-      float pv[32];  // the forward walk's part of dg for these tokens
-      float qxn = 0.f;
-      if (row_owner) {
-        const float4* src = reinterpret_cast<const float4*>(part + ((size_t)i * DK + d) * C + rb);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float4 u = src[c];
-          pv[4 * c] = u.x;
-          pv[4 * c + 1] = u.y;
-          pv[4 * c + 2] = u.z;
-          pv[4 * c + 3] = u.w;
-        }
-        if (n > 0) qxn = qx_sums[(size_t)(i + 1) * DK + d];
-      }
-      float z[32], w[32];  // rows of Z^T and W^T
-      tmem_ld32(tmem + L::T_X + lane_off + half * 32, z);
-      if (!safe) tmem_ld32(tmem + L::T_Y + lane_off + half * 32, w);
+    if (n + 1 < NC)
+      safe_next = prepare(false, b ^ 1, !safe);
+    else if (!safe)
+      wait_m2();
+    float w[32];  // this thread's row of W^T
+    if (!safe) {
+      tmem_ld32(tmem + L::T_Y + lane_off + tb, w);
       tmem_ld_wait();
-      float tot_k = 0.f, tot_s = 0.f;
-      if (row_owner) {
-        if (safe) {
-          const float* XB = reinterpret_cast<const float*>(sm + L::XB);
-          const float* XA = reinterpret_cast<const float*>(sm + L::XA);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int r = rb + c;
-            const float br = XB[r * KT + d];
-            float acc = 0.f;
-            for (int j = r; j < C; ++j) acc += XA[j * C + r] * raw(L::PB_Q, j, d) * __expf(XB[j * KT + d] - br);
-            w[c] = acc;  // exact intra term
-          }
-        } else {
-          const float inv = 1.f / DEC[d];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) w[c] *= EF[(rb + c) * L::FS + d] * inv;
-        }
-        __nv_bfloat16* dst = a.dk + ((size_t)bh * T + i * C + rb) * DK + d0 + d;
+    }
+    float tot_k = 0.f, tot_s = 0.f;
+    if (row_owner) {  // dk; per-token terms Kh Z (-> z) and Kh Z + k dk^intra without j = r (-> w)
+      const int d = row;
+      const uint32_t pk = pbo(b) + L::PB_K, pg = pbo(b) + L::PB_G, pq = pbo(b) + L::PB_Q;
+      const float* tot = TOT + b * NS * KT;
+      if (safe) {  // exact intra term w_r = sum_{j>=r} dA_jr q_j e^{B_j - B_r}
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const int r = rb + c;
-          const float qv = raw(L::PB_Q, r, d), kv = raw(L::PB_K, r, d), ev = EF[r * L::FS + d];
+          const int r = tb + c;
+          float acc = dA_at(r, r) * raw(pq, r, d), bd = 0.f;
+          for (int j = r + 1; j < C; ++j) {
+            bd += raw(pg, j, d);
+            acc += dA_at(j, r) * raw(pq, j, d) * __expf(bd);
+          }
+          w[c] = acc;
+        }
+      }
+      const float inv = 1.f / DEC[b * KT + d];
+      __nv_bfloat16* dst = a.dk + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const int h = half * 4 + rr;
+        float al[TS], e2[TS];
+#pragma unroll
+        for (int u = 0; u < TS; ++u) al[u] = ex2(raw(pg, h * TS + u, d) * kLog2e);
+        float e = 1.f;  // E2 = e^{gamma - B_r}, formed as GateRun::backward forms it
+        for (int hh = h + 1; hh < NS; ++hh) e *= tot[hh * KT + d];
+#pragma unroll
+        for (int u = TS - 1; u >= 0; --u) {
+          e2[u] = e;
+          e *= al[u];
+        }
+#pragma unroll
+        for (int u = 0; u < TS; ++u) {
+          const int c = rr * TS + u, r = tb + c;
+          const float ev = e2[u];
+          if (!safe) w[c] *= ev * inv;
+          const float qv = raw(pq, r, d), kv = raw(pk, r, d);
           if (i * C + r < T) dst[(size_t)c * DK] = __float2bfloat16_rn(ev * z[c] + w[c]);
           const float kz = bf_split_sum(kv * ev) * z[c];  // Kh Z, with Kh as the S update sees it
           w[c] = kz + kv * (w[c] - DIAG[r] * qv);        // plus k dk^intra without j = r
           tot_k += kz;
           tot_s += w[c];
         }
-        XCH[half * KT + d] = make_float2(tot_k, tot_s);
       }
-      __syncthreads();
-      if (tid == 0 && n + 1 < NC) {
-        if (safe) load_a(i - 1);
-        load_b(i - 1);
-      }
-      if (row_owner) {  // dg = c_i + prefix (exclusive) of (Kh Z + k dk^intra) + the forward walk's part
-        const float2 o = XCH[(half ^ 1) * KT + d];
-        const float ci = CARRY[(n & 1) * KT + d] + qxn - (tot_k + o.x);
-        float pre = half == 1 ? o.y : 0.f;
-        __nv_bfloat16* dst = a.dg + ((size_t)bh * T + i * C + rb) * DK + d0 + d;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          if (i * C + rb + c < T) dst[(size_t)c * DK] = __float2bfloat16_rn(ci + pre + pv[c]);
-          pre += w[c];
-        }
-        if (half == 0) CARRY[((n + 1) & 1) * KT + d] = ci;
-      }
+      XCH[half * KT + d] = make_float2(tot_k, tot_s);
     }
-    tc_fence_before();
     __syncthreads();
+    if (tid == 0 && n + 2 < NC) load_b(i - 2, b);
+    if (row_owner) {  // dg = c_i + prefix (exclusive) of (Kh Z + k dk^intra) + the forward walk's part
+      const int d = row;
+      const float2 o = XCH[(half ^ 1) * KT + d];
+      const float ci = CARRY[(n & 1) * KT + d] + qxn - (tot_k + o.x);
+      float pre = half == 1 ? o.y : 0.f;
+      __nv_bfloat16* dst = a.dg + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        if (i * C + tb + c < T) dst[(size_t)c * DK] = __float2bfloat16_rn(ci + pre + pv[c]);
+        pre += w[c];
+      }
+      if (half == 0) CARRY[((n + 1) & 1) * KT + d] = ci;
+    }
   }
   // dh0 rows = G_0
   if (a.dh0) {
-    tc_fence_after();
     float v[32];
     for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 32) {
       tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
