@@ -26,6 +26,15 @@
 // Operand layouts are the 128-byte-swizzled forms described in sm100.cuh; V comes straight from a
 // TMA tile load and serves as the MN-major B operand of two MMAs; Kh, stored [token][dim], is the
 // K-major B operand of A and the MN-major A operand of dS.
+//
+// Sequence split.  When the (head, value tile) CTAs alone would leave most SMs idle (few heads, long
+// sequences), the chunks are cut into nseg segments and the state recurrence is evaluated as an
+// affine scan over them ("MS-GLA ...", section 2.1: the state update S <- diag(decay) S + dS is an
+// affine map, so maps compose): (1) a state-only pass gives, per segment, the end state reached from
+// zero (from h0 for the first segment) and the segment's decay product Gamma; (2) a scan
+// S_in(s+1) = Gamma_s * S_in(s) + S_local(s) gives every segment's entry state; (3) the full kernel
+// runs each segment from its entry state.  Nothing else changes: the per-chunk arithmetic of (3)
+// is the one above, so the outputs differ from the unsplit run only by rounding.
 #include "fast_path.cuh"
 #include "fused_common.cuh"
 
@@ -65,13 +74,28 @@ struct FwdLayout {
   static_assert(C * DK * 4 <= KH - QS_HI && C * C * 4 <= SB_LO - KH, "exact-path scratch");
 };
 
-template <int DK>
+struct FwdArgs {
+  const float* h0;     // [BH][DK][DV] or null (zeros)
+  float* sbuf;         // [BH][nseg][DK][DV]: segment end states (state-only pass), then entry states
+  float* gam;          // [BH][nseg][DK]: segment decay products
+  __nv_bfloat16* o;
+  float* hT;           // [BH][DK][DV] or null
+  int T, DV, seg_chunks, nseg;
+  unsigned int* latch;
+};
+
+// One CTA per (64 value columns, head, segment).  STATE_ONLY: the state recurrence alone (no
+// queries, no outputs), writing the segment's end state and decay product.
+template <int DK, bool STATE_ONLY>
 __global__ void __launch_bounds__(NTHREADS, 1)
     fwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
-                     const float* __restrict__ h0, __nv_bfloat16* __restrict__ o, float* __restrict__ hT, int T,
-                     int DV, unsigned int* latch) {
+                     const FwdArgs args) {
   using L = FwdLayout<DK>;
+  const float* h0 = args.h0;
+  __nv_bfloat16* o = args.o;
+  const int T = args.T, DV = args.DV;
+  unsigned int* latch = args.latch;
   using Gate = GateRun<DK, NTHREADS>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_load[2], bar_mma1, bar_mma2;
@@ -80,8 +104,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
-  const int dv0 = blockIdx.x * DVT, bh = blockIdx.y;
+  const int dv0 = blockIdx.x * DVT, bh = blockIdx.y, seg = blockIdx.z;
   const int NC = (T + C - 1) / C;
+  const int c_begin = seg * args.seg_chunks;
+  const int nloc = min(NC, c_begin + args.seg_chunks) - c_begin;  // chunks of this segment
   float* decay_sm = reinterpret_cast<float*>(sm + L::DECAY);
   float* tot_sm = reinterpret_cast<float*>(sm + L::TOT);
 
@@ -101,18 +127,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     fence_mbar_init();
   }
   __syncthreads();
-  auto issue_load = [&](int chunk) {
-    const int s = chunk & 1;
+  // Local chunk li of the segment into stage li & 1 (the state-only pass skips q).
+  auto issue_load = [&](int li) {
+    const int s = li & 1, chunk = c_begin + li;
     uint8_t* st = sm + s * L::STAGE;
-    mbar_arrive_expect_tx(&bar_load[s], L::STAGE);
-    tma_load_3d(st, &tm_q, &bar_load[s], 0, chunk * C, bh);
+    mbar_arrive_expect_tx(&bar_load[s], STATE_ONLY ? L::STAGE - L::RAW : L::STAGE);
+    if (!STATE_ONLY) tma_load_3d(st, &tm_q, &bar_load[s], 0, chunk * C, bh);
     tma_load_3d(st + L::RAW, &tm_k, &bar_load[s], 0, chunk * C, bh);
     tma_load_3d(st + 2 * L::RAW, &tm_g, &bar_load[s], 0, chunk * C, bh);
     tma_load_3d(st + 3 * L::RAW, &tm_v, &bar_load[s], dv0, chunk * C, bh);
   };
   if (tid == 0) {
     issue_load(0);
-    if (NC > 1) issue_load(1);
+    if (nloc > 1) issue_load(1);
   }
 
   // State owned by this thread: row s_row (lane layout of the dS accumulator, M = DK), columns
@@ -124,8 +151,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   float S[SW];
 #pragma unroll
   for (int c = 0; c < SW; ++c) S[c] = 0.f;
-  if (s_owner && h0) {
-    const float4* src = reinterpret_cast<const float4*>(h0 + ((size_t)bh * DK + s_row) * DV + dv0 + sc0);
+  // Entry state: h0 for the first segment; the scanned entry state for the others (full pass).
+  const float* init = seg == 0 ? (h0 ? h0 + (size_t)bh * DK * DV : nullptr)
+                      : STATE_ONLY ? nullptr
+                                   : args.sbuf + ((size_t)bh * args.nseg + seg - 1) * DK * DV;
+  float gamma_acc = 1.f;  // decay product of the segment for row s_row (state-only pass)
+  if (s_owner && init) {
+    const float4* src = reinterpret_cast<const float4*>(init + (size_t)s_row * DV + dv0 + sc0);
 #pragma unroll
     for (int c = 0; c < SW / 4; ++c) {
       const float4 x = src[c];
@@ -143,10 +175,58 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t t_A = tmem, t_O = tmem + 64, t_dS = tmem + 128;
   const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
 
-  for (int i = 0; i < NC; ++i) {
-    const int s = i & 1;
+  for (int li = 0; li < nloc; ++li) {
+    const int s = li & 1, i = c_begin + li;
     uint8_t* st = sm + s * L::STAGE;
-    mbar_wait(&bar_load[s], (i >> 1) & 1, latch);
+    mbar_wait(&bar_load[s], (li >> 1) & 1, latch);
+
+    if constexpr (STATE_ONLY) {  // gates, Kh, dS = Kh^T V, S = e^{gamma} S + dS
+      Gate gr;
+      gr.run(st + 2 * L::RAW, DK, tot_sm);
+      if (gr.h == 0) {
+        decay_sm[gr.d] = gr.dec0;
+        decay_sm[gr.d + 1] = gr.dec1;
+      }
+      {
+        const uint32_t blk = (gr.d >> 6) * (C * 128), col = gr.d & 63;
+        gr.backward([&](int j, float e0, float e1) {
+          const uint32_t wk = *reinterpret_cast<const uint32_t*>(st + L::RAW + (j * DK + gr.d) * 2);
+          *reinterpret_cast<uint32_t*>(sm + L::KH + blk + sw128(j, col)) = pack2(bf_lo(wk) * e0, bf_hi(wk) * e1);
+        });
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (tid == 0) {
+        const uint32_t base = smem_u32(sm);
+        const uint32_t vbase = base + s * L::STAGE + 3 * L::RAW;
+        constexpr uint32_t id_S = idesc_bf16_f32(DK, DVT, true, true);
+#pragma unroll
+        for (int k = 0; k < C / 16; ++k)
+          umma_bf16(t_dS, desc_sw128(base + L::KH + k * 2048, C * 128, 1024), desc_sw128(vbase + k * 2048, 16, 1024),
+                    id_S, k > 0);
+        umma_commit(&bar_mma1);
+      }
+      __syncwarp();
+      mbar_wait(&bar_mma1, li & 1, latch);
+      tc_fence_after();
+      {
+        float ds[SW];
+        tmem_ld32(t_dS + lane_off + sc0, ds);
+        tmem_ld_wait();
+        if (s_owner) {
+          const float dec = decay_sm[s_row];
+          gamma_acc *= dec;
+#pragma unroll
+          for (int c = 0; c < SW; ++c) S[c] = dec * S[c] + ds[c];
+        }
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0 && li + 2 < nloc) issue_load(li + 2);
+      continue;
+    }
 
     // ---------------- gate math: one ex2 per (token, dim); decays from running products -------
     Gate gr;
@@ -214,7 +294,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       umma_commit(&bar_mma1);
     }
     __syncwarp();
-    mbar_wait(&bar_mma1, i & 1, latch);
+    mbar_wait(&bar_mma1, li & 1, latch);
     tc_fence_after();
 
     // ---------------- safe mode: exact intra-chunk matrix ----------------
@@ -288,7 +368,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       umma_commit(&bar_mma2);
     }
     __syncwarp();
-    mbar_wait(&bar_mma2, i & 1, latch);
+    mbar_wait(&bar_mma2, li & 1, latch);
     tc_fence_after();
 
     // ---------------- O epilogue: bf16 rows straight to global ----------------
@@ -302,14 +382,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && i + 2 < NC) issue_load(i + 2);
+    if (tid == 0 && li + 2 < nloc) issue_load(li + 2);
   }
 
-  if (s_owner && hT) {
-    float4* dst = reinterpret_cast<float4*>(hT + ((size_t)bh * DK + s_row) * DV + dv0 + sc0);
+  float* out = STATE_ONLY ? args.sbuf + ((size_t)bh * args.nseg + seg) * DK * DV
+                          : (seg == args.nseg - 1 && args.hT ? args.hT + (size_t)bh * DK * DV : nullptr);
+  if (s_owner && out) {
+    float4* dst = reinterpret_cast<float4*>(out + (size_t)s_row * DV + dv0 + sc0);
 #pragma unroll
     for (int c = 0; c < SW / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
   }
+  if (STATE_ONLY && s_owner && half == 0 && blockIdx.x == 0)
+    args.gam[((size_t)bh * args.nseg + seg) * DK + s_row] = gamma_acc;
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 256);
@@ -326,32 +410,107 @@ bool fwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype) {
   return encode_fn() != nullptr;
 }
 
-size_t fwd_workspace(int, int, int, int) { return 0; }
+// Entry states of segments 1 .. nseg-1, in place: entry s-1 of sbuf holds S_local(s-1) on input and
+// the state entering segment s on output, S_in(s) = Gamma_{s-1} * S_in(s-1) + S_local(s-1) per row.
+__global__ void segment_scan_kernel(float* __restrict__ sbuf, const float* __restrict__ gam, int BH, int DK, int DV,
+                                    int nseg) {
+  const size_t per = (size_t)DK * DV, n = (size_t)BH * per;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+    const size_t bh = e / per, rem = e % per;
+    const int d = (int)(rem / DV);
+    float* p = sbuf + bh * nseg * per + rem;
+    float acc = p[0];
+    for (int sg = 1; sg < nseg - 1; ++sg) {
+      acc = gam[(bh * nseg + sg) * DK + d] * acc + p[sg * per];
+      p[sg * per] = acc;
+    }
+  }
+}
 
-template <int DK>
-static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o,
-                              float* hT, int BH, int T, int dv, cudaStream_t st) {
-  CUtensorMap mq, mk, mg, mv;
-  if (!make_map(&mq, q, BH, T, DK, DK, false) || !make_map(&mk, k, BH, T, DK, DK, false) ||
-      !make_map(&mg, g, BH, T, DK, DK, false) || !make_map(&mv, v, BH, T, dv, DVT, true))
-    return cudaErrorInvalidValue;
-  auto kern = fwd_fused_kernel<DK>;
+static int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+// Segments of the sequence split: as many as fill the SMs once with (head, value tile, segment)
+// CTAs; 1 (no split) when the heads alone fill at least half of them.
+static void plan_segments(int BH, int T, int dv, int* nseg, int* seg_chunks) {
+  const int NC = (T + C - 1) / C, base = BH * (dv / DVT), sms = sm_count();
+  int n = 1;
+  if (2 * base <= sms) n = sms / base;
+  if (n > NC) n = NC;
+  if (n < 1) n = 1;
+  const int per = (NC + n - 1) / n;
+  *seg_chunks = per;
+  *nseg = (NC + per - 1) / per;
+}
+
+size_t fwd_workspace(int BH, int T, int dk, int dv) {
+  int nseg, per;
+  plan_segments(BH, T, dv, &nseg, &per);
+  if (nseg == 1) return 0;
+  return align256((size_t)BH * nseg * dk * dv * sizeof(float)) + align256((size_t)BH * nseg * dk * sizeof(float));
+}
+
+template <int DK, bool STATE_ONLY>
+static cudaError_t launch_fwd_pass(const CUtensorMap* m, const FwdArgs& args, int BH, int dv, int nz, cudaStream_t st) {
+  auto kern = fwd_fused_kernel<DK, STATE_ONLY>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdLayout<DK>::ALLOC);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid(dv / DVT, BH);
-  kern<<<grid, NTHREADS, FwdLayout<DK>::ALLOC, st>>>(mq, mk, mg, mv, h0, static_cast<__nv_bfloat16*>(o), hT, T, dv,
-                                                     device_error_latch());
+  dim3 grid(dv / DVT, BH, nz);
+  kern<<<grid, NTHREADS, FwdLayout<DK>::ALLOC, st>>>(m[0], m[1], m[2], m[3], args);
   return cudaGetLastError();
 }
 
+template <int DK>
+static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o,
+                              float* hT, int BH, int T, int dv, void* ws, cudaStream_t st) {
+  CUtensorMap m[4];
+  if (!make_map(&m[0], q, BH, T, DK, DK, false) || !make_map(&m[1], k, BH, T, DK, DK, false) ||
+      !make_map(&m[2], g, BH, T, DK, DK, false) || !make_map(&m[3], v, BH, T, dv, DVT, true))
+    return cudaErrorInvalidValue;
+  FwdArgs a;
+  a.h0 = h0;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.hT = hT;
+  a.T = T;
+  a.DV = dv;
+  a.latch = device_error_latch();
+  plan_segments(BH, T, dv, &a.nseg, &a.seg_chunks);
+  a.sbuf = nullptr;
+  a.gam = nullptr;
+  if (a.nseg > 1) {
+    if (!ws) return cudaErrorInvalidValue;
+    a.sbuf = static_cast<float*>(ws);
+    a.gam = a.sbuf + align256((size_t)BH * a.nseg * DK * dv * sizeof(float)) / sizeof(float);
+    cudaError_t e = launch_fwd_pass<DK, true>(m, a, BH, dv, a.nseg - 1, st);
+    if (e != cudaSuccess) return e;
+    if (a.nseg > 2) {
+      const size_t n = (size_t)BH * DK * dv;
+      const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+      segment_scan_kernel<<<blocks, 256, 0, st>>>(a.sbuf, a.gam, BH, DK, dv, a.nseg);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+  }
+  return launch_fwd_pass<DK, false>(m, a, BH, dv, a.nseg, st);
+}
+
 cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
-                int BH, int T, int dk, int dv, void*, cudaStream_t st) {
-  if (dk == 64) return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, st);
-  if (dk == 128) return launch_fwd<128>(q, k, v, g, h0, o, hT, BH, T, dv, st);
+                int BH, int T, int dk, int dv, void* ws, cudaStream_t st) {
+  if (dk == 64) return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, ws, st);
+  if (dk == 128) return launch_fwd<128>(q, k, v, g, h0, o, hT, BH, T, dv, ws, st);
   return cudaErrorNotSupported;
 }
 

@@ -157,10 +157,23 @@ def test_deterministic_repeat():
 
 
 def test_fused_forward_is_selected_for_bf16_shapes():
-    """bf16, chunk 64, d_k in {64, 128}, d_v a multiple of 64: the fused kernel (no workspace) runs."""
+    """bf16, chunk 64, d_k in {64, 128}, d_v a multiple of 64: the fused kernel runs.  With enough
+    heads to fill the GPU it needs no workspace; with few heads it splits the sequence and keeps one
+    fp32 state and one decay vector per (head, segment)."""
     assert gla.workspace_bytes("gla_chunk_fwd", 8, 4, 2048, 128, 256, 64, 1) == 0
-    assert gla.workspace_bytes("gla_chunk_fwd", 1, 1, 100, 64, 64, 64, 1) == 0
+    nseg = 2  # 2 chunks, one head: one segment per chunk
+    expect = -(-nseg * 64 * 64 * 4 // 256) * 256 + -(-nseg * 64 * 4 // 256) * 256
+    assert gla.workspace_bytes("gla_chunk_fwd", 1, 1, 100, 64, 64, 64, 1) == expect
     assert gla.workspace_bytes("gla_chunk_fwd", 1, 1, 100, 64, 64, 64, 0) > 0  # fp32: generic passes
+
+
+@pytest.mark.parametrize("dk,dv,T", [(128, 64, 64 * 23 + 5), (64, 128, 64 * 9), (128, 256, 64 * 40 + 63),
+                                     (128, 128, 64 * 2)])
+def test_fused_forward_sequence_split(dk, dv, T):
+    """Few heads and many chunks: the forward runs as segments (state-only pass, scan of the segment
+    entry states, full pass per segment).  o and hT against the oracle, with an initial state."""
+    inp = make_gla_inputs(1, 2, T, dk, dv, torch.bfloat16, seed=40 + dk + T, with_h0=True, with_do=False)
+    _run_fwd_bwd(inp, 64, check_bwd=False)
 
 
 @pytest.mark.parametrize("dv", [128, 256])
