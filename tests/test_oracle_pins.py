@@ -13,6 +13,8 @@
 * GSA reduces to known forms for alpha == 1 and for a single slot (m = 1, softmax == 1).
 * a few plausible mistakes planted in copies of the recurrence fail these pins.
 """
+import math
+
 import numpy as np
 import pytest
 
@@ -347,3 +349,78 @@ def test_planted_mistakes_fail_the_bruteforce_pin(rng, kind):
     bo, _ = _brute_gla(q, k, v, g, h0)
     mo, _ = _mutant(q, k, v, g, h0, kind)
     assert np.max(np.abs(mo - bo)) > 1e-3
+
+
+# ---------------------------------------------------------------------------------------
+# raw-logit gate: g = logsigmoid(x) / tau and its derivative
+# ---------------------------------------------------------------------------------------
+def test_gate_logsigmoid_values():
+    """logsigmoid(0) = -ln 2; logsigmoid(x) - logsigmoid(-x) = x; -> 0 for large x, -> x for very negative x."""
+    tau = 16.0
+    assert abs(O.gate_logsigmoid(0.0, tau) * tau + math.log(2.0)) < 1e-15
+    x = np.linspace(-30, 30, 121)
+    np.testing.assert_allclose((O.gate_logsigmoid(x, 1.0) - O.gate_logsigmoid(-x, 1.0)), x, rtol=0, atol=1e-12)
+    assert abs(O.gate_logsigmoid(60.0, 1.0)) < 1e-25
+    assert abs(O.gate_logsigmoid(-700.0, 8.0) - (-700.0 / 8.0)) < 1e-12
+    assert np.all(np.diff(O.gate_logsigmoid(x, tau)) > 0) and np.all(O.gate_logsigmoid(x, tau) < 0)
+
+
+def test_gate_logsigmoid_bwd_finite_differences(rng):
+    x = rng.normal(size=50) * 4
+    dg = rng.normal(size=50)
+    tau, h = 8.0, 1e-6
+    fd = dg * (O.gate_logsigmoid(x + h, tau) - O.gate_logsigmoid(x - h, tau)) / (2 * h)
+    np.testing.assert_allclose(O.gate_logsigmoid_bwd(x, dg, tau), fd, rtol=1e-7, atol=1e-10)
+    # sigmoid(-x) + sigmoid(x) = 1
+    np.testing.assert_allclose(O.gate_logsigmoid_bwd(x, dg, tau) + O.gate_logsigmoid_bwd(-x, dg, tau), dg / tau,
+                               rtol=1e-13, atol=1e-15)
+
+
+def test_planted_gate_mistake_fails():
+    """A gate built as log(sigmoid(x)) * tau (scale applied the wrong way) fails the ln 2 pin."""
+    wrong = -math.log1p(math.exp(0.0)) * 16.0
+    assert abs(wrong * 16.0 + math.log(2.0)) > 1e-3
+
+
+# ---------------------------------------------------------------------------------------
+# MS-GLA pooling and causal hold
+# ---------------------------------------------------------------------------------------
+def test_msgla_pool_hand_example():
+    """T = 5, s = 2: blocks {1,2}, {3,4}, {5} -> 1.5, 3.5, 5 (the short block averages its one token)."""
+    x = np.arange(1.0, 6.0).reshape(1, 1, 5, 1)
+    np.testing.assert_array_equal(O.msgla_pool(x, 2).ravel(), [1.5, 3.5, 5.0])
+    np.testing.assert_array_equal(O.msgla_pool(x, 5).ravel(), [3.0])
+    np.testing.assert_array_equal(O.msgla_pool(x, 1), x)
+
+
+def test_msgla_hold_hand_example():
+    """Pooled outputs [a, b, c] at s = 2, T = 5: token t sees block (t+1)//2 - 1 -> [0, a, a, b, b]."""
+    y = np.array([10.0, 20.0, 30.0]).reshape(1, 1, 3, 1)
+    np.testing.assert_array_equal(O.msgla_hold(y, 5, 2).ravel(), [0, 10, 10, 20, 20])
+    np.testing.assert_array_equal(O.msgla_hold(y, 3, 1).ravel(), [10, 20, 30])
+
+
+def test_msgla_pool_then_hold_is_causal(rng):
+    """hold(pool(x)) at token t depends on x only through tokens <= t, and a block shows up
+    exactly at its last token."""
+    T, s = 13, 4
+    x = rng.normal(size=(1, 2, T, 3))
+    base = O.msgla_hold(O.msgla_pool(x, s), T, s)
+    for t0 in range(T):
+        x2 = x.copy()
+        x2[..., t0, :] += 1.0
+        diff = np.abs(O.msgla_hold(O.msgla_pool(x2, s), T, s) - base).max(axis=(0, 1, 3))
+        changed = np.nonzero(diff > 1e-12)[0]
+        if changed.size:
+            first = (t0 // s + 1) * s - 1  # last token of t0's block
+            assert changed.min() == first and changed.min() >= t0
+
+
+@pytest.mark.parametrize("T,s", [(13, 4), (8, 8), (7, 1), (5, 9)])
+def test_msgla_backward_is_the_adjoint(rng, T, s):
+    """<pool(x), dy> = <x, pool_bwd(dy)> and <hold(y), dz> = <y, hold_bwd(dz)>."""
+    P = -(-T // s)
+    x, dy = rng.normal(size=(2, 1, T, 4)), rng.normal(size=(2, 1, P, 4))
+    assert abs((O.msgla_pool(x, s) * dy).sum() - (x * O.msgla_pool_bwd(dy, T, s)).sum()) < 1e-12
+    y, dz = rng.normal(size=(2, 1, P, 4)), rng.normal(size=(2, 1, T, 4))
+    assert abs((O.msgla_hold(y, T, s) * dz).sum() - (y * O.msgla_hold_bwd(dz, s)).sum()) < 1e-12
