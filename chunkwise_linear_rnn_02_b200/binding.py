@@ -40,6 +40,12 @@ _SIGNATURES = {
     "gsa_recurrent_step": (_i, [_vp] * 8 + [_i] * 6 + [_vp]),
     "gla_device_error": (_i, [_vp, _i, ctypes.POINTER(_i)]),
     "gla_chunk_bwd_noalloc": (_i, [_vp] * 12 + [_i] * 7 + [_vp]),
+    "gla_gate_logsigmoid": (_i, [_vp, _vp, ctypes.c_size_t, ctypes.c_float, _i, _vp]),
+    "gla_gate_logsigmoid_bwd": (_i, [_vp, _vp, _vp, ctypes.c_size_t, ctypes.c_float, _i, _vp]),
+    "gla_msgla_pool": (_i, [_vp, _vp] + [_i] * 6 + [_vp]),
+    "gla_msgla_pool_bwd": (_i, [_vp, _vp] + [_i] * 6 + [_vp]),
+    "gla_msgla_hold": (_i, [_vp, _vp] + [_i] * 6 + [_vp]),
+    "gla_msgla_hold_bwd": (_i, [_vp, _vp] + [_i] * 6 + [_vp]),
 }
 
 
@@ -244,3 +250,51 @@ def device_error(reset: bool = True, device=None) -> int:
     dev = device or torch.device("cuda", torch.cuda.current_device())
     _check(load_library().gla_device_error(_stream(dev), int(reset), ctypes.byref(code)), "gla_device_error")
     return code.value
+
+
+# ------------------------------------------------------------------------------------------
+def gate_logsigmoid(x, tau: float):
+    """Raw-logit gate: g = logsigmoid(x) / tau (same shape and dtype as x)."""
+    _need_cuda(x)
+    g = torch.empty_like(x)
+    _check(load_library().gla_gate_logsigmoid(_ptr(x), _ptr(g), x.numel(), float(tau), _dtype_code(x),
+                                             _stream(x.device)), "gla_gate_logsigmoid")
+    return g
+
+
+def gate_logsigmoid_bwd(x, dg, tau: float):
+    """dx = dg * sigmoid(-x) / tau."""
+    _need_cuda(x, dg)
+    dx = torch.empty_like(x)
+    _check(load_library().gla_gate_logsigmoid_bwd(_ptr(x), _ptr(dg), _ptr(dx), x.numel(), float(tau),
+                                                 _dtype_code(x), _stream(x.device)), "gla_gate_logsigmoid_bwd")
+    return dx
+
+
+def _msgla(name, inp, rows_out, T, s):
+    _need_cuda(inp)
+    B, H, _, D = inp.shape
+    out = torch.empty(B, H, rows_out, D, dtype=inp.dtype, device=inp.device)
+    _check(getattr(load_library(), name)(_ptr(inp), _ptr(out), B, H, T, D, int(s), _dtype_code(inp),
+                                         _stream(inp.device)), name)
+    return out
+
+
+def msgla_pool(x, s: int):
+    """Average pooling of non-overlapping blocks of s tokens: [B,H,T,D] -> [B,H,ceil(T/s),D]."""
+    T = x.shape[2]
+    return _msgla("gla_msgla_pool", x, -(-T // s), T, s)
+
+
+def msgla_pool_bwd(dy, T: int, s: int):
+    return _msgla("gla_msgla_pool_bwd", dy, T, T, s)
+
+
+def msgla_hold(y, T: int, s: int):
+    """Causal hold back to T tokens: token t gets pooled row (t+1)//s - 1 (zeros before that)."""
+    return _msgla("gla_msgla_hold", y, T, T, s)
+
+
+def msgla_hold_bwd(dout, s: int):
+    T = dout.shape[2]
+    return _msgla("gla_msgla_hold_bwd", dout, -(-T // s), T, s)

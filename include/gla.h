@@ -169,13 +169,49 @@ int gsa_recurrent_step(const void* q, const void* k, const void* v, const void* 
  * (different streams or host threads) race on it.  Nothing in it needs to start at zero.
  * Arguments, layouts and outputs are those of gla_chunk_bwd.  Supported: bf16, chunk 64,
  * d_k = 128, d_v in {128, 256}, T >= 1 (else GLA_ERR_UNSUPPORTED / GLA_ERR_INVALID_ARG), and
- * B*H*(T + ceil(T/64))*d_k*4 bytes of scratch within the 64 MiB (else GLA_ERR_WORKSPACE).
+ * 65*B*H*ceil(T/64)*d_k*4 bytes of scratch (two parts, each rounded up to 256 bytes) within
+ * the 64 MiB (else GLA_ERR_WORKSPACE).
  * It allocates nothing.
  * ------------------------------------------------------------------------------------- */
 int gla_chunk_bwd_noalloc(const void* q, const void* k, const void* v, const void* g, const float* h0,
                           const void* dO, const float* dhT, void* dq, void* dk, void* dv, void* dg,
                           float* dh0, int B, int H, int T, int dk_dim, int dv_dim, int chunk, int dtype,
                           void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * gla_gate_logsigmoid - raw-logit gate entry: g = logsigmoid(x) / tau, element by element.
+ * The operators take the log-gate g (alpha = exp g <= 1); models build it from a logit x as
+ * log(sigmoid(x)) / tau ("MS-GLA ...", section 2.1: data-dependent forget gate; "Gated Slot
+ * Attention ...", "Approach": sigmoid forget gates, alpha = sigmoid(x)^(1/tau)).
+ *   x, g   n values of `dtype` (any layout; g may alias x).  tau > 0 and finite.
+ * n == 0 enqueues nothing.  Errors: GLA_ERR_INVALID_ARG (NULL or misaligned pointer with
+ * n > 0, tau not positive), GLA_ERR_UNSUPPORTED (dtype).  No workspace.
+ * ------------------------------------------------------------------------------------- */
+int gla_gate_logsigmoid(const void* x, void* g, size_t n, float tau, int dtype, void* stream);
+
+/* gla_gate_logsigmoid_bwd - its backward: dx = dg * sigmoid(-x) / tau (dx may alias dg). */
+int gla_gate_logsigmoid_bwd(const void* x, const void* dg, void* dx, size_t n, float tau, int dtype,
+                            void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * MS-GLA temporal pooling and causal hold ("MS-GLA: Multi-Scale Gated Linear Attention ...",
+ * sections 3.1 and 3.3), the reshaping around a GLA branch that runs at scale s.
+ *   gla_msgla_pool       x [B,H,T,D] -> y [B,H,P,D], P = ceil(T/s): y_p is the mean of tokens
+ *                        p*s .. min(T,(p+1)*s)-1 (a short last block averages only its tokens).
+ *   gla_msgla_pool_bwd   dy [B,H,P,D] -> dx [B,H,T,D]: dx_t = dy_{t/s} / (tokens in block t/s).
+ *   gla_msgla_hold       y [B,H,P,D] -> out [B,H,T,D]: out_t = y_{(t+1)/s - 1}, zeros while
+ *                        (t+1)/s = 0 (a block is visible from its last token on).
+ *   gla_msgla_hold_bwd   dout [B,H,T,D] -> dy [B,H,P,D]: the transpose (sum over the tokens that
+ *                        read block p).
+ * Arguments are (in, out, B, H, T, D, s, dtype, stream) for all four; in and out must not
+ * overlap.  D in 8..512, a multiple of 8; s >= 1; T == 0 enqueues nothing.  Errors as for the
+ * operators.  No workspace.
+ * ------------------------------------------------------------------------------------- */
+int gla_msgla_pool(const void* x, void* y, int B, int H, int T, int D, int s, int dtype, void* stream);
+int gla_msgla_pool_bwd(const void* dy, void* dx, int B, int H, int T, int D, int s, int dtype, void* stream);
+int gla_msgla_hold(const void* y, void* out, int B, int H, int T, int D, int s, int dtype, void* stream);
+int gla_msgla_hold_bwd(const void* dout, void* dy, int B, int H, int T, int D, int s, int dtype,
+                       void* stream);
 
 /* ---------------------------------------------------------------------------------------
  * gla_device_error - read (and optionally clear) the device-side error latch.

@@ -105,3 +105,25 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 1, 8, 8)
     with pytest.raises(binding.GLAError):
         binding.chunk_fwd(x, x, x, x)
+
+
+def test_gate_and_msgla_argument_checks(lib):
+    """Every call here fails a check (or has nothing to do) before any launch."""
+    vp = ctypes.c_void_p
+    # gate: tau must be positive, dtype known, pointers non-NULL and aligned when n > 0
+    assert lib.gla_gate_logsigmoid(vp(P), vp(P), 16, 0.0, 1, None) == INVALID
+    assert lib.gla_gate_logsigmoid(vp(P), vp(P), 16, float("nan"), 1, None) == INVALID
+    assert lib.gla_gate_logsigmoid(vp(P), vp(P), 16, 16.0, 5, None) == UNSUPPORTED
+    assert lib.gla_gate_logsigmoid(None, vp(P), 16, 16.0, 1, None) == INVALID
+    assert lib.gla_gate_logsigmoid(vp(P), vp(BAD), 16, 16.0, 1, None) == INVALID
+    assert lib.gla_gate_logsigmoid(None, None, 0, 16.0, 1, None) == OK  # nothing to do
+    assert lib.gla_gate_logsigmoid_bwd(vp(P), None, vp(P), 16, 8.0, 0, None) == INVALID
+    for name in ("gla_msgla_pool", "gla_msgla_pool_bwd", "gla_msgla_hold", "gla_msgla_hold_bwd"):
+        f = getattr(lib, name)
+        assert f(vp(P), vp(P), 1, 1, 10, 12, 2, 1, None) == UNSUPPORTED   # D not a multiple of 8
+        assert f(vp(P), vp(P), 1, 1, 10, 16, 0, 1, None) == INVALID       # s = 0
+        assert f(vp(P), vp(P), 0, 1, 10, 16, 2, 1, None) == INVALID       # B = 0
+        assert f(None, vp(P), 1, 1, 10, 16, 2, 1, None) == INVALID        # NULL input
+        assert f(vp(P), vp(BAD), 1, 1, 10, 16, 2, 1, None) == INVALID     # misaligned output
+        assert f(vp(P), vp(P), 1, 1, 10, 16, 2, 3, None) == UNSUPPORTED   # dtype
+        assert f(None, None, 1, 1, 0, 16, 2, 1, None) == OK               # T = 0: nothing to do

@@ -55,3 +55,28 @@ def test_gsa_decode_continues_forward(dtype):
     assert_close("o", torch.stack(outs, 2), ro[:, :, T:], tol)
     assert_close("S1", S1, rhT1, tol)
     assert_close("S2", S2, rhT2, tol)
+
+
+@pytest.mark.parametrize("variant", ["abc_no_gate", "data_independent_gate"])
+def test_gsa_gate_variants(variant):
+    """The ABC form (no forget gate, g = 0) and a data-independent gate (one log-decay per slot,
+    the same at every step) run through the same kernels."""
+    B, H, T, dk, dv, m = 1, 2, 150, 64, 64, 32
+    dtype = torch.bfloat16
+    inp = make_gsa_inputs(B, H, T, dk, dv, m, dtype, seed=17)
+    if variant == "abc_no_gate":
+        inp["g"] = torch.zeros_like(inp["g"])
+    else:
+        per_slot = inp["g"][:, :, :1, :].float()  # one value per (batch, head, slot)
+        inp["g"] = per_slot.expand(B, H, T, m).contiguous().to(dtype)
+    d = cuda(inp)
+    o, p, hT1, hT2 = gla.gsa_fwd(d["q"], d["k"], d["v"], d["phi"], d["g"], save_p=True)
+    a = [f64(inp[n]) for n in ["q", "k", "v", "phi", "g"]]
+    ro, rp, rhT1, rhT2 = O.gsa_fwd(*a)
+    tol = tol_for(dtype)
+    assert_close("o", o, ro, tol)
+    assert_close("hT2", hT2, rhT2, tol)
+    grads = gla.gsa_bwd(d["q"], d["k"], d["v"], d["phi"], d["g"], d["do"])
+    ref = O.gsa_bwd(*a, None, None, f64(inp["do"]))
+    for name, x, r in zip(["dq", "dk", "dv", "dphi", "dg"], grads, ref):
+        assert_close(name, x, r, tol)
