@@ -1,7 +1,7 @@
 // Fused sm_100a chunkwise GLA kernels (bf16 in, fp32 accumulate, chunk 64).
 //
-// Forward, one CTA per (head, 64 value columns); the CTA walks the chunks of its head in order
-// and keeps the recurrent state on chip ("MS-GLA ...", section 2.1: sequential inter-chunk
+// Forward, one CTA per (head, 64 value columns, sequence segment); the CTA walks the chunks of its
+// segment in order and keeps the recurrent state on chip ("MS-GLA ...", section 2.1: sequential inter-chunk
 // updates, parallel intra-chunk work; "Gated Linear Attention for Efficient Long Sequences":
 // chunking with on-chip reuse so that only inputs and outputs cross HBM).
 //
@@ -16,10 +16,10 @@
 //     O   = Qs (e^{gamma} S_i)        [64 x 64]   = (q e^{B}) S_i  (state copy pre-scaled by e^{gamma})
 //     dS  = Kh^T V                    [dk x 64]
 //     O  += A V
-//   state (fp32 registers, one thread per row d):   S_{i+1} = e^{gamma} S_i + dS
+//   state (fp32 registers; a thread holds half a row d):   S_{i+1} = e^{gamma} S_i + dS
 //
 // Qs carries e^{B - gamma} <= e^{|gamma|}; it stays finite (and e^{gamma} S_i stays normal) while
-// the chunk keeps at least e^-80 of its state in every key dimension.  A chunk below that bound
+// the chunk keeps at least e^-40 of its state in every key dimension.  A chunk below that bound
 // (near-reset gates) switches to a safe form for that chunk: Qs = q e^{B} with an unscaled state
 // copy, and the intra-chunk matrix recomputed exactly in fp32 from e^{B_j - B_r} (r <= j).
 //
@@ -47,33 +47,8 @@ constexpr int DVT = 64;      // value columns per CTA
 constexpr int NTHREADS = 256;  // warps w and w+4 share TMEM lanes and split accumulator columns
 
 // ------------------------------------------------------------------------------------------
-// Forward kernel
+// Arguments of the forward passes
 // ------------------------------------------------------------------------------------------
-template <int DK>
-struct FwdLayout {
-  static constexpr uint32_t RAW = C * DK * 2;               // one raw q / k / g tile
-  static constexpr uint32_t RAW_V = C * DVT * 2;            // raw v tile (swizzled)
-  static constexpr uint32_t STAGE = 3 * RAW + RAW_V;
-  static constexpr uint32_t OPS = 2 * STAGE;                // operand area
-  static constexpr uint32_t QS_HI = OPS;                    // Qs hi / lo [64 x DK]  K-major
-  static constexpr uint32_t QS_LO = QS_HI + C * DK * 2;
-  static constexpr uint32_t KH = QS_LO + C * DK * 2;        // Kh [64 x DK]  K-major B / MN-major A
-  static constexpr uint32_t SB_HI = KH + C * DK * 2;        // scaled state copy hi / lo [DK x 64] MN-major
-  static constexpr uint32_t SB_LO = SB_HI + DK * DVT * 2;
-  static constexpr uint32_t AB_HI = SB_LO + DK * DVT * 2;   // A hi / lo [64 x 64] K-major
-  static constexpr uint32_t AB_LO = AB_HI + C * C * 2;
-  static constexpr uint32_t DECAY = AB_LO + C * C * 2;      // float[DK]       e^{gamma_d}
-  static constexpr uint32_t TOT = DECAY + DK * 4;           // float[NSPLIT][DK] run products
-  static constexpr uint32_t TOTAL = TOT + GateRun<DK, NTHREADS>::NSPLIT * DK * 4;
-  static constexpr uint32_t ALLOC = TOTAL + 1024;           // slack for 1024-byte alignment
-  // Exact-path scratch, used after the first MMA group of a chunk has completed: fp32
-  // cumulative log-gates [64 x DK] over QS_HI..QS_LO, exact A [64 x 64] fp32 over KH..SB_HI.
-  static constexpr uint32_t XB = QS_HI, XA = KH;
-  static_assert(STAGE % 1024 == 0 && RAW % 1024 == 0, "stage alignment");
-  static_assert(ALLOC <= 227 * 1024, "shared memory");
-  static_assert(C * DK * 4 <= KH - QS_HI && C * C * 4 <= SB_LO - KH, "exact-path scratch");
-};
-
 struct FwdArgs {
   const float* h0;     // [BH][DK][DV] or null (zeros)
   float* sbuf;         // [BH][nseg][DK][DV]: segment end states (state-only pass), then entry states
@@ -84,30 +59,206 @@ struct FwdArgs {
   unsigned int* latch;
 };
 
-// One CTA per (64 value columns, head, segment).  STATE_ONLY: the state recurrence alone (no
-// queries, no outputs), writing the segment's end state and decay product.
-template <int DK, bool STATE_ONLY>
+// ------------------------------------------------------------------------------------------
+// State-only pass of the sequence split: one CTA per (64 value columns, head, segment) runs the
+// state recurrence alone (gates, Kh, dS = Kh^T V, S = e^{gamma} S + dS; no queries, no outputs)
+// and writes the segment's end state and decay product.  Kh is finite for every gate (E2 <= 1),
+// so this pass needs no exact path.
+// ------------------------------------------------------------------------------------------
+template <int DK>
+struct StateLayout {
+  static constexpr uint32_t RAW = C * DK * 2;          // one raw k / g tile
+  static constexpr uint32_t STAGE = 2 * RAW + C * DVT * 2;  // k, g, v
+  static constexpr uint32_t KH = 2 * STAGE;            // Kh [64 x DK], MN-major A operand of dS
+  static constexpr uint32_t DECAY = KH + C * DK * 2;
+  static constexpr uint32_t TOT = DECAY + DK * 4;
+  static constexpr uint32_t TOTAL = TOT + GateRun<DK, NTHREADS>::NSPLIT * DK * 4;
+  static constexpr uint32_t ALLOC = TOTAL + 1024;
+  static_assert(STAGE % 1024 == 0 && RAW % 1024 == 0, "stage alignment");
+};
+
+template <int DK>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    fwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
-                     const FwdArgs args) {
-  using L = FwdLayout<DK>;
-  const float* h0 = args.h0;
-  __nv_bfloat16* o = args.o;
-  const int T = args.T, DV = args.DV;
-  unsigned int* latch = args.latch;
+    fwd_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_g,
+                     const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
+  using L = StateLayout<DK>;
   using Gate = GateRun<DK, NTHREADS>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_load[2], bar_mma1, bar_mma2;
+  __shared__ uint64_t bar_load[2], bar_mma;
   __shared__ uint32_t tmem_base_sh;
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3, half = warp >> 2;
+  const int dv0 = blockIdx.x * DVT, bh = blockIdx.y, seg = blockIdx.z;
+  const int T = args.T, DV = args.DV, NC = (T + C - 1) / C;
+  const int c_begin = seg * args.seg_chunks;
+  const int nloc = min(NC, c_begin + args.seg_chunks) - c_begin;
+  float* decay_sm = reinterpret_cast<float*>(sm + L::DECAY);
+  float* tot_sm = reinterpret_cast<float*>(sm + L::TOT);
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, 64);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bar_load[0], 1);
+    mbar_init(&bar_load[1], 1);
+    mbar_init(&bar_mma, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue_load = [&](int li) {
+    const int s = li & 1, chunk = c_begin + li;
+    uint8_t* st = sm + s * L::STAGE;
+    mbar_arrive_expect_tx(&bar_load[s], L::STAGE);
+    tma_load_3d(st, &tm_k, &bar_load[s], 0, chunk * C, bh);
+    tma_load_3d(st + L::RAW, &tm_g, &bar_load[s], 0, chunk * C, bh);
+    tma_load_3d(st + 2 * L::RAW, &tm_v, &bar_load[s], dv0, chunk * C, bh);
+  };
+  if (tid == 0) {
+    issue_load(0);
+    if (nloc > 1) issue_load(1);
+  }
+  constexpr int SW = DVT / 2;
+  const bool s_owner = (DK == 128) ? true : (lane < 16);
+  const int s_row = (DK == 128) ? (q4 * 32 + lane) : (q4 * 16 + lane);
+  const int sc0 = half * SW;
+  float S[SW];
+#pragma unroll
+  for (int c = 0; c < SW; ++c) S[c] = 0.f;
+  if (seg == 0 && s_owner && args.h0) {
+    const float4* src = reinterpret_cast<const float4*>(args.h0 + ((size_t)bh * DK + s_row) * DV + dv0 + sc0);
+#pragma unroll
+    for (int c = 0; c < SW / 4; ++c) {
+      const float4 x = src[c];
+      S[4 * c] = x.x;
+      S[4 * c + 1] = x.y;
+      S[4 * c + 2] = x.z;
+      S[4 * c + 3] = x.w;
+    }
+  }
+  float gamma_acc = 1.f;  // decay product of the segment for row s_row
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t t_dS = tmem_base_sh;
+  const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+  for (int li = 0; li < nloc; ++li) {
+    const int s = li & 1;
+    uint8_t* st = sm + s * L::STAGE;
+    mbar_wait(&bar_load[s], (li >> 1) & 1, args.latch);
+    Gate gr;
+    gr.run(st + L::RAW, DK, tot_sm);
+    if (gr.h == 0) {
+      decay_sm[gr.d] = gr.dec0;
+      decay_sm[gr.d + 1] = gr.dec1;
+    }
+    {
+      const uint32_t blk = (gr.d >> 6) * (C * 128), col = gr.d & 63;
+      gr.backward([&](int j, float e0, float e1) {
+        const uint32_t wk = *reinterpret_cast<const uint32_t*>(st + (j * DK + gr.d) * 2);
+        *reinterpret_cast<uint32_t*>(sm + L::KH + blk + sw128(j, col)) = pack2(bf_lo(wk) * e0, bf_hi(wk) * e1);
+      });
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      const uint32_t base = smem_u32(sm);
+      const uint32_t vbase = base + s * L::STAGE + 2 * L::RAW;
+      constexpr uint32_t id_S = idesc_bf16_f32(DK, DVT, true, true);
+#pragma unroll
+      for (int k = 0; k < C / 16; ++k)
+        umma_bf16(t_dS, desc_sw128(base + L::KH + k * 2048, C * 128, 1024), desc_sw128(vbase + k * 2048, 16, 1024),
+                  id_S, k > 0);
+      umma_commit(&bar_mma);
+    }
+    __syncwarp();
+    mbar_wait(&bar_mma, li & 1, args.latch);
+    tc_fence_after();
+    float ds[SW];
+    tmem_ld32(t_dS + lane_off + sc0, ds);
+    tmem_ld_wait();
+    if (s_owner) {
+      const float dec = decay_sm[s_row];
+      gamma_acc *= dec;
+#pragma unroll
+      for (int c = 0; c < SW; ++c) S[c] = dec * S[c] + ds[c];
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && li + 2 < nloc) issue_load(li + 2);
+  }
+  float* out = args.sbuf + ((size_t)bh * args.nseg + seg) * DK * DV;
+  if (s_owner) {
+    float4* dst = reinterpret_cast<float4*>(out + (size_t)s_row * DV + dv0 + sc0);
+#pragma unroll
+    for (int c = 0; c < SW / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
+    if (half == 0 && blockIdx.x == 0) args.gam[((size_t)bh * args.nseg + seg) * DK + s_row] = gamma_acc;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(t_dS, 64);
+}
+
+// ------------------------------------------------------------------------------------------
+// Pipelined forward (the full pass).  Per chunk i the two MMA groups run while the CTA works on
+// its neighbours: during group 1 of chunk i (A, O_i = Qs S', dS) the threads store the outputs of
+// chunk i-1 and run the gate math of chunk i+1 into registers; during group 2 of chunk i
+// (O_i += A V) they store chunk i+1's operands (Qs, Kh, the scaled state copy) and group 1 of
+// chunk i+1 is issued right behind it.  O is double-buffered in TMEM; q/k/g come through a
+// two-stage ring and v through a three-deep ring, so a raw tile is free as soon as its own
+// chunk's math is done.  MMAs issued by one thread complete in order, so waiting for group 1 of
+// chunk i+1 also covers group 2 of chunk i.
+// ------------------------------------------------------------------------------------------
+template <int DK>
+struct FwdPipeLayout {
+  static constexpr uint32_t RAW = C * DK * 2;               // one raw q / k / g tile
+  static constexpr uint32_t QKG = 3 * RAW;                  // a q/k/g stage (two stages)
+  static constexpr uint32_t VTB = C * DVT * 2;              // a v tile (three buffers)
+  static constexpr uint32_t V0 = 2 * QKG;
+  static constexpr uint32_t QS_HI = V0 + 3 * VTB;           // Qs hi / lo [64 x DK]  K-major
+  static constexpr uint32_t QS_LO = QS_HI + C * DK * 2;
+  static constexpr uint32_t KH = QS_LO + C * DK * 2;        // Kh [64 x DK]  K-major B / MN-major A
+  static constexpr uint32_t SB_HI = KH + C * DK * 2;        // scaled state copy hi / lo [DK x 64]
+  static constexpr uint32_t SB_LO = SB_HI + DK * DVT * 2;
+  static constexpr uint32_t AB_HI = SB_LO + DK * DVT * 2;   // A hi / lo [64 x 64] K-major
+  static constexpr uint32_t AB_LO = AB_HI + C * C * 2;
+  static constexpr uint32_t DECAY = AB_LO + C * C * 2;      // float[2][DK]: e^{gamma_d} per chunk parity
+  static constexpr int NS = GateRun<DK, NTHREADS>::NSPLIT;
+  static constexpr uint32_t TOT = DECAY + 2 * DK * 4;       // float[NS][DK] run products
+  static constexpr uint32_t TOTAL = TOT + NS * DK * 4;
+  static constexpr uint32_t ALLOC = TOTAL + 1024;
+  // Exact-path scratch during the A epilogue of a chunk (its Qs / Kh are consumed by then, the
+  // next chunk's are still in registers): cumulative log-gates over QS_HI.., exact A over KH..
+  static constexpr uint32_t XB = QS_HI, XA = KH;
+  static_assert(QKG % 1024 == 0 && VTB % 1024 == 0 && QS_HI % 1024 == 0, "alignment");
+  static_assert(ALLOC <= 227 * 1024, "shared memory");
+  static_assert(C * DK * 4 <= KH - QS_HI && C * C * 4 <= SB_LO - KH, "exact-path scratch");
+};
+
+template <int DK>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    fwd_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
+                    const FwdArgs args) {
+  using L = FwdPipeLayout<DK>;
+  using Gate = GateRun<DK, NTHREADS>;
+  constexpr int TS = Gate::TS;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_qkg[2], bar_v[3], bar_mma1, bar_mma2;
+  __shared__ uint32_t tmem_base_sh;
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  const uint32_t base = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
   const int dv0 = blockIdx.x * DVT, bh = blockIdx.y, seg = blockIdx.z;
-  const int NC = (T + C - 1) / C;
+  const int T = args.T, DV = args.DV, NC = (T + C - 1) / C;
   const int c_begin = seg * args.seg_chunks;
-  const int nloc = min(NC, c_begin + args.seg_chunks) - c_begin;  // chunks of this segment
+  const int nloc = min(NC, c_begin + args.seg_chunks) - c_begin;
+  unsigned int* latch = args.latch;
   float* decay_sm = reinterpret_cast<float*>(sm + L::DECAY);
   float* tot_sm = reinterpret_cast<float*>(sm + L::TOT);
 
@@ -120,26 +271,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_g);
     prefetch_tmap(&tm_v);
-    mbar_init(&bar_load[0], 1);
-    mbar_init(&bar_load[1], 1);
+    for (int b = 0; b < 2; ++b) mbar_init(&bar_qkg[b], 1);
+    for (int b = 0; b < 3; ++b) mbar_init(&bar_v[b], 1);
     mbar_init(&bar_mma1, 1);
     mbar_init(&bar_mma2, 1);
     fence_mbar_init();
   }
   __syncthreads();
-  // Local chunk li of the segment into stage li & 1 (the state-only pass skips q).
-  auto issue_load = [&](int li) {
+  auto load_qkg = [&](int li) {
     const int s = li & 1, chunk = c_begin + li;
-    uint8_t* st = sm + s * L::STAGE;
-    mbar_arrive_expect_tx(&bar_load[s], STATE_ONLY ? L::STAGE - L::RAW : L::STAGE);
-    if (!STATE_ONLY) tma_load_3d(st, &tm_q, &bar_load[s], 0, chunk * C, bh);
-    tma_load_3d(st + L::RAW, &tm_k, &bar_load[s], 0, chunk * C, bh);
-    tma_load_3d(st + 2 * L::RAW, &tm_g, &bar_load[s], 0, chunk * C, bh);
-    tma_load_3d(st + 3 * L::RAW, &tm_v, &bar_load[s], dv0, chunk * C, bh);
+    uint8_t* st = sm + s * L::QKG;
+    mbar_arrive_expect_tx(&bar_qkg[s], L::QKG);
+    tma_load_3d(st, &tm_q, &bar_qkg[s], 0, chunk * C, bh);
+    tma_load_3d(st + L::RAW, &tm_k, &bar_qkg[s], 0, chunk * C, bh);
+    tma_load_3d(st + 2 * L::RAW, &tm_g, &bar_qkg[s], 0, chunk * C, bh);
+  };
+  auto load_v = [&](int li) {
+    const int b = li % 3;
+    mbar_arrive_expect_tx(&bar_v[b], L::VTB);
+    tma_load_3d(sm + L::V0 + b * L::VTB, &tm_v, &bar_v[b], dv0, (c_begin + li) * C, bh);
   };
   if (tid == 0) {
-    issue_load(0);
-    if (nloc > 1) issue_load(1);
+    load_qkg(0);
+    load_v(0);
+    if (nloc > 1) {
+      load_qkg(1);
+      load_v(1);
+    }
+    if (nloc > 2) load_v(2);
   }
 
   // State owned by this thread: row s_row (lane layout of the dS accumulator, M = DK), columns
@@ -151,11 +310,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   float S[SW];
 #pragma unroll
   for (int c = 0; c < SW; ++c) S[c] = 0.f;
-  // Entry state: h0 for the first segment; the scanned entry state for the others (full pass).
-  const float* init = seg == 0 ? (h0 ? h0 + (size_t)bh * DK * DV : nullptr)
-                      : STATE_ONLY ? nullptr
-                                   : args.sbuf + ((size_t)bh * args.nseg + seg - 1) * DK * DV;
-  float gamma_acc = 1.f;  // decay product of the segment for row s_row (state-only pass)
+  const float* init = seg == 0 ? (args.h0 ? args.h0 + (size_t)bh * DK * DV : nullptr)
+                               : args.sbuf + ((size_t)bh * args.nseg + seg - 1) * DK * DV;
   if (s_owner && init) {
     const float4* src = reinterpret_cast<const float4*>(init + (size_t)s_row * DV + dv0 + sc0);
 #pragma unroll
@@ -167,140 +323,132 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       S[4 * c + 3] = x.w;
     }
   }
-
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t t_A = tmem, t_O = tmem + 64, t_dS = tmem + 128;
+  const uint32_t t_A = tmem, t_O0 = tmem + 64, t_dS = tmem + 192;
   const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
 
-  for (int li = 0; li < nloc; ++li) {
-    const int s = li & 1, i = c_begin + li;
-    uint8_t* st = sm + s * L::STAGE;
-    mbar_wait(&bar_load[s], (li >> 1) & 1, latch);
-
-    if constexpr (STATE_ONLY) {  // gates, Kh, dS = Kh^T V, S = e^{gamma} S + dS
-      Gate gr;
-      gr.run(st + 2 * L::RAW, DK, tot_sm);
-      if (gr.h == 0) {
-        decay_sm[gr.d] = gr.dec0;
-        decay_sm[gr.d + 1] = gr.dec1;
-      }
-      {
-        const uint32_t blk = (gr.d >> 6) * (C * 128), col = gr.d & 63;
-        gr.backward([&](int j, float e0, float e1) {
-          const uint32_t wk = *reinterpret_cast<const uint32_t*>(st + L::RAW + (j * DK + gr.d) * 2);
-          *reinterpret_cast<uint32_t*>(sm + L::KH + blk + sw128(j, col)) = pack2(bf_lo(wk) * e0, bf_hi(wk) * e1);
-        });
-      }
-      fence_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      tc_fence_after();
-      if (tid == 0) {
-        const uint32_t base = smem_u32(sm);
-        const uint32_t vbase = base + s * L::STAGE + 3 * L::RAW;
-        constexpr uint32_t id_S = idesc_bf16_f32(DK, DVT, true, true);
-#pragma unroll
-        for (int k = 0; k < C / 16; ++k)
-          umma_bf16(t_dS, desc_sw128(base + L::KH + k * 2048, C * 128, 1024), desc_sw128(vbase + k * 2048, 16, 1024),
-                    id_S, k > 0);
-        umma_commit(&bar_mma1);
-      }
-      __syncwarp();
-      mbar_wait(&bar_mma1, li & 1, latch);
-      tc_fence_after();
-      {
-        float ds[SW];
-        tmem_ld32(t_dS + lane_off + sc0, ds);
-        tmem_ld_wait();
-        if (s_owner) {
-          const float dec = decay_sm[s_row];
-          gamma_acc *= dec;
-#pragma unroll
-          for (int c = 0; c < SW; ++c) S[c] = dec * S[c] + ds[c];
-        }
-      }
-      tc_fence_before();
-      __syncthreads();
-      if (tid == 0 && li + 2 < nloc) issue_load(li + 2);
-      continue;
-    }
-
-    // ---------------- gate math: one ex2 per (token, dim); decays from running products -------
+  // Gate math of local chunk li (stage li & 1) into registers: Qs hi / lo and Kh for the two
+  // dims gd, gd+1 and the tokens gh*TS .. gh*TS+TS-1 owned by this thread.  Returns the chunk's
+  // exact-path flag (CTA-uniform).
+  uint32_t qh[TS], ql[TS], kh[TS];
+  int gd = 0, gh = 0;
+  auto gate_regs = [&](int li) {
+    const uint8_t* st = sm + (li & 1) * L::QKG;
     Gate gr;
     const bool weak = gr.run(st + 2 * L::RAW, DK, tot_sm);
+    float* dec = decay_sm + (li & 1) * DK;
     if (gr.h == 0) {
-      decay_sm[gr.d] = gr.dec0;
-      decay_sm[gr.d + 1] = gr.dec1;
+      dec[gr.d] = gr.dec0;
+      dec[gr.d + 1] = gr.dec1;
     }
     const int safe = __syncthreads_or(weak);
-    {
-      const float inv0 = safe ? 1.f : 1.f / gr.dec0, inv1 = safe ? 1.f : 1.f / gr.dec1;
-      const uint32_t blk = (gr.d >> 6) * (C * 128), col = gr.d & 63;
-      gr.forward([&](int j, float e0, float e1) {
-        const uint32_t wq = *reinterpret_cast<const uint32_t*>(st + (j * DK + gr.d) * 2);
-        uint32_t hi, lo;
-        split2(bf_lo(wq) * e0 * inv0, bf_hi(wq) * e1 * inv1, hi, lo);
-        *reinterpret_cast<uint32_t*>(sm + L::QS_HI + blk + sw128(j, col)) = hi;
-        *reinterpret_cast<uint32_t*>(sm + L::QS_LO + blk + sw128(j, col)) = lo;
-      });
-      gr.backward([&](int j, float e0, float e1) {
-        const uint32_t wk = *reinterpret_cast<const uint32_t*>(st + L::RAW + (j * DK + gr.d) * 2);
-        *reinterpret_cast<uint32_t*>(sm + L::KH + blk + sw128(j, col)) = pack2(bf_lo(wk) * e0, bf_hi(wk) * e1);
-      });
+    gd = gr.d;
+    gh = gr.h;
+    float e0 = gr.pre0 * (safe ? 1.f : 1.f / gr.dec0), e1 = gr.pre1 * (safe ? 1.f : 1.f / gr.dec1);
+#pragma unroll
+    for (int u = 0; u < TS; ++u) {
+      e0 *= gr.a0[u];
+      e1 *= gr.a1[u];
+      const uint32_t wq = *reinterpret_cast<const uint32_t*>(st + ((gh * TS + u) * DK + gd) * 2);
+      split2(bf_lo(wq) * e0, bf_hi(wq) * e1, qh[u], ql[u]);
     }
-    // ---------------- state copy for the inter-chunk term: e^{gamma} S_i (or S_i in safe mode) ----
+    float f0 = gr.suf0, f1 = gr.suf1;
+#pragma unroll
+    for (int u = TS - 1; u >= 0; --u) {
+      const uint32_t wk = *reinterpret_cast<const uint32_t*>(st + L::RAW + ((gh * TS + u) * DK + gd) * 2);
+      kh[u] = pack2(bf_lo(wk) * f0, bf_hi(wk) * f1);
+      f0 *= gr.a0[u];
+      f1 *= gr.a1[u];
+    }
+    return safe;
+  };
+  // Operands of local chunk li into shared memory: Qs, Kh (from registers) and the state copy.
+  auto store_ops = [&](int li, int safe) {
+    const uint32_t blk = (gd >> 6) * (C * 128), col = gd & 63;
+#pragma unroll
+    for (int u = 0; u < TS; ++u) {
+      const uint32_t off = blk + sw128(gh * TS + u, col);
+      *reinterpret_cast<uint32_t*>(sm + L::QS_HI + off) = qh[u];
+      *reinterpret_cast<uint32_t*>(sm + L::QS_LO + off) = ql[u];
+      *reinterpret_cast<uint32_t*>(sm + L::KH + off) = kh[u];
+    }
     if (s_owner) {
-      const float sc = safe ? 1.f : decay_sm[s_row];
+      const float sc = safe ? 1.f : decay_sm[(li & 1) * DK + s_row];
       float sv[SW];
 #pragma unroll
       for (int c = 0; c < SW; ++c) sv[c] = S[c] * sc;
       store_half_split(sm + L::SB_HI, sm + L::SB_LO, s_row, sv, half);
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
+  };
+  // MMA group 1 of local chunk li: A = Qs Kh^T, O_li = Qs S', dS = Kh^T V.
+  auto issue_m1 = [&](int li) {
+    mbar_wait(&bar_v[li % 3], (li / 3) & 1, latch);
     tc_fence_after();
-
-    // ---------------- MMA group 1: A, O = Qs S', dS = Kh^T V ----------------
-    if (tid == 0) {
-      const uint32_t base = smem_u32(sm);
-      const uint32_t vbase = base + s * L::STAGE + 3 * L::RAW;
-      constexpr uint32_t id_A = idesc_bf16_f32(C, C, false, false);
-      constexpr uint32_t id_O = idesc_bf16_f32(C, DVT, false, true);
-      constexpr uint32_t id_S = idesc_bf16_f32(DK, DVT, true, true);
+    const uint32_t vbase = base + L::V0 + (li % 3) * L::VTB;
+    const uint32_t t_O = t_O0 + (li & 1) * 64;
+    constexpr uint32_t id_A = idesc_bf16_f32(C, C, false, false);
+    constexpr uint32_t id_O = idesc_bf16_f32(C, DVT, false, true);
+    constexpr uint32_t id_S = idesc_bf16_f32(DK, DVT, true, true);
 #pragma unroll
-      for (int k = 0; k < DK / 16; ++k) {
-        const uint32_t koff = (k >> 2) * (C * 128) + (k & 3) * 32;
-        const uint64_t kd = desc_sw128(base + L::KH + koff, 16, 1024);
-        umma_bf16(t_A, desc_sw128(base + L::QS_HI + koff, 16, 1024), kd, id_A, k > 0);
-        umma_bf16(t_A, desc_sw128(base + L::QS_LO + koff, 16, 1024), kd, id_A, 1);
-      }
-#pragma unroll
-      for (int k = 0; k < DK / 16; ++k) {
-        const uint32_t koff = (k >> 2) * (C * 128) + (k & 3) * 32;
-        const uint64_t qh = desc_sw128(base + L::QS_HI + koff, 16, 1024);
-        const uint64_t sh = desc_sw128(base + L::SB_HI + k * 2048, 16, 1024);
-        umma_bf16(t_O, qh, sh, id_O, k > 0);
-        umma_bf16(t_O, qh, desc_sw128(base + L::SB_LO + k * 2048, 16, 1024), id_O, 1);
-        umma_bf16(t_O, desc_sw128(base + L::QS_LO + koff, 16, 1024), sh, id_O, 1);
-      }
-#pragma unroll
-      for (int k = 0; k < C / 16; ++k)
-        umma_bf16(t_dS, desc_sw128(base + L::KH + k * 2048, C * 128, 1024), desc_sw128(vbase + k * 2048, 16, 1024),
-                  id_S, k > 0);
-      umma_commit(&bar_mma1);
+    for (int k = 0; k < DK / 16; ++k) {
+      const uint32_t koff = (k >> 2) * (C * 128) + (k & 3) * 32;
+      const uint64_t kd = desc_sw128(base + L::KH + koff, 16, 1024);
+      const uint64_t qh_d = desc_sw128(base + L::QS_HI + koff, 16, 1024);
+      const uint64_t ql_d = desc_sw128(base + L::QS_LO + koff, 16, 1024);
+      umma_bf16(t_A, qh_d, kd, id_A, k > 0);
+      umma_bf16(t_A, ql_d, kd, id_A, 1);
+      const uint64_t sh = desc_sw128(base + L::SB_HI + k * 2048, 16, 1024);
+      umma_bf16(t_O, qh_d, sh, id_O, k > 0);
+      umma_bf16(t_O, qh_d, desc_sw128(base + L::SB_LO + k * 2048, 16, 1024), id_O, 1);
+      umma_bf16(t_O, ql_d, sh, id_O, 1);
     }
-    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < C / 16; ++k)
+      umma_bf16(t_dS, desc_sw128(base + L::KH + k * 2048, C * 128, 1024), desc_sw128(vbase + k * 2048, 16, 1024),
+                id_S, k > 0);
+    umma_commit(&bar_mma1);
+  };
+  // O rows of local chunk li (after its group 2): bf16 straight to global.
+  auto store_o = [&](int li) {
+    mbar_wait(&bar_mma2, li & 1, latch);
+    tc_fence_after();
+    const int j = q4 * 16 + lane, cb = half * 32;
+    float ov[32];
+    tmem_ld32(t_O0 + (li & 1) * 64 + lane_off + cb, ov);
+    tmem_ld_wait();
+    const int t = (c_begin + li) * C + j;
+    if (lane < 16 && t < T) store_half_global_bf16(args.o + ((size_t)bh * T + t) * DV + dv0 + cb, ov);
+  };
+
+  mbar_wait(&bar_qkg[0], 0, latch);
+  int safe = gate_regs(0);
+  store_ops(0, safe);
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0) issue_m1(0);
+  for (int li = 0; li < nloc; ++li) {
+    const uint8_t* st = sm + (li & 1) * L::QKG;
+    // ---- while group 1 of chunk li runs: outputs of chunk li-1, gate math of chunk li+1 ----
+    if (li > 0) {
+      store_o(li - 1);
+      if (tid == 0 && li + 2 < nloc) load_v(li + 2);  // its buffer held chunk li-1's v
+    }
+    int safe_next = 0;
+    if (li + 1 < nloc) {
+      mbar_wait(&bar_qkg[(li + 1) & 1], ((li + 1) >> 1) & 1, latch);
+      safe_next = gate_regs(li + 1);
+    }
+    // ---- group 1 done: exact A if needed, A epilogue, state update, group 2 ----
     mbar_wait(&bar_mma1, li & 1, latch);
     tc_fence_after();
-
-    // ---------------- safe mode: exact intra-chunk matrix ----------------
-    float* Aex = reinterpret_cast<float*>(sm + L::XA);  // 64 x 64 fp32
+    float* Aex = reinterpret_cast<float*>(sm + L::XA);
     if (safe) {
-      float* Bf = reinterpret_cast<float*>(sm + L::XB);  // 64 x DK fp32 cumulative log-gates
+      float* Bf = reinterpret_cast<float*>(sm + L::XB);
       if (tid < DK) {
         float b = 0.f;
         for (int j = 0; j < C; ++j) {
@@ -320,8 +468,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       __syncthreads();
     }
-
-    // ---------------- A epilogue: mask, hi/lo bf16, store as the K-major A operand ----------------
     {
       const int j = q4 * 16 + lane, cb = half * 32;
       float a[32];
@@ -337,14 +483,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (cb + c > j) a[c] = 0.f;
         store_half_split(sm + L::AB_HI, sm + L::AB_LO, j, a, half);
       }
-    }
-    // ---------------- state update: S = e^gamma S + dS (fp32 registers) ----------------
-    {
       float ds[SW];
       tmem_ld32(t_dS + lane_off + sc0, ds);
       tmem_ld_wait();
       if (s_owner) {
-        const float dec = decay_sm[s_row];
+        const float dec = decay_sm[(li & 1) * DK + s_row];
 #pragma unroll
         for (int c = 0; c < SW; ++c) S[c] = dec * S[c] + ds[c];
       }
@@ -353,11 +496,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-
-    // ---------------- MMA group 2: O += A V ----------------
     if (tid == 0) {
-      const uint32_t base = smem_u32(sm);
-      const uint32_t vbase = base + s * L::STAGE + 3 * L::RAW;
+      const uint32_t vbase = base + L::V0 + (li % 3) * L::VTB;
+      const uint32_t t_O = t_O0 + (li & 1) * 64;
       constexpr uint32_t id_O = idesc_bf16_f32(C, DVT, false, true);
 #pragma unroll
       for (int k = 0; k < C / 16; ++k) {
@@ -366,34 +507,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         umma_bf16(t_O, desc_sw128(base + L::AB_LO + k * 32, 16, 1024), vd, id_O, 1);
       }
       umma_commit(&bar_mma2);
+      if (li + 2 < nloc) load_qkg(li + 2);  // chunk li's raw tiles are no longer read
     }
-    __syncwarp();
-    mbar_wait(&bar_mma2, li & 1, latch);
-    tc_fence_after();
-
-    // ---------------- O epilogue: bf16 rows straight to global ----------------
-    {
-      const int j = q4 * 16 + lane, cb = half * 32;
-      float ov[32];
-      tmem_ld32(t_O + lane_off + cb, ov);
-      tmem_ld_wait();
-      const int t = i * C + j;
-      if (lane < 16 && t < T) store_half_global_bf16(o + ((size_t)bh * T + t) * DV + dv0 + cb, ov);
+    // ---- while group 2 of chunk li runs: operands of chunk li+1, then its group 1 ----
+    if (li + 1 < nloc) {
+      store_ops(li + 1, safe_next);
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (tid == 0) issue_m1(li + 1);
     }
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && li + 2 < nloc) issue_load(li + 2);
+    safe = safe_next;
   }
+  store_o(nloc - 1);
 
-  float* out = STATE_ONLY ? args.sbuf + ((size_t)bh * args.nseg + seg) * DK * DV
-                          : (seg == args.nseg - 1 && args.hT ? args.hT + (size_t)bh * DK * DV : nullptr);
+  float* out = (seg == args.nseg - 1 && args.hT) ? args.hT + (size_t)bh * DK * DV : nullptr;
   if (s_owner && out) {
     float4* dst = reinterpret_cast<float4*>(out + (size_t)s_row * DV + dv0 + sc0);
 #pragma unroll
     for (int c = 0; c < SW / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
   }
-  if (STATE_ONLY && s_owner && half == 0 && blockIdx.x == 0)
-    args.gam[((size_t)bh * args.nseg + seg) * DK + s_row] = gamma_acc;
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 256);
@@ -459,17 +593,17 @@ size_t fwd_workspace(int BH, int T, int dk, int dv) {
   return align256((size_t)BH * nseg * dk * dv * sizeof(float)) + align256((size_t)BH * nseg * dk * sizeof(float));
 }
 
-template <int DK, bool STATE_ONLY>
-static cudaError_t launch_fwd_pass(const CUtensorMap* m, const FwdArgs& args, int BH, int dv, int nz, cudaStream_t st) {
-  auto kern = fwd_fused_kernel<DK, STATE_ONLY>;
+template <int DK>
+static cudaError_t launch_state_pass(const CUtensorMap* m, const FwdArgs& args, int BH, int dv, cudaStream_t st) {
+  auto kern = fwd_state_kernel<DK>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdLayout<DK>::ALLOC);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK>::ALLOC);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid(dv / DVT, BH, nz);
-  kern<<<grid, NTHREADS, FwdLayout<DK>::ALLOC, st>>>(m[0], m[1], m[2], m[3], args);
+  dim3 grid(dv / DVT, BH, args.nseg - 1);
+  kern<<<grid, NTHREADS, StateLayout<DK>::ALLOC, st>>>(m[1], m[2], m[3], args);
   return cudaGetLastError();
 }
 
@@ -494,7 +628,7 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
     if (!ws) return cudaErrorInvalidValue;
     a.sbuf = static_cast<float*>(ws);
     a.gam = a.sbuf + align256((size_t)BH * a.nseg * DK * dv * sizeof(float)) / sizeof(float);
-    cudaError_t e = launch_fwd_pass<DK, true>(m, a, BH, dv, a.nseg - 1, st);
+    cudaError_t e = launch_state_pass<DK>(m, a, BH, dv, st);
     if (e != cudaSuccess) return e;
     if (a.nseg > 2) {
       const size_t n = (size_t)BH * DK * dv;
@@ -504,7 +638,16 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
       if (e != cudaSuccess) return e;
     }
   }
-  return launch_fwd_pass<DK, false>(m, a, BH, dv, a.nseg, st);
+  auto kern = fwd_pipe_kernel<DK>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdPipeLayout<DK>::ALLOC);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid(dv / DVT, BH, a.nseg);
+  kern<<<grid, NTHREADS, FwdPipeLayout<DK>::ALLOC, st>>>(m[0], m[1], m[2], m[3], a);
+  return cudaGetLastError();
 }
 
 cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
