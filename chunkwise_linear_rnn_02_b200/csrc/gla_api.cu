@@ -146,7 +146,14 @@ size_t carve_gsa_fwd(Carve& c, int BH, int T, int dk, int dv, int m, int chunk, 
   GsaFwdWs x;
   x.S1 = c.take<float>((size_t)BH * NC * m * dk);
   x.o1 = c.take<float>((size_t)BH * T * m);
-  x.S2 = c.take<float>((size_t)BH * NC * m * dv);
+  // pass 2 is a plain key-gated GLA: per-chunk states for the generic kernels, or the fused
+  // forward's workspace when it serves the shape
+  size_t s2 = (size_t)BH * NC * m * dv;
+  if (gla::fast::fwd_supported(BH, T, m, dv, chunk, dtype)) {
+    const size_t fw = (gla::fast::fwd_workspace(BH, T, m, dv) + sizeof(float) - 1) / sizeof(float);
+    if (fw > s2) s2 = fw;
+  }
+  x.S2 = c.take<float>(s2);
   x.p = need_p ? (void*)c.take<char>((size_t)BH * T * m * esize(dtype)) : nullptr;
   if (w) *w = x;
   return c.used;
@@ -191,6 +198,12 @@ int gsa_fwd_impl(const TI* q, const TI* k, const TI* v, const TI* phi, const TI*
   GLA_CUDA((gk::bwd_dqdk<TI, TI, float>(s1, phi, phi, k, g, q, w.S1, nullptr, w.o1, nullptr, nullptr, nullptr,
                                         st)));
   GLA_CUDA(gk::softmax_fwd<TI>(w.o1, p, nullptr, (long)BH * T, m, st));
+  // pass 2: GLA with queries p, keys phi, values v and the same slot gates (key axis)
+  const int dtype = sizeof(TI) == 2 ? GLA_DTYPE_BF16 : GLA_DTYPE_F32;
+  if (gla::fast::fwd_supported(BH, T, m, dv, C, dtype)) {
+    GLA_CUDA(gla::fast::fwd(p, phi, v, g, h02, o, hT2, BH, T, m, dv, w.S2, st));
+    return GLA_OK;
+  }
   GLA_CUDA(gk::state_fwd<TI>(s2, phi, v, g, h02, 0, w.S2, hT2, 0, st));
   GLA_CUDA((gk::out<TI, TI, TI>(s2, p, phi, v, g, w.S2, o, st)));
   return GLA_OK;
