@@ -213,8 +213,8 @@ def traffic_from_profiles(kernel_key):
         for line in open(os.path.join(pdir, fn)):
             if line.strip().startswith(tag):
                 try:
-                    return float(line.split(":", 1)[1].split()[0])
-                except ValueError:
+                    return float(line.strip()[len(tag):].split()[0])
+                except (ValueError, IndexError):
                     return None
     return None
 
