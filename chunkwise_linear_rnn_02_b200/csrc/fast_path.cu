@@ -211,6 +211,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 // two-stage ring and v through a three-deep ring, so a raw tile is free as soon as its own
 // chunk's math is done.  MMAs issued by one thread complete in order, so waiting for group 1 of
 // chunk i+1 also covers group 2 of chunk i.
+//
+// A ninth warp issues the TMA loads and the MMAs.  tcgen05.mma issue proceeds at the rate the
+// tensor pipe executes (about 48 cycles per 64-wide MMA), so the issuing thread is held for a
+// group's whole duration; in its own warp it holds up no other work.  The 256 compute threads
+// hand over with named barriers: they arrive at kBarOps once a chunk's group-1 operands are in
+// shared memory and at kBarAB once its A operand is, and the producer waits at both.
 // ------------------------------------------------------------------------------------------
 template <int DK>
 struct FwdPipeLayout {
@@ -238,14 +244,18 @@ struct FwdPipeLayout {
   static_assert(C * DK * 4 <= KH - QS_HI && C * C * 4 <= SB_LO - KH, "exact-path scratch");
 };
 
+constexpr int PIPE_THREADS = NTHREADS + 32;  // 8 compute warps + the producer warp
+constexpr int kBarOps = 2, kBarAB = 3;       // compute threads -> producer handoffs
+
 template <int DK>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(PIPE_THREADS, 1)
     fwd_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
                     const FwdArgs args) {
   using L = FwdPipeLayout<DK>;
   using Gate = GateRun<DK, NTHREADS>;
   constexpr int TS = Gate::TS;
+  constexpr int NHAND = NTHREADS + 32;  // threads taking part in a handoff barrier
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_qkg[2], bar_v[3], bar_mma1, bar_mma2;
   __shared__ uint32_t tmem_base_sh;
@@ -253,7 +263,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t base = smem_u32(sm);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int q4 = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
+  const int q4 = warp & 3, half = (warp >> 2) & 1;  // TMEM lane quarter, column half
   const int dv0 = blockIdx.x * DVT, bh = blockIdx.y, seg = blockIdx.z;
   const int T = args.T, DV = args.DV, NC = (T + C - 1) / C;
   const int c_begin = seg * args.seg_chunks;
@@ -277,52 +287,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&bar_mma2, 1);
     fence_mbar_init();
   }
-  __syncthreads();
-  auto load_qkg = [&](int li) {
-    const int s = li & 1, chunk = c_begin + li;
-    uint8_t* st = sm + s * L::QKG;
-    mbar_arrive_expect_tx(&bar_qkg[s], L::QKG);
-    tma_load_3d(st, &tm_q, &bar_qkg[s], 0, chunk * C, bh);
-    tma_load_3d(st + L::RAW, &tm_k, &bar_qkg[s], 0, chunk * C, bh);
-    tma_load_3d(st + 2 * L::RAW, &tm_g, &bar_qkg[s], 0, chunk * C, bh);
-  };
-  auto load_v = [&](int li) {
-    const int b = li % 3;
-    mbar_arrive_expect_tx(&bar_v[b], L::VTB);
-    tma_load_3d(sm + L::V0 + b * L::VTB, &tm_v, &bar_v[b], dv0, (c_begin + li) * C, bh);
-  };
-  if (tid == 0) {
-    load_qkg(0);
-    load_v(0);
-    if (nloc > 1) {
-      load_qkg(1);
-      load_v(1);
-    }
-    if (nloc > 2) load_v(2);
-  }
-
-  // State owned by this thread: row s_row (lane layout of the dS accumulator, M = DK), columns
-  // sc0 .. sc0+31 of the CTA's 64.
-  constexpr int SW = DVT / 2;
-  const bool s_owner = (DK == 128) ? true : (lane < 16);
-  const int s_row = (DK == 128) ? (q4 * 32 + lane) : (q4 * 16 + lane);
-  const int sc0 = half * SW;
-  float S[SW];
-#pragma unroll
-  for (int c = 0; c < SW; ++c) S[c] = 0.f;
-  const float* init = seg == 0 ? (args.h0 ? args.h0 + (size_t)bh * DK * DV : nullptr)
-                               : args.sbuf + ((size_t)bh * args.nseg + seg - 1) * DK * DV;
-  if (s_owner && init) {
-    const float4* src = reinterpret_cast<const float4*>(init + (size_t)s_row * DV + dv0 + sc0);
-#pragma unroll
-    for (int c = 0; c < SW / 4; ++c) {
-      const float4 x = src[c];
-      S[4 * c] = x.x;
-      S[4 * c + 1] = x.y;
-      S[4 * c + 2] = x.z;
-      S[4 * c + 3] = x.w;
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -330,203 +294,262 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t t_A = tmem, t_O0 = tmem + 64, t_dS = tmem + 192;
   const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
 
-  // Gate math of local chunk li (stage li & 1) into registers: Qs hi / lo and Kh for the two
-  // dims gd, gd+1 and the tokens gh*TS .. gh*TS+TS-1 owned by this thread.  Returns the chunk's
-  // exact-path flag (CTA-uniform).
-  uint32_t qh[TS], ql[TS], kh[TS];
-  int gd = 0, gh = 0;
-  auto gate_regs = [&](int li) {
-    const uint8_t* st = sm + (li & 1) * L::QKG;
-    Gate gr;
-    const bool weak = gr.run(st + 2 * L::RAW, DK, tot_sm);
-    float* dec = decay_sm + (li & 1) * DK;
-    if (gr.h == 0) {
-      dec[gr.d] = gr.dec0;
-      dec[gr.d + 1] = gr.dec1;
+  if (warp == NTHREADS / 32) {
+    // ------------------------------ producer warp ------------------------------
+    auto load_qkg = [&](int li) {
+      const int s = li & 1, chunk = c_begin + li;
+      uint8_t* st = sm + s * L::QKG;
+      mbar_arrive_expect_tx(&bar_qkg[s], L::QKG);
+      tma_load_3d(st, &tm_q, &bar_qkg[s], 0, chunk * C, bh);
+      tma_load_3d(st + L::RAW, &tm_k, &bar_qkg[s], 0, chunk * C, bh);
+      tma_load_3d(st + 2 * L::RAW, &tm_g, &bar_qkg[s], 0, chunk * C, bh);
+    };
+    auto load_v = [&](int li) {
+      const int b = li % 3;
+      mbar_arrive_expect_tx(&bar_v[b], L::VTB);
+      tma_load_3d(sm + L::V0 + b * L::VTB, &tm_v, &bar_v[b], dv0, (c_begin + li) * C, bh);
+    };
+    if (lane == 0) {
+      load_qkg(0);
+      load_v(0);
+      if (nloc > 1) {
+        load_qkg(1);
+        load_v(1);
+      }
+      if (nloc > 2) load_v(2);
     }
-    const int safe = __syncthreads_or(weak);
-    gd = gr.d;
-    gh = gr.h;
-    float e0 = gr.pre0 * (safe ? 1.f : 1.f / gr.dec0), e1 = gr.pre1 * (safe ? 1.f : 1.f / gr.dec1);
+    for (int li = 0; li < nloc; ++li) {
+      bar_sync(kBarOps, NHAND);  // chunk li's Qs, Kh and state copy are in shared memory
+      if (lane == 0) {
+        // group 1: A = Qs Kh^T, O_li = Qs S', dS = Kh^T V
+        mbar_wait(&bar_v[li % 3], (li / 3) & 1, latch);
+        tc_fence_after();
+        const uint32_t vbase = base + L::V0 + (li % 3) * L::VTB;
+        const uint32_t t_O = t_O0 + (li & 1) * 64;
+        constexpr uint32_t id_A = idesc_bf16_f32(C, C, false, false);
+        constexpr uint32_t id_O = idesc_bf16_f32(C, DVT, false, true);
+        constexpr uint32_t id_S = idesc_bf16_f32(DK, DVT, true, true);
 #pragma unroll
-    for (int u = 0; u < TS; ++u) {
-      e0 *= gr.a0[u];
-      e1 *= gr.a1[u];
-      const uint32_t wq = *reinterpret_cast<const uint32_t*>(st + ((gh * TS + u) * DK + gd) * 2);
-      split2(bf_lo(wq) * e0, bf_hi(wq) * e1, qh[u], ql[u]);
+        for (int k = 0; k < DK / 16; ++k) {
+          const uint32_t koff = (k >> 2) * (C * 128) + (k & 3) * 32;
+          const uint64_t kd = desc_sw128(base + L::KH + koff, 16, 1024);
+          const uint64_t qh_d = desc_sw128(base + L::QS_HI + koff, 16, 1024);
+          const uint64_t ql_d = desc_sw128(base + L::QS_LO + koff, 16, 1024);
+          umma_bf16(t_A, qh_d, kd, id_A, k > 0);
+          umma_bf16(t_A, ql_d, kd, id_A, 1);
+          const uint64_t sh = desc_sw128(base + L::SB_HI + k * 2048, 16, 1024);
+          umma_bf16(t_O, qh_d, sh, id_O, k > 0);
+          umma_bf16(t_O, qh_d, desc_sw128(base + L::SB_LO + k * 2048, 16, 1024), id_O, 1);
+          umma_bf16(t_O, ql_d, sh, id_O, 1);
+        }
+#pragma unroll
+        for (int k = 0; k < C / 16; ++k)
+          umma_bf16(t_dS, desc_sw128(base + L::KH + k * 2048, C * 128, 1024),
+                    desc_sw128(vbase + k * 2048, 16, 1024), id_S, k > 0);
+        umma_commit(&bar_mma1);
+      }
+      bar_sync(kBarAB, NHAND);  // chunk li's A operand is in shared memory; its raw tiles are free
+      if (lane == 0) {
+        // group 2: O_li += A V
+        tc_fence_after();
+        const uint32_t vbase = base + L::V0 + (li % 3) * L::VTB;
+        const uint32_t t_O = t_O0 + (li & 1) * 64;
+        constexpr uint32_t id_O = idesc_bf16_f32(C, DVT, false, true);
+#pragma unroll
+        for (int k = 0; k < C / 16; ++k) {
+          const uint64_t vd = desc_sw128(vbase + k * 2048, 16, 1024);
+          umma_bf16(t_O, desc_sw128(base + L::AB_HI + k * 32, 16, 1024), vd, id_O, 1);
+          umma_bf16(t_O, desc_sw128(base + L::AB_LO + k * 32, 16, 1024), vd, id_O, 1);
+        }
+        umma_commit(&bar_mma2);
+        if (li + 2 < nloc) {
+          load_qkg(li + 2);
+          if (li >= 1) {
+            // The v buffer of chunk li+2 held chunk li-1's v, read by its group 2.  Group 1 of
+            // chunk li was issued after that group 2 and MMAs complete in order, so its completion
+            // frees the buffer.  (A parity wait on group 2's barrier could be two phases behind
+            // here, since group 2 of chunk li may already have completed; group 1 of chunk li+1
+            // has not been issued yet, so this wait is at most one phase behind.)
+            mbar_wait(&bar_mma1, li & 1, latch);
+            load_v(li + 2);
+          }
+        }
+      }
+      __syncwarp();
     }
-    float f0 = gr.suf0, f1 = gr.suf1;
+  } else {
+    // ------------------------------ compute warps ------------------------------
+    // State owned by this thread: row s_row (lane layout of the dS accumulator, M = DK), columns
+    // sc0 .. sc0+31 of the CTA's 64.
+    constexpr int SW = DVT / 2;
+    const bool s_owner = (DK == 128) ? true : (lane < 16);
+    const int s_row = (DK == 128) ? (q4 * 32 + lane) : (q4 * 16 + lane);
+    const int sc0 = half * SW;
+    float S[SW];
 #pragma unroll
-    for (int u = TS - 1; u >= 0; --u) {
-      const uint32_t wk = *reinterpret_cast<const uint32_t*>(st + L::RAW + ((gh * TS + u) * DK + gd) * 2);
-      kh[u] = pack2(bf_lo(wk) * f0, bf_hi(wk) * f1);
-      f0 *= gr.a0[u];
-      f1 *= gr.a1[u];
+    for (int c = 0; c < SW; ++c) S[c] = 0.f;
+    const float* init = seg == 0 ? (args.h0 ? args.h0 + (size_t)bh * DK * DV : nullptr)
+                                 : args.sbuf + ((size_t)bh * args.nseg + seg - 1) * DK * DV;
+    if (s_owner && init) {
+      const float4* src = reinterpret_cast<const float4*>(init + (size_t)s_row * DV + dv0 + sc0);
+#pragma unroll
+      for (int c = 0; c < SW / 4; ++c) {
+        const float4 x = src[c];
+        S[4 * c] = x.x;
+        S[4 * c + 1] = x.y;
+        S[4 * c + 2] = x.z;
+        S[4 * c + 3] = x.w;
+      }
     }
-    return safe;
-  };
-  // Operands of local chunk li into shared memory: Qs, Kh (from registers) and the state copy.
-  auto store_ops = [&](int li, int safe) {
-    const uint32_t blk = (gd >> 6) * (C * 128), col = gd & 63;
-#pragma unroll
-    for (int u = 0; u < TS; ++u) {
-      const uint32_t off = blk + sw128(gh * TS + u, col);
-      *reinterpret_cast<uint32_t*>(sm + L::QS_HI + off) = qh[u];
-      *reinterpret_cast<uint32_t*>(sm + L::QS_LO + off) = ql[u];
-      *reinterpret_cast<uint32_t*>(sm + L::KH + off) = kh[u];
-    }
-    if (s_owner) {
-      const float sc = safe ? 1.f : decay_sm[(li & 1) * DK + s_row];
-      float sv[SW];
-#pragma unroll
-      for (int c = 0; c < SW; ++c) sv[c] = S[c] * sc;
-      store_half_split(sm + L::SB_HI, sm + L::SB_LO, s_row, sv, half);
-    }
-  };
-  // MMA group 1 of local chunk li: A = Qs Kh^T, O_li = Qs S', dS = Kh^T V.
-  auto issue_m1 = [&](int li) {
-    mbar_wait(&bar_v[li % 3], (li / 3) & 1, latch);
-    tc_fence_after();
-    const uint32_t vbase = base + L::V0 + (li % 3) * L::VTB;
-    const uint32_t t_O = t_O0 + (li & 1) * 64;
-    constexpr uint32_t id_A = idesc_bf16_f32(C, C, false, false);
-    constexpr uint32_t id_O = idesc_bf16_f32(C, DVT, false, true);
-    constexpr uint32_t id_S = idesc_bf16_f32(DK, DVT, true, true);
-#pragma unroll
-    for (int k = 0; k < DK / 16; ++k) {
-      const uint32_t koff = (k >> 2) * (C * 128) + (k & 3) * 32;
-      const uint64_t kd = desc_sw128(base + L::KH + koff, 16, 1024);
-      const uint64_t qh_d = desc_sw128(base + L::QS_HI + koff, 16, 1024);
-      const uint64_t ql_d = desc_sw128(base + L::QS_LO + koff, 16, 1024);
-      umma_bf16(t_A, qh_d, kd, id_A, k > 0);
-      umma_bf16(t_A, ql_d, kd, id_A, 1);
-      const uint64_t sh = desc_sw128(base + L::SB_HI + k * 2048, 16, 1024);
-      umma_bf16(t_O, qh_d, sh, id_O, k > 0);
-      umma_bf16(t_O, qh_d, desc_sw128(base + L::SB_LO + k * 2048, 16, 1024), id_O, 1);
-      umma_bf16(t_O, ql_d, sh, id_O, 1);
-    }
-#pragma unroll
-    for (int k = 0; k < C / 16; ++k)
-      umma_bf16(t_dS, desc_sw128(base + L::KH + k * 2048, C * 128, 1024), desc_sw128(vbase + k * 2048, 16, 1024),
-                id_S, k > 0);
-    umma_commit(&bar_mma1);
-  };
-  // O rows of local chunk li (after its group 2): bf16 straight to global.
-  auto store_o = [&](int li) {
-    mbar_wait(&bar_mma2, li & 1, latch);
-    tc_fence_after();
-    const int j = q4 * 16 + lane, cb = half * 32;
-    float ov[32];
-    tmem_ld32(t_O0 + (li & 1) * 64 + lane_off + cb, ov);
-    tmem_ld_wait();
-    const int t = (c_begin + li) * C + j;
-    if (lane < 16 && t < T) store_half_global_bf16(args.o + ((size_t)bh * T + t) * DV + dv0 + cb, ov);
-  };
 
-  mbar_wait(&bar_qkg[0], 0, latch);
-  int safe = gate_regs(0);
-  store_ops(0, safe);
-  fence_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (tid == 0) issue_m1(0);
-  for (int li = 0; li < nloc; ++li) {
-    const uint8_t* st = sm + (li & 1) * L::QKG;
-    // ---- while group 1 of chunk li runs: outputs of chunk li-1, gate math of chunk li+1 ----
-    if (li > 0) {
-      store_o(li - 1);
-      if (tid == 0 && li + 2 < nloc) load_v(li + 2);  // its buffer held chunk li-1's v
-    }
-    int safe_next = 0;
-    if (li + 1 < nloc) {
-      mbar_wait(&bar_qkg[(li + 1) & 1], ((li + 1) >> 1) & 1, latch);
-      safe_next = gate_regs(li + 1);
-    }
-    // ---- group 1 done: exact A if needed, A epilogue, state update, group 2 ----
-    mbar_wait(&bar_mma1, li & 1, latch);
-    tc_fence_after();
-    float* Aex = reinterpret_cast<float*>(sm + L::XA);
-    if (safe) {
-      float* Bf = reinterpret_cast<float*>(sm + L::XB);
-      if (tid < DK) {
-        float b = 0.f;
-        for (int j = 0; j < C; ++j) {
-          b += bf2f(st + 2 * L::RAW + (j * DK + tid) * 2);
-          Bf[j * DK + tid] = b;
-        }
+    // Gate math of local chunk li (stage li & 1) into registers: Qs hi / lo and Kh for the two
+    // dims gd, gd+1 and the tokens gh*TS .. gh*TS+TS-1 owned by this thread.  Returns the chunk's
+    // exact-path flag (CTA-uniform).
+    uint32_t qh[TS], ql[TS], kh[TS];
+    int gd = 0, gh = 0;
+    auto gate_regs = [&](int li) {
+      const uint8_t* st = sm + (li & 1) * L::QKG;
+      Gate gr;
+      const bool weak = gr.run(st + 2 * L::RAW, DK, tot_sm);
+      float* dec = decay_sm + (li & 1) * DK;
+      if (gr.h == 0) {
+        dec[gr.d] = gr.dec0;
+        dec[gr.d + 1] = gr.dec1;
       }
-      __syncthreads();
-      for (int e = tid; e < C * C; e += NTHREADS) {
-        const int j = e / C, r = e % C;
-        float acc = 0.f;
-        if (r <= j)
-          for (int d = 0; d < DK; ++d)
-            acc += bf2f(st + (j * DK + d) * 2) * bf2f(st + L::RAW + (r * DK + d) * 2) *
-                   __expf(Bf[j * DK + d] - Bf[r * DK + d]);
-        Aex[e] = acc;
-      }
-      __syncthreads();
-    }
-    {
-      const int j = q4 * 16 + lane, cb = half * 32;
-      float a[32];
-      tmem_ld32(t_A + lane_off + cb, a);
-      tmem_ld_wait();
-      if (lane < 16) {
-        if (safe) {
+      const int safe = bar_or(kBarCompute, NTHREADS, weak);
+      gd = gr.d;
+      gh = gr.h;
+      float e0 = gr.pre0 * (safe ? 1.f : 1.f / gr.dec0), e1 = gr.pre1 * (safe ? 1.f : 1.f / gr.dec1);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) a[c] = Aex[j * C + cb + c];
-        }
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (cb + c > j) a[c] = 0.f;
-        store_half_split(sm + L::AB_HI, sm + L::AB_LO, j, a, half);
+      for (int u = 0; u < TS; ++u) {
+        e0 *= gr.a0[u];
+        e1 *= gr.a1[u];
+        const uint32_t wq = *reinterpret_cast<const uint32_t*>(st + ((gh * TS + u) * DK + gd) * 2);
+        split2(bf_lo(wq) * e0, bf_hi(wq) * e1, qh[u], ql[u]);
       }
-      float ds[SW];
-      tmem_ld32(t_dS + lane_off + sc0, ds);
-      tmem_ld_wait();
+      float f0 = gr.suf0, f1 = gr.suf1;
+#pragma unroll
+      for (int u = TS - 1; u >= 0; --u) {
+        const uint32_t wk = *reinterpret_cast<const uint32_t*>(st + L::RAW + ((gh * TS + u) * DK + gd) * 2);
+        kh[u] = pack2(bf_lo(wk) * f0, bf_hi(wk) * f1);
+        f0 *= gr.a0[u];
+        f1 *= gr.a1[u];
+      }
+      return safe;
+    };
+    // Operands of local chunk li into shared memory (Qs, Kh from registers; the state copy), then
+    // hand them to the producer.
+    auto store_ops = [&](int li, int safe) {
+      const uint32_t blk = (gd >> 6) * (C * 128), col = gd & 63;
+#pragma unroll
+      for (int u = 0; u < TS; ++u) {
+        const uint32_t off = blk + sw128(gh * TS + u, col);
+        *reinterpret_cast<uint32_t*>(sm + L::QS_HI + off) = qh[u];
+        *reinterpret_cast<uint32_t*>(sm + L::QS_LO + off) = ql[u];
+        *reinterpret_cast<uint32_t*>(sm + L::KH + off) = kh[u];
+      }
       if (s_owner) {
-        const float dec = decay_sm[(li & 1) * DK + s_row];
+        const float sc = safe ? 1.f : decay_sm[(li & 1) * DK + s_row];
+        float sv[SW];
 #pragma unroll
-        for (int c = 0; c < SW; ++c) S[c] = dec * S[c] + ds[c];
+        for (int c = 0; c < SW; ++c) sv[c] = S[c] * sc;
+        store_half_split(sm + L::SB_HI, sm + L::SB_LO, s_row, sv, half);
       }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (tid == 0) {
-      const uint32_t vbase = base + L::V0 + (li % 3) * L::VTB;
-      const uint32_t t_O = t_O0 + (li & 1) * 64;
-      constexpr uint32_t id_O = idesc_bf16_f32(C, DVT, false, true);
-#pragma unroll
-      for (int k = 0; k < C / 16; ++k) {
-        const uint64_t vd = desc_sw128(vbase + k * 2048, 16, 1024);
-        umma_bf16(t_O, desc_sw128(base + L::AB_HI + k * 32, 16, 1024), vd, id_O, 1);
-        umma_bf16(t_O, desc_sw128(base + L::AB_LO + k * 32, 16, 1024), vd, id_O, 1);
-      }
-      umma_commit(&bar_mma2);
-      if (li + 2 < nloc) load_qkg(li + 2);  // chunk li's raw tiles are no longer read
-    }
-    // ---- while group 2 of chunk li runs: operands of chunk li+1, then its group 1 ----
-    if (li + 1 < nloc) {
-      store_ops(li + 1, safe_next);
       fence_async_smem();
       tc_fence_before();
-      __syncthreads();
+      bar_arrive(kBarOps, NHAND);
+    };
+    // O rows of local chunk li (after its group 2): bf16 straight to global.
+    auto store_o = [&](int li) {
+      mbar_wait(&bar_mma2, li & 1, latch);
       tc_fence_after();
-      if (tid == 0) issue_m1(li + 1);
-    }
-    safe = safe_next;
-  }
-  store_o(nloc - 1);
+      const int j = q4 * 16 + lane, cb = half * 32;
+      float ov[32];
+      tmem_ld32(t_O0 + (li & 1) * 64 + lane_off + cb, ov);
+      tmem_ld_wait();
+      const int t = (c_begin + li) * C + j;
+      if (lane < 16 && t < T) store_half_global_bf16(args.o + ((size_t)bh * T + t) * DV + dv0 + cb, ov);
+    };
 
-  float* out = (seg == args.nseg - 1 && args.hT) ? args.hT + (size_t)bh * DK * DV : nullptr;
-  if (s_owner && out) {
-    float4* dst = reinterpret_cast<float4*>(out + (size_t)s_row * DV + dv0 + sc0);
+    mbar_wait(&bar_qkg[0], 0, latch);
+    int safe = gate_regs(0);
+    store_ops(0, safe);
+    for (int li = 0; li < nloc; ++li) {
+      const uint8_t* st = sm + (li & 1) * L::QKG;
+      // ---- while group 1 of chunk li runs: outputs of chunk li-1, gate math of chunk li+1 ----
+      if (li > 0) store_o(li - 1);
+      int safe_next = 0;
+      if (li + 1 < nloc) {
+        mbar_wait(&bar_qkg[(li + 1) & 1], ((li + 1) >> 1) & 1, latch);
+        safe_next = gate_regs(li + 1);
+      }
+      // ---- group 1 done: exact A if needed, A epilogue, state update; group 2 next ----
+      mbar_wait(&bar_mma1, li & 1, latch);
+      tc_fence_after();
+      float* Aex = reinterpret_cast<float*>(sm + L::XA);
+      if (safe) {
+        float* Bf = reinterpret_cast<float*>(sm + L::XB);
+        if (tid < DK) {
+          float b = 0.f;
+          for (int j = 0; j < C; ++j) {
+            b += bf2f(st + 2 * L::RAW + (j * DK + tid) * 2);
+            Bf[j * DK + tid] = b;
+          }
+        }
+        bar_sync(kBarCompute, NTHREADS);
+        for (int e = tid; e < C * C; e += NTHREADS) {
+          const int j = e / C, r = e % C;
+          float acc = 0.f;
+          if (r <= j)
+            for (int d = 0; d < DK; ++d)
+              acc += bf2f(st + (j * DK + d) * 2) * bf2f(st + L::RAW + (r * DK + d) * 2) *
+                     __expf(Bf[j * DK + d] - Bf[r * DK + d]);
+          Aex[e] = acc;
+        }
+        bar_sync(kBarCompute, NTHREADS);
+      }
+      {
+        const int j = q4 * 16 + lane, cb = half * 32;
+        float a[32];
+        tmem_ld32(t_A + lane_off + cb, a);
+        tmem_ld_wait();
+        if (lane < 16) {
+          if (safe) {
 #pragma unroll
-    for (int c = 0; c < SW / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
+            for (int c = 0; c < 32; ++c) a[c] = Aex[j * C + cb + c];
+          }
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (cb + c > j) a[c] = 0.f;
+          store_half_split(sm + L::AB_HI, sm + L::AB_LO, j, a, half);
+        }
+        float ds[SW];
+        tmem_ld32(t_dS + lane_off + sc0, ds);
+        tmem_ld_wait();
+        if (s_owner) {
+          const float dec = decay_sm[(li & 1) * DK + s_row];
+#pragma unroll
+          for (int c = 0; c < SW; ++c) S[c] = dec * S[c] + ds[c];
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      bar_arrive(kBarAB, NHAND);
+      // ---- while group 2 of chunk li runs: operands of chunk li+1 (group 1 follows) ----
+      // Exact-path scratch over Qs / Kh: every compute thread has finished with it before any
+      // thread stores chunk li+1's operands.
+      if (safe) bar_sync(kBarCompute, NTHREADS);
+      if (li + 1 < nloc) store_ops(li + 1, safe_next);
+      safe = safe_next;
+    }
+    store_o(nloc - 1);
+
+    float* out = (seg == args.nseg - 1 && args.hT) ? args.hT + (size_t)bh * DK * DV : nullptr;
+    if (s_owner && out) {
+      float4* dst = reinterpret_cast<float4*>(out + (size_t)s_row * DV + dv0 + sc0);
+#pragma unroll
+      for (int c = 0; c < SW / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -646,7 +669,7 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
     attr_set = true;
   }
   dim3 grid(dv / DVT, BH, a.nseg);
-  kern<<<grid, NTHREADS, FwdPipeLayout<DK>::ALLOC, st>>>(m[0], m[1], m[2], m[3], a);
+  kern<<<grid, PIPE_THREADS, FwdPipeLayout<DK>::ALLOC, st>>>(m[0], m[1], m[2], m[3], a);
   return cudaGetLastError();
 }
 

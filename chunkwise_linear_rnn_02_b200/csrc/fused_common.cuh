@@ -161,6 +161,25 @@ __device__ __forceinline__ void store_half_global_bf16(__nv_bfloat16* dst, const
   }
 }
 
+// Named barriers (id 0 is __syncthreads).  bar_sync waits; bar_arrive signals without waiting (a
+// producer warp syncs on a barrier that the consumer threads only arrive at); bar_or is a barrier
+// that also ORs a predicate over the participating threads.  Counts are in threads; every warp
+// taking part executes the instruction with all its lanes.
+__device__ __forceinline__ void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+__device__ __forceinline__ void bar_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ int bar_or(int id, int n, int pred) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %3, 0;\n\tbar.red.or.pred q, %1, %2, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(id), "r"(n), "r"(pred)
+      : "memory");
+  return r;
+}
+constexpr int kBarCompute = 1;  // named barrier of the threads that run the gate math
+
 // Gate math shared by the fused kernels.  The CTA's NTH threads cover ND key dimensions of one
 // chunk: thread t owns dimensions (2p, 2p+1), p = t % (ND/2), and the run of TS = 64 * (ND/2) / NTH
 // tokens starting at h * TS, h = t / (ND/2).  It loads the raw log-gates g (row-major [64][gstride]
@@ -202,7 +221,7 @@ struct GateRun {
     }
     tot[h * ND + d] = r0;
     tot[h * ND + d + 1] = r1;
-    __syncthreads();
+    bar_sync(kBarCompute, NTH);  // the NTH threads running the gate math
     pre0 = pre1 = suf0 = suf1 = 1.f;
 #pragma unroll
     for (int hh = 0; hh < NSPLIT; ++hh) {

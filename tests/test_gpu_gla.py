@@ -192,3 +192,13 @@ def test_fused_shapes_mixed_strong_gates():
     g[:, 1, 200:210, :7] = -9.0  # part of chunk 3, a few dimensions
     inp["g"] = g.to(torch.bfloat16)
     _run_fwd_bwd(inp, 64)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128)])
+def test_fused_forward_long_walk(dk, dv):
+    """Enough heads to fill the GPU (no sequence split), so one CTA walks every chunk of its head:
+    exercises the pipelined forward's ring buffers and barrier phases over many chunks."""
+    H = 80 if dv == 64 else 40
+    inp = make_gla_inputs(1, H, 64 * 9 + 7, dk, dv, torch.bfloat16, seed=50 + dk, with_h0=True, with_do=False)
+    assert gla.workspace_bytes("gla_chunk_fwd", 1, H, 64 * 9 + 7, dk, dv, 64, 1) == 0  # no split
+    _run_fwd_bwd(inp, 64, check_bwd=False)
