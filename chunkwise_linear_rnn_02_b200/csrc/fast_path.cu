@@ -50,12 +50,14 @@ constexpr int NTHREADS = 256;  // warps w and w+4 share TMEM lanes and split acc
 // Arguments of the forward passes
 // ------------------------------------------------------------------------------------------
 struct FwdArgs {
-  const float* h0;     // [BH][DK][DV] or null (zeros)
+  const float* h0;     // [BH][DK][DV] or null (zeros); element strides st_bh (head), st_row (row)
   float* sbuf;         // [BH][nseg][DK][DV]: segment end states (state-only pass), then entry states
   float* gam;          // [BH][nseg][DK]: segment decay products
   __nv_bfloat16* o;
   float* hT;           // [BH][DK][DV] or null
   int T, DV, seg_chunks, nseg;
+  long long st_bh, st_row;  // h0 / hT strides (a sub-block of a larger state when the shape is split)
+  float* acc_o;             // optional fp32 output [BH*T][DV] in place of o (split shapes)
   unsigned int* latch;
 };
 
@@ -127,7 +129,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
   for (int c = 0; c < SW; ++c) S[c] = 0.f;
   if (seg == 0 && s_owner && args.h0) {
-    const float4* src = reinterpret_cast<const float4*>(args.h0 + ((size_t)bh * DK + s_row) * DV + dv0 + sc0);
+    const float4* src = reinterpret_cast<const float4*>(args.h0 + bh * args.st_bh + s_row * args.st_row + dv0 + sc0);
 #pragma unroll
     for (int c = 0; c < SW / 4; ++c) {
       const float4 x = src[c];
@@ -388,10 +390,11 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     float S[SW];
 #pragma unroll
     for (int c = 0; c < SW; ++c) S[c] = 0.f;
-    const float* init = seg == 0 ? (args.h0 ? args.h0 + (size_t)bh * DK * DV : nullptr)
+    const float* init = seg == 0 ? (args.h0 ? args.h0 + bh * args.st_bh : nullptr)
                                  : args.sbuf + ((size_t)bh * args.nseg + seg - 1) * DK * DV;
+    const long long ipitch = seg == 0 ? args.st_row : DV;
     if (s_owner && init) {
-      const float4* src = reinterpret_cast<const float4*>(init + (size_t)s_row * DV + dv0 + sc0);
+      const float4* src = reinterpret_cast<const float4*>(init + s_row * ipitch + dv0 + sc0);
 #pragma unroll
       for (int c = 0; c < SW / 4; ++c) {
         const float4 x = src[c];
@@ -468,7 +471,15 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       tmem_ld32(t_O0 + (li & 1) * 64 + lane_off + cb, ov);
       tmem_ld_wait();
       const int t = (c_begin + li) * C + j;
-      if (lane < 16 && t < T) store_half_global_bf16(args.o + ((size_t)bh * T + t) * DV + dv0 + cb, ov);
+      if (lane < 16 && t < T) {
+        if (args.acc_o) {
+          float4* p = reinterpret_cast<float4*>(args.acc_o + ((size_t)bh * T + t) * DV + dv0 + cb);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) p[c] = make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3]);
+        } else {
+          store_half_global_bf16(args.o + ((size_t)bh * T + t) * DV + dv0 + cb, ov);
+        }
+      }
     };
 
     mbar_wait(&bar_qkg[0], 0, latch);
@@ -544,9 +555,9 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     }
     store_o(nloc - 1);
 
-    float* out = (seg == args.nseg - 1 && args.hT) ? args.hT + (size_t)bh * DK * DV : nullptr;
+    float* out = (seg == args.nseg - 1 && args.hT) ? args.hT + bh * args.st_bh : nullptr;
     if (s_owner && out) {
-      float4* dst = reinterpret_cast<float4*>(out + (size_t)s_row * DV + dv0 + sc0);
+      float4* dst = reinterpret_cast<float4*>(out + s_row * args.st_row + dv0 + sc0);
 #pragma unroll
       for (int c = 0; c < SW / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
     }
@@ -632,7 +643,8 @@ static cudaError_t launch_state_pass(const CUtensorMap* m, const FwdArgs& args, 
 
 template <int DK>
 static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o,
-                              float* hT, int BH, int T, int dv, void* ws, cudaStream_t st) {
+                              float* hT, int BH, int T, int dv, long long st_bh, long long st_row, float* acc_o,
+                              void* ws, cudaStream_t st) {
   CUtensorMap m[4];
   if (!make_map(&m[0], q, BH, T, DK, DK, false) || !make_map(&m[1], k, BH, T, DK, DK, false) ||
       !make_map(&m[2], g, BH, T, DK, DK, false) || !make_map(&m[3], v, BH, T, dv, DVT, true))
@@ -643,6 +655,9 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
   a.hT = hT;
   a.T = T;
   a.DV = dv;
+  a.st_bh = st_bh;
+  a.st_row = st_row;
+  a.acc_o = acc_o;
   a.latch = device_error_latch();
   plan_segments(BH, T, dv, &a.nseg, &a.seg_chunks);
   a.sbuf = nullptr;
@@ -674,9 +689,12 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
 }
 
 cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
-                int BH, int T, int dk, int dv, void* ws, cudaStream_t st) {
-  if (dk == 64) return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, ws, st);
-  if (dk == 128) return launch_fwd<128>(q, k, v, g, h0, o, hT, BH, T, dv, ws, st);
+                int BH, int T, int dk, int dv, void* ws, cudaStream_t st, long long st_bh, long long st_row,
+                float* acc_o) {
+  if (st_bh < 0) st_bh = (long long)dk * dv;
+  if (st_row < 0) st_row = dv;
+  if (dk == 64) return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st);
+  if (dk == 128) return launch_fwd<128>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st);
   return cudaErrorNotSupported;
 }
 

@@ -13,14 +13,26 @@ namespace fast {
 
 bool fwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype);
 size_t fwd_workspace(int BH, int T, int dk, int dv);
+// st_bh / st_row: element strides of the fp32 states per head and per row (defaults, when
+// negative: dk*dv and dv).  A split shape passes a sub-block of the caller's states this way, and
+// an fp32 array acc_o [BH*T][dv] that receives o in place of the bf16 output.
 cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
-                int BH, int T, int dk, int dv, void* ws, cudaStream_t st);
+                int BH, int T, int dk, int dv, void* ws, cudaStream_t st, long long st_bh = -1,
+                long long st_row = -1, float* acc_o = nullptr);
+
+// fp32 outputs of a backward sub-problem (split shapes): dq / dk / dg go to columns ck.. of
+// [BH*T][pk] arrays, dv to columns cv.. of a [BH*T][pv] array.
+struct BwdAccum {
+  float *q, *k, *g, *v;
+  int pk, ck, pv, cv;
+};
 
 bool bwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype);
 size_t bwd_workspace(int BH, int T, int dk, int dv);
 cudaError_t bwd(const void* q, const void* k, const void* v, const void* g, const float* h0, const void* dO,
                 const float* dhT, void* dq, void* dk, void* dv, void* dg, float* dh0, int BH, int T, int dkd,
-                int dvd, void* ws, cudaStream_t st);
+                int dvd, void* ws, cudaStream_t st, long long st_bh = -1, long long st_row = -1,
+                const BwdAccum* acc = nullptr);
 
 }  // namespace fast
 }  // namespace gla

@@ -48,8 +48,15 @@ struct BwdArgs {
   float* ws_qx;    // [BH][NC][DK] chunk sums of Qt X
   float* ws_part;  // [BH][NC][DK][64] forward-walk part of dg, one row of 64 tokens per chunk and dim
   int T, n_key_ctas;
+  long long st_bh, st_row;  // h0 / dhT / dh0 strides (a sub-block of a larger state when split)
+  // Optional fp32 outputs for a split shape: when set, dq / dk / dg go to columns acc_ck + key dim
+  // of [BH*T][acc_pk] arrays and dv to columns acc_cv + value col of a [BH*T][acc_pv] array, in
+  // place of the bf16 outputs.
+  float *acc_q, *acc_k, *acc_g, *acc_v;
+  int acc_pk, acc_ck, acc_pv, acc_cv;
   unsigned int* latch;
 };
+
 
 // ------------------------------------------------------------------------------------------
 // Key-tile CTA
@@ -105,7 +112,7 @@ struct KeyLayout {
 // buffer, Kh or Qt operand, state copy and rescale) and issue its group 1; then finish chunk i's
 // outputs.  The epilogue forms E1 / E2 itself from the raw gates and the run products of the gate
 // run, multiplying in the same order, so its values equal the ones behind the MMA operands.
-template <int DK, int DV>
+template <int DK, int DV, bool ACC>
 __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int tau, uint64_t* bars,
                               uint32_t tmem) {
   using L = KeyLayout<DK, DV>;
@@ -185,7 +192,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 64) {
 #pragma unroll
       for (int c = 0; c < 64; ++c)
-        v[c] = (src && row_owner) ? src[((size_t)bh * DK + d0 + row) * DV + c0 + c] : 0.f;
+        v[c] = (src && row_owner) ? src[bh * a.st_bh + (d0 + row) * a.st_row + c0 + c] : 0.f;
       tmem_st32(tmem + L::T_SG + lane_off + c0, v);
       tmem_st32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
     }
@@ -345,6 +352,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       }
       const float inv = 1.f / DEC[b * KT + d];
       __nv_bfloat16* dst = a.dq + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
+      float* dst32 = ACC ? a.acc_q + ((size_t)bh * T + i * C + tb) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
 #pragma unroll
       for (int rr = 0; rr < 4; ++rr) {
         float e = 1.f;  // E1 = e^{B_j}, formed as GateRun::forward forms it
@@ -355,7 +363,12 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
           e *= ex2(raw(pg, j, d) * kLog2e);
           if (!safe) y[c] *= e * inv;
           const float qv = raw(pq, j, d), kv = raw(pk, j, d);
-          if (i * C + j < T) dst[(size_t)c * DK] = __float2bfloat16_rn(e * x[c] + y[c]);
+          if (i * C + j < T) {
+            if (ACC)
+              dst32[(size_t)c * a.acc_pk] = e * x[c] + y[c];
+            else
+              dst[(size_t)c * DK] = __float2bfloat16_rn(e * x[c] + y[c]);
+          }
           x[c] = bf_split_sum(qv * e) * x[c];  // Qt X, with Qt as the G update sees it
           y[c] = qv * (y[c] - DIAG[j] * kv);   // q dq^intra without j = r
           tot_s += x[c];
@@ -396,7 +409,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
       tmem_ld_wait();
       if (row_owner && a.dhT) {
-        const float* src = a.dhT + ((size_t)bh * DK + d0 + row) * DV + c0;
+        const float* src = a.dhT + bh * a.st_bh + (d0 + row) * a.st_row + c0;
 #pragma unroll
         for (int c = 0; c < 32; ++c) acc += src[c] * v[c];
       }
@@ -471,6 +484,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       }
       const float inv = 1.f / DEC[b * KT + d];
       __nv_bfloat16* dst = a.dk + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
+      float* dst32 = ACC ? a.acc_k + ((size_t)bh * T + i * C + tb) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
 #pragma unroll
       for (int rr = 0; rr < 4; ++rr) {
         const int h = half * 4 + rr;
@@ -490,7 +504,12 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
           const float ev = e2[u];
           if (!safe) w[c] *= ev * inv;
           const float qv = raw(pq, r, d), kv = raw(pk, r, d);
-          if (i * C + r < T) dst[(size_t)c * DK] = __float2bfloat16_rn(ev * z[c] + w[c]);
+          if (i * C + r < T) {
+            if (ACC)
+              dst32[(size_t)c * a.acc_pk] = ev * z[c] + w[c];
+            else
+              dst[(size_t)c * DK] = __float2bfloat16_rn(ev * z[c] + w[c]);
+          }
           const float kz = bf_split_sum(kv * ev) * z[c];  // Kh Z, with Kh as the S update sees it
           w[c] = kz + kv * (w[c] - DIAG[r] * qv);        // plus k dk^intra without j = r
           tot_k += kz;
@@ -507,9 +526,15 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       const float ci = CARRY[(n & 1) * KT + d] + qxn - (tot_k + o.x);
       float pre = half == 1 ? o.y : 0.f;
       __nv_bfloat16* dst = a.dg + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
+      float* dst32 = ACC ? a.acc_g + ((size_t)bh * T + i * C + tb) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        if (i * C + tb + c < T) dst[(size_t)c * DK] = __float2bfloat16_rn(ci + pre + pv[c]);
+        if (i * C + tb + c < T) {
+          if (ACC)
+            dst32[(size_t)c * a.acc_pk] = ci + pre + pv[c];
+          else
+            dst[(size_t)c * DK] = __float2bfloat16_rn(ci + pre + pv[c]);
+        }
         pre += w[c];
       }
       if (half == 0) CARRY[((n + 1) & 1) * KT + d] = ci;
@@ -522,7 +547,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
       tmem_ld_wait();
       if (row_owner) {
-        float4* dst = reinterpret_cast<float4*>(a.dh0 + ((size_t)bh * DK + d0 + row) * DV + c0);
+        float4* dst = reinterpret_cast<float4*>(a.dh0 + bh * a.st_bh + (d0 + row) * a.st_row + c0);
 #pragma unroll
         for (int c = 0; c < 8; ++c) dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
       }
@@ -558,7 +583,7 @@ struct ValLayout {
   static_assert(C * DK * 4 <= KH_HI - QP_HI && C * C * 4 <= GC_HI - KH_HI, "exact-path scratch");
 };
 
-template <int DK>
+template <int DK, bool ACC>
 __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int vt, int DV,
                               uint64_t* bars, uint32_t tmem) {
   using L = ValLayout<DK>;
@@ -610,7 +635,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     float v[64];
     for (int cb = half * HT; cb < (half + 1) * HT; cb += 64) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) v[c] = a.dhT ? a.dhT[((size_t)bh * DK + grow) * DV + c0 + cb + c] : 0.f;
+      for (int c = 0; c < 64; ++c) v[c] = a.dhT ? a.dhT[bh * a.st_bh + grow * a.st_row + c0 + cb + c] : 0.f;
       tmem_st32(tmem + L::T_G + lane_off + cb, v);
       tmem_st32(tmem + L::T_G + lane_off + cb + 32, v + 32);
       store_row_split(sm + L::GC_HI + (cb / 64) * (DK * 128), sm + L::GC_LO + (cb / 64) * (DK * 128), grow, v, 1.f);
@@ -751,7 +776,15 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         tmem_ld32(tmem + L::T_DV + lane_off + cb, v);
         tmem_ld32(tmem + L::T_DV + lane_off + cb + 32, v + 32);
         tmem_ld_wait();
-        if (row_owner && t < T) store_row_global_bf16(a.dv + ((size_t)bh * T + t) * DV + c0 + cb, v);
+        if (row_owner && t < T) {
+          if (ACC) {
+            float4* p = reinterpret_cast<float4*>(a.acc_v + ((size_t)bh * T + t) * a.acc_pv + a.acc_cv + c0 + cb);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) p[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+          } else {
+            store_row_global_bf16(a.dv + ((size_t)bh * T + t) * DV + c0 + cb, v);
+          }
+        }
       }
     }
     tc_fence_before();
@@ -770,7 +803,7 @@ struct BwdSmem {
   static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
 
-template <int DK, int DV>
+template <int DK, int DV, bool ACC>
 __global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bars[5];
@@ -793,9 +826,9 @@ __global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant_
   constexpr int per_head = DK / KT + DV / VT;
   const int bh = blockIdx.x / per_head, role = blockIdx.x % per_head;
   if (role < DK / KT)
-    key_tile_body<DK, DV>(sm, mp, a, bh, role, bars, tmem);
+    key_tile_body<DK, DV, ACC>(sm, mp, a, bh, role, bars, tmem);
   else
-    val_tile_body<DK>(sm, mp, a, bh, role - DK / KT, DV, bars, tmem);
+    val_tile_body<DK, ACC>(sm, mp, a, bh, role - DK / KT, DV, bars, tmem);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -816,7 +849,8 @@ size_t bwd_workspace(int BH, int T, int dk, int) {
 template <int DK, int DV>
 static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* g, const float* h0,
                               const void* dO, const float* dhT, void* dq, void* dk, void* dv, void* dg, float* dh0,
-                              int BH, int T, void* ws, cudaStream_t st) {
+                              int BH, int T, void* ws, cudaStream_t st, long long st_bh, long long st_row,
+                              const BwdAccum* acc) {
   BwdMaps mp;
   if (!make_map(&mp.v, v, BH, T, DV, 64, true) || !make_map(&mp.dO, dO, BH, T, DV, 64, true) ||
       !make_map(&mp.k64, k, BH, T, DK, KT, true) || !make_map(&mp.g64, g, BH, T, DK, KT, true) ||
@@ -833,27 +867,52 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
   a.dg = static_cast<__nv_bfloat16*>(dg);
   a.dh0 = dh0;
   a.T = T;
+  a.st_bh = st_bh;
+  a.st_row = st_row;
+  a.acc_q = acc ? acc->q : nullptr;
+  a.acc_k = acc ? acc->k : nullptr;
+  a.acc_g = acc ? acc->g : nullptr;
+  a.acc_v = acc ? acc->v : nullptr;
+  a.acc_pk = acc ? acc->pk : 0;
+  a.acc_ck = acc ? acc->ck : 0;
+  a.acc_pv = acc ? acc->pv : 0;
+  a.acc_cv = acc ? acc->cv : 0;
   a.n_key_ctas = BH * (DK / KT);
   a.ws_qx = static_cast<float*>(ws);
   a.ws_part = a.ws_qx + align256((size_t)BH * ((T + C - 1) / C) * DK * sizeof(float)) / sizeof(float);
   a.latch = device_error_latch();
-  auto kern = bwd_fused_kernel<DK, DV>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<DK, DV>::ALLOC);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
   const int grid = BH * (DK / KT + DV / VT);
-  kern<<<grid, BT, BwdSmem<DK, DV>::ALLOC, st>>>(mp, a);
+  if (acc) {
+    auto kern = bwd_fused_kernel<DK, DV, true>;
+    static bool attr_acc = false;
+    if (!attr_acc) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<DK, DV>::ALLOC);
+      if (e != cudaSuccess) return e;
+      attr_acc = true;
+    }
+    kern<<<grid, BT, BwdSmem<DK, DV>::ALLOC, st>>>(mp, a);
+  } else {
+    auto kern = bwd_fused_kernel<DK, DV, false>;
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<DK, DV>::ALLOC);
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    kern<<<grid, BT, BwdSmem<DK, DV>::ALLOC, st>>>(mp, a);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t bwd(const void* q, const void* k, const void* v, const void* g, const float* h0, const void* dO,
                 const float* dhT, void* dq, void* dk, void* dv, void* dg, float* dh0, int BH, int T, int dkd, int dvd,
-                void* ws, cudaStream_t st) {
-  if (dkd == 128 && dvd == 256) return launch_bwd<128, 256>(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, ws, st);
-  if (dkd == 128 && dvd == 128) return launch_bwd<128, 128>(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, ws, st);
+                void* ws, cudaStream_t st, long long st_bh, long long st_row, const BwdAccum* acc) {
+  if (st_bh < 0) st_bh = (long long)dkd * dvd;
+  if (st_row < 0) st_row = dvd;
+  if (dkd == 128 && dvd == 256)
+    return launch_bwd<128, 256>(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, ws, st, st_bh, st_row, acc);
+  if (dkd == 128 && dvd == 128)
+    return launch_bwd<128, 128>(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, ws, st, st_bh, st_row, acc);
   return cudaErrorNotSupported;
 }
 

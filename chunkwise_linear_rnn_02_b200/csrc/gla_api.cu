@@ -8,6 +8,7 @@
 #include "../../include/gla.h"
 #include "common.cuh"
 #include "fast_path.cuh"
+#include "split.cuh"
 #include "generic_kernels.cuh"
 
 using gla::bf16;
@@ -68,6 +69,147 @@ struct Carve {
     return p;
   }
 };
+
+// ----------------------------------------------------------------------------------------
+// Wide bf16 shapes as sub-problems of the fused kernels
+//
+// The recurrence decays every row of S on its own, so the forward is linear in a split of the key
+// dimension: o = sum over key blocks of the output of the key block alone, and each block's hT is
+// its rows of hT.  The loss <dO, o> is a sum over value columns, so the backward is also a sum of
+// sub-problems over value blocks: dq, dk, dg of a key block sum over the value blocks, dv of a
+// value block sums over the key blocks, and dh0 / dhT are the (key, value) blocks of the state.
+// Key blocks are 128 wide; value blocks 256 (or 128) wide for the backward.  Inputs are gathered
+// into contiguous blocks, sub-results accumulate in fp32.
+// ----------------------------------------------------------------------------------------
+constexpr int kSplitK = 128;
+int split_vblock(int dv) { return dv % 256 == 0 ? 256 : 128; }
+
+bool split_fwd_ok(int BH, int T, int dk, int dv, int chunk, int dtype) {
+  if (gla::fast::fwd_supported(BH, T, dk, dv, chunk, dtype)) return false;  // served directly
+  return dk > kSplitK && dk % kSplitK == 0 && gla::fast::fwd_supported(BH, T, kSplitK, dv, chunk, dtype);
+}
+bool split_bwd_ok(int BH, int T, int dk, int dv, int chunk, int dtype) {
+  if (gla::fast::bwd_supported(BH, T, dk, dv, chunk, dtype)) return false;
+  if (dk % kSplitK != 0 || dv % 128 != 0) return false;
+  return gla::fast::bwd_supported(BH, T, kSplitK, split_vblock(dv), chunk, dtype);
+}
+
+struct SplitFwdWs {
+  bf16 *q, *k, *g;
+  float *acc, *part;
+  void* fws;
+};
+size_t carve_split_fwd(Carve& c, int BH, int T, int dk, int dv, SplitFwdWs* w) {
+  const size_t rows = (size_t)BH * T;
+  SplitFwdWs x;
+  x.q = c.take<bf16>(rows * kSplitK);
+  x.k = c.take<bf16>(rows * kSplitK);
+  x.g = c.take<bf16>(rows * kSplitK);
+  x.acc = c.take<float>(rows * dv);
+  x.part = c.take<float>(rows * dv);
+  x.fws = c.take<char>(gla::fast::fwd_workspace(BH, T, kSplitK, dv));
+  if (w) *w = x;
+  return c.used;
+}
+
+int split_fwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const float* h0, bf16* o, float* hT,
+              int BH, int T, int dk, int dv, void* ws, cudaStream_t st) {
+  Carve c(ws);
+  SplitFwdWs w;
+  carve_split_fwd(c, BH, T, dk, dv, &w);
+  const long long rows = (long long)BH * T;
+  for (int kb = 0; kb < dk / kSplitK; ++kb) {
+    const int c0 = kb * kSplitK;
+    GLA_CUDA(gla::split::gather_cols(q, w.q, rows, dk, c0, kSplitK, st));
+    GLA_CUDA(gla::split::gather_cols(k, w.k, rows, dk, c0, kSplitK, st));
+    GLA_CUDA(gla::split::gather_cols(g, w.g, rows, dk, c0, kSplitK, st));
+    GLA_CUDA(gla::fast::fwd(w.q, w.k, v, w.g, h0 ? h0 + (size_t)c0 * dv : nullptr, nullptr,
+                            hT ? hT + (size_t)c0 * dv : nullptr, BH, T, kSplitK, dv, w.fws, st, (long long)dk * dv,
+                            dv, kb == 0 ? w.acc : w.part));
+    if (kb > 0) GLA_CUDA(gla::split::add_cols(w.part, w.acc, rows, dv, dv, 0, st));
+  }
+  GLA_CUDA(gla::split::to_bf16(w.acc, o, rows * dv, st));
+  return GLA_OK;
+}
+
+struct SplitBwdWs {
+  bf16 *q, *k, *g, *v, *dO;
+  float *aq, *ak, *ag, *av;  // accumulators, full width
+  float *pq, *pk, *pg, *pv;  // one sub-problem's outputs, block width
+  void* bws;
+};
+size_t carve_split_bwd(Carve& c, int BH, int T, int dk, int dv, SplitBwdWs* w) {
+  const size_t rows = (size_t)BH * T;
+  const int vb = split_vblock(dv), nv = dv / vb;
+  SplitBwdWs x;
+  x.q = c.take<bf16>(rows * kSplitK);
+  x.k = c.take<bf16>(rows * kSplitK);
+  x.g = c.take<bf16>(rows * kSplitK);
+  x.v = nv > 1 ? c.take<bf16>(rows * dv) : nullptr;  // all value blocks, gathered once
+  x.dO = nv > 1 ? c.take<bf16>(rows * dv) : nullptr;
+  x.aq = c.take<float>(rows * dk);
+  x.ak = c.take<float>(rows * dk);
+  x.ag = c.take<float>(rows * dk);
+  x.av = c.take<float>(rows * dv);
+  x.pq = c.take<float>(rows * kSplitK);
+  x.pk = c.take<float>(rows * kSplitK);
+  x.pg = c.take<float>(rows * kSplitK);
+  x.pv = c.take<float>(rows * vb);
+  x.bws = c.take<char>(gla::fast::bwd_workspace(BH, T, kSplitK, vb));
+  if (w) *w = x;
+  return c.used;
+}
+
+int split_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const float* h0, const bf16* dO,
+              const float* dhT, bf16* dq, bf16* dk, bf16* dv, bf16* dg, float* dh0, int BH, int T, int dkd, int dvd,
+              void* ws, cudaStream_t st) {
+  Carve c(ws);
+  SplitBwdWs w;
+  carve_split_bwd(c, BH, T, dkd, dvd, &w);
+  const long long rows = (long long)BH * T;
+  const int vb = split_vblock(dvd), nv = dvd / vb, nk = dkd / kSplitK;
+  for (int vi = 0; nv > 1 && vi < nv; ++vi) {
+    GLA_CUDA(gla::split::gather_cols(v, w.v + (size_t)vi * rows * vb, rows, dvd, vi * vb, vb, st));
+    GLA_CUDA(gla::split::gather_cols(dO, w.dO + (size_t)vi * rows * vb, rows, dvd, vi * vb, vb, st));
+  }
+  for (int kb = 0; kb < nk; ++kb) {
+    const int k0 = kb * kSplitK;
+    const bf16 *qb = q, *kbp = k, *gb = g;
+    if (nk > 1) {
+      GLA_CUDA(gla::split::gather_cols(q, w.q, rows, dkd, k0, kSplitK, st));
+      GLA_CUDA(gla::split::gather_cols(k, w.k, rows, dkd, k0, kSplitK, st));
+      GLA_CUDA(gla::split::gather_cols(g, w.g, rows, dkd, k0, kSplitK, st));
+      qb = w.q;
+      kbp = w.k;
+      gb = w.g;
+    }
+    for (int vi = 0; vi < nv; ++vi) {
+      const int v0 = vi * vb;
+      const bf16* vvb = nv > 1 ? w.v + (size_t)vi * rows * vb : v;
+      const bf16* dob = nv > 1 ? w.dO + (size_t)vi * rows * vb : dO;
+      const size_t so = (size_t)k0 * dvd + v0;  // state block (k0.., v0..) of every head
+      // the first sub-problem of a block writes straight into the accumulator's columns, later ones
+      // into a block-wide buffer that is then added
+      const bool fk = vi == 0, fv = kb == 0;
+      const gla::fast::BwdAccum out{fk ? w.aq : w.pq, fk ? w.ak : w.pk, fk ? w.ag : w.pg, fv ? w.av : w.pv,
+                                    fk ? dkd : kSplitK, fk ? k0 : 0, fv ? dvd : vb, fv ? v0 : 0};
+      GLA_CUDA(gla::fast::bwd(qb, kbp, vvb, gb, h0 ? h0 + so : nullptr, dob, dhT ? dhT + so : nullptr, nullptr,
+                              nullptr, nullptr, nullptr, dh0 ? dh0 + so : nullptr, BH, T, kSplitK, vb, w.bws, st,
+                              (long long)dkd * dvd, dvd, &out));
+      if (!fk) {
+        GLA_CUDA(gla::split::add_cols(w.pq, w.aq, rows, kSplitK, dkd, k0, st));
+        GLA_CUDA(gla::split::add_cols(w.pk, w.ak, rows, kSplitK, dkd, k0, st));
+        GLA_CUDA(gla::split::add_cols(w.pg, w.ag, rows, kSplitK, dkd, k0, st));
+      }
+      if (!fv) GLA_CUDA(gla::split::add_cols(w.pv, w.av, rows, vb, dvd, v0, st));
+    }
+  }
+  GLA_CUDA(gla::split::to_bf16(w.aq, dq, rows * dkd, st));
+  GLA_CUDA(gla::split::to_bf16(w.ak, dk, rows * dkd, st));
+  GLA_CUDA(gla::split::to_bf16(w.ag, dg, rows * dkd, st));
+  GLA_CUDA(gla::split::to_bf16(w.av, dv, rows * dvd, st));
+  return GLA_OK;
+}
 
 // ----------------------------------------------------------------------------------------
 // GLA forward / backward (generic chunk-parallel passes)
@@ -267,6 +409,7 @@ size_t gla_chunk_fwd_workspace(int B, int H, int T, int dk, int dv, int chunk, i
   if (T == 0) return 0;
   if (gla::fast::fwd_supported(B * H, T, dk, dv, chunk, dtype)) return gla::fast::fwd_workspace(B * H, T, dk, dv);
   Carve c(nullptr);
+  if (split_fwd_ok(B * H, T, dk, dv, chunk, dtype)) return carve_split_fwd(c, B * H, T, dk, dv, nullptr);
   return carve_gla_fwd(c, B * H, T, dk, dv, chunk, nullptr);
 }
 
@@ -291,6 +434,9 @@ int gla_chunk_fwd(const void* q, const void* k, const void* v, const void* g, co
   if (T == 0) return copy_or_zero(hT, h0, (size_t)BH * dk * dv, st);
   if (gla::fast::fwd_supported(BH, T, dk, dv, chunk, dtype))
     return gla::fast::fwd(q, k, v, g, h0, o, hT, BH, T, dk, dv, ws, st) == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+  if (split_fwd_ok(BH, T, dk, dv, chunk, dtype))
+    return split_fwd((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)g, h0, (bf16*)o, hT, BH, T, dk, dv,
+                     ws, st);
   const gk::Shape s{BH, T, dk, dv, chunk};
   if (dtype == GLA_DTYPE_BF16)
     return gla_fwd_generic<bf16>((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)g, h0, (bf16*)o, hT,
@@ -304,6 +450,7 @@ size_t gla_chunk_bwd_workspace(int B, int H, int T, int dk, int dv, int chunk, i
   if (T == 0) return 0;
   if (gla::fast::bwd_supported(B * H, T, dk, dv, chunk, dtype)) return gla::fast::bwd_workspace(B * H, T, dk, dv);
   Carve c(nullptr);
+  if (split_bwd_ok(B * H, T, dk, dv, chunk, dtype)) return carve_split_bwd(c, B * H, T, dk, dv, nullptr);
   return carve_gla_bwd(c, B * H, T, dk, dv, chunk, nullptr);
 }
 
@@ -328,6 +475,9 @@ int gla_chunk_bwd(const void* q, const void* k, const void* v, const void* g, co
     return gla::fast::bwd(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, dkd, dvd, ws, st) == cudaSuccess
                ? GLA_OK
                : GLA_ERR_CUDA;
+  if (split_bwd_ok(BH, T, dkd, dvd, chunk, dtype))
+    return split_bwd((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)g, h0, (const bf16*)dO, dhT,
+                     (bf16*)dq, (bf16*)dk, (bf16*)dv, (bf16*)dg, dh0, BH, T, dkd, dvd, ws, st);
   const gk::Shape s{BH, T, dkd, dvd, chunk};
   if (dtype == GLA_DTYPE_BF16)
     return gla_bwd_generic<bf16>((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)g, h0,

@@ -202,3 +202,13 @@ def test_fused_forward_long_walk(dk, dv):
     inp = make_gla_inputs(1, H, 64 * 9 + 7, dk, dv, torch.bfloat16, seed=50 + dk, with_h0=True, with_do=False)
     assert gla.workspace_bytes("gla_chunk_fwd", 1, H, 64 * 9 + 7, dk, dv, 64, 1) == 0  # no split
     _run_fwd_bwd(inp, 64, check_bwd=False)
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 150, 256, 512), (1, 2, 100, 128, 384), (2, 1, 70, 384, 128)])
+def test_wide_shapes_run_as_fused_blocks(shape):
+    """bf16 shapes wider than the fused kernels run as key-block / value-block sub-problems whose
+    outputs add up (GLA is linear in a split of the key axis, its loss in a split of the value
+    axis); checked against the oracle with initial and final states."""
+    B, H, T, dk, dv = shape
+    inp = make_gla_inputs(B, H, T, dk, dv, torch.bfloat16, seed=60 + dk + dv, with_h0=True, with_dhT=True)
+    _run_fwd_bwd(inp, 64)
