@@ -9,19 +9,20 @@
 //   dk  = E2 (V G_{i+1}^T) + (E2 / dec) (dA^T Qt)
 //   dv  = Kh G_{i+1} + A^T dO
 //   G_i = dec G_{i+1} + Qt^T dO               S_{i+1} = dec S_i + Kh^T V
-//   db  = q (dq - dA_jj k) - k (dk - dA_jj q) ;  dg_t = sum_{s>=t} db_s + rowsum(dhT * hT)
-//
-// (the dA_jj terms of dq_j and dk_j cancel exactly in q dq - k dk and are left out of db).
+//   dg: chunk-local parts plus a carry across chunk boundaries (see the key tile below), so
+//       that no rounding accumulates over the sequence.
 //
 // One launch, two kinds of CTA, all resident at once:
 //   * key-tile CTAs, one per (head, 64 key dimensions): a forward walk that rebuilds S on chip
-//     and writes dq, then a reverse walk that carries G on chip and writes dk, dg and dh0 (dg
-//     needs dq, which it reads back with TMA);
+//     and writes dq and the forward part of dg (fp32, workspace), then a reverse walk that
+//     carries G on chip and writes dk, dg and dh0;
 //   * value-tile CTAs, one per (head, 128 value columns): one reverse walk carrying G[:, tile]
 //     that writes dv.
-// States live in TMEM as fp32 accumulators; their bf16 copies in shared memory feed the MMAs.
-// A chunk that keeps less than e^-40 of its state in some dimension computes its intra-chunk
-// terms exactly in fp32 (CUDA cores) instead of through the scaled operands.
+// States live in TMEM as fp32 accumulators; their bf16 hi / lo copies in shared memory feed the
+// MMAs.  A chunk that keeps less than e^-40 of its state in some dimension computes its
+// intra-chunk terms exactly in fp32 (CUDA cores) instead of through the scaled operands.  A
+// compile-time variant writes fp32 outputs into caller-provided arrays (wide shapes run as
+// blocks and add the blocks' results).
 #include "fast_path.cuh"
 #include "fused_common.cuh"
 
