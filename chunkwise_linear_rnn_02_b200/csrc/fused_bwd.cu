@@ -12,12 +12,19 @@
 //   dg: chunk-local parts plus a carry across chunk boundaries (see the key tile below), so
 //       that no rounding accumulates over the sequence.
 //
-// One launch, two kinds of CTA, all resident at once:
-//   * key-tile CTAs, one per (head, 64 key dimensions): a forward walk that rebuilds S on chip
-//     and writes dq and the forward part of dg (fp32, workspace), then a reverse walk that
-//     carries G on chip and writes dk, dg and dh0;
-//   * value-tile CTAs, one per (head, 128 value columns): one reverse walk carrying G[:, tile]
-//     that writes dv.
+// Two launches on the caller's stream:
+//   1. two kinds of CTA, all resident at once:
+//      * key-tile CTAs, one per (head, 64 key dimensions): a forward walk that rebuilds S on chip
+//        and writes dq, the forward part of dg (fp32, workspace) and the carry's start value;
+//      * value-tile CTAs, one per (head, 128 value columns): a reverse walk carrying G[:, tile]
+//        that writes dv, dh0[:, tile] and this tile's part of Z^T = G V^T for every chunk
+//        (fp32, workspace; Z sums over the value tiles);
+//      The value tiles also write, per chunk, their part of sum_r Kh_r Z_r (the chunk sums that
+//      drive the dg carry);
+//   2. a scan over chunks per (head, key dim) that turns the chunk sums into the carry c_i of
+//      every chunk;
+//   3. one CTA per (head, 64 key dimensions, chunk), all independent: dk and the rest of dg
+//      from Z^T, a recomputed dA, the forward walk's part and c_i.
 // States live in TMEM as fp32 accumulators; their bf16 hi / lo copies in shared memory feed the
 // MMAs.  A chunk that keeps less than e^-40 of its state in some dimension computes its
 // intra-chunk terms exactly in fp32 (CUDA cores) instead of through the scaled operands.  A
@@ -47,6 +54,10 @@ struct BwdArgs {
   __nv_bfloat16 *dq, *dk, *dv, *dg;
   float* dh0;
   float* ws_qx;    // [BH][NC][DK] chunk sums of Qt X
+  float* ws_carry; // [BH][DK] rowsum(dhT * hT): the start of the dg carry
+  float* ws_z;     // [BH][DV/VT][NC][DK][64] value tiles' parts of Z^T
+  float* ws_kz;    // [BH][DV/VT][NC][2][DK] value tiles' parts of the chunk sums of Kh Z (per token half)
+  float* ws_c;     // [BH][NC][DK] the dg carry c_i of every chunk
   float* ws_part;  // [BH][NC][DK][64] forward-walk part of dg, one row of 64 tokens per chunk and dim
   int T, n_key_ctas;
   long long st_bh, st_row;  // h0 / dhT / dh0 strides (a sub-block of a larger state when split)
@@ -423,137 +434,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   __syncthreads();
   tc_fence_after();
 
-  // ============================ reverse walk: dk, dg, dh0 ============================
-  if (tid == 0) {
-    load_a(NC - 1);
-    load_b(NC - 1, 0);
-    if (NC > 1) load_b(NC - 2, 1);
-  }
-  init_state(a.dhT);
-  safe_next = prepare(false, 0, 0);
-  for (int n = 0; n < NC; ++n) {
-    const int i = NC - 1 - n, b = n & 1, safe = safe_next;
-    mbar_wait(bar_m1, ph_m1, a.latch);
-    ph_m1 ^= 1;
-    tc_fence_after();
-    if (tid == 0 && n + 1 < NC) load_a(i - 1);
-    float z[32];  // this thread's row of Z^T: key dim d = row, tokens tb .. tb+31
-    tmem_ld32(tmem + L::T_X + lane_off + tb, z);
-    dA_epilogue();
-    fence_async_smem();
-    sync_tc();
-    if (!safe) issue_m2(false);
-    float pv[32];  // the forward walk's part of dg for these tokens
-    float qxn = 0.f;
-    if (row_owner) {
-      const float4* src = reinterpret_cast<const float4*>(part + ((size_t)i * DK + row) * C + tb);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float4 u = src[c];
-        pv[4 * c] = u.x;
-        pv[4 * c + 1] = u.y;
-        pv[4 * c + 2] = u.z;
-        pv[4 * c + 3] = u.w;
-      }
-      if (n > 0) qxn = qx_sums[(size_t)(i + 1) * DK + row];
-    }
-    if (n + 1 < NC)
-      safe_next = prepare(false, b ^ 1, !safe);
-    else if (!safe)
-      wait_m2();
-    float w[32];  // this thread's row of W^T
-    if (!safe) {
-      tmem_ld32(tmem + L::T_Y + lane_off + tb, w);
-      tmem_ld_wait();
-    }
-    float tot_k = 0.f, tot_s = 0.f;
-    if (row_owner) {  // dk; per-token terms Kh Z (-> z) and Kh Z + k dk^intra without j = r (-> w)
-      const int d = row;
-      const uint32_t pk = pbo(b) + L::PB_K, pg = pbo(b) + L::PB_G, pq = pbo(b) + L::PB_Q;
-      const float* tot = TOT + b * NS * KT;
-      if (safe) {  // exact intra term w_r = sum_{j>=r} dA_jr q_j e^{B_j - B_r}
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int r = tb + c;
-          float acc = dA_at(r, r) * raw(pq, r, d), bd = 0.f;
-          for (int j = r + 1; j < C; ++j) {
-            bd += raw(pg, j, d);
-            acc += dA_at(j, r) * raw(pq, j, d) * __expf(bd);
-          }
-          w[c] = acc;
-        }
-      }
-      const float inv = 1.f / DEC[b * KT + d];
-      __nv_bfloat16* dst = a.dk + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
-      float* dst32 = ACC ? a.acc_k + ((size_t)bh * T + i * C + tb) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
-#pragma unroll
-      for (int rr = 0; rr < 4; ++rr) {
-        const int h = half * 4 + rr;
-        float al[TS], e2[TS];
-#pragma unroll
-        for (int u = 0; u < TS; ++u) al[u] = ex2(raw(pg, h * TS + u, d) * kLog2e);
-        float e = 1.f;  // E2 = e^{gamma - B_r}, formed as GateRun::backward forms it
-        for (int hh = h + 1; hh < NS; ++hh) e *= tot[hh * KT + d];
-#pragma unroll
-        for (int u = TS - 1; u >= 0; --u) {
-          e2[u] = e;
-          e *= al[u];
-        }
-#pragma unroll
-        for (int u = 0; u < TS; ++u) {
-          const int c = rr * TS + u, r = tb + c;
-          const float ev = e2[u];
-          if (!safe) w[c] *= ev * inv;
-          const float qv = raw(pq, r, d), kv = raw(pk, r, d);
-          if (i * C + r < T) {
-            if (ACC)
-              dst32[(size_t)c * a.acc_pk] = ev * z[c] + w[c];
-            else
-              dst[(size_t)c * DK] = __float2bfloat16_rn(ev * z[c] + w[c]);
-          }
-          const float kz = bf_split_sum(kv * ev) * z[c];  // Kh Z, with Kh as the S update sees it
-          w[c] = kz + kv * (w[c] - DIAG[r] * qv);        // plus k dk^intra without j = r
-          tot_k += kz;
-          tot_s += w[c];
-        }
-      }
-      XCH[half * KT + d] = make_float2(tot_k, tot_s);
-    }
-    __syncthreads();
-    if (tid == 0 && n + 2 < NC) load_b(i - 2, b);
-    if (row_owner) {  // dg = c_i + prefix (exclusive) of (Kh Z + k dk^intra) + the forward walk's part
-      const int d = row;
-      const float2 o = XCH[(half ^ 1) * KT + d];
-      const float ci = CARRY[(n & 1) * KT + d] + qxn - (tot_k + o.x);
-      float pre = half == 1 ? o.y : 0.f;
-      __nv_bfloat16* dst = a.dg + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
-      float* dst32 = ACC ? a.acc_g + ((size_t)bh * T + i * C + tb) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        if (i * C + tb + c < T) {
-          if (ACC)
-            dst32[(size_t)c * a.acc_pk] = ci + pre + pv[c];
-          else
-            dst[(size_t)c * DK] = __float2bfloat16_rn(ci + pre + pv[c]);
-        }
-        pre += w[c];
-      }
-      if (half == 0) CARRY[((n + 1) & 1) * KT + d] = ci;
-    }
-  }
-  // dh0 rows = G_0
-  if (a.dh0) {
-    float v[32];
-    for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 32) {
-      tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
-      tmem_ld_wait();
-      if (row_owner) {
-        float4* dst = reinterpret_cast<float4*>(a.dh0 + bh * a.st_bh + (d0 + row) * a.st_row + c0);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-      }
-    }
-  }
+  if (tid < KT) a.ws_carry[(size_t)bh * DK + d0 + tid] = CARRY[tid];
 }
 
 // ------------------------------------------------------------------------------------------
@@ -579,7 +460,10 @@ struct ValLayout {
   static constexpr uint32_t TOT = DEC + DK * 4;
   static constexpr uint32_t TOTAL = TOT + GateRun<DK, BT>::NSPLIT * DK * 4;
   static constexpr uint32_t XB = QP_HI, XA = KH_HI;  // exact-path scratch (after the first MMA group)
-  static constexpr uint32_t T_G = 0, T_A = VT, T_DV = VT + 64;
+  // v tile [64 x VT] for Z^T = G V^T: read by the first MMA group only, so it shares A's space
+  static constexpr uint32_t VZ = AB_HI;
+  static constexpr uint32_t T_G = 0, T_A = VT, T_DV = VT + 64, T_Z = 2 * VT + 64;
+  static_assert(C * VT * 2 <= DEC - AB_HI && T_Z + 64 <= 512, "v tile / TMEM columns");
   static_assert(STAGE % 1024 == 0, "stage alignment");
   static_assert(C * DK * 4 <= KH_HI - QP_HI && C * C * 4 <= GC_HI - KH_HI, "exact-path scratch");
 };
@@ -606,12 +490,14 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   float* TOT = reinterpret_cast<float*>(sm + L::TOT);
 
   auto load = [&](int chunk) {
-    mbar_arrive_expect_tx(bar_ld, L::STAGE);
+    mbar_arrive_expect_tx(bar_ld, L::STAGE + C * VT * 2);
     tma_load_3d(sm, &mp.q_all, bar_ld, 0, chunk * C, bh);
     tma_load_3d(sm + L::RAW, &mp.k_all, bar_ld, 0, chunk * C, bh);
     tma_load_3d(sm + 2 * L::RAW, &mp.g_all, bar_ld, 0, chunk * C, bh);
-    for (int b = 0; b < VT / 64; ++b)
+    for (int b = 0; b < VT / 64; ++b) {
       tma_load_3d(sm + 3 * L::RAW + b * (C * 128), &mp.dO, bar_ld, c0 + b * 64, chunk * C, bh);
+      tma_load_3d(sm + L::VZ + b * (C * 128), &mp.v, bar_ld, c0 + b * 64, chunk * C, bh);
+    }
   };
   auto sync_tc = [&]() {
     tc_fence_before();
@@ -700,6 +586,15 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         umma_bf16(tmem + L::T_G, desc_sw128(base + L::QP_HI + k * 2048, C * 128, 1024), dd, id_G, 1);
         umma_bf16(tmem + L::T_G, desc_sw128(base + L::QP_LO + k * 2048, C * 128, 1024), dd, id_G, 1);
       }
+      // Z^T part of this value tile: G_{i+1}[:, tile] V[:, tile]^T (G copy hi + lo)
+      constexpr uint32_t id_Z = idesc_bf16_f32(DK, C, false, false);
+#pragma unroll
+      for (int k = 0; k < VT / 16; ++k) {
+        const uint32_t ko = (k >> 2) * (DK * 128) + (k & 3) * 32;
+        const uint64_t vd = desc_sw128(base + L::VZ + (k >> 2) * (C * 128) + (k & 3) * 32, 16, 1024);
+        umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_HI + ko, 16, 1024), vd, id_Z, k > 0);
+        umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_LO + ko, 16, 1024), vd, id_Z, 1);
+      }
       umma_commit(bar_m1);
     }
     __syncwarp();
@@ -707,6 +602,24 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     ph_m1 ^= 1;
     tc_fence_after();
     if (!safe) rescale_G();
+    {  // this tile's part of Z^T for chunk i: row grow of the M=128 accumulator, 32 tokens
+      float zv[32];
+      tmem_ld32(tmem + L::T_Z + lane_off + half * 32, zv);
+      tmem_ld_wait();
+      float4* dst = reinterpret_cast<float4*>(
+          a.ws_z + ((((size_t)bh * (DV / VT) + vt) * NC + i) * DK + grow) * C + half * 32);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) dst[c] = make_float4(zv[4 * c], zv[4 * c + 1], zv[4 * c + 2], zv[4 * c + 3]);
+      // this tile's part of sum_r Kh_r Z_r over the thread's 32 tokens (Kh as hi + lo)
+      const uint32_t kblk = (grow >> 6) * (C * 128), kcol = grow & 63;
+      float kz = 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const uint32_t off = kblk + sw128(half * 32 + c, kcol);
+        kz += (bf2f(sm + L::KH_HI + off) + bf2f(sm + L::KH_LO + off)) * zv[c];
+      }
+      a.ws_kz[((((size_t)bh * (DV / VT) + vt) * NC + i) * 2 + half) * DK + grow] = kz;
+    }
     float* XA = reinterpret_cast<float*>(sm + L::XA);
     if (safe) {  // exact A = sum_d q_jd k_rd e^{B_jd - B_rd}, r <= j
       float* XB = reinterpret_cast<float*>(sm + L::XB);
@@ -792,6 +705,287 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     __syncthreads();
     if (tid == 0 && n + 1 < NC) load(i - 1);
   }
+  // dh0[:, tile] = G_0
+  if (a.dh0) {
+    tc_fence_after();
+    float dv0v[32];
+    for (int cb = half * HT; cb < (half + 1) * HT; cb += 32) {
+      tmem_ld32(tmem + L::T_G + lane_off + cb, dv0v);
+      tmem_ld_wait();
+      float4* dst = reinterpret_cast<float4*>(a.dh0 + bh * a.st_bh + grow * a.st_row + c0 + cb);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) dst[c] = make_float4(dv0v[4 * c], dv0v[4 * c + 1], dv0v[4 * c + 2], dv0v[4 * c + 3]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Carry scan: per (head, key dim), c_{N-1} = rowsum(dhT * hT) - K_{N-1} and
+// c_i = c_{i+1} + Q_{i+1} - K_i, with Q the forward walk's chunk sums of Qt X and K the chunk
+// sums of Kh Z (summed over value tiles and token halves).
+// ------------------------------------------------------------------------------------------
+__global__ void carry_scan_kernel(const BwdArgs a, int BH, int DK, int NVT) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= BH * DK) return;
+  const int bh = e / DK, d = e % DK, NC = (a.T + C - 1) / C;
+  float c = a.ws_carry[e];
+  for (int i = NC - 1; i >= 0; --i) {
+    float k = 0.f;
+    for (int vt = 0; vt < NVT; ++vt)
+      for (int h = 0; h < 2; ++h) k += a.ws_kz[((((size_t)bh * NVT + vt) * NC + i) * 2 + h) * DK + d];
+    if (i < NC - 1) c += a.ws_qx[((size_t)bh * NC + i + 1) * DK + d];
+    c -= k;
+    a.ws_c[((size_t)bh * NC + i) * DK + d] = c;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Third launch: one CTA per (head, 64 key dimensions, chunk).  Gate run of the key slab (Qt, E2,
+// decays), dA = dO V^T recomputed, W^T = Qt^T dA, and the epilogue
+//   dk = E2 Z + (E2 / dec) W,   dg = c_i + prefix(Kh Z + k dk^intra) + the forward walk's part,
+// with Z^T summed over the value tiles' parts.  No state: every chunk is independent.
+// ------------------------------------------------------------------------------------------
+template <int DK, int DV>
+struct ChunkLayout {
+  static constexpr uint32_t VB = C * DV * 2;        // a v or dO tile [64 x DV]
+  static constexpr uint32_t TILE = C * KT * 2;      // a [64 x 64] bf16 tile
+  static constexpr uint32_t PA_V = 0, PA_DO = VB;
+  static constexpr uint32_t PB = 2 * VB;            // k, g, q tiles
+  static constexpr uint32_t PB_K = PB, PB_G = PB + TILE, PB_Q = PB + 2 * TILE;
+  static constexpr uint32_t KQ_HI = PB + 3 * TILE;  // Qt hi / lo
+  static constexpr uint32_t KQ_LO = KQ_HI + TILE;
+  static constexpr uint32_t DA_HI = PA_V;           // masked dA hi / lo: v is dead once dA is formed
+  static constexpr uint32_t DA_LO = DA_HI + TILE;
+  static constexpr int NS = GateRun<KT, BT>::NSPLIT;
+  static constexpr uint32_t XCH = KQ_LO + TILE;
+  static constexpr uint32_t DEC = XCH + 2 * KT * 8;
+  static constexpr uint32_t TOT = DEC + KT * 4;
+  static constexpr uint32_t DIAG = TOT + NS * KT * 4;
+  static constexpr uint32_t TOTAL = DIAG + C * 4;
+  static constexpr uint32_t T_DA = 0, T_Y = 64;  // TMEM columns (128 allocated)
+  static_assert(PB % 1024 == 0 && KQ_HI % 1024 == 0 && 2 * TILE <= VB, "operand layout");
+};
+
+template <int DK, int DV, bool ACC>
+__global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
+  using L = ChunkLayout<DK, DV>;
+  using Gate = GateRun<KT, BT>;
+  constexpr int NS = L::NS, TS = Gate::TS, NVT = DV / VT;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_ld, bar_m1, bar_m2;
+  __shared__ uint32_t tmem_base_sh;
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  const uint32_t base = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3, half = warp >> 2;
+  const int T = a.T, NC = (T + C - 1) / C;
+  const int i = blockIdx.x % NC, slab = blockIdx.x / NC;
+  const int tau = slab % (DK / KT), bh = slab / (DK / KT), d0 = tau * KT;
+  const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+  const bool row_owner = lane < 16;
+  const int row = q4 * 16 + lane;
+  const int tb = half * 32;
+  float* DEC = reinterpret_cast<float*>(sm + L::DEC);
+  float* TOT = reinterpret_cast<float*>(sm + L::TOT);
+  float2* XCH = reinterpret_cast<float2*>(sm + L::XCH);
+  float* DIAG = reinterpret_cast<float*>(sm + L::DIAG);
+
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, 128);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bar_ld, 1);
+    mbar_init(&bar_m1, 1);
+    mbar_init(&bar_m2, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bar_ld, 2 * L::VB + 3 * L::TILE);
+    for (int bb = 0; bb < DV / 64; ++bb) {
+      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, &bar_ld, bb * 64, i * C, bh);
+      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, &bar_ld, bb * 64, i * C, bh);
+    }
+    tma_load_3d(sm + L::PB_K, &mp.k64, &bar_ld, d0, i * C, bh);
+    tma_load_3d(sm + L::PB_G, &mp.g64, &bar_ld, d0, i * C, bh);
+    tma_load_3d(sm + L::PB_Q, &mp.q64, &bar_ld, d0, i * C, bh);
+  }
+  // global inputs of the epilogue, loaded while the tiles arrive
+  float pv[32], z[32];
+  float ci = 0.f;
+  if (row_owner) {
+    const float4* src = reinterpret_cast<const float4*>(a.ws_part + (((size_t)bh * NC + i) * DK + d0 + row) * C + tb);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 u = src[c];
+      pv[4 * c] = u.x;
+      pv[4 * c + 1] = u.y;
+      pv[4 * c + 2] = u.z;
+      pv[4 * c + 3] = u.w;
+    }
+    ci = a.ws_c[((size_t)bh * NC + i) * DK + d0 + row];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) z[c] = 0.f;
+    for (int vt = 0; vt < NVT; ++vt) {
+      const float4* zs = reinterpret_cast<const float4*>(
+          a.ws_z + ((((size_t)bh * NVT + vt) * NC + i) * DK + d0 + row) * C + tb);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float4 u = zs[c];
+        z[4 * c] += u.x;
+        z[4 * c + 1] += u.y;
+        z[4 * c + 2] += u.z;
+        z[4 * c + 3] += u.w;
+      }
+    }
+  }
+  auto raw = [&](uint32_t off, int j, int d) { return bf2f(sm + off + sw128(j, d)); };
+  auto raw2 = [&](uint32_t off, int j, int d) { return *reinterpret_cast<const uint32_t*>(sm + off + sw128(j, d)); };
+  auto dA_at = [&](int j, int r) { return raw(L::DA_HI, j, r) + raw(L::DA_LO, j, r); };
+
+  mbar_wait(&bar_ld, 0, a.latch);
+  if (tid == 0) {  // dA = dO V^T (operands as loaded)
+    tc_fence_after();
+    constexpr uint32_t id_dA = idesc_bf16_f32(C, C, false, false);
+#pragma unroll
+    for (int k = 0; k < DV / 16; ++k) {
+      const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
+      umma_bf16(tmem + L::T_DA, desc_sw128(base + L::PA_DO + ko, 16, 1024), desc_sw128(base + L::PA_V + ko, 16, 1024),
+                id_dA, k > 0);
+    }
+    umma_commit(&bar_m1);
+  }
+  // gate run of the key slab: Qt hi / lo, decays, run products
+  Gate gr;
+  const bool weak = gr.run_swizzled(sm + L::PB_G, TOT);
+  if (gr.h == 0) {
+    DEC[gr.d] = gr.dec0;
+    DEC[gr.d + 1] = gr.dec1;
+  }
+  const int safe = __syncthreads_or(weak);
+  gr.forward([&](int j, float e0, float e1) {
+    const uint32_t w = raw2(L::PB_Q, j, gr.d);
+    uint32_t hi, lo;
+    split2(bf_lo(w) * e0, bf_hi(w) * e1, hi, lo);
+    *reinterpret_cast<uint32_t*>(sm + L::KQ_HI + sw128(j, gr.d)) = hi;
+    *reinterpret_cast<uint32_t*>(sm + L::KQ_LO + sw128(j, gr.d)) = lo;
+  });
+  __syncwarp();
+  mbar_wait(&bar_m1, 0, a.latch);
+  tc_fence_after();
+  {  // dA epilogue: masked hi / lo operand (over the dead v tile) and its diagonal
+    float v[32];
+    tmem_ld32(tmem + L::T_DA + lane_off + tb, v);
+    tmem_ld_wait();
+    if (row_owner) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        if (tb + c > row) v[c] = 0.f;
+        if (tb + c == row) DIAG[row] = v[c];
+      }
+      store_half_split(sm + L::DA_HI, sm + L::DA_LO, row, v, half);
+    }
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0 && !safe) {  // W^T = Qt^T dA
+    constexpr uint32_t id_W = idesc_bf16_f32(KT, C, true, true);
+#pragma unroll
+    for (int k = 0; k < C / 16; ++k) {
+      const uint64_t ah = desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024);
+      const uint64_t bh2 = desc_sw128(base + L::DA_HI + k * 2048, C * 128, 1024);
+      umma_bf16(tmem + L::T_Y, ah, bh2, id_W, k > 0);
+      umma_bf16(tmem + L::T_Y, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), bh2, id_W, 1);
+      umma_bf16(tmem + L::T_Y, ah, desc_sw128(base + L::DA_LO + k * 2048, C * 128, 1024), id_W, 1);
+    }
+    umma_commit(&bar_m2);
+  }
+  float w[32];
+  if (!safe) {
+    __syncwarp();
+    mbar_wait(&bar_m2, 0, a.latch);
+    tc_fence_after();
+    tmem_ld32(tmem + L::T_Y + lane_off + tb, w);
+    tmem_ld_wait();
+  }
+  float tot_k = 0.f, tot_s = 0.f;
+  if (row_owner) {  // dk; per-token terms Kh Z and Kh Z + k dk^intra without j = r (-> w)
+    const int d = row;
+    if (safe) {  // exact intra term w_r = sum_{j>=r} dA_jr q_j e^{B_j - B_r}
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const int r = tb + c;
+        float acc = dA_at(r, r) * raw(L::PB_Q, r, d), bd = 0.f;
+        for (int j = r + 1; j < C; ++j) {
+          bd += raw(L::PB_G, j, d);
+          acc += dA_at(j, r) * raw(L::PB_Q, j, d) * __expf(bd);
+        }
+        w[c] = acc;
+      }
+    }
+    const float inv = 1.f / DEC[d];
+    __nv_bfloat16* dst = a.dk + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
+    float* dst32 = ACC ? a.acc_k + ((size_t)bh * T + i * C + tb) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      const int h = half * 4 + rr;
+      float al[TS], e2[TS];
+#pragma unroll
+      for (int u = 0; u < TS; ++u) al[u] = ex2(raw(L::PB_G, h * TS + u, d) * kLog2e);
+      float e = 1.f;  // E2 = e^{gamma - B_r}, formed as GateRun::backward forms it
+      for (int hh = h + 1; hh < NS; ++hh) e *= TOT[hh * KT + d];
+#pragma unroll
+      for (int u = TS - 1; u >= 0; --u) {
+        e2[u] = e;
+        e *= al[u];
+      }
+#pragma unroll
+      for (int u = 0; u < TS; ++u) {
+        const int c = rr * TS + u, r = tb + c;
+        const float ev = e2[u];
+        if (!safe) w[c] *= ev * inv;
+        const float qv = raw(L::PB_Q, r, d), kv = raw(L::PB_K, r, d);
+        if (i * C + r < T) {
+          if (ACC)
+            dst32[(size_t)c * a.acc_pk] = ev * z[c] + w[c];
+          else
+            dst[(size_t)c * DK] = __float2bfloat16_rn(ev * z[c] + w[c]);
+        }
+        const float kz = bf_split_sum(kv * ev) * z[c];  // Kh Z, with Kh as the S update sees it
+        w[c] = kz + kv * (w[c] - DIAG[r] * qv);        // plus k dk^intra without j = r
+        tot_s += w[c];
+      }
+    }
+    XCH[half * KT + d] = make_float2(tot_k, tot_s);
+  }
+  __syncthreads();
+  if (row_owner) {  // dg = c_i + prefix (exclusive) of (Kh Z + k dk^intra) + the forward walk's part
+    const int d = row;
+    const float2 o = XCH[(half ^ 1) * KT + d];
+    float pre = half == 1 ? o.y : 0.f;
+    __nv_bfloat16* dst = a.dg + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
+    float* dst32 = ACC ? a.acc_g + ((size_t)bh * T + i * C + tb) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      if (i * C + tb + c < T) {
+        if (ACC)
+          dst32[(size_t)c * a.acc_pk] = ci + pre + pv[c];
+        else
+          dst[(size_t)c * DK] = __float2bfloat16_rn(ci + pre + pv[c]);
+      }
+      pre += w[c];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -835,6 +1029,30 @@ __global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant_
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+template <int DK, int DV, bool ACC>
+static cudaError_t launch_all(const BwdMaps& mp, const BwdArgs& a, int BH, cudaStream_t st) {
+  constexpr uint32_t CHK = ChunkLayout<DK, DV>::TOTAL + 1024;
+  static_assert(2 * CHK <= 228 * 1024, "two chunk CTAs per SM");
+  auto k1 = bwd_fused_kernel<DK, DV, ACC>;
+  auto k3 = bwd_chunk_kernel<DK, DV, ACC>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<DK, DV>::ALLOC);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, CHK);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  k1<<<BH * (DK / KT + DV / VT), BT, BwdSmem<DK, DV>::ALLOC, st>>>(mp, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  carry_scan_kernel<<<(BH * DK + 127) / 128, 128, 0, st>>>(a, BH, DK, DV / VT);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int NC = (a.T + C - 1) / C;
+  k3<<<BH * (DK / KT) * NC, BT, CHK, st>>>(mp, a);
+  return cudaGetLastError();
+}
+
 bool bwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype) {
   if (force_generic()) return false;
   if (dtype != 1 || chunk != C || T < 1 || BH < 1) return false;
@@ -842,9 +1060,11 @@ bool bwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype) {
   return encode_fn() != nullptr;
 }
 
-size_t bwd_workspace(int BH, int T, int dk, int) {
+size_t bwd_workspace(int BH, int T, int dk, int dv) {
   const size_t NC = (T + C - 1) / C;
-  return align256((size_t)BH * NC * dk * sizeof(float)) + align256((size_t)BH * NC * C * dk * sizeof(float));
+  return align256((size_t)BH * NC * dk * sizeof(float)) + align256((size_t)BH * NC * C * dk * sizeof(float)) +
+         align256((size_t)BH * dk * sizeof(float)) + align256((size_t)BH * (dv / VT) * NC * dk * C * sizeof(float)) +
+         align256((size_t)BH * (dv / VT) * NC * 2 * dk * sizeof(float)) + align256((size_t)BH * NC * dk * sizeof(float));
 }
 
 template <int DK, int DV>
@@ -879,30 +1099,15 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
   a.acc_pv = acc ? acc->pv : 0;
   a.acc_cv = acc ? acc->cv : 0;
   a.n_key_ctas = BH * (DK / KT);
+  const size_t NC = (T + C - 1) / C;
   a.ws_qx = static_cast<float*>(ws);
-  a.ws_part = a.ws_qx + align256((size_t)BH * ((T + C - 1) / C) * DK * sizeof(float)) / sizeof(float);
+  a.ws_part = a.ws_qx + align256((size_t)BH * NC * DK * sizeof(float)) / sizeof(float);
+  a.ws_carry = a.ws_part + align256((size_t)BH * NC * C * DK * sizeof(float)) / sizeof(float);
+  a.ws_z = a.ws_carry + align256((size_t)BH * DK * sizeof(float)) / sizeof(float);
+  a.ws_kz = a.ws_z + align256((size_t)BH * (DV / VT) * NC * DK * C * sizeof(float)) / sizeof(float);
+  a.ws_c = a.ws_kz + align256((size_t)BH * (DV / VT) * NC * 2 * DK * sizeof(float)) / sizeof(float);
   a.latch = device_error_latch();
-  const int grid = BH * (DK / KT + DV / VT);
-  if (acc) {
-    auto kern = bwd_fused_kernel<DK, DV, true>;
-    static bool attr_acc = false;
-    if (!attr_acc) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<DK, DV>::ALLOC);
-      if (e != cudaSuccess) return e;
-      attr_acc = true;
-    }
-    kern<<<grid, BT, BwdSmem<DK, DV>::ALLOC, st>>>(mp, a);
-  } else {
-    auto kern = bwd_fused_kernel<DK, DV, false>;
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<DK, DV>::ALLOC);
-      if (e != cudaSuccess) return e;
-      attr_set = true;
-    }
-    kern<<<grid, BT, BwdSmem<DK, DV>::ALLOC, st>>>(mp, a);
-  }
-  return cudaGetLastError();
+  return acc ? launch_all<DK, DV, true>(mp, a, BH, st) : launch_all<DK, DV, false>(mp, a, BH, st);
 }
 
 cudaError_t bwd(const void* q, const void* k, const void* v, const void* g, const float* h0, const void* dO,

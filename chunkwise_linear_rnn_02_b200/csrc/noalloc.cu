@@ -23,7 +23,7 @@
 
 namespace {
 
-constexpr size_t kScratchBytes = size_t(64) << 20;  // 64 MiB
+constexpr size_t kScratchBytes = size_t(128) << 20;  // 128 MiB
 __device__ __align__(256) unsigned char g_bwd_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;

@@ -162,15 +162,15 @@ int gsa_recurrent_step(const void* q, const void* k, const void* v, const void* 
  * plain C host without a device allocator, a runtime that has carved up device memory in advance
  * and hands it out only for tensors, or code that must not call cudaMalloc because that call may
  * synchronise the device while its work is in flight.
- * What it uses instead: a fixed 64 MiB scratch array compiled into the library, reserved on every
- * device that loads this part of the library and held until the process exits.  The first call on
- * a device looks up that array's device address (cudaGetSymbolAddress); make the first call on each
- * device before any stream capture.  All calls share the array: calls that overlap on the GPU
- * (different streams or host threads) race on it.  Nothing in it needs to start at zero.
+ * What it uses instead: a fixed 128 MiB scratch array compiled into the library, reserved on
+ * every device that loads this part of the library and held until the process exits.  The first
+ * call on a device looks up that array's device address (cudaGetSymbolAddress); make the first
+ * call on each device before any stream capture.  All calls share the array: calls that overlap
+ * on the GPU (different streams or host threads) race on it.  Nothing in it needs to start at zero.
  * Arguments, layouts and outputs are those of gla_chunk_bwd.  Supported: bf16, chunk 64,
  * d_k = 128, d_v in {128, 256}, T >= 1 (else GLA_ERR_UNSUPPORTED / GLA_ERR_INVALID_ARG), and
- * 65*B*H*ceil(T/64)*d_k*4 bytes of scratch (two parts, each rounded up to 256 bytes) within
- * the 64 MiB (else GLA_ERR_WORKSPACE).
+ * (66 + d_v/2 + d_v/64)*B*H*ceil(T/64)*d_k*4 + B*H*d_k*4 bytes of scratch (six parts, each
+ * rounded up to 256 bytes) within the 128 MiB (else GLA_ERR_WORKSPACE).
  * It allocates nothing.
  * ------------------------------------------------------------------------------------- */
 int gla_chunk_bwd_noalloc(const void* q, const void* k, const void* v, const void* g, const float* h0,
