@@ -157,8 +157,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     {
       const uint32_t blk = (gr.d >> 6) * (C * 128), col = gr.d & 63;
+      uint32_t w[Gate::TS];
+      gr.load_pairs(st, DK, false, w);
       gr.backward([&](int j, float e0, float e1) {
-        const uint32_t wk = *reinterpret_cast<const uint32_t*>(st + (j * DK + gr.d) * 2);
+        const uint32_t wk = w[j - gr.h * Gate::TS];
         *reinterpret_cast<uint32_t*>(sm + L::KH + blk + sw128(j, col)) = pack2(bf_lo(wk) * e0, bf_hi(wk) * e1);
       });
     }

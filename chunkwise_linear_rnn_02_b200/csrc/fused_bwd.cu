@@ -191,8 +191,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     }
     return __syncthreads_or(weak);
   };
-  auto write_kq = [&](uint32_t off, int j, int d, float e0, float e1) {
-    const uint32_t w = raw2(off, j, d);
+  auto write_kq = [&](uint32_t w, int j, int d, float e0, float e1) {
     uint32_t hi, lo;
     split2(bf_lo(w) * e0, bf_hi(w) * e1, hi, lo);
     *reinterpret_cast<uint32_t*>(sm + L::KQ_HI + sw128(j, d)) = hi;
@@ -301,12 +300,13 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     wait_b(nb);
     Gate gr;
     const int safe = gate(gr, nb);
+    uint32_t w[Gate::TS];
+    gr.load_pairs(sm + pbo(nb) + (fwd ? L::PB_K : L::PB_Q), KT, true, w);
     if (m2_pending) wait_m2();
-    const uint32_t off = pbo(nb) + (fwd ? L::PB_K : L::PB_Q);
     if (fwd)
-      gr.backward([&](int j, float e0, float e1) { write_kq(off, j, gr.d, e0, e1); });
+      gr.backward([&](int j, float e0, float e1) { write_kq(w[j - gr.h * Gate::TS], j, gr.d, e0, e1); });
     else
-      gr.forward([&](int j, float e0, float e1) { write_kq(off, j, gr.d, e0, e1); });
+      gr.forward([&](int j, float e0, float e1) { write_kq(w[j - gr.h * Gate::TS], j, gr.d, e0, e1); });
     state_pass(nb);
     fence_async_smem();
     sync_tc();
@@ -482,21 +482,27 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   const int row = q4 * 16 + lane;   // row of an M=64 accumulator
   const int grow = q4 * 32 + lane;  // row of the M=128 G accumulator
   constexpr int HT = VT / 2;        // G / dv columns per warp
-  uint64_t* bar_ld = bars + 0;
+  uint64_t* bar_ld = bars + 0;  // q, k, g of a chunk
+  uint64_t* bar_dv = bars + 1;  // dO, v of a chunk
   uint64_t* bar_m1 = bars + 3;
   uint64_t* bar_m2 = bars + 4;
-  uint32_t ph_ld = 0, ph_m1 = 0, ph_m2 = 0;
+  uint32_t ph_ld = 0, ph_dv = 0, ph_m1 = 0, ph_m2 = 0;
   float* DEC = reinterpret_cast<float*>(sm + L::DEC);
   float* TOT = reinterpret_cast<float*>(sm + L::TOT);
 
-  auto load = [&](int chunk) {
-    mbar_arrive_expect_tx(bar_ld, L::STAGE + C * VT * 2);
+  // q, k, g are read only by the gate run (and the exact path), so the next chunk's copies are
+  // issued as soon as those reads are done; dO and v once the second MMA group has completed.
+  auto load_qkg = [&](int chunk) {
+    mbar_arrive_expect_tx(bar_ld, 3 * L::RAW);
     tma_load_3d(sm, &mp.q_all, bar_ld, 0, chunk * C, bh);
     tma_load_3d(sm + L::RAW, &mp.k_all, bar_ld, 0, chunk * C, bh);
     tma_load_3d(sm + 2 * L::RAW, &mp.g_all, bar_ld, 0, chunk * C, bh);
+  };
+  auto load_dov = [&](int chunk) {
+    mbar_arrive_expect_tx(bar_dv, L::DOT + C * VT * 2);
     for (int b = 0; b < VT / 64; ++b) {
-      tma_load_3d(sm + 3 * L::RAW + b * (C * 128), &mp.dO, bar_ld, c0 + b * 64, chunk * C, bh);
-      tma_load_3d(sm + L::VZ + b * (C * 128), &mp.v, bar_ld, c0 + b * 64, chunk * C, bh);
+      tma_load_3d(sm + 3 * L::RAW + b * (C * 128), &mp.dO, bar_dv, c0 + b * 64, chunk * C, bh);
+      tma_load_3d(sm + L::VZ + b * (C * 128), &mp.v, bar_dv, c0 + b * 64, chunk * C, bh);
     }
   };
   auto sync_tc = [&]() {
@@ -529,7 +535,10 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     }
     tmem_st_wait();
   }
-  if (tid == 0) load(NC - 1);
+  if (tid == 0) {
+    load_qkg(NC - 1);
+    load_dov(NC - 1);
+  }
   for (int n = 0; n < NC; ++n) {
     const int i = NC - 1 - n;
     mbar_wait(bar_ld, ph_ld, a.latch);
@@ -544,15 +553,18 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     {
       const float inv0 = safe ? 1.f : 1.f / gr.dec0, inv1 = safe ? 1.f : 1.f / gr.dec1;
       const uint32_t blk = (gr.d >> 6) * (C * 128), col = gr.d & 63;
+      uint32_t w[Gate::TS];
+      gr.load_pairs(sm, DK, false, w);
       gr.forward([&](int j, float e0, float e1) {
-        const uint32_t wq = *reinterpret_cast<const uint32_t*>(sm + (j * DK + gr.d) * 2);
+        const uint32_t wq = w[j - gr.h * Gate::TS];
         uint32_t hi, lo;
         split2(bf_lo(wq) * e0 * inv0, bf_hi(wq) * e1 * inv1, hi, lo);
         *reinterpret_cast<uint32_t*>(sm + L::QP_HI + blk + sw128(j, col)) = hi;
         *reinterpret_cast<uint32_t*>(sm + L::QP_LO + blk + sw128(j, col)) = lo;
       });
+      gr.load_pairs(sm + L::RAW, DK, false, w);
       gr.backward([&](int j, float e0, float e1) {
-        const uint32_t wk = *reinterpret_cast<const uint32_t*>(sm + L::RAW + (j * DK + gr.d) * 2);
+        const uint32_t wk = w[j - gr.h * Gate::TS];
         uint32_t hi, lo;
         split2(bf_lo(wk) * e0, bf_hi(wk) * e1, hi, lo);
         *reinterpret_cast<uint32_t*>(sm + L::KH_HI + blk + sw128(j, col)) = hi;
@@ -560,6 +572,8 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       });
     }
     if (safe) rescale_G();
+    mbar_wait(bar_dv, ph_dv, a.latch);
+    ph_dv ^= 1;
     fence_async_smem();
     sync_tc();
     if (tid == 0) {
@@ -596,12 +610,12 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_LO + ko, 16, 1024), vd, id_Z, 1);
       }
       umma_commit(bar_m1);
+      if (!safe && n + 1 < NC) load_qkg(i - 1);
     }
     __syncwarp();
     mbar_wait(bar_m1, ph_m1, a.latch);
     ph_m1 ^= 1;
     tc_fence_after();
-    if (!safe) rescale_G();
     {  // this tile's part of Z^T for chunk i: row grow of the M=128 accumulator, 32 tokens
       float zv[32];
       tmem_ld32(tmem + L::T_Z + lane_off + half * 32, zv);
@@ -657,18 +671,27 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         store_half_split(sm + L::AB_HI, sm + L::AB_LO, row, v, half);
       }
     }
-    {  // hi / lo copy of G_i for the next (earlier) chunk
+    {  // G_i = dec * G (chunks off the exact path, whose rescale came first) and its hi / lo copy
+      const float sc = safe ? 1.f : DEC[grow];
       float v[64];
       for (int cb = half * HT; cb < (half + 1) * HT; cb += 64) {
         tmem_ld32(tmem + L::T_G + lane_off + cb, v);
         tmem_ld32(tmem + L::T_G + lane_off + cb + 32, v + 32);
         tmem_ld_wait();
+        if (!safe) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) v[c] *= sc;
+          tmem_st32(tmem + L::T_G + lane_off + cb, v);
+          tmem_st32(tmem + L::T_G + lane_off + cb + 32, v + 32);
+        }
         store_row_split(sm + L::GC_HI + (cb / 64) * (DK * 128), sm + L::GC_LO + (cb / 64) * (DK * 128), grow, v, 1.f);
       }
+      tmem_st_wait();
     }
     fence_async_smem();
     sync_tc();
     if (tid == 0) {
+      if (safe && n + 1 < NC) load_qkg(i - 1);
       const uint32_t dob = base + 3 * L::RAW;
       constexpr uint32_t id_dv2 = idesc_bf16_f32(C, VT, true, true);
 #pragma unroll
@@ -683,6 +706,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     mbar_wait(bar_m2, ph_m2, a.latch);
     ph_m2 ^= 1;
     tc_fence_after();
+    if (tid == 0 && n + 1 < NC) load_dov(i - 1);  // dO and A (over v) are no longer read
     {  // dv epilogue
       float v[64];
       const int t = i * C + row;
@@ -703,7 +727,6 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     }
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && n + 1 < NC) load(i - 1);
   }
   // dh0[:, tile] = G_0
   if (a.dh0) {
@@ -724,19 +747,36 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
 // c_i = c_{i+1} + Q_{i+1} - K_i, with Q the forward walk's chunk sums of Qt X and K the chunk
 // sums of Kh Z (summed over value tiles and token halves).
 // ------------------------------------------------------------------------------------------
-__global__ void carry_scan_kernel(const BwdArgs a, int BH, int DK, int NVT) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= BH * DK) return;
-  const int bh = e / DK, d = e % DK, NC = (a.T + C - 1) / C;
-  float c = a.ws_carry[e];
-  for (int i = NC - 1; i >= 0; --i) {
-    float k = 0.f;
-    for (int vt = 0; vt < NVT; ++vt)
-      for (int h = 0; h < 2; ++h) k += a.ws_kz[((((size_t)bh * NVT + vt) * NC + i) * 2 + h) * DK + d];
-    if (i < NC - 1) c += a.ws_qx[((size_t)bh * NC + i + 1) * DK + d];
-    c -= k;
-    a.ws_c[((size_t)bh * NC + i) * DK + d] = c;
-  }
+// One block per (head, 32 key dims); its 8 warps each take a slice of the chunks: the slice sums
+// are exchanged in shared memory, then every warp walks its own slice from the right start.
+template <int NVT>
+__global__ void __launch_bounds__(256) carry_scan_kernel(const float* __restrict__ carry, const float* __restrict__ qx,
+                                                         const float* __restrict__ kz, float* __restrict__ cout,
+                                                         int DK, int NC) {
+  __shared__ float slice_sum[8][32];
+  const int dl = threadIdx.x & 31, s = threadIdx.x >> 5;
+  const int bh = blockIdx.x / (DK / 32), d = (blockIdx.x % (DK / 32)) * 32 + dl;
+  const int G = (NC + 7) / 8, top = NC - 1 - s * G;  // slice s: chunks top, top - 1, ..., top - G + 1
+  // change of the carry from chunk i + 1 to chunk i
+  auto delta = [&](int i) {
+    float v = i < NC - 1 ? qx[((size_t)bh * NC + i + 1) * DK + d] : 0.f;
+#pragma unroll
+    for (int h = 0; h < 2 * NVT; ++h) v -= kz[(((size_t)bh * NVT * NC + (h >> 1) * NC + i) * 2 + (h & 1)) * DK + d];
+    return v;
+  };
+  float sum = 0.f;
+#pragma unroll 4
+  for (int u = 0; u < G; ++u)
+    if (top - u >= 0) sum += delta(top - u);
+  slice_sum[s][dl] = sum;
+  __syncthreads();
+  float c = carry[(size_t)bh * DK + d];
+  for (int t = 0; t < s; ++t) c += slice_sum[t][dl];
+  for (int u = 0; u < G; ++u)
+    if (top - u >= 0) {
+      c += delta(top - u);
+      cout[((size_t)bh * NC + top - u) * DK + d] = c;
+    }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -868,8 +908,10 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
     DEC[gr.d + 1] = gr.dec1;
   }
   const int safe = __syncthreads_or(weak);
+  uint32_t wq[Gate::TS];
+  gr.load_pairs(sm + L::PB_Q, KT, true, wq);
   gr.forward([&](int j, float e0, float e1) {
-    const uint32_t w = raw2(L::PB_Q, j, gr.d);
+    const uint32_t w = wq[j - gr.h * Gate::TS];
     uint32_t hi, lo;
     split2(bf_lo(w) * e0, bf_hi(w) * e1, hi, lo);
     *reinterpret_cast<uint32_t*>(sm + L::KQ_HI + sw128(j, gr.d)) = hi;
@@ -1045,10 +1087,10 @@ static cudaError_t launch_all(const BwdMaps& mp, const BwdArgs& a, int BH, cudaS
   k1<<<BH * (DK / KT + DV / VT), BT, BwdSmem<DK, DV>::ALLOC, st>>>(mp, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  carry_scan_kernel<<<(BH * DK + 127) / 128, 128, 0, st>>>(a, BH, DK, DV / VT);
+  const int NC = (a.T + C - 1) / C;
+  carry_scan_kernel<DV / VT><<<BH * (DK / 32), 256, 0, st>>>(a.ws_carry, a.ws_qx, a.ws_kz, a.ws_c, DK, NC);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int NC = (a.T + C - 1) / C;
   k3<<<BH * (DK / KT) * NC, BT, CHK, st>>>(mp, a);
   return cudaGetLastError();
 }

@@ -239,6 +239,17 @@ struct GateRun {
     return !(dec0 >= kMinDecay && dec1 >= kMinDecay);
   }
 
+  // The thread's pair of bf16 values for every token of its run, from a [64][ND] tile (row stride
+  // `stride` elements, or the 128-byte swizzle), all loaded before any is used: the loops that
+  // consume them store to shared memory, and a load cannot move above such a store.
+  __device__ __forceinline__ void load_pairs(const uint8_t* src, int stride, bool swz, uint32_t (&w)[TS]) const {
+#pragma unroll
+    for (int u = 0; u < TS; ++u) {
+      const int j = h * TS + u;
+      w[u] = *reinterpret_cast<const uint32_t*>(src + (swz ? sm100::sw128(j, d) : (j * stride + d) * 2));
+    }
+  }
+
   // For each token j of the run: f(j, E1_0, E1_1) with E1 = e^{B_j} (inclusive products).
   template <typename F>
   __device__ __forceinline__ void forward(F f) const {
