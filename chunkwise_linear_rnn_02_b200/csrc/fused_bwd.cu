@@ -616,7 +616,8 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     mbar_wait(bar_m1, ph_m1, a.latch);
     ph_m1 ^= 1;
     tc_fence_after();
-    {  // this tile's part of Z^T for chunk i: row grow of the M=128 accumulator, 32 tokens
+    // this tile's part of Z^T for chunk i: row grow of the M=128 accumulator, 32 tokens
+    auto z_epilogue = [&]() {
       float zv[32];
       tmem_ld32(tmem + L::T_Z + lane_off + half * 32, zv);
       tmem_ld_wait();
@@ -633,7 +634,8 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         kz += (bf2f(sm + L::KH_HI + off) + bf2f(sm + L::KH_LO + off)) * zv[c];
       }
       a.ws_kz[((((size_t)bh * (DV / VT) + vt) * NC + i) * 2 + half) * DK + grow] = kz;
-    }
+    };
+    if (safe) z_epilogue();  // the exact path below overwrites Kh
     float* XA = reinterpret_cast<float*>(sm + L::XA);
     if (safe) {  // exact A = sum_d q_jd k_rd e^{B_jd - B_rd}, r <= j
       float* XB = reinterpret_cast<float*>(sm + L::XB);
@@ -671,6 +673,22 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         store_half_split(sm + L::AB_HI, sm + L::AB_LO, row, v, half);
       }
     }
+    fence_async_smem();
+    sync_tc();
+    if (tid == 0) {
+      if (safe && n + 1 < NC) load_qkg(i - 1);
+      const uint32_t dob = base + 3 * L::RAW;
+      constexpr uint32_t id_dv2 = idesc_bf16_f32(C, VT, true, true);
+#pragma unroll
+      for (int k = 0; k < C / 16; ++k) {
+        const uint64_t dd = desc_sw128(dob + k * 2048, C * 128, 1024);
+        umma_bf16(tmem + L::T_DV, desc_sw128(base + L::AB_HI + k * 2048, C * 128, 1024), dd, id_dv2, 1);
+        umma_bf16(tmem + L::T_DV, desc_sw128(base + L::AB_LO + k * 2048, C * 128, 1024), dd, id_dv2, 1);
+      }
+      umma_commit(bar_m2);
+    }
+    // while the second group runs: the Z^T epilogue and the G pass (neither touches A, dO or dv)
+    if (!safe) z_epilogue();
     {  // G_i = dec * G (chunks off the exact path, whose rescale came first) and its hi / lo copy
       const float sc = safe ? 1.f : DEC[grow];
       float v[64];
@@ -687,20 +705,6 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         store_row_split(sm + L::GC_HI + (cb / 64) * (DK * 128), sm + L::GC_LO + (cb / 64) * (DK * 128), grow, v, 1.f);
       }
       tmem_st_wait();
-    }
-    fence_async_smem();
-    sync_tc();
-    if (tid == 0) {
-      if (safe && n + 1 < NC) load_qkg(i - 1);
-      const uint32_t dob = base + 3 * L::RAW;
-      constexpr uint32_t id_dv2 = idesc_bf16_f32(C, VT, true, true);
-#pragma unroll
-      for (int k = 0; k < C / 16; ++k) {
-        const uint64_t dd = desc_sw128(dob + k * 2048, C * 128, 1024);
-        umma_bf16(tmem + L::T_DV, desc_sw128(base + L::AB_HI + k * 2048, C * 128, 1024), dd, id_dv2, 1);
-        umma_bf16(tmem + L::T_DV, desc_sw128(base + L::AB_LO + k * 2048, C * 128, 1024), dd, id_dv2, 1);
-      }
-      umma_commit(bar_m2);
     }
     __syncwarp();
     mbar_wait(bar_m2, ph_m2, a.latch);
@@ -828,7 +832,6 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   const int tb = half * 32;
   float* DEC = reinterpret_cast<float*>(sm + L::DEC);
   float* TOT = reinterpret_cast<float*>(sm + L::TOT);
-  float2* XCH = reinterpret_cast<float2*>(sm + L::XCH);
   float* DIAG = reinterpret_cast<float*>(sm + L::DIAG);
 
   if (warp == 0) {
@@ -855,37 +858,45 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
     tma_load_3d(sm + L::PB_G, &mp.g64, &bar_ld, d0, i * C, bh);
     tma_load_3d(sm + L::PB_Q, &mp.q64, &bar_ld, d0, i * C, bh);
   }
+  // The epilogue runs on all 32 lanes: lane l < 16 owns key dim row = q4 * 16 + l for tokens
+  // tb .. tb + 15, lane l + 16 the same dim for tokens tb + 16 .. tb + 31 (the M = 64 accumulators
+  // sit in TMEM lanes 0-15 of each quarter, so those values reach the upper lanes by shuffle).
+  const int sub = lane >> 4, tq = tb + sub * 16, qi = half * 2 + sub;
+  const int erow = q4 * 16 + (lane & 15);
   // global inputs of the epilogue, loaded while the tiles arrive
-  float pv[32], z[32];
-  float ci = 0.f;
-  if (row_owner) {
-    const float4* src = reinterpret_cast<const float4*>(a.ws_part + (((size_t)bh * NC + i) * DK + d0 + row) * C + tb);
+  float pv[16], z[16];
+  {
+    const float4* src = reinterpret_cast<const float4*>(a.ws_part + (((size_t)bh * NC + i) * DK + d0 + erow) * C + tq);
+    float4 u[4], zz[NVT][4];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const float4 u = src[c];
-      pv[4 * c] = u.x;
-      pv[4 * c + 1] = u.y;
-      pv[4 * c + 2] = u.z;
-      pv[4 * c + 3] = u.w;
-    }
-    ci = a.ws_c[((size_t)bh * NC + i) * DK + d0 + row];
+    for (int c = 0; c < 4; ++c) u[c] = src[c];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) z[c] = 0.f;
     for (int vt = 0; vt < NVT; ++vt) {
       const float4* zs = reinterpret_cast<const float4*>(
-          a.ws_z + ((((size_t)bh * NVT + vt) * NC + i) * DK + d0 + row) * C + tb);
+          a.ws_z + ((((size_t)bh * NVT + vt) * NC + i) * DK + d0 + erow) * C + tq);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float4 u = zs[c];
-        z[4 * c] += u.x;
-        z[4 * c + 1] += u.y;
-        z[4 * c + 2] += u.z;
-        z[4 * c + 3] += u.w;
-      }
+      for (int c = 0; c < 4; ++c) zz[vt][c] = zs[c];
     }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      pv[4 * c] = u[c].x;
+      pv[4 * c + 1] = u[c].y;
+      pv[4 * c + 2] = u[c].z;
+      pv[4 * c + 3] = u[c].w;
+      z[4 * c] = z[4 * c + 1] = z[4 * c + 2] = z[4 * c + 3] = 0.f;
+    }
+#pragma unroll
+    for (int vt = 0; vt < NVT; ++vt)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        z[4 * c] += zz[vt][c].x;
+        z[4 * c + 1] += zz[vt][c].y;
+        z[4 * c + 2] += zz[vt][c].z;
+        z[4 * c + 3] += zz[vt][c].w;
+      }
   }
+  const float ci = a.ws_c[((size_t)bh * NC + i) * DK + d0 + erow];
   auto raw = [&](uint32_t off, int j, int d) { return bf2f(sm + off + sw128(j, d)); };
-  auto raw2 = [&](uint32_t off, int j, int d) { return *reinterpret_cast<const uint32_t*>(sm + off + sw128(j, d)); };
   auto dA_at = [&](int j, int r) { return raw(L::DA_HI, j, r) + raw(L::DA_LO, j, r); };
 
   mbar_wait(&bar_ld, 0, a.latch);
@@ -949,35 +960,40 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
     }
     umma_commit(&bar_m2);
   }
-  float w[32];
+  const int d = erow;
+  float w[16];
   if (!safe) {
+    float wr[32];
     __syncwarp();
     mbar_wait(&bar_m2, 0, a.latch);
     tc_fence_after();
-    tmem_ld32(tmem + L::T_Y + lane_off + tb, w);
+    tmem_ld32(tmem + L::T_Y + lane_off + tb, wr);
     tmem_ld_wait();
-  }
-  float tot_k = 0.f, tot_s = 0.f;
-  if (row_owner) {  // dk; per-token terms Kh Z and Kh Z + k dk^intra without j = r (-> w)
-    const int d = row;
-    if (safe) {  // exact intra term w_r = sum_{j>=r} dA_jr q_j e^{B_j - B_r}
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int r = tb + c;
-        float acc = dA_at(r, r) * raw(L::PB_Q, r, d), bd = 0.f;
-        for (int j = r + 1; j < C; ++j) {
-          bd += raw(L::PB_G, j, d);
-          acc += dA_at(j, r) * raw(L::PB_Q, j, d) * __expf(bd);
-        }
-        w[c] = acc;
-      }
+    for (int c = 0; c < 16; ++c) {
+      const float x = __shfl_sync(0xffffffffu, wr[16 + c], lane & 15);
+      w[c] = sub ? x : wr[c];
     }
-    const float inv = 1.f / DEC[d];
-    __nv_bfloat16* dst = a.dk + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
-    float* dst32 = ACC ? a.acc_k + ((size_t)bh * T + i * C + tb) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
+  } else {  // exact intra term w_r = sum_{j>=r} dA_jr q_j e^{B_j - B_r}
 #pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {
-      const int h = half * 4 + rr;
+    for (int c = 0; c < 16; ++c) {
+      const int r = tq + c;
+      float acc = dA_at(r, r) * raw(L::PB_Q, r, d), bd = 0.f;
+      for (int j = r + 1; j < C; ++j) {
+        bd += raw(L::PB_G, j, d);
+        acc += dA_at(j, r) * raw(L::PB_Q, j, d) * __expf(bd);
+      }
+      w[c] = acc;
+    }
+  }
+  float tot_s = 0.f;
+  {  // dk; per-token terms Kh Z + k dk^intra without j = r (-> w)
+    const float inv = 1.f / DEC[d];
+    __nv_bfloat16* dst = a.dk + ((size_t)bh * T + i * C + tq) * DK + d0 + d;
+    float* dst32 = ACC ? a.acc_k + ((size_t)bh * T + i * C + tq) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
+#pragma unroll
+    for (int rr = 0; rr < 16 / TS; ++rr) {
+      const int h = tq / TS + rr;
       float al[TS], e2[TS];
 #pragma unroll
       for (int u = 0; u < TS; ++u) al[u] = ex2(raw(L::PB_G, h * TS + u, d) * kLog2e);
@@ -990,7 +1006,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
       }
 #pragma unroll
       for (int u = 0; u < TS; ++u) {
-        const int c = rr * TS + u, r = tb + c;
+        const int c = rr * TS + u, r = tq + c;
         const float ev = e2[u];
         if (!safe) w[c] *= ev * inv;
         const float qv = raw(L::PB_Q, r, d), kv = raw(L::PB_K, r, d);
@@ -1005,18 +1021,18 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
         tot_s += w[c];
       }
     }
-    XCH[half * KT + d] = make_float2(tot_k, tot_s);
   }
+  float* XQ = reinterpret_cast<float*>(sm + L::XCH);  // [4 token quarters][KT] sums of w
+  XQ[qi * KT + d] = tot_s;
   __syncthreads();
-  if (row_owner) {  // dg = c_i + prefix (exclusive) of (Kh Z + k dk^intra) + the forward walk's part
-    const int d = row;
-    const float2 o = XCH[(half ^ 1) * KT + d];
-    float pre = half == 1 ? o.y : 0.f;
-    __nv_bfloat16* dst = a.dg + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
-    float* dst32 = ACC ? a.acc_g + ((size_t)bh * T + i * C + tb) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
+  {  // dg = c_i + prefix (exclusive) of (Kh Z + k dk^intra) + the forward walk's part
+    float pre = 0.f;
+    for (int t = 0; t < qi; ++t) pre += XQ[t * KT + d];
+    __nv_bfloat16* dst = a.dg + ((size_t)bh * T + i * C + tq) * DK + d0 + d;
+    float* dst32 = ACC ? a.acc_g + ((size_t)bh * T + i * C + tq) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      if (i * C + tb + c < T) {
+    for (int c = 0; c < 16; ++c) {
+      if (i * C + tq + c < T) {
         if (ACC)
           dst32[(size_t)c * a.acc_pk] = ci + pre + pv[c];
         else
