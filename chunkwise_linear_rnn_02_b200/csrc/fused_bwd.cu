@@ -9,18 +9,17 @@
 //   dk  = E2 (V G_{i+1}^T) + (E2 / dec) (dA^T Qt)
 //   dv  = Kh G_{i+1} + A^T dO
 //   G_i = dec G_{i+1} + Qt^T dO               S_{i+1} = dec S_i + Kh^T V
-//   dg: chunk-local parts plus a carry across chunk boundaries (see the key tile below), so
-//       that no rounding accumulates over the sequence.
+//   dg: chunk-local parts plus a carry across chunk boundaries (the carry scan below), so that
+//       no rounding accumulates over the sequence.
 //
-// Two launches on the caller's stream:
-//   1. two kinds of CTA, all resident at once:
+// Three launches on the caller's stream:
+//   1. two kinds of CTA, independent of each other:
 //      * key-tile CTAs, one per (head, 64 key dimensions): a forward walk that rebuilds S on chip
-//        and writes dq, the forward part of dg (fp32, workspace) and the carry's start value;
+//        and writes dq, the forward part of dg and the chunk sums of Qt X (fp32, workspace), and
+//        the carry's start value rowsum(dhT * hT);
 //      * value-tile CTAs, one per (head, 128 value columns): a reverse walk carrying G[:, tile]
-//        that writes dv, dh0[:, tile] and this tile's part of Z^T = G V^T for every chunk
-//        (fp32, workspace; Z sums over the value tiles);
-//      The value tiles also write, per chunk, their part of sum_r Kh_r Z_r (the chunk sums that
-//      drive the dg carry);
+//        that writes dv, dh0[:, tile], and for every chunk this tile's part of Z^T = G V^T and of
+//        the chunk sums of Kh Z (fp32, workspace; both are summed over the value tiles later);
 //   2. a scan over chunks per (head, key dim) that turns the chunk sums into the carry c_i of
 //      every chunk;
 //   3. one CTA per (head, 64 key dimensions, chunk), all independent: dk and the rest of dg
@@ -59,7 +58,7 @@ struct BwdArgs {
   float* ws_kz;    // [BH][DV/VT][NC][2][DK] value tiles' parts of the chunk sums of Kh Z (per token half)
   float* ws_c;     // [BH][NC][DK] the dg carry c_i of every chunk
   float* ws_part;  // [BH][NC][DK][64] forward-walk part of dg, one row of 64 tokens per chunk and dim
-  int T, n_key_ctas;
+  int T;
   long long st_bh, st_row;  // h0 / dhT / dh0 strides (a sub-block of a larger state when split)
   // Optional fp32 outputs for a split shape: when set, dq / dk / dg go to columns acc_ck + key dim
   // of [BH*T][acc_pk] arrays and dv to columns acc_cv + value col of a [BH*T][acc_pv] array, in
@@ -80,13 +79,13 @@ struct BwdArgs {
 //   c_i  = e^{gamma_i} rowsum(G_{i+1} * S_i), carried backwards over chunk boundaries as
 //   c_{N-1} = rowsum(dhT * hT) - sum_r (Kh Z)_{N-1},  c_i = c_{i+1} + sum_j (Qt X)_{i+1} - sum_r (Kh Z)_i.
 // The forward walk writes the Qt X and q dq^intra parts (chunk-local, fp32) and the chunk sums of
-// Qt X into the workspace; the reverse walk adds the rest.  The chunk sums use Qt and Kh exactly as
-// the G and S updates see them (bf16 hi + lo), so the recurrence for c telescopes exactly for the
-// states the kernel carries and its rounding does not accumulate over chunks.  Because the four
-// parts of dg are several times larger than dg, every MMA operand of this CTA is a bf16 hi + lo
-// pair (three products per MMA), which keeps them near fp32 accuracy.  The state copies feeding X and Z
-// are split into bf16 hi + lo parts, because the chunk sums they produce are carried over the
-// whole sequence.
+// Qt X into the workspace; the value tiles write the chunk sums of Kh Z, the carry scan forms every
+// c_i and the chunk kernel adds the rest.  The chunk sums use Qt and Kh as the G and S updates see
+// them (bf16 hi + lo), so the recurrence for c telescopes for the states the kernels carry and its
+// rounding does not accumulate over chunks.  Because the four parts of dg are several times
+// larger than dg, every MMA operand is a bf16 hi + lo pair (three products per MMA, two where one
+// side is exact), which keeps them near fp32 accuracy; the state copies feeding X and Z are split
+// the same way, because the chunk sums they produce are carried over the whole sequence.
 // ------------------------------------------------------------------------------------------
 template <int DK, int DV>
 struct KeyLayout {
@@ -96,9 +95,9 @@ struct KeyLayout {
   static constexpr uint32_t PB = 2 * VB;            // part B: k, g, q tiles (two buffers)
   static constexpr uint32_t PB_STAGE = 3 * TILE;
   static constexpr uint32_t PB_K = 0, PB_G = TILE, PB_Q = 2 * TILE;  // offsets inside a part-B buffer
-  static constexpr uint32_t KQ_HI = PB + 2 * PB_STAGE;  // Kh (forward walk) / Qt (reverse walk), hi / lo
+  static constexpr uint32_t KQ_HI = PB + 2 * PB_STAGE;  // Kh hi / lo
   static constexpr uint32_t KQ_LO = KQ_HI + TILE;
-  static constexpr uint32_t SG_HI = KQ_LO + TILE;   // bf16 hi / lo copies of S or G rows [64 x DV], K-major
+  static constexpr uint32_t SG_HI = KQ_LO + TILE;   // bf16 hi / lo copies of the S rows [64 x DV], K-major
   static constexpr uint32_t SG_LO = SG_HI + KT * DV * 2;
   static constexpr uint32_t DA_HI = SG_LO + KT * DV * 2;  // masked dA, bf16 hi / lo [64 x 64]
   static constexpr uint32_t DA_LO = DA_HI + TILE;
@@ -107,8 +106,7 @@ struct KeyLayout {
   static constexpr uint32_t DEC = XCH + 2 * KT * 8;     // float [2][64]: chunk decays, per part-B buffer
   static constexpr uint32_t TOT = DEC + 2 * KT * 4;     // float [2][NS][64]: gate run products, per buffer
   static constexpr uint32_t DIAG = TOT + 2 * NS * KT * 4;
-  static constexpr uint32_t CARRY = DIAG + C * 4;       // [2][64] c_i, double-buffered over chunks
-  static constexpr uint32_t CARRYP = CARRY + 2 * KT * 4;  // [2][64] per-column-half partial row sums
+  static constexpr uint32_t CARRYP = DIAG + C * 4;      // [2][64] per-column-half partial row sums
   static constexpr uint32_t TOTAL = CARRYP + 2 * KT * 4;
   // TMEM columns
   static constexpr uint32_t T_SG = 0, T_DA = DV, T_X = DV + 64, T_Y = DV + 128;
@@ -119,9 +117,9 @@ struct KeyLayout {
 };
 
 // Key-tile schedule: chunk i's epilogue runs while chunk i+1's first MMA group is on the tensor
-// pipe.  Per chunk step: wait for MMA group 1 of chunk i, move its dA and X^T (Z^T) rows into
-// registers, issue group 2 (Y^T or W^T); then prepare chunk i+1 (gate run from the second part-B
-// buffer, Kh or Qt operand, state copy and rescale) and issue its group 1; then finish chunk i's
+// pipe.  Per chunk step: wait for MMA group 1 of chunk i, move its dA and X^T rows into
+// registers, issue group 2 (Y^T); then prepare chunk i+1 (gate run from the second part-B
+// buffer, Kh operand, state copy and rescale) and issue its group 1; then finish chunk i's
 // outputs.  The epilogue forms E1 / E2 itself from the raw gates and the run products of the gate
 // run, multiplying in the same order, so its values equal the ones behind the MMA operands.
 template <int DK, int DV, bool ACC>
@@ -149,7 +147,6 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   float* TOT = reinterpret_cast<float*>(sm + L::TOT);
   float2* XCH = reinterpret_cast<float2*>(sm + L::XCH);
   float* DIAG = reinterpret_cast<float*>(sm + L::DIAG);
-  float* CARRY = reinterpret_cast<float*>(sm + L::CARRY);
   float* qx_sums = a.ws_qx + (size_t)bh * NC * DK + d0;          // [NC][DK] slice of this head and key tile
   float* part = a.ws_part + ((size_t)bh * NC * DK + d0) * C;  // [NC][DK][64] slice: forward-walk part of dg
 
@@ -241,9 +238,8 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       store_half_split(sm + L::DA_HI, sm + L::DA_LO, row, v, half);
     }
   };
-  // MMA group 1: dA = dO V^T; X^T = S dO^T (forward) or Z^T = G V^T (reverse); and the state
-  // update S += Kh^T V (forward) or G += Qt^T dO (reverse).
-  auto issue_m1 = [&](bool fwd) {
+  // MMA group 1: dA = dO V^T, X^T = S dO^T and the state update S += Kh^T V.
+  auto issue_m1 = [&]() {
     if (tid != 0) return;
     mbar_wait(bar_pa, ph_pa, a.latch);
     ph_pa ^= 1;
@@ -251,11 +247,10 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     constexpr uint32_t id_dA = idesc_bf16_f32(C, C, false, false);
     constexpr uint32_t id_X = idesc_bf16_f32(KT, C, false, false);
     constexpr uint32_t id_S = idesc_bf16_f32(KT, DV, true, true);
-    const uint32_t xb = fwd ? L::PA_DO : L::PA_V, sb = fwd ? L::PA_V : L::PA_DO;
 #pragma unroll
     for (int k = 0; k < DV / 16; ++k) {
       const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
-      const uint64_t bd = desc_sw128(base + xb + ko, 16, 1024);
+      const uint64_t bd = desc_sw128(base + L::PA_DO + ko, 16, 1024);
       umma_bf16(tmem + L::T_DA, desc_sw128(base + L::PA_DO + ko, 16, 1024),
                 desc_sw128(base + L::PA_V + ko, 16, 1024), id_dA, k > 0);
       umma_bf16(tmem + L::T_X, desc_sw128(base + L::SG_HI + ko, 16, 1024), bd, id_X, k > 0);
@@ -263,29 +258,25 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     }
 #pragma unroll
     for (int k = 0; k < C / 16; ++k) {
-      const uint64_t dd = desc_sw128(base + sb + k * 2048, C * 128, 1024);
+      const uint64_t dd = desc_sw128(base + L::PA_V + k * 2048, C * 128, 1024);
       umma_bf16(tmem + L::T_SG, desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024), dd, id_S, 1);
       umma_bf16(tmem + L::T_SG, desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024), dd, id_S, 1);
     }
     umma_commit(bar_m1);
   };
-  // MMA group 2: Y^T = Kh^T dA^T (forward) or W^T = Qt^T dA (reverse).
-  auto issue_m2 = [&](bool fwd) {
+  // MMA group 2: Y^T = Kh^T dA^T.
+  auto issue_m2 = [&]() {
     if (tid != 0) return;
     constexpr uint32_t id_Y = idesc_bf16_f32(KT, C, true, false);
-    constexpr uint32_t id_W = idesc_bf16_f32(KT, C, true, true);
 #pragma unroll
     for (int k = 0; k < C / 16; ++k) {
       const uint64_t ah = desc_sw128(base + L::KQ_HI + k * 2048, C * 128, 1024);
       const uint64_t al = desc_sw128(base + L::KQ_LO + k * 2048, C * 128, 1024);
-      const uint64_t bh = fwd ? desc_sw128(base + L::DA_HI + k * 32, 16, 1024)
-                              : desc_sw128(base + L::DA_HI + k * 2048, C * 128, 1024);
-      const uint64_t bl = fwd ? desc_sw128(base + L::DA_LO + k * 32, 16, 1024)
-                              : desc_sw128(base + L::DA_LO + k * 2048, C * 128, 1024);
-      const uint32_t id = fwd ? id_Y : id_W;
-      umma_bf16(tmem + L::T_Y, ah, bh, id, k > 0);
-      umma_bf16(tmem + L::T_Y, al, bh, id, 1);
-      umma_bf16(tmem + L::T_Y, ah, bl, id, 1);
+      const uint64_t bh = desc_sw128(base + L::DA_HI + k * 32, 16, 1024);
+      const uint64_t bl = desc_sw128(base + L::DA_LO + k * 32, 16, 1024);
+      umma_bf16(tmem + L::T_Y, ah, bh, id_Y, k > 0);
+      umma_bf16(tmem + L::T_Y, al, bh, id_Y, 1);
+      umma_bf16(tmem + L::T_Y, ah, bl, id_Y, 1);
     }
     umma_commit(bar_m2);
   };
@@ -294,34 +285,31 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     ph_m2 ^= 1;
     tc_fence_after();
   };
-  // Chunk i+1 (or i-1): gate run from buffer nb, Kh / Qt operand, state copy + rescale, group 1.
-  // The operand area KQ is free once group 2 of the current chunk has completed.
-  auto prepare = [&](bool fwd, int nb, int m2_pending) {
+  // Chunk i+1: gate run from buffer nb, Kh operand, state copy + rescale, group 1.  The operand
+  // area KQ is free once group 2 of the current chunk has completed.
+  auto prepare = [&](int nb, int m2_pending) {
     wait_b(nb);
     Gate gr;
     const int safe = gate(gr, nb);
     uint32_t w[Gate::TS];
-    gr.load_pairs(sm + pbo(nb) + (fwd ? L::PB_K : L::PB_Q), KT, true, w);
+    gr.load_pairs(sm + pbo(nb) + L::PB_K, KT, true, w);
     if (m2_pending) wait_m2();
-    if (fwd)
-      gr.backward([&](int j, float e0, float e1) { write_kq(w[j - gr.h * Gate::TS], j, gr.d, e0, e1); });
-    else
-      gr.forward([&](int j, float e0, float e1) { write_kq(w[j - gr.h * Gate::TS], j, gr.d, e0, e1); });
+    gr.backward([&](int j, float e0, float e1) { write_kq(w[j - gr.h * Gate::TS], j, gr.d, e0, e1); });
     state_pass(nb);
     fence_async_smem();
     sync_tc();
-    issue_m1(fwd);
+    issue_m1();
     return safe;
   };
 
-  // ============================ forward walk: dq, first part of dg ============================
+  // ================================ forward walk: dq, first part of dg ================================
   if (tid == 0) {
     load_a(0);
     load_b(0, 0);
     if (NC > 1) load_b(1, 1);
   }
   init_state(a.h0);
-  int safe_next = prepare(true, 0, 0);
+  int safe_next = prepare(0, 0);
   for (int i = 0; i < NC; ++i) {
     const int b = i & 1, safe = safe_next;
     mbar_wait(bar_m1, ph_m1, a.latch);
@@ -333,9 +321,9 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     dA_epilogue();
     fence_async_smem();
     sync_tc();
-    if (!safe) issue_m2(true);
+    if (!safe) issue_m2();
     if (i + 1 < NC)
-      safe_next = prepare(true, b ^ 1, !safe);
+      safe_next = prepare(b ^ 1, !safe);
     else if (!safe)
       wait_m2();
     float y[32];  // this thread's row of Y^T
@@ -428,13 +416,8 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     }
     if (row_owner) CARRYP[half * KT + row] = acc;
     __syncthreads();
-    if (tid < KT) CARRY[tid] = CARRYP[tid] + CARRYP[KT + tid];  // c for the last chunk: buffer 0
+    if (tid < KT) a.ws_carry[(size_t)bh * DK + d0 + tid] = CARRYP[tid] + CARRYP[KT + tid];
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-
-  if (tid < KT) a.ws_carry[(size_t)bh * DK + d0 + tid] = CARRY[tid];
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1156,7 +1139,6 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
   a.acc_ck = acc ? acc->ck : 0;
   a.acc_pv = acc ? acc->pv : 0;
   a.acc_cv = acc ? acc->cv : 0;
-  a.n_key_ctas = BH * (DK / KT);
   const size_t NC = (T + C - 1) / C;
   a.ws_qx = static_cast<float*>(ws);
   a.ws_part = a.ws_qx + align256((size_t)BH * NC * DK * sizeof(float)) / sizeof(float);
