@@ -66,24 +66,32 @@ struct FwdArgs {
 // state recurrence alone (gates, Kh, dS = Kh^T V, S = e^{gamma} S + dS; no queries, no outputs)
 // and writes the segment's end state and decay product.  Kh is finite for every gate (E2 <= 1),
 // so this pass needs no exact path.
+//
+// REV: the same pass for the backward's state gradient G = dL/dS, which runs the other way:
+// G_i = e^{gamma} G_{i+1} + Qt^T dO with Qt = q e^{B} (E1 <= 1, again finite for every gate).  Its
+// CTAs take segments 1 .. nseg-1, walk their chunks last to first, start the last segment from
+// dhT (args.h0) and write the G at each segment's start from its end G of zero (from dhT).
+// HILO: the operand enters the MMA as a bf16 hi + lo pair (the backward's gate gradient takes
+// sums several times larger than itself from these states).
 // ------------------------------------------------------------------------------------------
-template <int DK>
+template <int DK, bool HILO>
 struct StateLayout {
   static constexpr uint32_t RAW = C * DK * 2;          // one raw k / g tile
   static constexpr uint32_t STAGE = 2 * RAW + C * DVT * 2;  // k, g, v
-  static constexpr uint32_t KH = 2 * STAGE;            // Kh [64 x DK], MN-major A operand of dS
-  static constexpr uint32_t DECAY = KH + C * DK * 2;
+  static constexpr uint32_t KH = 2 * STAGE;            // Kh [64 x DK], MN-major A operand of dS (hi part)
+  static constexpr uint32_t KH_LO = KH + C * DK * 2;   // its lo part (HILO)
+  static constexpr uint32_t DECAY = KH + (HILO ? 2 : 1) * C * DK * 2;
   static constexpr uint32_t TOT = DECAY + DK * 4;
   static constexpr uint32_t TOTAL = TOT + GateRun<DK, NTHREADS>::NSPLIT * DK * 4;
   static constexpr uint32_t ALLOC = TOTAL + 1024;
   static_assert(STAGE % 1024 == 0 && RAW % 1024 == 0, "stage alignment");
 };
 
-template <int DK>
+template <int DK, bool HILO, bool REV>
 __global__ void __launch_bounds__(NTHREADS, 1)
     fwd_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_g,
                      const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
-  using L = StateLayout<DK>;
+  using L = StateLayout<DK, HILO>;
   using Gate = GateRun<DK, NTHREADS>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_load[2], bar_mma;
@@ -92,10 +100,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, half = warp >> 2;
-  const int dv0 = blockIdx.x * DVT, bh = blockIdx.y, seg = blockIdx.z;
+  const int dv0 = blockIdx.x * DVT, bh = blockIdx.y, seg = REV ? blockIdx.z + 1 : blockIdx.z;
   const int T = args.T, DV = args.DV, NC = (T + C - 1) / C;
   const int c_begin = seg * args.seg_chunks;
-  const int nloc = min(NC, c_begin + args.seg_chunks) - c_begin;
+  const int c_end = min(NC, c_begin + args.seg_chunks);
+  const int nloc = c_end - c_begin;
   float* decay_sm = reinterpret_cast<float*>(sm + L::DECAY);
   float* tot_sm = reinterpret_cast<float*>(sm + L::TOT);
   if (warp == 0) {
@@ -110,7 +119,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
   __syncthreads();
   auto issue_load = [&](int li) {
-    const int s = li & 1, chunk = c_begin + li;
+    const int s = li & 1, chunk = REV ? c_end - 1 - li : c_begin + li;
     uint8_t* st = sm + s * L::STAGE;
     mbar_arrive_expect_tx(&bar_load[s], L::STAGE);
     tma_load_3d(st, &tm_k, &bar_load[s], 0, chunk * C, bh);
@@ -128,7 +137,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   float S[SW];
 #pragma unroll
   for (int c = 0; c < SW; ++c) S[c] = 0.f;
-  if (seg == 0 && s_owner && args.h0) {
+  if (seg == (REV ? args.nseg - 1 : 0) && s_owner && args.h0) {
     const float4* src = reinterpret_cast<const float4*>(args.h0 + bh * args.st_bh + s_row * args.st_row + dv0 + sc0);
 #pragma unroll
     for (int c = 0; c < SW / 4; ++c) {
@@ -159,10 +168,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t blk = (gr.d >> 6) * (C * 128), col = gr.d & 63;
       uint32_t w[Gate::TS];
       gr.load_pairs(st, DK, false, w);
-      gr.backward([&](int j, float e0, float e1) {
+      auto put = [&](int j, float e0, float e1) {  // Kh = k E2, or Qt = q E1 (REV)
         const uint32_t wk = w[j - gr.h * Gate::TS];
-        *reinterpret_cast<uint32_t*>(sm + L::KH + blk + sw128(j, col)) = pack2(bf_lo(wk) * e0, bf_hi(wk) * e1);
-      });
+        if (HILO) {
+          uint32_t hi, lo;
+          split2(bf_lo(wk) * e0, bf_hi(wk) * e1, hi, lo);
+          *reinterpret_cast<uint32_t*>(sm + L::KH + blk + sw128(j, col)) = hi;
+          *reinterpret_cast<uint32_t*>(sm + L::KH_LO + blk + sw128(j, col)) = lo;
+        } else {
+          *reinterpret_cast<uint32_t*>(sm + L::KH + blk + sw128(j, col)) = pack2(bf_lo(wk) * e0, bf_hi(wk) * e1);
+        }
+      };
+      if (REV)
+        gr.forward(put);
+      else
+        gr.backward(put);
     }
     fence_async_smem();
     tc_fence_before();
@@ -173,9 +193,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t vbase = base + s * L::STAGE + 2 * L::RAW;
       constexpr uint32_t id_S = idesc_bf16_f32(DK, DVT, true, true);
 #pragma unroll
-      for (int k = 0; k < C / 16; ++k)
-        umma_bf16(t_dS, desc_sw128(base + L::KH + k * 2048, C * 128, 1024), desc_sw128(vbase + k * 2048, 16, 1024),
-                  id_S, k > 0);
+      for (int k = 0; k < C / 16; ++k) {
+        const uint64_t vd = desc_sw128(vbase + k * 2048, 16, 1024);
+        umma_bf16(t_dS, desc_sw128(base + L::KH + k * 2048, C * 128, 1024), vd, id_S, k > 0);
+        if (HILO) umma_bf16(t_dS, desc_sw128(base + L::KH_LO + k * 2048, C * 128, 1024), vd, id_S, 1);
+      }
       umma_commit(&bar_mma);
     }
     __syncwarp();
@@ -194,12 +216,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     if (tid == 0 && li + 2 < nloc) issue_load(li + 2);
   }
-  float* out = args.sbuf + ((size_t)bh * args.nseg + seg) * DK * DV;
+  float* out = args.sbuf + ((size_t)bh * args.nseg + (REV ? seg - 1 : seg)) * DK * DV;
   if (s_owner) {
     float4* dst = reinterpret_cast<float4*>(out + (size_t)s_row * DV + dv0 + sc0);
 #pragma unroll
     for (int c = 0; c < SW / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
-    if (half == 0 && blockIdx.x == 0) args.gam[((size_t)bh * args.nseg + seg) * DK + s_row] = gamma_acc;
+    if (!REV && half == 0 && blockIdx.x == 0) args.gam[((size_t)bh * args.nseg + seg) * DK + s_row] = gamma_acc;
   }
   tc_fence_before();
   __syncthreads();
@@ -629,17 +651,20 @@ size_t fwd_workspace(int BH, int T, int dk, int dv) {
   return align256((size_t)BH * nseg * dk * dv * sizeof(float)) + align256((size_t)BH * nseg * dk * sizeof(float));
 }
 
-template <int DK>
-static cudaError_t launch_state_pass(const CUtensorMap* m, const FwdArgs& args, int BH, int dv, cudaStream_t st) {
-  auto kern = fwd_state_kernel<DK>;
+// m: maps of the operand ([64 x DK] rows), the gates, and the 64-column value tiles.
+template <int DK, bool HILO, bool REV>
+static cudaError_t launch_state_pass(const CUtensorMap& mk, const CUtensorMap& mg, const CUtensorMap& mv,
+                                     const FwdArgs& args, int BH, int dv, cudaStream_t st) {
+  auto kern = fwd_state_kernel<DK, HILO, REV>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK>::ALLOC);
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK, HILO>::ALLOC);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   dim3 grid(dv / DVT, BH, args.nseg - 1);
-  kern<<<grid, NTHREADS, StateLayout<DK>::ALLOC, st>>>(m[1], m[2], m[3], args);
+  kern<<<grid, NTHREADS, StateLayout<DK, HILO>::ALLOC, st>>>(mk, mg, mv, args);
   return cudaGetLastError();
 }
 
@@ -668,7 +693,7 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
     if (!ws) return cudaErrorInvalidValue;
     a.sbuf = static_cast<float*>(ws);
     a.gam = a.sbuf + align256((size_t)BH * a.nseg * DK * dv * sizeof(float)) / sizeof(float);
-    cudaError_t e = launch_state_pass<DK>(m, a, BH, dv, st);
+    cudaError_t e = launch_state_pass<DK, false, false>(m[1], m[2], m[3], a, BH, dv, st);
     if (e != cudaSuccess) return e;
     if (a.nseg > 2) {
       const size_t n = (size_t)BH * DK * dv;
@@ -688,6 +713,71 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
   dim3 grid(dv / DVT, BH, a.nseg);
   kern<<<grid, PIPE_THREADS, FwdPipeLayout<DK>::ALLOC, st>>>(m[0], m[1], m[2], m[3], a);
   return cudaGetLastError();
+}
+
+// Segments of the backward's sequence split: as many as fill the SMs once when each segment takes
+// ctas_per_seg CTAs of the backward's first launch; 1 when those alone fill half of the SMs.
+void plan_bwd_segments(int ctas_per_seg, int T, int* nseg, int* seg_chunks) {
+  const int NC = (T + C - 1) / C, sms = sm_count();
+  int n = 1;
+  if (2 * ctas_per_seg <= sms) n = sms / ctas_per_seg;
+  if (n > NC) n = NC;
+  if (n < 1) n = 1;
+  const int per = (NC + n - 1) / n;
+  *seg_chunks = per;
+  *nseg = (NC + per - 1) / per;
+}
+
+// End gradients of segments nseg-3 .. 0, in place: entry s of gbuf holds the gradient at the start
+// of segment s+1 reached from a zero end gradient (from dhT for the last segment) on input, and
+// the gradient at the end of segment s on output: G_end(s) = Gamma_{s+1} * G_end(s+1) + entry s.
+__global__ void segment_scan_rev_kernel(float* __restrict__ gbuf, const float* __restrict__ gam, int BH, int DK,
+                                        int DV, int nseg) {
+  const size_t per = (size_t)DK * DV, n = (size_t)BH * per;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+    const size_t bh = e / per, rem = e % per;
+    const int d = (int)(rem / DV);
+    float* p = gbuf + bh * nseg * per + rem;
+    float acc = p[(nseg - 2) * per];
+    for (int sg = nseg - 3; sg >= 0; --sg) {
+      acc = gam[(bh * nseg + sg + 1) * DK + d] * acc + p[sg * per];
+      p[sg * per] = acc;
+    }
+  }
+}
+
+cudaError_t segment_states(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mg,
+                           const CUtensorMap& mv, const CUtensorMap& mdo, const float* h0, const float* dhT,
+                           float* sbuf, float* gbuf, float* gam, int BH, int T, int dk, int dv, int nseg,
+                           int seg_chunks, long long st_bh, long long st_row, cudaStream_t st) {
+  if (dk != 128 || nseg < 2) return cudaErrorNotSupported;
+  FwdArgs a = {};
+  a.T = T;
+  a.DV = dv;
+  a.seg_chunks = seg_chunks;
+  a.nseg = nseg;
+  a.st_bh = st_bh;
+  a.st_row = st_row;
+  a.latch = device_error_latch();
+  a.h0 = h0;
+  a.sbuf = sbuf;
+  a.gam = gam;
+  cudaError_t e = launch_state_pass<128, true, false>(mk, mg, mv, a, BH, dv, st);
+  if (e != cudaSuccess) return e;
+  FwdArgs r = a;
+  r.h0 = dhT;
+  r.sbuf = gbuf;
+  r.gam = nullptr;
+  e = launch_state_pass<128, true, true>(mq, mg, mdo, r, BH, dv, st);
+  if (e != cudaSuccess) return e;
+  if (nseg > 2) {
+    const size_t n = (size_t)BH * dk * dv;
+    const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+    segment_scan_kernel<<<blocks, 256, 0, st>>>(sbuf, gam, BH, dk, dv, nseg);
+    segment_scan_rev_kernel<<<blocks, 256, 0, st>>>(gbuf, gam, BH, dk, dv, nseg);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,

@@ -2,6 +2,8 @@
 // The API layer asks *_supported() first and otherwise runs the generic kernels.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace gla {
@@ -26,6 +28,16 @@ struct BwdAccum {
   float *q, *k, *g, *v;
   int pk, ck, pv, cv;
 };
+
+// Sequence split of the backward (d_k = 128): segment count and length, and the segment states
+// (fp32 [BH][nseg][DK][DV]): sbuf[s-1] = the forward state entering segment s (s >= 1, from h0),
+// gbuf[s] = dL/dS at the end of segment s (s <= nseg-2, from dhT), gam[s] = the decay product of
+// segment s (s <= nseg-2).  Maps: q, k, g as [64 x DK] row tiles, v and dO as 64-column tiles.
+void plan_bwd_segments(int ctas_per_seg, int T, int* nseg, int* seg_chunks);
+cudaError_t segment_states(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mg,
+                           const CUtensorMap& mv, const CUtensorMap& mdo, const float* h0, const float* dhT,
+                           float* sbuf, float* gbuf, float* gam, int BH, int T, int dk, int dv, int nseg,
+                           int seg_chunks, long long st_bh, long long st_row, cudaStream_t st);
 
 bool bwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype);
 size_t bwd_workspace(int BH, int T, int dk, int dv);

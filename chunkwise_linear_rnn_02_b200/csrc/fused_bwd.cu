@@ -53,12 +53,16 @@ struct BwdArgs {
   __nv_bfloat16 *dq, *dk, *dv, *dg;
   float* dh0;
   float* ws_qx;    // [BH][NC][DK] chunk sums of Qt X
-  float* ws_carry; // [BH][DK] rowsum(dhT * hT): the start of the dg carry
+  float* ws_carry; // [BH][nseg][DK] rowsum(G_end * S_end) per segment: where the dg carry starts
   float* ws_z;     // [BH][DV/VT][NC][DK][64] value tiles' parts of Z^T
   float* ws_kz;    // [BH][DV/VT][NC][2][DK] value tiles' parts of the chunk sums of Kh Z (per token half)
   float* ws_c;     // [BH][NC][DK] the dg carry c_i of every chunk
   float* ws_part;  // [BH][NC][DK][64] forward-walk part of dg, one row of 64 tokens per chunk and dim
   int T;
+  // Sequence split: nseg segments of seg_chunks chunks; s_in / g_end hold the segment states
+  // ([BH][nseg][DK][DV] fp32: s_in[s-1] enters segment s, g_end[s] = dL/dS at the end of s).
+  int nseg, seg_chunks, n_bh;
+  const float *s_in, *g_end;
   long long st_bh, st_row;  // h0 / dhT / dh0 strides (a sub-block of a larger state when split)
   // Optional fp32 outputs for a split shape: when set, dq / dk / dg go to columns acc_ck + key dim
   // of [BH*T][acc_pk] arrays and dv to columns acc_cv + value col of a [BH*T][acc_pv] array, in
@@ -123,8 +127,8 @@ struct KeyLayout {
 // outputs.  The epilogue forms E1 / E2 itself from the raw gates and the run products of the gate
 // run, multiplying in the same order, so its values equal the ones behind the MMA operands.
 template <int DK, int DV, bool ACC>
-__device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int tau, uint64_t* bars,
-                              uint32_t tmem) {
+__device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int tau, int seg,
+                              uint64_t* bars, uint32_t tmem) {
   using L = KeyLayout<DK, DV>;
   using Gate = GateRun<KT, BT>;
   constexpr int NS = L::NS, TS = Gate::TS;
@@ -132,6 +136,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
   const int T = a.T, NC = (T + C - 1) / C, d0 = tau * KT;
+  const int ch0 = seg * a.seg_chunks, ch1 = min(NC, ch0 + a.seg_chunks);  // this segment's chunks
   const uint32_t base = smem_u32(sm);
   const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
   const bool row_owner = lane < 16;
@@ -194,13 +199,12 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     *reinterpret_cast<uint32_t*>(sm + L::KQ_HI + sw128(j, d)) = hi;
     *reinterpret_cast<uint32_t*>(sm + L::KQ_LO + sw128(j, d)) = lo;
   };
-  // Initialise the TMEM state rows from a [DK x DV] fp32 source (or zeros).
-  auto init_state = [&](const float* src) {
+  // Initialise the TMEM state rows from a [DK x DV] fp32 source with row stride srow (or zeros).
+  auto init_state = [&](const float* src, long long srow) {
     float v[64];
     for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 64) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c)
-        v[c] = (src && row_owner) ? src[bh * a.st_bh + (d0 + row) * a.st_row + c0 + c] : 0.f;
+      for (int c = 0; c < 64; ++c) v[c] = (src && row_owner) ? src[(d0 + row) * srow + c0 + c] : 0.f;
       tmem_st32(tmem + L::T_SG + lane_off + c0, v);
       tmem_st32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
     }
@@ -304,25 +308,28 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
 
   // ================================ forward walk: dq, first part of dg ================================
   if (tid == 0) {
-    load_a(0);
-    load_b(0, 0);
-    if (NC > 1) load_b(1, 1);
+    load_a(ch0);
+    load_b(ch0, 0);
+    if (ch1 - ch0 > 1) load_b(ch0 + 1, 1);
   }
-  init_state(a.h0);
+  if (seg == 0)
+    init_state(a.h0 ? a.h0 + bh * a.st_bh : nullptr, a.st_row);
+  else
+    init_state(a.s_in + ((size_t)bh * a.nseg + seg - 1) * DK * DV, DV);
   int safe_next = prepare(0, 0);
-  for (int i = 0; i < NC; ++i) {
-    const int b = i & 1, safe = safe_next;
+  for (int i = ch0; i < ch1; ++i) {
+    const int b = (i - ch0) & 1, safe = safe_next;
     mbar_wait(bar_m1, ph_m1, a.latch);
     ph_m1 ^= 1;
     tc_fence_after();
-    if (tid == 0 && i + 1 < NC) load_a(i + 1);
+    if (tid == 0 && i + 1 < ch1) load_a(i + 1);
     float x[32];  // this thread's row of X^T: key dim d = row, tokens tb .. tb+31
     tmem_ld32(tmem + L::T_X + lane_off + tb, x);
     dA_epilogue();
     fence_async_smem();
     sync_tc();
     if (!safe) issue_m2();
-    if (i + 1 < NC)
+    if (i + 1 < ch1)
       safe_next = prepare(b ^ 1, !safe);
     else if (!safe)
       wait_m2();
@@ -378,7 +385,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       XCH[half * KT + d] = make_float2(tot_s, tot_e);
     }
     __syncthreads();
-    if (tid == 0 && i + 2 < NC) load_b(i + 2, b);
+    if (tid == 0 && i + 2 < ch1) load_b(i + 2, b);
     if (row_owner) {  // part = suffix (inclusive) of Qt X minus prefix (exclusive) of q dq^intra
       const int d = row;
       const float2 o = XCH[(half ^ 1) * KT + d];
@@ -400,23 +407,28 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     }
   }
 
-  // rowsum(dhT * hT): hT rows = the state after the forward walk
+  // rowsum(G_end * S_end): S_end rows = the state after this segment's walk, G_end = dhT for the
+  // last segment, else the gradient at the segment's end from the segment scan
   {
     float* CARRYP = reinterpret_cast<float*>(sm + L::CARRYP);
+    const bool last = seg == a.nseg - 1;
+    const float* gsrc = last ? (a.dhT ? a.dhT + bh * a.st_bh : nullptr)
+                             : a.g_end + ((size_t)bh * a.nseg + seg) * DK * DV;
+    const long long grs = last ? a.st_row : DV;
     float v[32];
     float acc = 0.f;
     for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 32) {
       tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
       tmem_ld_wait();
-      if (row_owner && a.dhT) {
-        const float* src = a.dhT + bh * a.st_bh + (d0 + row) * a.st_row + c0;
+      if (row_owner && gsrc) {
+        const float* src = gsrc + (d0 + row) * grs + c0;
 #pragma unroll
         for (int c = 0; c < 32; ++c) acc += src[c] * v[c];
       }
     }
     if (row_owner) CARRYP[half * KT + row] = acc;
     __syncthreads();
-    if (tid < KT) a.ws_carry[(size_t)bh * DK + d0 + tid] = CARRYP[tid] + CARRYP[KT + tid];
+    if (tid < KT) a.ws_carry[((size_t)bh * a.nseg + seg) * DK + d0 + tid] = CARRYP[tid] + CARRYP[KT + tid];
   }
 }
 
@@ -452,12 +464,13 @@ struct ValLayout {
 };
 
 template <int DK, bool ACC>
-__device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int vt, int DV,
+__device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int vt, int DV, int seg,
                               uint64_t* bars, uint32_t tmem) {
   using L = ValLayout<DK>;
   using Gate = GateRun<DK, BT>;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = a.T, NC = (T + C - 1) / C, c0 = vt * VT;
+  const int ch0 = seg * a.seg_chunks, ch1 = min(NC, ch0 + a.seg_chunks), nl = ch1 - ch0;  // segment
   const uint32_t base = smem_u32(sm);
   const int q4 = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
   const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
@@ -506,12 +519,16 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     }
     tmem_st_wait();
   };
-  // G rows (this thread owns row grow of the M=128 accumulator): init from dhT[:, tile]
+  // G rows (this thread owns row grow of the M=128 accumulator): init from dhT[:, tile] (last
+  // segment) or from the gradient at the segment's end
   {
+    const bool last = seg == a.nseg - 1;
+    const float* gsrc = last ? (a.dhT ? a.dhT + bh * a.st_bh + grow * a.st_row : nullptr)
+                             : a.g_end + (((size_t)bh * a.nseg + seg) * DK + grow) * DV;
     float v[64];
     for (int cb = half * HT; cb < (half + 1) * HT; cb += 64) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) v[c] = a.dhT ? a.dhT[bh * a.st_bh + grow * a.st_row + c0 + cb + c] : 0.f;
+      for (int c = 0; c < 64; ++c) v[c] = gsrc ? gsrc[c0 + cb + c] : 0.f;
       tmem_st32(tmem + L::T_G + lane_off + cb, v);
       tmem_st32(tmem + L::T_G + lane_off + cb + 32, v + 32);
       store_row_split(sm + L::GC_HI + (cb / 64) * (DK * 128), sm + L::GC_LO + (cb / 64) * (DK * 128), grow, v, 1.f);
@@ -519,11 +536,11 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     tmem_st_wait();
   }
   if (tid == 0) {
-    load_qkg(NC - 1);
-    load_dov(NC - 1);
+    load_qkg(ch1 - 1);
+    load_dov(ch1 - 1);
   }
-  for (int n = 0; n < NC; ++n) {
-    const int i = NC - 1 - n;
+  for (int n = 0; n < nl; ++n) {
+    const int i = ch1 - 1 - n;
     mbar_wait(bar_ld, ph_ld, a.latch);
     ph_ld ^= 1;
     Gate gr;
@@ -593,7 +610,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_LO + ko, 16, 1024), vd, id_Z, 1);
       }
       umma_commit(bar_m1);
-      if (!safe && n + 1 < NC) load_qkg(i - 1);
+      if (!safe && n + 1 < nl) load_qkg(i - 1);
     }
     __syncwarp();
     mbar_wait(bar_m1, ph_m1, a.latch);
@@ -659,7 +676,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     fence_async_smem();
     sync_tc();
     if (tid == 0) {
-      if (safe && n + 1 < NC) load_qkg(i - 1);
+      if (safe && n + 1 < nl) load_qkg(i - 1);
       const uint32_t dob = base + 3 * L::RAW;
       constexpr uint32_t id_dv2 = idesc_bf16_f32(C, VT, true, true);
 #pragma unroll
@@ -693,7 +710,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     mbar_wait(bar_m2, ph_m2, a.latch);
     ph_m2 ^= 1;
     tc_fence_after();
-    if (tid == 0 && n + 1 < NC) load_dov(i - 1);  // dO and A (over v) are no longer read
+    if (tid == 0 && n + 1 < nl) load_dov(i - 1);  // dO and A (over v) are no longer read
     {  // dv epilogue
       float v[64];
       const int t = i * C + row;
@@ -716,7 +733,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     __syncthreads();
   }
   // dh0[:, tile] = G_0
-  if (a.dh0) {
+  if (a.dh0 && seg == 0) {
     tc_fence_after();
     float dv0v[32];
     for (int cb = half * HT; cb < (half + 1) * HT; cb += 32) {
@@ -734,19 +751,23 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
 // c_i = c_{i+1} + Q_{i+1} - K_i, with Q the forward walk's chunk sums of Qt X and K the chunk
 // sums of Kh Z (summed over value tiles and token halves).
 // ------------------------------------------------------------------------------------------
-// One block per (head, 32 key dims); its 8 warps each take a slice of the chunks: the slice sums
-// are exchanged in shared memory, then every warp walks its own slice from the right start.
+// One block per (head, 32 key dims, segment); its 8 warps each take a slice of the segment's
+// chunks: the slice sums are exchanged in shared memory, then every warp walks its own slice from
+// the right start.  Each segment's carry starts at its last chunk from rowsum(G_end * S_end) of
+// the states its walks used, so the recurrence telescopes within the segment.
 template <int NVT>
 __global__ void __launch_bounds__(256) carry_scan_kernel(const float* __restrict__ carry, const float* __restrict__ qx,
                                                          const float* __restrict__ kz, float* __restrict__ cout,
-                                                         int DK, int NC) {
+                                                         int DK, int NC, int seg_chunks) {
   __shared__ float slice_sum[8][32];
   const int dl = threadIdx.x & 31, s = threadIdx.x >> 5;
   const int bh = blockIdx.x / (DK / 32), d = (blockIdx.x % (DK / 32)) * 32 + dl;
-  const int G = (NC + 7) / 8, top = NC - 1 - s * G;  // slice s: chunks top, top - 1, ..., top - G + 1
-  // change of the carry from chunk i + 1 to chunk i
+  const int seg = blockIdx.y, nseg = gridDim.y;
+  const int ch0 = seg * seg_chunks, ch1 = min(NC, ch0 + seg_chunks);
+  const int G = (ch1 - ch0 + 7) / 8, top = ch1 - 1 - s * G;  // slice s: chunks top, top - 1, ... (>= ch0)
+  // change of the carry from chunk i + 1 to chunk i (none from beyond the segment)
   auto delta = [&](int i) {
-    float v = i < NC - 1 ? qx[((size_t)bh * NC + i + 1) * DK + d] : 0.f;
+    float v = i < ch1 - 1 ? qx[((size_t)bh * NC + i + 1) * DK + d] : 0.f;
 #pragma unroll
     for (int h = 0; h < 2 * NVT; ++h) v -= kz[(((size_t)bh * NVT * NC + (h >> 1) * NC + i) * 2 + (h & 1)) * DK + d];
     return v;
@@ -754,13 +775,13 @@ __global__ void __launch_bounds__(256) carry_scan_kernel(const float* __restrict
   float sum = 0.f;
 #pragma unroll 4
   for (int u = 0; u < G; ++u)
-    if (top - u >= 0) sum += delta(top - u);
+    if (top - u >= ch0) sum += delta(top - u);
   slice_sum[s][dl] = sum;
   __syncthreads();
-  float c = carry[(size_t)bh * DK + d];
+  float c = carry[((size_t)bh * nseg + seg) * DK + d];
   for (int t = 0; t < s; ++t) c += slice_sum[t][dl];
   for (int u = 0; u < G; ++u)
-    if (top - u >= 0) {
+    if (top - u >= ch0) {
       c += delta(top - u);
       cout[((size_t)bh * NC + top - u) * DK + d] = c;
     }
@@ -1060,11 +1081,12 @@ __global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   constexpr int per_head = DK / KT + DV / VT;
-  const int bh = blockIdx.x / per_head, role = blockIdx.x % per_head;
+  const int per_seg = a.n_bh * per_head;
+  const int seg = blockIdx.x / per_seg, bh = (blockIdx.x % per_seg) / per_head, role = blockIdx.x % per_head;
   if (role < DK / KT)
-    key_tile_body<DK, DV, ACC>(sm, mp, a, bh, role, bars, tmem);
+    key_tile_body<DK, DV, ACC>(sm, mp, a, bh, role, seg, bars, tmem);
   else
-    val_tile_body<DK, ACC>(sm, mp, a, bh, role - DK / KT, DV, bars, tmem);
+    val_tile_body<DK, ACC>(sm, mp, a, bh, role - DK / KT, DV, seg, bars, tmem);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -1083,11 +1105,12 @@ static cudaError_t launch_all(const BwdMaps& mp, const BwdArgs& a, int BH, cudaS
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k1<<<BH * (DK / KT + DV / VT), BT, BwdSmem<DK, DV>::ALLOC, st>>>(mp, a);
+  k1<<<BH * (DK / KT + DV / VT) * a.nseg, BT, BwdSmem<DK, DV>::ALLOC, st>>>(mp, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int NC = (a.T + C - 1) / C;
-  carry_scan_kernel<DV / VT><<<BH * (DK / 32), 256, 0, st>>>(a.ws_carry, a.ws_qx, a.ws_kz, a.ws_c, DK, NC);
+  carry_scan_kernel<DV / VT><<<dim3(BH * (DK / 32), a.nseg), 256, 0, st>>>(a.ws_carry, a.ws_qx, a.ws_kz, a.ws_c, DK,
+                                                                          NC, a.seg_chunks);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   k3<<<BH * (DK / KT) * NC, BT, CHK, st>>>(mp, a);
@@ -1101,11 +1124,30 @@ bool bwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype) {
   return encode_fn() != nullptr;
 }
 
+// Workspace parts, in order: Qt X chunk sums, forward part of dg, carry starts, Z^T parts, Kh Z
+// chunk sums, carries; with a sequence split also the segment states (forward, gradient) and the
+// segment decay products.
+static void bwd_parts(int BH, int T, int dk, int dv, size_t* sz, int* nseg, int* seg_chunks) {
+  plan_bwd_segments(BH * (dk / KT + dv / VT), T, nseg, seg_chunks);
+  const size_t NC = (T + C - 1) / C, ns = *nseg, f = sizeof(float);
+  sz[0] = align256((size_t)BH * NC * dk * f);
+  sz[1] = align256((size_t)BH * NC * C * dk * f);
+  sz[2] = align256((size_t)BH * ns * dk * f);
+  sz[3] = align256((size_t)BH * (dv / VT) * NC * dk * C * f);
+  sz[4] = align256((size_t)BH * (dv / VT) * NC * 2 * dk * f);
+  sz[5] = align256((size_t)BH * NC * dk * f);
+  sz[6] = ns > 1 ? align256((size_t)BH * ns * dk * dv * f) : 0;
+  sz[7] = sz[6];
+  sz[8] = ns > 1 ? align256((size_t)BH * ns * dk * f) : 0;
+}
+
 size_t bwd_workspace(int BH, int T, int dk, int dv) {
-  const size_t NC = (T + C - 1) / C;
-  return align256((size_t)BH * NC * dk * sizeof(float)) + align256((size_t)BH * NC * C * dk * sizeof(float)) +
-         align256((size_t)BH * dk * sizeof(float)) + align256((size_t)BH * (dv / VT) * NC * dk * C * sizeof(float)) +
-         align256((size_t)BH * (dv / VT) * NC * 2 * dk * sizeof(float)) + align256((size_t)BH * NC * dk * sizeof(float));
+  size_t sz[9];
+  int nseg, per;
+  bwd_parts(BH, T, dk, dv, sz, &nseg, &per);
+  size_t n = 0;
+  for (size_t x : sz) n += x;
+  return n;
 }
 
 template <int DK, int DV>
@@ -1139,14 +1181,26 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
   a.acc_ck = acc ? acc->ck : 0;
   a.acc_pv = acc ? acc->pv : 0;
   a.acc_cv = acc ? acc->cv : 0;
-  const size_t NC = (T + C - 1) / C;
-  a.ws_qx = static_cast<float*>(ws);
-  a.ws_part = a.ws_qx + align256((size_t)BH * NC * DK * sizeof(float)) / sizeof(float);
-  a.ws_carry = a.ws_part + align256((size_t)BH * NC * C * DK * sizeof(float)) / sizeof(float);
-  a.ws_z = a.ws_carry + align256((size_t)BH * DK * sizeof(float)) / sizeof(float);
-  a.ws_kz = a.ws_z + align256((size_t)BH * (DV / VT) * NC * DK * C * sizeof(float)) / sizeof(float);
-  a.ws_c = a.ws_kz + align256((size_t)BH * (DV / VT) * NC * 2 * DK * sizeof(float)) / sizeof(float);
+  size_t sz[9];
+  bwd_parts(BH, T, DK, DV, sz, &a.nseg, &a.seg_chunks);
+  float* p[9];
+  p[0] = static_cast<float*>(ws);
+  for (int j = 1; j < 9; ++j) p[j] = p[j - 1] + sz[j - 1] / sizeof(float);
+  a.ws_qx = p[0];
+  a.ws_part = p[1];
+  a.ws_carry = p[2];
+  a.ws_z = p[3];
+  a.ws_kz = p[4];
+  a.ws_c = p[5];
+  a.s_in = a.nseg > 1 ? p[6] : nullptr;
+  a.g_end = a.nseg > 1 ? p[7] : nullptr;
+  a.n_bh = BH;
   a.latch = device_error_latch();
+  if (a.nseg > 1) {
+    const cudaError_t e = segment_states(mp.q_all, mp.k_all, mp.g_all, mp.v, mp.dO, h0, dhT, p[6], p[7], p[8], BH, T,
+                                         DK, DV, a.nseg, a.seg_chunks, st_bh, st_row, st);
+    if (e != cudaSuccess) return e;
+  }
   return acc ? launch_all<DK, DV, true>(mp, a, BH, st) : launch_all<DK, DV, false>(mp, a, BH, st);
 }
 

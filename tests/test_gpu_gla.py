@@ -194,6 +194,33 @@ def test_fused_shapes_mixed_strong_gates():
     _run_fwd_bwd(inp, 64)
 
 
+def _bwd_workspace_bytes(BH, T, dk, dv, nseg):
+    """Size of the fused backward's workspace: six parts, plus the segment states when split."""
+    NC = -(-T // 64)
+    parts = [BH * NC * dk, BH * NC * 64 * dk, BH * nseg * dk, BH * (dv // 128) * NC * dk * 64,
+             BH * (dv // 128) * NC * 2 * dk, BH * NC * dk]
+    if nseg > 1:
+        parts += [BH * nseg * dk * dv, BH * nseg * dk * dv, BH * nseg * dk]
+    return sum(-(-4 * p // 256) * 256 for p in parts)
+
+
+@pytest.mark.parametrize("B,H,T,dv,nseg", [(2, 4, 64 * 40 + 17, 256, 4), (1, 4, 64 * 30, 128, 10)])
+def test_fused_backward_sequence_split(B, H, T, dv, nseg):
+    """Few heads: the backward's walks run as segments of several chunks (state entry from the
+    forward's segment scan, state gradient from the reverse one, the dg carry restarting per
+    segment).  Every gradient against the oracle, with initial and final states."""
+    assert gla.workspace_bytes("gla_chunk_bwd", B, H, T, 128, dv, 64, 1) == \
+        _bwd_workspace_bytes(B * H, T, 128, dv, nseg)
+    inp = make_gla_inputs(B, H, T, 128, dv, torch.bfloat16, seed=70 + dv, with_h0=True, with_dhT=True)
+    _run_fwd_bwd(inp, 64)
+
+
+def test_fused_backward_unsplit_workspace():
+    """Enough heads to fill the GPU: one segment, no segment states."""
+    assert gla.workspace_bytes("gla_chunk_bwd", 8, 4, 2048, 128, 256, 64, 1) == \
+        _bwd_workspace_bytes(32, 2048, 128, 256, 1)
+
+
 @pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128)])
 def test_fused_forward_long_walk(dk, dv):
     """Enough heads to fill the GPU (no sequence split), so one CTA walks every chunk of its head:
