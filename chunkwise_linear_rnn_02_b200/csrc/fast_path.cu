@@ -656,13 +656,9 @@ template <int DK, bool HILO, bool REV>
 static cudaError_t launch_state_pass(const CUtensorMap& mk, const CUtensorMap& mg, const CUtensorMap& mv,
                                      const FwdArgs& args, int BH, int dv, cudaStream_t st) {
   auto kern = fwd_state_kernel<DK, HILO, REV>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<DK, HILO>::ALLOC);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static bool attr_set[64] = {};
+  const cudaError_t e = ensure_smem_attr(kern, StateLayout<DK, HILO>::ALLOC, attr_set);
+  if (e != cudaSuccess) return e;
   dim3 grid(dv / DVT, BH, args.nseg - 1);
   kern<<<grid, NTHREADS, StateLayout<DK, HILO>::ALLOC, st>>>(mk, mg, mv, args);
   return cudaGetLastError();
@@ -704,11 +700,10 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
     }
   }
   auto kern = fwd_pipe_kernel<DK>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdPipeLayout<DK>::ALLOC);
+  static bool attr_set[64] = {};
+  {
+    const cudaError_t e = ensure_smem_attr(kern, FwdPipeLayout<DK>::ALLOC, attr_set);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   dim3 grid(dv / DVT, BH, a.nseg);
   kern<<<grid, PIPE_THREADS, FwdPipeLayout<DK>::ALLOC, st>>>(m[0], m[1], m[2], m[3], a);

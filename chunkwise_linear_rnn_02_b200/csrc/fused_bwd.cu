@@ -1098,12 +1098,11 @@ static cudaError_t launch_all(const BwdMaps& mp, const BwdArgs& a, int BH, cudaS
   static_assert(2 * CHK <= 228 * 1024, "two chunk CTAs per SM");
   auto k1 = bwd_fused_kernel<DK, DV, ACC>;
   auto k3 = bwd_chunk_kernel<DK, DV, ACC>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<DK, DV>::ALLOC);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, CHK);
+  static bool attr1[64] = {}, attr3[64] = {};
+  {
+    cudaError_t e = ensure_smem_attr(k1, BwdSmem<DK, DV>::ALLOC, attr1);
+    if (e == cudaSuccess) e = ensure_smem_attr(k3, CHK, attr3);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   k1<<<BH * (DK / KT + DV / VT) * a.nseg, BT, BwdSmem<DK, DV>::ALLOC, st>>>(mp, a);
   cudaError_t e = cudaGetLastError();

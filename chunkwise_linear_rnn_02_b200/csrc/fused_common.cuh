@@ -33,6 +33,19 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// Raise a kernel's dynamic shared-memory limit to `bytes`, once per device (the attribute belongs
+// to the kernel as loaded on the current device; `done` holds one flag per device ordinal).
+template <typename K>
+inline cudaError_t ensure_smem_attr(K kern, uint32_t bytes, bool (&done)[64]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+  return e;
+}
+
 // 3-D map over a [BH, T, D] bf16 tensor with box (box_d, 64 tokens, 1 head); tokens past T read
 // as zeros.
 inline bool make_map(CUtensorMap* m, const void* base, int BH, int T, int D, int box_d, bool swizzle128) {
