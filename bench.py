@@ -42,6 +42,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-heads", type=int, default=24, help="heads in the oracle's CPU sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-slices", type=int, default=E2E_PARTS,
+                    help="batch slices, each on its own stream, in the end-to-end measurement")
     ap.add_argument("--no-launch-count", action="store_true", help="skip the CUDA-profiler launch count")
     return ap.parse_args(argv)
 
@@ -281,13 +283,13 @@ def run_ours(args, cfg, name):
     step_ms, fwd_ms, bwd_ms = max_over_ranks([step_ms, fwd_ms, bwd_ms], dev)
 
     # end-to-end through the public API with host buffers: H2D inputs, fwd, bwd, D2H results.
-    # The batch goes through in E2E_PARTS slices of whole sequences, each on its own stream, so
+    # The batch goes through in --e2e-slices slices of whole sequences, each on its own stream, so
     # that one slice's host->device copy, another's kernels and a third's device->host copy
     # overlap (the sequences are independent; every byte still crosses PCIe inside the region).
     names_in = ["q", "k", "v", "g", "do"]
     host_in = {k: inp[k].pin_memory() for k in names_in}
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    parts = E2E_PARTS if cfg.B % E2E_PARTS == 0 else 1
+    parts = args.e2e_slices if args.e2e_slices > 0 and cfg.B % args.e2e_slices == 0 else 1
     rows = cfg.B // parts
     streams = [torch.cuda.Stream(device=dev) for _ in range(parts)]
     e2e_times = []
