@@ -433,7 +433,9 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
 }
 
 // ------------------------------------------------------------------------------------------
-// Value-tile CTA: reverse walk carrying G[:, tile] (fp32, TMEM); dv = Kh G_{i+1} + A^T dO.
+// Value-tile CTA: reverse walk carrying G[:, tile] (fp32, TMEM); dv = Kh G_{i+1} + A^T dO, formed
+// transposed (dv^T = G^T Kh^T + dO^T A: 128 value columns on the MMA's M axis, 64 tokens on N,
+// because an M = 64 MMA takes as long as an M = 128 one).
 // Qs, Kh, the G copy and A enter the MMAs as bf16 hi + lo pairs.  One array holds the queries of
 // both A and the G update: Qs = Qt / dec (then G <- dec (G + Qs^T dO)), or Qt itself in a chunk on
 // the exact path (then G <- dec G + Qt^T dO, the intra-chunk A computed exactly in fp32).
@@ -457,7 +459,7 @@ struct ValLayout {
   static constexpr uint32_t XB = QP_HI, XA = KH_HI;  // exact-path scratch (after the first MMA group)
   // v tile [64 x VT] for Z^T = G V^T: read by the first MMA group only, so it shares A's space
   static constexpr uint32_t VZ = AB_HI;
-  static constexpr uint32_t T_G = 0, T_A = VT, T_DV = VT + 64, T_Z = 2 * VT + 64;
+  static constexpr uint32_t T_G = 0, T_A = VT, T_DV = VT + 64, T_Z = 2 * VT + 64;  // dv^T takes 64 columns
   static_assert(C * VT * 2 <= DEC - AB_HI && T_Z + 64 <= 512, "v tile / TMEM columns");
   static_assert(STAGE % 1024 == 0, "stage alignment");
   static_assert(C * DK * 4 <= KH_HI - QP_HI && C * C * 4 <= GC_HI - KH_HI, "exact-path scratch");
@@ -477,7 +479,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   const bool row_owner = lane < 16;
   const int row = q4 * 16 + lane;   // row of an M=64 accumulator
   const int grow = q4 * 32 + lane;  // row of the M=128 G accumulator
-  constexpr int HT = VT / 2;        // G / dv columns per warp
+  constexpr int HT = VT / 2;        // G columns per warp
   uint64_t* bar_ld = bars + 0;  // q, k, g of a chunk
   uint64_t* bar_dv = bars + 1;  // dO, v of a chunk
   uint64_t* bar_m1 = bars + 3;
@@ -579,7 +581,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     if (tid == 0) {
       const uint32_t dob = base + 3 * L::RAW;
       constexpr uint32_t id_A = idesc_bf16_f32(C, C, false, false);
-      constexpr uint32_t id_dv = idesc_bf16_f32(C, VT, false, true);
+      constexpr uint32_t id_dv = idesc_bf16_f32(VT, C, true, false);  // dv^T = G^T Kh^T: value columns on M
       constexpr uint32_t id_G = idesc_bf16_f32(DK, VT, true, true);
 #pragma unroll
       for (int k = 0; k < DK / 16; ++k) {
@@ -590,9 +592,9 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         umma_bf16(tmem + L::T_A, qh, kl, id_A, 1);
         umma_bf16(tmem + L::T_A, ql, kh, id_A, 1);
         const uint64_t gh = desc_sw128(base + L::GC_HI + k * 2048, DK * 128, 1024);
-        umma_bf16(tmem + L::T_DV, kh, gh, id_dv, k > 0);
-        umma_bf16(tmem + L::T_DV, kh, desc_sw128(base + L::GC_LO + k * 2048, DK * 128, 1024), id_dv, 1);
-        umma_bf16(tmem + L::T_DV, kl, gh, id_dv, 1);
+        umma_bf16(tmem + L::T_DV, gh, kh, id_dv, k > 0);
+        umma_bf16(tmem + L::T_DV, desc_sw128(base + L::GC_LO + k * 2048, DK * 128, 1024), kh, id_dv, 1);
+        umma_bf16(tmem + L::T_DV, gh, kl, id_dv, 1);
       }
 #pragma unroll
       for (int k = 0; k < C / 16; ++k) {
@@ -678,12 +680,12 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     if (tid == 0) {
       if (safe && n + 1 < nl) load_qkg(i - 1);
       const uint32_t dob = base + 3 * L::RAW;
-      constexpr uint32_t id_dv2 = idesc_bf16_f32(C, VT, true, true);
+      constexpr uint32_t id_dv2 = idesc_bf16_f32(VT, C, true, true);  // dv^T += dO^T A
 #pragma unroll
       for (int k = 0; k < C / 16; ++k) {
         const uint64_t dd = desc_sw128(dob + k * 2048, C * 128, 1024);
-        umma_bf16(tmem + L::T_DV, desc_sw128(base + L::AB_HI + k * 2048, C * 128, 1024), dd, id_dv2, 1);
-        umma_bf16(tmem + L::T_DV, desc_sw128(base + L::AB_LO + k * 2048, C * 128, 1024), dd, id_dv2, 1);
+        umma_bf16(tmem + L::T_DV, dd, desc_sw128(base + L::AB_HI + k * 2048, C * 128, 1024), id_dv2, 1);
+        umma_bf16(tmem + L::T_DV, dd, desc_sw128(base + L::AB_LO + k * 2048, C * 128, 1024), id_dv2, 1);
       }
       umma_commit(bar_m2);
     }
@@ -711,22 +713,22 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     ph_m2 ^= 1;
     tc_fence_after();
     if (tid == 0 && n + 1 < nl) load_dov(i - 1);  // dO and A (over v) are no longer read
-    {  // dv epilogue
-      float v[64];
-      const int t = i * C + row;
-      for (int cb = half * HT; cb < (half + 1) * HT; cb += 64) {
-        tmem_ld32(tmem + L::T_DV + lane_off + cb, v);
-        tmem_ld32(tmem + L::T_DV + lane_off + cb + 32, v + 32);
-        tmem_ld_wait();
-        if (row_owner && t < T) {
-          if (ACC) {
-            float4* p = reinterpret_cast<float4*>(a.acc_v + ((size_t)bh * T + t) * a.acc_pv + a.acc_cv + c0 + cb);
+    {  // dv epilogue: row vcol of dv^T (value column c0 + vcol), tokens half*32 .. half*32+31; a
+       // warp's store covers 32 adjacent value columns of one token
+      float v[32];
+      const int vcol = q4 * 32 + lane, t0 = i * C + half * 32;
+      tmem_ld32(tmem + L::T_DV + lane_off + half * 32, v);
+      tmem_ld_wait();
+      if (ACC) {
+        float* p = a.acc_v + ((size_t)bh * T + t0) * a.acc_pv + a.acc_cv + c0 + vcol;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) p[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-          } else {
-            store_row_global_bf16(a.dv + ((size_t)bh * T + t) * DV + c0 + cb, v);
-          }
-        }
+        for (int c = 0; c < 32; ++c)
+          if (t0 + c < T) p[(size_t)c * a.acc_pv] = v[c];
+      } else {
+        __nv_bfloat16* p = a.dv + ((size_t)bh * T + t0) * DV + c0 + vcol;
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (t0 + c < T) p[(size_t)c * DV] = __float2bfloat16_rn(v[c]);
       }
     }
     tc_fence_before();
