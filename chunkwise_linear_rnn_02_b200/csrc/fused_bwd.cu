@@ -181,7 +181,6 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   };
   // Element (token j, dim d) of a raw tile at shared-memory offset off (TMA 128-byte swizzle).
   auto raw = [&](uint32_t off, int j, int d) { return bf2f(sm + off + sw128(j, d)); };
-  auto raw2 = [&](uint32_t off, int j, int d) { return *reinterpret_cast<const uint32_t*>(sm + off + sw128(j, d)); };
   // dA (masked, as the MMAs see it: hi + lo) at (j, r).
   auto dA_at = [&](int j, int r) { return raw(L::DA_HI, j, r) + raw(L::DA_LO, j, r); };
   // Gate run of the chunk in part-B buffer b: run products into TOT[b], decays into DEC[b].

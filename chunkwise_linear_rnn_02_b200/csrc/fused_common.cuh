@@ -112,20 +112,6 @@ __device__ __forceinline__ void store_row_sw128(uint8_t* tile, int r, const floa
   }
 }
 
-// Store 64 fp32 values as bf16 to global (16-byte aligned destination).
-__device__ __forceinline__ void store_row_global_bf16(__nv_bfloat16* dst, const float* v) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int cc = 0; cc < 8; ++cc) {
-    uint4 w;
-    w.x = pack2(v[8 * cc + 0], v[8 * cc + 1]);
-    w.y = pack2(v[8 * cc + 2], v[8 * cc + 3]);
-    w.z = pack2(v[8 * cc + 4], v[8 * cc + 5]);
-    w.w = pack2(v[8 * cc + 6], v[8 * cc + 7]);
-    d[cc] = w;
-  }
-}
-
 // hi + lo bf16 split of a pair of fp32 values: hi = bf16(x), lo = bf16(x - hi).
 __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
   hi = pack2(a, b);
