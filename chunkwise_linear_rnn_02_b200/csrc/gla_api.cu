@@ -100,6 +100,7 @@ struct SplitFwdWs {
   void* fws;
 };
 size_t carve_split_fwd(Carve& c, int BH, int T, int dk, int dv, SplitFwdWs* w) {
+  (void)dk;  // key blocks are gathered one at a time, so no part depends on d_k
   const size_t rows = (size_t)BH * T;
   SplitFwdWs x;
   x.q = c.take<bf16>(rows * kSplitK);
