@@ -302,9 +302,39 @@ size_t carve_gsa_fwd(Carve& c, int BH, int T, int dk, int dv, int m, int chunk, 
   return c.used;
 }
 
+// GSA's second pass (queries p, keys phi, values v, slot gates on its key axis) on the fused
+// backward: the m slots zero-padded to one 128-wide key block.  Exact: padded dimensions have zero
+// keys, queries, gates (decay 1) and states, so they add nothing to any output of the m real ones.
+bool gsa_pass2_fused_ok(int BH, int T, int m, int dv, int chunk, int dtype) {
+  return m <= 128 && m % 8 == 0 && gla::fast::bwd_supported(BH, T, 128, dv, chunk, dtype);
+}
+struct GsaFusedWs {
+  bf16 *p, *phi, *g;                 // [BH*T][128] padded operands
+  float *dq, *dk, *dg, *dv;          // fp32 outputs: [BH*T][128] (dp, dphi2, dg2) and [BH*T][dv]
+  float *h0, *dhT, *dh0;             // [BH][128][dv] padded states
+  void* ws;                          // the fused backward's workspace
+};
+void carve_gsa_fused(Carve& c, int BH, int T, int dv, GsaFusedWs* w) {
+  const size_t rows = (size_t)BH * T, st = (size_t)BH * 128 * dv;
+  GsaFusedWs x;
+  x.p = c.take<bf16>(rows * 128);
+  x.phi = c.take<bf16>(rows * 128);
+  x.g = c.take<bf16>(rows * 128);
+  x.dq = c.take<float>(rows * 128);
+  x.dk = c.take<float>(rows * 128);
+  x.dg = c.take<float>(rows * 128);
+  x.dv = c.take<float>(rows * dv);
+  x.h0 = c.take<float>(st);
+  x.dhT = c.take<float>(st);
+  x.dh0 = c.take<float>(st);
+  x.ws = c.take<char>(gla::fast::bwd_workspace(BH, T, 128, dv));
+  if (w) *w = x;
+}
+
 struct GsaBwdWs {
   float *S1, *o1, *S2, *dS2, *hT2, *db, *dp, *dphi2, *dg2, *do1, *dS1, *hT1;
   void* p;
+  GsaFusedWs f;
 };
 size_t carve_gsa_bwd(Carve& c, int BH, int T, int dk, int dv, int m, int chunk, int dtype, GsaBwdWs* w) {
   const size_t NC = gla::num_chunks(T, chunk);
@@ -323,6 +353,7 @@ size_t carve_gsa_bwd(Carve& c, int BH, int T, int dk, int dv, int m, int chunk, 
   x.dS1 = c.take<float>((size_t)BH * NC * m * dk);
   x.hT1 = c.take<float>((size_t)BH * m * dk);
   x.p = (void*)c.take<char>(tm * esize(dtype));
+  if (gsa_pass2_fused_ok(BH, T, m, dv, chunk, dtype)) carve_gsa_fused(c, BH, T, dv, &x.f);
   if (w) *w = x;
   return c.used;
 }
@@ -368,11 +399,35 @@ int gsa_bwd_impl(const TI* q, const TI* k, const TI* v, const TI* phi, const TI*
                                         st)));
   GLA_CUDA(gk::softmax_fwd<TI>(w.o1, p, nullptr, (long)BH * T, m, st));
   // pass 2 backward (queries p, keys phi, values v)
-  GLA_CUDA(gk::state_fwd<TI>(s2, phi, v, g, h02, 0, w.S2, w.hT2, 0, st));
-  GLA_CUDA((gk::dstate_bwd<TI, TI>(s2, p, g, dO, dhT2, 0, w.dS2, dh02, 0, st)));
-  GLA_CUDA((gk::bwd_dqdk<TI, TI, float>(s2, p, phi, v, g, dO, w.S2, w.dS2, w.dp, w.dphi2, nullptr, w.db, st)));
-  GLA_CUDA((gk::bwd_dv<TI, TI, TI>(s2, p, phi, g, dO, w.dS2, dv, st)));
-  GLA_CUDA(gk::dg<float>(s2, w.db, w.hT2, dhT2, 0, nullptr, w.dg2, st));
+  bool pass2_done = false;
+  if constexpr (sizeof(TI) == 2) {
+    if (gsa_pass2_fused_ok(BH, T, m, dvd, C, GLA_DTYPE_BF16)) {
+      const GsaFusedWs& f = w.f;
+      const long long rows = (long long)BH * T, sz = (long long)m * dvd, sp = 128LL * dvd;
+      GLA_CUDA(gla::split::copy_cols(p, m, f.p, 128, rows, m, 128, st));
+      GLA_CUDA(gla::split::copy_cols(phi, m, f.phi, 128, rows, m, 128, st));
+      GLA_CUDA(gla::split::copy_cols(g, m, f.g, 128, rows, m, 128, st));
+      if (h02) GLA_CUDA(gla::split::copy_cols(h02, sz, f.h0, sp, BH, sz, sp, st));
+      if (dhT2) GLA_CUDA(gla::split::copy_cols(dhT2, sz, f.dhT, sp, BH, sz, sp, st));
+      const gla::fast::BwdAccum acc{f.dq, f.dk, f.dg, f.dv, 128, 0, dvd, 0};
+      GLA_CUDA(gla::fast::bwd(f.p, f.phi, v, f.g, h02 ? f.h0 : nullptr, dO, dhT2 ? f.dhT : nullptr, nullptr,
+                              nullptr, nullptr, nullptr, dh02 ? f.dh0 : nullptr, BH, T, 128, dvd, f.ws, st, -1, -1,
+                              &acc));
+      GLA_CUDA(gla::split::copy_cols(f.dq, 128, w.dp, m, rows, m, m, st));
+      GLA_CUDA(gla::split::copy_cols(f.dk, 128, w.dphi2, m, rows, m, m, st));
+      GLA_CUDA(gla::split::copy_cols(f.dg, 128, w.dg2, m, rows, m, m, st));
+      GLA_CUDA(gla::split::to_bf16(f.dv, dv, rows * dvd, st));
+      if (dh02) GLA_CUDA(gla::split::copy_cols(f.dh0, sp, dh02, sz, BH, sz, sz, st));
+      pass2_done = true;
+    }
+  }
+  if (!pass2_done) {
+    GLA_CUDA(gk::state_fwd<TI>(s2, phi, v, g, h02, 0, w.S2, w.hT2, 0, st));
+    GLA_CUDA((gk::dstate_bwd<TI, TI>(s2, p, g, dO, dhT2, 0, w.dS2, dh02, 0, st)));
+    GLA_CUDA((gk::bwd_dqdk<TI, TI, float>(s2, p, phi, v, g, dO, w.S2, w.dS2, w.dp, w.dphi2, nullptr, w.db, st)));
+    GLA_CUDA((gk::bwd_dv<TI, TI, TI>(s2, p, phi, g, dO, w.dS2, dv, st)));
+    GLA_CUDA(gk::dg<float>(s2, w.db, w.hT2, dhT2, 0, nullptr, w.dg2, st));
+  }
   // slot softmax Jacobian
   GLA_CUDA(gk::softmax_bwd(w.o1, w.dp, w.do1, (long)BH * T, m, st));
   // pass 1 backward with roles exchanged

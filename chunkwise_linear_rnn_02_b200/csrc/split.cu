@@ -45,6 +45,20 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__
   }
 }
 
+// dst[r][c] = src[r][c] for c < ncols, 0 for ncols <= c < dst_cols (16-byte vectors of 8 bf16 / 4 fp32)
+template <typename T>
+__global__ void copy_kernel(const T* __restrict__ src, long long src_pitch, T* __restrict__ dst, long long dst_pitch,
+                            long long rows, long long ncols, long long dst_cols) {
+  constexpr int V = 16 / sizeof(T);
+  const long long vpr = dst_cols / V, n = rows * vpr;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const long long r = e / vpr, c = (e % vpr) * V;
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (c < ncols) x = *reinterpret_cast<const uint4*>(src + r * src_pitch + c);
+    *reinterpret_cast<uint4*>(dst + r * dst_pitch + c) = x;
+  }
+}
+
 int grid_for(long long items) {
   const long long blocks = (items + 255) / 256, cap = 148LL * 16;
   return (int)(blocks < 1 ? 1 : blocks > cap ? cap : blocks);
@@ -61,6 +75,20 @@ cudaError_t gather_cols(const bf16* src, bf16* dst, long long rows, int pitch, i
 cudaError_t add_cols(const float* part, float* acc, long long rows, int ncols, int acc_pitch, int col0,
                      cudaStream_t st) {
   add_kernel<<<grid_for(rows * (ncols / 4)), 256, 0, st>>>(part, acc, rows, ncols, acc_pitch, col0);
+  return cudaGetLastError();
+}
+
+cudaError_t copy_cols(const bf16* src, long long src_pitch, bf16* dst, long long dst_pitch, long long rows,
+                      long long ncols, long long dst_cols, cudaStream_t st) {
+  copy_kernel<bf16><<<grid_for(rows * (dst_cols / 8)), 256, 0, st>>>(src, src_pitch, dst, dst_pitch, rows, ncols,
+                                                                     dst_cols);
+  return cudaGetLastError();
+}
+
+cudaError_t copy_cols(const float* src, long long src_pitch, float* dst, long long dst_pitch, long long rows,
+                      long long ncols, long long dst_cols, cudaStream_t st) {
+  copy_kernel<float><<<grid_for(rows * (dst_cols / 4)), 256, 0, st>>>(src, src_pitch, dst, dst_pitch, rows, ncols,
+                                                                      dst_cols);
   return cudaGetLastError();
 }
 

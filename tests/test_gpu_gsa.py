@@ -41,6 +41,25 @@ def test_gsa_fwd_bwd(dtype, shape):
     assert gla.device_error() == 0
 
 
+@pytest.mark.parametrize("shape", [(1, 2, 150, 128, 128, 64), (2, 1, 100, 64, 256, 32)])
+def test_gsa_bwd_second_pass_on_fused_kernels(shape):
+    """bf16, d_v in {128, 256}: the second pass's backward runs on the fused kernels with its m slots
+    zero-padded to a 128-wide key block; every gradient against the oracle, with initial and final
+    states for both passes."""
+    B, H, T, dk, dv, m = shape
+    tol = tol_for(torch.bfloat16)
+    inp = make_gsa_inputs(B, H, T, dk, dv, m, torch.bfloat16, seed=19)
+    h1, h2, d1, d2 = _states(B, H, dk, dv, m, 20)
+    d = cuda(inp)
+    grads = gla.gsa_bwd(d["q"], d["k"], d["v"], d["phi"], d["g"], d["do"], h0_1=h1.cuda(), h0_2=h2.cuda(),
+                        dhT1=d1.cuda(), dhT2=d2.cuda())
+    a = [f64(inp[n]) for n in ["q", "k", "v", "phi", "g"]]
+    ref = O.gsa_bwd(*a, f64(h1), f64(h2), f64(inp["do"]), f64(d1), f64(d2))
+    for name, x, r in zip(["dq", "dk", "dv", "dphi", "dg", "dh0_1", "dh0_2"], grads, ref):
+        assert_close(name, x, r, tol)
+    assert gla.device_error() == 0
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_gsa_decode_continues_forward(dtype):
     B, H, T, n, dk, dv, m = 1, 2, 100, 12, 64, 64, 32
