@@ -276,8 +276,9 @@ int copy_or_zero(float* dst, const float* src, size_t n, cudaStream_t st) {
 }
 
 // ----------------------------------------------------------------------------------------
-// GSA (generic passes; pass 1 is the key-gated pass with roles exchanged: its state is kept
-// transposed, [m x dk], so that the slot axis is the gated row axis)
+// GSA.  Pass 1 runs on the generic kernels as the key-gated pass with roles exchanged (its state
+// kept transposed, [m x dk], so that the slot axis is the gated row axis); pass 2, a plain
+// key-gated GLA, runs on the fused kernels where they serve the shape, else on the generic ones.
 // ----------------------------------------------------------------------------------------
 struct GsaFwdWs {
   float *S1, *o1, *S2;
