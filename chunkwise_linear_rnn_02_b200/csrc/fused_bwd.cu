@@ -24,6 +24,10 @@
 //      every chunk;
 //   3. one CTA per (head, 64 key dimensions, chunk), all independent: dk and the rest of dg
 //      from Z^T, a recomputed dA, the forward walk's part and c_i.
+// With few heads the chunks are cut into segments, each walked by its own key and value tiles:
+// state-only passes and scans first give every segment its entry state S and its end gradient G
+// (segment_states), and each segment's carry starts from rowsum(G_end * S_end) of the states its
+// own walks used.
 // States live in TMEM as fp32 accumulators; their bf16 hi / lo copies in shared memory feed the
 // MMAs.  A chunk that keeps less than e^-40 of its state in some dimension computes its
 // intra-chunk terms exactly in fp32 (CUDA cores) instead of through the scaled operands.  A
@@ -81,7 +85,8 @@ struct BwdArgs {
 //   dg_t = c_i + sum_{r<tau} Kh_r Z_r + sum_{j>=tau} Qt_j X_j
 //              + sum_{r<tau} ( k_r dk^intra_r - q_r dq^intra_r )        (intra terms without j = r)
 //   c_i  = e^{gamma_i} rowsum(G_{i+1} * S_i), carried backwards over chunk boundaries as
-//   c_{N-1} = rowsum(dhT * hT) - sum_r (Kh Z)_{N-1},  c_i = c_{i+1} + sum_j (Qt X)_{i+1} - sum_r (Kh Z)_i.
+//   c_{N-1} = rowsum(dhT * hT) - sum_r (Kh Z)_{N-1},  c_i = c_{i+1} + sum_j (Qt X)_{i+1} - sum_r (Kh Z)_i
+//   (per segment when the sequence is split: G_end * S_end of the segment in place of dhT * hT).
 // The forward walk writes the Qt X and q dq^intra parts (chunk-local, fp32) and the chunk sums of
 // Qt X into the workspace; the value tiles write the chunk sums of Kh Z, the carry scan forms every
 // c_i and the chunk kernel adds the rest.  The chunk sums use Qt and Kh as the G and S updates see
