@@ -82,3 +82,46 @@ def test_chunk_local_gate_gradient_with_segment_carries(segments):
                 dg[t] = c[i] + pre + suf
         scale = np.abs(dg_ref[0, h]).max()
         np.testing.assert_allclose(dg, dg_ref[0, h], rtol=0, atol=1e-10 * scale)
+
+
+def test_segment_scans_reproduce_the_boundary_states():
+    """The sequence split's two affine scans: segment-local states from zero (the forward one from
+    h0 in the first segment, the reverse one from dhT in the last) and the segments' decay
+    products Gamma compose to the exact state entering every segment and the exact dL/dS at the
+    end of every segment."""
+    inp = make_gla_inputs(1, 1, 64 * 7 + 9, 4, 3, torch.float32, seed=6, with_h0=True, with_dhT=True)
+    a = {n: np.asarray(inp[n], dtype=np.float64)[0, 0] for n in ["q", "k", "v", "g", "do", "h0", "dhT"]}
+    T = a["q"].shape[0]
+    NC = -(-T // C)
+    S, G, B, gam = _chunk_terms(a["q"], a["k"], a["v"], a["g"], a["h0"], a["do"], a["dhT"])
+    per = 3
+    segs = [(s0, min(NC, s0 + per)) for s0 in range(0, NC, per)]  # chunk ranges [s0, s1)
+    ns = len(segs)
+    Gam = [np.prod([np.exp(gam[i]) for i in range(s0, s1)], axis=0) for s0, s1 in segs]
+
+    def walk_fwd(s0, s1, start):
+        s = start.copy()
+        for t in range(s0 * C, min(T, s1 * C)):
+            s = np.exp(a["g"][t])[:, None] * s + np.outer(a["k"][t], a["v"][t])
+        return s
+
+    def walk_rev(s0, s1, end):
+        x = end.copy()
+        for i in range(s1 - 1, s0 - 1, -1):
+            ts = range(i * C, min(T, (i + 1) * C))
+            x = np.exp(gam[i])[:, None] * x + sum(np.outer(a["q"][t] * np.exp(B[t]), a["do"][t]) for t in ts)
+        return x
+
+    zero = np.zeros_like(a["h0"])
+    s_in = [a["h0"]]
+    for s in range(ns - 1):  # S_in(s+1) = Gamma_s * S_in(s) + S_local(s), S_local(0) from h0
+        local = walk_fwd(*segs[s], a["h0"] if s == 0 else zero)
+        s_in.append(local if s == 0 else Gam[s][:, None] * s_in[s] + local)
+    g_end = [None] * ns
+    g_end[ns - 1] = a["dhT"]
+    for s in range(ns - 2, -1, -1):  # G_end(s) = Gamma_{s+1} * G_end(s+1) + G_local(s+1)
+        local = walk_rev(*segs[s + 1], a["dhT"] if s + 1 == ns - 1 else zero)
+        g_end[s] = local if s + 1 == ns - 1 else Gam[s + 1][:, None] * g_end[s + 1] + local
+    for s, (s0, s1) in enumerate(segs):
+        np.testing.assert_allclose(s_in[s], S[s0], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(g_end[s], G[s1], rtol=1e-12, atol=1e-12)
