@@ -2,22 +2,27 @@
 """Benchmark of the chunkwise GLA operator: forward + backward on one B200 per rank.
 
 One step = gla_chunk_fwd then gla_chunk_bwd (the whole hot path) over one synthetic batch of the
-340M-model layer shape (B=8, H=4, T=2048, d_k=128, d_v=256, chunk 64, bf16), inputs resident in
-HBM.  L2 is flushed (256 MiB memset) between steps, outside the per-step CUDA events.
+1.3B-model layer shape (B=8, H=4, T=2048, d_k=256, d_v=512, chunk 64, bf16; the largest
+forward+backward workload), inputs resident in HBM.  L2 is flushed (256 MiB memset) between
+steps, outside the per-step CUDA events.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
 Prints ONE JSON line on rank 0.  With N > 1 (torchrun, one rank per GPU) every rank runs the same
 per-GPU workload on its own batch (weak scaling; the heads are independent, so there is no data
 exchange); the step time is the max over ranks and `value` counts the tokens of all ranks.
+At N = 1 the line also carries, under `extra`, the other timed workloads: the 340M-model shape
+(forward + backward), the long sequence (forward over 32768 tokens, then the microseconds per
+gla_recurrent_step call over 256 decode steps) and GSA with 64 slots (forward + backward).
 `--impl reference` times the fp64 CPU oracle (the only other implementation of this operator)
-on rank 0, on a bounded sample of the same workload.
+on rank 0, on a bounded sample of the same workload, spread over the host cores.
 """
 from __future__ import annotations
 
 import argparse
 import datetime
 import json
+import multiprocessing
 import os
 import statistics
 import subprocess
@@ -30,17 +35,23 @@ sys.path.insert(0, ROOT)
 METRIC = "GLA chunk fwd+bwd tokens/s and % of roofline, 1 B200, vs host oracle"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 E2E_PARTS = 4  # batch slices (each on its own stream) in the end-to-end measurement
+GATE_DESC = {"gla": "g=logsigmoid(N(0,1))/16", "gsa": "g=logsigmoid(N(0,1))/8"}
 
 
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="gla_340m", choices=["gla_340m", "gla_1p3b"])
-    ap.add_argument("--cpu-heads", type=int, default=24, help="heads in the oracle's CPU sample")
+    ap.add_argument("--workload", default="gla_1p3b", choices=["gla_1p3b", "gla_340m"])
+    ap.add_argument("--cpu-tokens", type=int, default=512,
+                    help="tokens per head (a prefix of the sequence) in the oracle's cpu_baseline sample")
+    ap.add_argument("--ref-tokens", type=int, default=128,
+                    help="tokens per head in each step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' figures")
+    ap.add_argument("--extra-steps", type=int, default=10)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--e2e-slices", type=int, default=E2E_PARTS,
                     help="batch slices, each on its own stream, in the end-to-end measurement")
@@ -61,7 +72,11 @@ def load_peaks():
 
 
 def algorithmic(cfg):
-    """Compulsory bytes and algorithmic FLOPs of one fwd and one bwd call (per call, all heads)."""
+    """Compulsory bytes and algorithmic FLOPs of one GLA fwd and one bwd call (per call, all heads).
+
+    Bytes: the forward reads q, k, g, v and writes o and the fp32 final state; the backward reads
+    q, k, g, v, dO and writes dq, dk, dg, dv.  FLOPs: the chunk form's contractions (causal half of
+    the intra-chunk products)."""
     e = 2 if cfg.dtype.is_floating_point and cfg.dtype.itemsize == 2 else 4
     th = cfg.B * cfg.H * cfg.T
     dk, dv, C = cfg.dk, cfg.dv, cfg.chunk
@@ -72,12 +87,37 @@ def algorithmic(cfg):
     return fwd_bytes, bwd_bytes, fwd_flops, bwd_flops
 
 
+def gsa_algorithmic(cfg):
+    """Compulsory bytes and FLOPs of one GSA fwd and bwd call: both passes' contractions; the
+    forward reads q, k, v, phi, g and writes o and both fp32 final states, the backward reads
+    q, k, v, phi, g, dO and writes dq, dk, dv, dphi, dg."""
+    th = cfg.B * cfg.H * cfg.T
+    dk, dv, m, C = cfg.dk, cfg.dv, cfg.m, cfg.chunk
+    fwd_bytes = th * (2 * dk + dv + 2 * m) * 2 + th * dv * 2 + cfg.B * cfg.H * (dk * m + m * dv) * 4
+    bwd_bytes = th * (2 * dk + 2 * dv + 2 * m) * 2 + th * (2 * dk + dv + 2 * m) * 2
+
+    def f(a, b):
+        return 4 * a * b + C * (a + b), 8 * a * b + C * (3 * a + 2 * b)
+
+    (f1, b1), (f2, b2) = f(dk, m), f(m, dv)
+    return fwd_bytes, bwd_bytes, th * (f1 + f2), th * (b1 + b2)
+
+
+def roofline_ms(nbytes, flops, peaks):
+    return 1e3 * max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+
+
 def workload_desc(cfg, name):
     return {"workload": f"{name}: GLA fwd+bwd B={cfg.B} H={cfg.H} T={cfg.T} d_k={cfg.dk} d_v={cfg.dv} "
-                        f"chunk={cfg.chunk} bf16, q,k,v,dO~N(0,1), q*d_k^-0.5, g=logsigmoid(N(0,1))/16, h0=0",
+                        f"chunk={cfg.chunk} bf16, q,k,v,dO~N(0,1), q*d_k^-0.5, {GATE_DESC['gla']}, h0=0",
             "B": cfg.B, "H": cfg.H, "T": cfg.T, "d_k": cfg.dk, "d_v": cfg.dv, "chunk": cfg.chunk,
             "tokens_per_step_per_gpu": cfg.B * cfg.T,
             "l2": "flushed between steps (256 MiB memset outside the per-step events)"}
+
+
+def config_desc(cfg, name, world):
+    """The `config` object of both arms' JSON lines (identical for the same workload and N)."""
+    return dict(workload_desc(cfg, name), parallelism=f"replicas x{world} (independent heads)")
 
 
 # ---------------------------------------------------------------------------------------------
@@ -141,46 +181,95 @@ def gpu_id_for_smi(dev_index):
 
 
 # ---------------------------------------------------------------------------------------------
-# CPU oracle timing (cpu_baseline leg and the reference arm)
+# CPU oracle timing (cpu_baseline leg and the reference arm), over the host cores
 # ---------------------------------------------------------------------------------------------
-def time_oracle(cfg, n_heads, seed=0):
-    """Time the fp64 oracle fwd + bwd on the first n_heads heads of the workload; 1 thread."""
-    import numpy as np
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_piece(a):
+    """One head of the oracle's fp64 fwd + bwd, single-threaded (runs in a pool worker)."""
     from threadpoolctl import threadpool_limits
 
     import oracle as O
-    from chunkwise_linear_rnn_02_b200.inputs import make_gla_inputs
-
-    nb = max(1, (n_heads + cfg.H - 1) // cfg.H)
-    inp = make_gla_inputs(nb, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.dtype, seed=seed)
-    a = {k: v.reshape(nb * cfg.H, 1, cfg.T, -1)[:n_heads].double().numpy() for k, v in inp.items()}
     with threadpool_limits(limits=1):
+        if a is None:  # warm-up: imports done, nothing timed
+            return 0.0
         t0 = time.perf_counter()
         O.gla_fwd(a["q"], a["k"], a["v"], a["g"])
         O.gla_bwd(a["q"], a["k"], a["v"], a["g"], None, a["do"])
-        dt = time.perf_counter() - t0
-    tokens = n_heads * cfg.T / cfg.H  # a token of the workload carries H heads
-    return dt, tokens / dt, np
+        return time.perf_counter() - t0
+
+
+class OraclePool:
+    """A spawn-started process pool (safe next to a CUDA context) running oracle head pieces."""
+
+    def __init__(self, workers):
+        self.workers = max(1, workers)
+        self.pool = multiprocessing.get_context("spawn").Pool(self.workers)
+        self.pool.map(_oracle_piece, [None] * self.workers)
+
+    def pieces(self, cfg, n_heads, tokens, seed):
+        from chunkwise_linear_rnn_02_b200.inputs import make_gla_inputs
+
+        inp = make_gla_inputs(n_heads, 1, tokens, cfg.dk, cfg.dv, cfg.dtype, seed=seed)
+        return [{n: inp[n][h:h + 1].double().numpy() for n in ["q", "k", "v", "g", "do"]} for h in range(n_heads)]
+
+    def time(self, pieces):
+        """Wall time of all pieces spread over the workers, and the summed single-thread times."""
+        t0 = time.perf_counter()
+        per = self.pool.map(_oracle_piece, pieces, chunksize=1)
+        return time.perf_counter() - t0, sum(per)
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def cpu_baseline(cfg, name, tokens):
+    """The oracle on min(B*H, host cores) heads x the first `tokens` tokens, one process per core."""
+    heads = min(cfg.B * cfg.H, host_cores())
+    tokens = min(tokens, cfg.T)
+    pool = OraclePool(heads)
+    try:
+        wall, cpu_s = pool.time(pool.pieces(cfg, heads, tokens, seed=7))
+    finally:
+        pool.close()
+    tok = heads * tokens / cfg.H  # a token of the workload carries H heads
+    return {"value": tok / wall, "unit": "tokens/s", "cores": heads, "kind": "oracle",
+            "sample": f"{heads} of {cfg.B * cfg.H} heads x the first {tokens} of {cfg.T} tokens of {name}, "
+                      f"fwd+bwd, float64 numpy, one spawn process per core (1 BLAS thread each), wall {wall:.2f} s, "
+                      f"{cpu_s:.1f} CPU-s; tokens = heads*tokens/H",
+            "single_thread_value": tok / cpu_s, "host_cores": host_cores()}
 
 
 def run_reference(args, cfg, name):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if int(os.environ.get("RANK", "0")) != 0:
         return
+    heads = min(cfg.B * cfg.H, host_cores())
+    tokens = min(args.ref_tokens, cfg.T)
+    pool = OraclePool(heads)
     steps = []
-    for i in range(args.warmup + args.steps):
-        dt, _, _ = time_oracle(cfg, 1, seed=i)
-        if i >= args.warmup:
-            steps.append(dt)
+    try:
+        for i in range(args.warmup + args.steps):
+            wall, _ = pool.time(pool.pieces(cfg, heads, tokens, seed=100 + i))
+            if i >= args.warmup:
+                steps.append(wall)
+    finally:
+        pool.close()
     ms = 1e3 * statistics.mean(steps)
-    tokens = cfg.T / cfg.H
-    value = tokens / (ms / 1e3)
-    sample = f"1 of {cfg.B * cfg.H} heads per step (T={cfg.T}), fwd+bwd, float64 numpy, 1 thread"
+    value = heads * tokens / cfg.H / (ms / 1e3)
+    sample = (f"{heads} of {cfg.B * cfg.H} heads x {tokens} of {cfg.T} tokens per step, fwd+bwd, float64 numpy, "
+              f"one spawn process per core (1 BLAS thread each); tokens = heads*tokens/H")
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_desc(cfg, name),
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_desc(cfg, name, world),
             "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": heads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -220,6 +309,100 @@ def traffic_from_profiles(kernel_key):
                 except (ValueError, IndexError):
                     return None
     return None
+
+
+def time_pair(first, second, steps, warmup, flush):
+    """Mean CUDA-event times (ms) of first() and second() over `steps` steps, L2 flushed between."""
+    import torch
+
+    for _ in range(max(3, warmup)):
+        first()
+        second()
+        flush.zero_()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        evs[i][0].record()
+        first()
+        evs[i][1].record()
+        second()
+        evs[i][2].record()
+        flush.zero_()
+    torch.cuda.synchronize()
+    a = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+    b = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
+    return a, b
+
+
+def extra_workloads(args, dev, flush, peaks):
+    """The other timed workloads, each with its own roofline (same device-timing rules)."""
+    import torch
+
+    from chunkwise_linear_rnn_02_b200 import binding as gla
+    from chunkwise_linear_rnn_02_b200.inputs import CONFIGS, make_gla_inputs, make_gsa_inputs
+
+    out = {}
+    steps = args.extra_steps
+    # the 340M-model shape (or the 1.3B one when that is not the main workload)
+    other = "gla_340m" if args.workload != "gla_340m" else "gla_1p3b"
+    cfg = CONFIGS[other]
+    d = {k: v.to(dev) for k, v in make_gla_inputs(cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.dtype, seed=1).items()}
+    f_ms, b_ms = time_pair(lambda: gla.chunk_fwd(d["q"], d["k"], d["v"], d["g"], chunk=cfg.chunk),
+                           lambda: gla.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["do"], chunk=cfg.chunk),
+                           steps, 3, flush)
+    fb, bb, ff, bf = algorithmic(cfg)
+    roof = roofline_ms(fb + bb, ff + bf, peaks)
+    out[other] = {"what": workload_desc(cfg, other)["workload"], "fwd_ms": f_ms, "bwd_ms": b_ms,
+                  "step_ms": f_ms + b_ms, "tokens_per_s": cfg.B * cfg.T / ((f_ms + b_ms) / 1e3),
+                  "roofline_ms": roof, "pct_of_roofline": 100 * roof / (f_ms + b_ms), "steps": steps}
+    del d
+    # the long sequence: forward over T tokens, then 256 decode steps from its final state
+    cfg = CONFIGS["gla_long"]
+    n_dec = 256
+    inp = make_gla_inputs(cfg.B, cfg.H, cfg.T + n_dec, cfg.dk, cfg.dv, cfg.dtype, seed=2, with_do=False)
+    d = {k: v.to(dev) for k, v in inp.items()}
+    head = {k: v[:, :, :cfg.T].contiguous() for k, v in d.items()}
+    toks = [{k: v[:, :, t].contiguous() for k, v in d.items()} for t in range(cfg.T, cfg.T + n_dec)]
+    state = {}
+
+    def long_fwd():
+        state["S"] = gla.chunk_fwd(head["q"], head["k"], head["v"], head["g"], chunk=cfg.chunk)[1]
+
+    def decode():
+        S = state["S"]
+        for t in toks:
+            gla.recurrent_step(t["q"], t["k"], t["v"], t["g"], S)
+
+    f_ms, dec_ms = time_pair(long_fwd, decode, max(3, steps // 2), 3, flush)
+    fb, _, ff, _ = algorithmic(cfg)
+    roof = roofline_ms(fb, ff, peaks)
+    dec_bytes = cfg.B * cfg.H * (2 * cfg.dk * cfg.dv * 4 + (3 * cfg.dk + 2 * cfg.dv) * 2)
+    out["gla_long"] = {"what": f"gla_long: GLA fwd B={cfg.B} H={cfg.H} T={cfg.T} d_k={cfg.dk} d_v={cfg.dv} bf16, "
+                               f"then {n_dec} gla_recurrent_step calls from its final state",
+                       "fwd_ms": f_ms, "fwd_tokens_per_s": cfg.B * cfg.T / (f_ms / 1e3), "fwd_roofline_ms": roof,
+                       "fwd_pct_of_roofline": 100 * roof / f_ms,
+                       "decode_us_per_step": 1e3 * dec_ms / n_dec,
+                       "decode_roofline_us_per_step": 1e6 * dec_bytes / (peaks["hbm_gbs"] * 1e9),
+                       "decode_note": "one launch per token, L2 not flushed between decode steps (the 0.5 MB "
+                                      "state stays resident, as in serving)"}
+    del d, head, toks, state
+    # GSA with 64 slots
+    cfg = CONFIGS["gsa_64slots"]
+    d = {k: v.to(dev) for k, v in make_gsa_inputs(cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.m, cfg.dtype,
+                                                  seed=3).items()}
+    f_ms, b_ms = time_pair(lambda: gla.gsa_fwd(d["q"], d["k"], d["v"], d["phi"], d["g"], chunk=cfg.chunk),
+                           lambda: gla.gsa_bwd(d["q"], d["k"], d["v"], d["phi"], d["g"], d["do"], chunk=cfg.chunk),
+                           steps, 3, flush)
+    fb, bb, ff, bf = gsa_algorithmic(cfg)
+    roof = roofline_ms(fb + bb, ff + bf, peaks)
+    out["gsa_64slots"] = {"what": f"gsa_64slots: GSA fwd+bwd B={cfg.B} H={cfg.H} T={cfg.T} d_k={cfg.dk} "
+                                  f"d_v={cfg.dv} m={cfg.m} bf16, {GATE_DESC['gsa']}",
+                          "fwd_ms": f_ms, "bwd_ms": b_ms, "step_ms": f_ms + b_ms,
+                          "tokens_per_s": cfg.B * cfg.T / ((f_ms + b_ms) / 1e3), "roofline_ms": roof,
+                          "pct_of_roofline": 100 * roof / (f_ms + b_ms), "steps": steps}
+    del d
+    torch.cuda.synchronize()
+    return out
 
 
 def run_ours(args, cfg, name):
@@ -326,12 +509,13 @@ def run_ours(args, cfg, name):
     d2h = sum(x.numel() * x.element_size() for x in outs_host)
     e2e_ms = statistics.mean(e2e_times)
     (e2e_ms,) = max_over_ranks([e2e_ms], dev)
+    del host_in, outs_host, streams
 
     launches_per_step, kernel_names = (None, ["not counted"]) if args.no_launch_count else count_launches(step)
     peaks = load_peaks()
     fb, bb, ff, bf = algorithmic(cfg)
     (tokens,) = sum_over_ranks([cfg.B * cfg.T], dev)
-    t_roof = max((fb + bb) / (peaks["hbm_gbs"] * 1e9), (ff + bf) / (peaks["bf16_tflops"] * 1e12))
+    t_roof = roofline_ms(fb + bb, ff + bf, peaks) / 1e3
     # dominant call: the larger of the fwd and bwd device times
     if bwd_ms >= fwd_ms:
         key, byt, ms, fl = "gla_chunk_bwd", bb, bwd_ms, bf
@@ -343,28 +527,30 @@ def run_ours(args, cfg, name):
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "kernel": key,
                 "algorithmic_bytes_per_call": byt, "call_ms": ms,
                 "tensor_tflops_achieved": fl / (ms / 1e3) / 1e12,
+                "flop_roofline_ms": 1e3 * fl / (peaks["bf16_tflops"] * 1e12),
                 "peak_source": f"{peaks['source']} (HBM copy bandwidth)"}
+    extra = None
+    if world == 1 and not args.no_extra:
+        del d
+        extra = extra_workloads(args, dev, flush, peaks)
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
         return
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        n = min(args.cpu_heads, cfg.B * cfg.H)
-        dt, val, _ = time_oracle(cfg, n)
-        cpu = {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-               "sample": f"{n} of {cfg.B * cfg.H} heads, T={cfg.T}, fwd+bwd, float64 numpy, 1 thread, "
-                         f"{dt:.1f} s; tokens = heads*T/H"}
+        cpu = cpu_baseline(cfg, name, args.cpu_tokens)
     line = {"metric": METRIC, "value": tokens / (step_ms / 1e3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": step_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(workload_desc(cfg, name), parallelism=f"replicas x{world} (independent heads)"),
+            "config": config_desc(cfg, name, world),
             "pct_of_roofline": 100.0 * t_roof / (step_ms / 1e3), "roofline_step_ms": t_roof * 1e3,
             "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "roofline": roofline, "cpu_baseline": cpu,
             "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "batch_slices_on_streams": parts},
             "gpu_launches": None if launches_per_step is None else launches_per_step * args.steps,
-            "launches_per_step": launches_per_step, "kernels": kernel_names, "clocks": clocks}
+            "launches_per_step": launches_per_step, "kernels": kernel_names, "clocks": clocks,
+            "extra": extra}
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -199,13 +199,14 @@ __global__ void hold_bwd_kernel(const T* __restrict__ dout, T* __restrict__ dy, 
 }
 
 int grid_for(long long items) {
-  static int sms = 0;
-  if (!sms) {
+  // Function-local static: looked up once (thread-safe initialisation).
+  static const int sms = []() {
     int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
-      sms = n;
-    if (sms <= 0) sms = 148;
-  }
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+        n > 0)
+      return n;
+    return 148;
+  }();
   const long long blocks = (items + 255) / 256, cap = (long long)sms * 8;
   return (int)(blocks < 1 ? 1 : blocks > cap ? cap : blocks);
 }

@@ -595,7 +595,6 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
 // Host entry points
 // ------------------------------------------------------------------------------------------
 bool fwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype) {
-  if (force_generic()) return false;
   if (dtype != 1 || chunk != C || T < 1 || BH < 1 || BH > 65535) return false;
   if (dk != 64 && dk != 128) return false;
   if (dv % DVT != 0) return false;
@@ -620,15 +619,15 @@ __global__ void segment_scan_kernel(float* __restrict__ sbuf, const float* __res
 }
 
 static int sm_count() {
-  static int cached[64] = {};
+  static std::atomic<int> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (!n) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 // Segments of the sequence split: as many as fill the SMs once with (head, value tile, segment)
@@ -656,7 +655,7 @@ template <int DK, bool HILO, bool REV>
 static cudaError_t launch_state_pass(const CUtensorMap& mk, const CUtensorMap& mg, const CUtensorMap& mv,
                                      const FwdArgs& args, int BH, int dv, cudaStream_t st) {
   auto kern = fwd_state_kernel<DK, HILO, REV>;
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64] = {};
   const cudaError_t e = ensure_smem_attr(kern, StateLayout<DK, HILO>::ALLOC, attr_set);
   if (e != cudaSuccess) return e;
   dim3 grid(dv / DVT, BH, args.nseg - 1);
@@ -700,7 +699,7 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
     }
   }
   auto kern = fwd_pipe_kernel<DK>;
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64] = {};
   {
     const cudaError_t e = ensure_smem_attr(kern, FwdPipeLayout<DK>::ALLOC, attr_set);
     if (e != cudaSuccess) return e;

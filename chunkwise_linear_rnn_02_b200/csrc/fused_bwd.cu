@@ -1104,7 +1104,7 @@ static cudaError_t launch_all(const BwdMaps& mp, const BwdArgs& a, int BH, cudaS
   static_assert(2 * CHK <= 228 * 1024, "two chunk CTAs per SM");
   auto k1 = bwd_fused_kernel<DK, DV, ACC>;
   auto k3 = bwd_chunk_kernel<DK, DV, ACC>;
-  static bool attr1[64] = {}, attr3[64] = {};
+  static std::atomic<bool> attr1[64] = {}, attr3[64] = {};
   {
     cudaError_t e = ensure_smem_attr(k1, BwdSmem<DK, DV>::ALLOC, attr1);
     if (e == cudaSuccess) e = ensure_smem_attr(k3, CHK, attr3);
@@ -1123,7 +1123,6 @@ static cudaError_t launch_all(const BwdMaps& mp, const BwdArgs& a, int BH, cudaS
 }
 
 bool bwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype) {
-  if (force_generic()) return false;
   if (dtype != 1 || chunk != C || T < 1 || BH < 1) return false;
   if (dk != 128 || (dv != 128 && dv != 256)) return false;
   return encode_fn() != nullptr;

@@ -6,6 +6,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -22,27 +24,30 @@ constexpr float kMinDecay = 4.248354255291589e-18f;
 // Host
 // ------------------------------------------------------------------------------------------
 inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  // Function-local static: initialised once, thread-safe.
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return nullptr;
+  }();
   return fn;
 }
 
 // Raise a kernel's dynamic shared-memory limit to `bytes`, once per device (the attribute belongs
-// to the kernel as loaded on the current device; `done` holds one flag per device ordinal).
+// to the kernel as loaded on the current device; `done` holds one flag per device ordinal).  Two
+// host threads may race here: both then set the same attribute, which is harmless, and the flag is
+// atomic.
 template <typename K>
-inline cudaError_t ensure_smem_attr(K kern, uint32_t bytes, bool (&done)[64]) {
+inline cudaError_t ensure_smem_attr(K kern, uint32_t bytes, std::atomic<bool> (&done)[64]) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev].store(true, std::memory_order_release);
   return e;
 }
 
@@ -60,12 +65,6 @@ inline bool make_map(CUtensorMap* m, const void* base, int BH, int T, int D, int
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
-}
-
-// GLA_B200_GENERIC=1 in the environment routes every call to the generic kernels.
-inline bool force_generic() {
-  const char* e = getenv("GLA_B200_GENERIC");
-  return e && e[0] && e[0] != '0';
 }
 
 // ------------------------------------------------------------------------------------------

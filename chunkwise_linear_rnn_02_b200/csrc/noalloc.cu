@@ -63,8 +63,10 @@ extern "C" int gla_chunk_bwd_noalloc(const void* q, const void* k, const void* v
   for (const void* p : opt)
     if (p && !aligned16(p)) return GLA_ERR_INVALID_ARG;
   const int BH = B * H;
-  if (!gla::fast::bwd_supported(BH, T, dk_dim, dv_dim, chunk, dtype)) return GLA_ERR_UNSUPPORTED;
+  // The size limit is plain host arithmetic on the sizes, so it is checked before anything that
+  // needs the driver.
   if (gla::fast::bwd_workspace(BH, T, dk_dim, dv_dim) > kScratchBytes) return GLA_ERR_WORKSPACE;
+  if (!gla::fast::bwd_supported(BH, T, dk_dim, dv_dim, chunk, dtype)) return GLA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   const int st = scratch_on_current_device(&scratch);
   if (st != GLA_OK) return st;

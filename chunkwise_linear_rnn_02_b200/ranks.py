@@ -1,8 +1,10 @@
 """Rank bookkeeping for running the GLA operator on several GPUs, one process per GPU.
 
 The recurrence runs along time inside one (batch, head) sequence and couples nothing across
-sequences ("Gated Linear Attention Transformers with Hardware-Efficient Training", section 4:
-the state and gates are per head), so a multi-GPU run is plain data parallelism: every rank owns
+sequences: each head keeps its own compressed matrix memory that its own gates keep, decay or
+overwrite ("Gated Linear Attention for Efficient Long Sequences", "Step-by-step memory update";
+"MS-GLA ...", section 2.1: the gate scales the rows of that memory), so a multi-GPU run is plain
+data parallelism: every rank owns
 whole sequences, computes them with the single-GPU kernels and exchanges no data.  What remains
 to agree on is which rows of a batch a rank owns, which seed its synthetic batch uses, and how
 the per-rank step times and token counts combine into one figure (the slowest rank sets the

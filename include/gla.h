@@ -96,6 +96,11 @@ int gla_chunk_fwd(const void* q, const void* k, const void* v, const void* g, co
  *   out: dq, dk, dg [B,H,T,dk]; dv [B,H,T,dv]; dh0 [B,H,dk,dv] fp32 (optional)
  * The reverse-mode recurrence is derived from the forward recurrence; dg is the reverse
  * cumulative sum over t of q*dq - k*dk plus, for every t, sum_j dhT[i,j] hT[i,j].
+ * It is the gradient of the same chunkwise form ("MS-GLA", section 2.1: chunkwise parallel
+ * training of the gated recurrence, sequential across chunks and parallel inside a chunk),
+ * evaluated chunk by chunk in reverse with the state gradient kept on chip ("Gated Linear
+ * Attention for Efficient Long Sequences", "Why chunking and SRAM locality matter": only
+ * inputs and gradients cross HBM, no per-step state is written).
  * ------------------------------------------------------------------------------------- */
 size_t gla_chunk_bwd_workspace(int B, int H, int T, int dk, int dv, int chunk, int dtype);
 int gla_chunk_bwd(const void* q, const void* k, const void* v, const void* g, const float* h0,
@@ -119,6 +124,11 @@ int gla_recurrent_step(const void* q, const void* k, const void* v, const void* 
  *        h0_1 [B,H,dk,m], h0_2 [B,H,m,dv] fp32 (optional)
  *   out: o [B,H,T,dv]; p_save [B,H,T,m] (optional: the slot softmax p, in dtype);
  *        hT1 [B,H,dk,m], hT2 [B,H,m,dv] fp32 (optional)
+ * "Gated Slot Attention ...", abstract (a two-layer GLA linked via softmax) and "Approach"
+ * (two-pass linear attention with a softmax in between; a data-dependent forget gate per
+ * slot; reuses GLA's chunkwise training form): pass 1 writes k into the m slots weighted by
+ * phi under the slot gates and reads them with q; the softmax over the slots gives p; pass 2
+ * reads the values written under the same gates with p.
  * ------------------------------------------------------------------------------------- */
 size_t gsa_fwd_workspace(int B, int H, int T, int dk, int dv, int m, int chunk, int dtype);
 int gsa_fwd(const void* q, const void* k, const void* v, const void* phi, const void* g,
@@ -132,7 +142,10 @@ int gsa_fwd(const void* q, const void* k, const void* v, const void* phi, const 
  *   out: dq, dk [B,H,T,dk]; dv [B,H,T,dv]; dphi, dg [B,H,T,m];
  *        dh0_1 [B,H,dk,m], dh0_2 [B,H,m,dv] fp32 (optional)
  * Pass 2 is differentiated first, then the softmax Jacobian do1 = p * (dp - <p, dp>), then
- * pass 1; dphi and dg sum the contributions of both passes.
+ * pass 1; dphi and dg sum the contributions of both passes.  The reverse mode of the two-pass
+ * form of "Gated Slot Attention ...", "Approach" (two GLA passes sharing the per-slot forget
+ * gates, joined by a softmax over the slots); each pass's gradient is that of a chunkwise GLA
+ * ("MS-GLA", section 2.1).
  * ------------------------------------------------------------------------------------- */
 size_t gsa_bwd_workspace(int B, int H, int T, int dk, int dv, int m, int chunk, int dtype);
 int gsa_bwd(const void* q, const void* k, const void* v, const void* phi, const void* g,

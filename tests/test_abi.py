@@ -85,6 +85,11 @@ def test_bwd_and_gsa_argument_checks(lib):
     bad_nb = list(nb)
     bad_nb[0] = None
     assert lib.gla_chunk_bwd_noalloc(*bad_nb, 1, 1, 64, 128, 256, 64, 1, None) == INVALID
+    # a supported shape whose scratch exceeds the fixed 128 MiB: B=8, H=8, T=2048, d_v=256 needs
+    # (66 + 256/2 + 256/64) * 64 * 32 * 128 * 4 bytes (six parts, each a multiple of 256 bytes)
+    need = (66 + 128 + 4) * 64 * 32 * 128 * 4 + 64 * 128 * 4
+    assert need > 128 << 20
+    assert lib.gla_chunk_bwd_noalloc(*nb, 8, 8, 2048, 128, 256, 64, 1, None) == WORKSPACE
 
 
 def test_workspace_queries(lib):

@@ -23,6 +23,18 @@ def test_compulsory_bytes_of_the_benchmark_workload():
     assert ff > 0 and bf > ff
 
 
+def test_gsa_compulsory_bytes_and_flops():
+    """gsa_64slots (B=4, H=4, T=4096, d_k=d_v=128, m=64): 3,600 bytes per token-head in all (reads of
+    q, k, v, phi, g (+ dO) and writes of o (+ dq, dk, dv, dphi, dg)), plus the two fp32 final
+    states; FLOPs are both passes' chunk-form contractions (d_k x m, then m x d_v)."""
+    cfg = CONFIGS["gsa_64slots"]
+    fb, bb, ff, bf = bench.gsa_algorithmic(cfg)
+    th = 4 * 4 * 4096
+    assert fb == th * 1280 + 16 * (128 * 64 + 64 * 128) * 4
+    assert bb == th * 2304
+    assert ff == th * 90112 and bf == th * 192512
+
+
 def test_traffic_is_read_from_the_profile_summaries():
     """The roofline's `traffic` comes from a line of the committed ncu summary; it must parse to a
     byte count of the same order as the compulsory bytes (above them: workspace and re-reads)."""
@@ -34,7 +46,8 @@ def test_traffic_is_read_from_the_profile_summaries():
 
 
 def test_reference_arm_prints_one_json_line():
-    """`--impl reference` times the oracle on one head per step and prints the contract's line."""
+    """`--impl reference` times the oracle on a sample of heads per step, spread over the host cores,
+    and prints the contract's line."""
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
                         "--warmup", "0"], capture_output=True, text=True, timeout=600, cwd=ROOT)
     assert r.returncode == 0, r.stderr[-2000:]
@@ -45,4 +58,7 @@ def test_reference_arm_prints_one_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
-    assert d["config"]["workload"].startswith("gla_340m")
+    assert d["config"]["workload"].startswith("gla_1p3b")
+    # the same config object as the GPU arm's line for this workload and GPU count
+    assert d["config"] == bench.config_desc(CONFIGS["gla_1p3b"], "gla_1p3b", 1)
+    assert d["cpu_baseline"]["cores"] >= 1

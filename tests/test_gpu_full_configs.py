@@ -33,13 +33,19 @@ def _check_gla(cfg, idx, mu=0.0, seed=0, check_bwd=True):
     assert gla.device_error() == 0
 
 
+def _ends(cfg):
+    """The first and the last head of the grid, so that an off-by-one head or tile index at either
+    end cannot hide."""
+    return [(0, 0), (cfg.B - 1, cfg.H - 1)]
+
+
 def test_gla_340m_shape_fwd_bwd():
-    _check_gla(CONFIGS["gla_340m"], [(0, 0), (7, 3)])
+    _check_gla(CONFIGS["gla_340m"], _ends(CONFIGS["gla_340m"]))
 
 
 @pytest.mark.parametrize("mu", [-2.0, 0.0, 3.0])
 def test_gla_1p3b_shape_gate_sweep(mu):
-    _check_gla(CONFIGS["gla_1p3b"], [(3, 1)], mu=mu)
+    _check_gla(CONFIGS["gla_1p3b"], _ends(CONFIGS["gla_1p3b"]), mu=mu)
 
 
 def test_gla_long_sequence_then_decode():
@@ -56,8 +62,8 @@ def test_gla_long_sequence_then_decode():
     # GPU decode against the GPU chunked run over T + 256 tokens
     assert_close("decode vs chunked o", o_dec, o_full[:, :, cfg.T:], TOL_BF16)
     assert_close("decode vs chunked hT", S, hT_full, TOL_BF16)
-    # and both against the oracle on one sampled head
-    idx = [(0, 2)]
+    # and both against the oracle on the first and the last head
+    idx = _ends(cfg)
     sub = {nm: _heads(inp[nm], idx) for nm in ["q", "k", "v", "g"]}
     ro, rhT = O.gla_fwd(sub["q"], sub["k"], sub["v"], sub["g"])
     assert_close("o (oracle)", _heads(o_full.cpu(), idx), ro, TOL_BF16)
@@ -71,7 +77,7 @@ def test_gsa_64_slots_fwd_bwd():
     d = cuda(inp)
     o, p, hT1, hT2 = gla.gsa_fwd(d["q"], d["k"], d["v"], d["phi"], d["g"], chunk=cfg.chunk, save_p=True)
     grads = gla.gsa_bwd(d["q"], d["k"], d["v"], d["phi"], d["g"], d["do"], chunk=cfg.chunk)
-    idx = [(1, 2)]
+    idx = _ends(cfg)
     sub = [_heads(inp[nm], idx) for nm in ["q", "k", "v", "phi", "g"]]
     ro, rp, rhT1, rhT2 = O.gsa_fwd(*sub)
     for name, x, r in [("o", o, ro), ("p", p, rp), ("hT1", hT1, rhT1), ("hT2", hT2, rhT2)]:
