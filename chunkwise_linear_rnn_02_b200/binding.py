@@ -14,7 +14,7 @@ import torch
 
 __all__ = [
     "GLAError", "load_library", "library_path", "header_symbols", "status_string", "version",
-    "chunk_fwd", "chunk_bwd", "recurrent_step", "gsa_fwd", "gsa_bwd", "gsa_recurrent_step",
+    "chunk_fwd", "chunk_bwd", "chunk_fwd_logit", "chunk_bwd_logit", "recurrent_step", "gsa_fwd", "gsa_bwd", "gsa_recurrent_step",
     "device_error", "workspace_bytes",
 ]
 
@@ -32,6 +32,10 @@ _SIGNATURES = {
     "gla_chunk_fwd": (_i, [_vp] * 7 + [_i] * 7 + [_vp, _sz, _vp]),
     "gla_chunk_bwd_workspace": (_sz, [_i] * 7),
     "gla_chunk_bwd": (_i, [_vp] * 12 + [_i] * 7 + [_vp, _sz, _vp]),
+    "gla_chunk_fwd_logit_workspace": (_sz, [_i] * 7),
+    "gla_chunk_fwd_logit": (_i, [_vp] * 4 + [ctypes.c_float] + [_vp] * 3 + [_i] * 7 + [_vp, _sz, _vp]),
+    "gla_chunk_bwd_logit_workspace": (_sz, [_i] * 7),
+    "gla_chunk_bwd_logit": (_i, [_vp] * 4 + [ctypes.c_float] + [_vp] * 8 + [_i] * 7 + [_vp, _sz, _vp]),
     "gla_recurrent_step": (_i, [_vp] * 6 + [_i] * 5 + [_vp]),
     "gsa_fwd_workspace": (_sz, [_i] * 8),
     "gsa_fwd": (_i, [_vp] * 11 + [_i] * 8 + [_vp, _sz, _vp]),
@@ -171,6 +175,43 @@ def chunk_bwd(q, k, v, g, do, h0=None, dhT=None, chunk: int = 64, need_dh0: bool
                              _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg), _ptr(dh0), B, H, T, dk, dv, chunk, dt,
                              _ptr(ws), nb, _stream(dev)), "gla_chunk_bwd")
     return dq, dkk, dvv, dg, dh0
+
+
+def chunk_fwd_logit(q, k, v, x, tau: float, h0=None, chunk: int = 64, output_final_state: bool = True):
+    """GLA forward from raw gate logits x (g = logsigmoid(x) / tau formed inside the kernels)."""
+    _need_cuda(q, k, v, x)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    lib = load_library()
+    dev = q.device
+    h0 = _state(h0, (B, H, dk, dv), dev)
+    o = torch.empty(B, H, T, dv, dtype=q.dtype, device=dev)
+    hT = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev) if output_final_state else None
+    ws, nb = _workspace(lib.gla_chunk_fwd_logit_workspace(B, H, T, dk, dv, chunk, dt), dev)
+    _check(lib.gla_chunk_fwd_logit(_ptr(q), _ptr(k), _ptr(v), _ptr(x), float(tau), _ptr(h0), _ptr(o), _ptr(hT),
+                                   B, H, T, dk, dv, chunk, dt, _ptr(ws), nb, _stream(dev)), "gla_chunk_fwd_logit")
+    return o, hT
+
+
+def chunk_bwd_logit(q, k, v, x, tau: float, do, h0=None, dhT=None, chunk: int = 64, need_dh0: bool = True):
+    """Backward of chunk_fwd_logit: returns (dq, dk, dv, dx, dh0 or None)."""
+    _need_cuda(q, k, v, x, do)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    lib = load_library()
+    dev = q.device
+    h0 = _state(h0, (B, H, dk, dv), dev)
+    dhT = _state(dhT, (B, H, dk, dv), dev)
+    dq, dkk, dx = (torch.empty_like(q) for _ in range(3))
+    dvv = torch.empty_like(v)
+    dh0 = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev) if need_dh0 else None
+    ws, nb = _workspace(lib.gla_chunk_bwd_logit_workspace(B, H, T, dk, dv, chunk, dt), dev)
+    _check(lib.gla_chunk_bwd_logit(_ptr(q), _ptr(k), _ptr(v), _ptr(x), float(tau), _ptr(h0), _ptr(do), _ptr(dhT),
+                                   _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dx), _ptr(dh0), B, H, T, dk, dv, chunk, dt,
+                                   _ptr(ws), nb, _stream(dev)), "gla_chunk_bwd_logit")
+    return dq, dkk, dvv, dx, dh0
 
 
 def recurrent_step(q, k, v, g, S):

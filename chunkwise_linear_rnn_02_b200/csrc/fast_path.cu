@@ -58,6 +58,7 @@ struct FwdArgs {
   int T, DV, seg_chunks, nseg;
   long long st_bh, st_row;  // h0 / hT strides (a sub-block of a larger state when the shape is split)
   float* acc_o;             // optional fp32 output [BH*T][DV] in place of o (split shapes)
+  float inv_tau;            // > 0: the gate tensor holds raw logits x, g = logsigmoid(x) / tau
   unsigned int* latch;
 };
 
@@ -159,6 +160,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint8_t* st = sm + s * L::STAGE;
     mbar_wait(&bar_load[s], (li >> 1) & 1, args.latch);
     Gate gr;
+    gr.set_logit(args.inv_tau, T - (REV ? c_end - 1 - li : c_begin + li) * C);
     gr.run(st + L::RAW, DK, tot_sm);
     if (gr.h == 0) {
       decay_sm[gr.d] = gr.dec0;
@@ -437,6 +439,7 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     auto gate_regs = [&](int li) {
       const uint8_t* st = sm + (li & 1) * L::QKG;
       Gate gr;
+      gr.set_logit(args.inv_tau, T - (c_begin + li) * C);
       const bool weak = gr.run(st + 2 * L::RAW, DK, tot_sm);
       float* dec = decay_sm + (li & 1) * DK;
       if (gr.h == 0) {
@@ -618,7 +621,7 @@ __global__ void segment_scan_kernel(float* __restrict__ sbuf, const float* __res
   }
 }
 
-static int sm_count() {
+int sm_count() {
   static std::atomic<int> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
@@ -666,7 +669,7 @@ static cudaError_t launch_state_pass(const CUtensorMap& mk, const CUtensorMap& m
 template <int DK>
 static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o,
                               float* hT, int BH, int T, int dv, long long st_bh, long long st_row, float* acc_o,
-                              void* ws, cudaStream_t st) {
+                              void* ws, cudaStream_t st, float inv_tau) {
   CUtensorMap m[4];
   if (!make_map(&m[0], q, BH, T, DK, DK, false) || !make_map(&m[1], k, BH, T, DK, DK, false) ||
       !make_map(&m[2], g, BH, T, DK, DK, false) || !make_map(&m[3], v, BH, T, dv, DVT, true))
@@ -680,6 +683,7 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
   a.st_bh = st_bh;
   a.st_row = st_row;
   a.acc_o = acc_o;
+  a.inv_tau = inv_tau;
   a.latch = device_error_latch();
   plan_segments(BH, T, dv, &a.nseg, &a.seg_chunks);
   a.sbuf = nullptr;
@@ -743,9 +747,10 @@ __global__ void segment_scan_rev_kernel(float* __restrict__ gbuf, const float* _
 cudaError_t segment_states(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mg,
                            const CUtensorMap& mv, const CUtensorMap& mdo, const float* h0, const float* dhT,
                            float* sbuf, float* gbuf, float* gam, int BH, int T, int dk, int dv, int nseg,
-                           int seg_chunks, long long st_bh, long long st_row, cudaStream_t st) {
+                           int seg_chunks, long long st_bh, long long st_row, cudaStream_t st, float inv_tau) {
   if (dk != 128 || nseg < 2) return cudaErrorNotSupported;
   FwdArgs a = {};
+  a.inv_tau = inv_tau;
   a.T = T;
   a.DV = dv;
   a.seg_chunks = seg_chunks;
@@ -774,13 +779,40 @@ cudaError_t segment_states(const CUtensorMap& mq, const CUtensorMap& mk, const C
   return e;
 }
 
+cudaError_t segment_entry_states(const void* k, const void* g, const void* v, const float* h0, float* sbuf,
+                                 float* gam, int BH, int T, int dk, int dv, int nseg, int seg_chunks,
+                                 cudaStream_t st) {
+  if (dk != 64 || dv % DVT != 0 || nseg < 2) return cudaErrorNotSupported;
+  CUtensorMap m[3];
+  if (!make_map(&m[0], k, BH, T, dk, dk, false) || !make_map(&m[1], g, BH, T, dk, dk, false) ||
+      !make_map(&m[2], v, BH, T, dv, DVT, true))
+    return cudaErrorInvalidValue;
+  FwdArgs a = {};
+  a.h0 = h0;
+  a.sbuf = sbuf;
+  a.gam = gam;
+  a.T = T;
+  a.DV = dv;
+  a.seg_chunks = seg_chunks;
+  a.nseg = nseg;
+  a.st_bh = (long long)dk * dv;
+  a.st_row = dv;
+  a.latch = device_error_latch();
+  cudaError_t e = launch_state_pass<64, false, false>(m[0], m[1], m[2], a, BH, dv, st);
+  if (e != cudaSuccess || nseg < 3) return e;
+  const size_t n = (size_t)BH * dk * dv;
+  const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  segment_scan_kernel<<<blocks, 256, 0, st>>>(sbuf, gam, BH, dk, dv, nseg);
+  return cudaGetLastError();
+}
+
 cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
                 int BH, int T, int dk, int dv, void* ws, cudaStream_t st, long long st_bh, long long st_row,
-                float* acc_o) {
+                float* acc_o, float inv_tau) {
   if (st_bh < 0) st_bh = (long long)dk * dv;
   if (st_row < 0) st_row = dv;
-  if (dk == 64) return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st);
-  if (dk == 128) return launch_fwd<128>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st);
+  if (dk == 64) return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st, inv_tau);
+  if (dk == 128) return launch_fwd<128>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st, inv_tau);
   return cudaErrorNotSupported;
 }
 

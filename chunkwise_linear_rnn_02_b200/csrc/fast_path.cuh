@@ -17,10 +17,11 @@ bool fwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype);
 size_t fwd_workspace(int BH, int T, int dk, int dv);
 // st_bh / st_row: element strides of the fp32 states per head and per row (defaults, when
 // negative: dk*dv and dv).  A split shape passes a sub-block of the caller's states this way, and
-// an fp32 array acc_o [BH*T][dv] that receives o in place of the bf16 output.
+// an fp32 array acc_o [BH*T][dv] that receives o in place of the bf16 output.  inv_tau > 0: g holds
+// raw logits x and the kernels use g = bf16(logsigmoid(x) * inv_tau).
 cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
                 int BH, int T, int dk, int dv, void* ws, cudaStream_t st, long long st_bh = -1,
-                long long st_row = -1, float* acc_o = nullptr);
+                long long st_row = -1, float* acc_o = nullptr, float inv_tau = 0.f);
 
 // fp32 outputs of a backward sub-problem (split shapes): dq / dk / dg go to columns ck.. of
 // [BH*T][pk] arrays, dv to columns cv.. of a [BH*T][pv] array.
@@ -37,14 +38,27 @@ void plan_bwd_segments(int ctas_per_seg, int T, int* nseg, int* seg_chunks);
 cudaError_t segment_states(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mg,
                            const CUtensorMap& mv, const CUtensorMap& mdo, const float* h0, const float* dhT,
                            float* sbuf, float* gbuf, float* gam, int BH, int T, int dk, int dv, int nseg,
-                           int seg_chunks, long long st_bh, long long st_row, cudaStream_t st);
+                           int seg_chunks, long long st_bh, long long st_row, cudaStream_t st, float inv_tau);
+
+// SM count of the current device (cached per device).
+int sm_count();
+
+// Sequence split of a key-gated recurrence S <- diag(e^{g_t}) S + k_t^T v_t with d_k = 64 rows
+// (k, g: bf16 [BH][T][64]; v: bf16 [BH][T][dv], dv a multiple of 64), for a caller that walks the
+// segments itself: sbuf [BH][nseg][64][dv] receives in entry s-1 the state entering segment s
+// (s >= 1; the first segment starts from h0 [BH][64][dv] or zeros), gam [BH][nseg][64] the
+// segments' decay products.
+cudaError_t segment_entry_states(const void* k, const void* g, const void* v, const float* h0, float* sbuf,
+                                 float* gam, int BH, int T, int dk, int dv, int nseg, int seg_chunks,
+                                 cudaStream_t st);
 
 bool bwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype);
 size_t bwd_workspace(int BH, int T, int dk, int dv);
+// inv_tau > 0: g holds raw logits x (as for fwd) and dg receives dx = dg * sigmoid(-x) / tau.
 cudaError_t bwd(const void* q, const void* k, const void* v, const void* g, const float* h0, const void* dO,
                 const float* dhT, void* dq, void* dk, void* dv, void* dg, float* dh0, int BH, int T, int dkd,
                 int dvd, void* ws, cudaStream_t st, long long st_bh = -1, long long st_row = -1,
-                const BwdAccum* acc = nullptr);
+                const BwdAccum* acc = nullptr, float inv_tau = 0.f);
 
 }  // namespace fast
 }  // namespace gla

@@ -73,6 +73,9 @@ struct BwdArgs {
   // place of the bf16 outputs.
   float *acc_q, *acc_k, *acc_g, *acc_v;
   int acc_pk, acc_ck, acc_pv, acc_cv;
+  // > 0: the gate tensor holds raw logits x (g = logsigmoid(x) / tau) and the gate-gradient output
+  // receives dx = dg sigmoid(-x) / tau in place of dg
+  float inv_tau;
   unsigned int* latch;
 };
 
@@ -189,7 +192,8 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   // dA (masked, as the MMAs see it: hi + lo) at (j, r).
   auto dA_at = [&](int j, int r) { return raw(L::DA_HI, j, r) + raw(L::DA_LO, j, r); };
   // Gate run of the chunk in part-B buffer b: run products into TOT[b], decays into DEC[b].
-  auto gate = [&](Gate& gr, int b) {
+  auto gate = [&](Gate& gr, int b, int chunk) {
+    gr.set_logit(a.inv_tau, T - chunk * C);
     const bool weak = gr.run_swizzled(sm + pbo(b) + L::PB_G, TOT + b * NS * KT);
     if (gr.h == 0) {
       DEC[b * KT + gr.d] = gr.dec0;
@@ -295,10 +299,10 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   };
   // Chunk i+1: gate run from buffer nb, Kh operand, state copy + rescale, group 1.  The operand
   // area KQ is free once group 2 of the current chunk has completed.
-  auto prepare = [&](int nb, int m2_pending) {
+  auto prepare = [&](int nb, int m2_pending, int chunk) {
     wait_b(nb);
     Gate gr;
-    const int safe = gate(gr, nb);
+    const int safe = gate(gr, nb, chunk);
     uint32_t w[Gate::TS];
     gr.load_pairs(sm + pbo(nb) + L::PB_K, KT, true, w);
     if (m2_pending) wait_m2();
@@ -320,7 +324,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     init_state(a.h0 ? a.h0 + bh * a.st_bh : nullptr, a.st_row);
   else
     init_state(a.s_in + ((size_t)bh * a.nseg + seg - 1) * DK * DV, DV);
-  int safe_next = prepare(0, 0);
+  int safe_next = prepare(0, 0, ch0);
   for (int i = ch0; i < ch1; ++i) {
     const int b = (i - ch0) & 1, safe = safe_next;
     mbar_wait(bar_m1, ph_m1, a.latch);
@@ -334,7 +338,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     sync_tc();
     if (!safe) issue_m2();
     if (i + 1 < ch1)
-      safe_next = prepare(b ^ 1, !safe);
+      safe_next = prepare(b ^ 1, !safe, i + 1);
     else if (!safe)
       wait_m2();
     float y[32];  // this thread's row of Y^T
@@ -550,6 +554,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     mbar_wait(bar_ld, ph_ld, a.latch);
     ph_ld ^= 1;
     Gate gr;
+    gr.set_logit(a.inv_tau, T - i * C);
     const bool weak = gr.run(sm + 2 * L::RAW, DK, TOT);
     if (gr.h == 0) {
       DEC[gr.d] = gr.dec0;
@@ -923,6 +928,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   }
   // gate run of the key slab: Qt hi / lo, decays, run products
   Gate gr;
+  gr.set_logit(a.inv_tau, T - i * C);
   const bool weak = gr.run_swizzled(sm + L::PB_G, TOT);
   if (gr.h == 0) {
     DEC[gr.d] = gr.dec0;
@@ -1040,13 +1046,17 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
     for (int t = 0; t < qi; ++t) pre += XQ[t * KT + d];
     __nv_bfloat16* dst = a.dg + ((size_t)bh * T + i * C + tq) * DK + d0 + d;
     float* dst32 = ACC ? a.acc_g + ((size_t)bh * T + i * C + tq) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
+    const float tau = a.inv_tau > 0.f ? 1.f / a.inv_tau : 0.f;
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       if (i * C + tq + c < T) {
+        float dgv = ci + pre + pv[c];
+        // raw logits: dx = dg sigmoid(-x) / tau, with sigmoid(-x) = 1 - e^{tau g} = -expm1(tau g)
+        if (a.inv_tau > 0.f) dgv *= -expm1f(tau * raw(L::PB_G, tq + c, d)) * a.inv_tau;
         if (ACC)
-          dst32[(size_t)c * a.acc_pk] = ci + pre + pv[c];
+          dst32[(size_t)c * a.acc_pk] = dgv;
         else
-          dst[(size_t)c * DK] = __float2bfloat16_rn(ci + pre + pv[c]);
+          dst[(size_t)c * DK] = __float2bfloat16_rn(dgv);
       }
       pre += w[c];
     }
@@ -1158,7 +1168,7 @@ template <int DK, int DV>
 static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* g, const float* h0,
                               const void* dO, const float* dhT, void* dq, void* dk, void* dv, void* dg, float* dh0,
                               int BH, int T, void* ws, cudaStream_t st, long long st_bh, long long st_row,
-                              const BwdAccum* acc) {
+                              const BwdAccum* acc, float inv_tau) {
   BwdMaps mp;
   if (!make_map(&mp.v, v, BH, T, DV, 64, true) || !make_map(&mp.dO, dO, BH, T, DV, 64, true) ||
       !make_map(&mp.k64, k, BH, T, DK, KT, true) || !make_map(&mp.g64, g, BH, T, DK, KT, true) ||
@@ -1185,6 +1195,7 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
   a.acc_ck = acc ? acc->ck : 0;
   a.acc_pv = acc ? acc->pv : 0;
   a.acc_cv = acc ? acc->cv : 0;
+  a.inv_tau = inv_tau;
   size_t sz[9];
   bwd_parts(BH, T, DK, DV, sz, &a.nseg, &a.seg_chunks);
   float* p[9];
@@ -1202,7 +1213,7 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
   a.latch = device_error_latch();
   if (a.nseg > 1) {
     const cudaError_t e = segment_states(mp.q_all, mp.k_all, mp.g_all, mp.v, mp.dO, h0, dhT, p[6], p[7], p[8], BH, T,
-                                         DK, DV, a.nseg, a.seg_chunks, st_bh, st_row, st);
+                                         DK, DV, a.nseg, a.seg_chunks, st_bh, st_row, st, inv_tau);
     if (e != cudaSuccess) return e;
   }
   return acc ? launch_all<DK, DV, true>(mp, a, BH, st) : launch_all<DK, DV, false>(mp, a, BH, st);
@@ -1210,13 +1221,15 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
 
 cudaError_t bwd(const void* q, const void* k, const void* v, const void* g, const float* h0, const void* dO,
                 const float* dhT, void* dq, void* dk, void* dv, void* dg, float* dh0, int BH, int T, int dkd, int dvd,
-                void* ws, cudaStream_t st, long long st_bh, long long st_row, const BwdAccum* acc) {
+                void* ws, cudaStream_t st, long long st_bh, long long st_row, const BwdAccum* acc, float inv_tau) {
   if (st_bh < 0) st_bh = (long long)dkd * dvd;
   if (st_row < 0) st_row = dvd;
   if (dkd == 128 && dvd == 256)
-    return launch_bwd<128, 256>(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, ws, st, st_bh, st_row, acc);
+    return launch_bwd<128, 256>(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, ws, st, st_bh, st_row, acc,
+                                inv_tau);
   if (dkd == 128 && dvd == 128)
-    return launch_bwd<128, 128>(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, ws, st, st_bh, st_row, acc);
+    return launch_bwd<128, 128>(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, ws, st, st_bh, st_row, acc,
+                                inv_tau);
   return cudaErrorNotSupported;
 }
 

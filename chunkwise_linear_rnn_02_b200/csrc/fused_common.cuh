@@ -184,6 +184,16 @@ constexpr int kBarCompute = 1;  // named barrier of the threads that run the gat
 // bf16 at `graw`, columns col0..), computes alpha = e^g with one ex2 per value, and leaves in
 // registers the run's alphas and, via the shared buffer `tot` (NSPLIT x ND floats), the products of
 // the other runs: pre = prod of earlier runs, suf = prod of later runs, dec = e^{gamma}.
+//
+// Raw-logit gates: with inv_tau > 0 the tile holds logits x instead of log-gates, and the run first
+// replaces every element of it, in place, by g = bf16(logsigmoid(x) * inv_tau) (0 for the tokens
+// at or past `valid`, which lie beyond the end of the sequence), the values the standalone gate
+// entry would store; everything that reads the tile afterwards sees those log-gates.  The caller
+// runs exactly one gate run per loaded tile, before any other reader of it.
+__device__ __forceinline__ float logsigmoid_scaled(float x, float inv_tau) {
+  return (fminf(x, 0.f) - log1pf(expf(-fabsf(x)))) * inv_tau;
+}
+
 template <int ND, int NTH>
 struct GateRun {
   static constexpr int NPAIR = ND / 2;
@@ -193,6 +203,13 @@ struct GateRun {
   float a0[TS], a1[TS];
   float pre0, pre1, suf0, suf1, dec0, dec1;
   int p, h, d;
+  float inv_tau = 0.f;  // > 0: the tile holds raw logits (see above)
+  int valid = C;        // tokens of the tile inside the sequence (raw-logit mode)
+
+  __device__ __forceinline__ void set_logit(float inv_tau_, int tokens_left) {
+    inv_tau = inv_tau_;
+    valid = tokens_left < C ? tokens_left : C;
+  }
 
   // Returns true when this thread's dimensions keep less than kMinDecay of the state.
   __device__ __forceinline__ bool run(const uint8_t* graw, int gstride, float* tot) {
@@ -211,7 +228,12 @@ struct GateRun {
 #pragma unroll
     for (int u = 0; u < TS; ++u) {
       const int j = h * TS + u;
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(graw + (swz ? sm100::sw128(j, d) : (j * gstride + d) * 2));
+      const uint32_t off = swz ? sm100::sw128(j, d) : (j * gstride + d) * 2;
+      uint32_t w = *reinterpret_cast<const uint32_t*>(graw + off);
+      if (inv_tau > 0.f) {
+        w = j < valid ? pack2(logsigmoid_scaled(bf_lo(w), inv_tau), logsigmoid_scaled(bf_hi(w), inv_tau)) : 0u;
+        *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(graw) + off) = w;
+      }
       a0[u] = ex2(bf_lo(w) * kLog2e);
       a1[u] = ex2(bf_hi(w) * kLog2e);
       r0 *= a0[u];

@@ -10,6 +10,7 @@
 #include "fast_path.cuh"
 #include "split.cuh"
 #include "generic_kernels.cuh"
+#include "gsa_fused.cuh"
 
 using gla::bf16;
 namespace gk = gla::generic;
@@ -114,7 +115,7 @@ size_t carve_split_fwd(Carve& c, int BH, int T, int dk, int dv, SplitFwdWs* w) {
 }
 
 int split_fwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const float* h0, bf16* o, float* hT,
-              int BH, int T, int dk, int dv, void* ws, cudaStream_t st) {
+              int BH, int T, int dk, int dv, void* ws, cudaStream_t st, float inv_tau = 0.f) {
   Carve c(ws);
   SplitFwdWs w;
   carve_split_fwd(c, BH, T, dk, dv, &w);
@@ -126,7 +127,7 @@ int split_fwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const 
     GLA_CUDA(gla::split::gather_cols(g, w.g, rows, dk, c0, kSplitK, st));
     GLA_CUDA(gla::fast::fwd(w.q, w.k, v, w.g, h0 ? h0 + (size_t)c0 * dv : nullptr, nullptr,
                             hT ? hT + (size_t)c0 * dv : nullptr, BH, T, kSplitK, dv, w.fws, st, (long long)dk * dv,
-                            dv, kb == 0 ? w.acc : w.part));
+                            dv, kb == 0 ? w.acc : w.part, inv_tau));
     if (kb > 0) GLA_CUDA(gla::split::add_cols(w.part, w.acc, rows, dv, dv, 0, st));
   }
   GLA_CUDA(gla::split::to_bf16(w.acc, o, rows * dv, st));
@@ -163,7 +164,7 @@ size_t carve_split_bwd(Carve& c, int BH, int T, int dk, int dv, SplitBwdWs* w) {
 
 int split_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const float* h0, const bf16* dO,
               const float* dhT, bf16* dq, bf16* dk, bf16* dv, bf16* dg, float* dh0, int BH, int T, int dkd, int dvd,
-              void* ws, cudaStream_t st) {
+              void* ws, cudaStream_t st, float inv_tau = 0.f) {
   Carve c(ws);
   SplitBwdWs w;
   carve_split_bwd(c, BH, T, dkd, dvd, &w);
@@ -196,7 +197,7 @@ int split_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const 
                                     fk ? dkd : kSplitK, fk ? k0 : 0, fv ? dvd : vb, fv ? v0 : 0};
       GLA_CUDA(gla::fast::bwd(qb, kbp, vvb, gb, h0 ? h0 + so : nullptr, dob, dhT ? dhT + so : nullptr, nullptr,
                               nullptr, nullptr, nullptr, dh0 ? dh0 + so : nullptr, BH, T, kSplitK, vb, w.bws, st,
-                              (long long)dkd * dvd, dvd, &out));
+                              (long long)dkd * dvd, dvd, &out, inv_tau));
       if (!fk) {
         GLA_CUDA(gla::split::add_cols(w.pq, w.aq, rows, kSplitK, dkd, k0, st));
         GLA_CUDA(gla::split::add_cols(w.pk, w.ak, rows, kSplitK, dkd, k0, st));
@@ -315,7 +316,7 @@ struct GsaFusedWs {
   float *h0, *dhT, *dh0;             // [BH][128][dv] padded states
   void* ws;                          // the fused backward's workspace
 };
-void carve_gsa_fused(Carve& c, int BH, int T, int dv, GsaFusedWs* w) {
+void carve_gsa_fused(Carve& c, int BH, int T, int dv, GsaFusedWs* w, size_t bwd_ws = 0) {
   const size_t rows = (size_t)BH * T, st = (size_t)BH * 128 * dv;
   GsaFusedWs x;
   x.p = c.take<bf16>(rows * 128);
@@ -328,7 +329,8 @@ void carve_gsa_fused(Carve& c, int BH, int T, int dv, GsaFusedWs* w) {
   x.h0 = c.take<float>(st);
   x.dhT = c.take<float>(st);
   x.dh0 = c.take<float>(st);
-  x.ws = c.take<char>(gla::fast::bwd_workspace(BH, T, 128, dv));
+  const size_t need = gla::fast::bwd_workspace(BH, T, 128, dv);
+  x.ws = c.take<char>(need > bwd_ws ? need : bwd_ws);
   if (w) *w = x;
 }
 
@@ -357,6 +359,118 @@ size_t carve_gsa_bwd(Carve& c, int BH, int T, int dk, int dv, int m, int chunk, 
   if (gsa_pass2_fused_ok(BH, T, m, dv, chunk, dtype)) carve_gsa_fused(c, BH, T, dv, &x.f);
   if (w) *w = x;
   return c.used;
+}
+
+// ----------------------------------------------------------------------------------------
+// GSA with both passes on the fused kernels (bf16, chunk 64, d_k = 128, m = 64): pass 1 and the
+// slot softmax on the pass-1 kernel, pass 2 on the GLA forward.  The backward differentiates pass
+// 2 on the GLA backward (slots zero-padded to a 128-wide key block), applies the softmax Jacobian,
+// and differentiates pass 1 as a GLA with the roles exchanged: <do1, o1(q, k, phi, g)> equals
+// <q, o'> for o' = GLA(queries do1, keys phi, values k, the slot gates on the key axis) with the
+// initial state h0_1^T, so pass 1's gradients for phi, k, g and h0_1 are that GLA's gradients for
+// its keys, values, gates and initial state with dO' = q, and dq = S1 do1 is that GLA's output.
+// ----------------------------------------------------------------------------------------
+bool gsa_fused_fwd_ok(int BH, int T, int dk, int dv, int m, int chunk, int dtype) {
+  return gla::gsa::pass1_supported(BH, T, dk, m, chunk, dtype) && gla::fast::fwd_supported(BH, T, m, dv, chunk, dtype);
+}
+bool gsa_fused_bwd_ok(int BH, int T, int dk, int dv, int m, int chunk, int dtype) {
+  return gsa_fused_fwd_ok(BH, T, dk, dv, m, chunk, dtype) && gsa_pass2_fused_ok(BH, T, m, dv, chunk, dtype) &&
+         gla::fast::bwd_supported(BH, T, 128, dk, chunk, dtype) && gla::fast::fwd_supported(BH, T, m, dk, chunk, dtype);
+}
+
+struct GsaFusedFwdWs {
+  bf16* p;
+  void *p1ws, *fws;
+};
+size_t carve_gsa_fused_fwd(Carve& c, int BH, int T, int dk, int dv, int m, bool need_p, GsaFusedFwdWs* w) {
+  GsaFusedFwdWs x;
+  x.p = need_p ? c.take<bf16>((size_t)BH * T * m) : nullptr;
+  x.p1ws = c.take<char>(gla::gsa::pass1_workspace(BH, T, dk));
+  x.fws = c.take<char>(gla::fast::fwd_workspace(BH, T, m, dv));
+  if (w) *w = x;
+  return c.used;
+}
+
+struct GsaFusedBwdWs {
+  GsaFusedWs f;                   // pass 2: padded operands, fp32 gradients, padded states, bwd workspace
+  bf16 *p, *do1, *do1_pad;        // [rows][m], [rows][m], [rows][128]
+  float *dq1, *dphi1, *dg1, *dkf;  // pass-1 backward outputs: [rows][128] x 3, [rows][dk]
+  float *h0p, *dhTp, *dh0p, *h0t;  // [BH][128][dk] x 3, [BH][m][dk]
+  void *p1ws, *fws;
+};
+size_t carve_gsa_fused_bwd(Carve& c, int BH, int T, int dk, int dv, int m, GsaFusedBwdWs* w) {
+  const size_t rows = (size_t)BH * T, sp = (size_t)BH * 128 * dk;
+  GsaFusedBwdWs x;
+  carve_gsa_fused(c, BH, T, dv, &x.f, gla::fast::bwd_workspace(BH, T, 128, dk));
+  x.p = c.take<bf16>(rows * m);
+  x.do1 = c.take<bf16>(rows * m);
+  x.do1_pad = c.take<bf16>(rows * 128);
+  x.dq1 = c.take<float>(rows * 128);
+  x.dphi1 = c.take<float>(rows * 128);
+  x.dg1 = c.take<float>(rows * 128);
+  x.dkf = c.take<float>(rows * dk);
+  x.h0p = c.take<float>(sp);
+  x.dhTp = c.take<float>(sp);
+  x.dh0p = c.take<float>(sp);
+  x.h0t = c.take<float>((size_t)BH * m * dk);
+  x.p1ws = c.take<char>(gla::gsa::pass1_workspace(BH, T, dk));
+  x.fws = c.take<char>(gla::fast::fwd_workspace(BH, T, m, dk));
+  if (w) *w = x;
+  return c.used;
+}
+
+int gsa_fwd_fused(const bf16* q, const bf16* k, const bf16* v, const bf16* phi, const bf16* g, const float* h01,
+                  const float* h02, bf16* o, bf16* p_save, float* hT1, float* hT2, int BH, int T, int dk, int dv,
+                  int m, void* ws, cudaStream_t st) {
+  Carve c(ws);
+  GsaFusedFwdWs w;
+  carve_gsa_fused_fwd(c, BH, T, dk, dv, m, p_save == nullptr, &w);
+  bf16* p = p_save ? p_save : w.p;
+  GLA_CUDA(gla::gsa::pass1_fwd(q, k, phi, g, h01, p, hT1, BH, T, dk, w.p1ws, st));
+  GLA_CUDA(gla::fast::fwd(p, phi, v, g, h02, o, hT2, BH, T, m, dv, w.fws, st));
+  return GLA_OK;
+}
+
+int gsa_bwd_fused(const bf16* q, const bf16* k, const bf16* v, const bf16* phi, const bf16* g, const float* h01,
+                  const float* h02, const bf16* dO, const float* dhT1, const float* dhT2, bf16* dq, bf16* dk, bf16* dv,
+                  bf16* dphi, bf16* dg, float* dh01, float* dh02, int BH, int T, int dkd, int dvd, int m, void* ws,
+                  cudaStream_t st) {
+  Carve c(ws);
+  GsaFusedBwdWs w;
+  carve_gsa_fused_bwd(c, BH, T, dkd, dvd, m, &w);
+  const GsaFusedWs& f = w.f;
+  const long long rows = (long long)BH * T, sz = (long long)m * dvd, sp = 128LL * dvd, s1 = (long long)dkd * m;
+  // pass 1 forward again: the slot softmax p
+  GLA_CUDA(gla::gsa::pass1_fwd(q, k, phi, g, h01, w.p, nullptr, BH, T, dkd, w.p1ws, st));
+  // pass 2 backward (queries p, keys phi, values v), slots zero-padded to 128 keys
+  GLA_CUDA(gla::split::copy_cols(w.p, m, f.p, 128, rows, m, 128, st));
+  GLA_CUDA(gla::split::copy_cols(phi, m, f.phi, 128, rows, m, 128, st));
+  GLA_CUDA(gla::split::copy_cols(g, m, f.g, 128, rows, m, 128, st));
+  if (h02) GLA_CUDA(gla::split::copy_cols(h02, sz, f.h0, sp, BH, sz, sp, st));
+  if (dhT2) GLA_CUDA(gla::split::copy_cols(dhT2, sz, f.dhT, sp, BH, sz, sp, st));
+  const gla::fast::BwdAccum acc2{f.dq, f.dk, f.dg, f.dv, 128, 0, dvd, 0};
+  GLA_CUDA(gla::fast::bwd(f.p, f.phi, v, f.g, h02 ? f.h0 : nullptr, dO, dhT2 ? f.dhT : nullptr, nullptr, nullptr,
+                          nullptr, nullptr, dh02 ? f.dh0 : nullptr, BH, T, 128, dvd, f.ws, st, -1, -1, &acc2));
+  GLA_CUDA(gla::split::to_bf16(f.dv, dv, rows * dvd, st));
+  if (dh02) GLA_CUDA(gla::split::copy_cols(f.dh0, sp, dh02, sz, BH, sz, sz, st));
+  // slot softmax Jacobian: do1 = p (dp - <p, dp>)
+  GLA_CUDA(gla::gsa::softmax_jacobian(w.p, f.dq, 128, w.do1, w.do1_pad, rows, m, 128, st));
+  // pass 1 backward as a GLA backward: queries do1, keys phi, values k, dO' = q, states transposed
+  if (h01) GLA_CUDA(gla::gsa::transpose_states(h01, s1, w.h0p, BH, dkd, m, 128, st));
+  if (dhT1) GLA_CUDA(gla::gsa::transpose_states(dhT1, s1, w.dhTp, BH, dkd, m, 128, st));
+  const gla::fast::BwdAccum acc1{w.dq1, w.dphi1, w.dg1, w.dkf, 128, 0, dkd, 0};
+  GLA_CUDA(gla::fast::bwd(w.do1_pad, f.phi, k, f.g, h01 ? w.h0p : nullptr, q, dhT1 ? w.dhTp : nullptr, nullptr,
+                          nullptr, nullptr, nullptr, dh01 ? w.dh0p : nullptr, BH, T, 128, dkd, f.ws, st, -1, -1,
+                          &acc1));
+  // dq = S1 do1: the output of the GLA with queries do1, keys phi, values k from h0_1^T
+  if (h01) GLA_CUDA(gla::gsa::transpose_states(h01, s1, w.h0t, BH, dkd, m, m, st));
+  GLA_CUDA(gla::fast::fwd(w.do1, phi, k, g, h01 ? w.h0t : nullptr, dq, nullptr, BH, T, m, dkd, w.fws, st));
+  // both passes' contributions to dphi and dg; dk and dh0_1 back to the caller's layouts
+  GLA_CUDA(gla::gsa::add_cols_bf16(w.dphi1, f.dk, 128, dphi, rows, m, st));
+  GLA_CUDA(gla::gsa::add_cols_bf16(w.dg1, f.dg, 128, dg, rows, m, st));
+  GLA_CUDA(gla::split::to_bf16(w.dkf, dk, rows * dkd, st));
+  if (dh01) GLA_CUDA(gla::gsa::transpose_states(w.dh0p, 128LL * dkd, dh01, BH, m, dkd, dkd, st));
+  return GLA_OK;
 }
 
 template <typename TI>
@@ -470,9 +584,41 @@ size_t gla_chunk_fwd_workspace(int B, int H, int T, int dk, int dv, int chunk, i
   return carve_gla_fwd(c, B * H, T, dk, dv, chunk, nullptr);
 }
 
-int gla_chunk_fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
-                  int B, int H, int T, int dk, int dv, int chunk, int dtype, void* ws, size_t ws_bytes,
-                  void* stream) {
+size_t gla_chunk_bwd_workspace(int B, int H, int T, int dk, int dv, int chunk, int dtype) {
+  if (check_common(B, H, T, chunk, dtype) || check_dim(dk) || check_dim(dv)) return 0;
+  if (T == 0) return 0;
+  if (gla::fast::bwd_supported(B * H, T, dk, dv, chunk, dtype)) return gla::fast::bwd_workspace(B * H, T, dk, dv);
+  Carve c(nullptr);
+  if (split_bwd_ok(B * H, T, dk, dv, chunk, dtype)) return carve_split_bwd(c, B * H, T, dk, dv, nullptr);
+  return carve_gla_bwd(c, B * H, T, dk, dv, chunk, nullptr);
+}
+
+// Raw-logit entries: the fused and blocked paths form g = logsigmoid(x) / tau inside their gate
+// runs; the generic kernels take g from the standalone gate pass, written behind their workspace.
+size_t gla_chunk_fwd_logit_workspace(int B, int H, int T, int dk, int dv, int chunk, int dtype) {
+  const size_t base = gla_chunk_fwd_workspace(B, H, T, dk, dv, chunk, dtype);
+  if (T <= 0 || check_common(B, H, T, chunk, dtype) || check_dim(dk) || check_dim(dv)) return base;
+  if (gla::fast::fwd_supported(B * H, T, dk, dv, chunk, dtype) || split_fwd_ok(B * H, T, dk, dv, chunk, dtype))
+    return base;
+  return gla::align256(base) + gla::align256((size_t)B * H * T * dk * esize(dtype));
+}
+
+size_t gla_chunk_bwd_logit_workspace(int B, int H, int T, int dk, int dv, int chunk, int dtype) {
+  const size_t base = gla_chunk_bwd_workspace(B, H, T, dk, dv, chunk, dtype);
+  if (T <= 0 || check_common(B, H, T, chunk, dtype) || check_dim(dk) || check_dim(dv)) return base;
+  if (gla::fast::bwd_supported(B * H, T, dk, dv, chunk, dtype) || split_bwd_ok(B * H, T, dk, dv, chunk, dtype))
+    return base;
+  return gla::align256(base) + gla::align256((size_t)B * H * T * dk * esize(dtype));
+}
+
+}  // extern "C"
+
+namespace {
+
+// tau == 0: g holds log-gates; tau > 0: g holds raw logits x and the operator uses logsigmoid(x) / tau.
+int chunk_fwd_entry(const void* q, const void* k, const void* v, const void* g, float tau, const float* h0, void* o,
+                    float* hT, int B, int H, int T, int dk, int dv, int chunk, int dtype, void* ws, size_t ws_bytes,
+                    void* stream) {
   GLA_TRY(check_common(B, H, T, chunk, dtype));
   GLA_TRY(check_dim(dk));
   GLA_TRY(check_dim(dv));
@@ -484,16 +630,27 @@ int gla_chunk_fwd(const void* q, const void* k, const void* v, const void* g, co
   GLA_TRY(check_ptr(o, tok));
   GLA_TRY(check_ptr(h0, false));
   GLA_TRY(check_ptr(hT, false));
-  const size_t need = gla_chunk_fwd_workspace(B, H, T, dk, dv, chunk, dtype);
+  const bool logit = tau != 0.f;
+  if (logit && !(tau > 0.f && tau < 3.0e38f)) return GLA_ERR_INVALID_ARG;
+  const size_t need = logit ? gla_chunk_fwd_logit_workspace(B, H, T, dk, dv, chunk, dtype)
+                            : gla_chunk_fwd_workspace(B, H, T, dk, dv, chunk, dtype);
   if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return GLA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = B * H;
   if (T == 0) return copy_or_zero(hT, h0, (size_t)BH * dk * dv, st);
+  const float inv_tau = logit ? 1.f / tau : 0.f;
   if (gla::fast::fwd_supported(BH, T, dk, dv, chunk, dtype))
-    return gla::fast::fwd(q, k, v, g, h0, o, hT, BH, T, dk, dv, ws, st) == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+    return gla::fast::fwd(q, k, v, g, h0, o, hT, BH, T, dk, dv, ws, st, -1, -1, nullptr, inv_tau) == cudaSuccess
+               ? GLA_OK
+               : GLA_ERR_CUDA;
   if (split_fwd_ok(BH, T, dk, dv, chunk, dtype))
     return split_fwd((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)g, h0, (bf16*)o, hT, BH, T, dk, dv,
-                     ws, st);
+                     ws, st, inv_tau);
+  if (logit) {  // the standalone gate pass into the space behind the generic kernels' workspace
+    void* gbuf = static_cast<char*>(ws) + gla::align256(gla_chunk_fwd_workspace(B, H, T, dk, dv, chunk, dtype));
+    GLA_TRY(gla_gate_logsigmoid(g, gbuf, (size_t)BH * T * dk, tau, dtype, stream));
+    g = gbuf;
+  }
   const gk::Shape s{BH, T, dk, dv, chunk};
   if (dtype == GLA_DTYPE_BF16)
     return gla_fwd_generic<bf16>((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)g, h0, (bf16*)o, hT,
@@ -502,18 +659,9 @@ int gla_chunk_fwd(const void* q, const void* k, const void* v, const void* g, co
                                 hT, s, ws, st);
 }
 
-size_t gla_chunk_bwd_workspace(int B, int H, int T, int dk, int dv, int chunk, int dtype) {
-  if (check_common(B, H, T, chunk, dtype) || check_dim(dk) || check_dim(dv)) return 0;
-  if (T == 0) return 0;
-  if (gla::fast::bwd_supported(B * H, T, dk, dv, chunk, dtype)) return gla::fast::bwd_workspace(B * H, T, dk, dv);
-  Carve c(nullptr);
-  if (split_bwd_ok(B * H, T, dk, dv, chunk, dtype)) return carve_split_bwd(c, B * H, T, dk, dv, nullptr);
-  return carve_gla_bwd(c, B * H, T, dk, dv, chunk, nullptr);
-}
-
-int gla_chunk_bwd(const void* q, const void* k, const void* v, const void* g, const float* h0, const void* dO,
-                  const float* dhT, void* dq, void* dk, void* dv, void* dg, float* dh0, int B, int H, int T,
-                  int dkd, int dvd, int chunk, int dtype, void* ws, size_t ws_bytes, void* stream) {
+int chunk_bwd_entry(const void* q, const void* k, const void* v, const void* g, float tau, const float* h0,
+                    const void* dO, const float* dhT, void* dq, void* dk, void* dv, void* dg, float* dh0, int B, int H,
+                    int T, int dkd, int dvd, int chunk, int dtype, void* ws, size_t ws_bytes, void* stream) {
   GLA_TRY(check_common(B, H, T, chunk, dtype));
   GLA_TRY(check_dim(dkd));
   GLA_TRY(check_dim(dvd));
@@ -523,25 +671,72 @@ int gla_chunk_bwd(const void* q, const void* k, const void* v, const void* g, co
   GLA_TRY(check_ptr(h0, false));
   GLA_TRY(check_ptr(dhT, false));
   GLA_TRY(check_ptr(dh0, false));
-  const size_t need = gla_chunk_bwd_workspace(B, H, T, dkd, dvd, chunk, dtype);
+  const bool logit = tau != 0.f;
+  if (logit && !(tau > 0.f && tau < 3.0e38f)) return GLA_ERR_INVALID_ARG;
+  const size_t need = logit ? gla_chunk_bwd_logit_workspace(B, H, T, dkd, dvd, chunk, dtype)
+                            : gla_chunk_bwd_workspace(B, H, T, dkd, dvd, chunk, dtype);
   if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return GLA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = B * H;
   if (T == 0) return copy_or_zero(dh0, dhT, (size_t)BH * dkd * dvd, st);
+  const float inv_tau = logit ? 1.f / tau : 0.f;
   if (gla::fast::bwd_supported(BH, T, dkd, dvd, chunk, dtype))
-    return gla::fast::bwd(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, dkd, dvd, ws, st) == cudaSuccess
+    return gla::fast::bwd(q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, BH, T, dkd, dvd, ws, st, -1, -1, nullptr,
+                          inv_tau) == cudaSuccess
                ? GLA_OK
                : GLA_ERR_CUDA;
   if (split_bwd_ok(BH, T, dkd, dvd, chunk, dtype))
     return split_bwd((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)g, h0, (const bf16*)dO, dhT,
-                     (bf16*)dq, (bf16*)dk, (bf16*)dv, (bf16*)dg, dh0, BH, T, dkd, dvd, ws, st);
+                     (bf16*)dq, (bf16*)dk, (bf16*)dv, (bf16*)dg, dh0, BH, T, dkd, dvd, ws, st, inv_tau);
+  const void* x = g;
+  if (logit) {
+    void* gbuf = static_cast<char*>(ws) + gla::align256(gla_chunk_bwd_workspace(B, H, T, dkd, dvd, chunk, dtype));
+    GLA_TRY(gla_gate_logsigmoid(x, gbuf, (size_t)BH * T * dkd, tau, dtype, stream));
+    g = gbuf;
+  }
   const gk::Shape s{BH, T, dkd, dvd, chunk};
+  int r;
   if (dtype == GLA_DTYPE_BF16)
-    return gla_bwd_generic<bf16>((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)g, h0,
-                                 (const bf16*)dO, dhT, (bf16*)dq, (bf16*)dk, (bf16*)dv, (bf16*)dg, dh0, s, ws, st);
-  return gla_bwd_generic<float>((const float*)q, (const float*)k, (const float*)v, (const float*)g, h0,
-                                (const float*)dO, dhT, (float*)dq, (float*)dk, (float*)dv, (float*)dg, dh0, s, ws,
-                                st);
+    r = gla_bwd_generic<bf16>((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)g, h0, (const bf16*)dO, dhT,
+                              (bf16*)dq, (bf16*)dk, (bf16*)dv, (bf16*)dg, dh0, s, ws, st);
+  else
+    r = gla_bwd_generic<float>((const float*)q, (const float*)k, (const float*)v, (const float*)g, h0,
+                               (const float*)dO, dhT, (float*)dq, (float*)dk, (float*)dv, (float*)dg, dh0, s, ws, st);
+  if (r != GLA_OK || !logit) return r;
+  return gla_gate_logsigmoid_bwd(x, dg, dg, (size_t)BH * T * dkd, tau, dtype, stream);  // dx = dg sigmoid(-x) / tau
+}
+
+}  // namespace
+
+extern "C" {
+
+int gla_chunk_fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
+                  int B, int H, int T, int dk, int dv, int chunk, int dtype, void* ws, size_t ws_bytes,
+                  void* stream) {
+  return chunk_fwd_entry(q, k, v, g, 0.f, h0, o, hT, B, H, T, dk, dv, chunk, dtype, ws, ws_bytes, stream);
+}
+
+int gla_chunk_fwd_logit(const void* q, const void* k, const void* v, const void* x, float tau, const float* h0,
+                        void* o, float* hT, int B, int H, int T, int dk, int dv, int chunk, int dtype, void* ws,
+                        size_t ws_bytes, void* stream) {
+  if (!(tau > 0.f)) return GLA_ERR_INVALID_ARG;
+  return chunk_fwd_entry(q, k, v, x, tau, h0, o, hT, B, H, T, dk, dv, chunk, dtype, ws, ws_bytes, stream);
+}
+
+int gla_chunk_bwd(const void* q, const void* k, const void* v, const void* g, const float* h0, const void* dO,
+                  const float* dhT, void* dq, void* dk, void* dv, void* dg, float* dh0, int B, int H, int T,
+                  int dkd, int dvd, int chunk, int dtype, void* ws, size_t ws_bytes, void* stream) {
+  return chunk_bwd_entry(q, k, v, g, 0.f, h0, dO, dhT, dq, dk, dv, dg, dh0, B, H, T, dkd, dvd, chunk, dtype, ws,
+                         ws_bytes, stream);
+}
+
+int gla_chunk_bwd_logit(const void* q, const void* k, const void* v, const void* x, float tau, const float* h0,
+                        const void* dO, const float* dhT, void* dq, void* dk, void* dv, void* dx, float* dh0, int B,
+                        int H, int T, int dkd, int dvd, int chunk, int dtype, void* ws, size_t ws_bytes,
+                        void* stream) {
+  if (!(tau > 0.f)) return GLA_ERR_INVALID_ARG;
+  return chunk_bwd_entry(q, k, v, x, tau, h0, dO, dhT, dq, dk, dv, dx, dh0, B, H, T, dkd, dvd, chunk, dtype, ws,
+                         ws_bytes, stream);
 }
 
 int gla_recurrent_step(const void* q, const void* k, const void* v, const void* g, float* S, void* o, int B, int H,
@@ -566,6 +761,8 @@ size_t gsa_fwd_workspace(int B, int H, int T, int dk, int dv, int m, int chunk, 
   if (check_common(B, H, T, chunk, dtype) || check_dim(dk) || check_dim(dv) || check_dim(m)) return 0;
   if (T == 0) return 0;
   Carve c(nullptr);
+  if (gsa_fused_fwd_ok(B * H, T, dk, dv, m, chunk, dtype))
+    return carve_gsa_fused_fwd(c, B * H, T, dk, dv, m, true, nullptr);
   return carve_gsa_fwd(c, B * H, T, dk, dv, m, chunk, dtype, true, nullptr);
 }
 
@@ -589,6 +786,9 @@ int gsa_fwd(const void* q, const void* k, const void* v, const void* phi, const 
     GLA_TRY(copy_or_zero(hT1, h0_1, (size_t)BH * dk * m, st));
     return copy_or_zero(hT2, h0_2, (size_t)BH * m * dv, st);
   }
+  if (gsa_fused_fwd_ok(BH, T, dk, dv, m, chunk, dtype))
+    return gsa_fwd_fused((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)phi, (const bf16*)g, h0_1, h0_2,
+                         (bf16*)o, (bf16*)p_save, hT1, hT2, BH, T, dk, dv, m, ws, st);
   if (dtype == GLA_DTYPE_BF16)
     return gsa_fwd_impl<bf16>((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)phi, (const bf16*)g,
                               h0_1, h0_2, (bf16*)o, (bf16*)p_save, hT1, hT2, BH, T, dk, dv, m, chunk, ws, st);
@@ -601,6 +801,7 @@ size_t gsa_bwd_workspace(int B, int H, int T, int dk, int dv, int m, int chunk, 
   if (check_common(B, H, T, chunk, dtype) || check_dim(dk) || check_dim(dv) || check_dim(m)) return 0;
   if (T == 0) return 0;
   Carve c(nullptr);
+  if (gsa_fused_bwd_ok(B * H, T, dk, dv, m, chunk, dtype)) return carve_gsa_fused_bwd(c, B * H, T, dk, dv, m, nullptr);
   return carve_gsa_bwd(c, B * H, T, dk, dv, m, chunk, dtype, nullptr);
 }
 
@@ -625,6 +826,10 @@ int gsa_bwd(const void* q, const void* k, const void* v, const void* phi, const 
     GLA_TRY(copy_or_zero(dh0_1, dhT1, (size_t)BH * dkd * m, st));
     return copy_or_zero(dh0_2, dhT2, (size_t)BH * m * dvd, st);
   }
+  if (gsa_fused_bwd_ok(BH, T, dkd, dvd, m, chunk, dtype))
+    return gsa_bwd_fused((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)phi, (const bf16*)g, h0_1, h0_2,
+                         (const bf16*)dO, dhT1, dhT2, (bf16*)dq, (bf16*)dk, (bf16*)dv, (bf16*)dphi, (bf16*)dg, dh0_1,
+                         dh0_2, BH, T, dkd, dvd, m, ws, st);
   if (dtype == GLA_DTYPE_BF16)
     return gsa_bwd_impl<bf16>((const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)phi, (const bf16*)g,
                               h0_1, h0_2, (const bf16*)dO, dhT1, dhT2, (bf16*)dq, (bf16*)dk, (bf16*)dv, (bf16*)dphi,

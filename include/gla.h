@@ -109,6 +109,29 @@ int gla_chunk_bwd(const void* q, const void* k, const void* v, const void* g, co
                   void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * gla_chunk_fwd_logit / gla_chunk_bwd_logit - gla_chunk_fwd / gla_chunk_bwd with the gate given
+ * as raw logits: x [B,H,T,dk] in place of g, with g = logsigmoid(x) / tau formed inside the
+ * kernels' gate runs ("MS-GLA", section 2.1: a data-dependent forget gate; "Gated Slot
+ * Attention ...", "Approach": sigmoid forget gates, alpha = sigmoid(x)^(1/tau)).  The log-gates
+ * equal, value for value, what gla_gate_logsigmoid stores for x (so these calls return exactly
+ * what gla_gate_logsigmoid followed by gla_chunk_fwd / gla_chunk_bwd returns), without that
+ * pass's trip through memory.  The backward writes dx = dg * sigmoid(-x) / tau into `dx` in
+ * place of dg.  tau > 0 and finite (else GLA_ERR_INVALID_ARG).  Everything else, including the
+ * errors, as for gla_chunk_fwd / gla_chunk_bwd; the workspace is what the *_logit_workspace()
+ * query returns (the shapes the generic kernels serve need room for g behind their own).
+ * ------------------------------------------------------------------------------------- */
+size_t gla_chunk_fwd_logit_workspace(int B, int H, int T, int dk, int dv, int chunk, int dtype);
+int gla_chunk_fwd_logit(const void* q, const void* k, const void* v, const void* x, float tau,
+                        const float* h0, void* o, float* hT, int B, int H, int T, int dk, int dv,
+                        int chunk, int dtype, void* workspace, size_t workspace_bytes, void* stream);
+size_t gla_chunk_bwd_logit_workspace(int B, int H, int T, int dk, int dv, int chunk, int dtype);
+int gla_chunk_bwd_logit(const void* q, const void* k, const void* v, const void* x, float tau,
+                        const float* h0, const void* dO, const float* dhT, void* dq, void* dk,
+                        void* dv, void* dx, float* dh0, int B, int H, int T, int dk_dim,
+                        int dv_dim, int chunk, int dtype, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * gla_recurrent_step - one token of recurrent inference, in place on the state.
  *   in : q, k, g [B,H,dk]; v [B,H,dv]; S [B,H,dk,dv] fp32 (read, then overwritten)
  *   out: o [B,H,dv];  S <- diag(exp g) S + k^T v ; o = q S

@@ -99,3 +99,55 @@ def test_gsa_gate_variants(variant):
     ref = O.gsa_bwd(*a, None, None, f64(inp["do"]))
     for name, x, r in zip(["dq", "dk", "dv", "dphi", "dg"], grads, ref):
         assert_close(name, x, r, tol)
+
+
+def test_gsa_fused_near_reset_slots():
+    """bf16 at the fused shape (d_k = 128, m = 64, d_v = 128), with a few slots that forget (g = -30)
+    over a whole chunk or a short stretch: those chunks take the first pass's exact path (its
+    intra-chunk terms formed in fp32 from products of the decays).  Initial and final states on
+    both passes; every output and gradient against the oracle."""
+    B, H, T, dk, dv, m = 1, 2, 200, 128, 128, 64
+    tol = tol_for(torch.bfloat16)
+    inp = make_gsa_inputs(B, H, T, dk, dv, m, torch.bfloat16, seed=21)
+    g = inp["g"].float()
+    g[:, :, 64:128, 5] = -30.0
+    g[:, 1, 150:160, 40] = -30.0
+    inp["g"] = g.to(torch.bfloat16)
+    h1, h2, d1, d2 = _states(B, H, dk, dv, m, 22)
+    d = cuda(inp)
+    o, p, hT1, hT2 = gla.gsa_fwd(d["q"], d["k"], d["v"], d["phi"], d["g"], h0_1=h1.cuda(), h0_2=h2.cuda(),
+                                 save_p=True)
+    a = [f64(inp[n]) for n in ["q", "k", "v", "phi", "g"]]
+    ro, rp, rhT1, rhT2 = O.gsa_fwd(*a, f64(h1), f64(h2))
+    for name, x, r in [("o", o, ro), ("p", p, rp), ("hT1", hT1, rhT1), ("hT2", hT2, rhT2)]:
+        assert_close(name, x, r, tol)
+    grads = gla.gsa_bwd(d["q"], d["k"], d["v"], d["phi"], d["g"], d["do"], h0_1=h1.cuda(), h0_2=h2.cuda(),
+                        dhT1=d1.cuda(), dhT2=d2.cuda())
+    ref = O.gsa_bwd(*a, f64(h1), f64(h2), f64(inp["do"]), f64(d1), f64(d2))
+    for name, x, r in zip(["dq", "dk", "dv", "dphi", "dg", "dh0_1", "dh0_2"], grads, ref):
+        assert_close(name, x, r, tol)
+    assert gla.device_error() == 0
+
+
+def test_gsa_fused_many_heads_unsplit():
+    """80 heads fill the SMs, so the first pass runs one CTA per head over the whole sequence (no
+    sequence split); the first and the last head against the oracle."""
+    B, H, T, dk, dv, m = 4, 20, 130, 128, 128, 64
+    tol = tol_for(torch.bfloat16)
+    inp = make_gsa_inputs(B, H, T, dk, dv, m, torch.bfloat16, seed=23)
+    d = cuda(inp)
+    o, p, hT1, hT2 = gla.gsa_fwd(d["q"], d["k"], d["v"], d["phi"], d["g"], save_p=True)
+    grads = gla.gsa_bwd(d["q"], d["k"], d["v"], d["phi"], d["g"], d["do"])
+    idx = [(0, 0), (B - 1, H - 1)]
+
+    def heads(x):
+        return f64(torch.stack([x[b, h].cpu() for b, h in idx])[:, None])
+
+    sub = [heads(inp[n]) for n in ["q", "k", "v", "phi", "g"]]
+    ro, rp, rhT1, rhT2 = O.gsa_fwd(*sub)
+    for name, x, r in [("o", o, ro), ("p", p, rp), ("hT1", hT1, rhT1), ("hT2", hT2, rhT2)]:
+        assert_close(name, heads(x), r, tol)
+    ref = O.gsa_bwd(*sub, None, None, heads(inp["do"]))
+    for name, x, r in zip(["dq", "dk", "dv", "dphi", "dg", "dh0_1", "dh0_2"], grads, ref):
+        assert_close(name, heads(x), r, tol)
+    assert gla.device_error() == 0
