@@ -58,6 +58,8 @@ struct FwdArgs {
   int T, DV, seg_chunks, nseg;
   long long st_bh, st_row;  // h0 / hT strides (a sub-block of a larger state when the shape is split)
   float* acc_o;             // optional fp32 output [BH*T][DV] in place of o (split shapes)
+  const float* add_o;       // optional fp32 [BH*T][DV] added to o before it is stored (split shapes)
+  int ck, cv;               // first column of the CTA's key block in q / k / g and of v (wider tensors)
   float inv_tau;            // > 0: the gate tensor holds raw logits x, g = logsigmoid(x) / tau
   unsigned int* latch;
 };
@@ -123,9 +125,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int s = li & 1, chunk = REV ? c_end - 1 - li : c_begin + li;
     uint8_t* st = sm + s * L::STAGE;
     mbar_arrive_expect_tx(&bar_load[s], L::STAGE);
-    tma_load_3d(st, &tm_k, &bar_load[s], 0, chunk * C, bh);
-    tma_load_3d(st + L::RAW, &tm_g, &bar_load[s], 0, chunk * C, bh);
-    tma_load_3d(st + 2 * L::RAW, &tm_v, &bar_load[s], dv0, chunk * C, bh);
+    tma_load_3d(st, &tm_k, &bar_load[s], args.ck, chunk * C, bh);
+    tma_load_3d(st + L::RAW, &tm_g, &bar_load[s], args.ck, chunk * C, bh);
+    tma_load_3d(st + 2 * L::RAW, &tm_v, &bar_load[s], args.cv + dv0, chunk * C, bh);
   };
   if (tid == 0) {
     issue_load(0);
@@ -328,14 +330,14 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       const int s = li & 1, chunk = c_begin + li;
       uint8_t* st = sm + s * L::QKG;
       mbar_arrive_expect_tx(&bar_qkg[s], L::QKG);
-      tma_load_3d(st, &tm_q, &bar_qkg[s], 0, chunk * C, bh);
-      tma_load_3d(st + L::RAW, &tm_k, &bar_qkg[s], 0, chunk * C, bh);
-      tma_load_3d(st + 2 * L::RAW, &tm_g, &bar_qkg[s], 0, chunk * C, bh);
+      tma_load_3d(st, &tm_q, &bar_qkg[s], args.ck, chunk * C, bh);
+      tma_load_3d(st + L::RAW, &tm_k, &bar_qkg[s], args.ck, chunk * C, bh);
+      tma_load_3d(st + 2 * L::RAW, &tm_g, &bar_qkg[s], args.ck, chunk * C, bh);
     };
     auto load_v = [&](int li) {
       const int b = li % 3;
       mbar_arrive_expect_tx(&bar_v[b], L::VTB);
-      tma_load_3d(sm + L::V0 + b * L::VTB, &tm_v, &bar_v[b], dv0, (c_begin + li) * C, bh);
+      tma_load_3d(sm + L::V0 + b * L::VTB, &tm_v, &bar_v[b], args.cv + dv0, (c_begin + li) * C, bh);
     };
     if (lane == 0) {
       load_qkg(0);
@@ -499,12 +501,24 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       tmem_ld_wait();
       const int t = (c_begin + li) * C + j;
       if (lane < 16 && t < T) {
+        const size_t off = ((size_t)bh * T + t) * DV + dv0 + cb;
+        if (args.add_o) {  // a partial output of earlier key blocks
+          const float4* ad = reinterpret_cast<const float4*>(args.add_o + off);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float4 u = ad[c];
+            ov[4 * c] += u.x;
+            ov[4 * c + 1] += u.y;
+            ov[4 * c + 2] += u.z;
+            ov[4 * c + 3] += u.w;
+          }
+        }
         if (args.acc_o) {
-          float4* p = reinterpret_cast<float4*>(args.acc_o + ((size_t)bh * T + t) * DV + dv0 + cb);
+          float4* p = reinterpret_cast<float4*>(args.acc_o + off);
 #pragma unroll
           for (int c = 0; c < 8; ++c) p[c] = make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3]);
         } else {
-          store_half_global_bf16(args.o + ((size_t)bh * T + t) * DV + dv0 + cb, ov);
+          store_half_global_bf16(args.o + off, ov);
         }
       }
     };
@@ -669,10 +683,10 @@ static cudaError_t launch_state_pass(const CUtensorMap& mk, const CUtensorMap& m
 template <int DK>
 static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o,
                               float* hT, int BH, int T, int dv, long long st_bh, long long st_row, float* acc_o,
-                              void* ws, cudaStream_t st, float inv_tau) {
+                              void* ws, cudaStream_t st, float inv_tau, int dk_total, int k0, const float* add_o) {
   CUtensorMap m[4];
-  if (!make_map(&m[0], q, BH, T, DK, DK, false) || !make_map(&m[1], k, BH, T, DK, DK, false) ||
-      !make_map(&m[2], g, BH, T, DK, DK, false) || !make_map(&m[3], v, BH, T, dv, DVT, true))
+  if (!make_map(&m[0], q, BH, T, dk_total, DK, false) || !make_map(&m[1], k, BH, T, dk_total, DK, false) ||
+      !make_map(&m[2], g, BH, T, dk_total, DK, false) || !make_map(&m[3], v, BH, T, dv, DVT, true))
     return cudaErrorInvalidValue;
   FwdArgs a;
   a.h0 = h0;
@@ -683,6 +697,9 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
   a.st_bh = st_bh;
   a.st_row = st_row;
   a.acc_o = acc_o;
+  a.add_o = add_o;
+  a.ck = k0;
+  a.cv = 0;
   a.inv_tau = inv_tau;
   a.latch = device_error_latch();
   plan_segments(BH, T, dv, &a.nseg, &a.seg_chunks);
@@ -747,10 +764,13 @@ __global__ void segment_scan_rev_kernel(float* __restrict__ gbuf, const float* _
 cudaError_t segment_states(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mg,
                            const CUtensorMap& mv, const CUtensorMap& mdo, const float* h0, const float* dhT,
                            float* sbuf, float* gbuf, float* gam, int BH, int T, int dk, int dv, int nseg,
-                           int seg_chunks, long long st_bh, long long st_row, cudaStream_t st, float inv_tau) {
+                           int seg_chunks, long long st_bh, long long st_row, cudaStream_t st, float inv_tau, int ck,
+                           int cv) {
   if (dk != 128 || nseg < 2) return cudaErrorNotSupported;
   FwdArgs a = {};
   a.inv_tau = inv_tau;
+  a.ck = ck;
+  a.cv = cv;
   a.T = T;
   a.DV = dv;
   a.seg_chunks = seg_chunks;
@@ -808,11 +828,16 @@ cudaError_t segment_entry_states(const void* k, const void* g, const void* v, co
 
 cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
                 int BH, int T, int dk, int dv, void* ws, cudaStream_t st, long long st_bh, long long st_row,
-                float* acc_o, float inv_tau) {
+                float* acc_o, float inv_tau, int dk_total, int k0, const float* add_o) {
   if (st_bh < 0) st_bh = (long long)dk * dv;
   if (st_row < 0) st_row = dv;
-  if (dk == 64) return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st, inv_tau);
-  if (dk == 128) return launch_fwd<128>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st, inv_tau);
+  if (dk_total < 0) dk_total = dk;
+  if (k0 < 0 || k0 + dk > dk_total || k0 % 8 != 0) return cudaErrorInvalidValue;
+  if (dk == 64)
+    return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st, inv_tau, dk_total, k0, add_o);
+  if (dk == 128)
+    return launch_fwd<128>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st, inv_tau, dk_total, k0,
+                           add_o);
   return cudaErrorNotSupported;
 }
 

@@ -18,16 +18,23 @@ size_t fwd_workspace(int BH, int T, int dk, int dv);
 // st_bh / st_row: element strides of the fp32 states per head and per row (defaults, when
 // negative: dk*dv and dv).  A split shape passes a sub-block of the caller's states this way, and
 // an fp32 array acc_o [BH*T][dv] that receives o in place of the bf16 output.  inv_tau > 0: g holds
-// raw logits x and the kernels use g = bf16(logsigmoid(x) * inv_tau).
+// raw logits x and the kernels use g = bf16(logsigmoid(x) * inv_tau).  A key block of wider
+// tensors: q, k, g are [BH][T][dk_total] and the call uses columns k0 .. k0+dk-1 (read in place by
+// the tile loads); add_o ([BH*T][dv] fp32) is added to o before it is stored (to acc_o or as bf16).
 cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
                 int BH, int T, int dk, int dv, void* ws, cudaStream_t st, long long st_bh = -1,
-                long long st_row = -1, float* acc_o = nullptr, float inv_tau = 0.f);
+                long long st_row = -1, float* acc_o = nullptr, float inv_tau = 0.f, int dk_total = -1, int k0 = 0,
+                const float* add_o = nullptr);
 
-// fp32 outputs of a backward sub-problem (split shapes): dq / dk / dg go to columns ck.. of
-// [BH*T][pk] arrays, dv to columns cv.. of a [BH*T][pv] array.
+// A backward sub-problem inside wider tensors (split shapes, padded operands): its key dimensions
+// are columns ck.. of [BH*T][pk] arrays (the q, k, g inputs and every key-side output array), its
+// value columns are cv.. of [BH*T][pv] arrays (v, dO and the dv arrays).  A non-null q / k / g / v
+// receives that gradient in fp32 (a partial sum) in place of the bf16 output; otherwise the bf16
+// output is written, after adding add_q / add_k / add_g / add_v (fp32 partial sums) where given.
 struct BwdAccum {
   float *q, *k, *g, *v;
   int pk, ck, pv, cv;
+  const float *add_q, *add_k, *add_g, *add_v;
 };
 
 // Sequence split of the backward (d_k = 128): segment count and length, and the segment states
@@ -38,7 +45,8 @@ void plan_bwd_segments(int ctas_per_seg, int T, int* nseg, int* seg_chunks);
 cudaError_t segment_states(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mg,
                            const CUtensorMap& mv, const CUtensorMap& mdo, const float* h0, const float* dhT,
                            float* sbuf, float* gbuf, float* gam, int BH, int T, int dk, int dv, int nseg,
-                           int seg_chunks, long long st_bh, long long st_row, cudaStream_t st, float inv_tau);
+                           int seg_chunks, long long st_bh, long long st_row, cudaStream_t st, float inv_tau, int ck,
+                           int cv);
 
 // SM count of the current device (cached per device).
 int sm_count();

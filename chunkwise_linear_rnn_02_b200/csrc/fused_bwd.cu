@@ -68,17 +68,30 @@ struct BwdArgs {
   int nseg, seg_chunks, n_bh;
   const float *s_in, *g_end;
   long long st_bh, st_row;  // h0 / dhT / dh0 strides (a sub-block of a larger state when split)
-  // Optional fp32 outputs for a split shape: when set, dq / dk / dg go to columns acc_ck + key dim
-  // of [BH*T][acc_pk] arrays and dv to columns acc_cv + value col of a [BH*T][acc_pv] array, in
-  // place of the bf16 outputs.
+  // Outputs: with acc_x set, x goes in fp32 to acc_x (a partial sum of a split shape); else in bf16
+  // to the output, plus add_x (fp32: the partial sum of earlier sub-problems) where that is set.
+  // Key-side arrays (the q, k, g inputs, dq, dk, dg and their acc / add arrays) are [BH*T][pk] with
+  // this call's key dimensions from column ck; value-side ones (v, dO, dv, acc_v, add_v) are
+  // [BH*T][pv] with this call's value columns from cv.  The tile loads read them in place.
   float *acc_q, *acc_k, *acc_g, *acc_v;
-  int acc_pk, acc_ck, acc_pv, acc_cv;
+  const float *add_q, *add_k, *add_g, *add_v;
+  int pk, ck, pv, cv;
   // > 0: the gate tensor holds raw logits x (g = logsigmoid(x) / tau) and the gate-gradient output
   // receives dx = dg sigmoid(-x) / tau in place of dg
   float inv_tau;
   unsigned int* latch;
 };
 
+
+// One gradient value plus the partial sum in add (if any): fp32 into acc (itself a partial sum, which
+// may be add's own element) or bf16 into out.
+__device__ __forceinline__ void store_out(float* acc, const float* add, __nv_bfloat16* out, size_t idx, float val) {
+  if (add) val += add[idx];
+  if (acc)
+    acc[idx] = val;
+  else
+    out[idx] = __float2bfloat16_rn(val);
+}
 
 // ------------------------------------------------------------------------------------------
 // Key-tile CTA
@@ -134,7 +147,7 @@ struct KeyLayout {
 // buffer, Kh operand, state copy and rescale) and issue its group 1; then finish chunk i's
 // outputs.  The epilogue forms E1 / E2 itself from the raw gates and the run products of the gate
 // run, multiplying in the same order, so its values equal the ones behind the MMA operands.
-template <int DK, int DV, bool ACC>
+template <int DK, int DV>
 __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int tau, int seg,
                               uint64_t* bars, uint32_t tmem) {
   using L = KeyLayout<DK, DV>;
@@ -167,16 +180,16 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   auto load_a = [&](int chunk) {
     mbar_arrive_expect_tx(bar_pa, 2 * L::VB);
     for (int bb = 0; bb < DV / 64; ++bb) {
-      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, bar_pa, bb * 64, chunk * C, bh);
-      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, bar_pa, bb * 64, chunk * C, bh);
+      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, bar_pa, a.cv + bb * 64, chunk * C, bh);
+      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, bar_pa, a.cv + bb * 64, chunk * C, bh);
     }
   };
   auto load_b = [&](int chunk, int b) {
     uint8_t* pb = sm + pbo(b);
     mbar_arrive_expect_tx(bar_pb + b, L::PB_STAGE);
-    tma_load_3d(pb + L::PB_K, &mp.k64, bar_pb + b, d0, chunk * C, bh);
-    tma_load_3d(pb + L::PB_G, &mp.g64, bar_pb + b, d0, chunk * C, bh);
-    tma_load_3d(pb + L::PB_Q, &mp.q64, bar_pb + b, d0, chunk * C, bh);
+    tma_load_3d(pb + L::PB_K, &mp.k64, bar_pb + b, a.ck + d0, chunk * C, bh);
+    tma_load_3d(pb + L::PB_G, &mp.g64, bar_pb + b, a.ck + d0, chunk * C, bh);
+    tma_load_3d(pb + L::PB_Q, &mp.q64, bar_pb + b, a.ck + d0, chunk * C, bh);
   };
   auto wait_b = [&](int b) {
     mbar_wait(bar_pb + b, (ph_pb >> b) & 1u, a.latch);
@@ -366,8 +379,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         }
       }
       const float inv = 1.f / DEC[b * KT + d];
-      __nv_bfloat16* dst = a.dq + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
-      float* dst32 = ACC ? a.acc_q + ((size_t)bh * T + i * C + tb) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
+      const size_t ob = ((size_t)bh * T + i * C + tb) * a.pk + a.ck + d0 + d;  // output index, token tb
 #pragma unroll
       for (int rr = 0; rr < 4; ++rr) {
         float e = 1.f;  // E1 = e^{B_j}, formed as GateRun::forward forms it
@@ -379,10 +391,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
           if (!safe) y[c] *= e * inv;
           const float qv = raw(pq, j, d), kv = raw(pk, j, d);
           if (i * C + j < T) {
-            if (ACC)
-              dst32[(size_t)c * a.acc_pk] = e * x[c] + y[c];
-            else
-              dst[(size_t)c * DK] = __float2bfloat16_rn(e * x[c] + y[c]);
+            store_out(a.acc_q, a.add_q, a.dq, ob + (size_t)c * a.pk, e * x[c] + y[c]);
           }
           x[c] = bf_split_sum(qv * e) * x[c];  // Qt X, with Qt as the G update sees it
           y[c] = qv * (y[c] - DIAG[j] * kv);   // q dq^intra without j = r
@@ -473,7 +482,7 @@ struct ValLayout {
   static_assert(C * DK * 4 <= KH_HI - QP_HI && C * C * 4 <= GC_HI - KH_HI, "exact-path scratch");
 };
 
-template <int DK, bool ACC>
+template <int DK>
 __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int vt, int DV, int seg,
                               uint64_t* bars, uint32_t tmem) {
   using L = ValLayout<DK>;
@@ -500,15 +509,15 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   // issued as soon as those reads are done; dO and v once the second MMA group has completed.
   auto load_qkg = [&](int chunk) {
     mbar_arrive_expect_tx(bar_ld, 3 * L::RAW);
-    tma_load_3d(sm, &mp.q_all, bar_ld, 0, chunk * C, bh);
-    tma_load_3d(sm + L::RAW, &mp.k_all, bar_ld, 0, chunk * C, bh);
-    tma_load_3d(sm + 2 * L::RAW, &mp.g_all, bar_ld, 0, chunk * C, bh);
+    tma_load_3d(sm, &mp.q_all, bar_ld, a.ck, chunk * C, bh);
+    tma_load_3d(sm + L::RAW, &mp.k_all, bar_ld, a.ck, chunk * C, bh);
+    tma_load_3d(sm + 2 * L::RAW, &mp.g_all, bar_ld, a.ck, chunk * C, bh);
   };
   auto load_dov = [&](int chunk) {
     mbar_arrive_expect_tx(bar_dv, L::DOT + C * VT * 2);
     for (int b = 0; b < VT / 64; ++b) {
-      tma_load_3d(sm + 3 * L::RAW + b * (C * 128), &mp.dO, bar_dv, c0 + b * 64, chunk * C, bh);
-      tma_load_3d(sm + L::VZ + b * (C * 128), &mp.v, bar_dv, c0 + b * 64, chunk * C, bh);
+      tma_load_3d(sm + 3 * L::RAW + b * (C * 128), &mp.dO, bar_dv, a.cv + c0 + b * 64, chunk * C, bh);
+      tma_load_3d(sm + L::VZ + b * (C * 128), &mp.v, bar_dv, a.cv + c0 + b * 64, chunk * C, bh);
     }
   };
   auto sync_tc = [&]() {
@@ -728,17 +737,10 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       const int vcol = q4 * 32 + lane, t0 = i * C + half * 32;
       tmem_ld32(tmem + L::T_DV + lane_off + half * 32, v);
       tmem_ld_wait();
-      if (ACC) {
-        float* p = a.acc_v + ((size_t)bh * T + t0) * a.acc_pv + a.acc_cv + c0 + vcol;
+      const size_t ob = ((size_t)bh * T + t0) * a.pv + a.cv + c0 + vcol;  // output index, token t0
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (t0 + c < T) p[(size_t)c * a.acc_pv] = v[c];
-      } else {
-        __nv_bfloat16* p = a.dv + ((size_t)bh * T + t0) * DV + c0 + vcol;
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (t0 + c < T) p[(size_t)c * DV] = __float2bfloat16_rn(v[c]);
-      }
+      for (int c = 0; c < 32; ++c)
+        if (t0 + c < T) store_out(a.acc_v, a.add_v, a.dv, ob + (size_t)c * a.pv, v[c]);
     }
     tc_fence_before();
     __syncthreads();
@@ -825,7 +827,7 @@ struct ChunkLayout {
   static_assert(PB % 1024 == 0 && KQ_HI % 1024 == 0 && 2 * TILE <= VB, "operand layout");
 };
 
-template <int DK, int DV, bool ACC>
+template <int DK, int DV>
 __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
   using L = ChunkLayout<DK, DV>;
   using Gate = GateRun<KT, BT>;
@@ -866,12 +868,12 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   if (tid == 0) {
     mbar_arrive_expect_tx(&bar_ld, 2 * L::VB + 3 * L::TILE);
     for (int bb = 0; bb < DV / 64; ++bb) {
-      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, &bar_ld, bb * 64, i * C, bh);
-      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, &bar_ld, bb * 64, i * C, bh);
+      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, &bar_ld, a.cv + bb * 64, i * C, bh);
+      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, &bar_ld, a.cv + bb * 64, i * C, bh);
     }
-    tma_load_3d(sm + L::PB_K, &mp.k64, &bar_ld, d0, i * C, bh);
-    tma_load_3d(sm + L::PB_G, &mp.g64, &bar_ld, d0, i * C, bh);
-    tma_load_3d(sm + L::PB_Q, &mp.q64, &bar_ld, d0, i * C, bh);
+    tma_load_3d(sm + L::PB_K, &mp.k64, &bar_ld, a.ck + d0, i * C, bh);
+    tma_load_3d(sm + L::PB_G, &mp.g64, &bar_ld, a.ck + d0, i * C, bh);
+    tma_load_3d(sm + L::PB_Q, &mp.q64, &bar_ld, a.ck + d0, i * C, bh);
   }
   // The epilogue runs on all 32 lanes: lane l < 16 owns key dim row = q4 * 16 + l for tokens
   // tb .. tb + 15, lane l + 16 the same dim for tokens tb + 16 .. tb + 31 (the M = 64 accumulators
@@ -1005,8 +1007,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   float tot_s = 0.f;
   {  // dk; per-token terms Kh Z + k dk^intra without j = r (-> w)
     const float inv = 1.f / DEC[d];
-    __nv_bfloat16* dst = a.dk + ((size_t)bh * T + i * C + tq) * DK + d0 + d;
-    float* dst32 = ACC ? a.acc_k + ((size_t)bh * T + i * C + tq) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
+    const size_t ob = ((size_t)bh * T + i * C + tq) * a.pk + a.ck + d0 + d;  // output index, token tq
 #pragma unroll
     for (int rr = 0; rr < 16 / TS; ++rr) {
       const int h = tq / TS + rr;
@@ -1027,10 +1028,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
         if (!safe) w[c] *= ev * inv;
         const float qv = raw(L::PB_Q, r, d), kv = raw(L::PB_K, r, d);
         if (i * C + r < T) {
-          if (ACC)
-            dst32[(size_t)c * a.acc_pk] = ev * z[c] + w[c];
-          else
-            dst[(size_t)c * DK] = __float2bfloat16_rn(ev * z[c] + w[c]);
+          store_out(a.acc_k, a.add_k, a.dk, ob + (size_t)c * a.pk, ev * z[c] + w[c]);
         }
         const float kz = bf_split_sum(kv * ev) * z[c];  // Kh Z, with Kh as the S update sees it
         w[c] = kz + kv * (w[c] - DIAG[r] * qv);        // plus k dk^intra without j = r
@@ -1044,8 +1042,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   {  // dg = c_i + prefix (exclusive) of (Kh Z + k dk^intra) + the forward walk's part
     float pre = 0.f;
     for (int t = 0; t < qi; ++t) pre += XQ[t * KT + d];
-    __nv_bfloat16* dst = a.dg + ((size_t)bh * T + i * C + tq) * DK + d0 + d;
-    float* dst32 = ACC ? a.acc_g + ((size_t)bh * T + i * C + tq) * a.acc_pk + a.acc_ck + d0 + d : nullptr;
+    const size_t ob = ((size_t)bh * T + i * C + tq) * a.pk + a.ck + d0 + d;  // output index, token tq
     const float tau = a.inv_tau > 0.f ? 1.f / a.inv_tau : 0.f;
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
@@ -1053,10 +1050,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
         float dgv = ci + pre + pv[c];
         // raw logits: dx = dg sigmoid(-x) / tau, with sigmoid(-x) = 1 - e^{tau g} = -expm1(tau g)
         if (a.inv_tau > 0.f) dgv *= -expm1f(tau * raw(L::PB_G, tq + c, d)) * a.inv_tau;
-        if (ACC)
-          dst32[(size_t)c * a.acc_pk] = dgv;
-        else
-          dst[(size_t)c * DK] = __float2bfloat16_rn(dgv);
+        store_out(a.acc_g, a.add_g, a.dg, ob + (size_t)c * a.pk, dgv);
       }
       pre += w[c];
     }
@@ -1076,7 +1070,7 @@ struct BwdSmem {
   static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
 
-template <int DK, int DV, bool ACC>
+template <int DK, int DV>
 __global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bars[5];
@@ -1100,20 +1094,20 @@ __global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant_
   const int per_seg = a.n_bh * per_head;
   const int seg = blockIdx.x / per_seg, bh = (blockIdx.x % per_seg) / per_head, role = blockIdx.x % per_head;
   if (role < DK / KT)
-    key_tile_body<DK, DV, ACC>(sm, mp, a, bh, role, seg, bars, tmem);
+    key_tile_body<DK, DV>(sm, mp, a, bh, role, seg, bars, tmem);
   else
-    val_tile_body<DK, ACC>(sm, mp, a, bh, role - DK / KT, DV, seg, bars, tmem);
+    val_tile_body<DK>(sm, mp, a, bh, role - DK / KT, DV, seg, bars, tmem);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-template <int DK, int DV, bool ACC>
+template <int DK, int DV>
 static cudaError_t launch_all(const BwdMaps& mp, const BwdArgs& a, int BH, cudaStream_t st) {
   constexpr uint32_t CHK = ChunkLayout<DK, DV>::TOTAL + 1024;
   static_assert(2 * CHK <= 228 * 1024, "two chunk CTAs per SM");
-  auto k1 = bwd_fused_kernel<DK, DV, ACC>;
-  auto k3 = bwd_chunk_kernel<DK, DV, ACC>;
+  auto k1 = bwd_fused_kernel<DK, DV>;
+  auto k3 = bwd_chunk_kernel<DK, DV>;
   static std::atomic<bool> attr1[64] = {}, attr3[64] = {};
   {
     cudaError_t e = ensure_smem_attr(k1, BwdSmem<DK, DV>::ALLOC, attr1);
@@ -1169,12 +1163,15 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
                               const void* dO, const float* dhT, void* dq, void* dk, void* dv, void* dg, float* dh0,
                               int BH, int T, void* ws, cudaStream_t st, long long st_bh, long long st_row,
                               const BwdAccum* acc, float inv_tau) {
+  // pitch and first column of this sub-problem's key dims and value columns in the tensors given
+  const int PK = acc ? acc->pk : DK, CK = acc ? acc->ck : 0, PV = acc ? acc->pv : DV, CV = acc ? acc->cv : 0;
+  if (CK < 0 || CK + DK > PK || CK % 8 || CV < 0 || CV + DV > PV || CV % 8) return cudaErrorInvalidValue;
   BwdMaps mp;
-  if (!make_map(&mp.v, v, BH, T, DV, 64, true) || !make_map(&mp.dO, dO, BH, T, DV, 64, true) ||
-      !make_map(&mp.k64, k, BH, T, DK, KT, true) || !make_map(&mp.g64, g, BH, T, DK, KT, true) ||
-      !make_map(&mp.q64, q, BH, T, DK, KT, true) ||
-      !make_map(&mp.q_all, q, BH, T, DK, DK, false) || !make_map(&mp.k_all, k, BH, T, DK, DK, false) ||
-      !make_map(&mp.g_all, g, BH, T, DK, DK, false))
+  if (!make_map(&mp.v, v, BH, T, PV, 64, true) || !make_map(&mp.dO, dO, BH, T, PV, 64, true) ||
+      !make_map(&mp.k64, k, BH, T, PK, KT, true) || !make_map(&mp.g64, g, BH, T, PK, KT, true) ||
+      !make_map(&mp.q64, q, BH, T, PK, KT, true) ||
+      !make_map(&mp.q_all, q, BH, T, PK, DK, false) || !make_map(&mp.k_all, k, BH, T, PK, DK, false) ||
+      !make_map(&mp.g_all, g, BH, T, PK, DK, false))
     return cudaErrorInvalidValue;
   BwdArgs a;
   a.h0 = h0;
@@ -1191,10 +1188,14 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
   a.acc_k = acc ? acc->k : nullptr;
   a.acc_g = acc ? acc->g : nullptr;
   a.acc_v = acc ? acc->v : nullptr;
-  a.acc_pk = acc ? acc->pk : 0;
-  a.acc_ck = acc ? acc->ck : 0;
-  a.acc_pv = acc ? acc->pv : 0;
-  a.acc_cv = acc ? acc->cv : 0;
+  a.add_q = acc ? acc->add_q : nullptr;
+  a.add_k = acc ? acc->add_k : nullptr;
+  a.add_g = acc ? acc->add_g : nullptr;
+  a.add_v = acc ? acc->add_v : nullptr;
+  a.pk = PK;
+  a.ck = CK;
+  a.pv = PV;
+  a.cv = CV;
   a.inv_tau = inv_tau;
   size_t sz[9];
   bwd_parts(BH, T, DK, DV, sz, &a.nseg, &a.seg_chunks);
@@ -1213,10 +1214,10 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
   a.latch = device_error_latch();
   if (a.nseg > 1) {
     const cudaError_t e = segment_states(mp.q_all, mp.k_all, mp.g_all, mp.v, mp.dO, h0, dhT, p[6], p[7], p[8], BH, T,
-                                         DK, DV, a.nseg, a.seg_chunks, st_bh, st_row, st, inv_tau);
+                                         DK, DV, a.nseg, a.seg_chunks, st_bh, st_row, st, inv_tau, CK, CV);
     if (e != cudaSuccess) return e;
   }
-  return acc ? launch_all<DK, DV, true>(mp, a, BH, st) : launch_all<DK, DV, false>(mp, a, BH, st);
+  return launch_all<DK, DV>(mp, a, BH, st);
 }
 
 cudaError_t bwd(const void* q, const void* k, const void* v, const void* g, const float* h0, const void* dO,

@@ -79,8 +79,10 @@ struct Carve {
 // its rows of hT.  The loss <dO, o> is a sum over value columns, so the backward is also a sum of
 // sub-problems over value blocks: dq, dk, dg of a key block sum over the value blocks, dv of a
 // value block sums over the key blocks, and dh0 / dhT are the (key, value) blocks of the state.
-// Key blocks are 128 wide; value blocks 256 (or 128) wide for the backward.  Inputs are gathered
-// into contiguous blocks, sub-results accumulate in fp32.
+// Key blocks are 128 wide; value blocks 256 (or 128) wide for the backward.  The kernels read
+// their blocks of q, k, g, v, dO in place (the tile loads take the block's first column); every
+// sub-problem but the last of an output block leaves an fp32 partial sum, which the next one adds
+// in its epilogue; the last writes the bf16 result.
 // ----------------------------------------------------------------------------------------
 constexpr int kSplitK = 128;
 int split_vblock(int dv) { return dv % 256 == 0 ? 256 : 128; }
@@ -96,19 +98,13 @@ bool split_bwd_ok(int BH, int T, int dk, int dv, int chunk, int dtype) {
 }
 
 struct SplitFwdWs {
-  bf16 *q, *k, *g;
-  float *acc, *part;
+  float* acc;  // [BH*T][dv] partial output of the key blocks so far
   void* fws;
 };
 size_t carve_split_fwd(Carve& c, int BH, int T, int dk, int dv, SplitFwdWs* w) {
-  (void)dk;  // key blocks are gathered one at a time, so no part depends on d_k
-  const size_t rows = (size_t)BH * T;
+  (void)dk;
   SplitFwdWs x;
-  x.q = c.take<bf16>(rows * kSplitK);
-  x.k = c.take<bf16>(rows * kSplitK);
-  x.g = c.take<bf16>(rows * kSplitK);
-  x.acc = c.take<float>(rows * dv);
-  x.part = c.take<float>(rows * dv);
+  x.acc = c.take<float>((size_t)BH * T * dv);
   x.fws = c.take<char>(gla::fast::fwd_workspace(BH, T, kSplitK, dv));
   if (w) *w = x;
   return c.used;
@@ -119,44 +115,29 @@ int split_fwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const 
   Carve c(ws);
   SplitFwdWs w;
   carve_split_fwd(c, BH, T, dk, dv, &w);
-  const long long rows = (long long)BH * T;
-  for (int kb = 0; kb < dk / kSplitK; ++kb) {
+  const int nk = dk / kSplitK;
+  for (int kb = 0; kb < nk; ++kb) {
     const int c0 = kb * kSplitK;
-    GLA_CUDA(gla::split::gather_cols(q, w.q, rows, dk, c0, kSplitK, st));
-    GLA_CUDA(gla::split::gather_cols(k, w.k, rows, dk, c0, kSplitK, st));
-    GLA_CUDA(gla::split::gather_cols(g, w.g, rows, dk, c0, kSplitK, st));
-    GLA_CUDA(gla::fast::fwd(w.q, w.k, v, w.g, h0 ? h0 + (size_t)c0 * dv : nullptr, nullptr,
-                            hT ? hT + (size_t)c0 * dv : nullptr, BH, T, kSplitK, dv, w.fws, st, (long long)dk * dv,
-                            dv, kb == 0 ? w.acc : w.part, inv_tau));
-    if (kb > 0) GLA_CUDA(gla::split::add_cols(w.part, w.acc, rows, dv, dv, 0, st));
+    GLA_CUDA(gla::fast::fwd(q, k, v, g, h0 ? h0 + (size_t)c0 * dv : nullptr, o, hT ? hT + (size_t)c0 * dv : nullptr, BH,
+                            T, kSplitK, dv, w.fws, st, (long long)dk * dv, dv, kb < nk - 1 ? w.acc : nullptr, inv_tau,
+                            dk, c0, kb > 0 ? w.acc : nullptr));
   }
-  GLA_CUDA(gla::split::to_bf16(w.acc, o, rows * dv, st));
   return GLA_OK;
 }
 
 struct SplitBwdWs {
-  bf16 *q, *k, *g, *v, *dO;
-  float *aq, *ak, *ag, *av;  // accumulators, full width
-  float *pq, *pk, *pg, *pv;  // one sub-problem's outputs, block width
+  float *aq, *ak, *ag;  // [BH*T][dk] partial key-side gradients (over value blocks)
+  float* av;            // [BH*T][dv] partial dv (over key blocks)
   void* bws;
 };
 size_t carve_split_bwd(Carve& c, int BH, int T, int dk, int dv, SplitBwdWs* w) {
   const size_t rows = (size_t)BH * T;
-  const int vb = split_vblock(dv), nv = dv / vb;
+  const int vb = split_vblock(dv), nv = dv / vb, nk = dk / kSplitK;
   SplitBwdWs x;
-  x.q = c.take<bf16>(rows * kSplitK);
-  x.k = c.take<bf16>(rows * kSplitK);
-  x.g = c.take<bf16>(rows * kSplitK);
-  x.v = nv > 1 ? c.take<bf16>(rows * dv) : nullptr;  // all value blocks, gathered once
-  x.dO = nv > 1 ? c.take<bf16>(rows * dv) : nullptr;
-  x.aq = c.take<float>(rows * dk);
-  x.ak = c.take<float>(rows * dk);
-  x.ag = c.take<float>(rows * dk);
-  x.av = c.take<float>(rows * dv);
-  x.pq = c.take<float>(rows * kSplitK);
-  x.pk = c.take<float>(rows * kSplitK);
-  x.pg = c.take<float>(rows * kSplitK);
-  x.pv = c.take<float>(rows * vb);
+  x.aq = nv > 1 ? c.take<float>(rows * dk) : nullptr;
+  x.ak = nv > 1 ? c.take<float>(rows * dk) : nullptr;
+  x.ag = nv > 1 ? c.take<float>(rows * dk) : nullptr;
+  x.av = nk > 1 ? c.take<float>(rows * dv) : nullptr;
   x.bws = c.take<char>(gla::fast::bwd_workspace(BH, T, kSplitK, vb));
   if (w) *w = x;
   return c.used;
@@ -168,48 +149,24 @@ int split_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const 
   Carve c(ws);
   SplitBwdWs w;
   carve_split_bwd(c, BH, T, dkd, dvd, &w);
-  const long long rows = (long long)BH * T;
   const int vb = split_vblock(dvd), nv = dvd / vb, nk = dkd / kSplitK;
-  for (int vi = 0; nv > 1 && vi < nv; ++vi) {
-    GLA_CUDA(gla::split::gather_cols(v, w.v + (size_t)vi * rows * vb, rows, dvd, vi * vb, vb, st));
-    GLA_CUDA(gla::split::gather_cols(dO, w.dO + (size_t)vi * rows * vb, rows, dvd, vi * vb, vb, st));
-  }
   for (int kb = 0; kb < nk; ++kb) {
     const int k0 = kb * kSplitK;
-    const bf16 *qb = q, *kbp = k, *gb = g;
-    if (nk > 1) {
-      GLA_CUDA(gla::split::gather_cols(q, w.q, rows, dkd, k0, kSplitK, st));
-      GLA_CUDA(gla::split::gather_cols(k, w.k, rows, dkd, k0, kSplitK, st));
-      GLA_CUDA(gla::split::gather_cols(g, w.g, rows, dkd, k0, kSplitK, st));
-      qb = w.q;
-      kbp = w.k;
-      gb = w.g;
-    }
     for (int vi = 0; vi < nv; ++vi) {
       const int v0 = vi * vb;
-      const bf16* vvb = nv > 1 ? w.v + (size_t)vi * rows * vb : v;
-      const bf16* dob = nv > 1 ? w.dO + (size_t)vi * rows * vb : dO;
       const size_t so = (size_t)k0 * dvd + v0;  // state block (k0.., v0..) of every head
-      // the first sub-problem of a block writes straight into the accumulator's columns, later ones
-      // into a block-wide buffer that is then added
-      const bool fk = vi == 0, fv = kb == 0;
-      const gla::fast::BwdAccum out{fk ? w.aq : w.pq, fk ? w.ak : w.pk, fk ? w.ag : w.pg, fv ? w.av : w.pv,
-                                    fk ? dkd : kSplitK, fk ? k0 : 0, fv ? dvd : vb, fv ? v0 : 0};
-      GLA_CUDA(gla::fast::bwd(qb, kbp, vvb, gb, h0 ? h0 + so : nullptr, dob, dhT ? dhT + so : nullptr, nullptr,
-                              nullptr, nullptr, nullptr, dh0 ? dh0 + so : nullptr, BH, T, kSplitK, vb, w.bws, st,
-                              (long long)dkd * dvd, dvd, &out, inv_tau));
-      if (!fk) {
-        GLA_CUDA(gla::split::add_cols(w.pq, w.aq, rows, kSplitK, dkd, k0, st));
-        GLA_CUDA(gla::split::add_cols(w.pk, w.ak, rows, kSplitK, dkd, k0, st));
-        GLA_CUDA(gla::split::add_cols(w.pg, w.ag, rows, kSplitK, dkd, k0, st));
-      }
-      if (!fv) GLA_CUDA(gla::split::add_cols(w.pv, w.av, rows, vb, dvd, v0, st));
+      // key-side gradients sum over the value blocks, dv over the key blocks: every sub-problem but
+      // the last of a block leaves an fp32 partial sum that the next one adds
+      const bool kpart = vi < nv - 1, kadd = vi > 0, vpart = kb < nk - 1, vadd = kb > 0;
+      const gla::fast::BwdAccum out{kpart ? w.aq : nullptr, kpart ? w.ak : nullptr, kpart ? w.ag : nullptr,
+                                    vpart ? w.av : nullptr, dkd, k0, dvd, v0,
+                                    kadd ? w.aq : nullptr, kadd ? w.ak : nullptr, kadd ? w.ag : nullptr,
+                                    vadd ? w.av : nullptr};
+      GLA_CUDA(gla::fast::bwd(q, k, v, g, h0 ? h0 + so : nullptr, dO, dhT ? dhT + so : nullptr, dq, dk, dv, dg,
+                              dh0 ? dh0 + so : nullptr, BH, T, kSplitK, vb, w.bws, st, (long long)dkd * dvd, dvd, &out,
+                              inv_tau));
     }
   }
-  GLA_CUDA(gla::split::to_bf16(w.aq, dq, rows * dkd, st));
-  GLA_CUDA(gla::split::to_bf16(w.ak, dk, rows * dkd, st));
-  GLA_CUDA(gla::split::to_bf16(w.ag, dg, rows * dkd, st));
-  GLA_CUDA(gla::split::to_bf16(w.av, dv, rows * dvd, st));
   return GLA_OK;
 }
 
@@ -394,7 +351,7 @@ size_t carve_gsa_fused_fwd(Carve& c, int BH, int T, int dk, int dv, int m, bool 
 struct GsaFusedBwdWs {
   GsaFusedWs f;                   // pass 2: padded operands, fp32 gradients, padded states, bwd workspace
   bf16 *p, *do1, *do1_pad;        // [rows][m], [rows][m], [rows][128]
-  float *dq1, *dphi1, *dg1, *dkf;  // pass-1 backward outputs: [rows][128] x 3, [rows][dk]
+  float *dq1, *dphi1, *dg1;        // pass-1 backward outputs: [rows][128] x 3
   float *h0p, *dhTp, *dh0p, *h0t;  // [BH][128][dk] x 3, [BH][m][dk]
   void *p1ws, *fws;
 };
@@ -408,7 +365,6 @@ size_t carve_gsa_fused_bwd(Carve& c, int BH, int T, int dk, int dv, int m, GsaFu
   x.dq1 = c.take<float>(rows * 128);
   x.dphi1 = c.take<float>(rows * 128);
   x.dg1 = c.take<float>(rows * 128);
-  x.dkf = c.take<float>(rows * dk);
   x.h0p = c.take<float>(sp);
   x.dhTp = c.take<float>(sp);
   x.dh0p = c.take<float>(sp);
@@ -448,27 +404,24 @@ int gsa_bwd_fused(const bf16* q, const bf16* k, const bf16* v, const bf16* phi, 
   GLA_CUDA(gla::split::copy_cols(g, m, f.g, 128, rows, m, 128, st));
   if (h02) GLA_CUDA(gla::split::copy_cols(h02, sz, f.h0, sp, BH, sz, sp, st));
   if (dhT2) GLA_CUDA(gla::split::copy_cols(dhT2, sz, f.dhT, sp, BH, sz, sp, st));
-  const gla::fast::BwdAccum acc2{f.dq, f.dk, f.dg, f.dv, 128, 0, dvd, 0};
-  GLA_CUDA(gla::fast::bwd(f.p, f.phi, v, f.g, h02 ? f.h0 : nullptr, dO, dhT2 ? f.dhT : nullptr, nullptr, nullptr,
-                          nullptr, nullptr, dh02 ? f.dh0 : nullptr, BH, T, 128, dvd, f.ws, st, -1, -1, &acc2));
-  GLA_CUDA(gla::split::to_bf16(f.dv, dv, rows * dvd, st));
+  const gla::fast::BwdAccum acc2{f.dq, f.dk, f.dg, nullptr, 128, 0, dvd, 0};  // dv straight to bf16
+  GLA_CUDA(gla::fast::bwd(f.p, f.phi, v, f.g, h02 ? f.h0 : nullptr, dO, dhT2 ? f.dhT : nullptr, nullptr, nullptr, dv,
+                          nullptr, dh02 ? f.dh0 : nullptr, BH, T, 128, dvd, f.ws, st, -1, -1, &acc2));
   if (dh02) GLA_CUDA(gla::split::copy_cols(f.dh0, sp, dh02, sz, BH, sz, sz, st));
   // slot softmax Jacobian: do1 = p (dp - <p, dp>)
   GLA_CUDA(gla::gsa::softmax_jacobian(w.p, f.dq, 128, w.do1, w.do1_pad, rows, m, 128, st));
   // pass 1 backward as a GLA backward: queries do1, keys phi, values k, dO' = q, states transposed
   if (h01) GLA_CUDA(gla::gsa::transpose_states(h01, s1, w.h0p, BH, dkd, m, 128, st));
   if (dhT1) GLA_CUDA(gla::gsa::transpose_states(dhT1, s1, w.dhTp, BH, dkd, m, 128, st));
-  const gla::fast::BwdAccum acc1{w.dq1, w.dphi1, w.dg1, w.dkf, 128, 0, dkd, 0};
+  const gla::fast::BwdAccum acc1{w.dq1, w.dphi1, w.dg1, nullptr, 128, 0, dkd, 0};  // dk (its dv) straight to bf16
   GLA_CUDA(gla::fast::bwd(w.do1_pad, f.phi, k, f.g, h01 ? w.h0p : nullptr, q, dhT1 ? w.dhTp : nullptr, nullptr,
-                          nullptr, nullptr, nullptr, dh01 ? w.dh0p : nullptr, BH, T, 128, dkd, f.ws, st, -1, -1,
-                          &acc1));
+                          nullptr, dk, nullptr, dh01 ? w.dh0p : nullptr, BH, T, 128, dkd, f.ws, st, -1, -1, &acc1));
   // dq = S1 do1: the output of the GLA with queries do1, keys phi, values k from h0_1^T
   if (h01) GLA_CUDA(gla::gsa::transpose_states(h01, s1, w.h0t, BH, dkd, m, m, st));
   GLA_CUDA(gla::fast::fwd(w.do1, phi, k, g, h01 ? w.h0t : nullptr, dq, nullptr, BH, T, m, dkd, w.fws, st));
   // both passes' contributions to dphi and dg; dk and dh0_1 back to the caller's layouts
   GLA_CUDA(gla::gsa::add_cols_bf16(w.dphi1, f.dk, 128, dphi, rows, m, st));
   GLA_CUDA(gla::gsa::add_cols_bf16(w.dg1, f.dg, 128, dg, rows, m, st));
-  GLA_CUDA(gla::split::to_bf16(w.dkf, dk, rows * dkd, st));
   if (dh01) GLA_CUDA(gla::gsa::transpose_states(w.dh0p, 128LL * dkd, dh01, BH, m, dkd, dkd, st));
   return GLA_OK;
 }
