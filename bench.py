@@ -374,6 +374,32 @@ def extra_workloads(args, dev, flush, peaks):
             gla.recurrent_step(t["q"], t["k"], t["v"], t["g"], S)
 
     f_ms, dec_ms = time_pair(long_fwd, decode, max(3, steps // 2), 3, flush)
+    # the same 256 steps captured once as a CUDA graph and replayed: the device time per step
+    # without the host's per-call overhead (the state is rewritten in place by every replay)
+    graph_us = None
+    try:
+        S0 = state["S"].clone()
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            decode()  # warm-up on the capturing stream
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            decode()
+        reps = 10
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        state["S"].copy_(S0)
+        graph.replay()
+        e0.record()
+        for _ in range(reps):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        graph_us = 1e3 * e0.elapsed_time(e1) / (reps * n_dec)
+        del graph
+    except Exception as exc:  # capture unavailable: keep the eager figure only
+        graph_us = f"not captured: {exc}"
     fb, _, ff, _ = algorithmic(cfg)
     roof = roofline_ms(fb, ff, peaks)
     dec_bytes = cfg.B * cfg.H * (2 * cfg.dk * cfg.dv * 4 + (3 * cfg.dk + 2 * cfg.dv) * 2)
@@ -382,8 +408,11 @@ def extra_workloads(args, dev, flush, peaks):
                        "fwd_ms": f_ms, "fwd_tokens_per_s": cfg.B * cfg.T / (f_ms / 1e3), "fwd_roofline_ms": roof,
                        "fwd_pct_of_roofline": 100 * roof / f_ms,
                        "decode_us_per_step": 1e3 * dec_ms / n_dec,
+                       "decode_graph_us_per_step": graph_us,
                        "decode_roofline_us_per_step": 1e6 * dec_bytes / (peaks["hbm_gbs"] * 1e9),
-                       "decode_note": "one launch per token, L2 not flushed between decode steps (the 0.5 MB "
+                       "decode_note": "one launch per token; decode_us_per_step from eager calls (host-bound: "
+                                      "Python and ctypes per call), decode_graph_us_per_step from a CUDA-graph "
+                                      "replay of the 256 calls; L2 not flushed between decode steps (the 0.5 MB "
                                       "state stays resident, as in serving)"}
     del d, head, toks, state
     # GSA with 64 slots

@@ -90,12 +90,13 @@ struct StateLayout {
   static_assert(STAGE % 1024 == 0 && RAW % 1024 == 0, "stage alignment");
 };
 
-template <int DK, bool HILO, bool REV>
+template <int DK, bool HILO, bool REV, bool FLEX>
 __global__ void __launch_bounds__(NTHREADS, 1)
     fwd_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_g,
                      const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
   using L = StateLayout<DK, HILO>;
-  using Gate = GateRun<DK, NTHREADS>;
+  using Gate = GateRun<DK, NTHREADS, FLEX>;
+  const int ck = FLEX ? args.ck : 0, cv = FLEX ? args.cv : 0;  // column offsets into wider tensors
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_load[2], bar_mma;
   __shared__ uint32_t tmem_base_sh;
@@ -125,9 +126,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int s = li & 1, chunk = REV ? c_end - 1 - li : c_begin + li;
     uint8_t* st = sm + s * L::STAGE;
     mbar_arrive_expect_tx(&bar_load[s], L::STAGE);
-    tma_load_3d(st, &tm_k, &bar_load[s], args.ck, chunk * C, bh);
-    tma_load_3d(st + L::RAW, &tm_g, &bar_load[s], args.ck, chunk * C, bh);
-    tma_load_3d(st + 2 * L::RAW, &tm_v, &bar_load[s], args.cv + dv0, chunk * C, bh);
+    tma_load_3d(st, &tm_k, &bar_load[s], ck, chunk * C, bh);
+    tma_load_3d(st + L::RAW, &tm_g, &bar_load[s], ck, chunk * C, bh);
+    tma_load_3d(st + 2 * L::RAW, &tm_v, &bar_load[s], cv + dv0, chunk * C, bh);
   };
   if (tid == 0) {
     issue_load(0);
@@ -277,13 +278,16 @@ struct FwdPipeLayout {
 constexpr int PIPE_THREADS = NTHREADS + 32;  // 8 compute warps + the producer warp
 constexpr int kBarOps = 2, kBarAB = 3;       // compute threads -> producer handoffs
 
-template <int DK>
+// FLEX: the build for wider tensors (column offsets, fp32 partial outputs with an added partial) and
+// raw-logit gates; the plain build has none of that code.
+template <int DK, bool FLEX>
 __global__ void __launch_bounds__(PIPE_THREADS, 1)
     fwd_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
                     const FwdArgs args) {
   using L = FwdPipeLayout<DK>;
-  using Gate = GateRun<DK, NTHREADS>;
+  using Gate = GateRun<DK, NTHREADS, FLEX>;
+  const int ck = FLEX ? args.ck : 0, cv = FLEX ? args.cv : 0;  // column offsets into wider tensors
   constexpr int TS = Gate::TS;
   constexpr int NHAND = NTHREADS + 32;  // threads taking part in a handoff barrier
   extern __shared__ uint8_t smem_raw[];
@@ -330,14 +334,14 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       const int s = li & 1, chunk = c_begin + li;
       uint8_t* st = sm + s * L::QKG;
       mbar_arrive_expect_tx(&bar_qkg[s], L::QKG);
-      tma_load_3d(st, &tm_q, &bar_qkg[s], args.ck, chunk * C, bh);
-      tma_load_3d(st + L::RAW, &tm_k, &bar_qkg[s], args.ck, chunk * C, bh);
-      tma_load_3d(st + 2 * L::RAW, &tm_g, &bar_qkg[s], args.ck, chunk * C, bh);
+      tma_load_3d(st, &tm_q, &bar_qkg[s], ck, chunk * C, bh);
+      tma_load_3d(st + L::RAW, &tm_k, &bar_qkg[s], ck, chunk * C, bh);
+      tma_load_3d(st + 2 * L::RAW, &tm_g, &bar_qkg[s], ck, chunk * C, bh);
     };
     auto load_v = [&](int li) {
       const int b = li % 3;
       mbar_arrive_expect_tx(&bar_v[b], L::VTB);
-      tma_load_3d(sm + L::V0 + b * L::VTB, &tm_v, &bar_v[b], args.cv + dv0, (c_begin + li) * C, bh);
+      tma_load_3d(sm + L::V0 + b * L::VTB, &tm_v, &bar_v[b], cv + dv0, (c_begin + li) * C, bh);
     };
     if (lane == 0) {
       load_qkg(0);
@@ -502,7 +506,7 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       const int t = (c_begin + li) * C + j;
       if (lane < 16 && t < T) {
         const size_t off = ((size_t)bh * T + t) * DV + dv0 + cb;
-        if (args.add_o) {  // a partial output of earlier key blocks
+        if (FLEX && args.add_o) {  // a partial output of earlier key blocks
           const float4* ad = reinterpret_cast<const float4*>(args.add_o + off);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -513,7 +517,7 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
             ov[4 * c + 3] += u.w;
           }
         }
-        if (args.acc_o) {
+        if (FLEX && args.acc_o) {
           float4* p = reinterpret_cast<float4*>(args.acc_o + off);
 #pragma unroll
           for (int c = 0; c < 8; ++c) p[c] = make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3]);
@@ -668,10 +672,10 @@ size_t fwd_workspace(int BH, int T, int dk, int dv) {
 }
 
 // m: maps of the operand ([64 x DK] rows), the gates, and the 64-column value tiles.
-template <int DK, bool HILO, bool REV>
+template <int DK, bool HILO, bool REV, bool FLEX>
 static cudaError_t launch_state_pass(const CUtensorMap& mk, const CUtensorMap& mg, const CUtensorMap& mv,
                                      const FwdArgs& args, int BH, int dv, cudaStream_t st) {
-  auto kern = fwd_state_kernel<DK, HILO, REV>;
+  auto kern = fwd_state_kernel<DK, HILO, REV, FLEX>;
   static std::atomic<bool> attr_set[64] = {};
   const cudaError_t e = ensure_smem_attr(kern, StateLayout<DK, HILO>::ALLOC, attr_set);
   if (e != cudaSuccess) return e;
@@ -702,6 +706,7 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
   a.cv = 0;
   a.inv_tau = inv_tau;
   a.latch = device_error_latch();
+  const bool flex = inv_tau > 0.f || acc_o || add_o || k0 != 0 || dk_total != DK;
   plan_segments(BH, T, dv, &a.nseg, &a.seg_chunks);
   a.sbuf = nullptr;
   a.gam = nullptr;
@@ -709,7 +714,8 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
     if (!ws) return cudaErrorInvalidValue;
     a.sbuf = static_cast<float*>(ws);
     a.gam = a.sbuf + align256((size_t)BH * a.nseg * DK * dv * sizeof(float)) / sizeof(float);
-    cudaError_t e = launch_state_pass<DK, false, false>(m[1], m[2], m[3], a, BH, dv, st);
+    cudaError_t e = flex ? launch_state_pass<DK, false, false, true>(m[1], m[2], m[3], a, BH, dv, st)
+                         : launch_state_pass<DK, false, false, false>(m[1], m[2], m[3], a, BH, dv, st);
     if (e != cudaSuccess) return e;
     if (a.nseg > 2) {
       const size_t n = (size_t)BH * DK * dv;
@@ -719,10 +725,10 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
       if (e != cudaSuccess) return e;
     }
   }
-  auto kern = fwd_pipe_kernel<DK>;
-  static std::atomic<bool> attr_set[64] = {};
+  auto kern = flex ? fwd_pipe_kernel<DK, true> : fwd_pipe_kernel<DK, false>;
+  static std::atomic<bool> attr_set[2][64] = {};
   {
-    const cudaError_t e = ensure_smem_attr(kern, FwdPipeLayout<DK>::ALLOC, attr_set);
+    const cudaError_t e = ensure_smem_attr(kern, FwdPipeLayout<DK>::ALLOC, attr_set[flex ? 1 : 0]);
     if (e != cudaSuccess) return e;
   }
   dim3 grid(dv / DVT, BH, a.nseg);
@@ -781,13 +787,16 @@ cudaError_t segment_states(const CUtensorMap& mq, const CUtensorMap& mk, const C
   a.h0 = h0;
   a.sbuf = sbuf;
   a.gam = gam;
-  cudaError_t e = launch_state_pass<128, true, false>(mk, mg, mv, a, BH, dv, st);
+  const bool flex = inv_tau > 0.f || ck != 0 || cv != 0;
+  cudaError_t e = flex ? launch_state_pass<128, true, false, true>(mk, mg, mv, a, BH, dv, st)
+                       : launch_state_pass<128, true, false, false>(mk, mg, mv, a, BH, dv, st);
   if (e != cudaSuccess) return e;
   FwdArgs r = a;
   r.h0 = dhT;
   r.sbuf = gbuf;
   r.gam = nullptr;
-  e = launch_state_pass<128, true, true>(mq, mg, mdo, r, BH, dv, st);
+  e = flex ? launch_state_pass<128, true, true, true>(mq, mg, mdo, r, BH, dv, st)
+           : launch_state_pass<128, true, true, false>(mq, mg, mdo, r, BH, dv, st);
   if (e != cudaSuccess) return e;
   if (nseg > 2) {
     const size_t n = (size_t)BH * dk * dv;
@@ -818,7 +827,7 @@ cudaError_t segment_entry_states(const void* k, const void* g, const void* v, co
   a.st_bh = (long long)dk * dv;
   a.st_row = dv;
   a.latch = device_error_latch();
-  cudaError_t e = launch_state_pass<64, false, false>(m[0], m[1], m[2], a, BH, dv, st);
+  cudaError_t e = launch_state_pass<64, false, false, false>(m[0], m[1], m[2], a, BH, dv, st);
   if (e != cudaSuccess || nseg < 3) return e;
   const size_t n = (size_t)BH * dk * dv;
   const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);

@@ -83,14 +83,18 @@ struct BwdArgs {
 };
 
 
-// One gradient value plus the partial sum in add (if any): fp32 into acc (itself a partial sum, which
-// may be add's own element) or bf16 into out.
+// One gradient value.  FLEX builds: plus the partial sum in add (if any), then fp32 into acc (itself
+// a partial sum, which may be add's own element) or bf16 into out; the plain build stores bf16.
+template <bool FLEX>
 __device__ __forceinline__ void store_out(float* acc, const float* add, __nv_bfloat16* out, size_t idx, float val) {
-  if (add) val += add[idx];
-  if (acc)
-    acc[idx] = val;
-  else
-    out[idx] = __float2bfloat16_rn(val);
+  if (FLEX) {
+    if (add) val += add[idx];
+    if (acc) {
+      acc[idx] = val;
+      return;
+    }
+  }
+  out[idx] = __float2bfloat16_rn(val);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -147,12 +151,14 @@ struct KeyLayout {
 // buffer, Kh operand, state copy and rescale) and issue its group 1; then finish chunk i's
 // outputs.  The epilogue forms E1 / E2 itself from the raw gates and the run products of the gate
 // run, multiplying in the same order, so its values equal the ones behind the MMA operands.
-template <int DK, int DV>
+template <int DK, int DV, bool FLEX>
 __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int tau, int seg,
                               uint64_t* bars, uint32_t tmem) {
   using L = KeyLayout<DK, DV>;
-  using Gate = GateRun<KT, BT>;
+  using Gate = GateRun<KT, BT, FLEX>;
   constexpr int NS = L::NS, TS = Gate::TS;
+  // column offsets into wider tensors and the key-side row pitch (FLEX builds only)
+  const int ck = FLEX ? a.ck : 0, cv = FLEX ? a.cv : 0, pk = FLEX ? a.pk : DK;
   static_assert(TS == 8 && NS == 8, "epilogue runs: four gate runs of eight tokens per token half");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
@@ -180,16 +186,16 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   auto load_a = [&](int chunk) {
     mbar_arrive_expect_tx(bar_pa, 2 * L::VB);
     for (int bb = 0; bb < DV / 64; ++bb) {
-      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, bar_pa, a.cv + bb * 64, chunk * C, bh);
-      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, bar_pa, a.cv + bb * 64, chunk * C, bh);
+      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, bar_pa, cv + bb * 64, chunk * C, bh);
+      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, bar_pa, cv + bb * 64, chunk * C, bh);
     }
   };
   auto load_b = [&](int chunk, int b) {
     uint8_t* pb = sm + pbo(b);
     mbar_arrive_expect_tx(bar_pb + b, L::PB_STAGE);
-    tma_load_3d(pb + L::PB_K, &mp.k64, bar_pb + b, a.ck + d0, chunk * C, bh);
-    tma_load_3d(pb + L::PB_G, &mp.g64, bar_pb + b, a.ck + d0, chunk * C, bh);
-    tma_load_3d(pb + L::PB_Q, &mp.q64, bar_pb + b, a.ck + d0, chunk * C, bh);
+    tma_load_3d(pb + L::PB_K, &mp.k64, bar_pb + b, ck + d0, chunk * C, bh);
+    tma_load_3d(pb + L::PB_G, &mp.g64, bar_pb + b, ck + d0, chunk * C, bh);
+    tma_load_3d(pb + L::PB_Q, &mp.q64, bar_pb + b, ck + d0, chunk * C, bh);
   };
   auto wait_b = [&](int b) {
     mbar_wait(bar_pb + b, (ph_pb >> b) & 1u, a.latch);
@@ -379,7 +385,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         }
       }
       const float inv = 1.f / DEC[b * KT + d];
-      const size_t ob = ((size_t)bh * T + i * C + tb) * a.pk + a.ck + d0 + d;  // output index, token tb
+      const size_t ob = ((size_t)bh * T + i * C + tb) * pk + ck + d0 + d;  // output index, token tb
 #pragma unroll
       for (int rr = 0; rr < 4; ++rr) {
         float e = 1.f;  // E1 = e^{B_j}, formed as GateRun::forward forms it
@@ -391,7 +397,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
           if (!safe) y[c] *= e * inv;
           const float qv = raw(pq, j, d), kv = raw(pk, j, d);
           if (i * C + j < T) {
-            store_out(a.acc_q, a.add_q, a.dq, ob + (size_t)c * a.pk, e * x[c] + y[c]);
+            store_out<FLEX>(a.acc_q, a.add_q, a.dq, ob + (size_t)c * pk, e * x[c] + y[c]);
           }
           x[c] = bf_split_sum(qv * e) * x[c];  // Qt X, with Qt as the G update sees it
           y[c] = qv * (y[c] - DIAG[j] * kv);   // q dq^intra without j = r
@@ -482,11 +488,13 @@ struct ValLayout {
   static_assert(C * DK * 4 <= KH_HI - QP_HI && C * C * 4 <= GC_HI - KH_HI, "exact-path scratch");
 };
 
-template <int DK>
+template <int DK, bool FLEX>
 __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int vt, int DV, int seg,
                               uint64_t* bars, uint32_t tmem) {
   using L = ValLayout<DK>;
-  using Gate = GateRun<DK, BT>;
+  using Gate = GateRun<DK, BT, FLEX>;
+  // column offsets into wider tensors and the value-side row pitch (FLEX builds only)
+  const int ck = FLEX ? a.ck : 0, cv = FLEX ? a.cv : 0, pv = FLEX ? a.pv : DV;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = a.T, NC = (T + C - 1) / C, c0 = vt * VT;
   const int ch0 = seg * a.seg_chunks, ch1 = min(NC, ch0 + a.seg_chunks), nl = ch1 - ch0;  // segment
@@ -509,15 +517,15 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   // issued as soon as those reads are done; dO and v once the second MMA group has completed.
   auto load_qkg = [&](int chunk) {
     mbar_arrive_expect_tx(bar_ld, 3 * L::RAW);
-    tma_load_3d(sm, &mp.q_all, bar_ld, a.ck, chunk * C, bh);
-    tma_load_3d(sm + L::RAW, &mp.k_all, bar_ld, a.ck, chunk * C, bh);
-    tma_load_3d(sm + 2 * L::RAW, &mp.g_all, bar_ld, a.ck, chunk * C, bh);
+    tma_load_3d(sm, &mp.q_all, bar_ld, ck, chunk * C, bh);
+    tma_load_3d(sm + L::RAW, &mp.k_all, bar_ld, ck, chunk * C, bh);
+    tma_load_3d(sm + 2 * L::RAW, &mp.g_all, bar_ld, ck, chunk * C, bh);
   };
   auto load_dov = [&](int chunk) {
     mbar_arrive_expect_tx(bar_dv, L::DOT + C * VT * 2);
     for (int b = 0; b < VT / 64; ++b) {
-      tma_load_3d(sm + 3 * L::RAW + b * (C * 128), &mp.dO, bar_dv, a.cv + c0 + b * 64, chunk * C, bh);
-      tma_load_3d(sm + L::VZ + b * (C * 128), &mp.v, bar_dv, a.cv + c0 + b * 64, chunk * C, bh);
+      tma_load_3d(sm + 3 * L::RAW + b * (C * 128), &mp.dO, bar_dv, cv + c0 + b * 64, chunk * C, bh);
+      tma_load_3d(sm + L::VZ + b * (C * 128), &mp.v, bar_dv, cv + c0 + b * 64, chunk * C, bh);
     }
   };
   auto sync_tc = [&]() {
@@ -737,10 +745,10 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       const int vcol = q4 * 32 + lane, t0 = i * C + half * 32;
       tmem_ld32(tmem + L::T_DV + lane_off + half * 32, v);
       tmem_ld_wait();
-      const size_t ob = ((size_t)bh * T + t0) * a.pv + a.cv + c0 + vcol;  // output index, token t0
+      const size_t ob = ((size_t)bh * T + t0) * pv + cv + c0 + vcol;  // output index, token t0
 #pragma unroll
       for (int c = 0; c < 32; ++c)
-        if (t0 + c < T) store_out(a.acc_v, a.add_v, a.dv, ob + (size_t)c * a.pv, v[c]);
+        if (t0 + c < T) store_out<FLEX>(a.acc_v, a.add_v, a.dv, ob + (size_t)c * pv, v[c]);
     }
     tc_fence_before();
     __syncthreads();
@@ -827,10 +835,12 @@ struct ChunkLayout {
   static_assert(PB % 1024 == 0 && KQ_HI % 1024 == 0 && 2 * TILE <= VB, "operand layout");
 };
 
-template <int DK, int DV>
+template <int DK, int DV, bool FLEX>
 __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
   using L = ChunkLayout<DK, DV>;
-  using Gate = GateRun<KT, BT>;
+  using Gate = GateRun<KT, BT, FLEX>;
+  // column offsets into wider tensors and the key-side row pitch (FLEX builds only)
+  const int ck = FLEX ? a.ck : 0, cv = FLEX ? a.cv : 0, pk = FLEX ? a.pk : DK;
   constexpr int NS = L::NS, TS = Gate::TS, NVT = DV / VT;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_ld, bar_m1, bar_m2;
@@ -868,12 +878,12 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   if (tid == 0) {
     mbar_arrive_expect_tx(&bar_ld, 2 * L::VB + 3 * L::TILE);
     for (int bb = 0; bb < DV / 64; ++bb) {
-      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, &bar_ld, a.cv + bb * 64, i * C, bh);
-      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, &bar_ld, a.cv + bb * 64, i * C, bh);
+      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, &bar_ld, cv + bb * 64, i * C, bh);
+      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, &bar_ld, cv + bb * 64, i * C, bh);
     }
-    tma_load_3d(sm + L::PB_K, &mp.k64, &bar_ld, a.ck + d0, i * C, bh);
-    tma_load_3d(sm + L::PB_G, &mp.g64, &bar_ld, a.ck + d0, i * C, bh);
-    tma_load_3d(sm + L::PB_Q, &mp.q64, &bar_ld, a.ck + d0, i * C, bh);
+    tma_load_3d(sm + L::PB_K, &mp.k64, &bar_ld, ck + d0, i * C, bh);
+    tma_load_3d(sm + L::PB_G, &mp.g64, &bar_ld, ck + d0, i * C, bh);
+    tma_load_3d(sm + L::PB_Q, &mp.q64, &bar_ld, ck + d0, i * C, bh);
   }
   // The epilogue runs on all 32 lanes: lane l < 16 owns key dim row = q4 * 16 + l for tokens
   // tb .. tb + 15, lane l + 16 the same dim for tokens tb + 16 .. tb + 31 (the M = 64 accumulators
@@ -1007,7 +1017,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   float tot_s = 0.f;
   {  // dk; per-token terms Kh Z + k dk^intra without j = r (-> w)
     const float inv = 1.f / DEC[d];
-    const size_t ob = ((size_t)bh * T + i * C + tq) * a.pk + a.ck + d0 + d;  // output index, token tq
+    const size_t ob = ((size_t)bh * T + i * C + tq) * pk + ck + d0 + d;  // output index, token tq
 #pragma unroll
     for (int rr = 0; rr < 16 / TS; ++rr) {
       const int h = tq / TS + rr;
@@ -1028,7 +1038,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
         if (!safe) w[c] *= ev * inv;
         const float qv = raw(L::PB_Q, r, d), kv = raw(L::PB_K, r, d);
         if (i * C + r < T) {
-          store_out(a.acc_k, a.add_k, a.dk, ob + (size_t)c * a.pk, ev * z[c] + w[c]);
+          store_out<FLEX>(a.acc_k, a.add_k, a.dk, ob + (size_t)c * pk, ev * z[c] + w[c]);
         }
         const float kz = bf_split_sum(kv * ev) * z[c];  // Kh Z, with Kh as the S update sees it
         w[c] = kz + kv * (w[c] - DIAG[r] * qv);        // plus k dk^intra without j = r
@@ -1042,15 +1052,15 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   {  // dg = c_i + prefix (exclusive) of (Kh Z + k dk^intra) + the forward walk's part
     float pre = 0.f;
     for (int t = 0; t < qi; ++t) pre += XQ[t * KT + d];
-    const size_t ob = ((size_t)bh * T + i * C + tq) * a.pk + a.ck + d0 + d;  // output index, token tq
-    const float tau = a.inv_tau > 0.f ? 1.f / a.inv_tau : 0.f;
+    const size_t ob = ((size_t)bh * T + i * C + tq) * pk + ck + d0 + d;  // output index, token tq
+    const float tau = FLEX && a.inv_tau > 0.f ? 1.f / a.inv_tau : 0.f;
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       if (i * C + tq + c < T) {
         float dgv = ci + pre + pv[c];
         // raw logits: dx = dg sigmoid(-x) / tau, with sigmoid(-x) = 1 - e^{tau g} = -expm1(tau g)
-        if (a.inv_tau > 0.f) dgv *= -expm1f(tau * raw(L::PB_G, tq + c, d)) * a.inv_tau;
-        store_out(a.acc_g, a.add_g, a.dg, ob + (size_t)c * a.pk, dgv);
+        if (FLEX && a.inv_tau > 0.f) dgv *= -expm1f(tau * raw(L::PB_G, tq + c, d)) * a.inv_tau;
+        store_out<FLEX>(a.acc_g, a.add_g, a.dg, ob + (size_t)c * pk, dgv);
       }
       pre += w[c];
     }
@@ -1070,7 +1080,7 @@ struct BwdSmem {
   static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
 
-template <int DK, int DV>
+template <int DK, int DV, bool FLEX>
 __global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bars[5];
@@ -1094,20 +1104,20 @@ __global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant_
   const int per_seg = a.n_bh * per_head;
   const int seg = blockIdx.x / per_seg, bh = (blockIdx.x % per_seg) / per_head, role = blockIdx.x % per_head;
   if (role < DK / KT)
-    key_tile_body<DK, DV>(sm, mp, a, bh, role, seg, bars, tmem);
+    key_tile_body<DK, DV, FLEX>(sm, mp, a, bh, role, seg, bars, tmem);
   else
-    val_tile_body<DK>(sm, mp, a, bh, role - DK / KT, DV, seg, bars, tmem);
+    val_tile_body<DK, FLEX>(sm, mp, a, bh, role - DK / KT, DV, seg, bars, tmem);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-template <int DK, int DV>
+template <int DK, int DV, bool FLEX>
 static cudaError_t launch_all(const BwdMaps& mp, const BwdArgs& a, int BH, cudaStream_t st) {
   constexpr uint32_t CHK = ChunkLayout<DK, DV>::TOTAL + 1024;
   static_assert(2 * CHK <= 228 * 1024, "two chunk CTAs per SM");
-  auto k1 = bwd_fused_kernel<DK, DV>;
-  auto k3 = bwd_chunk_kernel<DK, DV>;
+  auto k1 = bwd_fused_kernel<DK, DV, FLEX>;
+  auto k3 = bwd_chunk_kernel<DK, DV, FLEX>;
   static std::atomic<bool> attr1[64] = {}, attr3[64] = {};
   {
     cudaError_t e = ensure_smem_attr(k1, BwdSmem<DK, DV>::ALLOC, attr1);
@@ -1217,7 +1227,9 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
                                          DK, DV, a.nseg, a.seg_chunks, st_bh, st_row, st, inv_tau, CK, CV);
     if (e != cudaSuccess) return e;
   }
-  return launch_all<DK, DV>(mp, a, BH, st);
+  // the plain build unless the call needs offsets, partial sums or raw-logit gates
+  if (acc || inv_tau > 0.f) return launch_all<DK, DV, true>(mp, a, BH, st);
+  return launch_all<DK, DV, false>(mp, a, BH, st);
 }
 
 cudaError_t bwd(const void* q, const void* k, const void* v, const void* g, const float* h0, const void* dO,

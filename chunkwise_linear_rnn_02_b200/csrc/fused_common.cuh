@@ -185,16 +185,18 @@ constexpr int kBarCompute = 1;  // named barrier of the threads that run the gat
 // registers the run's alphas and, via the shared buffer `tot` (NSPLIT x ND floats), the products of
 // the other runs: pre = prod of earlier runs, suf = prod of later runs, dec = e^{gamma}.
 //
-// Raw-logit gates: with inv_tau > 0 the tile holds logits x instead of log-gates, and the run first
-// replaces every element of it, in place, by g = bf16(logsigmoid(x) * inv_tau) (0 for the tokens
-// at or past `valid`, which lie beyond the end of the sequence), the values the standalone gate
-// entry would store; everything that reads the tile afterwards sees those log-gates.  The caller
-// runs exactly one gate run per loaded tile, before any other reader of it.
+// Raw-logit gates (LOGIT builds): with inv_tau > 0 the tile holds logits x instead of log-gates, and
+// the run first replaces every element of it, in place, by g = bf16(logsigmoid(x) * inv_tau) (0 for
+// the tokens at or past `valid`, which lie beyond the end of the sequence), the values the
+// standalone gate entry would store; everything that reads the tile afterwards sees those
+// log-gates.  The caller runs exactly one gate run per loaded tile, before any other reader of it.
+// The transform is a loop of its own ahead of the gate loop, so builds without it compile the gate
+// loop unchanged.
 __device__ __forceinline__ float logsigmoid_scaled(float x, float inv_tau) {
   return (fminf(x, 0.f) - log1pf(expf(-fabsf(x)))) * inv_tau;
 }
 
-template <int ND, int NTH>
+template <int ND, int NTH, bool LOGIT = false>
 struct GateRun {
   static constexpr int NPAIR = ND / 2;
   static constexpr int NSPLIT = NTH / NPAIR;
@@ -224,16 +226,21 @@ struct GateRun {
     p = tid % NPAIR;
     h = tid / NPAIR;
     d = 2 * p;
+    if (LOGIT && inv_tau > 0.f) {
+#pragma unroll
+      for (int u = 0; u < TS; ++u) {
+        const int j = h * TS + u;
+        uint32_t* ptr = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(graw) +
+                                                    (swz ? sm100::sw128(j, d) : (j * gstride + d) * 2));
+        const uint32_t w = *ptr;
+        *ptr = j < valid ? pack2(logsigmoid_scaled(bf_lo(w), inv_tau), logsigmoid_scaled(bf_hi(w), inv_tau)) : 0u;
+      }
+    }
     float r0 = 1.f, r1 = 1.f;
 #pragma unroll
     for (int u = 0; u < TS; ++u) {
       const int j = h * TS + u;
-      const uint32_t off = swz ? sm100::sw128(j, d) : (j * gstride + d) * 2;
-      uint32_t w = *reinterpret_cast<const uint32_t*>(graw + off);
-      if (inv_tau > 0.f) {
-        w = j < valid ? pack2(logsigmoid_scaled(bf_lo(w), inv_tau), logsigmoid_scaled(bf_hi(w), inv_tau)) : 0u;
-        *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(graw) + off) = w;
-      }
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(graw + (swz ? sm100::sw128(j, d) : (j * gstride + d) * 2));
       a0[u] = ex2(bf_lo(w) * kLog2e);
       a1[u] = ex2(bf_hi(w) * kLog2e);
       r0 *= a0[u];

@@ -331,8 +331,9 @@ bool gsa_fused_fwd_ok(int BH, int T, int dk, int dv, int m, int chunk, int dtype
   return gla::gsa::pass1_supported(BH, T, dk, m, chunk, dtype) && gla::fast::fwd_supported(BH, T, m, dv, chunk, dtype);
 }
 bool gsa_fused_bwd_ok(int BH, int T, int dk, int dv, int m, int chunk, int dtype) {
-  return gsa_fused_fwd_ok(BH, T, dk, dv, m, chunk, dtype) && gsa_pass2_fused_ok(BH, T, m, dv, chunk, dtype) &&
-         gla::fast::bwd_supported(BH, T, 128, dk, chunk, dtype) && gla::fast::fwd_supported(BH, T, m, dk, chunk, dtype);
+  return gsa_fused_fwd_ok(BH, T, dk, dv, m, chunk, dtype) && 2 * m == 128 &&
+         gla::fast::bwd_supported(BH, T, 128, dv, chunk, dtype) && gla::fast::bwd_supported(BH, T, 128, dk, chunk, dtype) &&
+         gla::fast::fwd_supported(BH, T, 128, dk, chunk, dtype);
 }
 
 struct GsaFusedFwdWs {
@@ -349,8 +350,9 @@ size_t carve_gsa_fused_fwd(Carve& c, int BH, int T, int dk, int dv, int m, bool 
 }
 
 struct GsaFusedBwdWs {
-  GsaFusedWs f;                   // pass 2: padded operands, fp32 gradients, padded states, bwd workspace
-  bf16 *p, *do1, *do1_pad;        // [rows][m], [rows][m], [rows][128]
+  GsaFusedWs f;                    // pass 2: widened operands, fp32 gradients, widened states, bwd workspace
+  float* p32;                      // [rows][m] the slot softmax in fp32
+  bf16* do1;                       // [rows][128]: do1 [hi | lo]
   float *dq1, *dphi1, *dg1;        // pass-1 backward outputs: [rows][128] x 3
   float *h0p, *dhTp, *dh0p, *h0t;  // [BH][128][dk] x 3, [BH][m][dk]
   void *p1ws, *fws;
@@ -359,9 +361,8 @@ size_t carve_gsa_fused_bwd(Carve& c, int BH, int T, int dk, int dv, int m, GsaFu
   const size_t rows = (size_t)BH * T, sp = (size_t)BH * 128 * dk;
   GsaFusedBwdWs x;
   carve_gsa_fused(c, BH, T, dv, &x.f, gla::fast::bwd_workspace(BH, T, 128, dk));
-  x.p = c.take<bf16>(rows * m);
-  x.do1 = c.take<bf16>(rows * m);
-  x.do1_pad = c.take<bf16>(rows * 128);
+  x.p32 = c.take<float>(rows * m);
+  x.do1 = c.take<bf16>(rows * 128);
   x.dq1 = c.take<float>(rows * 128);
   x.dphi1 = c.take<float>(rows * 128);
   x.dg1 = c.take<float>(rows * 128);
@@ -370,7 +371,7 @@ size_t carve_gsa_fused_bwd(Carve& c, int BH, int T, int dk, int dv, int m, GsaFu
   x.dh0p = c.take<float>(sp);
   x.h0t = c.take<float>((size_t)BH * m * dk);
   x.p1ws = c.take<char>(gla::gsa::pass1_workspace(BH, T, dk));
-  x.fws = c.take<char>(gla::fast::fwd_workspace(BH, T, m, dk));
+  x.fws = c.take<char>(gla::fast::fwd_workspace(BH, T, 128, dk));
   if (w) *w = x;
   return c.used;
 }
@@ -387,6 +388,10 @@ int gsa_fwd_fused(const bf16* q, const bf16* k, const bf16* v, const bf16* phi, 
   return GLA_OK;
 }
 
+// Both GLA passes of the backward run on 128-wide key blocks: the m = 64 slots, then a second copy of
+// them (same keys and gates) whose queries are the low bf16 parts of the real queries, so that p and
+// do1 enter at about 16 mantissa bits (the slot softmax and its Jacobian amplify a bf16 rounding of
+// either several times over).  The two copies' gradients add up.
 int gsa_bwd_fused(const bf16* q, const bf16* k, const bf16* v, const bf16* phi, const bf16* g, const float* h01,
                   const float* h02, const bf16* dO, const float* dhT1, const float* dhT2, bf16* dq, bf16* dk, bf16* dv,
                   bf16* dphi, bf16* dg, float* dh01, float* dh02, int BH, int T, int dkd, int dvd, int m, void* ws,
@@ -396,33 +401,42 @@ int gsa_bwd_fused(const bf16* q, const bf16* k, const bf16* v, const bf16* phi, 
   carve_gsa_fused_bwd(c, BH, T, dkd, dvd, m, &w);
   const GsaFusedWs& f = w.f;
   const long long rows = (long long)BH * T, sz = (long long)m * dvd, sp = 128LL * dvd, s1 = (long long)dkd * m;
-  // pass 1 forward again: the slot softmax p
-  GLA_CUDA(gla::gsa::pass1_fwd(q, k, phi, g, h01, w.p, nullptr, BH, T, dkd, w.p1ws, st));
-  // pass 2 backward (queries p, keys phi, values v), slots zero-padded to 128 keys
-  GLA_CUDA(gla::split::copy_cols(w.p, m, f.p, 128, rows, m, 128, st));
-  GLA_CUDA(gla::split::copy_cols(phi, m, f.phi, 128, rows, m, 128, st));
-  GLA_CUDA(gla::split::copy_cols(g, m, f.g, 128, rows, m, 128, st));
-  if (h02) GLA_CUDA(gla::split::copy_cols(h02, sz, f.h0, sp, BH, sz, sp, st));
+  const long long s1t = (long long)m * dkd, s1p = 128LL * dkd;
+  // pass 1 forward again: the slot softmax p, in fp32
+  GLA_CUDA(gla::gsa::pass1_fwd(q, k, phi, g, h01, nullptr, nullptr, BH, T, dkd, w.p1ws, st, w.p32));
+  // key blocks of 128: queries [p hi | p lo], keys [phi | phi], gates [g | g]
+  GLA_CUDA(gla::gsa::widen(w.p32, f.p, rows, m, true, st));
+  GLA_CUDA(gla::gsa::widen(phi, f.phi, rows, m, false, st));
+  GLA_CUDA(gla::gsa::widen(g, f.g, rows, m, false, st));
+  // pass 2 backward (queries p, keys phi, values v): both copies start from h0_2, the first alone
+  // carries dhT2
+  if (h02) {
+    GLA_CUDA(gla::split::copy_cols(h02, sz, f.h0, sp, BH, sz, sz, st));
+    GLA_CUDA(gla::split::copy_cols(h02, sz, f.h0 + sz, sp, BH, sz, sz, st));
+  }
   if (dhT2) GLA_CUDA(gla::split::copy_cols(dhT2, sz, f.dhT, sp, BH, sz, sp, st));
   const gla::fast::BwdAccum acc2{f.dq, f.dk, f.dg, nullptr, 128, 0, dvd, 0};  // dv straight to bf16
   GLA_CUDA(gla::fast::bwd(f.p, f.phi, v, f.g, h02 ? f.h0 : nullptr, dO, dhT2 ? f.dhT : nullptr, nullptr, nullptr, dv,
                           nullptr, dh02 ? f.dh0 : nullptr, BH, T, 128, dvd, f.ws, st, -1, -1, &acc2));
-  if (dh02) GLA_CUDA(gla::split::copy_cols(f.dh0, sp, dh02, sz, BH, sz, sz, st));
-  // slot softmax Jacobian: do1 = p (dp - <p, dp>)
-  GLA_CUDA(gla::gsa::softmax_jacobian(w.p, f.dq, 128, w.do1, w.do1_pad, rows, m, 128, st));
+  if (dh02) GLA_CUDA(gla::gsa::fold_rows(f.dh0, dh02, BH, m, dvd, st));
+  // slot softmax Jacobian: do1 = p (dp - <p, dp>), dp = the first copy's query gradient
+  GLA_CUDA(gla::gsa::softmax_jacobian(w.p32, f.dq, 128, w.do1, rows, m, st));
   // pass 1 backward as a GLA backward: queries do1, keys phi, values k, dO' = q, states transposed
-  if (h01) GLA_CUDA(gla::gsa::transpose_states(h01, s1, w.h0p, BH, dkd, m, 128, st));
+  if (h01) {
+    GLA_CUDA(gla::gsa::transpose_states(h01, s1, w.h0t, BH, dkd, m, m, st));
+    GLA_CUDA(gla::split::copy_cols(w.h0t, s1t, w.h0p, s1p, BH, s1t, s1t, st));
+    GLA_CUDA(gla::split::copy_cols(w.h0t, s1t, w.h0p + s1t, s1p, BH, s1t, s1t, st));
+  }
   if (dhT1) GLA_CUDA(gla::gsa::transpose_states(dhT1, s1, w.dhTp, BH, dkd, m, 128, st));
   const gla::fast::BwdAccum acc1{w.dq1, w.dphi1, w.dg1, nullptr, 128, 0, dkd, 0};  // dk (its dv) straight to bf16
-  GLA_CUDA(gla::fast::bwd(w.do1_pad, f.phi, k, f.g, h01 ? w.h0p : nullptr, q, dhT1 ? w.dhTp : nullptr, nullptr,
-                          nullptr, dk, nullptr, dh01 ? w.dh0p : nullptr, BH, T, 128, dkd, f.ws, st, -1, -1, &acc1));
+  GLA_CUDA(gla::fast::bwd(w.do1, f.phi, k, f.g, h01 ? w.h0p : nullptr, q, dhT1 ? w.dhTp : nullptr, nullptr, nullptr,
+                          dk, nullptr, dh01 ? w.dh0p : nullptr, BH, T, 128, dkd, f.ws, st, -1, -1, &acc1));
   // dq = S1 do1: the output of the GLA with queries do1, keys phi, values k from h0_1^T
-  if (h01) GLA_CUDA(gla::gsa::transpose_states(h01, s1, w.h0t, BH, dkd, m, m, st));
-  GLA_CUDA(gla::fast::fwd(w.do1, phi, k, g, h01 ? w.h0t : nullptr, dq, nullptr, BH, T, m, dkd, w.fws, st));
-  // both passes' contributions to dphi and dg; dk and dh0_1 back to the caller's layouts
-  GLA_CUDA(gla::gsa::add_cols_bf16(w.dphi1, f.dk, 128, dphi, rows, m, st));
-  GLA_CUDA(gla::gsa::add_cols_bf16(w.dg1, f.dg, 128, dg, rows, m, st));
-  if (dh01) GLA_CUDA(gla::gsa::transpose_states(w.dh0p, 128LL * dkd, dh01, BH, m, dkd, dkd, st));
+  GLA_CUDA(gla::fast::fwd(w.do1, f.phi, k, f.g, h01 ? w.h0p : nullptr, dq, nullptr, BH, T, 128, dkd, w.fws, st));
+  // both passes' and both copies' contributions to dphi and dg; dh0_1 back to [dk][m]
+  GLA_CUDA(gla::gsa::fold_add_bf16(w.dphi1, f.dk, dphi, rows, m, st));
+  GLA_CUDA(gla::gsa::fold_add_bf16(w.dg1, f.dg, dg, rows, m, st));
+  if (dh01) GLA_CUDA(gla::gsa::transpose_states(w.dh0p, s1p, dh01, BH, m, dkd, dkd, st, true));
   return GLA_OK;
 }
 

@@ -15,9 +15,9 @@
 //     S1_{i+1} = S1_i diag(dec) + K^T (Phi o E2)                   state on chip (fp32 registers)
 //
 // The gate enters only through column scalings, so q and k feed tcgen05.mma as TMA loads them
-// (raw bf16 tiles with the 128-byte swizzle) and A = Q K^T is exact in fp32.  The state copy and
-// the masked A are bf16 hi + lo pairs; Phi o E2 is one bf16 operand (the role the decayed keys play
-// in the GLA forward).  The epilogue scales X, takes the softmax over the 64 slots of each token
+// (raw bf16 tiles with the 128-byte swizzle) and A = Q K^T is exact in fp32.  The state copy, the
+// masked A and Phi o E2 are bf16 hi + lo pairs: the slot softmax turns absolute errors of o1 into
+// relative errors of p, and a single bf16 Phi o E2 alone put the output several percent off.  The epilogue scales X, takes the softmax over the 64 slots of each token
 // (the two threads that hold a token's halves exchange the row max and sum in shared memory) and
 // stores p in bf16; o1 never reaches HBM.
 //
@@ -66,8 +66,8 @@ struct Pass1Layout {
   static constexpr uint32_t ST = C * M * 2;                // a phi or g tile [64 x 64], swizzled
   static constexpr uint32_t Q_OFF = 0, K_OFF = QT, PHI_OFF = 2 * QT, G_OFF = 2 * QT + ST;
   static constexpr uint32_t STAGE = 2 * QT + 2 * ST;       // two stages
-  static constexpr uint32_t PH0 = 2 * STAGE;               // Phi o E2 [64 x 64], one per chunk parity
-  static constexpr uint32_t SB_HI = PH0 + 2 * ST;          // state copy hi / lo [DK x 64], MN-major B
+  static constexpr uint32_t PH0 = 2 * STAGE;               // Phi o E2 hi / lo [64 x 64], per chunk parity
+  static constexpr uint32_t SB_HI = PH0 + 4 * ST;          // state copy hi / lo [DK x 64], MN-major B
   static constexpr uint32_t SB_LO = SB_HI + DK * M * 2;
   static constexpr uint32_t AB_HI = SB_LO + DK * M * 2;    // masked A hi / lo [64 x 64], K-major A
   static constexpr uint32_t AB_LO = AB_HI + C * C * 2;
@@ -92,7 +92,8 @@ struct Pass1Layout {
 struct Pass1Args {
   const float* h0;        // [BH][DK][64] or null (zeros)
   const float* sin;       // [BH][nseg][64][DK]: transposed state entering segment s at entry s-1
-  __nv_bfloat16* p;       // [BH][T][64]
+  __nv_bfloat16* p;       // [BH][T][64], or
+  float* p32;             // [BH][T][64] in fp32 (when set, in place of p)
   float* hT;              // [BH][DK][64] or null
   int T, seg_chunks, nseg;
   unsigned int* latch;
@@ -175,7 +176,7 @@ __global__ void __launch_bounds__(NTH, 1)
         mbar_wait(&bar_ld[li & 1], (li >> 1) & 1, latch);
         tc_fence_after();
         const uint32_t st = base + (li & 1) * L::STAGE;
-        const uint32_t ph = base + L::PH0 + (li & 1) * L::ST;
+        const uint32_t ph = base + L::PH0 + (li & 1) * 2 * L::ST;  // hi, then lo at + ST
         const uint32_t t_X = t_X0 + (li & 1) * 64;
 #pragma unroll
         for (int k = 0; k < DK / 16; ++k) {
@@ -186,22 +187,26 @@ __global__ void __launch_bounds__(NTH, 1)
           umma_bf16(t_X, qd, desc_sw128(base + L::SB_LO + k * 2048, 16, 1024), id_X, 1);
         }
 #pragma unroll
-        for (int k = 0; k < C / 16; ++k)
-          umma_bf16(t_dS, desc_sw128(st + L::K_OFF + k * 2048, C * 128, 1024), desc_sw128(ph + k * 2048, 16, 1024),
-                    id_S, k > 0);
+        for (int k = 0; k < C / 16; ++k) {
+          const uint64_t kd = desc_sw128(st + L::K_OFF + k * 2048, C * 128, 1024);
+          umma_bf16(t_dS, kd, desc_sw128(ph + k * 2048, 16, 1024), id_S, k > 0);
+          umma_bf16(t_dS, kd, desc_sw128(ph + L::ST + k * 2048, 16, 1024), id_S, 1);
+        }
         umma_commit(&bar_mma1);
       }
       bar_sync(kBarAB, NHAND);  // chunk li's masked A is in shared memory; its stage is free
       if (lane == 0) {
         // group 2: X += mask(A) (Phi o E2)
         tc_fence_after();
-        const uint32_t ph = base + L::PH0 + (li & 1) * L::ST;
+        const uint32_t ph = base + L::PH0 + (li & 1) * 2 * L::ST;
         const uint32_t t_X = t_X0 + (li & 1) * 64;
 #pragma unroll
         for (int k = 0; k < C / 16; ++k) {
-          const uint64_t vd = desc_sw128(ph + k * 2048, 16, 1024);
-          umma_bf16(t_X, desc_sw128(base + L::AB_HI + k * 32, 16, 1024), vd, id_X, 1);
-          umma_bf16(t_X, desc_sw128(base + L::AB_LO + k * 32, 16, 1024), vd, id_X, 1);
+          const uint64_t vh = desc_sw128(ph + k * 2048, 16, 1024), vl = desc_sw128(ph + L::ST + k * 2048, 16, 1024);
+          const uint64_t ah = desc_sw128(base + L::AB_HI + k * 32, 16, 1024);
+          umma_bf16(t_X, ah, vh, id_X, 1);
+          umma_bf16(t_X, desc_sw128(base + L::AB_LO + k * 32, 16, 1024), vh, id_X, 1);
+          umma_bf16(t_X, ah, vl, id_X, 1);
         }
         umma_commit(&bar_mma2);
         // the stage of chunk li is read by nothing after its first group and the A epilogue
@@ -239,7 +244,7 @@ __global__ void __launch_bounds__(NTH, 1)
 
     // Gate math of local chunk li (stage li & 1): decays, Phi o E2 into registers, and the scale
     // table e^{B_j - gamma} (e^{B_j} on the exact path).  Returns the chunk's exact-path flag.
-    uint32_t phr[TS];
+    uint32_t phr[TS], phl[TS];
     int gd = 0, gh = 0;
     auto gate_regs = [&](int li) {
       const uint8_t* st = sm + (li & 1) * L::STAGE;
@@ -257,7 +262,7 @@ __global__ void __launch_bounds__(NTH, 1)
       gr.load_pairs(st + L::PHI_OFF, M, true, w);
       gr.backward([&](int j, float e0, float e1) {
         const uint32_t x = w[j - gh * TS];
-        phr[j - gh * TS] = pack2(bf_lo(x) * e0, bf_hi(x) * e1);
+        fast::split2(bf_lo(x) * e0, bf_hi(x) * e1, phr[j - gh * TS], phl[j - gh * TS]);
       });
       // written after the gate run's barrier: every compute thread has finished reading the table
       // of chunk li - 2 (same parity) by then
@@ -271,9 +276,12 @@ __global__ void __launch_bounds__(NTH, 1)
     };
     // Operands of local chunk li into shared memory, then hand them to the producer.
     auto store_ops = [&](int li, int safe) {
-      uint8_t* phb = sm + L::PH0 + (li & 1) * L::ST;
+      uint8_t* phb = sm + L::PH0 + (li & 1) * 2 * L::ST;
 #pragma unroll
-      for (int u = 0; u < TS; ++u) *reinterpret_cast<uint32_t*>(phb + sw128(gh * TS + u, gd)) = phr[u];
+      for (int u = 0; u < TS; ++u) {
+        *reinterpret_cast<uint32_t*>(phb + sw128(gh * TS + u, gd)) = phr[u];
+        *reinterpret_cast<uint32_t*>(phb + L::ST + sw128(gh * TS + u, gd)) = phl[u];
+      }
       const float* dec = decay_sm + (li & 1) * M;
       float sv[SW];
 #pragma unroll
@@ -379,7 +387,13 @@ __global__ void __launch_bounds__(NTH, 1)
         const float inv = 1.f / (ssum[j] + ssum[C + j]);
 #pragma unroll
         for (int c = 0; c < 32; ++c) x[c] *= inv;
-        fast::store_half_global_bf16(args.p + ((size_t)bh * T + t) * M + cb, x);
+        if (args.p32) {
+          float4* dst = reinterpret_cast<float4*>(args.p32 + ((size_t)bh * T + t) * M + cb);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+        } else {
+          fast::store_half_global_bf16(args.p + ((size_t)bh * T + t) * M + cb, x);
+        }
       }
     };
 
@@ -443,57 +457,105 @@ __global__ void __launch_bounds__(NTH, 1)
 }
 
 // ------------------------------------------------------------------------------------------
-// Elementwise glue
+// Elementwise glue.  The backward runs both GLA passes on 128-wide key blocks whose first 64 keys
+// are the slots; the other 64 carry a second copy of the slots (same keys phi, same gates) whose
+// queries are the low bf16 parts of the real queries: with queries [hi | lo] the pass computes
+// exactly what queries hi + lo give (the output is linear in the queries), so p and do1 enter with
+// about 16 mantissa bits instead of 8.  The gradients of the two copies add up.
 // ------------------------------------------------------------------------------------------
-// One warp per token: do1 = p (dp - <p, dp>) over the m <= 64 slots (each lane takes two).
-__global__ void jacobian_kernel(const __nv_bfloat16* __restrict__ p, const float* __restrict__ dp, int dp_pitch,
-                                __nv_bfloat16* __restrict__ do1, __nv_bfloat16* __restrict__ do1_pad, long long rows,
-                                int m, int pad) {
+// One warp per token: do1 = p (dp - <p, dp>) over the m <= 64 slots (each lane takes two), from
+// p in fp32 and dp (fp32, row pitch dp_pitch); do1 goes out as bf16 [hi | lo] rows of 2m.
+__global__ void jacobian_kernel(const float* __restrict__ p, const float* __restrict__ dp, int dp_pitch,
+                                __nv_bfloat16* __restrict__ do1, long long rows, int m) {
   const int lane = threadIdx.x & 31;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
   for (long long r = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
     const int c = 2 * lane;
     float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
     if (c < m) {
-      const __nv_bfloat162 pp = *reinterpret_cast<const __nv_bfloat162*>(p + r * m + c);
+      const float2 pp = *reinterpret_cast<const float2*>(p + r * m + c);
       const float2 dd = *reinterpret_cast<const float2*>(dp + r * dp_pitch + c);
-      p0 = __low2float(pp);
-      p1 = __high2float(pp);
+      p0 = pp.x;
+      p1 = pp.y;
       d0 = dd.x;
       d1 = dd.y;
     }
     float dot = p0 * d0 + p1 * d1;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    const __nv_bfloat162 out = __floats2bfloat162_rn(p0 * (d0 - dot), p1 * (d1 - dot));
-    if (c < m) *reinterpret_cast<__nv_bfloat162*>(do1 + r * m + c) = out;
-    for (int cc = c; cc < pad; cc += 64)
-      *reinterpret_cast<__nv_bfloat162*>(do1_pad + r * pad + cc) = cc < m ? out : __floats2bfloat162_rn(0.f, 0.f);
+    if (c < m) {
+      const float x0 = p0 * (d0 - dot), x1 = p1 * (d1 - dot);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(x0, x1);
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(x0 - __low2float(hi), x1 - __high2float(hi));
+      *reinterpret_cast<__nv_bfloat162*>(do1 + r * 2 * m + c) = hi;
+      *reinterpret_cast<__nv_bfloat162*>(do1 + r * 2 * m + m + c) = lo;
+    }
   }
 }
 
-// dst [nb][Cp][R]: dst[b][c][r] = src[b * sb + r * Cc + c] for c < Cc, zeros for Cc <= c < Cp.
-__global__ void transpose_kernel(const float* __restrict__ src, long long sb, float* __restrict__ dst, int nb, int R,
-                                 int Cc, int Cp) {
-  const long long n = (long long)nb * Cp * R;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
-    const int r = (int)(e % R);
-    const int c = (int)((e / R) % Cp);
-    const long long b = e / ((long long)R * Cp);
-    dst[e] = c < Cc ? src[b * sb + (long long)r * Cc + c] : 0.f;
-  }
-}
-
-__global__ void add_cols_kernel(const float* __restrict__ a, const float* __restrict__ b, int pitch,
-                                __nv_bfloat16* __restrict__ out, long long rows, int m) {
+// Rows of 2m bf16: [hi | lo] of fp32 rows of m (mode 0), or [x | x] of bf16 rows of m (mode 1).
+__global__ void widen_kernel(const void* __restrict__ src, __nv_bfloat16* __restrict__ dst, long long rows, int m,
+                             int mode) {
   const int vpr = m / 2;
   const long long n = rows * vpr;
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
     const long long r = e / vpr;
     const int c = (int)(e % vpr) * 2;
-    const float2 x = *reinterpret_cast<const float2*>(a + r * pitch + c);
-    const float2 y = *reinterpret_cast<const float2*>(b + r * pitch + c);
-    *reinterpret_cast<__nv_bfloat162*>(out + r * m + c) = __floats2bfloat162_rn(x.x + y.x, x.y + y.y);
+    __nv_bfloat162 a, b;
+    if (mode == 0) {
+      const float2 x = *reinterpret_cast<const float2*>(static_cast<const float*>(src) + r * m + c);
+      a = __floats2bfloat162_rn(x.x, x.y);
+      b = __floats2bfloat162_rn(x.x - __low2float(a), x.y - __high2float(a));
+    } else {
+      a = b = *reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(src) + r * m + c);
+    }
+    *reinterpret_cast<__nv_bfloat162*>(dst + r * 2 * m + c) = a;
+    *reinterpret_cast<__nv_bfloat162*>(dst + r * 2 * m + m + c) = b;
+  }
+}
+
+// dst [nb][Cp][R]: dst[b][c][r] = src[b * sb + r * Cc + c] (+ src[b * sb + (r + R) * Cc + c] when
+// fold, the second copy's row) for c < Cc, zeros for Cc <= c < Cp.
+__global__ void transpose_kernel(const float* __restrict__ src, long long sb, float* __restrict__ dst, int nb, int R,
+                                 int Cc, int Cp, int fold) {
+  const long long n = (long long)nb * Cp * R;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(e % R);
+    const int c = (int)((e / R) % Cp);
+    const long long b = e / ((long long)R * Cp);
+    float x = 0.f;
+    if (c < Cc) {
+      x = src[b * sb + (long long)r * Cc + c];
+      if (fold) x += src[b * sb + (long long)(r + R) * Cc + c];
+    }
+    dst[e] = x;
+  }
+}
+
+// dst[b][r][c] = src[b][r][c] + src[b][r + R][c]: the two copies' state gradients, [nb][2R][Cc] -> [nb][R][Cc].
+__global__ void fold_rows_kernel(const float* __restrict__ src, float* __restrict__ dst, int nb, int R, int Cc) {
+  const long long per = (long long)R * Cc, n = (long long)nb * per;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const long long b = e / per, i = e % per;
+    dst[e] = src[b * 2 * per + i] + src[b * 2 * per + per + i];
+  }
+}
+
+// out[r][c] = bf16(a[r][c] + a[r][m + c] + b[r][c] + b[r][m + c]) for c < m: both passes, both copies
+// (a, b fp32 with rows of 2m).
+__global__ void fold_add_kernel(const float* __restrict__ a, const float* __restrict__ b, __nv_bfloat16* __restrict__ out,
+                                long long rows, int m) {
+  const int vpr = m / 2;
+  const long long n = rows * vpr;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const long long r = e / vpr;
+    const int c = (int)(e % vpr) * 2;
+    const float* ar = a + r * 2 * m;
+    const float* br = b + r * 2 * m;
+    const float2 a0 = *reinterpret_cast<const float2*>(ar + c), a1 = *reinterpret_cast<const float2*>(ar + m + c);
+    const float2 b0 = *reinterpret_cast<const float2*>(br + c), b1 = *reinterpret_cast<const float2*>(br + m + c);
+    *reinterpret_cast<__nv_bfloat162*>(out + r * m + c) =
+        __floats2bfloat162_rn(a0.x + a1.x + b0.x + b1.x, a0.y + a1.y + b0.y + b1.y);
   }
 }
 
@@ -533,7 +595,7 @@ size_t pass1_workspace(int BH, int T, int dk) {
 }
 
 cudaError_t pass1_fwd(const void* q, const void* k, const void* phi, const void* g, const float* h0, void* p,
-                      float* hT, int BH, int T, int dk, void* ws, cudaStream_t st) {
+                      float* hT, int BH, int T, int dk, void* ws, cudaStream_t st, float* p32) {
   if (dk != 128) return cudaErrorNotSupported;
   constexpr int DK = 128;
   using L = Pass1Layout<DK>;
@@ -545,6 +607,7 @@ cudaError_t pass1_fwd(const void* q, const void* k, const void* phi, const void*
   a.h0 = h0;
   a.sin = nullptr;
   a.p = static_cast<__nv_bfloat16*>(p);
+  a.p32 = p32;
   a.hT = hT;
   a.T = T;
   a.latch = device_error_latch();
@@ -556,7 +619,7 @@ cudaError_t pass1_fwd(const void* q, const void* k, const void* phi, const void*
     float* h0t = gam + align256((size_t)BH * a.nseg * M * 4) / 4;
     if (h0) {
       transpose_kernel<<<grid_for((long long)BH * M * DK, 256), 256, 0, st>>>(h0, (long long)DK * M, h0t, BH, DK,
-                                                                            M, M);
+                                                                            M, M, 0);
       const cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
@@ -576,26 +639,35 @@ cudaError_t pass1_fwd(const void* q, const void* k, const void* phi, const void*
   return cudaGetLastError();
 }
 
-cudaError_t softmax_jacobian(const void* p, const float* dp, int dp_pitch, void* do1, void* do1_pad, long long rows,
-                             int m, int pad, cudaStream_t st) {
-  if (m > 64 || m % 2 != 0 || pad % 2 != 0 || pad < m) return cudaErrorNotSupported;
-  jacobian_kernel<<<grid_for(rows, 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(p), dp, dp_pitch,
-                                                     static_cast<__nv_bfloat16*>(do1),
-                                                     static_cast<__nv_bfloat16*>(do1_pad), rows, m, pad);
+cudaError_t softmax_jacobian(const float* p, const float* dp, int dp_pitch, void* do1, long long rows, int m,
+                             cudaStream_t st) {
+  if (m > 64 || m % 2 != 0) return cudaErrorNotSupported;
+  jacobian_kernel<<<grid_for(rows, 8), 256, 0, st>>>(p, dp, dp_pitch, static_cast<__nv_bfloat16*>(do1), rows, m);
+  return cudaGetLastError();
+}
+
+cudaError_t widen(const void* src, void* dst, long long rows, int m, bool hilo, cudaStream_t st) {
+  if (m % 2 != 0) return cudaErrorNotSupported;
+  widen_kernel<<<grid_for(rows * (m / 2), 256), 256, 0, st>>>(src, static_cast<__nv_bfloat16*>(dst), rows, m,
+                                                               hilo ? 0 : 1);
   return cudaGetLastError();
 }
 
 cudaError_t transpose_states(const float* src, long long src_bstride, float* dst, int nb, int R, int Cc, int Cp,
-                             cudaStream_t st) {
-  transpose_kernel<<<grid_for((long long)nb * Cp * R, 256), 256, 0, st>>>(src, src_bstride, dst, nb, R, Cc, Cp);
+                             cudaStream_t st, bool fold) {
+  transpose_kernel<<<grid_for((long long)nb * Cp * R, 256), 256, 0, st>>>(src, src_bstride, dst, nb, R, Cc, Cp,
+                                                                          fold ? 1 : 0);
   return cudaGetLastError();
 }
 
-cudaError_t add_cols_bf16(const float* a, const float* b, int pitch, void* out, long long rows, int m,
-                          cudaStream_t st) {
+cudaError_t fold_rows(const float* src, float* dst, int nb, int R, int Cc, cudaStream_t st) {
+  fold_rows_kernel<<<grid_for((long long)nb * R * Cc, 256), 256, 0, st>>>(src, dst, nb, R, Cc);
+  return cudaGetLastError();
+}
+
+cudaError_t fold_add_bf16(const float* a, const float* b, void* out, long long rows, int m, cudaStream_t st) {
   if (m % 2 != 0) return cudaErrorNotSupported;
-  add_cols_kernel<<<grid_for(rows * (m / 2), 256), 256, 0, st>>>(a, b, pitch, static_cast<__nv_bfloat16*>(out),
-                                                                 rows, m);
+  fold_add_kernel<<<grid_for(rows * (m / 2), 256), 256, 0, st>>>(a, b, static_cast<__nv_bfloat16*>(out), rows, m);
   return cudaGetLastError();
 }
 
