@@ -158,7 +158,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   using Gate = GateRun<KT, BT, FLEX>;
   constexpr int NS = L::NS, TS = Gate::TS;
   // column offsets into wider tensors and the key-side row pitch (FLEX builds only)
-  const int ck = FLEX ? a.ck : 0, cv = FLEX ? a.cv : 0, pk = FLEX ? a.pk : DK;
+  const int col_k = FLEX ? a.ck : 0, col_v = FLEX ? a.cv : 0, pitch_k = FLEX ? a.pk : DK;
   static_assert(TS == 8 && NS == 8, "epilogue runs: four gate runs of eight tokens per token half");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
@@ -186,16 +186,16 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   auto load_a = [&](int chunk) {
     mbar_arrive_expect_tx(bar_pa, 2 * L::VB);
     for (int bb = 0; bb < DV / 64; ++bb) {
-      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, bar_pa, cv + bb * 64, chunk * C, bh);
-      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, bar_pa, cv + bb * 64, chunk * C, bh);
+      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, bar_pa, col_v + bb * 64, chunk * C, bh);
+      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, bar_pa, col_v + bb * 64, chunk * C, bh);
     }
   };
   auto load_b = [&](int chunk, int b) {
     uint8_t* pb = sm + pbo(b);
     mbar_arrive_expect_tx(bar_pb + b, L::PB_STAGE);
-    tma_load_3d(pb + L::PB_K, &mp.k64, bar_pb + b, ck + d0, chunk * C, bh);
-    tma_load_3d(pb + L::PB_G, &mp.g64, bar_pb + b, ck + d0, chunk * C, bh);
-    tma_load_3d(pb + L::PB_Q, &mp.q64, bar_pb + b, ck + d0, chunk * C, bh);
+    tma_load_3d(pb + L::PB_K, &mp.k64, bar_pb + b, col_k + d0, chunk * C, bh);
+    tma_load_3d(pb + L::PB_G, &mp.g64, bar_pb + b, col_k + d0, chunk * C, bh);
+    tma_load_3d(pb + L::PB_Q, &mp.q64, bar_pb + b, col_k + d0, chunk * C, bh);
   };
   auto wait_b = [&](int b) {
     mbar_wait(bar_pb + b, (ph_pb >> b) & 1u, a.latch);
@@ -385,7 +385,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         }
       }
       const float inv = 1.f / DEC[b * KT + d];
-      const size_t ob = ((size_t)bh * T + i * C + tb) * pk + ck + d0 + d;  // output index, token tb
+      const size_t ob = ((size_t)bh * T + i * C + tb) * pitch_k + col_k + d0 + d;  // output index, token tb
 #pragma unroll
       for (int rr = 0; rr < 4; ++rr) {
         float e = 1.f;  // E1 = e^{B_j}, formed as GateRun::forward forms it
@@ -397,7 +397,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
           if (!safe) y[c] *= e * inv;
           const float qv = raw(pq, j, d), kv = raw(pk, j, d);
           if (i * C + j < T) {
-            store_out<FLEX>(a.acc_q, a.add_q, a.dq, ob + (size_t)c * pk, e * x[c] + y[c]);
+            store_out<FLEX>(a.acc_q, a.add_q, a.dq, ob + (size_t)c * pitch_k, e * x[c] + y[c]);
           }
           x[c] = bf_split_sum(qv * e) * x[c];  // Qt X, with Qt as the G update sees it
           y[c] = qv * (y[c] - DIAG[j] * kv);   // q dq^intra without j = r
@@ -494,7 +494,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   using L = ValLayout<DK>;
   using Gate = GateRun<DK, BT, FLEX>;
   // column offsets into wider tensors and the value-side row pitch (FLEX builds only)
-  const int ck = FLEX ? a.ck : 0, cv = FLEX ? a.cv : 0, pv = FLEX ? a.pv : DV;
+  const int col_k = FLEX ? a.ck : 0, col_v = FLEX ? a.cv : 0, pitch_v = FLEX ? a.pv : DV;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = a.T, NC = (T + C - 1) / C, c0 = vt * VT;
   const int ch0 = seg * a.seg_chunks, ch1 = min(NC, ch0 + a.seg_chunks), nl = ch1 - ch0;  // segment
@@ -517,15 +517,15 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   // issued as soon as those reads are done; dO and v once the second MMA group has completed.
   auto load_qkg = [&](int chunk) {
     mbar_arrive_expect_tx(bar_ld, 3 * L::RAW);
-    tma_load_3d(sm, &mp.q_all, bar_ld, ck, chunk * C, bh);
-    tma_load_3d(sm + L::RAW, &mp.k_all, bar_ld, ck, chunk * C, bh);
-    tma_load_3d(sm + 2 * L::RAW, &mp.g_all, bar_ld, ck, chunk * C, bh);
+    tma_load_3d(sm, &mp.q_all, bar_ld, col_k, chunk * C, bh);
+    tma_load_3d(sm + L::RAW, &mp.k_all, bar_ld, col_k, chunk * C, bh);
+    tma_load_3d(sm + 2 * L::RAW, &mp.g_all, bar_ld, col_k, chunk * C, bh);
   };
   auto load_dov = [&](int chunk) {
     mbar_arrive_expect_tx(bar_dv, L::DOT + C * VT * 2);
     for (int b = 0; b < VT / 64; ++b) {
-      tma_load_3d(sm + 3 * L::RAW + b * (C * 128), &mp.dO, bar_dv, cv + c0 + b * 64, chunk * C, bh);
-      tma_load_3d(sm + L::VZ + b * (C * 128), &mp.v, bar_dv, cv + c0 + b * 64, chunk * C, bh);
+      tma_load_3d(sm + 3 * L::RAW + b * (C * 128), &mp.dO, bar_dv, col_v + c0 + b * 64, chunk * C, bh);
+      tma_load_3d(sm + L::VZ + b * (C * 128), &mp.v, bar_dv, col_v + c0 + b * 64, chunk * C, bh);
     }
   };
   auto sync_tc = [&]() {
@@ -745,10 +745,10 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       const int vcol = q4 * 32 + lane, t0 = i * C + half * 32;
       tmem_ld32(tmem + L::T_DV + lane_off + half * 32, v);
       tmem_ld_wait();
-      const size_t ob = ((size_t)bh * T + t0) * pv + cv + c0 + vcol;  // output index, token t0
+      const size_t ob = ((size_t)bh * T + t0) * pitch_v + col_v + c0 + vcol;  // output index, token t0
 #pragma unroll
       for (int c = 0; c < 32; ++c)
-        if (t0 + c < T) store_out<FLEX>(a.acc_v, a.add_v, a.dv, ob + (size_t)c * pv, v[c]);
+        if (t0 + c < T) store_out<FLEX>(a.acc_v, a.add_v, a.dv, ob + (size_t)c * pitch_v, v[c]);
     }
     tc_fence_before();
     __syncthreads();
@@ -840,7 +840,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   using L = ChunkLayout<DK, DV>;
   using Gate = GateRun<KT, BT, FLEX>;
   // column offsets into wider tensors and the key-side row pitch (FLEX builds only)
-  const int ck = FLEX ? a.ck : 0, cv = FLEX ? a.cv : 0, pk = FLEX ? a.pk : DK;
+  const int col_k = FLEX ? a.ck : 0, col_v = FLEX ? a.cv : 0, pitch_k = FLEX ? a.pk : DK;
   constexpr int NS = L::NS, TS = Gate::TS, NVT = DV / VT;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_ld, bar_m1, bar_m2;
@@ -878,12 +878,12 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   if (tid == 0) {
     mbar_arrive_expect_tx(&bar_ld, 2 * L::VB + 3 * L::TILE);
     for (int bb = 0; bb < DV / 64; ++bb) {
-      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, &bar_ld, cv + bb * 64, i * C, bh);
-      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, &bar_ld, cv + bb * 64, i * C, bh);
+      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, &bar_ld, col_v + bb * 64, i * C, bh);
+      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, &bar_ld, col_v + bb * 64, i * C, bh);
     }
-    tma_load_3d(sm + L::PB_K, &mp.k64, &bar_ld, ck + d0, i * C, bh);
-    tma_load_3d(sm + L::PB_G, &mp.g64, &bar_ld, ck + d0, i * C, bh);
-    tma_load_3d(sm + L::PB_Q, &mp.q64, &bar_ld, ck + d0, i * C, bh);
+    tma_load_3d(sm + L::PB_K, &mp.k64, &bar_ld, col_k + d0, i * C, bh);
+    tma_load_3d(sm + L::PB_G, &mp.g64, &bar_ld, col_k + d0, i * C, bh);
+    tma_load_3d(sm + L::PB_Q, &mp.q64, &bar_ld, col_k + d0, i * C, bh);
   }
   // The epilogue runs on all 32 lanes: lane l < 16 owns key dim row = q4 * 16 + l for tokens
   // tb .. tb + 15, lane l + 16 the same dim for tokens tb + 16 .. tb + 31 (the M = 64 accumulators
@@ -1017,7 +1017,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   float tot_s = 0.f;
   {  // dk; per-token terms Kh Z + k dk^intra without j = r (-> w)
     const float inv = 1.f / DEC[d];
-    const size_t ob = ((size_t)bh * T + i * C + tq) * pk + ck + d0 + d;  // output index, token tq
+    const size_t ob = ((size_t)bh * T + i * C + tq) * pitch_k + col_k + d0 + d;  // output index, token tq
 #pragma unroll
     for (int rr = 0; rr < 16 / TS; ++rr) {
       const int h = tq / TS + rr;
@@ -1038,7 +1038,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
         if (!safe) w[c] *= ev * inv;
         const float qv = raw(L::PB_Q, r, d), kv = raw(L::PB_K, r, d);
         if (i * C + r < T) {
-          store_out<FLEX>(a.acc_k, a.add_k, a.dk, ob + (size_t)c * pk, ev * z[c] + w[c]);
+          store_out<FLEX>(a.acc_k, a.add_k, a.dk, ob + (size_t)c * pitch_k, ev * z[c] + w[c]);
         }
         const float kz = bf_split_sum(kv * ev) * z[c];  // Kh Z, with Kh as the S update sees it
         w[c] = kz + kv * (w[c] - DIAG[r] * qv);        // plus k dk^intra without j = r
@@ -1052,7 +1052,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   {  // dg = c_i + prefix (exclusive) of (Kh Z + k dk^intra) + the forward walk's part
     float pre = 0.f;
     for (int t = 0; t < qi; ++t) pre += XQ[t * KT + d];
-    const size_t ob = ((size_t)bh * T + i * C + tq) * pk + ck + d0 + d;  // output index, token tq
+    const size_t ob = ((size_t)bh * T + i * C + tq) * pitch_k + col_k + d0 + d;  // output index, token tq
     const float tau = FLEX && a.inv_tau > 0.f ? 1.f / a.inv_tau : 0.f;
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
@@ -1060,7 +1060,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
         float dgv = ci + pre + pv[c];
         // raw logits: dx = dg sigmoid(-x) / tau, with sigmoid(-x) = 1 - e^{tau g} = -expm1(tau g)
         if (FLEX && a.inv_tau > 0.f) dgv *= -expm1f(tau * raw(L::PB_G, tq + c, d)) * a.inv_tau;
-        store_out<FLEX>(a.acc_g, a.add_g, a.dg, ob + (size_t)c * pk, dgv);
+        store_out<FLEX>(a.acc_g, a.add_g, a.dg, ob + (size_t)c * pitch_k, dgv);
       }
       pre += w[c];
     }
