@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 // hand over with named barriers: they arrive at kBarOps once a chunk's group-1 operands are in
 // shared memory and at kBarAB once its A operand is, and the producer waits at both.
 // ------------------------------------------------------------------------------------------
-template <int DK>
+template <int DK, bool KHILO = false>
 struct FwdPipeLayout {
   static constexpr uint32_t RAW = C * DK * 2;               // one raw q / k / g tile
   static constexpr uint32_t QKG = 3 * RAW;                  // a q/k/g stage (two stages)
@@ -258,7 +258,8 @@ struct FwdPipeLayout {
   static constexpr uint32_t QS_HI = V0 + 3 * VTB;           // Qs hi / lo [64 x DK]  K-major
   static constexpr uint32_t QS_LO = QS_HI + C * DK * 2;
   static constexpr uint32_t KH = QS_LO + C * DK * 2;        // Kh [64 x DK]  K-major B / MN-major A
-  static constexpr uint32_t SB_HI = KH + C * DK * 2;        // scaled state copy hi / lo [DK x 64]
+  static constexpr uint32_t KH_LO = KH + C * DK * 2;        // its lo part (KHILO builds)
+  static constexpr uint32_t SB_HI = KH_LO + (KHILO ? C * DK * 2 : 0);  // scaled state copy hi / lo [DK x 64]
   static constexpr uint32_t SB_LO = SB_HI + DK * DVT * 2;
   static constexpr uint32_t AB_HI = SB_LO + DK * DVT * 2;   // A hi / lo [64 x 64] K-major
   static constexpr uint32_t AB_LO = AB_HI + C * C * 2;
@@ -279,13 +280,15 @@ constexpr int PIPE_THREADS = NTHREADS + 32;  // 8 compute warps + the producer w
 constexpr int kBarOps = 2, kBarAB = 3;       // compute threads -> producer handoffs
 
 // FLEX: the build for wider tensors (column offsets, fp32 partial outputs with an added partial) and
-// raw-logit gates; the plain build has none of that code.
-template <int DK, bool FLEX>
+// raw-logit gates; the plain build has none of that code.  KHILO: Kh enters the MMAs as a bf16
+// hi + lo pair as well (for a caller whose output needs it, at the price of three more MMAs per
+// 16 keys in A and one more per 16 tokens in dS).
+template <int DK, bool FLEX, bool KHILO>
 __global__ void __launch_bounds__(PIPE_THREADS, 1)
     fwd_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
                     const FwdArgs args) {
-  using L = FwdPipeLayout<DK>;
+  using L = FwdPipeLayout<DK, KHILO>;
   using Gate = GateRun<DK, NTHREADS, FLEX>;
   const int ck = FLEX ? args.ck : 0, cv = FLEX ? args.cv : 0;  // column offsets into wider tensors
   constexpr int TS = Gate::TS;
@@ -371,15 +374,18 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
           const uint64_t ql_d = desc_sw128(base + L::QS_LO + koff, 16, 1024);
           umma_bf16(t_A, qh_d, kd, id_A, k > 0);
           umma_bf16(t_A, ql_d, kd, id_A, 1);
+          if (KHILO) umma_bf16(t_A, qh_d, desc_sw128(base + L::KH_LO + koff, 16, 1024), id_A, 1);
           const uint64_t sh = desc_sw128(base + L::SB_HI + k * 2048, 16, 1024);
           umma_bf16(t_O, qh_d, sh, id_O, k > 0);
           umma_bf16(t_O, qh_d, desc_sw128(base + L::SB_LO + k * 2048, 16, 1024), id_O, 1);
           umma_bf16(t_O, ql_d, sh, id_O, 1);
         }
 #pragma unroll
-        for (int k = 0; k < C / 16; ++k)
-          umma_bf16(t_dS, desc_sw128(base + L::KH + k * 2048, C * 128, 1024),
-                    desc_sw128(vbase + k * 2048, 16, 1024), id_S, k > 0);
+        for (int k = 0; k < C / 16; ++k) {
+          const uint64_t vd = desc_sw128(vbase + k * 2048, 16, 1024);
+          umma_bf16(t_dS, desc_sw128(base + L::KH + k * 2048, C * 128, 1024), vd, id_S, k > 0);
+          if (KHILO) umma_bf16(t_dS, desc_sw128(base + L::KH_LO + k * 2048, C * 128, 1024), vd, id_S, 1);
+        }
         umma_commit(&bar_mma1);
       }
       bar_sync(kBarAB, NHAND);  // chunk li's A operand is in shared memory; its raw tiles are free
@@ -440,7 +446,7 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     // Gate math of local chunk li (stage li & 1) into registers: Qs hi / lo and Kh for the two
     // dims gd, gd+1 and the tokens gh*TS .. gh*TS+TS-1 owned by this thread.  Returns the chunk's
     // exact-path flag (CTA-uniform).
-    uint32_t qh[TS], ql[TS], kh[TS];
+    uint32_t qh[TS], ql[TS], kh[TS], kl[KHILO ? TS : 1];
     int gd = 0, gh = 0;
     auto gate_regs = [&](int li) {
       const uint8_t* st = sm + (li & 1) * L::QKG;
@@ -467,7 +473,10 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
 #pragma unroll
       for (int u = TS - 1; u >= 0; --u) {
         const uint32_t wk = *reinterpret_cast<const uint32_t*>(st + L::RAW + ((gh * TS + u) * DK + gd) * 2);
-        kh[u] = pack2(bf_lo(wk) * f0, bf_hi(wk) * f1);
+        if (KHILO)
+          split2(bf_lo(wk) * f0, bf_hi(wk) * f1, kh[u], kl[KHILO ? u : 0]);
+        else
+          kh[u] = pack2(bf_lo(wk) * f0, bf_hi(wk) * f1);
         f0 *= gr.a0[u];
         f1 *= gr.a1[u];
       }
@@ -483,6 +492,7 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
         *reinterpret_cast<uint32_t*>(sm + L::QS_HI + off) = qh[u];
         *reinterpret_cast<uint32_t*>(sm + L::QS_LO + off) = ql[u];
         *reinterpret_cast<uint32_t*>(sm + L::KH + off) = kh[u];
+        if (KHILO) *reinterpret_cast<uint32_t*>(sm + L::KH_LO + off) = kl[KHILO ? u : 0];
       }
       if (s_owner) {
         const float sc = safe ? 1.f : decay_sm[(li & 1) * DK + s_row];
@@ -687,7 +697,8 @@ static cudaError_t launch_state_pass(const CUtensorMap& mk, const CUtensorMap& m
 template <int DK>
 static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o,
                               float* hT, int BH, int T, int dv, long long st_bh, long long st_row, float* acc_o,
-                              void* ws, cudaStream_t st, float inv_tau, int dk_total, int k0, const float* add_o) {
+                              void* ws, cudaStream_t st, float inv_tau, int dk_total, int k0, const float* add_o,
+                              bool kh_hilo) {
   CUtensorMap m[4];
   if (!make_map(&m[0], q, BH, T, dk_total, DK, false) || !make_map(&m[1], k, BH, T, dk_total, DK, false) ||
       !make_map(&m[2], g, BH, T, dk_total, DK, false) || !make_map(&m[3], v, BH, T, dv, DVT, true))
@@ -706,7 +717,7 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
   a.cv = 0;
   a.inv_tau = inv_tau;
   a.latch = device_error_latch();
-  const bool flex = inv_tau > 0.f || acc_o || add_o || k0 != 0 || dk_total != DK;
+  const bool flex = inv_tau > 0.f || acc_o || add_o || k0 != 0 || dk_total != DK || kh_hilo;
   plan_segments(BH, T, dv, &a.nseg, &a.seg_chunks);
   a.sbuf = nullptr;
   a.gam = nullptr;
@@ -714,8 +725,9 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
     if (!ws) return cudaErrorInvalidValue;
     a.sbuf = static_cast<float*>(ws);
     a.gam = a.sbuf + align256((size_t)BH * a.nseg * DK * dv * sizeof(float)) / sizeof(float);
-    cudaError_t e = flex ? launch_state_pass<DK, false, false, true>(m[1], m[2], m[3], a, BH, dv, st)
-                         : launch_state_pass<DK, false, false, false>(m[1], m[2], m[3], a, BH, dv, st);
+    cudaError_t e = kh_hilo ? launch_state_pass<DK, true, false, true>(m[1], m[2], m[3], a, BH, dv, st)
+                    : flex  ? launch_state_pass<DK, false, false, true>(m[1], m[2], m[3], a, BH, dv, st)
+                            : launch_state_pass<DK, false, false, false>(m[1], m[2], m[3], a, BH, dv, st);
     if (e != cudaSuccess) return e;
     if (a.nseg > 2) {
       const size_t n = (size_t)BH * DK * dv;
@@ -725,14 +737,17 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
       if (e != cudaSuccess) return e;
     }
   }
-  auto kern = flex ? fwd_pipe_kernel<DK, true> : fwd_pipe_kernel<DK, false>;
-  static std::atomic<bool> attr_set[2][64] = {};
+  // the split-Kh build exists for d_k = 64 only (its extra operand does not fit next to d_k = 128)
+  auto kern = kh_hilo ? fwd_pipe_kernel<DK, true, DK == 64> : flex ? fwd_pipe_kernel<DK, true, false>
+                                                                   : fwd_pipe_kernel<DK, false, false>;
+  const uint32_t alloc = kh_hilo ? FwdPipeLayout<DK, DK == 64>::ALLOC : FwdPipeLayout<DK>::ALLOC;
+  static std::atomic<bool> attr_set[3][64] = {};
   {
-    const cudaError_t e = ensure_smem_attr(kern, FwdPipeLayout<DK>::ALLOC, attr_set[flex ? 1 : 0]);
+    const cudaError_t e = ensure_smem_attr(kern, alloc, attr_set[kh_hilo ? 2 : flex ? 1 : 0]);
     if (e != cudaSuccess) return e;
   }
   dim3 grid(dv / DVT, BH, a.nseg);
-  kern<<<grid, PIPE_THREADS, FwdPipeLayout<DK>::ALLOC, st>>>(m[0], m[1], m[2], m[3], a);
+  kern<<<grid, PIPE_THREADS, alloc, st>>>(m[0], m[1], m[2], m[3], a);
   return cudaGetLastError();
 }
 
@@ -837,16 +852,18 @@ cudaError_t segment_entry_states(const void* k, const void* g, const void* v, co
 
 cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
                 int BH, int T, int dk, int dv, void* ws, cudaStream_t st, long long st_bh, long long st_row,
-                float* acc_o, float inv_tau, int dk_total, int k0, const float* add_o) {
+                float* acc_o, float inv_tau, int dk_total, int k0, const float* add_o, bool kh_hilo) {
   if (st_bh < 0) st_bh = (long long)dk * dv;
   if (st_row < 0) st_row = dv;
   if (dk_total < 0) dk_total = dk;
   if (k0 < 0 || k0 + dk > dk_total || k0 % 8 != 0) return cudaErrorInvalidValue;
+  if (kh_hilo && dk != 64) return cudaErrorNotSupported;
   if (dk == 64)
-    return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st, inv_tau, dk_total, k0, add_o);
+    return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st, inv_tau, dk_total, k0, add_o,
+                          kh_hilo);
   if (dk == 128)
     return launch_fwd<128>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st, inv_tau, dk_total, k0,
-                           add_o);
+                           add_o, false);
   return cudaErrorNotSupported;
 }
 

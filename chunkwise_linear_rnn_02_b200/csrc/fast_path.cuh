@@ -21,10 +21,11 @@ size_t fwd_workspace(int BH, int T, int dk, int dv);
 // raw logits x and the kernels use g = bf16(logsigmoid(x) * inv_tau).  A key block of wider
 // tensors: q, k, g are [BH][T][dk_total] and the call uses columns k0 .. k0+dk-1 (read in place by
 // the tile loads); add_o ([BH*T][dv] fp32) is added to o before it is stored (to acc_o or as bf16).
+// kh_hilo (d_k = 64 only): the decayed keys enter the MMAs as bf16 hi + lo pairs too.
 cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
                 int BH, int T, int dk, int dv, void* ws, cudaStream_t st, long long st_bh = -1,
                 long long st_row = -1, float* acc_o = nullptr, float inv_tau = 0.f, int dk_total = -1, int k0 = 0,
-                const float* add_o = nullptr);
+                const float* add_o = nullptr, bool kh_hilo = false);
 
 // A backward sub-problem inside wider tensors (split shapes, padded operands): its key dimensions
 // are columns ck.. of [BH*T][pk] arrays (the q, k, g inputs and every key-side output array), its

@@ -83,18 +83,24 @@ struct BwdArgs {
 };
 
 
-// One gradient value.  FLEX builds: plus the partial sum in add (if any), then fp32 into acc (itself
-// a partial sum, which may be add's own element) or bf16 into out; the plain build stores bf16.
+// One gradient value: FLEX builds store fp32 into acc (a partial sum) when it is set, else bf16
+// into out; the plain build stores bf16.
 template <bool FLEX>
-__device__ __forceinline__ void store_out(float* acc, const float* add, __nv_bfloat16* out, size_t idx, float val) {
-  if (FLEX) {
-    if (add) val += add[idx];
-    if (acc) {
-      acc[idx] = val;
-      return;
-    }
-  }
-  out[idx] = __float2bfloat16_rn(val);
+__device__ __forceinline__ void store_out(float* acc, __nv_bfloat16* out, size_t idx, float val) {
+  if (FLEX && acc)
+    acc[idx] = val;
+  else
+    out[idx] = __float2bfloat16_rn(val);
+}
+
+// FLEX builds: the partial sums (of earlier sub-problems) for N outputs at idx0 + c * pitch, 0 where
+// add is null or past the first `valid`; all loads are issued before any of them is used, so that
+// they are in flight together (the stores that follow may alias add, which would otherwise order
+// every load after the previous store).
+template <bool FLEX, int N>
+__device__ __forceinline__ void load_adds(const float* add, size_t idx0, long long pitch, int valid, float (&out)[N]) {
+#pragma unroll
+  for (int c = 0; c < N; ++c) out[c] = (FLEX && add && c < valid) ? add[idx0 + (size_t)c * pitch] : 0.f;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -388,6 +394,8 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       const size_t ob = ((size_t)bh * T + i * C + tb) * pitch_k + col_k + d0 + d;  // output index, token tb
 #pragma unroll
       for (int rr = 0; rr < 4; ++rr) {
+        float ad[TS];
+        load_adds<FLEX, TS>(a.add_q, ob + (size_t)(rr * TS) * pitch_k, pitch_k, T - (i * C + tb + rr * TS), ad);
         float e = 1.f;  // E1 = e^{B_j}, formed as GateRun::forward forms it
         for (int hh = 0; hh < half * 4 + rr; ++hh) e *= tot[hh * KT + d];
 #pragma unroll
@@ -397,7 +405,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
           if (!safe) y[c] *= e * inv;
           const float qv = raw(pq, j, d), kv = raw(pk, j, d);
           if (i * C + j < T) {
-            store_out<FLEX>(a.acc_q, a.add_q, a.dq, ob + (size_t)c * pitch_k, e * x[c] + y[c]);
+            store_out<FLEX>(a.acc_q, a.dq, ob + (size_t)c * pitch_k, e * x[c] + y[c] + ad[u]);
           }
           x[c] = bf_split_sum(qv * e) * x[c];  // Qt X, with Qt as the G update sees it
           y[c] = qv * (y[c] - DIAG[j] * kv);   // q dq^intra without j = r
@@ -747,8 +755,14 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       tmem_ld_wait();
       const size_t ob = ((size_t)bh * T + t0) * pitch_v + col_v + c0 + vcol;  // output index, token t0
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
-        if (t0 + c < T) store_out<FLEX>(a.acc_v, a.add_v, a.dv, ob + (size_t)c * pitch_v, v[c]);
+      for (int hh = 0; hh < 2; ++hh) {  // 16 tokens at a time keeps the register count down
+        float ad[16];
+        load_adds<FLEX, 16>(a.add_v, ob + (size_t)(16 * hh) * pitch_v, pitch_v, T - (t0 + 16 * hh), ad);
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          if (t0 + 16 * hh + c < T)
+            store_out<FLEX>(a.acc_v, a.dv, ob + (size_t)(16 * hh + c) * pitch_v, v[16 * hh + c] + ad[c]);
+      }
     }
     tc_fence_before();
     __syncthreads();
@@ -1021,7 +1035,8 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
 #pragma unroll
     for (int rr = 0; rr < 16 / TS; ++rr) {
       const int h = tq / TS + rr;
-      float al[TS], e2[TS];
+      float al[TS], e2[TS], ad[TS];
+      load_adds<FLEX, TS>(a.add_k, ob + (size_t)(rr * TS) * pitch_k, pitch_k, T - (i * C + tq + rr * TS), ad);
 #pragma unroll
       for (int u = 0; u < TS; ++u) al[u] = ex2(raw(L::PB_G, h * TS + u, d) * kLog2e);
       float e = 1.f;  // E2 = e^{gamma - B_r}, formed as GateRun::backward forms it
@@ -1038,7 +1053,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
         if (!safe) w[c] *= ev * inv;
         const float qv = raw(L::PB_Q, r, d), kv = raw(L::PB_K, r, d);
         if (i * C + r < T) {
-          store_out<FLEX>(a.acc_k, a.add_k, a.dk, ob + (size_t)c * pitch_k, ev * z[c] + w[c]);
+          store_out<FLEX>(a.acc_k, a.dk, ob + (size_t)c * pitch_k, ev * z[c] + w[c] + ad[u]);
         }
         const float kz = bf_split_sum(kv * ev) * z[c];  // Kh Z, with Kh as the S update sees it
         w[c] = kz + kv * (w[c] - DIAG[r] * qv);        // plus k dk^intra without j = r
@@ -1054,13 +1069,15 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
     for (int t = 0; t < qi; ++t) pre += XQ[t * KT + d];
     const size_t ob = ((size_t)bh * T + i * C + tq) * pitch_k + col_k + d0 + d;  // output index, token tq
     const float tau = FLEX && a.inv_tau > 0.f ? 1.f / a.inv_tau : 0.f;
+    float ad[16];
+    load_adds<FLEX, 16>(a.add_g, ob, pitch_k, T - (i * C + tq), ad);
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       if (i * C + tq + c < T) {
         float dgv = ci + pre + pv[c];
         // raw logits: dx = dg sigmoid(-x) / tau, with sigmoid(-x) = 1 - e^{tau g} = -expm1(tau g)
         if (FLEX && a.inv_tau > 0.f) dgv *= -expm1f(tau * raw(L::PB_G, tq + c, d)) * a.inv_tau;
-        store_out<FLEX>(a.acc_g, a.add_g, a.dg, ob + (size_t)c * pitch_k, dgv);
+        store_out<FLEX>(a.acc_g, a.dg, ob + (size_t)c * pitch_k, dgv + ad[c]);
       }
       pre += w[c];
     }

@@ -333,7 +333,7 @@ bool gsa_fused_fwd_ok(int BH, int T, int dk, int dv, int m, int chunk, int dtype
 bool gsa_fused_bwd_ok(int BH, int T, int dk, int dv, int m, int chunk, int dtype) {
   return gsa_fused_fwd_ok(BH, T, dk, dv, m, chunk, dtype) && 2 * m == 128 &&
          gla::fast::bwd_supported(BH, T, 128, dv, chunk, dtype) && gla::fast::bwd_supported(BH, T, 128, dk, chunk, dtype) &&
-         gla::fast::fwd_supported(BH, T, 128, dk, chunk, dtype);
+         gla::fast::fwd_supported(BH, T, m, dk, chunk, dtype);
 }
 
 struct GsaFusedFwdWs {
@@ -355,6 +355,7 @@ struct GsaFusedBwdWs {
   bf16* do1;                       // [rows][128]: do1 [hi | lo]
   float *dq1, *dphi1, *dg1;        // pass-1 backward outputs: [rows][128] x 3
   float *h0p, *dhTp, *dh0p, *h0t;  // [BH][128][dk] x 3, [BH][m][dk]
+  float* dqp;                      // [rows][dk] fp32: dq's partial from the queries' hi half
   void *p1ws, *fws;
 };
 size_t carve_gsa_fused_bwd(Carve& c, int BH, int T, int dk, int dv, int m, GsaFusedBwdWs* w) {
@@ -370,8 +371,9 @@ size_t carve_gsa_fused_bwd(Carve& c, int BH, int T, int dk, int dv, int m, GsaFu
   x.dhTp = c.take<float>(sp);
   x.dh0p = c.take<float>(sp);
   x.h0t = c.take<float>((size_t)BH * m * dk);
+  x.dqp = c.take<float>(rows * dk);
   x.p1ws = c.take<char>(gla::gsa::pass1_workspace(BH, T, dk));
-  x.fws = c.take<char>(gla::fast::fwd_workspace(BH, T, 128, dk));
+  x.fws = c.take<char>(gla::fast::fwd_workspace(BH, T, m, dk));
   if (w) *w = x;
   return c.used;
 }
@@ -431,8 +433,13 @@ int gsa_bwd_fused(const bf16* q, const bf16* k, const bf16* v, const bf16* phi, 
   const gla::fast::BwdAccum acc1{w.dq1, w.dphi1, w.dg1, nullptr, 128, 0, dkd, 0};  // dk (its dv) straight to bf16
   GLA_CUDA(gla::fast::bwd(w.do1, f.phi, k, f.g, h01 ? w.h0p : nullptr, q, dhT1 ? w.dhTp : nullptr, nullptr, nullptr,
                           dk, nullptr, dh01 ? w.dh0p : nullptr, BH, T, 128, dkd, f.ws, st, -1, -1, &acc1));
-  // dq = S1 do1: the output of the GLA with queries do1, keys phi, values k from h0_1^T
-  GLA_CUDA(gla::fast::fwd(w.do1, f.phi, k, f.g, h01 ? w.h0p : nullptr, dq, nullptr, BH, T, 128, dkd, w.fws, st));
+  // dq = S1 do1: the output of the GLA with queries do1, keys phi, values k from h0_1^T, as two
+  // d_k = 64 forwards over the queries' hi and lo halves (the second adds the first's partial), with
+  // the decayed keys as bf16 hi + lo pairs (a single bf16 put dq 2 % off in the emulation)
+  GLA_CUDA(gla::fast::fwd(w.do1, f.phi, k, f.g, h01 ? w.h0t : nullptr, nullptr, nullptr, BH, T, m, dkd, w.fws, st, -1,
+                          -1, w.dqp, 0.f, 128, 0, nullptr, true));
+  GLA_CUDA(gla::fast::fwd(w.do1, f.phi, k, f.g, h01 ? w.h0t : nullptr, dq, nullptr, BH, T, m, dkd, w.fws, st, -1, -1,
+                          nullptr, 0.f, 128, m, w.dqp, true));
   // both passes' and both copies' contributions to dphi and dg; dh0_1 back to [dk][m]
   GLA_CUDA(gla::gsa::fold_add_bf16(w.dphi1, f.dk, dphi, rows, m, st));
   GLA_CUDA(gla::gsa::fold_add_bf16(w.dg1, f.dg, dg, rows, m, st));
