@@ -90,12 +90,12 @@ struct StateLayout {
   static_assert(STAGE % 1024 == 0 && RAW % 1024 == 0, "stage alignment");
 };
 
-template <int DK, bool HILO, bool REV, bool FLEX>
+template <int DK, bool HILO, bool REV, bool FLEX, bool LOGIT>
 __global__ void __launch_bounds__(NTHREADS, 1)
     fwd_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_g,
                      const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
   using L = StateLayout<DK, HILO>;
-  using Gate = GateRun<DK, NTHREADS, FLEX>;
+  using Gate = GateRun<DK, NTHREADS, LOGIT>;
   const int ck = FLEX ? args.ck : 0, cv = FLEX ? args.cv : 0;  // column offsets into wider tensors
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_load[2], bar_mma;
@@ -283,13 +283,13 @@ constexpr int kBarOps = 2, kBarAB = 3;       // compute threads -> producer hand
 // raw-logit gates; the plain build has none of that code.  KHILO: Kh enters the MMAs as a bf16
 // hi + lo pair as well (for a caller whose output needs it, at the price of three more MMAs per
 // 16 keys in A and one more per 16 tokens in dS).
-template <int DK, bool FLEX, bool KHILO>
+template <int DK, bool FLEX, bool KHILO, bool LOGIT>
 __global__ void __launch_bounds__(PIPE_THREADS, 1)
     fwd_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
                     const FwdArgs args) {
   using L = FwdPipeLayout<DK, KHILO>;
-  using Gate = GateRun<DK, NTHREADS, FLEX>;
+  using Gate = GateRun<DK, NTHREADS, LOGIT>;
   const int ck = FLEX ? args.ck : 0, cv = FLEX ? args.cv : 0;  // column offsets into wider tensors
   constexpr int TS = Gate::TS;
   constexpr int NHAND = NTHREADS + 32;  // threads taking part in a handoff barrier
@@ -685,9 +685,11 @@ size_t fwd_workspace(int BH, int T, int dk, int dv) {
 template <int DK, bool HILO, bool REV, bool FLEX>
 static cudaError_t launch_state_pass(const CUtensorMap& mk, const CUtensorMap& mg, const CUtensorMap& mv,
                                      const FwdArgs& args, int BH, int dv, cudaStream_t st) {
-  auto kern = fwd_state_kernel<DK, HILO, REV, FLEX>;
-  static std::atomic<bool> attr_set[64] = {};
-  const cudaError_t e = ensure_smem_attr(kern, StateLayout<DK, HILO>::ALLOC, attr_set);
+  // raw-logit gates only in a build of their own
+  auto kern = args.inv_tau > 0.f ? fwd_state_kernel<DK, HILO, REV, FLEX, FLEX>
+                                 : fwd_state_kernel<DK, HILO, REV, FLEX, false>;
+  static std::atomic<bool> attr_set[2][64] = {};
+  const cudaError_t e = ensure_smem_attr(kern, StateLayout<DK, HILO>::ALLOC, attr_set[args.inv_tau > 0.f ? 1 : 0]);
   if (e != cudaSuccess) return e;
   dim3 grid(dv / DVT, BH, args.nseg - 1);
   kern<<<grid, NTHREADS, StateLayout<DK, HILO>::ALLOC, st>>>(mk, mg, mv, args);
@@ -738,12 +740,15 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
     }
   }
   // the split-Kh build exists for d_k = 64 only (its extra operand does not fit next to d_k = 128)
-  auto kern = kh_hilo ? fwd_pipe_kernel<DK, true, DK == 64> : flex ? fwd_pipe_kernel<DK, true, false>
-                                                                   : fwd_pipe_kernel<DK, false, false>;
+  const bool logit = inv_tau > 0.f;
+  auto kern = kh_hilo ? fwd_pipe_kernel<DK, true, DK == 64, false>
+              : logit ? fwd_pipe_kernel<DK, true, false, true>
+              : flex  ? fwd_pipe_kernel<DK, true, false, false>
+                      : fwd_pipe_kernel<DK, false, false, false>;
   const uint32_t alloc = kh_hilo ? FwdPipeLayout<DK, DK == 64>::ALLOC : FwdPipeLayout<DK>::ALLOC;
-  static std::atomic<bool> attr_set[3][64] = {};
+  static std::atomic<bool> attr_set[4][64] = {};
   {
-    const cudaError_t e = ensure_smem_attr(kern, alloc, attr_set[kh_hilo ? 2 : flex ? 1 : 0]);
+    const cudaError_t e = ensure_smem_attr(kern, alloc, attr_set[kh_hilo ? 3 : logit ? 2 : flex ? 1 : 0]);
     if (e != cudaSuccess) return e;
   }
   dim3 grid(dv / DVT, BH, a.nseg);
@@ -857,7 +862,7 @@ cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, cons
   if (st_row < 0) st_row = dv;
   if (dk_total < 0) dk_total = dk;
   if (k0 < 0 || k0 + dk > dk_total || k0 % 8 != 0) return cudaErrorInvalidValue;
-  if (kh_hilo && dk != 64) return cudaErrorNotSupported;
+  if (kh_hilo && (dk != 64 || inv_tau > 0.f)) return cudaErrorNotSupported;
   if (dk == 64)
     return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st, inv_tau, dk_total, k0, add_o,
                           kh_hilo);

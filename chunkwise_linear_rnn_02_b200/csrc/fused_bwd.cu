@@ -157,11 +157,11 @@ struct KeyLayout {
 // buffer, Kh operand, state copy and rescale) and issue its group 1; then finish chunk i's
 // outputs.  The epilogue forms E1 / E2 itself from the raw gates and the run products of the gate
 // run, multiplying in the same order, so its values equal the ones behind the MMA operands.
-template <int DK, int DV, bool FLEX>
+template <int DK, int DV, bool FLEX, bool LOGIT>
 __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int tau, int seg,
                               uint64_t* bars, uint32_t tmem) {
   using L = KeyLayout<DK, DV>;
-  using Gate = GateRun<KT, BT, FLEX>;
+  using Gate = GateRun<KT, BT, LOGIT>;
   constexpr int NS = L::NS, TS = Gate::TS;
   // column offsets into wider tensors and the key-side row pitch (FLEX builds only)
   const int col_k = FLEX ? a.ck : 0, col_v = FLEX ? a.cv : 0, pitch_k = FLEX ? a.pk : DK;
@@ -405,7 +405,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
           if (!safe) y[c] *= e * inv;
           const float qv = raw(pq, j, d), kv = raw(pk, j, d);
           if (i * C + j < T) {
-            store_out<FLEX>(a.acc_q, a.dq, ob + (size_t)c * pitch_k, e * x[c] + y[c] + ad[u]);
+            store_out<FLEX>(a.acc_q, a.dq, ob + (size_t)c * pitch_k, FLEX ? e * x[c] + y[c] + ad[u] : e * x[c] + y[c]);
           }
           x[c] = bf_split_sum(qv * e) * x[c];  // Qt X, with Qt as the G update sees it
           y[c] = qv * (y[c] - DIAG[j] * kv);   // q dq^intra without j = r
@@ -496,11 +496,11 @@ struct ValLayout {
   static_assert(C * DK * 4 <= KH_HI - QP_HI && C * C * 4 <= GC_HI - KH_HI, "exact-path scratch");
 };
 
-template <int DK, bool FLEX>
+template <int DK, bool FLEX, bool LOGIT>
 __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int vt, int DV, int seg,
                               uint64_t* bars, uint32_t tmem) {
   using L = ValLayout<DK>;
-  using Gate = GateRun<DK, BT, FLEX>;
+  using Gate = GateRun<DK, BT, LOGIT>;
   // column offsets into wider tensors and the value-side row pitch (FLEX builds only)
   const int col_k = FLEX ? a.ck : 0, col_v = FLEX ? a.cv : 0, pitch_v = FLEX ? a.pv : DV;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -761,7 +761,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
 #pragma unroll
         for (int c = 0; c < 16; ++c)
           if (t0 + 16 * hh + c < T)
-            store_out<FLEX>(a.acc_v, a.dv, ob + (size_t)(16 * hh + c) * pitch_v, v[16 * hh + c] + ad[c]);
+            store_out<FLEX>(a.acc_v, a.dv, ob + (size_t)(16 * hh + c) * pitch_v, FLEX ? v[16 * hh + c] + ad[c] : v[16 * hh + c]);
       }
     }
     tc_fence_before();
@@ -849,10 +849,10 @@ struct ChunkLayout {
   static_assert(PB % 1024 == 0 && KQ_HI % 1024 == 0 && 2 * TILE <= VB, "operand layout");
 };
 
-template <int DK, int DV, bool FLEX>
+template <int DK, int DV, bool FLEX, bool LOGIT>
 __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
   using L = ChunkLayout<DK, DV>;
-  using Gate = GateRun<KT, BT, FLEX>;
+  using Gate = GateRun<KT, BT, LOGIT>;
   // column offsets into wider tensors and the key-side row pitch (FLEX builds only)
   const int col_k = FLEX ? a.ck : 0, col_v = FLEX ? a.cv : 0, pitch_k = FLEX ? a.pk : DK;
   constexpr int NS = L::NS, TS = Gate::TS, NVT = DV / VT;
@@ -1053,7 +1053,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
         if (!safe) w[c] *= ev * inv;
         const float qv = raw(L::PB_Q, r, d), kv = raw(L::PB_K, r, d);
         if (i * C + r < T) {
-          store_out<FLEX>(a.acc_k, a.dk, ob + (size_t)c * pitch_k, ev * z[c] + w[c] + ad[u]);
+          store_out<FLEX>(a.acc_k, a.dk, ob + (size_t)c * pitch_k, FLEX ? ev * z[c] + w[c] + ad[u] : ev * z[c] + w[c]);
         }
         const float kz = bf_split_sum(kv * ev) * z[c];  // Kh Z, with Kh as the S update sees it
         w[c] = kz + kv * (w[c] - DIAG[r] * qv);        // plus k dk^intra without j = r
@@ -1068,7 +1068,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
     float pre = 0.f;
     for (int t = 0; t < qi; ++t) pre += XQ[t * KT + d];
     const size_t ob = ((size_t)bh * T + i * C + tq) * pitch_k + col_k + d0 + d;  // output index, token tq
-    const float tau = FLEX && a.inv_tau > 0.f ? 1.f / a.inv_tau : 0.f;
+    const float tau = LOGIT && a.inv_tau > 0.f ? 1.f / a.inv_tau : 0.f;
     float ad[16];
     load_adds<FLEX, 16>(a.add_g, ob, pitch_k, T - (i * C + tq), ad);
 #pragma unroll
@@ -1076,8 +1076,8 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
       if (i * C + tq + c < T) {
         float dgv = ci + pre + pv[c];
         // raw logits: dx = dg sigmoid(-x) / tau, with sigmoid(-x) = 1 - e^{tau g} = -expm1(tau g)
-        if (FLEX && a.inv_tau > 0.f) dgv *= -expm1f(tau * raw(L::PB_G, tq + c, d)) * a.inv_tau;
-        store_out<FLEX>(a.acc_g, a.dg, ob + (size_t)c * pitch_k, dgv + ad[c]);
+        if (LOGIT && a.inv_tau > 0.f) dgv *= -expm1f(tau * raw(L::PB_G, tq + c, d)) * a.inv_tau;
+        store_out<FLEX>(a.acc_g, a.dg, ob + (size_t)c * pitch_k, FLEX ? dgv + ad[c] : dgv);
       }
       pre += w[c];
     }
@@ -1097,7 +1097,7 @@ struct BwdSmem {
   static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
 
-template <int DK, int DV, bool FLEX>
+template <int DK, int DV, bool FLEX, bool LOGIT>
 __global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bars[5];
@@ -1121,20 +1121,20 @@ __global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant_
   const int per_seg = a.n_bh * per_head;
   const int seg = blockIdx.x / per_seg, bh = (blockIdx.x % per_seg) / per_head, role = blockIdx.x % per_head;
   if (role < DK / KT)
-    key_tile_body<DK, DV, FLEX>(sm, mp, a, bh, role, seg, bars, tmem);
+    key_tile_body<DK, DV, FLEX, LOGIT>(sm, mp, a, bh, role, seg, bars, tmem);
   else
-    val_tile_body<DK, FLEX>(sm, mp, a, bh, role - DK / KT, DV, seg, bars, tmem);
+    val_tile_body<DK, FLEX, LOGIT>(sm, mp, a, bh, role - DK / KT, DV, seg, bars, tmem);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-template <int DK, int DV, bool FLEX>
+template <int DK, int DV, bool FLEX, bool LOGIT>
 static cudaError_t launch_all(const BwdMaps& mp, const BwdArgs& a, int BH, cudaStream_t st) {
   constexpr uint32_t CHK = ChunkLayout<DK, DV>::TOTAL + 1024;
   static_assert(2 * CHK <= 228 * 1024, "two chunk CTAs per SM");
-  auto k1 = bwd_fused_kernel<DK, DV, FLEX>;
-  auto k3 = bwd_chunk_kernel<DK, DV, FLEX>;
+  auto k1 = bwd_fused_kernel<DK, DV, FLEX, LOGIT>;
+  auto k3 = bwd_chunk_kernel<DK, DV, FLEX, LOGIT>;
   static std::atomic<bool> attr1[64] = {}, attr3[64] = {};
   {
     cudaError_t e = ensure_smem_attr(k1, BwdSmem<DK, DV>::ALLOC, attr1);
@@ -1244,9 +1244,11 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
                                          DK, DV, a.nseg, a.seg_chunks, st_bh, st_row, st, inv_tau, CK, CV);
     if (e != cudaSuccess) return e;
   }
-  // the plain build unless the call needs offsets, partial sums or raw-logit gates
-  if (acc || inv_tau > 0.f) return launch_all<DK, DV, true>(mp, a, BH, st);
-  return launch_all<DK, DV, false>(mp, a, BH, st);
+  // the plain build unless the call needs offsets or partial sums (FLEX) or raw-logit gates (LOGIT,
+  // a build of its own so that the others carry none of its code)
+  if (inv_tau > 0.f) return launch_all<DK, DV, true, true>(mp, a, BH, st);
+  if (acc) return launch_all<DK, DV, true, false>(mp, a, BH, st);
+  return launch_all<DK, DV, false, false>(mp, a, BH, st);
 }
 
 cudaError_t bwd(const void* q, const void* k, const void* v, const void* g, const float* h0, const void* dO,

@@ -227,7 +227,7 @@ struct GateRun {
     h = tid / NPAIR;
     d = 2 * p;
     if (LOGIT && inv_tau > 0.f) {
-#pragma unroll
+#pragma unroll 1
       for (int u = 0; u < TS; ++u) {
         const int j = h * TS + u;
         uint32_t* ptr = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(graw) +
