@@ -28,14 +28,13 @@ cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, cons
                 const float* add_o = nullptr, bool kh_hilo = false);
 
 // A backward sub-problem inside wider tensors (split shapes, padded operands): its key dimensions
-// are columns ck.. of [BH*T][pk] arrays (the q, k, g inputs and every key-side output array), its
-// value columns are cv.. of [BH*T][pv] arrays (v, dO and the dv arrays).  A non-null q / k / g / v
-// receives that gradient in fp32 (a partial sum) in place of the bf16 output; otherwise the bf16
-// output is written, after adding add_q / add_k / add_g / add_v (fp32 partial sums) where given.
+// are columns ck.. of the [BH*T][pk] inputs q, k, g, its value columns cv.. of the [BH*T][pv] inputs
+// v and dO.  The key-side gradients go in fp32 to q / k / g (all required, [BH*T][dk] each) in place
+// of the bf16 outputs; dv goes in fp32 to v ([BH*T][dv]), or, with v null, in bf16 to the dv output,
+// then [BH*T][pv] and written at columns cv...
 struct BwdAccum {
   float *q, *k, *g, *v;
   int pk, ck, pv, cv;
-  const float *add_q, *add_k, *add_g, *add_v;
 };
 
 // Sequence split of the backward (d_k = 128): segment count and length, and the segment states

@@ -68,13 +68,12 @@ struct BwdArgs {
   int nseg, seg_chunks, n_bh;
   const float *s_in, *g_end;
   long long st_bh, st_row;  // h0 / dhT / dh0 strides (a sub-block of a larger state when split)
-  // Outputs: with acc_x set, x goes in fp32 to acc_x (a partial sum of a split shape); else in bf16
-  // to the output, plus add_x (fp32: the partial sum of earlier sub-problems) where that is set.
-  // Key-side arrays (the q, k, g inputs, dq, dk, dg and their acc / add arrays) are [BH*T][pk] with
-  // this call's key dimensions from column ck; value-side ones (v, dO, dv, acc_v, add_v) are
-  // [BH*T][pv] with this call's value columns from cv.  The tile loads read them in place.
+  // FLEX builds: the inputs are column blocks of wider arrays, read in place by the tile loads: q,
+  // k, g are [BH*T][pk] with this call's key dimensions from column ck, v and dO [BH*T][pv] with its
+  // value columns from cv.  The gradients go in fp32 to acc_q / acc_k / acc_g ([BH*T][DK] each) and
+  // acc_v ([BH*T][DV]) in place of the bf16 outputs; with acc_v null, dv goes in bf16 to the value
+  // columns of dv, [BH*T][pv].
   float *acc_q, *acc_k, *acc_g, *acc_v;
-  const float *add_q, *add_k, *add_g, *add_v;
   int pk, ck, pv, cv;
   // > 0: the gate tensor holds raw logits x (g = logsigmoid(x) / tau) and the gate-gradient output
   // receives dx = dg sigmoid(-x) / tau in place of dg
@@ -82,26 +81,6 @@ struct BwdArgs {
   unsigned int* latch;
 };
 
-
-// One gradient value: FLEX builds store fp32 into acc (a partial sum) when it is set, else bf16
-// into out; the plain build stores bf16.
-template <bool FLEX>
-__device__ __forceinline__ void store_out(float* acc, __nv_bfloat16* out, size_t idx, float val) {
-  if (FLEX && acc)
-    acc[idx] = val;
-  else
-    out[idx] = __float2bfloat16_rn(val);
-}
-
-// FLEX builds: the partial sums (of earlier sub-problems) for N outputs at idx0 + c * pitch, 0 where
-// add is null or past the first `valid`; all loads are issued before any of them is used, so that
-// they are in flight together (the stores that follow may alias add, which would otherwise order
-// every load after the previous store).
-template <bool FLEX, int N>
-__device__ __forceinline__ void load_adds(const float* add, size_t idx0, long long pitch, int valid, float (&out)[N]) {
-#pragma unroll
-  for (int c = 0; c < N; ++c) out[c] = (FLEX && add && c < valid) ? add[idx0 + (size_t)c * pitch] : 0.f;
-}
 
 // ------------------------------------------------------------------------------------------
 // Key-tile CTA
@@ -163,8 +142,8 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   using L = KeyLayout<DK, DV>;
   using Gate = GateRun<KT, BT, LOGIT>;
   constexpr int NS = L::NS, TS = Gate::TS;
-  // column offsets into wider tensors and the key-side row pitch (FLEX builds only)
-  const int col_k = FLEX ? a.ck : 0, col_v = FLEX ? a.cv : 0, pitch_k = FLEX ? a.pk : DK;
+  // column offsets into wider input tensors (FLEX builds only)
+  const int col_k = FLEX ? a.ck : 0, col_v = FLEX ? a.cv : 0;
   static_assert(TS == 8 && NS == 8, "epilogue runs: four gate runs of eight tokens per token half");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
@@ -218,7 +197,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   auto dA_at = [&](int j, int r) { return raw(L::DA_HI, j, r) + raw(L::DA_LO, j, r); };
   // Gate run of the chunk in part-B buffer b: run products into TOT[b], decays into DEC[b].
   auto gate = [&](Gate& gr, int b, int chunk) {
-    gr.set_logit(a.inv_tau, T - chunk * C);
+    if constexpr (LOGIT) gr.set_logit(a.inv_tau, T - chunk * C);
     const bool weak = gr.run_swizzled(sm + pbo(b) + L::PB_G, TOT + b * NS * KT);
     if (gr.h == 0) {
       DEC[b * KT + gr.d] = gr.dec0;
@@ -391,11 +370,10 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         }
       }
       const float inv = 1.f / DEC[b * KT + d];
-      const size_t ob = ((size_t)bh * T + i * C + tb) * pitch_k + col_k + d0 + d;  // output index, token tb
+      __nv_bfloat16* dst = a.dq + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
+      float* dst32 = FLEX ? a.acc_q + ((size_t)bh * T + i * C + tb) * DK + d0 + d : nullptr;
 #pragma unroll
       for (int rr = 0; rr < 4; ++rr) {
-        float ad[TS];
-        load_adds<FLEX, TS>(a.add_q, ob + (size_t)(rr * TS) * pitch_k, pitch_k, T - (i * C + tb + rr * TS), ad);
         float e = 1.f;  // E1 = e^{B_j}, formed as GateRun::forward forms it
         for (int hh = 0; hh < half * 4 + rr; ++hh) e *= tot[hh * KT + d];
 #pragma unroll
@@ -405,7 +383,10 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
           if (!safe) y[c] *= e * inv;
           const float qv = raw(pq, j, d), kv = raw(pk, j, d);
           if (i * C + j < T) {
-            store_out<FLEX>(a.acc_q, a.dq, ob + (size_t)c * pitch_k, FLEX ? e * x[c] + y[c] + ad[u] : e * x[c] + y[c]);
+            if constexpr (FLEX)
+              dst32[(size_t)c * DK] = e * x[c] + y[c];
+            else
+              dst[(size_t)c * DK] = __float2bfloat16_rn(e * x[c] + y[c]);
           }
           x[c] = bf_split_sum(qv * e) * x[c];  // Qt X, with Qt as the G update sees it
           y[c] = qv * (y[c] - DIAG[j] * kv);   // q dq^intra without j = r
@@ -579,7 +560,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     mbar_wait(bar_ld, ph_ld, a.latch);
     ph_ld ^= 1;
     Gate gr;
-    gr.set_logit(a.inv_tau, T - i * C);
+    if constexpr (LOGIT) gr.set_logit(a.inv_tau, T - i * C);
     const bool weak = gr.run(sm + 2 * L::RAW, DK, TOT);
     if (gr.h == 0) {
       DEC[gr.d] = gr.dec0;
@@ -753,15 +734,21 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       const int vcol = q4 * 32 + lane, t0 = i * C + half * 32;
       tmem_ld32(tmem + L::T_DV + lane_off + half * 32, v);
       tmem_ld_wait();
-      const size_t ob = ((size_t)bh * T + t0) * pitch_v + col_v + c0 + vcol;  // output index, token t0
+      if (FLEX && a.acc_v) {
+        float* p = a.acc_v + ((size_t)bh * T + t0) * DV + c0 + vcol;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {  // 16 tokens at a time keeps the register count down
-        float ad[16];
-        load_adds<FLEX, 16>(a.add_v, ob + (size_t)(16 * hh) * pitch_v, pitch_v, T - (t0 + 16 * hh), ad);
+        for (int c = 0; c < 32; ++c)
+          if (t0 + c < T) p[(size_t)c * DV] = v[c];
+      } else if (FLEX) {  // dv in bf16 at the value columns of a [BH*T][pv] array
+        __nv_bfloat16* p = a.dv + ((size_t)bh * T + t0) * pitch_v + col_v + c0 + vcol;
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-          if (t0 + 16 * hh + c < T)
-            store_out<FLEX>(a.acc_v, a.dv, ob + (size_t)(16 * hh + c) * pitch_v, FLEX ? v[16 * hh + c] + ad[c] : v[16 * hh + c]);
+        for (int c = 0; c < 32; ++c)
+          if (t0 + c < T) p[(size_t)c * pitch_v] = __float2bfloat16_rn(v[c]);
+      } else {
+        __nv_bfloat16* p = a.dv + ((size_t)bh * T + t0) * DV + c0 + vcol;
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (t0 + c < T) p[(size_t)c * DV] = __float2bfloat16_rn(v[c]);
       }
     }
     tc_fence_before();
@@ -853,8 +840,8 @@ template <int DK, int DV, bool FLEX, bool LOGIT>
 __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
   using L = ChunkLayout<DK, DV>;
   using Gate = GateRun<KT, BT, LOGIT>;
-  // column offsets into wider tensors and the key-side row pitch (FLEX builds only)
-  const int col_k = FLEX ? a.ck : 0, col_v = FLEX ? a.cv : 0, pitch_k = FLEX ? a.pk : DK;
+  // column offsets into wider input tensors (FLEX builds only)
+  const int col_k = FLEX ? a.ck : 0, col_v = FLEX ? a.cv : 0;
   constexpr int NS = L::NS, TS = Gate::TS, NVT = DV / VT;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_ld, bar_m1, bar_m2;
@@ -954,7 +941,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   }
   // gate run of the key slab: Qt hi / lo, decays, run products
   Gate gr;
-  gr.set_logit(a.inv_tau, T - i * C);
+  if constexpr (LOGIT) gr.set_logit(a.inv_tau, T - i * C);
   const bool weak = gr.run_swizzled(sm + L::PB_G, TOT);
   if (gr.h == 0) {
     DEC[gr.d] = gr.dec0;
@@ -1031,12 +1018,12 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   float tot_s = 0.f;
   {  // dk; per-token terms Kh Z + k dk^intra without j = r (-> w)
     const float inv = 1.f / DEC[d];
-    const size_t ob = ((size_t)bh * T + i * C + tq) * pitch_k + col_k + d0 + d;  // output index, token tq
+    __nv_bfloat16* dst = a.dk + ((size_t)bh * T + i * C + tq) * DK + d0 + d;
+    float* dst32 = FLEX ? a.acc_k + ((size_t)bh * T + i * C + tq) * DK + d0 + d : nullptr;
 #pragma unroll
     for (int rr = 0; rr < 16 / TS; ++rr) {
       const int h = tq / TS + rr;
-      float al[TS], e2[TS], ad[TS];
-      load_adds<FLEX, TS>(a.add_k, ob + (size_t)(rr * TS) * pitch_k, pitch_k, T - (i * C + tq + rr * TS), ad);
+      float al[TS], e2[TS];
 #pragma unroll
       for (int u = 0; u < TS; ++u) al[u] = ex2(raw(L::PB_G, h * TS + u, d) * kLog2e);
       float e = 1.f;  // E2 = e^{gamma - B_r}, formed as GateRun::backward forms it
@@ -1053,7 +1040,10 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
         if (!safe) w[c] *= ev * inv;
         const float qv = raw(L::PB_Q, r, d), kv = raw(L::PB_K, r, d);
         if (i * C + r < T) {
-          store_out<FLEX>(a.acc_k, a.dk, ob + (size_t)c * pitch_k, FLEX ? ev * z[c] + w[c] + ad[u] : ev * z[c] + w[c]);
+          if constexpr (FLEX)
+            dst32[(size_t)c * DK] = ev * z[c] + w[c];
+          else
+            dst[(size_t)c * DK] = __float2bfloat16_rn(ev * z[c] + w[c]);
         }
         const float kz = bf_split_sum(kv * ev) * z[c];  // Kh Z, with Kh as the S update sees it
         w[c] = kz + kv * (w[c] - DIAG[r] * qv);        // plus k dk^intra without j = r
@@ -1067,17 +1057,19 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   {  // dg = c_i + prefix (exclusive) of (Kh Z + k dk^intra) + the forward walk's part
     float pre = 0.f;
     for (int t = 0; t < qi; ++t) pre += XQ[t * KT + d];
-    const size_t ob = ((size_t)bh * T + i * C + tq) * pitch_k + col_k + d0 + d;  // output index, token tq
-    const float tau = LOGIT && a.inv_tau > 0.f ? 1.f / a.inv_tau : 0.f;
-    float ad[16];
-    load_adds<FLEX, 16>(a.add_g, ob, pitch_k, T - (i * C + tq), ad);
+    __nv_bfloat16* dst = a.dg + ((size_t)bh * T + i * C + tq) * DK + d0 + d;
+    float* dst32 = FLEX ? a.acc_g + ((size_t)bh * T + i * C + tq) * DK + d0 + d : nullptr;
+    const float tau = LOGIT ? 1.f / a.inv_tau : 0.f;
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       if (i * C + tq + c < T) {
         float dgv = ci + pre + pv[c];
         // raw logits: dx = dg sigmoid(-x) / tau, with sigmoid(-x) = 1 - e^{tau g} = -expm1(tau g)
-        if (LOGIT && a.inv_tau > 0.f) dgv *= -expm1f(tau * raw(L::PB_G, tq + c, d)) * a.inv_tau;
-        store_out<FLEX>(a.acc_g, a.dg, ob + (size_t)c * pitch_k, FLEX ? dgv + ad[c] : dgv);
+        if constexpr (LOGIT) dgv *= -expm1f(tau * raw(L::PB_G, tq + c, d)) * a.inv_tau;
+        if constexpr (FLEX)
+          dst32[(size_t)c * DK] = dgv;
+        else
+          dst[(size_t)c * DK] = __float2bfloat16_rn(dgv);
       }
       pre += w[c];
     }
@@ -1193,6 +1185,7 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
   // pitch and first column of this sub-problem's key dims and value columns in the tensors given
   const int PK = acc ? acc->pk : DK, CK = acc ? acc->ck : 0, PV = acc ? acc->pv : DV, CV = acc ? acc->cv : 0;
   if (CK < 0 || CK + DK > PK || CK % 8 || CV < 0 || CV + DV > PV || CV % 8) return cudaErrorInvalidValue;
+  if (acc && (!acc->q || !acc->k || !acc->g || (!acc->v && !dv))) return cudaErrorInvalidValue;
   BwdMaps mp;
   if (!make_map(&mp.v, v, BH, T, PV, 64, true) || !make_map(&mp.dO, dO, BH, T, PV, 64, true) ||
       !make_map(&mp.k64, k, BH, T, PK, KT, true) || !make_map(&mp.g64, g, BH, T, PK, KT, true) ||
@@ -1215,10 +1208,6 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
   a.acc_k = acc ? acc->k : nullptr;
   a.acc_g = acc ? acc->g : nullptr;
   a.acc_v = acc ? acc->v : nullptr;
-  a.add_q = acc ? acc->add_q : nullptr;
-  a.add_k = acc ? acc->add_k : nullptr;
-  a.add_g = acc ? acc->add_g : nullptr;
-  a.add_v = acc ? acc->add_v : nullptr;
   a.pk = PK;
   a.ck = CK;
   a.pv = PV;
@@ -1244,11 +1233,11 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
                                          DK, DV, a.nseg, a.seg_chunks, st_bh, st_row, st, inv_tau, CK, CV);
     if (e != cudaSuccess) return e;
   }
-  // the plain build unless the call needs offsets or partial sums (FLEX) or raw-logit gates (LOGIT,
-  // a build of its own so that the others carry none of its code)
-  if (inv_tau > 0.f) return launch_all<DK, DV, true, true>(mp, a, BH, st);
-  if (acc) return launch_all<DK, DV, true, false>(mp, a, BH, st);
-  return launch_all<DK, DV, false, false>(mp, a, BH, st);
+  // the plain build unless the call needs offsets and fp32 outputs (FLEX) or raw-logit gates (LOGIT);
+  // each build carries only its own code
+  const bool logit = inv_tau > 0.f;
+  if (acc) return logit ? launch_all<DK, DV, true, true>(mp, a, BH, st) : launch_all<DK, DV, true, false>(mp, a, BH, st);
+  return logit ? launch_all<DK, DV, false, true>(mp, a, BH, st) : launch_all<DK, DV, false, false>(mp, a, BH, st);
 }
 
 cudaError_t bwd(const void* q, const void* k, const void* v, const void* g, const float* h0, const void* dO,

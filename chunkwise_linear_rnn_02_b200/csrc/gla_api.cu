@@ -126,18 +126,18 @@ int split_fwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const 
 }
 
 struct SplitBwdWs {
-  float *aq, *ak, *ag;  // [BH*T][dk] partial key-side gradients (over value blocks)
-  float* av;            // [BH*T][dv] partial dv (over key blocks)
+  float *aq, *ak, *ag;  // [nk][nv] slices [BH*T][128]: each sub-problem's key-side gradients
+  float* av;            // [nk][nv] slices [BH*T][vb]: each sub-problem's dv (none with one key block)
   void* bws;
 };
 size_t carve_split_bwd(Carve& c, int BH, int T, int dk, int dv, SplitBwdWs* w) {
   const size_t rows = (size_t)BH * T;
   const int vb = split_vblock(dv), nv = dv / vb, nk = dk / kSplitK;
   SplitBwdWs x;
-  x.aq = nv > 1 ? c.take<float>(rows * dk) : nullptr;
-  x.ak = nv > 1 ? c.take<float>(rows * dk) : nullptr;
-  x.ag = nv > 1 ? c.take<float>(rows * dk) : nullptr;
-  x.av = nk > 1 ? c.take<float>(rows * dv) : nullptr;
+  x.aq = c.take<float>(nv * rows * dk);
+  x.ak = c.take<float>(nv * rows * dk);
+  x.ag = c.take<float>(nv * rows * dk);
+  x.av = nk > 1 ? c.take<float>(nk * rows * dv) : nullptr;
   x.bws = c.take<char>(gla::fast::bwd_workspace(BH, T, kSplitK, vb));
   if (w) *w = x;
   return c.used;
@@ -150,23 +150,26 @@ int split_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const 
   SplitBwdWs w;
   carve_split_bwd(c, BH, T, dkd, dvd, &w);
   const int vb = split_vblock(dvd), nv = dvd / vb, nk = dkd / kSplitK;
+  const long long rows = (long long)BH * T, ks = rows * kSplitK, vs = rows * vb;
   for (int kb = 0; kb < nk; ++kb) {
     const int k0 = kb * kSplitK;
     for (int vi = 0; vi < nv; ++vi) {
-      const int v0 = vi * vb;
+      const int v0 = vi * vb, s = kb * nv + vi;
       const size_t so = (size_t)k0 * dvd + v0;  // state block (k0.., v0..) of every head
-      // key-side gradients sum over the value blocks, dv over the key blocks: every sub-problem but
-      // the last of a block leaves an fp32 partial sum that the next one adds
-      const bool kpart = vi < nv - 1, kadd = vi > 0, vpart = kb < nk - 1, vadd = kb > 0;
-      const gla::fast::BwdAccum out{kpart ? w.aq : nullptr, kpart ? w.ak : nullptr, kpart ? w.ag : nullptr,
-                                    vpart ? w.av : nullptr, dkd, k0, dvd, v0,
-                                    kadd ? w.aq : nullptr, kadd ? w.ak : nullptr, kadd ? w.ag : nullptr,
-                                    vadd ? w.av : nullptr};
+      // key-side gradients sum over the value blocks, dv over the key blocks: each sub-problem writes
+      // its fp32 part into compact slices of its own (with one key block dv goes straight to bf16),
+      // and one pass per gradient sums the slices into the bf16 columns
+      const gla::fast::BwdAccum out{w.aq + s * ks, w.ak + s * ks, w.ag + s * ks, w.av ? w.av + s * vs : nullptr,
+                                    dkd, k0, dvd, v0};
       GLA_CUDA(gla::fast::bwd(q, k, v, g, h0 ? h0 + so : nullptr, dO, dhT ? dhT + so : nullptr, dq, dk, dv, dg,
                               dh0 ? dh0 + so : nullptr, BH, T, kSplitK, vb, w.bws, st, (long long)dkd * dvd, dvd, &out,
                               inv_tau));
     }
   }
+  GLA_CUDA(gla::split::sum_blocks_to_bf16(w.aq, rows, kSplitK, nk, nv, nv, 1, dq, st));
+  GLA_CUDA(gla::split::sum_blocks_to_bf16(w.ak, rows, kSplitK, nk, nv, nv, 1, dk, st));
+  GLA_CUDA(gla::split::sum_blocks_to_bf16(w.ag, rows, kSplitK, nk, nv, nv, 1, dg, st));
+  if (w.av) GLA_CUDA(gla::split::sum_blocks_to_bf16(w.av, rows, vb, nv, nk, 1, nv, dv, st));
   return GLA_OK;
 }
 

@@ -6,35 +6,6 @@ namespace gla {
 namespace split {
 namespace {
 
-__global__ void gather_kernel(const bf16* __restrict__ src, bf16* __restrict__ dst, long long rows, int pitch,
-                              int col0, int ncols) {
-  const int vpr = ncols / 8;
-  const long long n = rows * vpr;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
-    const long long r = e / vpr;
-    const int c = (int)(e % vpr) * 8;
-    *reinterpret_cast<uint4*>(dst + r * ncols + c) = *reinterpret_cast<const uint4*>(src + r * pitch + col0 + c);
-  }
-}
-
-__global__ void add_kernel(const float* __restrict__ part, float* __restrict__ acc, long long rows, int ncols,
-                           int acc_pitch, int col0) {
-  const int vpr = ncols / 4;
-  const long long n = rows * vpr;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
-    const long long r = e / vpr;
-    const int c = (int)(e % vpr) * 4;
-    const float4 u = *reinterpret_cast<const float4*>(part + r * ncols + c);
-    float4* a = reinterpret_cast<float4*>(acc + r * acc_pitch + col0 + c);
-    float4 x = *a;
-    x.x += u.x;
-    x.y += u.y;
-    x.z += u.z;
-    x.w += u.w;
-    *a = x;
-  }
-}
-
 __global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__ dst, long long n) {
   const long long nv = n / 8;
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < nv; e += (long long)gridDim.x * blockDim.x) {
@@ -42,6 +13,29 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__
     __nv_bfloat162 h[4] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w),
                            __floats2bfloat162_rn(b.x, b.y), __floats2bfloat162_rn(b.z, b.w)};
     reinterpret_cast<uint4*>(dst)[e] = *reinterpret_cast<const uint4*>(h);
+  }
+}
+
+// dst[r][c] (pitch nblocks * W) = sum over j < nparts of the slice (b * bstride + j * jstride) at
+// [r][c % W], b = c / W; slices are [rows][W] fp32, consecutive.
+__global__ void sum_blocks_kernel(const float* __restrict__ parts, long long rows, int W, int nblocks, int nparts,
+                                  int bstride, int jstride, bf16* __restrict__ dst) {
+  const int vpr = nblocks * W / 8;
+  const long long n = rows * vpr, slice = rows * W;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const long long r = e / vpr;
+    const int c = (int)(e % vpr) * 8, b = c / W, cc = c - b * W;
+    const float* src = parts + (long long)b * bstride * slice + r * W + cc;
+    float4 a = *reinterpret_cast<const float4*>(src), u = *reinterpret_cast<const float4*>(src + 4);
+    for (int j = 1; j < nparts; ++j) {
+      const float* s2 = src + (long long)j * jstride * slice;
+      const float4 x = *reinterpret_cast<const float4*>(s2), y = *reinterpret_cast<const float4*>(s2 + 4);
+      a.x += x.x, a.y += x.y, a.z += x.z, a.w += x.w;
+      u.x += y.x, u.y += y.y, u.z += y.z, u.w += y.w;
+    }
+    __nv_bfloat162 h[4] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w),
+                           __floats2bfloat162_rn(u.x, u.y), __floats2bfloat162_rn(u.z, u.w)};
+    *reinterpret_cast<uint4*>(dst + r * (nblocks * W) + c) = *reinterpret_cast<const uint4*>(h);
   }
 }
 
@@ -66,18 +60,6 @@ int grid_for(long long items) {
 
 }  // namespace
 
-cudaError_t gather_cols(const bf16* src, bf16* dst, long long rows, int pitch, int col0, int ncols,
-                        cudaStream_t st) {
-  gather_kernel<<<grid_for(rows * (ncols / 8)), 256, 0, st>>>(src, dst, rows, pitch, col0, ncols);
-  return cudaGetLastError();
-}
-
-cudaError_t add_cols(const float* part, float* acc, long long rows, int ncols, int acc_pitch, int col0,
-                     cudaStream_t st) {
-  add_kernel<<<grid_for(rows * (ncols / 4)), 256, 0, st>>>(part, acc, rows, ncols, acc_pitch, col0);
-  return cudaGetLastError();
-}
-
 cudaError_t copy_cols(const bf16* src, long long src_pitch, bf16* dst, long long dst_pitch, long long rows,
                       long long ncols, long long dst_cols, cudaStream_t st) {
   copy_kernel<bf16><<<grid_for(rows * (dst_cols / 8)), 256, 0, st>>>(src, src_pitch, dst, dst_pitch, rows, ncols,
@@ -89,6 +71,14 @@ cudaError_t copy_cols(const float* src, long long src_pitch, float* dst, long lo
                       long long ncols, long long dst_cols, cudaStream_t st) {
   copy_kernel<float><<<grid_for(rows * (dst_cols / 4)), 256, 0, st>>>(src, src_pitch, dst, dst_pitch, rows, ncols,
                                                                       dst_cols);
+  return cudaGetLastError();
+}
+
+cudaError_t sum_blocks_to_bf16(const float* parts, long long rows, int W, int nblocks, int nparts, int bstride,
+                               int jstride, bf16* dst, cudaStream_t st) {
+  if (W % 8 || nblocks < 1 || nparts < 1) return cudaErrorInvalidValue;
+  sum_blocks_kernel<<<grid_for(rows * (nblocks * W / 8)), 256, 0, st>>>(parts, rows, W, nblocks, nparts, bstride,
+                                                                         jstride, dst);
   return cudaGetLastError();
 }
 
