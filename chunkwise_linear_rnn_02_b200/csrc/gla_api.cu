@@ -5,6 +5,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "../../include/gla.h"
 #include "common.cuh"
 #include "fast_path.cuh"
@@ -125,10 +127,36 @@ int split_fwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const 
   return GLA_OK;
 }
 
+// A second stream per device, with fork / join events, for sub-problems that need not run after one
+// another; made on first use.  Its mutex is held while a call enqueues its work there, so that the
+// event records and waits of concurrent callers do not interleave.
+struct SideStream {
+  cudaStream_t s;
+  cudaEvent_t fork, join;
+  std::mutex mu;
+};
+int side_stream(SideStream** out) {
+  static std::mutex make_mu;
+  static SideStream per_dev[64];
+  static bool made[64];
+  int dev = 0;
+  GLA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return GLA_ERR_CUDA;
+  std::lock_guard<std::mutex> g(make_mu);
+  if (!made[dev]) {
+    GLA_CUDA(cudaStreamCreateWithFlags(&per_dev[dev].s, cudaStreamNonBlocking));
+    GLA_CUDA(cudaEventCreateWithFlags(&per_dev[dev].fork, cudaEventDisableTiming));
+    GLA_CUDA(cudaEventCreateWithFlags(&per_dev[dev].join, cudaEventDisableTiming));
+    made[dev] = true;
+  }
+  *out = &per_dev[dev];
+  return GLA_OK;
+}
+
 struct SplitBwdWs {
   float *aq, *ak, *ag;  // [nk][nv] slices [BH*T][128]: each sub-problem's key-side gradients
   float* av;            // [nk][nv] slices [BH*T][vb]: each sub-problem's dv (none with one key block)
-  void* bws;
+  void* bws[2];         // the fused kernels' workspace, one per stream
 };
 size_t carve_split_bwd(Carve& c, int BH, int T, int dk, int dv, SplitBwdWs* w) {
   const size_t rows = (size_t)BH * T;
@@ -138,7 +166,7 @@ size_t carve_split_bwd(Carve& c, int BH, int T, int dk, int dv, SplitBwdWs* w) {
   x.ak = c.take<float>(nv * rows * dk);
   x.ag = c.take<float>(nv * rows * dk);
   x.av = nk > 1 ? c.take<float>(nk * rows * dv) : nullptr;
-  x.bws = c.take<char>(gla::fast::bwd_workspace(BH, T, kSplitK, vb));
+  for (int j = 0; j < 2; ++j) x.bws[j] = c.take<char>(gla::fast::bwd_workspace(BH, T, kSplitK, vb));
   if (w) *w = x;
   return c.used;
 }
@@ -151,6 +179,14 @@ int split_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const 
   carve_split_bwd(c, BH, T, dkd, dvd, &w);
   const int vb = split_vblock(dvd), nv = dvd / vb, nk = dkd / kSplitK;
   const long long rows = (long long)BH * T, ks = rows * kSplitK, vs = rows * vb;
+  // The sub-problems write disjoint slices, so they run on two streams (the caller's and a side
+  // stream): the CTAs of one sub-problem's chunk-parallel launch fill the SMs that the other's
+  // walks leave idle.
+  SideStream* side = nullptr;
+  GLA_TRY(side_stream(&side));
+  std::lock_guard<std::mutex> lock(side->mu);
+  GLA_CUDA(cudaEventRecord(side->fork, st));
+  GLA_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
   for (int kb = 0; kb < nk; ++kb) {
     const int k0 = kb * kSplitK;
     for (int vi = 0; vi < nv; ++vi) {
@@ -162,10 +198,12 @@ int split_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const 
       const gla::fast::BwdAccum out{w.aq + s * ks, w.ak + s * ks, w.ag + s * ks, w.av ? w.av + s * vs : nullptr,
                                     dkd, k0, dvd, v0};
       GLA_CUDA(gla::fast::bwd(q, k, v, g, h0 ? h0 + so : nullptr, dO, dhT ? dhT + so : nullptr, dq, dk, dv, dg,
-                              dh0 ? dh0 + so : nullptr, BH, T, kSplitK, vb, w.bws, st, (long long)dkd * dvd, dvd, &out,
-                              inv_tau));
+                              dh0 ? dh0 + so : nullptr, BH, T, kSplitK, vb, w.bws[s & 1], s & 1 ? side->s : st,
+                              (long long)dkd * dvd, dvd, &out, inv_tau));
     }
   }
+  GLA_CUDA(cudaEventRecord(side->join, side->s));
+  GLA_CUDA(cudaStreamWaitEvent(st, side->join, 0));
   GLA_CUDA(gla::split::sum_blocks_to_bf16(w.aq, rows, kSplitK, nk, nv, nv, 1, dq, st));
   GLA_CUDA(gla::split::sum_blocks_to_bf16(w.ak, rows, kSplitK, nk, nv, nv, 1, dk, st));
   GLA_CUDA(gla::split::sum_blocks_to_bf16(w.ag, rows, kSplitK, nk, nv, nv, 1, dg, st));
