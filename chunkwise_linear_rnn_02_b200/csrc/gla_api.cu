@@ -471,20 +471,29 @@ int gsa_bwd_fused(const bf16* q, const bf16* k, const bf16* v, const bf16* phi, 
     GLA_CUDA(gla::split::copy_cols(w.h0t, s1t, w.h0p + s1t, s1p, BH, s1t, s1t, st));
   }
   if (dhT1) GLA_CUDA(gla::gsa::transpose_states(dhT1, s1, w.dhTp, BH, dkd, m, 128, st));
-  const gla::fast::BwdAccum acc1{w.dq1, w.dphi1, w.dg1, nullptr, 128, 0, dkd, 0};  // dk (its dv) straight to bf16
-  GLA_CUDA(gla::fast::bwd(w.do1, f.phi, k, f.g, h01 ? w.h0p : nullptr, q, dhT1 ? w.dhTp : nullptr, nullptr, nullptr,
-                          dk, nullptr, dh01 ? w.dh0p : nullptr, BH, T, 128, dkd, f.ws, st, -1, -1, &acc1));
+  // From here the pass-1 backward (caller's stream) and the dq forwards (side stream) read only do1
+  // and the inputs, and write disjoint outputs, so they run side by side.
+  SideStream* side = nullptr;
+  GLA_TRY(side_stream(&side));
+  std::lock_guard<std::mutex> lock(side->mu);
+  GLA_CUDA(cudaEventRecord(side->fork, st));
+  GLA_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
   // dq = S1 do1: the output of the GLA with queries do1, keys phi, values k from h0_1^T, as two
   // d_k = 64 forwards over the queries' hi and lo halves (the second adds the first's partial), with
   // the decayed keys as bf16 hi + lo pairs (a single bf16 put dq 2 % off in the emulation)
-  GLA_CUDA(gla::fast::fwd(w.do1, f.phi, k, f.g, h01 ? w.h0t : nullptr, nullptr, nullptr, BH, T, m, dkd, w.fws, st, -1,
-                          -1, w.dqp, 0.f, 128, 0, nullptr, true));
-  GLA_CUDA(gla::fast::fwd(w.do1, f.phi, k, f.g, h01 ? w.h0t : nullptr, dq, nullptr, BH, T, m, dkd, w.fws, st, -1, -1,
-                          nullptr, 0.f, 128, m, w.dqp, true));
+  GLA_CUDA(gla::fast::fwd(w.do1, f.phi, k, f.g, h01 ? w.h0t : nullptr, nullptr, nullptr, BH, T, m, dkd, w.fws, side->s,
+                          -1, -1, w.dqp, 0.f, 128, 0, nullptr, true));
+  GLA_CUDA(gla::fast::fwd(w.do1, f.phi, k, f.g, h01 ? w.h0t : nullptr, dq, nullptr, BH, T, m, dkd, w.fws, side->s, -1,
+                          -1, nullptr, 0.f, 128, m, w.dqp, true));
+  GLA_CUDA(cudaEventRecord(side->join, side->s));
+  const gla::fast::BwdAccum acc1{w.dq1, w.dphi1, w.dg1, nullptr, 128, 0, dkd, 0};  // dk (its dv) straight to bf16
+  GLA_CUDA(gla::fast::bwd(w.do1, f.phi, k, f.g, h01 ? w.h0p : nullptr, q, dhT1 ? w.dhTp : nullptr, nullptr, nullptr,
+                          dk, nullptr, dh01 ? w.dh0p : nullptr, BH, T, 128, dkd, f.ws, st, -1, -1, &acc1));
   // both passes' and both copies' contributions to dphi and dg; dh0_1 back to [dk][m]
   GLA_CUDA(gla::gsa::fold_add_bf16(w.dphi1, f.dk, dphi, rows, m, st));
   GLA_CUDA(gla::gsa::fold_add_bf16(w.dg1, f.dg, dg, rows, m, st));
   if (dh01) GLA_CUDA(gla::gsa::transpose_states(w.dh0p, s1p, dh01, BH, m, dkd, dkd, st, true));
+  GLA_CUDA(cudaStreamWaitEvent(st, side->join, 0));
   return GLA_OK;
 }
 
