@@ -498,7 +498,8 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   uint64_t* bar_dv = bars + 1;  // dO, v of a chunk
   uint64_t* bar_m1 = bars + 3;
   uint64_t* bar_m2 = bars + 4;
-  uint32_t ph_ld = 0, ph_dv = 0, ph_m1 = 0, ph_m2 = 0;
+  uint64_t* bar_mA = bars + 5;  // first part of group 1: Z^T and A
+  uint32_t ph_ld = 0, ph_dv = 0, ph_m1 = 0, ph_m2 = 0, ph_mA = 0;
   float* DEC = reinterpret_cast<float*>(sm + L::DEC);
   float* TOT = reinterpret_cast<float*>(sm + L::TOT);
 
@@ -598,6 +599,16 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       constexpr uint32_t id_A = idesc_bf16_f32(C, C, false, false);
       constexpr uint32_t id_dv = idesc_bf16_f32(VT, C, true, false);  // dv^T = G^T Kh^T: value columns on M
       constexpr uint32_t id_G = idesc_bf16_f32(DK, VT, true, true);
+      // Z^T part of this value tile: G_{i+1}[:, tile] V[:, tile]^T (G copy hi + lo); first, since the
+      // v tile shares A's space, which the A epilogue overwrites after the first commit
+      constexpr uint32_t id_Z = idesc_bf16_f32(DK, C, false, false);
+#pragma unroll
+      for (int k = 0; k < VT / 16; ++k) {
+        const uint32_t ko = (k >> 2) * (DK * 128) + (k & 3) * 32;
+        const uint64_t vd = desc_sw128(base + L::VZ + (k >> 2) * (C * 128) + (k & 3) * 32, 16, 1024);
+        umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_HI + ko, 16, 1024), vd, id_Z, k > 0);
+        umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_LO + ko, 16, 1024), vd, id_Z, 1);
+      }
 #pragma unroll
       for (int k = 0; k < DK / 16; ++k) {
         const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
@@ -606,6 +617,13 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         umma_bf16(tmem + L::T_A, qh, kh, id_A, k > 0);
         umma_bf16(tmem + L::T_A, qh, kl, id_A, 1);
         umma_bf16(tmem + L::T_A, ql, kh, id_A, 1);
+      }
+      umma_commit(bar_mA);
+      // dv^T = G^T Kh^T and the G update: the A epilogue runs while they execute
+#pragma unroll
+      for (int k = 0; k < DK / 16; ++k) {
+        const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
+        const uint64_t kh = desc_sw128(base + L::KH_HI + ko, 16, 1024), kl = desc_sw128(base + L::KH_LO + ko, 16, 1024);
         const uint64_t gh = desc_sw128(base + L::GC_HI + k * 2048, DK * 128, 1024);
         umma_bf16(tmem + L::T_DV, gh, kh, id_dv, k > 0);
         umma_bf16(tmem + L::T_DV, desc_sw128(base + L::GC_LO + k * 2048, DK * 128, 1024), kh, id_dv, 1);
@@ -617,21 +635,16 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         umma_bf16(tmem + L::T_G, desc_sw128(base + L::QP_HI + k * 2048, C * 128, 1024), dd, id_G, 1);
         umma_bf16(tmem + L::T_G, desc_sw128(base + L::QP_LO + k * 2048, C * 128, 1024), dd, id_G, 1);
       }
-      // Z^T part of this value tile: G_{i+1}[:, tile] V[:, tile]^T (G copy hi + lo)
-      constexpr uint32_t id_Z = idesc_bf16_f32(DK, C, false, false);
-#pragma unroll
-      for (int k = 0; k < VT / 16; ++k) {
-        const uint32_t ko = (k >> 2) * (DK * 128) + (k & 3) * 32;
-        const uint64_t vd = desc_sw128(base + L::VZ + (k >> 2) * (C * 128) + (k & 3) * 32, 16, 1024);
-        umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_HI + ko, 16, 1024), vd, id_Z, k > 0);
-        umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_LO + ko, 16, 1024), vd, id_Z, 1);
-      }
       umma_commit(bar_m1);
       if (!safe && n + 1 < nl) load_qkg(i - 1);
     }
     __syncwarp();
-    mbar_wait(bar_m1, ph_m1, a.latch);
-    ph_m1 ^= 1;
+    mbar_wait(bar_mA, ph_mA, a.latch);
+    ph_mA ^= 1;
+    if (safe) {  // the exact path overwrites Qs / Kh, which the rest of group 1 reads
+      mbar_wait(bar_m1, ph_m1, a.latch);
+      ph_m1 ^= 1;
+    }
     tc_fence_after();
     // this tile's part of Z^T for chunk i: row grow of the M=128 accumulator, 32 tokens
     auto z_epilogue = [&]() {
@@ -704,8 +717,14 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       }
       umma_commit(bar_m2);
     }
-    // while the second group runs: the Z^T epilogue and the G pass (neither touches A, dO or dv)
-    if (!safe) z_epilogue();
+    // while the rest of group 1 and the second group run: the Z^T epilogue; then (group 1 complete)
+    // the G pass (neither touches A, dO or dv)
+    if (!safe) {
+      z_epilogue();
+      mbar_wait(bar_m1, ph_m1, a.latch);
+      ph_m1 ^= 1;
+      tc_fence_after();
+    }
     {  // G_i = dec * G (chunks off the exact path, whose rescale came first) and its hi / lo copy
       const float sc = safe ? 1.f : DEC[grow];
       float v[64];
@@ -1092,7 +1111,7 @@ struct BwdSmem {
 template <int DK, int DV, bool FLEX, bool LOGIT>
 __global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bars[5];
+  __shared__ uint64_t bars[6];
   __shared__ uint32_t tmem_base_sh;
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -1102,7 +1121,7 @@ __global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant_
     tmem_relinquish();
   }
   if (threadIdx.x == 0) {
-    for (int b = 0; b < 5; ++b) mbar_init(&bars[b], 1);
+    for (int b = 0; b < 6; ++b) mbar_init(&bars[b], 1);
     fence_mbar_init();
   }
   tc_fence_before();

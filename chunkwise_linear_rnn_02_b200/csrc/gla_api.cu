@@ -180,11 +180,15 @@ int split_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const 
   const int vb = split_vblock(dvd), nv = dvd / vb, nk = dkd / kSplitK;
   const long long rows = (long long)BH * T, ks = rows * kSplitK, vs = rows * vb;
   // The sub-problems write disjoint slices, so they run on two streams (the caller's and a side
-  // stream): the CTAs of one sub-problem's chunk-parallel launch fill the SMs that the other's
-  // walks leave idle.
+  // stream, sub-problem s on stream s & 1): the CTAs of one sub-problem's chunk-parallel launch fill
+  // the SMs that the other's walks leave idle.  Each summing pass is enqueued as soon as its slices
+  // are: a key block's after its last sub-problem (waiting for the other stream's part of the block),
+  // a value block's at the end of the stream that ran all its sub-problems (nv even) or after the
+  // join.
   SideStream* side = nullptr;
   GLA_TRY(side_stream(&side));
   std::lock_guard<std::mutex> lock(side->mu);
+  cudaStream_t sts[2] = {st, side->s};
   GLA_CUDA(cudaEventRecord(side->fork, st));
   GLA_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
   for (int kb = 0; kb < nk; ++kb) {
@@ -194,20 +198,34 @@ int split_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const 
       const size_t so = (size_t)k0 * dvd + v0;  // state block (k0.., v0..) of every head
       // key-side gradients sum over the value blocks, dv over the key blocks: each sub-problem writes
       // its fp32 part into compact slices of its own (with one key block dv goes straight to bf16),
-      // and one pass per gradient sums the slices into the bf16 columns
+      // and the summing passes add the slices into the bf16 columns
       const gla::fast::BwdAccum out{w.aq + s * ks, w.ak + s * ks, w.ag + s * ks, w.av ? w.av + s * vs : nullptr,
                                     dkd, k0, dvd, v0};
       GLA_CUDA(gla::fast::bwd(q, k, v, g, h0 ? h0 + so : nullptr, dO, dhT ? dhT + so : nullptr, dq, dk, dv, dg,
-                              dh0 ? dh0 + so : nullptr, BH, T, kSplitK, vb, w.bws[s & 1], s & 1 ? side->s : st,
+                              dh0 ? dh0 + so : nullptr, BH, T, kSplitK, vb, w.bws[s & 1], sts[s & 1],
                               (long long)dkd * dvd, dvd, &out, inv_tau));
     }
+    // key block kb is complete once both streams are past its sub-problems
+    const int last = (kb * nv + nv - 1) & 1;
+    cudaStream_t ks_st = sts[last];
+    if (nv > 1) {
+      GLA_CUDA(cudaEventRecord(side->join, sts[last ^ 1]));
+      GLA_CUDA(cudaStreamWaitEvent(ks_st, side->join, 0));
+    }
+    const float* base[3] = {w.aq, w.ak, w.ag};
+    bf16* outs[3] = {dq, dk, dg};
+    for (int j = 0; j < 3; ++j)
+      GLA_CUDA(gla::split::sum_blocks_to_bf16(base[j] + (size_t)kb * nv * ks, rows, kSplitK, 1, nv, 0, 1,
+                                              outs[j] + k0, dkd, ks_st));
+  }
+  if (w.av && nv % 2 == 0) {  // value block vi ran on stream vi & 1 for every key block
+    for (int vi = 0; vi < nv; ++vi)
+      GLA_CUDA(gla::split::sum_blocks_to_bf16(w.av + (size_t)vi * vs, rows, vb, 1, nk, 0, nv, dv + vi * vb, dvd,
+                                              sts[vi & 1]));
   }
   GLA_CUDA(cudaEventRecord(side->join, side->s));
   GLA_CUDA(cudaStreamWaitEvent(st, side->join, 0));
-  GLA_CUDA(gla::split::sum_blocks_to_bf16(w.aq, rows, kSplitK, nk, nv, nv, 1, dq, st));
-  GLA_CUDA(gla::split::sum_blocks_to_bf16(w.ak, rows, kSplitK, nk, nv, nv, 1, dk, st));
-  GLA_CUDA(gla::split::sum_blocks_to_bf16(w.ag, rows, kSplitK, nk, nv, nv, 1, dg, st));
-  if (w.av) GLA_CUDA(gla::split::sum_blocks_to_bf16(w.av, rows, vb, nv, nk, 1, nv, dv, st));
+  if (w.av && nv % 2 != 0) GLA_CUDA(gla::split::sum_blocks_to_bf16(w.av, rows, vb, nv, nk, 1, nv, dv, dvd, st));
   return GLA_OK;
 }
 

@@ -16,10 +16,10 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__
   }
 }
 
-// dst[r][c] (pitch nblocks * W) = sum over j < nparts of the slice (b * bstride + j * jstride) at
-// [r][c % W], b = c / W; slices are [rows][W] fp32, consecutive.
+// dst[r][col0 + c] (row pitch dst_pitch), c < nblocks * W, = sum over j < nparts of the slice
+// (b * bstride + j * jstride) at [r][c % W], b = c / W; slices are [rows][W] fp32, consecutive.
 __global__ void sum_blocks_kernel(const float* __restrict__ parts, long long rows, int W, int nblocks, int nparts,
-                                  int bstride, int jstride, bf16* __restrict__ dst) {
+                                  int bstride, int jstride, bf16* __restrict__ dst, long long dst_pitch) {
   const int vpr = nblocks * W / 8;
   const long long n = rows * vpr, slice = rows * W;
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
@@ -35,7 +35,7 @@ __global__ void sum_blocks_kernel(const float* __restrict__ parts, long long row
     }
     __nv_bfloat162 h[4] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w),
                            __floats2bfloat162_rn(u.x, u.y), __floats2bfloat162_rn(u.z, u.w)};
-    *reinterpret_cast<uint4*>(dst + r * (nblocks * W) + c) = *reinterpret_cast<const uint4*>(h);
+    *reinterpret_cast<uint4*>(dst + r * dst_pitch + c) = *reinterpret_cast<const uint4*>(h);
   }
 }
 
@@ -75,10 +75,11 @@ cudaError_t copy_cols(const float* src, long long src_pitch, float* dst, long lo
 }
 
 cudaError_t sum_blocks_to_bf16(const float* parts, long long rows, int W, int nblocks, int nparts, int bstride,
-                               int jstride, bf16* dst, cudaStream_t st) {
-  if (W % 8 || nblocks < 1 || nparts < 1) return cudaErrorInvalidValue;
+                               int jstride, bf16* dst, long long dst_pitch, cudaStream_t st) {
+  if (W % 8 || dst_pitch % 8 || nblocks < 1 || nparts < 1 || (long long)nblocks * W > dst_pitch)
+    return cudaErrorInvalidValue;
   sum_blocks_kernel<<<grid_for(rows * (nblocks * W / 8)), 256, 0, st>>>(parts, rows, W, nblocks, nparts, bstride,
-                                                                         jstride, dst);
+                                                                         jstride, dst, dst_pitch);
   return cudaGetLastError();
 }
 
