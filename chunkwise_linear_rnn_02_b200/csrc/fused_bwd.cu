@@ -41,7 +41,12 @@ namespace fast {
 
 using namespace sm100;
 
-constexpr int BT = 256;  // threads per CTA: warps w and w+4 share TMEM lanes and split columns
+constexpr int BT = 256;  // compute threads per CTA: warps w and w+4 share TMEM lanes and split columns
+// The walk kernel adds a ninth warp that issues the MMAs: tcgen05.mma issue holds the issuing thread
+// for the group's execution, so the compute warps only hand over (named barriers kBarH1 / kBarH2:
+// the compute threads arrive, the producer warp syncs) and wait for the groups' mbarriers.
+constexpr int BTP = BT + 32;
+constexpr int kBarH1 = 2, kBarH2 = 3;
 constexpr int KT = 64;   // key dimensions per key-tile CTA
 constexpr int VT = 128;  // value columns per value-tile CTA
 
@@ -58,10 +63,10 @@ struct BwdArgs {
   float* dh0;
   float* ws_qx;    // [BH][NC][DK] chunk sums of Qt X
   float* ws_carry; // [BH][nseg][DK] rowsum(G_end * S_end) per segment: where the dg carry starts
-  float* ws_z;     // [BH][DV/VT][NC][DK][64] value tiles' parts of Z^T
+  float* ws_z;     // [BH][DV/VT][NC][64][DK] value tiles' parts of Z (token rows of DK dims)
   float* ws_kz;    // [BH][DV/VT][NC][2][DK] value tiles' parts of the chunk sums of Kh Z (per token half)
   float* ws_c;     // [BH][NC][DK] the dg carry c_i of every chunk
-  float* ws_part;  // [BH][NC][DK][64] forward-walk part of dg, one row of 64 tokens per chunk and dim
+  float* ws_part;  // [BH][NC][64][DK] forward-walk part of dg, one row of DK dims per token
   int T;
   // Sequence split: nseg segments of seg_chunks chunks; s_in / g_end hold the segment states
   // ([BH][nseg][DK][DV] fp32: s_in[s-1] enters segment s, g_end[s] = dL/dS at the end of s).
@@ -138,7 +143,7 @@ struct KeyLayout {
 // run, multiplying in the same order, so its values equal the ones behind the MMA operands.
 template <int DK, int DV, bool FLEX, bool LOGIT>
 __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int tau, int seg,
-                              uint64_t* bars, uint32_t tmem) {
+                              uint64_t* bars, uint32_t tmem, int* safe_flag) {
   using L = KeyLayout<DK, DV>;
   using Gate = GateRun<KT, BT, LOGIT>;
   constexpr int NS = L::NS, TS = Gate::TS;
@@ -165,7 +170,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   float2* XCH = reinterpret_cast<float2*>(sm + L::XCH);
   float* DIAG = reinterpret_cast<float*>(sm + L::DIAG);
   float* qx_sums = a.ws_qx + (size_t)bh * NC * DK + d0;          // [NC][DK] slice of this head and key tile
-  float* part = a.ws_part + ((size_t)bh * NC * DK + d0) * C;  // [NC][DK][64] slice: forward-walk part of dg
+  float* part = a.ws_part + (size_t)bh * NC * C * DK + d0;  // [NC][64][DK] slice: forward-walk part of dg
 
   auto pbo = [&](int b) { return L::PB + (uint32_t)b * L::PB_STAGE; };
   auto load_a = [&](int chunk) {
@@ -186,10 +191,11 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     mbar_wait(bar_pb + b, (ph_pb >> b) & 1u, a.latch);
     ph_pb ^= 1u << b;
   };
-  auto sync_tc = [&]() {
+  // operands in shared memory / TMEM are complete: hand them to the producer warp
+  auto handoff = [&](int id) {
+    fence_async_smem();
     tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+    bar_arrive(id, BTP);
   };
   // Element (token j, dim d) of a raw tile at shared-memory offset off (TMA 128-byte swizzle).
   auto raw = [&](uint32_t off, int j, int d) { return bf2f(sm + off + sw128(j, d)); };
@@ -203,7 +209,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       DEC[b * KT + gr.d] = gr.dec0;
       DEC[b * KT + gr.d + 1] = gr.dec1;
     }
-    return __syncthreads_or(weak);
+    return bar_or(kBarCompute, BT, weak);
   };
   auto write_kq = [&](uint32_t w, int j, int d, float e0, float e1) {
     uint32_t hi, lo;
@@ -254,9 +260,8 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       store_half_split(sm + L::DA_HI, sm + L::DA_LO, row, v, half);
     }
   };
-  // MMA group 1: dA = dO V^T, X^T = S dO^T and the state update S += Kh^T V.
+  // MMA group 1 (producer lane 0): dA = dO V^T, X^T = S dO^T and the state update S += Kh^T V.
   auto issue_m1 = [&]() {
-    if (tid != 0) return;
     mbar_wait(bar_pa, ph_pa, a.latch);
     ph_pa ^= 1;
     tc_fence_after();
@@ -280,9 +285,8 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     }
     umma_commit(bar_m1);
   };
-  // MMA group 2: Y^T = Kh^T dA^T.
+  // MMA group 2 (producer lane 0): Y^T = Kh^T dA^T.
   auto issue_m2 = [&]() {
-    if (tid != 0) return;
     constexpr uint32_t id_Y = idesc_bf16_f32(KT, C, true, false);
 #pragma unroll
     for (int k = 0; k < C / 16; ++k) {
@@ -301,8 +305,9 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     ph_m2 ^= 1;
     tc_fence_after();
   };
-  // Chunk i+1: gate run from buffer nb, Kh operand, state copy + rescale, group 1.  The operand
-  // area KQ is free once group 2 of the current chunk has completed.
+  // Chunk i+1: gate run from buffer nb, Kh operand, state copy + rescale, then group 1 (handed to
+  // the producer with the chunk's exact-path flag).  The operand area KQ is free once group 2 of
+  // the current chunk has completed.
   auto prepare = [&](int nb, int m2_pending, int chunk) {
     wait_b(nb);
     Gate gr;
@@ -312,11 +317,31 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     if (m2_pending) wait_m2();
     gr.backward([&](int j, float e0, float e1) { write_kq(w[j - gr.h * Gate::TS], j, gr.d, e0, e1); });
     state_pass(nb);
-    fence_async_smem();
-    sync_tc();
-    issue_m1();
+    if (tid == 0) safe_flag[nb] = safe;
+    handoff(kBarH1);
     return safe;
   };
+
+  if (tid >= BT) {  // ======== producer warp: the MMA groups, in the order the compute threads hand over
+    bar_sync(kBarH1, BTP);
+    tc_fence_after();
+    if (lane == 0) issue_m1();
+    __syncwarp();
+    for (int i = ch0; i < ch1; ++i) {
+      const int b = (i - ch0) & 1;
+      bar_sync(kBarH2, BTP);  // chunk i's dA operand is in shared memory
+      tc_fence_after();
+      if (lane == 0 && !safe_flag[b]) issue_m2();
+      __syncwarp();
+      if (i + 1 < ch1) {
+        bar_sync(kBarH1, BTP);  // chunk i+1's Kh and state copy are in shared memory
+        tc_fence_after();
+        if (lane == 0) issue_m1();
+        __syncwarp();
+      }
+    }
+    return;
+  }
 
   // ================================ forward walk: dq, first part of dg ================================
   if (tid == 0) {
@@ -338,47 +363,64 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     float x[32];  // this thread's row of X^T: key dim d = row, tokens tb .. tb+31
     tmem_ld32(tmem + L::T_X + lane_off + tb, x);
     dA_epilogue();
-    fence_async_smem();
-    sync_tc();
-    if (!safe) issue_m2();
-    if (i + 1 < ch1)
+    handoff(kBarH2);  // group 2 (chunk off the exact path)
+    // dA and DIAG of every thread are read below: the gate run's barrier in prepare orders them, or
+    // this one after the last chunk
+    if (i + 1 < ch1) {
       safe_next = prepare(b ^ 1, !safe, i + 1);
-    else if (!safe)
-      wait_m2();
+    } else {
+      bar_sync(kBarCompute, BT);
+      if (!safe) wait_m2();
+    }
     float y[32];  // this thread's row of Y^T
     if (!safe) {
       tmem_ld32(tmem + L::T_Y + lane_off + tb, y);
       tmem_ld_wait();
     }
+    // The M = 64 accumulators sit in TMEM lanes 0-15 of each quarter.  Split the row's 32 tokens
+    // over the warp: lane l < 16 keeps tokens tb .. tb+15 of key dim q4*16 + l, lane l + 16 takes
+    // tokens tb+16 .. tb+31 of the same dim (by shuffle), so that every lane works on 16 tokens.
+    const int sub = lane >> 4, tq = tb + sub * 16, d = q4 * 16 + (lane & 15);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const float xv = __shfl_sync(0xffffffffu, x[16 + c], lane & 15);
+      if (sub) x[c] = xv;
+    }
+    if (!safe) {  // (on the exact path y is formed below, per token)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float yv = __shfl_sync(0xffffffffu, y[16 + c], lane & 15);
+        if (sub) y[c] = yv;
+      }
+    }
     float tot_s = 0.f, tot_e = 0.f;
-    if (row_owner) {  // dq; per-token terms Qt X (-> x) and q dq^intra without j = r (-> y)
-      const int d = row;
+    {  // dq; per-token terms Qt X (-> x) and q dq^intra without j = r (-> y)
       const uint32_t pk = pbo(b) + L::PB_K, pg = pbo(b) + L::PB_G, pq = pbo(b) + L::PB_Q;
       const float* tot = TOT + b * NS * KT;
       if (safe) {  // exact intra term y_j = sum_{r<=j} dA_jr k_r e^{B_j - B_r}
         float bj = 0.f;
-        for (int t = 0; t < tb; ++t) bj += raw(pg, t, d);
+        for (int t = 0; t < tq; ++t) bj += raw(pg, t, d);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          bj += raw(pg, tb + c, d);
+        for (int c = 0; c < 16; ++c) {
+          bj += raw(pg, tq + c, d);
           float acc = 0.f, br = 0.f;
-          for (int r = 0; r <= tb + c; ++r) {
+          for (int r = 0; r <= tq + c; ++r) {
             br += raw(pg, r, d);
-            acc += dA_at(tb + c, r) * raw(pk, r, d) * __expf(bj - br);
+            acc += dA_at(tq + c, r) * raw(pk, r, d) * __expf(bj - br);
           }
           y[c] = acc;
         }
       }
       const float inv = 1.f / DEC[b * KT + d];
-      __nv_bfloat16* dst = a.dq + ((size_t)bh * T + i * C + tb) * DK + d0 + d;
-      float* dst32 = FLEX ? a.acc_q + ((size_t)bh * T + i * C + tb) * DK + d0 + d : nullptr;
+      __nv_bfloat16* dst = a.dq + ((size_t)bh * T + i * C + tq) * DK + d0 + d;
+      float* dst32 = FLEX ? a.acc_q + ((size_t)bh * T + i * C + tq) * DK + d0 + d : nullptr;
 #pragma unroll
-      for (int rr = 0; rr < 4; ++rr) {
+      for (int rr = 0; rr < 16 / TS; ++rr) {
         float e = 1.f;  // E1 = e^{B_j}, formed as GateRun::forward forms it
-        for (int hh = 0; hh < half * 4 + rr; ++hh) e *= tot[hh * KT + d];
+        for (int hh = 0; hh < tq / TS + rr; ++hh) e *= tot[hh * KT + d];
 #pragma unroll
         for (int u = 0; u < TS; ++u) {
-          const int c = rr * TS + u, j = tb + c;
+          const int c = rr * TS + u, j = tq + c;
           e *= ex2(raw(pg, j, d) * kLog2e);
           if (!safe) y[c] *= e * inv;
           const float qv = raw(pq, j, d), kv = raw(pk, j, d);
@@ -394,28 +436,31 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
           tot_e += y[c];
         }
       }
-      XCH[half * KT + d] = make_float2(tot_s, tot_e);
     }
-    __syncthreads();
+    // sums over the other 16 tokens of this half (the partner lane) and over the other half (XCH)
+    const float part_s = __shfl_xor_sync(0xffffffffu, tot_s, 16), part_e = __shfl_xor_sync(0xffffffffu, tot_e, 16);
+    if (!sub) XCH[half * KT + d] = make_float2(tot_s + part_s, tot_e + part_e);
+    bar_sync(kBarCompute, BT);
     if (tid == 0 && i + 2 < ch1) load_b(i + 2, b);
-    if (row_owner) {  // part = suffix (inclusive) of Qt X minus prefix (exclusive) of q dq^intra
-      const int d = row;
+    {  // part = suffix (inclusive) of Qt X minus prefix (exclusive) of q dq^intra
       const float2 o = XCH[(half ^ 1) * KT + d];
-      float suf = half == 0 ? o.x : 0.f, pre = half == 1 ? o.y : 0.f;
+      float suf = (half == 0 ? o.x : 0.f) + (sub == 0 ? part_s : 0.f);
+      float pre = (half == 1 ? o.y : 0.f) + (sub == 1 ? part_e : 0.f);
 #pragma unroll
-      for (int c = 31; c >= 0; --c) {
+      for (int c = 15; c >= 0; --c) {
         suf += x[c];
         x[c] = suf;
       }
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < 16; ++c) {
         x[c] -= pre;
         pre += y[c];
       }
-      float4* dst = reinterpret_cast<float4*>(part + ((size_t)i * DK + d) * C + tb);
+      // token-major rows: the lanes (consecutive dims) store adjacent words
+      float* dst = part + ((size_t)i * C + tq) * DK + d;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
-      if (half == 0) qx_sums[(size_t)i * DK + d] = suf;
+      for (int c = 0; c < 16; ++c) dst[(size_t)c * DK] = x[c];
+      if (half == 0 && sub == 0) qx_sums[(size_t)i * DK + d] = suf;
     }
   }
 
@@ -439,7 +484,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       }
     }
     if (row_owner) CARRYP[half * KT + row] = acc;
-    __syncthreads();
+    bar_sync(kBarCompute, BT);
     if (tid < KT) a.ws_carry[((size_t)bh * a.nseg + seg) * DK + d0 + tid] = CARRYP[tid] + CARRYP[KT + tid];
   }
 }
@@ -479,7 +524,7 @@ struct ValLayout {
 
 template <int DK, bool FLEX, bool LOGIT>
 __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, int bh, int vt, int DV, int seg,
-                              uint64_t* bars, uint32_t tmem) {
+                              uint64_t* bars, uint32_t tmem, int* safe_flag) {
   using L = ValLayout<DK>;
   using Gate = GateRun<DK, BT, LOGIT>;
   // column offsets into wider tensors and the value-side row pitch (FLEX builds only)
@@ -518,10 +563,11 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       tma_load_3d(sm + L::VZ + b * (C * 128), &mp.v, bar_dv, col_v + c0 + b * 64, chunk * C, bh);
     }
   };
-  auto sync_tc = [&]() {
+  // operands in shared memory / TMEM are complete: hand them to the producer warp
+  auto handoff = [&](int id) {
+    fence_async_smem();
     tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+    bar_arrive(id, BTP);
   };
   // G <- DEC[row] * G for this thread's row of the M=128 accumulator.
   auto rescale_G = [&]() {
@@ -536,6 +582,92 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     }
     tmem_st_wait();
   };
+  // MMA group 1 (producer lane 0): Z^T part, A (first commit), dv^T = G^T Kh^T and the G update
+  auto issue_g1 = [&]() {
+    const uint32_t dob = base + 3 * L::RAW;
+    constexpr uint32_t id_A = idesc_bf16_f32(C, C, false, false);
+    constexpr uint32_t id_dv = idesc_bf16_f32(VT, C, true, false);  // dv^T = G^T Kh^T: value columns on M
+    constexpr uint32_t id_G = idesc_bf16_f32(DK, VT, true, true);
+    // Z^T part of this value tile: G_{i+1}[:, tile] V[:, tile]^T (G copy hi + lo); first, since the
+    // v tile shares A's space, which the A epilogue overwrites after the first commit
+    constexpr uint32_t id_Z = idesc_bf16_f32(DK, C, false, false);
+#pragma unroll
+    for (int k = 0; k < VT / 16; ++k) {
+      const uint32_t ko = (k >> 2) * (DK * 128) + (k & 3) * 32;
+      const uint64_t vd = desc_sw128(base + L::VZ + (k >> 2) * (C * 128) + (k & 3) * 32, 16, 1024);
+      umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_HI + ko, 16, 1024), vd, id_Z, k > 0);
+      umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_LO + ko, 16, 1024), vd, id_Z, 1);
+    }
+#pragma unroll
+    for (int k = 0; k < DK / 16; ++k) {
+      const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
+      const uint64_t qh = desc_sw128(base + L::QP_HI + ko, 16, 1024), ql = desc_sw128(base + L::QP_LO + ko, 16, 1024);
+      const uint64_t kh = desc_sw128(base + L::KH_HI + ko, 16, 1024), kl = desc_sw128(base + L::KH_LO + ko, 16, 1024);
+      umma_bf16(tmem + L::T_A, qh, kh, id_A, k > 0);
+      umma_bf16(tmem + L::T_A, qh, kl, id_A, 1);
+      umma_bf16(tmem + L::T_A, ql, kh, id_A, 1);
+    }
+    umma_commit(bar_mA);
+    // dv^T = G^T Kh^T and the G update: the A epilogue runs while they execute
+#pragma unroll
+    for (int k = 0; k < DK / 16; ++k) {
+      const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
+      const uint64_t kh = desc_sw128(base + L::KH_HI + ko, 16, 1024), kl = desc_sw128(base + L::KH_LO + ko, 16, 1024);
+      const uint64_t gh = desc_sw128(base + L::GC_HI + k * 2048, DK * 128, 1024);
+      umma_bf16(tmem + L::T_DV, gh, kh, id_dv, k > 0);
+      umma_bf16(tmem + L::T_DV, desc_sw128(base + L::GC_LO + k * 2048, DK * 128, 1024), kh, id_dv, 1);
+      umma_bf16(tmem + L::T_DV, gh, kl, id_dv, 1);
+    }
+#pragma unroll
+    for (int k = 0; k < C / 16; ++k) {
+      const uint64_t dd = desc_sw128(dob + k * 2048, C * 128, 1024);
+      umma_bf16(tmem + L::T_G, desc_sw128(base + L::QP_HI + k * 2048, C * 128, 1024), dd, id_G, 1);
+      umma_bf16(tmem + L::T_G, desc_sw128(base + L::QP_LO + k * 2048, C * 128, 1024), dd, id_G, 1);
+    }
+    umma_commit(bar_m1);
+  };
+  // MMA group 2 (producer lane 0): dv^T += dO^T A
+  auto issue_g2 = [&]() {
+    const uint32_t dob = base + 3 * L::RAW;
+    constexpr uint32_t id_dv2 = idesc_bf16_f32(VT, C, true, true);  // dv^T += dO^T A
+#pragma unroll
+    for (int k = 0; k < C / 16; ++k) {
+      const uint64_t dd = desc_sw128(dob + k * 2048, C * 128, 1024);
+      umma_bf16(tmem + L::T_DV, dd, desc_sw128(base + L::AB_HI + k * 2048, C * 128, 1024), id_dv2, 1);
+      umma_bf16(tmem + L::T_DV, dd, desc_sw128(base + L::AB_LO + k * 2048, C * 128, 1024), id_dv2, 1);
+    }
+    umma_commit(bar_m2);
+  };
+
+  if (tid >= BT) {  // ======== producer warp: the MMA groups and the loads that wait for a handoff
+    for (int n = 0; n < nl; ++n) {
+      const int i = ch1 - 1 - n;
+      bar_sync(kBarH1, BTP);  // chunk i's Qs, Kh, G copy (and rescaled G) are ready
+      tc_fence_after();
+      const int safe = safe_flag[0];
+      if (lane == 0) {
+        if (!safe && n + 1 < nl) load_qkg(i - 1);  // the raw q, k, g tiles have been read
+        mbar_wait(bar_dv, ph_dv, a.latch);
+        ph_dv ^= 1;
+        tc_fence_after();
+        issue_g1();
+      }
+      __syncwarp();
+      bar_sync(kBarH2, BTP);  // chunk i's A operand is in shared memory
+      tc_fence_after();
+      if (lane == 0) {
+        if (safe && n + 1 < nl) load_qkg(i - 1);  // the exact path has read the raw tiles
+        issue_g2();
+        if (n + 1 < nl) {  // dO and v (over A) are free once group 2 has completed
+          mbar_wait(bar_m2, ph_m2, a.latch);
+          ph_m2 ^= 1;
+          load_dov(i - 1);
+        }
+      }
+      __syncwarp();
+    }
+    return;
+  }
   // G rows (this thread owns row grow of the M=128 accumulator): init from dhT[:, tile] (last
   // segment) or from the gradient at the segment's end
   {
@@ -567,7 +699,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       DEC[gr.d] = gr.dec0;
       DEC[gr.d + 1] = gr.dec1;
     }
-    const int safe = __syncthreads_or(weak);
+    const int safe = bar_or(kBarCompute, BT, weak);
     {
       const float inv0 = safe ? 1.f : 1.f / gr.dec0, inv1 = safe ? 1.f : 1.f / gr.dec1;
       const uint32_t blk = (gr.d >> 6) * (C * 128), col = gr.d & 63;
@@ -590,54 +722,8 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       });
     }
     if (safe) rescale_G();
-    mbar_wait(bar_dv, ph_dv, a.latch);
-    ph_dv ^= 1;
-    fence_async_smem();
-    sync_tc();
-    if (tid == 0) {
-      const uint32_t dob = base + 3 * L::RAW;
-      constexpr uint32_t id_A = idesc_bf16_f32(C, C, false, false);
-      constexpr uint32_t id_dv = idesc_bf16_f32(VT, C, true, false);  // dv^T = G^T Kh^T: value columns on M
-      constexpr uint32_t id_G = idesc_bf16_f32(DK, VT, true, true);
-      // Z^T part of this value tile: G_{i+1}[:, tile] V[:, tile]^T (G copy hi + lo); first, since the
-      // v tile shares A's space, which the A epilogue overwrites after the first commit
-      constexpr uint32_t id_Z = idesc_bf16_f32(DK, C, false, false);
-#pragma unroll
-      for (int k = 0; k < VT / 16; ++k) {
-        const uint32_t ko = (k >> 2) * (DK * 128) + (k & 3) * 32;
-        const uint64_t vd = desc_sw128(base + L::VZ + (k >> 2) * (C * 128) + (k & 3) * 32, 16, 1024);
-        umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_HI + ko, 16, 1024), vd, id_Z, k > 0);
-        umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_LO + ko, 16, 1024), vd, id_Z, 1);
-      }
-#pragma unroll
-      for (int k = 0; k < DK / 16; ++k) {
-        const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
-        const uint64_t qh = desc_sw128(base + L::QP_HI + ko, 16, 1024), ql = desc_sw128(base + L::QP_LO + ko, 16, 1024);
-        const uint64_t kh = desc_sw128(base + L::KH_HI + ko, 16, 1024), kl = desc_sw128(base + L::KH_LO + ko, 16, 1024);
-        umma_bf16(tmem + L::T_A, qh, kh, id_A, k > 0);
-        umma_bf16(tmem + L::T_A, qh, kl, id_A, 1);
-        umma_bf16(tmem + L::T_A, ql, kh, id_A, 1);
-      }
-      umma_commit(bar_mA);
-      // dv^T = G^T Kh^T and the G update: the A epilogue runs while they execute
-#pragma unroll
-      for (int k = 0; k < DK / 16; ++k) {
-        const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
-        const uint64_t kh = desc_sw128(base + L::KH_HI + ko, 16, 1024), kl = desc_sw128(base + L::KH_LO + ko, 16, 1024);
-        const uint64_t gh = desc_sw128(base + L::GC_HI + k * 2048, DK * 128, 1024);
-        umma_bf16(tmem + L::T_DV, gh, kh, id_dv, k > 0);
-        umma_bf16(tmem + L::T_DV, desc_sw128(base + L::GC_LO + k * 2048, DK * 128, 1024), kh, id_dv, 1);
-        umma_bf16(tmem + L::T_DV, gh, kl, id_dv, 1);
-      }
-#pragma unroll
-      for (int k = 0; k < C / 16; ++k) {
-        const uint64_t dd = desc_sw128(dob + k * 2048, C * 128, 1024);
-        umma_bf16(tmem + L::T_G, desc_sw128(base + L::QP_HI + k * 2048, C * 128, 1024), dd, id_G, 1);
-        umma_bf16(tmem + L::T_G, desc_sw128(base + L::QP_LO + k * 2048, C * 128, 1024), dd, id_G, 1);
-      }
-      umma_commit(bar_m1);
-      if (!safe && n + 1 < nl) load_qkg(i - 1);
-    }
+    if (tid == 0) safe_flag[0] = safe;
+    handoff(kBarH1);  // group 1
     __syncwarp();
     mbar_wait(bar_mA, ph_mA, a.latch);
     ph_mA ^= 1;
@@ -651,10 +737,10 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       float zv[32];
       tmem_ld32(tmem + L::T_Z + lane_off + half * 32, zv);
       tmem_ld_wait();
-      float4* dst = reinterpret_cast<float4*>(
-          a.ws_z + ((((size_t)bh * (DV / VT) + vt) * NC + i) * DK + grow) * C + half * 32);
+      // token-major rows: the lanes (consecutive key dims) store adjacent words
+      float* dst = a.ws_z + ((((size_t)bh * (DV / VT) + vt) * NC + i) * C + half * 32) * DK + grow;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) dst[c] = make_float4(zv[4 * c], zv[4 * c + 1], zv[4 * c + 2], zv[4 * c + 3]);
+      for (int c = 0; c < 32; ++c) dst[(size_t)c * DK] = zv[c];
       // this tile's part of sum_r Kh_r Z_r over the thread's 32 tokens (Kh as hi + lo)
       const uint32_t kblk = (grow >> 6) * (C * 128), kcol = grow & 63;
       float kz = 0.f;
@@ -676,7 +762,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
           XB[j * DK + tid] = b;
         }
       }
-      __syncthreads();
+      bar_sync(kBarCompute, BT);
       for (int e = tid; e < C * C; e += BT) {
         const int j = e / C, r = e % C;
         float acc = 0.f;
@@ -686,7 +772,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
                    __expf(XB[j * DK + d] - XB[r * DK + d]);
         XA[e] = acc;
       }
-      __syncthreads();
+      bar_sync(kBarCompute, BT);
     }
     {  // A epilogue
       float v[32];
@@ -703,27 +789,15 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         store_half_split(sm + L::AB_HI, sm + L::AB_LO, row, v, half);
       }
     }
-    fence_async_smem();
-    sync_tc();
-    if (tid == 0) {
-      if (safe && n + 1 < nl) load_qkg(i - 1);
-      const uint32_t dob = base + 3 * L::RAW;
-      constexpr uint32_t id_dv2 = idesc_bf16_f32(VT, C, true, true);  // dv^T += dO^T A
-#pragma unroll
-      for (int k = 0; k < C / 16; ++k) {
-        const uint64_t dd = desc_sw128(dob + k * 2048, C * 128, 1024);
-        umma_bf16(tmem + L::T_DV, dd, desc_sw128(base + L::AB_HI + k * 2048, C * 128, 1024), id_dv2, 1);
-        umma_bf16(tmem + L::T_DV, dd, desc_sw128(base + L::AB_LO + k * 2048, C * 128, 1024), id_dv2, 1);
-      }
-      umma_commit(bar_m2);
-    }
-    // while the rest of group 1 and the second group run: the Z^T epilogue; then (group 1 complete)
-    // the G pass (neither touches A, dO or dv)
+    handoff(kBarH2);  // group 2
+    // once group 1 has completed (the second group runs meanwhile): the Z^T epilogue and the G pass
+    // (neither touches A, dO or dv).  The Z^T epilogue waits for group 1 because its shared-memory
+    // reads would compete with the operand reads of group 1's last MMAs.
     if (!safe) {
-      z_epilogue();
       mbar_wait(bar_m1, ph_m1, a.latch);
       ph_m1 ^= 1;
       tc_fence_after();
+      z_epilogue();
     }
     {  // G_i = dec * G (chunks off the exact path, whose rescale came first) and its hi / lo copy
       const float sc = safe ? 1.f : DEC[grow];
@@ -746,7 +820,6 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     mbar_wait(bar_m2, ph_m2, a.latch);
     ph_m2 ^= 1;
     tc_fence_after();
-    if (tid == 0 && n + 1 < nl) load_dov(i - 1);  // dO and A (over v) are no longer read
     {  // dv epilogue: row vcol of dv^T (value column c0 + vcol), tokens half*32 .. half*32+31; a
        // warp's store covers 32 adjacent value columns of one token
       float v[32];
@@ -771,7 +844,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       }
     }
     tc_fence_before();
-    __syncthreads();
+    bar_sync(kBarCompute, BT);
   }
   // dh0[:, tile] = G_0
   if (a.dh0 && seg == 0) {
@@ -912,35 +985,23 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   const int erow = q4 * 16 + (lane & 15);
   // global inputs of the epilogue, loaded while the tiles arrive
   float pv[16], z[16];
-  {
-    const float4* src = reinterpret_cast<const float4*>(a.ws_part + (((size_t)bh * NC + i) * DK + d0 + erow) * C + tq);
-    float4 u[4], zz[NVT][4];
+  {  // token-major rows: for each token the lanes read adjacent words (two runs of 16 dims)
+    const float* src = a.ws_part + (((size_t)bh * NC + i) * C + tq) * DK + d0 + erow;
+    float zz[NVT][16];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) u[c] = src[c];
+    for (int c = 0; c < 16; ++c) pv[c] = src[(size_t)c * DK];
 #pragma unroll
     for (int vt = 0; vt < NVT; ++vt) {
-      const float4* zs = reinterpret_cast<const float4*>(
-          a.ws_z + ((((size_t)bh * NVT + vt) * NC + i) * DK + d0 + erow) * C + tq);
+      const float* zs = a.ws_z + ((((size_t)bh * NVT + vt) * NC + i) * C + tq) * DK + d0 + erow;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) zz[vt][c] = zs[c];
+      for (int c = 0; c < 16; ++c) zz[vt][c] = zs[(size_t)c * DK];
     }
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      pv[4 * c] = u[c].x;
-      pv[4 * c + 1] = u[c].y;
-      pv[4 * c + 2] = u[c].z;
-      pv[4 * c + 3] = u[c].w;
-      z[4 * c] = z[4 * c + 1] = z[4 * c + 2] = z[4 * c + 3] = 0.f;
+    for (int c = 0; c < 16; ++c) {
+      z[c] = 0.f;
+#pragma unroll
+      for (int vt = 0; vt < NVT; ++vt) z[c] += zz[vt][c];
     }
-#pragma unroll
-    for (int vt = 0; vt < NVT; ++vt)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        z[4 * c] += zz[vt][c].x;
-        z[4 * c + 1] += zz[vt][c].y;
-        z[4 * c + 2] += zz[vt][c].z;
-        z[4 * c + 3] += zz[vt][c].w;
-      }
   }
   const float ci = a.ws_c[((size_t)bh * NC + i) * DK + d0 + erow];
   auto raw = [&](uint32_t off, int j, int d) { return bf2f(sm + off + sw128(j, d)); };
@@ -1109,9 +1170,10 @@ struct BwdSmem {
 };
 
 template <int DK, int DV, bool FLEX, bool LOGIT>
-__global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
+__global__ void __launch_bounds__(BTP, 1) bwd_fused_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bars[6];
+  __shared__ int safe_flag[2];  // exact-path flag of a chunk, compute threads -> producer warp
   __shared__ uint32_t tmem_base_sh;
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -1132,9 +1194,9 @@ __global__ void __launch_bounds__(BT, 1) bwd_fused_kernel(const __grid_constant_
   const int per_seg = a.n_bh * per_head;
   const int seg = blockIdx.x / per_seg, bh = (blockIdx.x % per_seg) / per_head, role = blockIdx.x % per_head;
   if (role < DK / KT)
-    key_tile_body<DK, DV, FLEX, LOGIT>(sm, mp, a, bh, role, seg, bars, tmem);
+    key_tile_body<DK, DV, FLEX, LOGIT>(sm, mp, a, bh, role, seg, bars, tmem, safe_flag);
   else
-    val_tile_body<DK, FLEX, LOGIT>(sm, mp, a, bh, role - DK / KT, DV, seg, bars, tmem);
+    val_tile_body<DK, FLEX, LOGIT>(sm, mp, a, bh, role - DK / KT, DV, seg, bars, tmem, safe_flag);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -1152,7 +1214,7 @@ static cudaError_t launch_all(const BwdMaps& mp, const BwdArgs& a, int BH, cudaS
     if (e == cudaSuccess) e = ensure_smem_attr(k3, CHK, attr3);
     if (e != cudaSuccess) return e;
   }
-  k1<<<BH * (DK / KT + DV / VT) * a.nseg, BT, BwdSmem<DK, DV>::ALLOC, st>>>(mp, a);
+  k1<<<BH * (DK / KT + DV / VT) * a.nseg, BTP, BwdSmem<DK, DV>::ALLOC, st>>>(mp, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int NC = (a.T + C - 1) / C;
