@@ -542,6 +542,12 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     store_ops(0, safe);
     for (int li = 0; li < nloc; ++li) {
       const uint8_t* st = sm + (li & 1) * L::QKG;
+      if (FLEX && args.add_o && lane < 16) {
+        // the partial output that store_o(li) adds, one step ahead: this thread's 128-byte row
+        // segment into L1 (the dependent loads would otherwise stall the epilogue)
+        const int t = (c_begin + li) * C + q4 * 16 + lane;
+        if (t < T) prefetch_l1(args.add_o + ((size_t)bh * T + t) * DV + dv0 + half * 32);
+      }
       // ---- while group 1 of chunk li runs: outputs of chunk li-1, gate math of chunk li+1 ----
       if (li > 0) store_o(li - 1);
       int safe_next = 0;
