@@ -46,7 +46,7 @@ constexpr int BT = 256;  // compute threads per CTA: warps w and w+4 share TMEM 
 // for the group's execution, so the compute warps only hand over (named barriers kBarH1 / kBarH2:
 // the compute threads arrive, the producer warp syncs) and wait for the groups' mbarriers.
 constexpr int BTP = BT + 32;
-constexpr int kBarH1 = 2, kBarH2 = 3;
+constexpr int kBarH1 = 2, kBarH2 = 3, kBarH0 = 4;
 constexpr int KT = 64;   // key dimensions per key-tile CTA
 constexpr int VT = 128;  // value columns per value-tile CTA
 
@@ -516,7 +516,9 @@ struct ValLayout {
   static constexpr uint32_t XB = QP_HI, XA = KH_HI;  // exact-path scratch (after the first MMA group)
   // v tile [64 x VT] for Z^T = G V^T: read by the first MMA group only, so it shares A's space
   static constexpr uint32_t VZ = AB_HI;
-  static constexpr uint32_t T_G = 0, T_A = VT, T_DV = VT + 64, T_Z = 2 * VT + 64;  // dv^T takes 64 columns
+  // dv^T takes 64 columns, double-buffered by chunk parity (its epilogue runs during the next chunk)
+  static constexpr uint32_t T_G = 0, T_A = VT, T_DV = VT + 64, T_Z = 2 * VT + 64;
+  static_assert(T_DV + 128 <= T_Z, "two dv^T buffers");
   static_assert(C * VT * 2 <= DEC - AB_HI && T_Z + 64 <= 512, "v tile / TMEM columns");
   static_assert(STAGE % 1024 == 0, "stage alignment");
   static_assert(C * DK * 4 <= KH_HI - QP_HI && C * C * 4 <= GC_HI - KH_HI, "exact-path scratch");
@@ -582,14 +584,11 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     }
     tmem_st_wait();
   };
-  // MMA group 1 (producer lane 0): Z^T part, A (first commit), dv^T = G^T Kh^T and the G update
-  auto issue_g1 = [&]() {
-    const uint32_t dob = base + 3 * L::RAW;
-    constexpr uint32_t id_A = idesc_bf16_f32(C, C, false, false);
-    constexpr uint32_t id_dv = idesc_bf16_f32(VT, C, true, false);  // dv^T = G^T Kh^T: value columns on M
-    constexpr uint32_t id_G = idesc_bf16_f32(DK, VT, true, true);
-    // Z^T part of this value tile: G_{i+1}[:, tile] V[:, tile]^T (G copy hi + lo); first, since the
-    // v tile shares A's space, which the A epilogue overwrites after the first commit
+  // Z^T part of this value tile (producer lane 0): G_{i+1}[:, tile] V[:, tile]^T with the G copy
+  // hi + lo.  It needs only the G copy and the v tile, so it is issued as soon as the previous
+  // chunk's G pass has handed over; the A commit that follows covers it (MMAs of one thread
+  // complete in order), which matters because the v tile shares A's space.
+  auto issue_z = [&]() {
     constexpr uint32_t id_Z = idesc_bf16_f32(DK, C, false, false);
 #pragma unroll
     for (int k = 0; k < VT / 16; ++k) {
@@ -598,6 +597,14 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_HI + ko, 16, 1024), vd, id_Z, k > 0);
       umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_LO + ko, 16, 1024), vd, id_Z, 1);
     }
+  };
+  // MMA group 1 (producer lane 0): A (first commit, with the Z^T part before it), dv^T = G^T Kh^T
+  // and the G update
+  auto issue_g1 = [&](int n) {
+    const uint32_t dob = base + 3 * L::RAW, t_dv = tmem + L::T_DV + (n & 1) * 64;
+    constexpr uint32_t id_A = idesc_bf16_f32(C, C, false, false);
+    constexpr uint32_t id_dv = idesc_bf16_f32(VT, C, true, false);  // dv^T = G^T Kh^T: value columns on M
+    constexpr uint32_t id_G = idesc_bf16_f32(DK, VT, true, true);
 #pragma unroll
     for (int k = 0; k < DK / 16; ++k) {
       const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
@@ -614,9 +621,9 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
       const uint64_t kh = desc_sw128(base + L::KH_HI + ko, 16, 1024), kl = desc_sw128(base + L::KH_LO + ko, 16, 1024);
       const uint64_t gh = desc_sw128(base + L::GC_HI + k * 2048, DK * 128, 1024);
-      umma_bf16(tmem + L::T_DV, gh, kh, id_dv, k > 0);
-      umma_bf16(tmem + L::T_DV, desc_sw128(base + L::GC_LO + k * 2048, DK * 128, 1024), kh, id_dv, 1);
-      umma_bf16(tmem + L::T_DV, gh, kl, id_dv, 1);
+      umma_bf16(t_dv, gh, kh, id_dv, k > 0);
+      umma_bf16(t_dv, desc_sw128(base + L::GC_LO + k * 2048, DK * 128, 1024), kh, id_dv, 1);
+      umma_bf16(t_dv, gh, kl, id_dv, 1);
     }
 #pragma unroll
     for (int k = 0; k < C / 16; ++k) {
@@ -627,37 +634,47 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     umma_commit(bar_m1);
   };
   // MMA group 2 (producer lane 0): dv^T += dO^T A
-  auto issue_g2 = [&]() {
-    const uint32_t dob = base + 3 * L::RAW;
+  auto issue_g2 = [&](int n) {
+    const uint32_t dob = base + 3 * L::RAW, t_dv = tmem + L::T_DV + (n & 1) * 64;
     constexpr uint32_t id_dv2 = idesc_bf16_f32(VT, C, true, true);  // dv^T += dO^T A
 #pragma unroll
     for (int k = 0; k < C / 16; ++k) {
       const uint64_t dd = desc_sw128(dob + k * 2048, C * 128, 1024);
-      umma_bf16(tmem + L::T_DV, dd, desc_sw128(base + L::AB_HI + k * 2048, C * 128, 1024), id_dv2, 1);
-      umma_bf16(tmem + L::T_DV, dd, desc_sw128(base + L::AB_LO + k * 2048, C * 128, 1024), id_dv2, 1);
+      umma_bf16(t_dv, dd, desc_sw128(base + L::AB_HI + k * 2048, C * 128, 1024), id_dv2, 1);
+      umma_bf16(t_dv, dd, desc_sw128(base + L::AB_LO + k * 2048, C * 128, 1024), id_dv2, 1);
     }
     umma_commit(bar_m2);
   };
 
   if (tid >= BT) {  // ======== producer warp: the MMA groups and the loads that wait for a handoff
+    // the Z^T part of chunk i: after the G copy's handoff (H0) and the arrival of chunk i's v tile
+    auto z_part = [&]() {
+      bar_sync(kBarH0, BTP);
+      tc_fence_after();
+      if (lane == 0) {
+        mbar_wait(bar_dv, ph_dv, a.latch);
+        ph_dv ^= 1;
+        tc_fence_after();
+        issue_z();
+      }
+      __syncwarp();
+    };
+    if (nl > 0) z_part();
     for (int n = 0; n < nl; ++n) {
       const int i = ch1 - 1 - n;
-      bar_sync(kBarH1, BTP);  // chunk i's Qs, Kh, G copy (and rescaled G) are ready
+      bar_sync(kBarH1, BTP);  // chunk i's Qs, Kh (and rescaled G) are ready
       tc_fence_after();
       const int safe = safe_flag[0];
       if (lane == 0) {
         if (!safe && n + 1 < nl) load_qkg(i - 1);  // the raw q, k, g tiles have been read
-        mbar_wait(bar_dv, ph_dv, a.latch);
-        ph_dv ^= 1;
-        tc_fence_after();
-        issue_g1();
+        issue_g1(n);
       }
       __syncwarp();
       bar_sync(kBarH2, BTP);  // chunk i's A operand is in shared memory
       tc_fence_after();
       if (lane == 0) {
         if (safe && n + 1 < nl) load_qkg(i - 1);  // the exact path has read the raw tiles
-        issue_g2();
+        issue_g2(n);
         if (n + 1 < nl) {  // dO and v (over A) are free once group 2 has completed
           mbar_wait(bar_m2, ph_m2, a.latch);
           ph_m2 ^= 1;
@@ -665,6 +682,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
         }
       }
       __syncwarp();
+      if (n + 1 < nl) z_part();  // chunk i-1's Z^T part, after chunk i's G pass
     }
     return;
   }
@@ -688,6 +706,33 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     load_qkg(ch1 - 1);
     load_dov(ch1 - 1);
   }
+  if (nl > 0) handoff(kBarH0);  // the G copy: the first chunk's Z^T part
+  // dv epilogue of chunk ic from dv^T buffer buf (its group 2 has completed): row vcol of dv^T (value
+  // column c0 + vcol), tokens half*32 .. half*32+31; a warp's store covers 32 adjacent value columns
+  // of one token.  It runs during the next chunk's first MMA group.
+  auto dv_epilogue = [&](int ic, int buf) {
+    tc_fence_after();
+    float v[32];
+    const int vcol = q4 * 32 + lane, t0 = ic * C + half * 32;
+    tmem_ld32(tmem + L::T_DV + buf * 64 + lane_off + half * 32, v);
+    tmem_ld_wait();
+    if (FLEX && a.acc_v) {
+      float* p = a.acc_v + ((size_t)bh * T + t0) * DV + c0 + vcol;
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (t0 + c < T) p[(size_t)c * DV] = v[c];
+    } else if (FLEX) {  // dv in bf16 at the value columns of a [BH*T][pv] array
+      __nv_bfloat16* p = a.dv + ((size_t)bh * T + t0) * pitch_v + col_v + c0 + vcol;
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (t0 + c < T) p[(size_t)c * pitch_v] = __float2bfloat16_rn(v[c]);
+    } else {
+      __nv_bfloat16* p = a.dv + ((size_t)bh * T + t0) * DV + c0 + vcol;
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (t0 + c < T) p[(size_t)c * DV] = __float2bfloat16_rn(v[c]);
+    }
+  };
   for (int n = 0; n < nl; ++n) {
     const int i = ch1 - 1 - n;
     mbar_wait(bar_ld, ph_ld, a.latch);
@@ -724,6 +769,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     if (safe) rescale_G();
     if (tid == 0) safe_flag[0] = safe;
     handoff(kBarH1);  // group 1
+    if (n > 0) dv_epilogue(i + 1, (n - 1) & 1);  // the previous chunk's dv, while group 1 runs
     __syncwarp();
     mbar_wait(bar_mA, ph_mA, a.latch);
     ph_mA ^= 1;
@@ -790,14 +836,13 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       }
     }
     handoff(kBarH2);  // group 2
-    // once group 1 has completed (the second group runs meanwhile): the Z^T epilogue and the G pass
-    // (neither touches A, dO or dv).  The Z^T epilogue waits for group 1 because its shared-memory
-    // reads would compete with the operand reads of group 1's last MMAs.
+    // while the rest of group 1 runs: the Z^T epilogue (its part completed before A); then, group 1
+    // complete, the G pass (neither touches A, dO or dv)
     if (!safe) {
+      z_epilogue();
       mbar_wait(bar_m1, ph_m1, a.latch);
       ph_m1 ^= 1;
       tc_fence_after();
-      z_epilogue();
     }
     {  // G_i = dec * G (chunks off the exact path, whose rescale came first) and its hi / lo copy
       const float sc = safe ? 1.f : DEC[grow];
@@ -816,36 +861,15 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       }
       tmem_st_wait();
     }
+    if (n + 1 < nl) handoff(kBarH0);  // the G copy: the next chunk's Z^T part
     __syncwarp();
     mbar_wait(bar_m2, ph_m2, a.latch);
     ph_m2 ^= 1;
     tc_fence_after();
-    {  // dv epilogue: row vcol of dv^T (value column c0 + vcol), tokens half*32 .. half*32+31; a
-       // warp's store covers 32 adjacent value columns of one token
-      float v[32];
-      const int vcol = q4 * 32 + lane, t0 = i * C + half * 32;
-      tmem_ld32(tmem + L::T_DV + lane_off + half * 32, v);
-      tmem_ld_wait();
-      if (FLEX && a.acc_v) {
-        float* p = a.acc_v + ((size_t)bh * T + t0) * DV + c0 + vcol;
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (t0 + c < T) p[(size_t)c * DV] = v[c];
-      } else if (FLEX) {  // dv in bf16 at the value columns of a [BH*T][pv] array
-        __nv_bfloat16* p = a.dv + ((size_t)bh * T + t0) * pitch_v + col_v + c0 + vcol;
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (t0 + c < T) p[(size_t)c * pitch_v] = __float2bfloat16_rn(v[c]);
-      } else {
-        __nv_bfloat16* p = a.dv + ((size_t)bh * T + t0) * DV + c0 + vcol;
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (t0 + c < T) p[(size_t)c * DV] = __float2bfloat16_rn(v[c]);
-      }
-    }
     tc_fence_before();
     bar_sync(kBarCompute, BT);
   }
+  if (nl > 0) dv_epilogue(ch0, (nl - 1) & 1);
   // dh0[:, tile] = G_0
   if (a.dh0 && seg == 0) {
     tc_fence_after();
