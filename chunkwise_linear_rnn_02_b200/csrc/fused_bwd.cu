@@ -666,8 +666,8 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       tc_fence_after();
       const int safe = safe_flag[0];
       if (lane == 0) {
-        if (!safe && n + 1 < nl) load_qkg(i - 1);  // the raw q, k, g tiles have been read
         issue_g1(n);
+        if (!safe && n + 1 < nl) load_qkg(i - 1);  // the raw q, k, g tiles have been read
       }
       __syncwarp();
       bar_sync(kBarH2, BTP);  // chunk i's A operand is in shared memory
@@ -1209,6 +1209,16 @@ __global__ void __launch_bounds__(BTP, 1) bwd_fused_kernel(const __grid_constant
   if (threadIdx.x == 0) {
     for (int b = 0; b < 6; ++b) mbar_init(&bars[b], 1);
     fence_mbar_init();
+  }
+  if (threadIdx.x == BT) {  // the tensor maps, ahead of the first loads
+    prefetch_tmap(&mp.v);
+    prefetch_tmap(&mp.dO);
+    prefetch_tmap(&mp.k64);
+    prefetch_tmap(&mp.g64);
+    prefetch_tmap(&mp.q64);
+    prefetch_tmap(&mp.q_all);
+    prefetch_tmap(&mp.k_all);
+    prefetch_tmap(&mp.g_all);
   }
   tc_fence_before();
   __syncthreads();
