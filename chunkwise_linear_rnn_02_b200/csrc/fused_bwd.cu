@@ -49,6 +49,9 @@ constexpr int BTP = BT + 32;
 constexpr int kBarH1 = 2, kBarH2 = 3, kBarH0 = 4;
 constexpr int KT = 64;   // key dimensions per key-tile CTA
 constexpr int VT = 128;  // value columns per value-tile CTA
+// Per (head, chunk): the masked dA as the MMAs take it (bf16 hi and lo [64 x 64] tiles, 128-byte
+// swizzled) and its fp32 diagonal, written by the first key tile for the chunk kernel.
+constexpr uint32_t kDaBytes = 2 * C * KT * 2 + C * 4;
 
 struct BwdMaps {
   CUtensorMap v, dO;                 // box (64 cols, 64 tokens), 128-byte swizzle
@@ -67,6 +70,7 @@ struct BwdArgs {
   float* ws_kz;    // [BH][DV/VT][NC][2][DK] value tiles' parts of the chunk sums of Kh Z (per token half)
   float* ws_c;     // [BH][NC][DK] the dg carry c_i of every chunk
   float* ws_part;  // [BH][NC][64][DK] forward-walk part of dg, one row of DK dims per token
+  uint8_t* ws_da;  // [BH][NC] blocks of kDaBytes: masked dA hi / lo tiles and diagonal
   int T;
   // Sequence split: nseg segments of seg_chunks chunks; s_in / g_end hold the segment states
   // ([BH][nseg][DK][DV] fp32: s_in[s-1] enters segment s, g_end[s] = dL/dS at the end of s).
@@ -331,15 +335,29 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       const int b = (i - ch0) & 1;
       bar_sync(kBarH2, BTP);  // chunk i's dA operand is in shared memory
       tc_fence_after();
-      if (lane == 0 && !safe_flag[b]) issue_m2();
+      if (lane == 0) {
+        if (!safe_flag[b]) issue_m2();
+        if (tau == 0) {  // dA and its diagonal for the chunk kernel (one key tile per head writes)
+          uint8_t* dst = a.ws_da + ((size_t)bh * NC + i) * kDaBytes;
+          bulk_s2g(dst, sm + L::DA_HI, 2 * L::TILE);
+          bulk_s2g(dst + 2 * L::TILE, sm + L::DIAG, C * 4);
+          tma_store_commit();
+        }
+      }
       __syncwarp();
       if (i + 1 < ch1) {
         bar_sync(kBarH1, BTP);  // chunk i+1's Kh and state copy are in shared memory
         tc_fence_after();
-        if (lane == 0) issue_m1();
+        if (lane == 0) {
+          // the copies have read dA before group 1 of chunk i+1 is issued, whose completion the
+          // compute threads wait for before they write chunk i+1's dA
+          if (tau == 0) tma_store_wait_read_all();
+          issue_m1();
+        }
         __syncwarp();
       }
     }
+    if (lane == 0 && tau == 0) tma_store_wait_all();  // written before the CTA exits
     return;
   }
 
@@ -927,40 +945,40 @@ __global__ void __launch_bounds__(256) carry_scan_kernel(const float* __restrict
 
 // ------------------------------------------------------------------------------------------
 // Third launch: one CTA per (head, 64 key dimensions, chunk).  Gate run of the key slab (Qt, E2,
-// decays), dA = dO V^T recomputed, W^T = Qt^T dA, and the epilogue
+// decays), the masked dA of the chunk as the first key tile wrote it (hi / lo operand tiles and the
+// diagonal, one bulk copy), W^T = Qt^T dA, and the epilogue
 //   dk = E2 Z + (E2 / dec) W,   dg = c_i + prefix(Kh Z + k dk^intra) + the forward walk's part,
 // with Z^T summed over the value tiles' parts.  No state: every chunk is independent.
 // ------------------------------------------------------------------------------------------
 template <int DK, int DV>
 struct ChunkLayout {
-  static constexpr uint32_t VB = C * DV * 2;        // a v or dO tile [64 x DV]
   static constexpr uint32_t TILE = C * KT * 2;      // a [64 x 64] bf16 tile
-  static constexpr uint32_t PA_V = 0, PA_DO = VB;
-  static constexpr uint32_t PB = 2 * VB;            // k, g, q tiles
-  static constexpr uint32_t PB_K = PB, PB_G = PB + TILE, PB_Q = PB + 2 * TILE;
-  static constexpr uint32_t KQ_HI = PB + 3 * TILE;  // Qt hi / lo
+  static constexpr uint32_t PB_K = 0, PB_G = TILE, PB_Q = 2 * TILE;  // k, g, q tiles
+  static constexpr uint32_t KQ_HI = 3 * TILE;       // Qt hi / lo
   static constexpr uint32_t KQ_LO = KQ_HI + TILE;
-  static constexpr uint32_t DA_HI = PA_V;           // masked dA hi / lo: v is dead once dA is formed
-  static constexpr uint32_t DA_LO = DA_HI + TILE;
+  static constexpr uint32_t DA_HI = KQ_LO + TILE;   // masked dA hi / lo, then its diagonal: one
+  static constexpr uint32_t DA_LO = DA_HI + TILE;   // kDaBytes block as the key tile wrote it
+  static constexpr uint32_t DIAG = DA_LO + TILE;
   static constexpr int NS = GateRun<KT, BT>::NSPLIT;
-  static constexpr uint32_t XCH = KQ_LO + TILE;
+  static constexpr uint32_t XCH = DIAG + C * 4;
   static constexpr uint32_t DEC = XCH + 2 * KT * 8;
   static constexpr uint32_t TOT = DEC + KT * 4;
-  static constexpr uint32_t DIAG = TOT + NS * KT * 4;
-  static constexpr uint32_t TOTAL = DIAG + C * 4;
-  static constexpr uint32_t T_DA = 0, T_Y = 64;  // TMEM columns (128 allocated)
-  static_assert(PB % 1024 == 0 && KQ_HI % 1024 == 0 && 2 * TILE <= VB, "operand layout");
+  static constexpr uint32_t TOTAL = TOT + NS * KT * 4;
+  static constexpr uint32_t T_Y = 0;  // TMEM columns (64 allocated)
+  static_assert(KQ_HI % 1024 == 0 && DA_HI % 1024 == 0 && DIAG == DA_HI + 2 * TILE &&
+                    DIAG + C * 4 - DA_HI == kDaBytes,
+                "operand layout");
 };
 
 template <int DK, int DV, bool FLEX, bool LOGIT>
 __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
   using L = ChunkLayout<DK, DV>;
   using Gate = GateRun<KT, BT, LOGIT>;
-  // column offsets into wider input tensors (FLEX builds only)
-  const int col_k = FLEX ? a.ck : 0, col_v = FLEX ? a.cv : 0;
+  // column offset into wider input tensors (FLEX builds only)
+  const int col_k = FLEX ? a.ck : 0;
   constexpr int NS = L::NS, TS = Gate::TS, NVT = DV / VT;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_ld, bar_m1, bar_m2;
+  __shared__ uint64_t bar_ld, bar_m2;
   __shared__ uint32_t tmem_base_sh;
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -971,20 +989,17 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   const int i = blockIdx.x % NC, slab = blockIdx.x / NC;
   const int tau = slab % (DK / KT), bh = slab / (DK / KT), d0 = tau * KT;
   const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-  const bool row_owner = lane < 16;
-  const int row = q4 * 16 + lane;
   const int tb = half * 32;
   float* DEC = reinterpret_cast<float*>(sm + L::DEC);
   float* TOT = reinterpret_cast<float*>(sm + L::TOT);
   float* DIAG = reinterpret_cast<float*>(sm + L::DIAG);
 
   if (warp == 0) {
-    tmem_alloc(&tmem_base_sh, 128);
+    tmem_alloc(&tmem_base_sh, 64);
     tmem_relinquish();
   }
   if (tid == 0) {
     mbar_init(&bar_ld, 1);
-    mbar_init(&bar_m1, 1);
     mbar_init(&bar_m2, 1);
     fence_mbar_init();
   }
@@ -993,11 +1008,8 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   if (tid == 0) {
-    mbar_arrive_expect_tx(&bar_ld, 2 * L::VB + 3 * L::TILE);
-    for (int bb = 0; bb < DV / 64; ++bb) {
-      tma_load_3d(sm + L::PA_V + bb * (C * 128), &mp.v, &bar_ld, col_v + bb * 64, i * C, bh);
-      tma_load_3d(sm + L::PA_DO + bb * (C * 128), &mp.dO, &bar_ld, col_v + bb * 64, i * C, bh);
-    }
+    mbar_arrive_expect_tx(&bar_ld, 3 * L::TILE + kDaBytes);
+    bulk_g2s(sm + L::DA_HI, a.ws_da + ((size_t)bh * NC + i) * kDaBytes, kDaBytes, &bar_ld);
     tma_load_3d(sm + L::PB_K, &mp.k64, &bar_ld, col_k + d0, i * C, bh);
     tma_load_3d(sm + L::PB_G, &mp.g64, &bar_ld, col_k + d0, i * C, bh);
     tma_load_3d(sm + L::PB_Q, &mp.q64, &bar_ld, col_k + d0, i * C, bh);
@@ -1032,17 +1044,6 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   auto dA_at = [&](int j, int r) { return raw(L::DA_HI, j, r) + raw(L::DA_LO, j, r); };
 
   mbar_wait(&bar_ld, 0, a.latch);
-  if (tid == 0) {  // dA = dO V^T (operands as loaded)
-    tc_fence_after();
-    constexpr uint32_t id_dA = idesc_bf16_f32(C, C, false, false);
-#pragma unroll
-    for (int k = 0; k < DV / 16; ++k) {
-      const uint32_t ko = (k >> 2) * (C * 128) + (k & 3) * 32;
-      umma_bf16(tmem + L::T_DA, desc_sw128(base + L::PA_DO + ko, 16, 1024), desc_sw128(base + L::PA_V + ko, 16, 1024),
-                id_dA, k > 0);
-    }
-    umma_commit(&bar_m1);
-  }
   // gate run of the key slab: Qt hi / lo, decays, run products
   Gate gr;
   if constexpr (LOGIT) gr.set_logit(a.inv_tau, T - i * C);
@@ -1061,22 +1062,6 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
     *reinterpret_cast<uint32_t*>(sm + L::KQ_HI + sw128(j, gr.d)) = hi;
     *reinterpret_cast<uint32_t*>(sm + L::KQ_LO + sw128(j, gr.d)) = lo;
   });
-  __syncwarp();
-  mbar_wait(&bar_m1, 0, a.latch);
-  tc_fence_after();
-  {  // dA epilogue: masked hi / lo operand (over the dead v tile) and its diagonal
-    float v[32];
-    tmem_ld32(tmem + L::T_DA + lane_off + tb, v);
-    tmem_ld_wait();
-    if (row_owner) {
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        if (tb + c > row) v[c] = 0.f;
-        if (tb + c == row) DIAG[row] = v[c];
-      }
-      store_half_split(sm + L::DA_HI, sm + L::DA_LO, row, v, half);
-    }
-  }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -1180,7 +1165,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 128);
+  if (warp == 0) tmem_dealloc(tmem, 64);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1266,9 +1251,9 @@ bool bwd_supported(int BH, int T, int dk, int dv, int chunk, int dtype) {
   return encode_fn() != nullptr;
 }
 
-// Workspace parts, in order: Qt X chunk sums, forward part of dg, carry starts, Z^T parts, Kh Z
-// chunk sums, carries; with a sequence split also the segment states (forward, gradient) and the
-// segment decay products.
+// Workspace parts, in order: Qt X chunk sums, forward part of dg, carry starts, Z parts, Kh Z chunk
+// sums, carries; with a sequence split the segment states (forward, gradient) and the segment decay
+// products; the masked dA blocks.
 static void bwd_parts(int BH, int T, int dk, int dv, size_t* sz, int* nseg, int* seg_chunks) {
   plan_bwd_segments(BH * (dk / KT + dv / VT), T, nseg, seg_chunks);
   const size_t NC = (T + C - 1) / C, ns = *nseg, f = sizeof(float);
@@ -1281,10 +1266,11 @@ static void bwd_parts(int BH, int T, int dk, int dv, size_t* sz, int* nseg, int*
   sz[6] = ns > 1 ? align256((size_t)BH * ns * dk * dv * f) : 0;
   sz[7] = sz[6];
   sz[8] = ns > 1 ? align256((size_t)BH * ns * dk * f) : 0;
+  sz[9] = align256((size_t)BH * NC * kDaBytes);
 }
 
 size_t bwd_workspace(int BH, int T, int dk, int dv) {
-  size_t sz[9];
+  size_t sz[10];
   int nseg, per;
   bwd_parts(BH, T, dk, dv, sz, &nseg, &per);
   size_t n = 0;
@@ -1328,11 +1314,11 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
   a.pv = PV;
   a.cv = CV;
   a.inv_tau = inv_tau;
-  size_t sz[9];
+  size_t sz[10];
   bwd_parts(BH, T, DK, DV, sz, &a.nseg, &a.seg_chunks);
-  float* p[9];
+  float* p[10];
   p[0] = static_cast<float*>(ws);
-  for (int j = 1; j < 9; ++j) p[j] = p[j - 1] + sz[j - 1] / sizeof(float);
+  for (int j = 1; j < 10; ++j) p[j] = p[j - 1] + sz[j - 1] / sizeof(float);
   a.ws_qx = p[0];
   a.ws_part = p[1];
   a.ws_carry = p[2];
@@ -1341,6 +1327,7 @@ static cudaError_t launch_bwd(const void* q, const void* k, const void* v, const
   a.ws_c = p[5];
   a.s_in = a.nseg > 1 ? p[6] : nullptr;
   a.g_end = a.nseg > 1 ? p[7] : nullptr;
+  a.ws_da = reinterpret_cast<uint8_t*>(p[9]);
   a.n_bh = BH;
   a.latch = device_error_latch();
   if (a.nseg > 1) {

@@ -195,12 +195,14 @@ def test_fused_shapes_mixed_strong_gates():
 
 
 def _bwd_workspace_bytes(BH, T, dk, dv, nseg):
-    """Size of the fused backward's workspace: six parts, plus the segment states when split."""
+    """Size of the fused backward's workspace: six parts, the segment states when split, and per
+    (head, chunk) the masked dA block (bf16 hi and lo 64 x 64 tiles and the fp32 diagonal)."""
     NC = -(-T // 64)
     parts = [BH * NC * dk, BH * NC * 64 * dk, BH * nseg * dk, BH * (dv // 128) * NC * dk * 64,
              BH * (dv // 128) * NC * 2 * dk, BH * NC * dk]
     if nseg > 1:
         parts += [BH * nseg * dk * dv, BH * nseg * dk * dv, BH * nseg * dk]
+    parts += [BH * NC * (2 * 64 * 64 * 2 + 64 * 4) // 4]
     return sum(-(-4 * p // 256) * 256 for p in parts)
 
 
