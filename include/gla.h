@@ -206,9 +206,9 @@ int gsa_recurrent_step(const void* q, const void* k, const void* v, const void* 
  * Arguments, layouts and outputs are those of gla_chunk_bwd.  Supported: bf16, chunk 64,
  * d_k = 128, d_v in {128, 256}, T >= 1 (else GLA_ERR_UNSUPPORTED / GLA_ERR_INVALID_ARG), and
  * scratch within the 128 MiB (else GLA_ERR_WORKSPACE): the bytes gla_chunk_bwd_workspace()
- * reports for the same sizes, (66 + d_v/2 + d_v/64)*B*H*ceil(T/64)*d_k*4 + nseg*B*H*d_k*4 (six
- * parts, each rounded up to 256 bytes), plus 2*nseg*B*H*d_k*d_v*4 + nseg*B*H*d_k*4 when few heads
- * leave SMs idle and the sequence is split into nseg segments.
+ * reports for the same sizes, (66 + d_v/2 + d_v/64)*B*H*ceil(T/64)*d_k*4 + nseg*B*H*d_k*4 +
+ * 16640*B*H*ceil(T/64) (seven parts, each rounded up to 256 bytes), plus 2*nseg*B*H*d_k*d_v*4 +
+ * nseg*B*H*d_k*4 when few heads leave SMs idle and the sequence is split into nseg segments.
  * It allocates nothing.
  * ------------------------------------------------------------------------------------- */
 int gla_chunk_bwd_noalloc(const void* q, const void* k, const void* v, const void* g, const float* h0,
