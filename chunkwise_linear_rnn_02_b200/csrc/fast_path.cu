@@ -655,6 +655,26 @@ __global__ void segment_scan_kernel(float* __restrict__ sbuf, const float* __res
   }
 }
 
+cudaError_t side_stream(int pool, SideStream** out) {
+  static std::mutex make_mu;
+  static SideStream per_dev[2][64];
+  static bool made[2][64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || pool < 0 || pool > 1) return cudaErrorInvalidValue;
+  std::lock_guard<std::mutex> g(make_mu);
+  SideStream& x = per_dev[pool][dev];
+  if (!made[pool][dev]) {
+    if ((e = cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+    made[pool][dev] = true;
+  }
+  *out = &x;
+  return cudaSuccess;
+}
+
 int sm_count() {
   static std::atomic<int> cached[64] = {};
   int dev = 0;
@@ -814,16 +834,28 @@ cudaError_t segment_states(const CUtensorMap& mq, const CUtensorMap& mk, const C
   a.sbuf = sbuf;
   a.gam = gam;
   const bool flex = inv_tau > 0.f || ck != 0 || cv != 0;
-  cudaError_t e = flex ? launch_state_pass<128, true, false, true>(mk, mg, mv, a, BH, dv, st)
-                       : launch_state_pass<128, true, false, false>(mk, mg, mv, a, BH, dv, st);
+  // The two passes are independent (only the reverse scan below needs the forward pass's decay
+  // products): the reverse pass runs on a side stream, beside the forward one.
+  SideStream* side = nullptr;
+  cudaError_t e = side_stream(1, &side);
   if (e != cudaSuccess) return e;
-  FwdArgs r = a;
-  r.h0 = dhT;
-  r.sbuf = gbuf;
-  r.gam = nullptr;
-  e = flex ? launch_state_pass<128, true, true, true>(mq, mg, mdo, r, BH, dv, st)
-           : launch_state_pass<128, true, true, false>(mq, mg, mdo, r, BH, dv, st);
-  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lock(side->mu);
+    if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
+    FwdArgs r = a;
+    r.h0 = dhT;
+    r.sbuf = gbuf;
+    r.gam = nullptr;
+    e = flex ? launch_state_pass<128, true, true, true>(mq, mg, mdo, r, BH, dv, side->s)
+             : launch_state_pass<128, true, true, false>(mq, mg, mdo, r, BH, dv, side->s);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess) return e;
+    e = flex ? launch_state_pass<128, true, false, true>(mk, mg, mv, a, BH, dv, st)
+             : launch_state_pass<128, true, false, false>(mk, mg, mv, a, BH, dv, st);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(st, side->join, 0)) != cudaSuccess) return e;
+  }
   if (nseg > 2) {
     const size_t n = (size_t)BH * dk * dv;
     const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);

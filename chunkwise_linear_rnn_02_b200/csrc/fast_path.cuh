@@ -2,6 +2,8 @@
 // The API layer asks *_supported() first and otherwise runs the generic kernels.
 #pragma once
 
+#include <mutex>
+
 #include <cuda.h>
 
 #include "common.cuh"
@@ -50,6 +52,18 @@ cudaError_t segment_states(const CUtensorMap& mq, const CUtensorMap& mk, const C
 
 // SM count of the current device (cached per device).
 int sm_count();
+
+// A second stream per device and pool, with fork / join events, for launches that need not run after
+// one another; made on first use.  Its mutex is held while a call enqueues its work there, so that
+// the event records and waits of concurrent callers do not interleave.  Pool 0 serves the API layer
+// (wide-shape sub-problems, GSA), pool 1 the launches inside one fused call (the backward's segment
+// state passes), so that a call made while pool 0 is held never waits for it again.
+struct SideStream {
+  cudaStream_t s;
+  cudaEvent_t fork, join;
+  std::mutex mu;
+};
+cudaError_t side_stream(int pool, SideStream** out);
 
 // Sequence split of a key-gated recurrence S <- diag(e^{g_t}) S + k_t^T v_t with d_k = 64 rows
 // (k, g: bf16 [BH][T][64]; v: bf16 [BH][T][dv], dv a multiple of 64), for a caller that walks the

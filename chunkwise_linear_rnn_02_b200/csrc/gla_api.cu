@@ -127,32 +127,6 @@ int split_fwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const 
   return GLA_OK;
 }
 
-// A second stream per device, with fork / join events, for sub-problems that need not run after one
-// another; made on first use.  Its mutex is held while a call enqueues its work there, so that the
-// event records and waits of concurrent callers do not interleave.
-struct SideStream {
-  cudaStream_t s;
-  cudaEvent_t fork, join;
-  std::mutex mu;
-};
-int side_stream(SideStream** out) {
-  static std::mutex make_mu;
-  static SideStream per_dev[64];
-  static bool made[64];
-  int dev = 0;
-  GLA_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) return GLA_ERR_CUDA;
-  std::lock_guard<std::mutex> g(make_mu);
-  if (!made[dev]) {
-    GLA_CUDA(cudaStreamCreateWithFlags(&per_dev[dev].s, cudaStreamNonBlocking));
-    GLA_CUDA(cudaEventCreateWithFlags(&per_dev[dev].fork, cudaEventDisableTiming));
-    GLA_CUDA(cudaEventCreateWithFlags(&per_dev[dev].join, cudaEventDisableTiming));
-    made[dev] = true;
-  }
-  *out = &per_dev[dev];
-  return GLA_OK;
-}
-
 struct SplitBwdWs {
   float *aq, *ak, *ag;  // [nk][nv] slices [BH*T][128]: each sub-problem's key-side gradients
   float* av;            // [nk][nv] slices [BH*T][vb]: each sub-problem's dv (none with one key block)
@@ -185,8 +159,8 @@ int split_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const 
   // are: a key block's after its last sub-problem (waiting for the other stream's part of the block),
   // a value block's at the end of the stream that ran all its sub-problems (nv even) or after the
   // join.
-  SideStream* side = nullptr;
-  GLA_TRY(side_stream(&side));
+  gla::fast::SideStream* side = nullptr;
+  GLA_CUDA(gla::fast::side_stream(0, &side));
   std::lock_guard<std::mutex> lock(side->mu);
   cudaStream_t sts[2] = {st, side->s};
   GLA_CUDA(cudaEventRecord(side->fork, st));
@@ -491,8 +465,8 @@ int gsa_bwd_fused(const bf16* q, const bf16* k, const bf16* v, const bf16* phi, 
   if (dhT1) GLA_CUDA(gla::gsa::transpose_states(dhT1, s1, w.dhTp, BH, dkd, m, 128, st));
   // From here the pass-1 backward (caller's stream) and the dq forwards (side stream) read only do1
   // and the inputs, and write disjoint outputs, so they run side by side.
-  SideStream* side = nullptr;
-  GLA_TRY(side_stream(&side));
+  gla::fast::SideStream* side = nullptr;
+  GLA_CUDA(gla::fast::side_stream(0, &side));
   std::lock_guard<std::mutex> lock(side->mu);
   GLA_CUDA(cudaEventRecord(side->fork, st));
   GLA_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
