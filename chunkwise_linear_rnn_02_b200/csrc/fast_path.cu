@@ -726,7 +726,7 @@ template <int DK>
 static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o,
                               float* hT, int BH, int T, int dv, long long st_bh, long long st_row, float* acc_o,
                               void* ws, cudaStream_t st, float inv_tau, int dk_total, int k0, const float* add_o,
-                              bool kh_hilo) {
+                              bool kh_hilo, int phase) {
   CUtensorMap m[4];
   if (!make_map(&m[0], q, BH, T, dk_total, DK, false) || !make_map(&m[1], k, BH, T, dk_total, DK, false) ||
       !make_map(&m[2], g, BH, T, dk_total, DK, false) || !make_map(&m[3], v, BH, T, dv, DVT, true))
@@ -753,6 +753,8 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
     if (!ws) return cudaErrorInvalidValue;
     a.sbuf = static_cast<float*>(ws);
     a.gam = a.sbuf + align256((size_t)BH * a.nseg * DK * dv * sizeof(float)) / sizeof(float);
+  }
+  if (a.nseg > 1 && phase != kFwdWalk) {
     cudaError_t e = kh_hilo ? launch_state_pass<DK, true, false, true>(m[1], m[2], m[3], a, BH, dv, st)
                     : flex  ? launch_state_pass<DK, false, false, true>(m[1], m[2], m[3], a, BH, dv, st)
                             : launch_state_pass<DK, false, false, false>(m[1], m[2], m[3], a, BH, dv, st);
@@ -765,6 +767,7 @@ static cudaError_t launch_fwd(const void* q, const void* k, const void* v, const
       if (e != cudaSuccess) return e;
     }
   }
+  if (phase == kFwdStates) return cudaSuccess;
   // the split-Kh build exists for d_k = 64 only (its extra operand does not fit next to d_k = 128)
   const bool logit = inv_tau > 0.f;
   auto kern = kh_hilo ? fwd_pipe_kernel<DK, true, DK == 64, false>
@@ -895,7 +898,7 @@ cudaError_t segment_entry_states(const void* k, const void* g, const void* v, co
 
 cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
                 int BH, int T, int dk, int dv, void* ws, cudaStream_t st, long long st_bh, long long st_row,
-                float* acc_o, float inv_tau, int dk_total, int k0, const float* add_o, bool kh_hilo) {
+                float* acc_o, float inv_tau, int dk_total, int k0, const float* add_o, bool kh_hilo, int phase) {
   if (st_bh < 0) st_bh = (long long)dk * dv;
   if (st_row < 0) st_row = dv;
   if (dk_total < 0) dk_total = dk;
@@ -903,10 +906,10 @@ cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, cons
   if (kh_hilo && (dk != 64 || inv_tau > 0.f)) return cudaErrorNotSupported;
   if (dk == 64)
     return launch_fwd<64>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st, inv_tau, dk_total, k0, add_o,
-                          kh_hilo);
+                          kh_hilo, phase);
   if (dk == 128)
     return launch_fwd<128>(q, k, v, g, h0, o, hT, BH, T, dv, st_bh, st_row, acc_o, ws, st, inv_tau, dk_total, k0,
-                           add_o, false);
+                           add_o, false, phase);
   return cudaErrorNotSupported;
 }
 

@@ -24,10 +24,15 @@ size_t fwd_workspace(int BH, int T, int dk, int dv);
 // tensors: q, k, g are [BH][T][dk_total] and the call uses columns k0 .. k0+dk-1 (read in place by
 // the tile loads); add_o ([BH*T][dv] fp32) is added to o before it is stored (to acc_o or as bf16).
 // kh_hilo (d_k = 64 only): the decayed keys enter the MMAs as bf16 hi + lo pairs too.
+// phase: kFwdAll runs the whole forward; with a sequence split, kFwdStates runs only the segment
+// entry states (state pass and scan, into ws; they need k, g, v and h0, not q) and kFwdWalk only the
+// walks, from entry states an earlier kFwdStates call with the same arguments left in ws.  Without a
+// split kFwdStates does nothing and kFwdWalk is kFwdAll.
+enum FwdPhase { kFwdAll = 0, kFwdStates = 1, kFwdWalk = 2 };
 cudaError_t fwd(const void* q, const void* k, const void* v, const void* g, const float* h0, void* o, float* hT,
                 int BH, int T, int dk, int dv, void* ws, cudaStream_t st, long long st_bh = -1,
                 long long st_row = -1, float* acc_o = nullptr, float inv_tau = 0.f, int dk_total = -1, int k0 = 0,
-                const float* add_o = nullptr, bool kh_hilo = false);
+                const float* add_o = nullptr, bool kh_hilo = false, int phase = kFwdAll);
 
 // A backward sub-problem inside wider tensors (split shapes, padded operands): its key dimensions
 // are columns ck.. of the [BH*T][pk] inputs q, k, g, its value columns cv.. of the [BH*T][pv] inputs

@@ -418,8 +418,21 @@ int gsa_fwd_fused(const bf16* q, const bf16* k, const bf16* v, const bf16* phi, 
   GsaFusedFwdWs w;
   carve_gsa_fused_fwd(c, BH, T, dk, dv, m, p_save == nullptr, &w);
   bf16* p = p_save ? p_save : w.p;
-  GLA_CUDA(gla::gsa::pass1_fwd(q, k, phi, g, h01, p, hT1, BH, T, dk, w.p1ws, st));
-  GLA_CUDA(gla::fast::fwd(p, phi, v, g, h02, o, hT2, BH, T, m, dv, w.fws, st));
+  // Pass 2's segment entry states need phi, g and v, not p: on the side stream, beside pass 1.
+  gla::fast::SideStream* side = nullptr;
+  GLA_CUDA(gla::fast::side_stream(0, &side));
+  {
+    std::lock_guard<std::mutex> lock(side->mu);
+    GLA_CUDA(cudaEventRecord(side->fork, st));
+    GLA_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
+    GLA_CUDA(gla::fast::fwd(p, phi, v, g, h02, o, hT2, BH, T, m, dv, w.fws, side->s, -1, -1, nullptr, 0.f, -1, 0,
+                            nullptr, false, gla::fast::kFwdStates));
+    GLA_CUDA(cudaEventRecord(side->join, side->s));
+    GLA_CUDA(gla::gsa::pass1_fwd(q, k, phi, g, h01, p, hT1, BH, T, dk, w.p1ws, st));
+    GLA_CUDA(cudaStreamWaitEvent(st, side->join, 0));
+  }
+  GLA_CUDA(gla::fast::fwd(p, phi, v, g, h02, o, hT2, BH, T, m, dv, w.fws, st, -1, -1, nullptr, 0.f, -1, 0, nullptr,
+                          false, gla::fast::kFwdWalk));
   return GLA_OK;
 }
 
