@@ -564,7 +564,8 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   uint64_t* bar_m1 = bars + 3;
   uint64_t* bar_m2 = bars + 4;
   uint64_t* bar_mA = bars + 5;  // first part of group 1: Z^T and A
-  uint32_t ph_ld = 0, ph_dv = 0, ph_m1 = 0, ph_m2 = 0, ph_mA = 0;
+  uint64_t* bar_mZ = bars + 6;  // the Z^T part alone
+  uint32_t ph_ld = 0, ph_dv = 0, ph_m1 = 0, ph_m2 = 0, ph_mA = 0, ph_mZ = 0;
   float* DEC = reinterpret_cast<float*>(sm + L::DEC);
   float* TOT = reinterpret_cast<float*>(sm + L::TOT);
 
@@ -615,6 +616,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_HI + ko, 16, 1024), vd, id_Z, k > 0);
       umma_bf16(tmem + L::T_Z, desc_sw128(base + L::GC_LO + ko, 16, 1024), vd, id_Z, 1);
     }
+    umma_commit(bar_mZ);
   };
   // MMA group 1 (producer lane 0): A (first commit, with the Z^T part before it), dv^T = G^T Kh^T
   // and the G update
@@ -785,17 +787,6 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       });
     }
     if (safe) rescale_G();
-    if (tid == 0) safe_flag[0] = safe;
-    handoff(kBarH1);  // group 1
-    if (n > 0) dv_epilogue(i + 1, (n - 1) & 1);  // the previous chunk's dv, while group 1 runs
-    __syncwarp();
-    mbar_wait(bar_mA, ph_mA, a.latch);
-    ph_mA ^= 1;
-    if (safe) {  // the exact path overwrites Qs / Kh, which the rest of group 1 reads
-      mbar_wait(bar_m1, ph_m1, a.latch);
-      ph_m1 ^= 1;
-    }
-    tc_fence_after();
     // this tile's part of Z^T for chunk i: row grow of the M=128 accumulator, 32 tokens
     auto z_epilogue = [&]() {
       float zv[32];
@@ -815,6 +806,22 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       }
       a.ws_kz[((((size_t)bh * (DV / VT) + vt) * NC + i) * 2 + half) * DK + grow] = kz;
     };
+    if (tid == 0) safe_flag[0] = safe;
+    handoff(kBarH1);  // group 1
+    bar_sync(kBarCompute, BT);  // every thread's Kh is in shared memory (the Z^T epilogue reads it)
+    if (n > 0) dv_epilogue(i + 1, (n - 1) & 1);  // the previous chunk's dv, while group 1 runs
+    mbar_wait(bar_mZ, ph_mZ, a.latch);
+    ph_mZ ^= 1;
+    tc_fence_after();
+    if (!safe) z_epilogue();  // its part was issued after the previous chunk's G pass
+    __syncwarp();
+    mbar_wait(bar_mA, ph_mA, a.latch);
+    ph_mA ^= 1;
+    if (safe) {  // the exact path overwrites Qs / Kh, which the rest of group 1 reads
+      mbar_wait(bar_m1, ph_m1, a.latch);
+      ph_m1 ^= 1;
+    }
+    tc_fence_after();
     if (safe) z_epilogue();  // the exact path below overwrites Kh
     float* XA = reinterpret_cast<float*>(sm + L::XA);
     if (safe) {  // exact A = sum_d q_jd k_rd e^{B_jd - B_rd}, r <= j
@@ -854,10 +861,8 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       }
     }
     handoff(kBarH2);  // group 2
-    // while the rest of group 1 runs: the Z^T epilogue (its part completed before A); then, group 1
-    // complete, the G pass (neither touches A, dO or dv)
+    // group 1 complete: the G pass (it touches neither A, dO nor dv)
     if (!safe) {
-      z_epilogue();
       mbar_wait(bar_m1, ph_m1, a.latch);
       ph_m1 ^= 1;
       tc_fence_after();
@@ -1181,7 +1186,7 @@ struct BwdSmem {
 template <int DK, int DV, bool FLEX, bool LOGIT>
 __global__ void __launch_bounds__(BTP, 1) bwd_fused_kernel(const __grid_constant__ BwdMaps mp, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bars[6];
+  __shared__ uint64_t bars[7];
   __shared__ int safe_flag[2];  // exact-path flag of a chunk, compute threads -> producer warp
   __shared__ uint32_t tmem_base_sh;
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -1192,7 +1197,7 @@ __global__ void __launch_bounds__(BTP, 1) bwd_fused_kernel(const __grid_constant
     tmem_relinquish();
   }
   if (threadIdx.x == 0) {
-    for (int b = 0; b < 6; ++b) mbar_init(&bars[b], 1);
+    for (int b = 0; b < 7; ++b) mbar_init(&bars[b], 1);
     fence_mbar_init();
   }
   if (threadIdx.x == BT) {  // the tensor maps, ahead of the first loads
