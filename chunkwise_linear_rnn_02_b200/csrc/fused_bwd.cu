@@ -234,19 +234,27 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   };
   // TMEM state rows -> hi/lo bf16 K-major operand copy; then the rows scaled by DEC[b] (all lanes
   // take part; only owners' rows matter).
+  // The copy uses all 32 lanes, 32 columns at a time: lane l < 16 stores columns 0-15 of its row's
+  // piece, lane l + 16 columns 16-31 of the same row, received by shuffle (the M = 64 accumulator
+  // leaves TMEM lanes 16-31 empty, so those lanes' own values are unused).
   auto state_pass = [&](int b) {
     const float sc = row_owner ? DEC[b * KT + row] : 0.f;
-    float v[64];
-    for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 64) {
+    const int sub = lane >> 4, srow = q4 * 16 + (lane & 15);
+    float v[32];
+    for (int c0 = half * HV; c0 < (half + 1) * HV; c0 += 32) {
       tmem_ld32(tmem + L::T_SG + lane_off + c0, v);
-      tmem_ld32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
       tmem_ld_wait();
-      if (row_owner)
-        store_row_split(sm + L::SG_HI + (c0 / 64) * (KT * 128), sm + L::SG_LO + (c0 / 64) * (KT * 128), row, v, 1.f);
+      float u[16];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) v[c] *= sc;
+      for (int c = 0; c < 16; ++c) {
+        const float x = __shfl_sync(0xffffffffu, v[16 + c], lane & 15);
+        u[c] = sub ? x : v[c];
+      }
+      store_quarter_split(sm + L::SG_HI + (c0 / 64) * (KT * 128), sm + L::SG_LO + (c0 / 64) * (KT * 128), srow, u,
+                          ((c0 & 63) >> 4) + sub);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) v[c] *= sc;
       tmem_st32(tmem + L::T_SG + lane_off + c0, v);
-      tmem_st32(tmem + L::T_SG + lane_off + c0 + 32, v + 32);
     }
     tmem_st_wait();
   };

@@ -145,6 +145,20 @@ __device__ __forceinline__ void store_half_split(uint8_t* th, uint8_t* tl, int r
     *reinterpret_cast<uint4*>(tl + off) = l;
   }
 }
+// Store 16 fp32 values as hi / lo bf16 into columns 16*qb .. 16*qb+15 of swizzled 64-column row r.
+__device__ __forceinline__ void store_quarter_split(uint8_t* th, uint8_t* tl, int r, const float* v, int qb) {
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    uint4 h, l;
+    split2(v[8 * cc + 0], v[8 * cc + 1], h.x, l.x);
+    split2(v[8 * cc + 2], v[8 * cc + 3], h.y, l.y);
+    split2(v[8 * cc + 4], v[8 * cc + 5], h.z, l.z);
+    split2(v[8 * cc + 6], v[8 * cc + 7], h.w, l.w);
+    const uint32_t off = r * 128 + ((((2 * qb + cc) ^ (r & 7)) & 7) << 4);
+    *reinterpret_cast<uint4*>(th + off) = h;
+    *reinterpret_cast<uint4*>(tl + off) = l;
+  }
+}
 // Store 32 fp32 values as bf16 to global (16-byte aligned destination).
 __device__ __forceinline__ void store_half_global_bf16(__nv_bfloat16* dst, const float* v) {
   uint4* d = reinterpret_cast<uint4*>(dst);
