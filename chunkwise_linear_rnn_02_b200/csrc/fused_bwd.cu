@@ -130,7 +130,8 @@ struct KeyLayout {
   static constexpr uint32_t TOT = DEC + 2 * KT * 4;     // float [2][NS][64]: gate run products, per buffer
   static constexpr uint32_t DIAG = TOT + 2 * NS * KT * 4;
   static constexpr uint32_t CARRYP = DIAG + C * 4;      // [2][64] per-column-half partial row sums
-  static constexpr uint32_t TOTAL = CARRYP + 2 * KT * 4;
+  static constexpr uint32_t PRE = CARRYP + 2 * KT * 4;  // float [2][NS][64]: prefix products of TOT
+  static constexpr uint32_t TOTAL = PRE + 2 * NS * KT * 4;
   // TMEM columns
   static constexpr uint32_t T_SG = 0, T_DA = DV, T_X = DV + 64, T_Y = DV + 128;
   static_assert(DV + 192 <= 512, "TMEM columns");
@@ -171,6 +172,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   uint32_t ph_pa = 0, ph_pb = 0, ph_m1 = 0, ph_m2 = 0;
   float* DEC = reinterpret_cast<float*>(sm + L::DEC);
   float* TOT = reinterpret_cast<float*>(sm + L::TOT);
+  float* PRE = reinterpret_cast<float*>(sm + L::PRE);
   float2* XCH = reinterpret_cast<float2*>(sm + L::XCH);
   float* DIAG = reinterpret_cast<float*>(sm + L::DIAG);
   float* qx_sums = a.ws_qx + (size_t)bh * NC * DK + d0;          // [NC][DK] slice of this head and key tile
@@ -324,6 +326,16 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     wait_b(nb);
     Gate gr;
     const int safe = gate(gr, nb, chunk);
+    if (tid < KT) {  // E1 at each token group's start, multiplied in the order the epilogue used
+      float* pre = PRE + nb * NS * KT;
+      const float* tot = TOT + nb * NS * KT;
+      float e = 1.f;
+#pragma unroll
+      for (int hh = 0; hh < NS; ++hh) {
+        pre[hh * KT + tid] = e;
+        e *= tot[hh * KT + tid];
+      }
+    }
     uint32_t w[Gate::TS];
     gr.load_pairs(sm + pbo(nb) + L::PB_K, KT, true, w);
     if (m2_pending) wait_m2();
@@ -422,7 +434,6 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     float tot_s = 0.f, tot_e = 0.f;
     {  // dq; per-token terms Qt X (-> x) and q dq^intra without j = r (-> y)
       const uint32_t pk = pbo(b) + L::PB_K, pg = pbo(b) + L::PB_G, pq = pbo(b) + L::PB_Q;
-      const float* tot = TOT + b * NS * KT;
       if (safe) {  // exact intra term y_j = sum_{r<=j} dA_jr k_r e^{B_j - B_r}
         float bj = 0.f;
         for (int t = 0; t < tq; ++t) bj += raw(pg, t, d);
@@ -442,8 +453,9 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       float* dst32 = FLEX ? a.acc_q + ((size_t)bh * T + i * C + tq) * DK + d0 + d : nullptr;
 #pragma unroll
       for (int rr = 0; rr < 16 / TS; ++rr) {
-        float e = 1.f;  // E1 = e^{B_j}, formed as GateRun::forward forms it
-        for (int hh = 0; hh < tq / TS + rr; ++hh) e *= tot[hh * KT + d];
+        // E1 = e^{B_j}, formed as GateRun::forward forms it: the earlier groups' run products, then
+        // this group's factors one token at a time
+        float e = PRE[(b * NS + tq / TS + rr) * KT + d];
 #pragma unroll
         for (int u = 0; u < TS; ++u) {
           const int c = rr * TS + u, j = tq + c;
