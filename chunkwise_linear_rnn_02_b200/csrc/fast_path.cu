@@ -235,10 +235,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 // ------------------------------------------------------------------------------------------
 // Pipelined forward (the full pass).  Per chunk i the two MMA groups run while the CTA works on
-// its neighbours: during group 1 of chunk i (A, O_i = Qs S', dS) the threads store the outputs of
-// chunk i-1 and run the gate math of chunk i+1 into registers; during group 2 of chunk i
-// (O_i += A V) they store chunk i+1's operands (Qs, Kh, the scaled state copy) and group 1 of
-// chunk i+1 is issued right behind it.  O is double-buffered in TMEM; q/k/g come through a
+// its neighbours.  Group 1 is A = Qs Kh^T and dS = Kh^T V (first commit), then O_i = Qs S'
+// (second commit).  During group 1 the threads store the outputs of chunk i-1; once A and dS are
+// done they form A's operand and update the state while the O MMAs still run, hand A over for
+// group 2 (O_i += A V), and run the gate math of chunk i+1 into registers; once group 1 is done
+// they store chunk i+1's operands (Qs, Kh, the scaled state copy) and group 1 of chunk i+1 is
+// issued right behind group 2.  O is double-buffered in TMEM; q/k/g come through a
 // two-stage ring and v through a three-deep ring, so a raw tile is free as soon as its own
 // chunk's math is done.  MMAs issued by one thread complete in order, so waiting for group 1 of
 // chunk i+1 also covers group 2 of chunk i.
@@ -294,7 +296,7 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
   constexpr int TS = Gate::TS;
   constexpr int NHAND = NTHREADS + 32;  // threads taking part in a handoff barrier
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_qkg[2], bar_v[3], bar_mma1, bar_mma2;
+  __shared__ uint64_t bar_qkg[2], bar_v[3], bar_mmaA, bar_mma1, bar_mma2;
   __shared__ uint32_t tmem_base_sh;
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -320,6 +322,7 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     prefetch_tmap(&tm_v);
     for (int b = 0; b < 2; ++b) mbar_init(&bar_qkg[b], 1);
     for (int b = 0; b < 3; ++b) mbar_init(&bar_v[b], 1);
+    mbar_init(&bar_mmaA, 1);
     mbar_init(&bar_mma1, 1);
     mbar_init(&bar_mma2, 1);
     fence_mbar_init();
@@ -358,7 +361,8 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     for (int li = 0; li < nloc; ++li) {
       bar_sync(kBarOps, NHAND);  // chunk li's Qs, Kh and state copy are in shared memory
       if (lane == 0) {
-        // group 1: A = Qs Kh^T, O_li = Qs S', dS = Kh^T V
+        // group 1: A = Qs Kh^T and dS = Kh^T V (first commit: the A epilogue and the state update
+        // need only these), then O_li = Qs S' (second commit)
         mbar_wait(&bar_v[li % 3], (li / 3) & 1, latch);
         tc_fence_after();
         const uint32_t vbase = base + L::V0 + (li % 3) * L::VTB;
@@ -375,16 +379,22 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
           umma_bf16(t_A, qh_d, kd, id_A, k > 0);
           umma_bf16(t_A, ql_d, kd, id_A, 1);
           if (KHILO) umma_bf16(t_A, qh_d, desc_sw128(base + L::KH_LO + koff, 16, 1024), id_A, 1);
-          const uint64_t sh = desc_sw128(base + L::SB_HI + k * 2048, 16, 1024);
-          umma_bf16(t_O, qh_d, sh, id_O, k > 0);
-          umma_bf16(t_O, qh_d, desc_sw128(base + L::SB_LO + k * 2048, 16, 1024), id_O, 1);
-          umma_bf16(t_O, ql_d, sh, id_O, 1);
         }
 #pragma unroll
         for (int k = 0; k < C / 16; ++k) {
           const uint64_t vd = desc_sw128(vbase + k * 2048, 16, 1024);
           umma_bf16(t_dS, desc_sw128(base + L::KH + k * 2048, C * 128, 1024), vd, id_S, k > 0);
           if (KHILO) umma_bf16(t_dS, desc_sw128(base + L::KH_LO + k * 2048, C * 128, 1024), vd, id_S, 1);
+        }
+        umma_commit(&bar_mmaA);
+#pragma unroll
+        for (int k = 0; k < DK / 16; ++k) {
+          const uint32_t koff = (k >> 2) * (C * 128) + (k & 3) * 32;
+          const uint64_t qh_d = desc_sw128(base + L::QS_HI + koff, 16, 1024);
+          const uint64_t sh = desc_sw128(base + L::SB_HI + k * 2048, 16, 1024);
+          umma_bf16(t_O, qh_d, sh, id_O, k > 0);
+          umma_bf16(t_O, qh_d, desc_sw128(base + L::SB_LO + k * 2048, 16, 1024), id_O, 1);
+          umma_bf16(t_O, desc_sw128(base + L::QS_LO + koff, 16, 1024), sh, id_O, 1);
         }
         umma_commit(&bar_mma1);
       }
@@ -548,15 +558,12 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
         const int t = (c_begin + li) * C + q4 * 16 + lane;
         if (t < T) prefetch_l1(args.add_o + ((size_t)bh * T + t) * DV + dv0 + half * 32);
       }
-      // ---- while group 1 of chunk li runs: outputs of chunk li-1, gate math of chunk li+1 ----
+      // ---- while group 1 of chunk li runs: outputs of chunk li-1 ----
       if (li > 0) store_o(li - 1);
-      int safe_next = 0;
-      if (li + 1 < nloc) {
-        mbar_wait(&bar_qkg[(li + 1) & 1], ((li + 1) >> 1) & 1, latch);
-        safe_next = gate_regs(li + 1);
-      }
-      // ---- group 1 done: exact A if needed, A epilogue, state update; group 2 next ----
-      mbar_wait(&bar_mma1, li & 1, latch);
+      // ---- A and dS done (O may still run): exact A if needed, A epilogue, state update ----
+      mbar_wait(&bar_mmaA, li & 1, latch);
+      // the exact path's scratch lies over Qs and Kh, which the O MMAs read
+      if (safe) mbar_wait(&bar_mma1, li & 1, latch);
       tc_fence_after();
       float* Aex = reinterpret_cast<float*>(sm + L::XA);
       if (safe) {
@@ -607,7 +614,17 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       fence_async_smem();
       tc_fence_before();
       bar_arrive(kBarAB, NHAND);
-      // ---- while group 2 of chunk li runs: operands of chunk li+1 (group 1 follows) ----
+      // ---- while the O MMAs and group 2 of chunk li run: gate math of chunk li+1 ----
+      int safe_next = 0;
+      if (li + 1 < nloc) {
+        mbar_wait(&bar_qkg[(li + 1) & 1], ((li + 1) >> 1) & 1, latch);
+        safe_next = gate_regs(li + 1);
+      }
+      // ---- group 1 done (O read Qs and the state copy): operands of chunk li+1 (group 1 follows) ----
+      if (!safe) {
+        mbar_wait(&bar_mma1, li & 1, latch);
+        tc_fence_after();
+      }
       // Exact-path scratch over Qs / Kh: every compute thread has finished with it before any
       // thread stores chunk li+1's operands.
       if (safe) bar_sync(kBarCompute, NTHREADS);
