@@ -515,34 +515,38 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       tc_fence_before();
       bar_arrive(kBarOps, NHAND);
     };
-    // O rows of local chunk li (after its group 2): bf16 straight to global.
+    // O rows of local chunk li (after its group 2): bf16 straight to global.  The tile is read with
+    // the 16-lane TMEM shape, so each thread holds two rows x four column pairs and a warp's access
+    // covers 8 rows x 32 contiguous bytes (fp32) instead of 16 rows x 16 bytes.
     auto store_o = [&](int li) {
       mbar_wait(&bar_mma2, li & 1, latch);
       tc_fence_after();
-      const int j = q4 * 16 + lane, cb = half * 32;
-      float ov[32];
-      tmem_ld32(t_O0 + (li & 1) * 64 + lane_off + cb, ov);
+      const int cb = half * 32, r0 = q4 * 16 + (lane >> 2), cq = 2 * (lane & 3);
+      float ov[16];  // register 4k + 2h + e: row r0 + 8h, column cb + 8k + cq + e
+      tmem_ld16x32(t_O0 + (li & 1) * 64 + lane_off + cb, ov);
       tmem_ld_wait();
-      const int t = (c_begin + li) * C + j;
-      if (lane < 16 && t < T) {
-        const size_t off = ((size_t)bh * T + t) * DV + dv0 + cb;
-        if (FLEX && args.add_o) {  // a partial output of earlier key blocks
-          const float4* ad = reinterpret_cast<const float4*>(args.add_o + off);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const float4 u = ad[c];
-            ov[4 * c] += u.x;
-            ov[4 * c + 1] += u.y;
-            ov[4 * c + 2] += u.z;
-            ov[4 * c + 3] += u.w;
+      for (int h = 0; h < 2; ++h) {
+        const int t = (c_begin + li) * C + r0 + 8 * h;
+        if (t >= T) continue;
+        const size_t off = ((size_t)bh * T + t) * DV + dv0 + cb + cq;
+        float2 o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) o[k] = make_float2(ov[4 * k + 2 * h], ov[4 * k + 2 * h + 1]);
+        if (FLEX && args.add_o) {  // a partial output of earlier key blocks
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 u = *reinterpret_cast<const float2*>(args.add_o + off + 8 * k);
+            o[k].x += u.x;
+            o[k].y += u.y;
           }
         }
-        if (FLEX && args.acc_o) {
-          float4* p = reinterpret_cast<float4*>(args.acc_o + off);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) p[c] = make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3]);
-        } else {
-          store_half_global_bf16(args.o + off, ov);
+        for (int k = 0; k < 4; ++k) {
+          if (FLEX && args.acc_o)
+            *reinterpret_cast<float2*>(args.acc_o + off + 8 * k) = o[k];
+          else
+            *reinterpret_cast<__nv_bfloat162*>(args.o + off + 8 * k) = __floats2bfloat162_rn(o[k].x, o[k].y);
         }
       }
     };
