@@ -618,11 +618,31 @@ __global__ void decode_kernel(const TI* __restrict__ q, const TI* __restrict__ k
   if (c < DV) {
     const float vc = ldf(v + (size_t)bh * DV + c);
     float* Sb = S + (size_t)bh * DK * DV;
-    for (int d = threadIdx.y; d < DK; d += 8) {
-      const size_t qi = (size_t)bh * DK + d;
-      const float s = expf(ldf(g + qi)) * Sb[(size_t)d * DV + c] + ldf(k + qi) * vc;
-      Sb[(size_t)d * DV + c] = s;
-      acc += ldf(q + qi) * s;
+    constexpr int R = 16;  // rows per thread held in registers (d_k <= 128): all loads in flight at once
+    if (DK <= 8 * R) {
+      float sv[R];
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        const int d = threadIdx.y + 8 * j;
+        sv[j] = d < DK ? Sb[(size_t)d * DV + c] : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        const int d = threadIdx.y + 8 * j;
+        if (d < DK) {
+          const size_t qi = (size_t)bh * DK + d;
+          const float s = expf(ldf(g + qi)) * sv[j] + ldf(k + qi) * vc;
+          Sb[(size_t)d * DV + c] = s;
+          acc += ldf(q + qi) * s;
+        }
+      }
+    } else {
+      for (int d = threadIdx.y; d < DK; d += 8) {
+        const size_t qi = (size_t)bh * DK + d;
+        const float s = expf(ldf(g + qi)) * Sb[(size_t)d * DV + c] + ldf(k + qi) * vc;
+        Sb[(size_t)d * DV + c] = s;
+        acc += ldf(q + qi) * s;
+      }
     }
   }
   part[threadIdx.y][threadIdx.x] = acc;
