@@ -15,15 +15,17 @@
 // Three launches on the caller's stream:
 //   1. two kinds of CTA, independent of each other:
 //      * key-tile CTAs, one per (head, 64 key dimensions): a forward walk that rebuilds S on chip
-//        and writes dq, the forward part of dg and the chunk sums of Qt X (fp32, workspace), and
-//        the carry's start value rowsum(dhT * hT);
+//        and writes dq, the forward part of dg and the chunk sums of Qt X (fp32, workspace), the
+//        carry's start value rowsum(dhT * hT), and (the first key tile of a head) each chunk's
+//        masked dA for the third launch;
 //      * value-tile CTAs, one per (head, 128 value columns): a reverse walk carrying G[:, tile]
 //        that writes dv, dh0[:, tile], and for every chunk this tile's part of Z^T = G V^T and of
 //        the chunk sums of Kh Z (fp32, workspace; both are summed over the value tiles later);
 //   2. a scan over chunks per (head, key dim) that turns the chunk sums into the carry c_i of
 //      every chunk;
 //   3. one CTA per (head, 64 key dimensions, chunk), all independent: dk and the rest of dg
-//      from Z^T, a recomputed dA, the forward walk's part and c_i.
+//      from Z, the key tile's dA, the forward walk's part and c_i.
+// Each CTA of the first launch has 8 compute warps and a ninth warp that issues its MMA groups.
 // With few heads the chunks are cut into segments, each walked by its own key and value tiles:
 // state-only passes and scans first give every segment its entry state S and its end gradient G
 // (segment_states), and each segment's carry starts from rowsum(G_end * S_end) of the states its
@@ -31,8 +33,8 @@
 // States live in TMEM as fp32 accumulators; their bf16 hi / lo copies in shared memory feed the
 // MMAs.  A chunk that keeps less than e^-40 of its state in some dimension computes its
 // intra-chunk terms exactly in fp32 (CUDA cores) instead of through the scaled operands.  A
-// compile-time variant writes fp32 outputs into caller-provided arrays (wide shapes run as
-// blocks and add the blocks' results).
+// compile-time variant reads column blocks of wider tensors and writes fp32 outputs (wide shapes
+// run as blocks whose results are added afterwards).
 #include "fast_path.cuh"
 #include "fused_common.cuh"
 
@@ -552,7 +554,8 @@ struct ValLayout {
   static constexpr uint32_t TOT = DEC + DK * 4;
   static constexpr uint32_t TOTAL = TOT + GateRun<DK, BT>::NSPLIT * DK * 4;
   static constexpr uint32_t XB = QP_HI, XA = KH_HI;  // exact-path scratch (after the first MMA group)
-  // v tile [64 x VT] for Z^T = G V^T: read by the first MMA group only, so it shares A's space
+  // v tile [64 x VT] for Z^T = G V^T: read by the Z^T MMAs only, which complete before the A
+  // commit (MMAs of one thread complete in order), so it shares A's space
   static constexpr uint32_t VZ = AB_HI;
   // dv^T takes 64 columns, double-buffered by chunk parity (its epilogue runs during the next chunk)
   static constexpr uint32_t T_G = 0, T_A = VT, T_DV = VT + 64, T_Z = 2 * VT + 64;
@@ -583,7 +586,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   uint64_t* bar_dv = bars + 1;  // dO, v of a chunk
   uint64_t* bar_m1 = bars + 3;
   uint64_t* bar_m2 = bars + 4;
-  uint64_t* bar_mA = bars + 5;  // first part of group 1: Z^T and A
+  uint64_t* bar_mA = bars + 5;  // the A MMAs (and, completing before them, the Z^T part)
   uint64_t* bar_mZ = bars + 6;  // the Z^T part alone
   uint32_t ph_ld = 0, ph_dv = 0, ph_m1 = 0, ph_m2 = 0, ph_mA = 0, ph_mZ = 0;
   float* DEC = reinterpret_cast<float*>(sm + L::DEC);
