@@ -518,10 +518,23 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     // O rows of local chunk li (after its group 2): bf16 straight to global.  The tile is read with
     // the 16-lane TMEM shape, so each thread holds two rows x four column pairs and a warp's access
     // covers 8 rows x 32 contiguous bytes (fp32) instead of 16 rows x 16 bytes.
-    auto store_o = [&](int li) {
+    const int cb_o = half * 32, r0_o = q4 * 16 + (lane >> 2), cq_o = 2 * (lane & 3);
+    // The partial output of earlier key blocks for chunk li's rows as this thread adds them (see
+    // store_o), loaded a whole chunk step before it is used.
+    auto load_add = [&](int li, float2 (&ad)[8]) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = (c_begin + li) * C + r0_o + 8 * h;
+        const size_t off = ((size_t)bh * T + (t < T ? t : 0)) * DV + dv0 + cb_o + cq_o;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          ad[4 * h + k] = t < T ? *reinterpret_cast<const float2*>(args.add_o + off + 8 * k) : make_float2(0.f, 0.f);
+      }
+    };
+    auto store_o = [&](int li, const float2 (&ad)[8]) {
       mbar_wait(&bar_mma2, li & 1, latch);
       tc_fence_after();
-      const int cb = half * 32, r0 = q4 * 16 + (lane >> 2), cq = 2 * (lane & 3);
+      const int cb = cb_o, r0 = r0_o, cq = cq_o;
       float ov[16];  // register 4k + 2h + e: row r0 + 8h, column cb + 8k + cq + e
       tmem_ld16x32(t_O0 + (li & 1) * 64 + lane_off + cb, ov);
       tmem_ld_wait();
@@ -536,9 +549,8 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
         if (FLEX && args.add_o) {  // a partial output of earlier key blocks
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const float2 u = *reinterpret_cast<const float2*>(args.add_o + off + 8 * k);
-            o[k].x += u.x;
-            o[k].y += u.y;
+            o[k].x += ad[4 * h + k].x;
+            o[k].y += ad[4 * h + k].y;
           }
         }
 #pragma unroll
@@ -554,16 +566,14 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     mbar_wait(&bar_qkg[0], 0, latch);
     int safe = gate_regs(0);
     store_ops(0, safe);
+    float2 ad_cur[8], ad_next[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) ad_cur[k] = ad_next[k] = make_float2(0.f, 0.f);
     for (int li = 0; li < nloc; ++li) {
       const uint8_t* st = sm + (li & 1) * L::QKG;
-      if (FLEX && args.add_o && lane < 16) {
-        // the partial output that store_o(li) adds, one step ahead: this thread's 128-byte row
-        // segment into L1 (the dependent loads would otherwise stall the epilogue)
-        const int t = (c_begin + li) * C + q4 * 16 + lane;
-        if (t < T) prefetch_l1(args.add_o + ((size_t)bh * T + t) * DV + dv0 + half * 32);
-      }
+      if (FLEX && args.add_o) load_add(li, ad_next);  // used by store_o(li), one step later
       // ---- while group 1 of chunk li runs: outputs of chunk li-1 ----
-      if (li > 0) store_o(li - 1);
+      if (li > 0) store_o(li - 1, ad_cur);
       // ---- A and dS done (O may still run): exact A if needed, A epilogue, state update ----
       mbar_wait(&bar_mmaA, li & 1, latch);
       // the exact path's scratch lies over Qs and Kh, which the O MMAs read
@@ -634,8 +644,10 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       if (safe) bar_sync(kBarCompute, NTHREADS);
       if (li + 1 < nloc) store_ops(li + 1, safe_next);
       safe = safe_next;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ad_cur[k] = ad_next[k];
     }
-    store_o(nloc - 1);
+    store_o(nloc - 1, ad_cur);
 
     float* out = (seg == args.nseg - 1 && args.hT) ? args.hT + bh * args.st_bh : nullptr;
     if (s_owner && out) {

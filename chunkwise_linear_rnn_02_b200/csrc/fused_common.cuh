@@ -173,8 +173,6 @@ __device__ __forceinline__ void store_half_global_bf16(__nv_bfloat16* dst, const
   }
 }
 
-// Bring the 128-byte line holding p into L1 (no register result; the line arrives in the background).
-__device__ __forceinline__ void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 
 // Named barriers (id 0 is __syncthreads).  bar_sync waits; bar_arrive signals without waiting (a
 // producer warp syncs on a barrier that the consumer threads only arrive at); bar_or is a barrier
