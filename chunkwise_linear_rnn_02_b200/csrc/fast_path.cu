@@ -86,6 +86,7 @@ struct StateLayout {
   static constexpr uint32_t DECAY = KH + (HILO ? 2 : 1) * C * DK * 2;
   static constexpr uint32_t TOT = DECAY + DK * 4;
   static constexpr uint32_t TOTAL = TOT + GateRun<DK, NTHREADS>::NSPLIT * DK * 4;
+  static_assert(TOT % 8 == 0 && DECAY % 8 == 0, "gate tables are read as float2");
   static constexpr uint32_t ALLOC = TOTAL + 1024;
   static_assert(STAGE % 1024 == 0 && RAW % 1024 == 0, "stage alignment");
 };
@@ -165,10 +166,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     Gate gr;
     gr.set_logit(args.inv_tau, T - (REV ? c_end - 1 - li : c_begin + li) * C);
     gr.run(st + L::RAW, DK, tot_sm);
-    if (gr.h == 0) {
-      decay_sm[gr.d] = gr.dec0;
-      decay_sm[gr.d + 1] = gr.dec1;
-    }
+    if (gr.h == 0) gr.store_decay(decay_sm);
     {
       const uint32_t blk = (gr.d >> 6) * (C * 128), col = gr.d & 63;
       uint32_t w[Gate::TS];
@@ -269,6 +267,7 @@ struct FwdPipeLayout {
   static constexpr int NS = GateRun<DK, NTHREADS>::NSPLIT;
   static constexpr uint32_t TOT = DECAY + 2 * DK * 4;       // float[NS][DK] run products
   static constexpr uint32_t TOTAL = TOT + NS * DK * 4;
+  static_assert(TOT % 8 == 0 && DECAY % 8 == 0, "gate tables are read as float2");
   static constexpr uint32_t ALLOC = TOTAL + 1024;
   // Exact-path scratch during the A epilogue of a chunk (its Qs / Kh are consumed by then, the
   // next chunk's are still in registers): cumulative log-gates over QS_HI.., exact A over KH..
@@ -464,10 +463,7 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       gr.set_logit(args.inv_tau, T - (c_begin + li) * C);
       const bool weak = gr.run(st + 2 * L::RAW, DK, tot_sm);
       float* dec = decay_sm + (li & 1) * DK;
-      if (gr.h == 0) {
-        dec[gr.d] = gr.dec0;
-        dec[gr.d + 1] = gr.dec1;
-      }
+      if (gr.h == 0) gr.store_decay(dec);
       const int safe = bar_or(kBarCompute, NTHREADS, weak);
       gd = gr.d;
       gh = gr.h;

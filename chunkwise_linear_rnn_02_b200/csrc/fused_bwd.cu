@@ -134,6 +134,7 @@ struct KeyLayout {
   static constexpr uint32_t CARRYP = DIAG + C * 4;      // [2][64] per-column-half partial row sums
   static constexpr uint32_t PRE = CARRYP + 2 * KT * 4;  // float [2][NS][64]: prefix products of TOT
   static constexpr uint32_t TOTAL = PRE + 2 * NS * KT * 4;
+  static_assert(TOT % 8 == 0 && DEC % 8 == 0, "gate tables are read as float2");
   // TMEM columns
   static constexpr uint32_t T_SG = 0, T_DA = DV, T_X = DV + 64, T_Y = DV + 128;
   static_assert(DV + 192 <= 512, "TMEM columns");
@@ -154,6 +155,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   using L = KeyLayout<DK, DV>;
   using Gate = GateRun<KT, BT, LOGIT>;
   constexpr int NS = L::NS, TS = Gate::TS;
+  static_assert(TS % 4 == 0, "token pairs u, u ^ 2 of the epilogue loads lie in one group");
   // column offsets into wider input tensors (FLEX builds only)
   const int col_k = FLEX ? a.ck : 0, col_v = FLEX ? a.cv : 0;
   static_assert(TS == 8 && NS == 8, "epilogue runs: four gate runs of eight tokens per token half");
@@ -213,10 +215,7 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
   auto gate = [&](Gate& gr, int b, int chunk) {
     if constexpr (LOGIT) gr.set_logit(a.inv_tau, T - chunk * C);
     const bool weak = gr.run_swizzled(sm + pbo(b) + L::PB_G, TOT + b * NS * KT);
-    if (gr.h == 0) {
-      DEC[b * KT + gr.d] = gr.dec0;
-      DEC[b * KT + gr.d + 1] = gr.dec1;
-    }
+    if (gr.h == 0) gr.store_decay(DEC + b * KT);
     return bar_or(kBarCompute, BT, weak);
   };
   auto write_kq = [&](uint32_t w, int j, int d, float e0, float e1) {
@@ -455,15 +454,27 @@ __device__ void key_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
       float* dst32 = FLEX ? a.acc_q + ((size_t)bh * T + i * C + tq) * DK + d0 + d : nullptr;
 #pragma unroll
       for (int rr = 0; rr < 16 / TS; ++rr) {
+        // The group's raw g, q and k values.  Lanes 16-31 read token rows 16 below those of lanes
+        // 0-15, which the 128-byte swizzle puts on the same banks; so at load step u they read
+        // token u ^ 2 of their group (the other 32-byte half of the row), and the values are put
+        // back in token order once loaded.
+        float gl[TS], ql[TS], kl[TS];
+#pragma unroll
+        for (int u = 0; u < TS; ++u) {
+          const int j = tq + rr * TS + (u ^ (2 * sub));
+          gl[u] = raw(pg, j, d);
+          ql[u] = raw(pq, j, d);
+          kl[u] = raw(pk, j, d);
+        }
         // E1 = e^{B_j}, formed as GateRun::forward forms it: the earlier groups' run products, then
         // this group's factors one token at a time
         float e = PRE[(b * NS + tq / TS + rr) * KT + d];
 #pragma unroll
         for (int u = 0; u < TS; ++u) {
           const int c = rr * TS + u, j = tq + c;
-          e *= ex2(raw(pg, j, d) * kLog2e);
+          e *= ex2((sub ? gl[u ^ 2] : gl[u]) * kLog2e);
           if (!safe) y[c] *= e * inv;
-          const float qv = raw(pq, j, d), kv = raw(pk, j, d);
+          const float qv = sub ? ql[u ^ 2] : ql[u], kv = sub ? kl[u ^ 2] : kl[u];
           if (i * C + j < T) {
             if constexpr (FLEX)
               dst32[(size_t)c * DK] = e * x[c] + y[c];
@@ -553,6 +564,7 @@ struct ValLayout {
   static constexpr uint32_t DEC = AB_LO + C * C * 2;
   static constexpr uint32_t TOT = DEC + DK * 4;
   static constexpr uint32_t TOTAL = TOT + GateRun<DK, BT>::NSPLIT * DK * 4;
+  static_assert(TOT % 8 == 0 && DEC % 8 == 0, "gate tables are read as float2");
   static constexpr uint32_t XB = QP_HI, XA = KH_HI;  // exact-path scratch (after the first MMA group)
   // v tile [64 x VT] for Z^T = G V^T: read by the Z^T MMAs only, which complete before the A
   // commit (MMAs of one thread complete in order), so it shares A's space
@@ -783,10 +795,7 @@ __device__ void val_tile_body(uint8_t* sm, const BwdMaps& mp, const BwdArgs& a, 
     Gate gr;
     if constexpr (LOGIT) gr.set_logit(a.inv_tau, T - i * C);
     const bool weak = gr.run(sm + 2 * L::RAW, DK, TOT);
-    if (gr.h == 0) {
-      DEC[gr.d] = gr.dec0;
-      DEC[gr.d + 1] = gr.dec1;
-    }
+    if (gr.h == 0) gr.store_decay(DEC);
     const int safe = bar_or(kBarCompute, BT, weak);
     {
       const float inv0 = safe ? 1.f : 1.f / gr.dec0, inv1 = safe ? 1.f : 1.f / gr.dec1;
@@ -992,6 +1001,7 @@ struct ChunkLayout {
   static constexpr uint32_t DEC = XCH + 2 * KT * 8;
   static constexpr uint32_t TOT = DEC + KT * 4;
   static constexpr uint32_t TOTAL = TOT + NS * KT * 4;
+  static_assert(TOT % 8 == 0 && DEC % 8 == 0, "gate tables are read as float2");
   static constexpr uint32_t T_Y = 0;  // TMEM columns (64 allocated)
   static_assert(KQ_HI % 1024 == 0 && DA_HI % 1024 == 0 && DIAG == DA_HI + 2 * TILE &&
                     DIAG + C * 4 - DA_HI == kDaBytes,
@@ -1005,6 +1015,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   // column offset into wider input tensors (FLEX builds only)
   const int col_k = FLEX ? a.ck : 0;
   constexpr int NS = L::NS, TS = Gate::TS, NVT = DV / VT;
+  static_assert(TS % 4 == 0, "token pairs u, u ^ 2 of the epilogue loads lie in one group");
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_ld, bar_m2;
   __shared__ uint32_t tmem_base_sh;
@@ -1076,10 +1087,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
   Gate gr;
   if constexpr (LOGIT) gr.set_logit(a.inv_tau, T - i * C);
   const bool weak = gr.run_swizzled(sm + L::PB_G, TOT);
-  if (gr.h == 0) {
-    DEC[gr.d] = gr.dec0;
-    DEC[gr.d + 1] = gr.dec1;
-  }
+  if (gr.h == 0) gr.store_decay(DEC);
   const int safe = __syncthreads_or(weak);
   uint32_t wq[Gate::TS];
   gr.load_pairs(sm + L::PB_Q, KT, true, wq);
@@ -1140,9 +1148,19 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
 #pragma unroll
     for (int rr = 0; rr < 16 / TS; ++rr) {
       const int h = tq / TS + rr;
+      // the group's raw g, q and k values; lanes 16-31 read token u ^ 2 at load step u, off the
+      // banks of lanes 0-15 (as in the key tile's dq epilogue), and take them back in token order
+      float gl[TS], ql[TS], kl[TS];
+#pragma unroll
+      for (int u = 0; u < TS; ++u) {
+        const int r = h * TS + (u ^ (2 * sub));
+        gl[u] = raw(L::PB_G, r, d);
+        ql[u] = raw(L::PB_Q, r, d);
+        kl[u] = raw(L::PB_K, r, d);
+      }
       float al[TS], e2[TS];
 #pragma unroll
-      for (int u = 0; u < TS; ++u) al[u] = ex2(raw(L::PB_G, h * TS + u, d) * kLog2e);
+      for (int u = 0; u < TS; ++u) al[u] = ex2((sub ? gl[u ^ 2] : gl[u]) * kLog2e);
       float e = 1.f;  // E2 = e^{gamma - B_r}, formed as GateRun::backward forms it
       for (int hh = h + 1; hh < NS; ++hh) e *= TOT[hh * KT + d];
 #pragma unroll
@@ -1155,7 +1173,7 @@ __global__ void __launch_bounds__(BT, 2) bwd_chunk_kernel(const __grid_constant_
         const int c = rr * TS + u, r = tq + c;
         const float ev = e2[u];
         if (!safe) w[c] *= ev * inv;
-        const float qv = raw(L::PB_Q, r, d), kv = raw(L::PB_K, r, d);
+        const float qv = sub ? ql[u ^ 2] : ql[u], kv = sub ? kl[u ^ 2] : kl[u];
         if (i * C + r < T) {
           if constexpr (FLEX)
             dst32[(size_t)c * DK] = ev * z[c] + w[c];

@@ -198,7 +198,8 @@ constexpr int kBarCompute = 1;  // named barrier of the threads that run the gat
 // tokens starting at h * TS, h = t / (ND/2).  It loads the raw log-gates g (row-major [64][gstride]
 // bf16 at `graw`, columns col0..), computes alpha = e^g with one ex2 per value, and leaves in
 // registers the run's alphas and, via the shared buffer `tot` (NSPLIT x ND floats), the products of
-// the other runs: pre = prod of earlier runs, suf = prod of later runs, dec = e^{gamma}.
+// the other runs: pre = prod of earlier runs, suf = prod of later runs, dec = e^{gamma}.  `tot` and
+// the decay arrays given to store_decay are 8-byte aligned (each thread moves its pair as a float2).
 //
 // Raw-logit gates (LOGIT builds): with inv_tau > 0 the tile holds logits x instead of log-gates, and
 // the run first replaces every element of it, in place, by g = bf16(logsigmoid(x) * inv_tau) (0 for
@@ -261,24 +262,30 @@ struct GateRun {
       r0 *= a0[u];
       r1 *= a1[u];
     }
-    tot[h * ND + d] = r0;
-    tot[h * ND + d + 1] = r1;
+    // one float2 per thread (tot is 8-byte aligned): a warp's 32 pairs take two wavefronts, where
+    // two scalar accesses of stride 8 bytes would each meet a 2-way bank conflict
+    *reinterpret_cast<float2*>(tot + h * ND + d) = make_float2(r0, r1);
     bar_sync(kBarCompute, NTH);  // the NTH threads running the gate math
     pre0 = pre1 = suf0 = suf1 = 1.f;
 #pragma unroll
     for (int hh = 0; hh < NSPLIT; ++hh) {
-      const float t0 = tot[hh * ND + d], t1 = tot[hh * ND + d + 1];
+      const float2 t = *reinterpret_cast<const float2*>(tot + hh * ND + d);
       if (hh < h) {
-        pre0 *= t0;
-        pre1 *= t1;
+        pre0 *= t.x;
+        pre1 *= t.y;
       } else if (hh > h) {
-        suf0 *= t0;
-        suf1 *= t1;
+        suf0 *= t.x;
+        suf1 *= t.y;
       }
     }
     dec0 = pre0 * r0 * suf0;
     dec1 = pre1 * r1 * suf1;
     return !(dec0 >= kMinDecay && dec1 >= kMinDecay);
+  }
+
+  // dec0, dec1 into dst[d], dst[d + 1].
+  __device__ __forceinline__ void store_decay(float* dst) const {
+    *reinterpret_cast<float2*>(dst + d) = make_float2(dec0, dec1);
   }
 
   // The thread's pair of bf16 values for every token of its run, from a [64][ND] tile (row stride

@@ -78,6 +78,7 @@ struct Pass1Layout {
   static constexpr int NS = fast::GateRun<M, NCOMP>::NSPLIT;
   static constexpr uint32_t TOT = SMX + 4 * C * 4;         // float [NS][64]: gate run products
   static constexpr uint32_t TOTAL = TOT + NS * M * 4;
+  static_assert(TOT % 8 == 0 && DECAY % 8 == 0, "gate tables are read as float2");
   static constexpr uint32_t ALLOC = TOTAL + 1024;
   // exact-path scratch while the A epilogue of a chunk runs (its state copy has been consumed):
   // A in fp32 and the decays alpha, both [64][64]
@@ -251,10 +252,7 @@ __global__ void __launch_bounds__(NTH, 1)
       Gate gr;
       const bool weak = gr.run_swizzled(st + L::G_OFF, tot_sm);
       float* dec = decay_sm + (li & 1) * M;
-      if (gr.h == 0) {
-        dec[gr.d] = gr.dec0;
-        dec[gr.d + 1] = gr.dec1;
-      }
+      if (gr.h == 0) gr.store_decay(dec);
       const int safe = bar_or(kBarCompute, NCOMP, weak);
       gd = gr.d;
       gh = gr.h;
